@@ -1,0 +1,647 @@
+/*
+ * gsa_oracle.c -- plain float64 CPU oracle for Gist Sparse Attention (GSA).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (long_context_gsa_b200, libgsa.so) never calls it, and the two share no
+ * code: no headers, helpers, tables or constants.
+ *
+ * Sources (web explainers of "Forget, Then Recall: Learnable Compression and
+ * Selective Unfolding via Gist Sparse Attention", Mao, Li and Fox):
+ *   [ja] gist.science/ja/paper/2604.20920, section 2.1 (basic mechanism,
+ *        steps 1-4) and section 2.2 (hierarchical extension, H-GSA)
+ *   [ko] gist.science/ko/paper/2604.20920, "2. Methodology"
+ *   [nl] gist.science/nl/paper/2604.20920, "Het Proces (Selectieve
+ *        Ontvouwing)": Compressie, Scoring (s_{t,m} = q_t^T k_{g_m}),
+ *        Selectie (top-k), Selectieve Ontvouwing; "Hierarchische Uitbreiding"
+ *
+ * What it computes, step by step, in the order the pages give:
+ *   1. Scoring   s_m = scale * q . k_gist[m] for every completed gist m
+ *                ([nl] Scoring; the 1/sqrt(d) factor is the adopted reading,
+ *                a positive factor does not change the ranking).
+ *   2. Selection the k highest scores; equal scores go to the lower chunk
+ *                index ([nl] Selectie, [ja] 2.1 step 3).
+ *   3. Unfolding the attended token set is: for each selected chunk its raw
+ *                tokens and its gist token (the SG+SR rule, [ja] 2.1 step 3
+ *                and the ablation in section 4); each unselected chunk keeps
+ *                its gist token only, or is dropped when `exclude` is set
+ *                ([nl] Selectieve Ontvouwing, [ko] 2 hybrid attention); plus
+ *                the raw tokens of the query's own unfinished chunk.
+ *   4. Attention exact softmax over that set: w_u = exp(z_u - Z) / sum,
+ *                z_u = scale * q . k_u, output = sum w_u v_u ([ja] 2.1
+ *                step 4, hybrid attention).
+ *   H-GSA ([ja] 2.2, [nl] Hierarchische Uitbreiding): meta-gists summarise
+ *   groups of g gists; the top meta groups are chosen first, then the top
+ *   gists among their children, then the chosen chunks are unfolded.
+ *   Prefill: the same steps for every position of a sequence with
+ *   interleaved gists; a gist position attends its own chunk's raw tokens
+ *   and the gists up to and including itself ([nl] Compressie: the causal
+ *   mask lets a gist see only its own block and the preceding gists).
+ *
+ * Everything is float64 with plain scalar loops; inputs are read from their
+ * storage type (float32, or bfloat16 bits) and widened exactly.  A pool of
+ * POSIX threads runs independent output rows in parallel.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+#define ORC_OK 0
+#define ORC_EINVAL 1
+#define ORC_ENOMEM 2
+
+/* Token kinds in the attended-set report. */
+#define TOK_RAW 0
+#define TOK_GIST 1
+#define TOK_META 2
+
+/* ------------------------------------------------------------------------ */
+/* Argument blocks (mirrored by ctypes in oracle/__init__.py).               */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk;
+  int32_t n_max, t_max, topk, exclude, dtype;
+  double scale;                       /* <= 0 selects 1/sqrt(d) */
+  const void *q, *gist_k, *gist_v, *raw_k, *raw_v;
+  const int32_t *n_gists, *own_len;   /* [batch] */
+  int32_t n_rows;                     /* rows to compute */
+  const int32_t *rows;                /* row id b*hq + h; NULL = all rows */
+  const int32_t *sel_in;              /* optional forced selection [n_rows][topk] */
+  double *out;                        /* [n_rows][d] */
+  double *lse;                        /* [n_rows] or NULL */
+  int32_t *sel_out;                   /* [n_rows][topk] or NULL */
+  double *sel_score;                  /* [n_rows][topk] or NULL */
+  double *scores;                     /* [n_rows][n_max] or NULL (NaN past N) */
+  int32_t set_cap;                    /* capacity of the set report per row */
+  int32_t *set_n, *set_kind, *set_idx;/* [n_rows], [n_rows][set_cap] x2 */
+  double *set_w;                      /* [n_rows][set_cap] */
+  int32_t n_threads;                  /* 0 = all online cores */
+} orc_decode_args;
+
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk;
+  int32_t n_max, t_max, m_max, topk, exclude, dtype;
+  int32_t group, topk_meta;
+  double scale;
+  const void *q, *meta_k, *meta_v, *gist_k, *gist_v, *raw_k, *raw_v;
+  const int32_t *n_gists, *own_len;
+  int32_t n_rows;
+  const int32_t *rows;
+  const int32_t *meta_sel_in;         /* optional [n_rows][topk_meta] */
+  const int32_t *sel_in;              /* optional [n_rows][topk] */
+  double *out, *lse;
+  int32_t *meta_sel_out;              /* [n_rows][topk_meta] or NULL */
+  int32_t *sel_out;                   /* [n_rows][topk] or NULL */
+  double *meta_scores;                /* [n_rows][m_max] or NULL */
+  double *cand_scores;                /* [n_rows][n_max] or NULL: child score by gist id, NaN if not a candidate */
+  int32_t set_cap;
+  int32_t *set_n, *set_kind, *set_idx;
+  double *set_w;
+  int32_t n_threads;
+} orc_hgsa_args;
+
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk;
+  int32_t n_chunks, topk, exclude, dtype;
+  double scale;
+  const void *q_raw, *k_raw, *v_raw;     /* [B][H][n_chunks*chunk][d] */
+  const void *q_gist, *k_gist, *v_gist;  /* [B][H][n_chunks][d] */
+  int32_t n_rows;
+  const int64_t *rows;                /* (b*hq + h) * (L + N) + pos; pos < L raw, else gist pos-L */
+  const int32_t *sel_in;              /* optional [n_rows][topk] */
+  double *out, *lse;
+  int32_t *sel_out;
+  double *sel_score;
+  int32_t set_cap;
+  int32_t *set_n, *set_kind, *set_idx;
+  double *set_w;
+  int32_t n_threads;
+} orc_prefill_args;
+
+/* ------------------------------------------------------------------------ */
+/* Element access and the two primitives: dot product, ranked order.        */
+/* ------------------------------------------------------------------------ */
+
+static double elem(const void *base, size_t i, int dtype) {
+  if (dtype == ORC_F32) return (double)((const float *)base)[i];
+  uint32_t bits = (uint32_t)((const uint16_t *)base)[i] << 16; /* bf16 -> f32, exact */
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+/* q . key, both d-vectors at element offsets qo and ko. */
+static double dot(const void *qb, size_t qo, const void *kb, size_t ko, int d, int dtype) {
+  double acc = 0.0;
+  for (int i = 0; i < d; ++i) acc += elem(qb, qo + i, dtype) * elem(kb, ko + i, dtype);
+  return acc;
+}
+
+typedef struct {
+  double s;
+  int32_t m;
+} scored_t;
+
+/* Ranking: higher score first; equal scores, lower index first. */
+static int cmp_rank(const void *x, const void *y) {
+  const scored_t *a = (const scored_t *)x, *b = (const scored_t *)y;
+  if (a->s > b->s) return -1;
+  if (a->s < b->s) return 1;
+  return (a->m < b->m) ? -1 : (a->m > b->m);
+}
+
+/* ------------------------------------------------------------------------ */
+/* The attended set and exact softmax attention over it.                    */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  const void *kb, *vb; /* key / value array */
+  size_t off;          /* element offset of the row */
+  int32_t kind, idx;   /* report only */
+} token_t;
+
+typedef struct {
+  token_t *tok;
+  int32_t n, cap;
+} tokset_t;
+
+static int push(tokset_t *S, const void *kb, const void *vb, size_t off, int kind, int idx) {
+  if (S->n == S->cap) {
+    int32_t nc = S->cap ? 2 * S->cap : 256;
+    token_t *t = (token_t *)realloc(S->tok, (size_t)nc * sizeof(token_t));
+    if (!t) return ORC_ENOMEM;
+    S->tok = t;
+    S->cap = nc;
+  }
+  token_t *t = &S->tok[S->n++];
+  t->kb = kb;
+  t->vb = vb;
+  t->off = off;
+  t->kind = kind;
+  t->idx = idx;
+  return ORC_OK;
+}
+
+/* z_u = scale * q.k_u ; Z = max z ; w_u = exp(z_u - Z) / sum_v exp(z_v - Z) ;
+ * out = sum_u w_u v_u ; lse = Z + log(sum_v exp(z_v - Z)).                  */
+static int attend(const void *qb, size_t qo, const tokset_t *S, int d, int dtype, double scale,
+                  double *out, double *lse, int32_t set_cap, int32_t *set_n, int32_t *set_kind,
+                  int32_t *set_idx, double *set_w) {
+  for (int i = 0; i < d; ++i) out[i] = 0.0;
+  if (S->n == 0) { /* empty set: defined as zero output, lse = -inf */
+    if (lse) *lse = -INFINITY;
+    if (set_n) *set_n = 0;
+    return ORC_OK;
+  }
+  double *z = (double *)malloc((size_t)S->n * sizeof(double));
+  if (!z) return ORC_ENOMEM;
+  double Z = -INFINITY;
+  for (int u = 0; u < S->n; ++u) {
+    z[u] = scale * dot(qb, qo, S->tok[u].kb, S->tok[u].off, d, dtype);
+    if (z[u] > Z) Z = z[u];
+  }
+  double denom = 0.0;
+  for (int u = 0; u < S->n; ++u) {
+    z[u] = exp(z[u] - Z);
+    denom += z[u];
+  }
+  for (int u = 0; u < S->n; ++u) {
+    double w = z[u] / denom;
+    for (int i = 0; i < d; ++i) out[i] += w * elem(S->tok[u].vb, S->tok[u].off + i, dtype);
+    if (set_w && u < set_cap) {
+      set_kind[u] = S->tok[u].kind;
+      set_idx[u] = S->tok[u].idx;
+      set_w[u] = w;
+    }
+  }
+  if (lse) *lse = Z + log(denom);
+  if (set_n) *set_n = S->n;
+  free(z);
+  return ORC_OK;
+}
+
+/* Select min(k, n) of the candidates by the ranking above.  `cand` is
+ * reordered in place so that the first min(k, n) entries are the selection
+ * in rank order.  Returns the number selected. */
+static int32_t select_topk(scored_t *cand, int32_t n, int32_t k) {
+  qsort(cand, (size_t)n, sizeof(scored_t), cmp_rank);
+  return k < n ? k : n;
+}
+
+/* A forced selection (the conditional oracle): the listed indices, in the
+ * given order, -1 entries ignored.  Returns the count, or -1 if an index is
+ * out of [0, n_valid) or repeated. */
+static int32_t forced_selection(const int32_t *in, int32_t k, int32_t n_valid, scored_t *sel,
+                                const double *score_of) {
+  int32_t n = 0;
+  for (int32_t i = 0; i < k; ++i) {
+    int32_t m = in[i];
+    if (m < 0) continue;
+    if (m >= n_valid) return -1;
+    for (int32_t j = 0; j < n; ++j)
+      if (sel[j].m == m) return -1;
+    sel[n].m = m;
+    sel[n].s = score_of ? score_of[m] : 0.0;
+    ++n;
+  }
+  return n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Thread pool over output rows.                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef int (*row_fn)(const void *args, int64_t row_slot);
+
+typedef struct {
+  row_fn fn;
+  const void *args;
+  int64_t n;
+  int64_t next; /* atomic */
+  int status;   /* atomic: first error */
+} pool_t;
+
+static void *pool_worker(void *p) {
+  pool_t *P = (pool_t *)p;
+  for (;;) {
+    int64_t r = __atomic_fetch_add(&P->next, 1, __ATOMIC_RELAXED);
+    if (r >= P->n) break;
+    int st = P->fn(P->args, r);
+    if (st) {
+      int zero = 0;
+      __atomic_compare_exchange_n(&P->status, &zero, st, 0, __ATOMIC_RELAXED, __ATOMIC_RELAXED);
+    }
+  }
+  return NULL;
+}
+
+int gsa_oracle_default_threads(void) {
+  long n = sysconf(_SC_NPROCESSORS_ONLN);
+  return n > 0 ? (int)n : 1;
+}
+
+static int run_pool(row_fn fn, const void *args, int64_t n, int32_t n_threads) {
+  pool_t P = {fn, args, n, 0, 0};
+  int nt = n_threads > 0 ? n_threads : gsa_oracle_default_threads();
+  if (nt > n) nt = (int)(n > 0 ? n : 1);
+  if (nt <= 1) {
+    pool_worker(&P);
+    return P.status;
+  }
+  pthread_t *th = (pthread_t *)malloc((size_t)nt * sizeof(pthread_t));
+  if (!th) return ORC_ENOMEM;
+  int started = 0;
+  for (int i = 0; i < nt; ++i) {
+    if (pthread_create(&th[i], NULL, pool_worker, &P) != 0) break;
+    ++started;
+  }
+  if (started == 0) pool_worker(&P);
+  for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+  free(th);
+  return P.status;
+}
+
+static double resolve_scale(double scale, int d) { return scale > 0.0 ? scale : 1.0 / sqrt((double)d); }
+
+/* ------------------------------------------------------------------------ */
+/* Flat GSA decode, one (b, h) row.                                          */
+/* ------------------------------------------------------------------------ */
+
+static int decode_row(const void *pa, int64_t slot) {
+  const orc_decode_args *a = (const orc_decode_args *)pa;
+  const int32_t row = a->rows ? a->rows[slot] : (int32_t)slot;
+  const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);
+  const int d = a->d, c = a->chunk, dt = a->dtype;
+  const double scale = resolve_scale(a->scale, d);
+  const int32_t N = a->n_gists[b], own = a->own_len[b];
+  const size_t qo = ((size_t)b * a->hq + h) * d;
+  const size_t gbase = ((size_t)b * a->hkv + kvh) * a->n_max;
+  const size_t rbase = ((size_t)b * a->hkv + kvh) * a->t_max;
+
+  /* 1. scores of every completed gist */
+  scored_t *cand = (scored_t *)malloc((size_t)(N > 0 ? N : 1) * sizeof(scored_t));
+  double *s = (double *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+  char *chosen = (char *)calloc((size_t)(N > 0 ? N : 1), 1);
+  if (!cand || !s || !chosen) return ORC_ENOMEM;
+  for (int32_t m = 0; m < N; ++m) {
+    s[m] = scale * dot(a->q, qo, a->gist_k, (gbase + m) * d, d, dt);
+    cand[m].s = s[m];
+    cand[m].m = m;
+  }
+  if (a->scores) {
+    double *sr = a->scores + (size_t)slot * a->n_max;
+    for (int32_t m = 0; m < a->n_max; ++m) sr[m] = m < N ? s[m] : NAN;
+  }
+
+  /* 2. top-k (or the forced selection) */
+  int32_t nsel;
+  if (a->sel_in) {
+    nsel = forced_selection(a->sel_in + (size_t)slot * a->topk, a->topk, N, cand, s);
+    if (nsel < 0) return ORC_EINVAL;
+  } else {
+    nsel = select_topk(cand, N, a->topk);
+  }
+  for (int32_t i = 0; i < nsel; ++i) chosen[cand[i].m] = 1;
+  if (a->sel_out) {
+    int32_t *so = a->sel_out + (size_t)slot * a->topk;
+    double *ss = a->sel_score ? a->sel_score + (size_t)slot * a->topk : NULL;
+    for (int32_t i = 0; i < a->topk; ++i) {
+      so[i] = i < nsel ? cand[i].m : -1;
+      if (ss) ss[i] = i < nsel ? cand[i].s : -INFINITY;
+    }
+  }
+
+  /* 3. the attended set, in interleaved-sequence order */
+  tokset_t S = {0};
+  int st = ORC_OK;
+  for (int32_t m = 0; m < N && !st; ++m) {
+    if (chosen[m]) {
+      for (int j = 0; j < c && !st; ++j)
+        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    } else if (!a->exclude) {
+      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    }
+  }
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+
+  /* 4. exact softmax attention over the set */
+  if (!st) {
+    const size_t so = (size_t)slot;
+    st = attend(a->q, qo, &S, d, dt, scale, a->out + so * d, a->lse ? a->lse + so : NULL, a->set_cap,
+                a->set_n ? a->set_n + so : NULL, a->set_kind ? a->set_kind + so * a->set_cap : NULL,
+                a->set_idx ? a->set_idx + so * a->set_cap : NULL, a->set_w ? a->set_w + so * a->set_cap : NULL);
+  }
+  free(S.tok);
+  free(cand);
+  free(s);
+  free(chosen);
+  return st;
+}
+
+static int check_common(int32_t B, int32_t hq, int32_t hkv, int32_t d, int32_t c, int32_t dtype) {
+  if (B <= 0 || hq <= 0 || hkv <= 0 || d <= 0 || c <= 0) return ORC_EINVAL;
+  if (hq % hkv) return ORC_EINVAL;
+  if (dtype != ORC_F32 && dtype != ORC_BF16) return ORC_EINVAL;
+  return ORC_OK;
+}
+
+int gsa_oracle_decode(const orc_decode_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (a->topk < 0 || !a->q || !a->gist_k || !a->gist_v || !a->raw_k || !a->raw_v || !a->out) return ORC_EINVAL;
+  if (!a->n_gists || !a->own_len) return ORC_EINVAL;
+  for (int b = 0; b < a->batch; ++b) {
+    int32_t N = a->n_gists[b], own = a->own_len[b];
+    if (N < 0 || N > a->n_max || own < 0 || own > a->chunk) return ORC_EINVAL;
+    if ((int64_t)N * a->chunk + own > a->t_max) return ORC_EINVAL;
+  }
+  int64_t n = a->rows ? a->n_rows : (int64_t)a->batch * a->hq;
+  if (a->rows)
+    for (int64_t i = 0; i < n; ++i)
+      if (a->rows[i] < 0 || a->rows[i] >= a->batch * a->hq) return ORC_EINVAL;
+  return run_pool(decode_row, a, n, a->n_threads);
+}
+
+/* ------------------------------------------------------------------------ */
+/* H-GSA decode, one (b, h) row: meta level, then gist level, then unfold.  */
+/* ------------------------------------------------------------------------ */
+
+static int hgsa_row(const void *pa, int64_t slot) {
+  const orc_hgsa_args *a = (const orc_hgsa_args *)pa;
+  const int32_t row = a->rows ? a->rows[slot] : (int32_t)slot;
+  const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);
+  const int d = a->d, c = a->chunk, dt = a->dtype, g = a->group;
+  const double scale = resolve_scale(a->scale, d);
+  const int32_t N = a->n_gists[b], own = a->own_len[b];
+  const int32_t M = N / g; /* complete meta groups */
+  const size_t qo = ((size_t)b * a->hq + h) * d;
+  const size_t gbase = ((size_t)b * a->hkv + kvh) * a->n_max;
+  const size_t mbase = ((size_t)b * a->hkv + kvh) * a->m_max;
+  const size_t rbase = ((size_t)b * a->hkv + kvh) * a->t_max;
+  int st = ORC_OK;
+
+  /* meta level: score the meta-gists, keep the top groups */
+  const int32_t Mc = M > 0 ? M : 1, Nc = N > 0 ? N : 1;
+  scored_t *mc = (scored_t *)malloc((size_t)Mc * sizeof(scored_t));
+  double *ms = (double *)malloc((size_t)Mc * sizeof(double));
+  char *meta_chosen = (char *)calloc((size_t)Mc, 1);
+  scored_t *gc = (scored_t *)malloc((size_t)Nc * sizeof(scored_t));
+  double *gs = (double *)malloc((size_t)Nc * sizeof(double));
+  char *is_cand = (char *)calloc((size_t)Nc, 1), *chosen = (char *)calloc((size_t)Nc, 1);
+  if (!mc || !ms || !meta_chosen || !gc || !gs || !is_cand || !chosen) return ORC_ENOMEM;
+
+  for (int32_t j = 0; j < M; ++j) {
+    ms[j] = scale * dot(a->q, qo, a->meta_k, (mbase + j) * d, d, dt);
+    mc[j].s = ms[j];
+    mc[j].m = j;
+  }
+  if (a->meta_scores) {
+    double *o = a->meta_scores + (size_t)slot * a->m_max;
+    for (int32_t j = 0; j < a->m_max; ++j) o[j] = j < M ? ms[j] : NAN;
+  }
+  int32_t nmeta;
+  if (a->meta_sel_in) {
+    nmeta = forced_selection(a->meta_sel_in + (size_t)slot * a->topk_meta, a->topk_meta, M, mc, ms);
+    if (nmeta < 0) return ORC_EINVAL;
+  } else {
+    nmeta = select_topk(mc, M, a->topk_meta);
+  }
+  for (int32_t i = 0; i < nmeta; ++i) meta_chosen[mc[i].m] = 1;
+  if (a->meta_sel_out) {
+    int32_t *o = a->meta_sel_out + (size_t)slot * a->topk_meta;
+    for (int32_t i = 0; i < a->topk_meta; ++i) o[i] = i < nmeta ? mc[i].m : -1;
+  }
+
+  /* gist level: candidates are the children of the chosen groups plus the
+   * gists of an incomplete trailing group (no meta-gist summarises them) */
+  int32_t ncand = 0;
+  for (int32_t m = 0; m < N; ++m) {
+    int32_t grp = m / g;
+    if (grp >= M || meta_chosen[grp]) {
+      is_cand[m] = 1;
+      gs[m] = scale * dot(a->q, qo, a->gist_k, (gbase + m) * d, d, dt);
+      gc[ncand].s = gs[m];
+      gc[ncand].m = m;
+      ++ncand;
+    }
+  }
+  if (a->cand_scores) {
+    double *o = a->cand_scores + (size_t)slot * a->n_max;
+    for (int32_t m = 0; m < a->n_max; ++m) o[m] = (m < N && is_cand[m]) ? gs[m] : NAN;
+  }
+  int32_t nsel;
+  if (a->sel_in) {
+    /* forced child selection must name candidates */
+    nsel = forced_selection(a->sel_in + (size_t)slot * a->topk, a->topk, N, gc, gs);
+    if (nsel < 0) return ORC_EINVAL;
+    for (int32_t i = 0; i < nsel; ++i)
+      if (!is_cand[gc[i].m]) return ORC_EINVAL;
+  } else {
+    nsel = select_topk(gc, ncand, a->topk);
+  }
+  for (int32_t i = 0; i < nsel; ++i) chosen[gc[i].m] = 1;
+  if (a->sel_out) {
+    int32_t *o = a->sel_out + (size_t)slot * a->topk;
+    for (int32_t i = 0; i < a->topk; ++i) o[i] = i < nsel ? gc[i].m : -1;
+  }
+
+  /* the attended set: unselected meta-gists, unselected candidate gists,
+   * selected chunks (raw + gist), own raw rows */
+  tokset_t S = {0};
+  if (!a->exclude)
+    for (int32_t j = 0; j < M && !st; ++j)
+      if (!meta_chosen[j]) st = push(&S, a->meta_k, a->meta_v, (mbase + j) * d, TOK_META, j);
+  for (int32_t m = 0; m < N && !st; ++m) {
+    if (chosen[m]) {
+      for (int j = 0; j < c && !st; ++j)
+        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    } else if (is_cand[m] && !a->exclude) {
+      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    }
+  }
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  if (!st) {
+    const size_t so = (size_t)slot;
+    st = attend(a->q, qo, &S, d, dt, scale, a->out + so * d, a->lse ? a->lse + so : NULL, a->set_cap,
+                a->set_n ? a->set_n + so : NULL, a->set_kind ? a->set_kind + so * a->set_cap : NULL,
+                a->set_idx ? a->set_idx + so * a->set_cap : NULL, a->set_w ? a->set_w + so * a->set_cap : NULL);
+  }
+  free(S.tok);
+  free(mc);
+  free(ms);
+  free(meta_chosen);
+  free(gc);
+  free(gs);
+  free(is_cand);
+  free(chosen);
+  return st;
+}
+
+int gsa_oracle_hgsa(const orc_hgsa_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (a->group <= 0 || a->topk < 0 || a->topk_meta < 0) return ORC_EINVAL;
+  if (!a->q || !a->meta_k || !a->meta_v || !a->gist_k || !a->gist_v || !a->raw_k || !a->raw_v || !a->out)
+    return ORC_EINVAL;
+  if (!a->n_gists || !a->own_len) return ORC_EINVAL;
+  for (int b = 0; b < a->batch; ++b) {
+    int32_t N = a->n_gists[b], own = a->own_len[b];
+    if (N < 0 || N > a->n_max || own < 0 || own > a->chunk) return ORC_EINVAL;
+    if (N / a->group > a->m_max) return ORC_EINVAL;
+    if ((int64_t)N * a->chunk + own > a->t_max) return ORC_EINVAL;
+  }
+  int64_t n = a->rows ? a->n_rows : (int64_t)a->batch * a->hq;
+  if (a->rows)
+    for (int64_t i = 0; i < n; ++i)
+      if (a->rows[i] < 0 || a->rows[i] >= a->batch * a->hq) return ORC_EINVAL;
+  return run_pool(hgsa_row, a, n, a->n_threads);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Causal prefill with interleaved gists, one (b, h, position) row.          */
+/* ------------------------------------------------------------------------ */
+
+static int prefill_row(const void *pa, int64_t slot) {
+  const orc_prefill_args *a = (const orc_prefill_args *)pa;
+  const int d = a->d, c = a->chunk, dt = a->dtype;
+  const int32_t N = a->n_chunks;
+  const int64_t L = (int64_t)N * c, P = L + N;
+  const int64_t row = a->rows ? a->rows[slot] : slot;
+  const int64_t bh = row / P, pos = row % P;
+  const int b = (int)(bh / a->hq), h = (int)(bh % a->hq), kvh = h / (a->hq / a->hkv);
+  const double scale = resolve_scale(a->scale, d);
+  const size_t rb = ((size_t)b * a->hkv + kvh) * (size_t)L;  /* raw rows of this kv head */
+  const size_t gb = ((size_t)b * a->hkv + kvh) * (size_t)N;  /* gist rows of this kv head */
+  tokset_t S = {0};
+  int st = ORC_OK;
+  const void *qarr;
+  size_t qo;
+  int32_t nsel = 0;
+  scored_t *cand = NULL;
+  double *s = NULL;
+  char *chosen = NULL;
+
+  if (pos >= L) {
+    /* gist query m: its own chunk's raw tokens and the gists 0..m */
+    const int32_t m = (int32_t)(pos - L);
+    qarr = a->q_gist;
+    qo = (((size_t)b * a->hq + h) * (size_t)N + m) * d;
+    for (int j = 0; j < c && !st; ++j) st = push(&S, a->k_raw, a->v_raw, (rb + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+    for (int32_t t = 0; t <= m && !st; ++t) st = push(&S, a->k_gist, a->v_gist, (gb + t) * d, TOK_GIST, t);
+  } else {
+    /* raw query at position i = m*c + j: completed chunks are 0..m-1 and the
+     * own chunk's raw tokens m*c .. i are visible */
+    const int32_t m = (int32_t)(pos / c), j = (int32_t)(pos % c);
+    qarr = a->q_raw;
+    qo = (((size_t)b * a->hq + h) * (size_t)L + pos) * d;
+    const int32_t mc = m > 0 ? m : 1;
+    cand = (scored_t *)malloc((size_t)mc * sizeof(scored_t));
+    s = (double *)malloc((size_t)mc * sizeof(double));
+    chosen = (char *)calloc((size_t)mc, 1);
+    if (!cand || !s || !chosen) return ORC_ENOMEM;
+    for (int32_t t = 0; t < m; ++t) {
+      s[t] = scale * dot(qarr, qo, a->k_gist, (gb + t) * d, d, dt);
+      cand[t].s = s[t];
+      cand[t].m = t;
+    }
+    if (a->sel_in) {
+      nsel = forced_selection(a->sel_in + (size_t)slot * a->topk, a->topk, m, cand, s);
+      if (nsel < 0) return ORC_EINVAL;
+    } else {
+      nsel = select_topk(cand, m, a->topk);
+    }
+    for (int32_t i = 0; i < nsel; ++i) chosen[cand[i].m] = 1;
+    for (int32_t t = 0; t < m && !st; ++t) {
+      if (chosen[t]) {
+        for (int r = 0; r < c && !st; ++r)
+          st = push(&S, a->k_raw, a->v_raw, (rb + (size_t)t * c + r) * d, TOK_RAW, t * c + r);
+        if (!st) st = push(&S, a->k_gist, a->v_gist, (gb + t) * d, TOK_GIST, t);
+      } else if (!a->exclude) {
+        st = push(&S, a->k_gist, a->v_gist, (gb + t) * d, TOK_GIST, t);
+      }
+    }
+    for (int32_t r = 0; r <= j && !st; ++r)
+      st = push(&S, a->k_raw, a->v_raw, (rb + (size_t)m * c + r) * d, TOK_RAW, m * c + r);
+  }
+  if (a->sel_out) {
+    int32_t *so = a->sel_out + (size_t)slot * a->topk;
+    double *ss = a->sel_score ? a->sel_score + (size_t)slot * a->topk : NULL;
+    for (int32_t i = 0; i < a->topk; ++i) {
+      so[i] = i < nsel ? cand[i].m : -1;
+      if (ss) ss[i] = i < nsel ? cand[i].s : -INFINITY;
+    }
+  }
+  if (!st) {
+    const size_t so = (size_t)slot;
+    st = attend(qarr, qo, &S, d, dt, scale, a->out + so * d, a->lse ? a->lse + so : NULL, a->set_cap,
+                a->set_n ? a->set_n + so : NULL, a->set_kind ? a->set_kind + so * a->set_cap : NULL,
+                a->set_idx ? a->set_idx + so * a->set_cap : NULL, a->set_w ? a->set_w + so * a->set_cap : NULL);
+  }
+  free(S.tok);
+  free(cand);
+  free(s);
+  free(chosen);
+  return st;
+}
+
+int gsa_oracle_prefill(const orc_prefill_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (a->n_chunks < 0 || a->topk < 0) return ORC_EINVAL;
+  if (!a->q_raw || !a->k_raw || !a->v_raw || !a->q_gist || !a->k_gist || !a->v_gist || !a->out) return ORC_EINVAL;
+  const int64_t P = (int64_t)a->n_chunks * a->chunk + a->n_chunks;
+  const int64_t total = (int64_t)a->batch * a->hq * P;
+  int64_t n = a->rows ? a->n_rows : total;
+  if (a->rows)
+    for (int64_t i = 0; i < n; ++i)
+      if (a->rows[i] < 0 || a->rows[i] >= total) return ORC_EINVAL;
+  return run_pool(prefill_row, a, n, a->n_threads);
+}

@@ -1,0 +1,475 @@
+"""Pins for the float64 oracle: checks that do not re-run the oracle's own code.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError on
+a mismatch.  ``test_oracle_pins.py`` runs them against the committed oracle
+(all must pass) and ``test_oracle_mutants.py`` runs them against copies of the
+oracle with a planted mistake (each mistake must fail at least one pin).
+
+The independent formulations used here:
+  * the attended set written as a dense mask over the interleaved sequence
+    [chunk 0 raw tokens, gist 0, chunk 1 raw tokens, gist 1, ..., own tokens]
+    and a numpy softmax over it (no gather, no per-token list);
+  * selection by brute-force enumeration of every k-subset, keeping the one
+    with the largest score sum, earliest in lexicographic order on ties;
+  * closed forms: all chunks selected = dense attention; k = 0 = compression
+    only; a zero query = uniform weights = the mean of the attended values,
+    with lse = log(set size);
+  * hand-derived examples in ``tests/golden/``.
+Sources: gist.science explainers of "Forget, Then Recall ... Gist Sparse
+Attention" -- Dutch page "Het Proces" (Compressie, Scoring, Selectie,
+Selectieve Ontvouwing, Hierarchische Uitbreiding), Japanese page sections 2.1
+and 2.2.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+from pathlib import Path
+
+import numpy as np
+
+GOLDEN = Path(__file__).resolve().parent / "golden"
+
+
+# ----------------------------------------------------------------- helpers
+def softmax_attend(q, K, V, mask, scale):
+    """Dense masked softmax attention in float64: returns (out, lse, w)."""
+    z = scale * (K @ q)
+    z = np.where(mask, z, -np.inf)
+    Z = z.max()
+    e = np.exp(z - Z)
+    w = e / e.sum()
+    return w @ V, Z + math.log(e.sum()), w
+
+
+def brute_topk(scores, k):
+    """Best k-subset by score sum; first in lexicographic order on ties."""
+    n = len(scores)
+    k = min(k, n)
+    best, best_sum = (), -np.inf
+    for sub in itertools.combinations(range(n), k):
+        s = float(sum(scores[i] for i in sub))
+        if s > best_sum:
+            best, best_sum = sub, s
+    return set(best)
+
+
+def interleaved(raw_k, raw_v, gk, gv, N, c, own):
+    """Keys/values of the interleaved sequence of one (b, kv head), plus labels."""
+    K, V, lab = [], [], []
+    for m in range(N):
+        for j in range(c):
+            K.append(raw_k[m * c + j]); V.append(raw_v[m * c + j]); lab.append(("raw", m))
+        K.append(gk[m]); V.append(gv[m]); lab.append(("gist", m))
+    for j in range(own):
+        K.append(raw_k[N * c + j]); V.append(raw_v[N * c + j]); lab.append(("own", j))
+    return np.array(K, dtype=np.float64), np.array(V, dtype=np.float64), lab
+
+
+def decode_mask(lab, S, exclude):
+    return np.array([(kind == "raw" and m in S) or (kind == "gist" and (m in S or not exclude)) or kind == "own"
+                     for kind, m in lab])
+
+
+def rand_decode(rng, B, Hq, Hkv, d, c, N, own, extra_gists=1, dtype="f32"):
+    n_max = N + extra_gists
+    t_max = n_max * c + c
+    arr = {
+        "q": rng.standard_normal((B, Hq, d)),
+        "gist_k": rng.standard_normal((B, Hkv, n_max, d)),
+        "gist_v": rng.standard_normal((B, Hkv, n_max, d)),
+        "raw_k": rng.standard_normal((B, Hkv, t_max, d)),
+        "raw_v": rng.standard_normal((B, Hkv, t_max, d)),
+    }
+    arr = {k: v.astype(np.float32) for k, v in arr.items()}
+    if dtype == "bf16":
+        from oracle import bf16_bits
+        arr = {k: bf16_bits(v) for k, v in arr.items()}
+    arr["n_gists"] = np.full(B, N, np.int32)
+    arr["own_len"] = np.full(B, own, np.int32)
+    return arr
+
+
+def as_f64(a):
+    if a.dtype == np.uint16:
+        from oracle import bf16_to_f32
+        return bf16_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def run_decode(orc, arr, c, k, exclude, **kw):
+    return orc.decode(arr["q"], arr["gist_k"], arr["gist_v"], arr["raw_k"], arr["raw_v"], arr["n_gists"],
+                      arr["own_len"], chunk=c, topk=k, exclude=exclude, **kw)
+
+
+def dense_decode_reference(arr, b, h, Hq, Hkv, c, k, exclude, scale=None, S=None):
+    """Brute-force selection + dense masked attention for one decode row."""
+    d = arr["q"].shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    kvh = h // (Hq // Hkv)
+    N, own = int(arr["n_gists"][b]), int(arr["own_len"][b])
+    q = as_f64(arr["q"])[b, h]
+    gk, gv = as_f64(arr["gist_k"])[b, kvh], as_f64(arr["gist_v"])[b, kvh]
+    rk, rv = as_f64(arr["raw_k"])[b, kvh], as_f64(arr["raw_v"])[b, kvh]
+    scores = scale * (gk[:N] @ q)
+    if S is None:
+        S = brute_topk(list(scores), k)
+    K, V, lab = interleaved(rk, rv, gk, gv, N, c, own)
+    out, lse, _ = softmax_attend(q, K, V, decode_mask(lab, S, exclude), scale)
+    return out, lse, S
+
+
+# ------------------------------------------------------------ decode pins
+def pin_decode_bruteforce(orc):
+    """Tiny problems: selection = best subset, output = dense masked softmax."""
+    rng = np.random.default_rng(11)
+    for trial in range(24):
+        c = int(rng.integers(1, 4))
+        N = int(rng.integers(0, 7))
+        k = int(rng.integers(0, 5))
+        own = int(rng.integers(1, c + 1))
+        Hkv = int(rng.integers(1, 3))
+        G = int(rng.integers(1, 3))
+        d = int(rng.choice([2, 3, 5]))
+        dtype = "bf16" if trial % 3 == 2 else "f32"
+        arr = rand_decode(rng, 2, Hkv * G, Hkv, d, c, N, own, dtype=dtype)
+        arr["n_gists"][1] = max(0, N - 1)  # ragged batch
+        arr["own_len"][1] = 1
+        for exclude in (False, True):
+            res = run_decode(orc, arr, c, k, exclude)
+            for r in range(2 * Hkv * G):
+                b, h = divmod(r, Hkv * G)
+                out, lse, S = dense_decode_reference(arr, b, h, Hkv * G, Hkv, c, k, exclude)
+                got = {int(x) for x in res["sel"][r] if x >= 0}
+                assert got == S, (trial, r, got, S)
+                np.testing.assert_allclose(res["out"][r], out, rtol=1e-12, atol=1e-12)
+                assert abs(res["lse"][r] - lse) < 1e-12
+
+
+def pin_decode_dense_limit(orc):
+    """k >= N: every chunk unfolded, the output is dense attention over the whole sequence."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, d, c, N, own = 2, 4, 2, 8, 4, 9, 3
+    arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+    for exclude in (False, True):
+        res = run_decode(orc, arr, c, N + 2, exclude)
+        for r in range(B * Hq):
+            b, h = divmod(r, Hq)
+            kvh = h // (Hq // Hkv)
+            q = arr["q"][b, h].astype(np.float64)
+            K = np.concatenate([arr["raw_k"][b, kvh, : N * c + own], arr["gist_k"][b, kvh, :N]]).astype(np.float64)
+            V = np.concatenate([arr["raw_v"][b, kvh, : N * c + own], arr["gist_v"][b, kvh, :N]]).astype(np.float64)
+            z = (K @ q) / math.sqrt(d)
+            w = np.exp(z - z.max())
+            w /= w.sum()
+            np.testing.assert_allclose(res["out"][r], w @ V, rtol=1e-12, atol=1e-12)
+            assert sorted(res["sel"][r][:N]) == list(range(N)) and (res["sel"][r][N:] == -1).all()
+
+
+def pin_decode_k0_compression_only(orc):
+    """k = 0: all gists + own tokens (default); own tokens only (exclude)."""
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, d, c, N, own = 1, 2, 1, 6, 3, 5, 2
+    arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+    for exclude in (False, True):
+        res = run_decode(orc, arr, c, 0, exclude)
+        for h in range(Hq):
+            q = arr["q"][0, h].astype(np.float64)
+            own_k = arr["raw_k"][0, 0, N * c: N * c + own]
+            own_v = arr["raw_v"][0, 0, N * c: N * c + own]
+            K = own_k if exclude else np.concatenate([arr["gist_k"][0, 0, :N], own_k])
+            V = own_v if exclude else np.concatenate([arr["gist_v"][0, 0, :N], own_v])
+            z = (K.astype(np.float64) @ q) / math.sqrt(d)
+            w = np.exp(z - z.max())
+            w /= w.sum()
+            np.testing.assert_allclose(res["out"][h], w @ V.astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def pin_decode_zero_query(orc):
+    """q = 0: all scores tie, so chunks 0..k-1 are chosen; weights are uniform,
+    the output is the plain mean of the attended values and lse = log(set size)."""
+    rng = np.random.default_rng(14)
+    d, c, N, own, k = 4, 3, 7, 2, 3
+    arr = rand_decode(rng, 1, 1, 1, d, c, N, own)
+    arr["q"][:] = 0
+    for exclude in (False, True):
+        res = run_decode(orc, arr, c, k, exclude, set_cap=64)
+        assert list(res["sel"][0]) == [0, 1, 2]
+        rows = [arr["raw_v"][0, 0, m * c + j] for m in range(k) for j in range(c)]
+        gists = list(range(N)) if not exclude else list(range(k))
+        rows += [arr["gist_v"][0, 0, m] for m in gists]
+        rows += [arr["raw_v"][0, 0, N * c + j] for j in range(own)]
+        expect = np.mean(np.array(rows, dtype=np.float64), axis=0)
+        np.testing.assert_allclose(res["out"][0], expect, rtol=1e-12, atol=1e-13)
+        size = k * (c + 1) + (0 if exclude else N - k) + own
+        assert abs(res["lse"][0] - math.log(size)) < 1e-12
+        assert res["set_n"][0] == size
+
+
+def pin_decode_invariants(orc):
+    """Weights >= 0 sum to 1; output in the coordinate-wise hull of the attended
+    values; consistent chunk permutation leaves the output unchanged; a positive
+    score scale leaves the selection unchanged."""
+    rng = np.random.default_rng(15)
+    B, Hq, Hkv, d, c, N, own, k = 1, 2, 1, 8, 4, 12, 2, 4
+    arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+    cap = 256
+    res = run_decode(orc, arr, c, k, False, set_cap=cap)
+    for r in range(Hq):
+        n = res["set_n"][r]
+        w = res["set_w"][r, :n]
+        assert (w >= 0).all() and abs(w.sum() - 1) < 1e-12
+        vals = []
+        for kind, idx in zip(res["set_kind"][r, :n], res["set_idx"][r, :n]):
+            src = arr["raw_v"] if kind == 0 else arr["gist_v"]
+            vals.append(src[0, 0, idx])
+        vals = np.array(vals, dtype=np.float64)
+        assert (res["out"][r] >= vals.min(0) - 1e-12).all() and (res["out"][r] <= vals.max(0) + 1e-12).all()
+    # permute whole chunks (raw rows + gist together)
+    perm = rng.permutation(N)
+    arr2 = {kk: v.copy() for kk, v in arr.items()}
+    for new, old in enumerate(perm):
+        arr2["gist_k"][:, :, new] = arr["gist_k"][:, :, old]
+        arr2["gist_v"][:, :, new] = arr["gist_v"][:, :, old]
+        arr2["raw_k"][:, :, new * c:(new + 1) * c] = arr["raw_k"][:, :, old * c:(old + 1) * c]
+        arr2["raw_v"][:, :, new * c:(new + 1) * c] = arr["raw_v"][:, :, old * c:(old + 1) * c]
+    res2 = run_decode(orc, arr2, c, k, False)
+    np.testing.assert_allclose(res2["out"], res["out"], rtol=1e-12, atol=1e-12)
+    for r in range(Hq):
+        assert {int(perm[x]) for x in res2["sel"][r]} == {int(x) for x in res["sel"][r]}
+    res3 = run_decode(orc, arr, c, k, False, scale=0.37)
+    assert (res3["sel"] == res["sel"]).all()
+
+
+def pin_decode_exact_ties(orc):
+    """Duplicate gist keys give exactly equal scores; the lower chunk index wins."""
+    rng = np.random.default_rng(16)
+    d, c, N, own = 4, 2, 6, 1
+    arr = rand_decode(rng, 1, 1, 1, d, c, N, own)
+    q = arr["q"][0, 0]
+    base = q / np.linalg.norm(q)
+    for m in (1, 3, 4):
+        arr["gist_k"][0, 0, m] = (3 * base).astype(np.float32)  # highest, tied
+    for m in (0, 2, 5):
+        arr["gist_k"][0, 0, m] = (-3 * base).astype(np.float32)
+    res = run_decode(orc, arr, c, 2, False)
+    assert list(res["sel"][0]) == [1, 3]
+    res = run_decode(orc, arr, c, 4, False)
+    assert list(res["sel"][0][:3]) == [1, 3, 4] and res["sel"][0][3] == 0
+
+
+def pin_decode_gqa_mapping(orc):
+    """Query head h reads kv head h // (Hq/Hkv): each head equals a one-head problem."""
+    rng = np.random.default_rng(17)
+    B, Hq, Hkv, d, c, N, own, k = 1, 6, 2, 4, 2, 5, 1, 2
+    arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+    res = run_decode(orc, arr, c, k, False)
+    for h in range(Hq):
+        kvh = h // (Hq // Hkv)
+        one = {"q": arr["q"][:, h:h + 1], "n_gists": arr["n_gists"], "own_len": arr["own_len"]}
+        for name in ("gist_k", "gist_v", "raw_k", "raw_v"):
+            one[name] = arr[name][:, kvh:kvh + 1]
+        r1 = run_decode(orc, one, c, k, False)
+        np.testing.assert_allclose(res["out"][h], r1["out"][0], rtol=0, atol=0)
+
+
+def pin_decode_golden(orc):
+    """Hand-derived example (tests/golden/decode_hand.json)."""
+    _check_golden(orc, json.loads((GOLDEN / "decode_hand.json").read_text()))
+
+
+# --------------------------------------------------------------- H-GSA pins
+def rand_hgsa(rng, B, Hq, Hkv, d, c, N, g, own):
+    arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+    M = max(1, N // g)
+    arr["meta_k"] = rng.standard_normal((B, Hkv, M + 1, d)).astype(np.float32)
+    arr["meta_v"] = rng.standard_normal((B, Hkv, M + 1, d)).astype(np.float32)
+    return arr
+
+
+def run_hgsa(orc, arr, c, g, km, k, exclude, **kw):
+    return orc.hgsa(arr["q"], arr["meta_k"], arr["meta_v"], arr["gist_k"], arr["gist_v"], arr["raw_k"],
+                    arr["raw_v"], arr["n_gists"], arr["own_len"], chunk=c, group=g, topk_meta=km, topk=k,
+                    exclude=exclude, **kw)
+
+
+def pin_hgsa_bruteforce(orc):
+    """Meta subsets then child subsets by enumeration; dense mask over raw, gist and meta tokens."""
+    rng = np.random.default_rng(21)
+    for trial in range(20):
+        c = int(rng.integers(1, 3))
+        g = int(rng.integers(1, 4))
+        N = int(rng.integers(0, 11))
+        km = int(rng.integers(0, 4))
+        k = int(rng.integers(0, 4))
+        own = int(rng.integers(1, c + 1))
+        d = 3
+        arr = rand_hgsa(rng, 1, 2, 1, d, c, N, g, own)
+        M = N // g
+        for exclude in (False, True):
+            res = run_hgsa(orc, arr, c, g, km, k, exclude)
+            for h in range(2):
+                q = arr["q"][0, h].astype(np.float64)
+                sc = 1 / math.sqrt(d)
+                mk, mv = arr["meta_k"][0, 0].astype(np.float64), arr["meta_v"][0, 0].astype(np.float64)
+                gk, gv = arr["gist_k"][0, 0].astype(np.float64), arr["gist_v"][0, 0].astype(np.float64)
+                rk, rv = arr["raw_k"][0, 0].astype(np.float64), arr["raw_v"][0, 0].astype(np.float64)
+                Sm = brute_topk(list(sc * (mk[:M] @ q)), km)
+                cand = [m for m in range(N) if m // g >= M or m // g in Sm]
+                cs = sc * (gk[cand] @ q) if cand else np.zeros(0)
+                S = {cand[i] for i in brute_topk(list(cs), k)}
+                K, V, lab = interleaved(rk, rv, gk, gv, N, c, own)
+                K = np.concatenate([K, mk[:M]]) if M else K
+                V = np.concatenate([V, mv[:M]]) if M else V
+                lab = lab + [("meta", j) for j in range(M)]
+                mask = np.array([(kind == "raw" and m in S)
+                                 or (kind == "gist" and m in cand and (m in S or not exclude))
+                                 or kind == "own"
+                                 or (kind == "meta" and m not in Sm and not exclude) for kind, m in lab])
+                out, lse, _ = softmax_attend(q, K, V, mask, sc)
+                assert {int(x) for x in res["meta_sel"][h] if x >= 0} == Sm
+                assert {int(x) for x in res["sel"][h] if x >= 0} == S
+                np.testing.assert_allclose(res["out"][h], out, rtol=1e-12, atol=1e-12)
+                assert abs(res["lse"][h] - lse) < 1e-12
+
+
+def pin_hgsa_reduces_to_flat(orc):
+    """All meta groups chosen -> flat GSA; g = 1 with meta = gist -> flat GSA."""
+    rng = np.random.default_rng(22)
+    B, Hq, Hkv, d, c, N, g, own, k = 1, 4, 2, 6, 2, 12, 3, 2, 3
+    arr = rand_hgsa(rng, B, Hq, Hkv, d, c, N, g, own)
+    for exclude in (False, True):
+        flat = run_decode(orc, arr, c, k, exclude)
+        res = run_hgsa(orc, arr, c, g, N // g, k, exclude)
+        np.testing.assert_allclose(res["out"], flat["out"], rtol=1e-12, atol=1e-12)
+        assert (res["sel"] == flat["sel"]).all()
+        arr1 = dict(arr)
+        arr1["meta_k"], arr1["meta_v"] = arr["gist_k"], arr["gist_v"]
+        res1 = run_hgsa(orc, arr1, c, 1, k + 2, k, exclude)
+        np.testing.assert_allclose(res1["out"], flat["out"], rtol=1e-12, atol=1e-12)
+
+
+def pin_hgsa_golden(orc):
+    """Hand-derived example (tests/golden/hgsa_hand.json)."""
+    _check_golden(orc, json.loads((GOLDEN / "hgsa_hand.json").read_text()))
+
+
+# ------------------------------------------------------------- prefill pins
+def rand_prefill(rng, B, Hq, Hkv, d, c, N):
+    L = N * c
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    return {"q_raw": f(B, Hq, L, d), "k_raw": f(B, Hkv, L, d), "v_raw": f(B, Hkv, L, d),
+            "q_gist": f(B, Hq, N, d), "k_gist": f(B, Hkv, N, d), "v_gist": f(B, Hkv, N, d)}
+
+
+def run_prefill(orc, arr, c, k, exclude, **kw):
+    return orc.prefill(arr["q_raw"], arr["k_raw"], arr["v_raw"], arr["q_gist"], arr["k_gist"], arr["v_gist"],
+                       chunk=c, topk=k, exclude=exclude, **kw)
+
+
+def pin_prefill_dense_and_gist_rows(orc):
+    """Rows with m <= k completed chunks = dense causal attention over the interleaved
+    prefix; gist rows = their own chunk's raw tokens + gists 0..m."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, d, c, N, k = 1, 2, 1, 4, 3, 6, 2
+    arr = rand_prefill(rng, B, Hq, Hkv, d, c, N)
+    L = N * c
+    sc = 1 / math.sqrt(d)
+    for exclude in (False, True):
+        res = run_prefill(orc, arr, c, k, exclude)
+        for h in range(Hq):
+            base = h * (L + N)
+            for pos in range(L + N):
+                r = base + pos
+                if pos < L:
+                    m, j = divmod(pos, c)
+                    if m > k:
+                        continue
+                    K = np.concatenate([arr["k_raw"][0, 0, : pos + 1], arr["k_gist"][0, 0, :m]])
+                    V = np.concatenate([arr["v_raw"][0, 0, : pos + 1], arr["v_gist"][0, 0, :m]])
+                    q = arr["q_raw"][0, h, pos]
+                else:
+                    m = pos - L
+                    K = np.concatenate([arr["k_raw"][0, 0, m * c:(m + 1) * c], arr["k_gist"][0, 0, : m + 1]])
+                    V = np.concatenate([arr["v_raw"][0, 0, m * c:(m + 1) * c], arr["v_gist"][0, 0, : m + 1]])
+                    q = arr["q_gist"][0, h, m]
+                z = sc * (K.astype(np.float64) @ q.astype(np.float64))
+                w = np.exp(z - z.max())
+                w /= w.sum()
+                np.testing.assert_allclose(res["out"][r], w @ V.astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def pin_prefill_bruteforce(orc):
+    """Raw rows with m > k: brute-force selection and a dense mask over the prefix."""
+    rng = np.random.default_rng(32)
+    B, Hq, Hkv, d, c, N, k = 1, 4, 2, 3, 2, 6, 2
+    arr = rand_prefill(rng, B, Hq, Hkv, d, c, N)
+    L = N * c
+    sc = 1 / math.sqrt(d)
+    for exclude in (False, True):
+        res = run_prefill(orc, arr, c, k, exclude)
+        for h in range(Hq):
+            kvh = h // (Hq // Hkv)
+            for pos in range(L):
+                m, j = divmod(pos, c)
+                q = arr["q_raw"][0, h, pos].astype(np.float64)
+                gk = arr["k_gist"][0, kvh].astype(np.float64)
+                S = brute_topk(list(sc * (gk[:m] @ q)), k)
+                K, V, lab = interleaved(arr["k_raw"][0, kvh].astype(np.float64), arr["v_raw"][0, kvh].astype(np.float64),
+                                        gk, arr["v_gist"][0, kvh].astype(np.float64), m, c, j + 1)
+                out, lse, _ = softmax_attend(q, K, V, decode_mask(lab, S, exclude), sc)
+                r = h * (L + N) + pos
+                assert {int(x) for x in res["sel"][r] if x >= 0} == S
+                np.testing.assert_allclose(res["out"][r], out, rtol=1e-12, atol=1e-12)
+
+
+def pin_prefill_golden(orc):
+    """Hand-derived example (tests/golden/prefill_hand.json)."""
+    _check_golden(orc, json.loads((GOLDEN / "prefill_hand.json").read_text()))
+
+
+# ------------------------------------------------------------- golden files
+def _arr(x, dtype=np.float32):
+    return np.array(x, dtype=dtype)
+
+
+def _expected_from_logits(tokens):
+    """out = sum e^z v / sum e^z and lse = log sum e^z over the listed tokens."""
+    z = np.array([t["logit"] for t in tokens], dtype=np.float64)
+    v = np.array([t["value"] for t in tokens], dtype=np.float64)
+    e = np.exp(z)
+    return (e @ v) / e.sum(), math.log(e.sum())
+
+
+def _check_golden(orc, G):
+    kind = G["kind"]
+    for case in G["cases"]:
+        inp = {k: _arr(v) for k, v in G["inputs"].items()}
+        p = dict(G["params"], **case.get("params", {}))
+        if kind == "decode":
+            inp["n_gists"] = _arr(G["n_gists"], np.int32)
+            inp["own_len"] = _arr(G["own_len"], np.int32)
+            res = run_decode(orc, inp, p["chunk"], p["topk"], p["exclude"], scale=p["scale"])
+            row = 0
+        elif kind == "hgsa":
+            inp["n_gists"] = _arr(G["n_gists"], np.int32)
+            inp["own_len"] = _arr(G["own_len"], np.int32)
+            res = run_hgsa(orc, inp, p["chunk"], p["group"], p["topk_meta"], p["topk"], p["exclude"], scale=p["scale"])
+            row = 0
+            assert [int(x) for x in res["meta_sel"][0]] == case["meta_selection"]
+        else:
+            res = run_prefill(orc, inp, p["chunk"], p["topk"], p["exclude"], scale=p["scale"], rows=[case["row"]])
+            row = 0
+        assert [int(x) for x in res["sel"][row]] == case["selection"], (case["name"], res["sel"][row])
+        out, lse = _expected_from_logits(case["tokens"])
+        np.testing.assert_allclose(res["out"][row], out, rtol=1e-13, atol=1e-14, err_msg=case["name"])
+        assert abs(res["lse"][row] - lse) < 1e-13, case["name"]
+
+
+DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
+               pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
+               pin_decode_golden]
+HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden]
+PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]
+ALL_PINS = DECODE_PINS + HGSA_PINS + PREFILL_PINS
