@@ -1,0 +1,368 @@
+"""GSA hot-path benchmark: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gsa|reference] [--workload NAME]
+
+A step is one GSA decode step (score every completed gist -> top-k ->
+unfold + attend) for the whole batch of the workload, through the C ABI of
+libgsa.so.  The default workload is the Llama-3.2-1B-shaped decode at 8x
+compression (16 sequences x 32 query heads / 8 kv heads, d=64, 32K raw
+context, chunk 8 -> 4096 gists, top-64).  Inputs are seeded synthetic
+tensors resident in HBM; L2 is flushed (a 2x-L2 buffer is written) between
+timed steps and the flush is outside the timed events.
+
+With --gpus N (launched under torch.distributed.run) every rank runs its own
+batch (different seed): decode rows are independent, so the work shards with
+no collective on the data path (weak scaling).  Step time is the maximum
+over ranks of the device-measured time.
+
+--impl reference times the float64 CPU oracle instead (rank 0 only), on a
+bounded sample of rows per step, with the same metric and workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "GSA decode head-queries/s"
+UNIT = "head-queries/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="gsa", choices=["gsa", "reference"])
+    p.add_argument("--workload", default="llama1b_8x")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    return p.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    f = ROOT / "MEASURED_PEAKS.json"
+    if f.exists():
+        d = json.loads(f.read_text())
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        rows = []
+        for line in Path(self.file.name).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def algorithmic_bytes(cfg, x, sel):
+    """Bytes the method must move for one step: every gist key (+ value in
+    the default set), the raw K/V rows of the union of selected chunks per
+    (b, kv head), selected gist values in exclude mode, own rows, q and out."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    B, hq, hkv, d, c = cfg.batch, cfg.hq, cfg.hkv, cfg.d, cfg.chunk
+    G = hq // hkv
+    N = cfg.n_gists
+    gist = B * hkv * N * d * e * (1 if cfg.exclude else 2)
+    s = sel.reshape(B, hkv, G, -1).cpu()
+    union = 0
+    for b in range(B):
+        for kv in range(hkv):
+            u = torch.unique(s[b, kv])
+            union += int((u >= 0).sum())
+    raw = union * c * d * e * 2
+    gsel = union * d * e if cfg.exclude else 0
+    own = B * hkv * 1 * d * e * 2
+    qo = B * hq * d * e + B * hq * d * 4
+    return {"gist": gist, "raw_union": raw, "gist_sel": gsel, "own": own, "q_out": qo,
+            "total": gist + raw + gsel + own + qo, "union_chunks": union}
+
+
+def score_kernel_bytes(cfg):
+    e = 2 if cfg.dtype == "bf16" else 4
+    return cfg.batch * cfg.hkv * cfg.n_gists * cfg.d * e * (1 if cfg.exclude else 2)
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_rate(x_host, cfg, rows_per_call, target_s, max_calls=1000):
+    """Time the float64 oracle on repeated calls of `rows_per_call` rows."""
+    import oracle
+    o = oracle.get()
+    n_rows = cfg.batch * cfg.hq
+    rows = np.arange(rows_per_call) % n_rows
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        o.decode(x_host["q"], x_host["gist_k"], x_host["gist_v"], x_host["raw_k"], x_host["raw_v"],
+                 x_host["n_gists"], x_host["own_len"], chunk=cfg.chunk, topk=cfg.topk, exclude=cfg.exclude,
+                 rows=rows)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= target_s or calls >= max_calls:
+            break
+    return calls * rows_per_call / el, calls, el, o.default_threads()
+
+
+def host_copy(x):
+    from long_context_gsa_b200.workloads import to_oracle
+    return {k: to_oracle(v) for k, v in x.items() if k in ("q", "gist_k", "gist_v", "raw_k", "raw_v", "n_gists",
+                                                           "own_len")}
+
+
+# ---------------------------------------------------------------- GSA arm
+def run_gsa(args, world, rank, local):
+    import long_context_gsa_b200 as G
+    import long_context_gsa_b200.workloads as W
+
+    G.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    cfg = W.CONFIGS[args.workload]
+    x = W.decode_inputs(cfg, device=dev, seed=cfg.seed + 1000 * rank)
+    B, hq, d = x["q"].shape
+    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
+    dt = G.GSA_BF16 if cfg.dtype == "bf16" else G.GSA_F32
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, cfg.exclude, 0.0, dt, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+    scores = torch.empty((B, hq, n_max), dtype=torch.float32, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    prior = G.GSA_PRIOR_NONE if cfg.exclude else G.GSA_PRIOR_GISTS
+
+    def step_fused():
+        G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
+                     out, None, sel, ssc, ws)
+
+    def step_split(evs):
+        evs[0].record(stream)
+        G.gsa_score_gists(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores, ws)
+        evs[1].record(stream)
+        G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
+        evs[2].record(stream)
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
+                            prior, out, None, ws)
+        evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step_fused()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    # (A) headline: fused decode steps, each bracketed by events, L2 flushed between
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier()
+        for s in range(args.steps):
+            flush.zero_()
+            ev[s][0].record(stream)
+            step_fused()
+            ev[s][1].record(stream)
+        barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    local_ms = sum(step_ms)
+    clocks = clk.summary()
+
+    # (B) per-kernel durations: the same steps through the three entry points
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    for s in range(args.steps):
+        flush.zero_()
+        step_split(kev[s])
+    barrier()
+    kern_ms = np.array([[kev[s][i].elapsed_time(kev[s][i + 1]) for i in range(3)] for s in range(args.steps)])
+
+    # (C) end to end through the public call with host buffers: H2D q, decode, D2H out
+    q_host = x["q"].cpu().pin_memory()
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    for s in range(args.steps):
+        flush.zero_()
+        eev[s][0].record(stream)
+        x["q"].copy_(q_host, non_blocking=True)
+        step_fused()
+        out_host.copy_(out, non_blocking=True)
+        eev[s][1].record(stream)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
+
+    t = torch.tensor([local_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, total_e2e_ms = float(t[0]), float(t[1])
+    ab = algorithmic_bytes(cfg, x, sel)
+    result = None
+    if rank == 0:
+        hbm, bf16, peak_kind = peaks()
+        hq_total = cfg.head_queries * world * args.steps
+        value = hq_total / (total_ms / 1e3)
+        ms_step = total_ms / args.steps
+        k_avg = kern_ms.mean(0)
+        names = ["score_gists", "topk_select", "unfold_attend"]
+        kb = score_kernel_bytes(cfg)
+        dom = int(np.argmax(k_avg))
+        dom_bytes = [kb, None, ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]][dom]
+        roof = None
+        if dom_bytes:
+            ach = dom_bytes / (k_avg[dom] / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": names[dom], "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(ach / hbm, 4), "traffic": None, "peak_kind": peak_kind}
+        step_gbs = ab["total"] / (ms_step / 1e3) / 1e9
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "batch_per_gpu": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv, "d": cfg.d,
+                       "context": cfg.context, "chunk": cfg.chunk, "n_gists": cfg.n_gists, "topk": cfg.topk,
+                       "exclude_unselected": cfg.exclude, "l2": "flushed between timed steps (2x L2 buffer written)",
+                       "parallelism": f"dp{world} (independent rows per GPU)"},
+            "roofline": roof,
+            "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(step_gbs, 1),
+                         "frac": round(step_gbs / hbm, 4), "union_chunks": ab["union_chunks"]},
+            "kernels_us": {n: round(float(v) * 1e3, 2) for n, v in zip(names, k_avg)},
+            "e2e": {"value": round(cfg.head_queries * world * args.steps / (total_e2e_ms / 1e3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": int(x["q"].numel() * x["q"].element_size()),
+                    "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+            "clocks": clocks,
+            "gpu_launches": 3 * args.steps,
+        }
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        xh = host_copy(x)
+        rate, calls, el, cores = oracle_rate(xh, cfg, cfg.head_queries, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(rate, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "sample": f"{calls} full steps of {cfg.head_queries} head-queries ({el:.1f} s)"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import long_context_gsa_b200.workloads as W
+    cfg = W.CONFIGS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = W.decode_inputs(cfg, device=dev)
+    xh = host_copy(x)
+    del x
+    rows_per_step = min(cfg.head_queries, 64)
+    import oracle
+    o = oracle.get()
+    rows = np.arange(rows_per_step)
+
+    def one():
+        o.decode(xh["q"], xh["gist_k"], xh["gist_v"], xh["raw_k"], xh["raw_v"], xh["n_gists"], xh["own_len"],
+                 chunk=cfg.chunk, topk=cfg.topk, exclude=cfg.exclude, rows=rows)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    value = args.steps * rows_per_step / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch_per_gpu": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv, "d": cfg.d,
+                   "context": cfg.context, "chunk": cfg.chunk, "topk": cfg.topk},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": o.default_threads(), "kind": "oracle",
+                         "sample": f"each step = {rows_per_step} of the {cfg.head_queries} head-queries"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+    else:
+        res = run_gsa(args, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

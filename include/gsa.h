@@ -1,0 +1,236 @@
+/*
+ * gsa.h -- C ABI of libgsa.so: the Gist Sparse Attention (GSA) hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web explainers of "Forget, Then Recall: Learnable
+ * Compression and Selective Unfolding via Gist Sparse Attention"):
+ *   [nl] gist.science/nl/paper/2604.20920, "Het Proces (Selectieve
+ *        Ontvouwing)": Compressie, Scoring (s_{t,m} = q_t^T k_{g_m}),
+ *        Selectie (top-k), Selectieve Ontvouwing; "Hierarchische
+ *        Uitbreiding (H-GSA)".
+ *   [ja] gist.science/ja/paper/2604.20920, section 2.1 (steps 1-4:
+ *        gist insertion, relevance scoring, selective unfolding, hybrid
+ *        attention) and section 2.2 (H-GSA, coarse-to-fine selection).
+ *   [ko] gist.science/ko/paper/2604.20920, "2. Methodology" (hybrid
+ *        attention over selected raw tokens plus all, or selected, gists).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  * Pointers named q, *_k, *_v, out*, scores, sel_*, ws, n_gists, own_len
+ *    are DEVICE pointers on the current CUDA device, 16-byte aligned,
+ *    densely packed in the layouts stated below (row-major, last index
+ *    fastest).  The caller allocates and owns all of them; the library
+ *    allocates nothing and keeps no per-call state.
+ *  * `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call only enqueues work on that stream and returns;
+ *    results are ready when the stream is synchronised.
+ *  * Argument checks run on the host before anything is enqueued and return
+ *    GSA_ERR_INVALID_ARG / GSA_ERR_UNSUPPORTED / GSA_ERR_WORKSPACE without
+ *    side effects.  A launch failure returns GSA_ERR_CUDA.  Errors that
+ *    only the device can see (an index in sel_idx out of range, a bounded
+ *    wait that expired) are recorded as bits in the workspace status word
+ *    (gsa_workspace_status) and the offending element is skipped; the
+ *    kernels never trap.
+ *  * Device-side counts n_gists[b] (completed gists, N) and own_len[b]
+ *    (raw tokens of the query's unfinished chunk, 0 <= own <= chunk) are
+ *    int32 arrays of length batch.  They must satisfy N <= n_max and
+ *    N*chunk + own <= t_max; the kernels clamp to these bounds.
+ *  * Query head h reads kv head h / (hq / hkv) (grouped-query layout).
+ *  * Scores and logits are scale * q.k with scale = 1/sqrt(d) unless
+ *    desc->scale > 0.  All accumulation is fp32.
+ *  * Selection per (b, h): the min(topk, N) chunks of highest score, ties
+ *    to the lower chunk index ([nl] Selectie); sel_idx rows are sorted by
+ *    (score desc, index asc) and padded with -1 (sel_score with -inf).
+ *  * Attended set per (b, h) ([ja] 2.1 steps 3-4, [nl] Selectieve
+ *    Ontvouwing): for each selected chunk its `chunk` raw tokens and its
+ *    gist token; each unselected chunk's gist token unless
+ *    exclude_unselected; the own chunk's raw tokens.  Output is the exact
+ *    softmax average of the values over that set; lse is its natural-log
+ *    normaliser (max + log sum exp).
+ *  * A workspace `ws` of gsa_workspace_bytes() bytes is passed to every
+ *    call.  Calls that consume another call's results (score -> select ->
+ *    unfold) must get the same ws.  One ws must not be used by two calls
+ *    that may run concurrently.
+ */
+#ifndef GSA_H
+#define GSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gsa_status {
+  GSA_OK = 0,
+  GSA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or count */
+  GSA_ERR_UNSUPPORTED = 2, /* valid but not built: d, dtype, chunk or topk outside the supported set */
+  GSA_ERR_WORKSPACE = 3,   /* ws too small (see gsa_workspace_bytes) */
+  GSA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  GSA_ERR_TIMEOUT = 5      /* reported by gsa_workspace_status: a bounded device wait expired */
+} gsa_status;
+
+typedef enum gsa_dtype { GSA_F32 = 0, GSA_BF16 = 1 } gsa_dtype;
+
+/* Which partial softmax result a producer left in ws for gsa_unfold_attend. */
+typedef enum gsa_prior {
+  GSA_PRIOR_NONE = 0,  /* nothing: only valid with exclude_unselected = 1 */
+  GSA_PRIOR_GISTS = 1, /* gsa_score_gists in default mode: all completed gists */
+  GSA_PRIOR_HGSA = 2   /* hgsa_select: unselected meta-gists + unselected candidate gists */
+} gsa_prior;
+
+/* Workspace sizing: which call sequence the workspace serves. */
+typedef enum gsa_op { GSA_OP_DECODE = 0, GSA_OP_HGSA = 1, GSA_OP_PREFILL = 2 } gsa_op;
+
+/* Device-side status bits (gsa_workspace_status). */
+#define GSA_DEVERR_BAD_INDEX 0x1u /* a sel_idx entry outside [0, N) or repeated was skipped */
+#define GSA_DEVERR_TIMEOUT 0x2u   /* an mbarrier wait exceeded its iteration bound */
+#define GSA_DEVERR_CAPACITY 0x4u  /* a count exceeded a capacity and was clamped */
+
+typedef struct gsa_desc {
+  int32_t batch;              /* B >= 1 */
+  int32_t hq, hkv;            /* query heads, kv heads; hq % hkv == 0, hq/hkv <= 16 */
+  int32_t d;                  /* head dim: 64 or 128 */
+  int32_t chunk;              /* c: raw tokens per chunk, 1..64 */
+  int32_t n_max;              /* gist capacity per (b, kv head); prefill: number of chunks N */
+  int32_t t_max;              /* raw-row capacity per (b, kv head); prefill: N*chunk */
+  int32_t topk;               /* k, 0..1024 */
+  int32_t exclude_unselected; /* 0: unselected chunks keep their gist; 1: dropped */
+  float scale;                /* <= 0 selects 1/sqrt(d) */
+  int32_t dtype;              /* gsa_dtype of q, gist, meta and raw keys/values */
+  int32_t out_dtype;          /* gsa_dtype of the attention output */
+} gsa_desc;
+
+typedef struct gsa_hdesc {
+  int32_t group;     /* g: gists summarised by one meta-gist, >= 1 */
+  int32_t topk_meta; /* meta groups kept per (b, h), 1..64, topk_meta*group <= 4096 */
+  int32_t m_max;     /* meta capacity per (b, kv head), >= n_max / group */
+} gsa_hdesc;
+
+/* Human-readable name of a status code (static string). */
+const char *gsa_status_string(int32_t status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t gsa_version(void);
+
+/* Bytes of workspace the call sequence `op` needs for these shapes
+ * (hdesc only for GSA_OP_HGSA, may be NULL otherwise).  Returns 0 if the
+ * shapes are invalid. */
+size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc);
+
+/* Zero the workspace on `stream` (cudaMemsetAsync).  Needed once after
+ * allocation; every call leaves the workspace reusable afterwards. */
+gsa_status gsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, copy the workspace status word (GSA_DEVERR_* bits)
+ * to *flags_out and clear it.  A nonzero TIMEOUT bit means results of the
+ * affected calls are invalid. */
+gsa_status gsa_workspace_status(void *ws, size_t ws_bytes, void *stream, uint32_t *flags_out);
+
+/* ---- Flat GSA decode: three steps ------------------------------------- */
+
+/* Step 1, relevance scoring ([nl] Scoring; [ja] 2.1 step 2).
+ *   q       [B, hq, d]
+ *   gist_k  [B, hkv, n_max, d]   gist keys; rows >= n_gists[b] are ignored
+ *   gist_v  [B, hkv, n_max, d]   gist values; may be NULL when
+ *                                exclude_unselected = 1
+ *   scores  [B, hq, n_max] fp32  out: scores[b,h,m] for m < n_gists[b];
+ *                                entries beyond are not written
+ * In default mode the same pass also leaves in ws the softmax partial over
+ * all completed gists (every gist is in the attended set, selected or not),
+ * consumed by gsa_unfold_attend with prior = GSA_PRIOR_GISTS. */
+gsa_status gsa_score_gists(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                           const int32_t *n_gists, float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/* Step 2, top-k chunk selection ([nl] Selectie; [ja] 2.1 step 3).
+ *   scores    [B, hq, n_max] fp32; row (b,h) uses its first n_gists[b]
+ *   sel_idx   [B, hq, topk] int32 out; sel_score [B, hq, topk] fp32 out
+ * Ties go to the lower chunk index.  Also re-arms the per-row counters in
+ * ws that gsa_unfold_attend uses. */
+gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, int32_t *sel_idx,
+                           float *sel_score, void *ws, size_t ws_bytes, void *stream);
+
+/* Step 3, selective unfolding + exact attention ([nl] Selectieve
+ * Ontvouwing; [ja] 2.1 steps 3-4).
+ *   raw_k, raw_v  [B, hkv, t_max, d]  chunk m occupies rows m*chunk ..
+ *                 m*chunk+chunk-1; the own chunk rows N*chunk .. +own-1
+ *   gist_v        [B, hkv, n_max, d]  read for selected chunks when
+ *                 exclude_unselected = 1 (NULL allowed otherwise)
+ *   sel_idx, sel_score  from gsa_topk_select or hgsa_select (the selected
+ *                 gist's logit is its score, so gist keys are not re-read)
+ *   prior         which partial result ws holds (gsa_prior)
+ *   out           [B, hq, d] in out_dtype; lse [B, hq] fp32 or NULL
+ * Selected entries that are -1 are skipped; entries >= N or repeated are
+ * skipped and flagged (GSA_DEVERR_BAD_INDEX). */
+gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *raw_k, const void *raw_v,
+                             const void *gist_v, const int32_t *n_gists, const int32_t *own_len,
+                             const int32_t *sel_idx, const float *sel_score, int32_t prior, void *out, float *lse,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* One decode step = score -> select -> unfold on `stream`.  sel_idx /
+ * sel_score ([B, hq, topk]) may be NULL, in which case ws holds them. */
+gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v, const void *raw_k,
+                      const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
+                      int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- H-GSA decode: one meta level ([ja] 2.2; [nl] Hierarchische
+ * Uitbreiding) -------------------------------------------------------- */
+
+/* Coarse-to-fine selection.  Meta-gist j (j < M = n_gists[b] / group)
+ * summarises gists j*group .. j*group+group-1; gists of an incomplete
+ * trailing group have no meta-gist and are always candidates.
+ *   meta_k, meta_v  [B, hkv, m_max, d]
+ *   meta_idx        [B, hq, topk_meta] int32 out (sorted, -1 padded)
+ *   sel_idx         [B, hq, topk] int32 out: chosen chunks (gist ids)
+ *   sel_score       [B, hq, topk] fp32 out
+ * In default mode ws receives the softmax partial over the unselected
+ * meta-gists and all candidate gists (selected candidates' gists are part
+ * of the set too), consumed with prior = GSA_PRIOR_HGSA. */
+gsa_status hgsa_select(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,
+                       const void *meta_v, const void *gist_k, const void *gist_v, const int32_t *n_gists,
+                       int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* One H-GSA decode step = hgsa_select -> gsa_unfold_attend.  meta_idx,
+ * sel_idx and sel_score may be NULL (ws holds them). */
+gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,
+                       const void *meta_v, const void *gist_k, const void *gist_v, const void *raw_k,
+                       const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
+                       int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* ---- Causal prefill with interleaved gists ([nl] Compressie + the
+ * decode steps applied at every position) ------------------------------ */
+
+/* Layouts (N = desc->n_max chunks, L = N*chunk = desc->t_max):
+ *   q_raw [B, hq, L, d]; k_raw, v_raw [B, hkv, L, d]
+ *   q_gist [B, hq, N, d]; k_gist, v_gist [B, hkv, N, d]
+ * Raw position i = m*chunk + j sees the completed gists 0..m-1 (top-k
+ * selection among them) and its own chunk's raw tokens m*chunk .. i.  Gist
+ * position m sees its chunk's raw tokens and gists 0..m (compression mask).
+ *
+ * Stage 1, scoring + selection for every raw position (tensor cores):
+ *   sel_idx [B, hq, L, topk] int32 out, sel_score [B, hq, L, topk] fp32
+ *   out; in default mode ws also receives each row's softmax partial over
+ *   its completed gists. */
+gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *k_gist, const void *v_gist,
+                             int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
+
+/* Stage 2, unfolding + attention for every raw and gist position:
+ *   out_raw [B, hq, L, d], out_gist [B, hq, N, d] in out_dtype. */
+gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
+                              const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,
+                              const float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* Both stages.  sel_idx / sel_score may be NULL (ws holds them). */
+gsa_status gsa_prefill(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
+                       const void *q_gist, const void *k_gist, const void *v_gist, int32_t *sel_idx,
+                       float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSA_H */

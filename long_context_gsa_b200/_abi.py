@@ -1,0 +1,257 @@
+"""ctypes binding of libgsa.so -- argument marshalling only.
+
+Each function here has the name of the C entry point it calls (see
+include/gsa.h for layouts and semantics), takes torch tensors, checks that
+they live on the current CUDA device with the dtype and contiguity the C
+ABI expects, passes their data pointers and the current (or given) stream,
+and raises GsaError on a non-OK status.  No arithmetic happens here; there
+is no CPU path: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from pathlib import Path
+
+import torch
+
+from .build import LIB
+
+GSA_OK, GSA_ERR_INVALID_ARG, GSA_ERR_UNSUPPORTED, GSA_ERR_WORKSPACE, GSA_ERR_CUDA, GSA_ERR_TIMEOUT = range(6)
+GSA_F32, GSA_BF16 = 0, 1
+GSA_PRIOR_NONE, GSA_PRIOR_GISTS, GSA_PRIOR_HGSA = 0, 1, 2
+GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL = 0, 1, 2
+GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
+
+EXPORTS = (
+    "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
+    "gsa_score_gists", "gsa_topk_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select", "hgsa_decode",
+    "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
+)
+
+
+class GsaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg}")
+        self.status = status
+
+
+class gsa_desc(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32),
+                ("chunk", C.c_int32), ("n_max", C.c_int32), ("t_max", C.c_int32), ("topk", C.c_int32),
+                ("exclude_unselected", C.c_int32), ("scale", C.c_float), ("dtype", C.c_int32),
+                ("out_dtype", C.c_int32)]
+
+
+class gsa_hdesc(C.Structure):
+    _fields_ = [("group", C.c_int32), ("topk_meta", C.c_int32), ("m_max", C.c_int32)]
+
+
+_lib = None
+
+
+def load(path: Path | None = None) -> C.CDLL:
+    """Load libgsa.so (built in-tree by long_context_gsa_b200.build)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = Path(path) if path else LIB
+    if not p.exists():
+        raise RuntimeError(f"{p} is missing: build it with `python -m long_context_gsa_b200.build` "
+                           "(the GSA kernels have no CPU fallback)")
+    lib = C.CDLL(str(p))
+    vp, sz, i32 = C.c_void_p, C.c_size_t, C.c_int32
+    D, H = C.POINTER(gsa_desc), C.POINTER(gsa_hdesc)
+    sig = {
+        "gsa_status_string": ([i32], C.c_char_p),
+        "gsa_version": ([], i32),
+        "gsa_workspace_bytes": ([D, i32, H], sz),
+        "gsa_workspace_init": ([vp, sz, vp], i32),
+        "gsa_workspace_status": ([vp, sz, vp, C.POINTER(C.c_uint32)], i32),
+        "gsa_score_gists": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_topk_select": ([D, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_unfold_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
+        "gsa_decode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "hgsa_select": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "hgsa_decode": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_prefill_score": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+    }
+    for name, (argt, rest) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = argt
+        fn.restype = rest
+    if path is None:
+        _lib = lib
+    return lib
+
+
+# ------------------------------------------------------------- marshalling
+_TORCH_DT = {GSA_F32: torch.float32, GSA_BF16: torch.bfloat16}
+
+
+def make_desc(batch, hq, hkv, d, chunk, n_max, t_max, topk, exclude_unselected=False, scale=0.0,
+              dtype=GSA_BF16, out_dtype=GSA_F32) -> gsa_desc:
+    return gsa_desc(batch, hq, hkv, d, chunk, n_max, t_max, topk, int(bool(exclude_unselected)), float(scale),
+                    dtype, out_dtype)
+
+
+def make_hdesc(group, topk_meta, m_max) -> gsa_hdesc:
+    return gsa_hdesc(group, topk_meta, m_max)
+
+
+def _ptr(t, dtype=None, name="tensor", optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the GSA path has no CPU implementation)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def _check(fn, st):
+    if st != GSA_OK:
+        raise GsaError(fn, st, load().gsa_status_string(st).decode())
+
+
+def _ws(ws):
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous CUDA tensor")
+    return C.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def gsa_status_string(status: int) -> str:
+    return load().gsa_status_string(status).decode()
+
+
+def gsa_version() -> int:
+    return int(load().gsa_version())
+
+
+def gsa_workspace_bytes(desc: gsa_desc, op: int = GSA_OP_DECODE, hdesc: gsa_hdesc | None = None) -> int:
+    return int(load().gsa_workspace_bytes(C.byref(desc), op, C.byref(hdesc) if hdesc is not None else None))
+
+
+def gsa_workspace_init(ws, stream=None):
+    p, n = _ws(ws)
+    _check("gsa_workspace_init", load().gsa_workspace_init(p, n, _stream(stream)))
+
+
+def gsa_workspace_status(ws, stream=None) -> int:
+    p, n = _ws(ws)
+    flags = C.c_uint32(0)
+    st = load().gsa_workspace_status(p, n, _stream(stream), C.byref(flags))
+    if st not in (GSA_OK, GSA_ERR_TIMEOUT):
+        _check("gsa_workspace_status", st)
+    return int(flags.value)
+
+
+def gsa_score_gists(desc, q, gist_k, gist_v, n_gists, scores, ws, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("gsa_score_gists", load().gsa_score_gists(
+        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True),
+        _ptr(n_gists, torch.int32, "n_gists"), _ptr(scores, torch.float32, "scores"), p, n, _stream(stream)))
+
+
+def gsa_topk_select(desc, scores, n_gists, sel_idx, sel_score, ws, stream=None):
+    p, n = _ws(ws)
+    _check("gsa_topk_select", load().gsa_topk_select(
+        C.byref(desc), _ptr(scores, torch.float32, "scores"), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
+        _stream(stream)))
+
+
+def gsa_unfold_attend(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, prior, out, lse, ws,
+                      stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("gsa_unfold_attend", load().gsa_unfold_attend(
+        C.byref(desc), _ptr(q, dt, "q"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
+        _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(own_len, torch.int32, "own_len"), _ptr(sel_idx, torch.int32, "sel_idx", True),
+        _ptr(sel_score, torch.float32, "sel_score", True), int(prior), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
+        _ptr(lse, torch.float32, "lse", True), p, n, _stream(stream)))
+
+
+def gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None, sel_idx=None,
+               sel_score=None, ws=None, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("gsa_decode", load().gsa_decode(
+        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
+        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(own_len, torch.int32, "own_len"), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
+        _ptr(lse, torch.float32, "lse", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
+        _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
+
+
+def hgsa_select(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, n_gists, meta_idx, sel_idx, sel_score, ws,
+                stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("hgsa_select", load().hgsa_select(
+        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q"), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v", True),
+        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(meta_idx, torch.int32, "meta_idx"), _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+
+
+def hgsa_decode(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None,
+                meta_idx=None, sel_idx=None, sel_score=None, ws=None, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("hgsa_decode", load().hgsa_decode(
+        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q"), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v"),
+        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
+        _ptr(n_gists, torch.int32, "n_gists"), _ptr(own_len, torch.int32, "own_len"),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True),
+        _ptr(meta_idx, torch.int32, "meta_idx", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
+        _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
+
+
+def gsa_prefill_score(desc, q_raw, k_gist, v_gist, sel_idx, sel_score, ws, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("gsa_prefill_score", load().gsa_prefill_score(
+        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist", True),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+
+
+def gsa_prefill_attend(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, sel_idx, sel_score, out_raw, out_gist, ws,
+                       stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    odt = _TORCH_DT[desc.out_dtype]
+    p, n = _ws(ws)
+    _check("gsa_prefill_attend", load().gsa_prefill_attend(
+        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_raw, dt, "k_raw"), _ptr(v_raw, dt, "v_raw"),
+        _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"),
+        _ptr(out_raw, odt, "out_raw"), _ptr(out_gist, odt, "out_gist"), p, n, _stream(stream)))
+
+
+def gsa_prefill(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, out_raw, out_gist, sel_idx=None, sel_score=None,
+                ws=None, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    odt = _TORCH_DT[desc.out_dtype]
+    p, n = _ws(ws)
+    _check("gsa_prefill", load().gsa_prefill(
+        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_raw, dt, "k_raw"), _ptr(v_raw, dt, "v_raw"),
+        _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist"),
+        _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True),
+        _ptr(out_raw, odt, "out_raw"), _ptr(out_gist, odt, "out_gist"), p, n, _stream(stream)))

@@ -1,0 +1,481 @@
+// gsa_api.cu -- the extern "C" boundary of libgsa.so (see include/gsa.h).
+//
+// Host side only: argument checks, workspace layout, split sizing and
+// kernel launches.  Every step of the computation runs in the kernels
+// included below; nothing here touches tensor data.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/gsa.h"
+#include "common.cuh"
+#include "k_score.cuh"
+#include "k_topk.cuh"
+#include "k_unfold.cuh"
+
+namespace gsa {
+namespace {
+
+constexpr int kScoreSplitMax = 64;   // partial slots per row from the scoring pass
+constexpr int kUnfoldSplitMax = 32;  // partial slots per row from the unfold pass
+constexpr int kHgsaSplitMax = 32;    // partial slots per row from the H-GSA pass
+constexpr int kTopkSmemCap = 16384;  // keys kept in shared memory by the top-k kernel
+constexpr int kMaxTopk = kTopkMax;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t elem_size(int32_t dt) { return dt == GSA_BF16 ? 2 : 4; }
+inline float resolve_scale(const gsa_desc *d) {
+  return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->d));
+}
+
+struct Layout {
+  size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
+  size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
+  size_t pf_stats = 0;
+  size_t total = 0;
+};
+
+gsa_status check_desc(const gsa_desc *d) {
+  if (!d) return GSA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->hq < 1 || d->hkv < 1 || d->hq % d->hkv) return GSA_ERR_INVALID_ARG;
+  if (d->hq / d->hkv > 16) return GSA_ERR_UNSUPPORTED;
+  if (d->d != 64 && d->d != 128) return GSA_ERR_UNSUPPORTED;
+  if (d->chunk < 1 || d->chunk > 64) return GSA_ERR_UNSUPPORTED;
+  if (d->n_max < 1 || d->t_max < 1 || d->n_max > (1 << 24) || d->t_max > (1 << 28)) return GSA_ERR_INVALID_ARG;
+  if (d->topk < 0) return GSA_ERR_INVALID_ARG;
+  if (d->topk > kMaxTopk) return GSA_ERR_UNSUPPORTED;
+  if (d->exclude_unselected != 0 && d->exclude_unselected != 1) return GSA_ERR_INVALID_ARG;
+  if (d->dtype != GSA_F32 && d->dtype != GSA_BF16) return GSA_ERR_INVALID_ARG;
+  if (d->out_dtype != GSA_F32 && d->out_dtype != GSA_BF16) return GSA_ERR_INVALID_ARG;
+  if (!std::isfinite(d->scale)) return GSA_ERR_INVALID_ARG;
+  if (static_cast<size_t>(d->chunk) * d->d * elem_size(d->dtype) > 32768) return GSA_ERR_UNSUPPORTED;
+  return GSA_OK;
+}
+
+gsa_status check_hdesc(const gsa_desc *d, const gsa_hdesc *h) {
+  if (!h) return GSA_ERR_INVALID_ARG;
+  if (h->group < 1 || h->topk_meta < 1 || h->m_max < 1) return GSA_ERR_INVALID_ARG;
+  if (h->topk_meta > 64 || static_cast<int64_t>(h->topk_meta) * h->group > 4096 || h->group > 4096)
+    return GSA_ERR_UNSUPPORTED;
+  if (h->m_max < d->n_max / h->group) return GSA_ERR_INVALID_ARG;
+  return GSA_OK;
+}
+
+inline int hgsa_cand_cap(const gsa_hdesc *h) { return h->topk_meta * h->group + h->group - 1; }
+
+Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
+  Layout L;
+  const size_t rows = static_cast<size_t>(d->batch) * d->hq;
+  const size_t rec = static_cast<size_t>(d->d + kPartHeader) * 4;
+  size_t off = 0;
+  auto take = [&](size_t &field, size_t bytes) {
+    field = off;
+    off = align256(off + bytes);
+  };
+  take(L.status, 256);
+  take(L.counters, rows * 4);
+  if (op == GSA_OP_PREFILL) {
+    const size_t prow = rows * static_cast<size_t>(d->t_max);
+    take(L.sel_idx, prow * d->topk * 4);
+    take(L.sel_score, prow * d->topk * 4);
+    take(L.pf_stats, prow * rec);
+    L.total = off;
+    return L;
+  }
+  take(L.scores, rows * d->n_max * 4);
+  take(L.sel_idx, rows * d->topk * 4);
+  take(L.sel_score, rows * d->topk * 4);
+  take(L.part_g, rows * kScoreSplitMax * rec);
+  take(L.part_u, rows * kUnfoldSplitMax * rec);
+  if (op == GSA_OP_HGSA && h) {
+    const size_t cap = hgsa_cand_cap(h);
+    take(L.meta_scores, rows * h->m_max * 4);
+    take(L.meta_idx, rows * h->topk_meta * 4);
+    take(L.cand_scores, rows * cap * 4);
+    take(L.cand_ids, rows * cap * 4);
+    take(L.cand_count, rows * 4);
+    take(L.part_h, rows * kHgsaSplitMax * rec);
+  }
+  L.total = off;
+  return L;
+}
+
+inline uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+inline int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+int score_splits(const gsa_desc *d, int head_split, int rows_cap) {
+  const int units = d->batch * d->hkv * head_split;
+  return clampi(cdiv(4 * sm_count(), units), 1, std::min(kScoreSplitMax, cdiv(rows_cap, 64)));
+}
+
+int unfold_splits(const gsa_desc *d) {
+  const int rows = d->batch * d->hq;
+  return clampi(cdiv(4 * sm_count(), rows), 1, std::min(kUnfoldSplitMax, std::max(1, d->topk)));
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// its predecessor drains; it calls griddepcontrol.wait before touching data.
+template <typename Kern, typename Arg>
+gsa_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, void *stream, const Arg &arg) {
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return GSA_OK;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, arg);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GSA_ERR_CUDA;
+  }
+  return GSA_OK;
+}
+
+#define GSA_TRY(x)                     \
+  do {                                 \
+    const gsa_status _s = (x);         \
+    if (_s != GSA_OK) return _s;       \
+  } while (0)
+
+gsa_status need_ptr(const void *p) { return (p && aligned16(p)) ? GSA_OK : GSA_ERR_INVALID_ARG; }
+gsa_status opt_ptr(const void *p) { return (!p || aligned16(p)) ? GSA_OK : GSA_ERR_INVALID_ARG; }
+
+// ---------------------------------------------------------------- scoring
+template <int D, int GH, bool V>
+gsa_status launch_score_mma_t(const ScoreArgs &sa, int splits, int B, void *stream) {
+  using Cfg = ScoreMmaCfg<D, GH, V>;
+  return launch(k_score_mma<D, GH, V>, dim3(splits, sa.hkv * sa.head_split, B), dim3(Cfg::kThreads), Cfg::kSmemBytes,
+                stream, sa);
+}
+
+template <int D, bool V>
+gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dtype, void *stream) {
+  if (dtype == GSA_BF16)
+    return launch(k_score_generic<D, __nv_bfloat16, V>, dim3(splits, sa.hkv, B), dim3(128), 0, stream, sa);
+  return launch(k_score_generic<D, float, V>, dim3(splits, sa.hkv, B), dim3(128), 0, stream, sa);
+}
+
+// Score rows of `keys` (gists or meta-gists) against q; optional partial.
+gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const void *vals, const int32_t *n_gists,
+                     int count_div, int rows_cap, float *scores, int score_stride, float *part, int *splits_out,
+                     uint32_t *status, void *stream) {
+  const int group = d->hq / d->hkv;
+  const bool with_v = part != nullptr;
+  const bool mma = d->dtype == GSA_BF16;
+  const int GH = group <= 4 ? 4 : 8;
+  const int head_split = mma ? cdiv(group, GH) : 1;
+  const int splits = score_splits(d, head_split, rows_cap);
+  if (splits_out) *splits_out = splits;
+  ScoreArgs sa;
+  sa.q = q;
+  sa.gk = keys;
+  sa.gv = vals;
+  sa.n_gists = n_gists;
+  sa.count_div = count_div;
+  sa.rows_cap = rows_cap;
+  sa.scores = scores;
+  sa.score_stride = score_stride;
+  sa.part = part;
+  sa.n_split = splits;
+  sa.status = status;
+  sa.hq = d->hq;
+  sa.hkv = d->hkv;
+  sa.group = group;
+  sa.head_split = head_split;
+  sa.scale = resolve_scale(d);
+  sa.scale_log2 = sa.scale * kLog2e;
+  if (!mma) {
+    if (d->d == 64)
+      return with_v ? launch_score_generic_t<64, true>(sa, splits, d->batch, d->dtype, stream)
+                    : launch_score_generic_t<64, false>(sa, splits, d->batch, d->dtype, stream);
+    return with_v ? launch_score_generic_t<128, true>(sa, splits, d->batch, d->dtype, stream)
+                  : launch_score_generic_t<128, false>(sa, splits, d->batch, d->dtype, stream);
+  }
+#define GSA_SCORE_CASE(DD, GG)                                                                         \
+  if (d->d == DD && GH == GG)                                                                          \
+    return with_v ? launch_score_mma_t<DD, GG, true>(sa, splits, d->batch, stream)                     \
+                  : launch_score_mma_t<DD, GG, false>(sa, splits, d->batch, stream);
+  GSA_SCORE_CASE(64, 4)
+  GSA_SCORE_CASE(64, 8)
+  GSA_SCORE_CASE(128, 4)
+  GSA_SCORE_CASE(128, 8)
+#undef GSA_SCORE_CASE
+  return GSA_ERR_UNSUPPORTED;
+}
+
+gsa_status run_topk(int rows, int hq, const float *scores, int stride, const int32_t *n_gists, int count_div,
+                    const int32_t *counts, int k, const int32_t *id_map, int32_t *sel_idx, float *sel_score,
+                    uint32_t *counters, void *stream) {
+  TopkArgs ta;
+  ta.scores = scores;
+  ta.stride = stride;
+  ta.n_gists = n_gists;
+  ta.count_div = count_div;
+  ta.counts = counts;
+  ta.hq = hq;
+  ta.k = k;
+  ta.id_map = id_map;
+  ta.sel_idx = sel_idx;
+  ta.sel_score = sel_score;
+  ta.counters = counters;
+  ta.smem_cap = std::min(stride, kTopkSmemCap);
+  return launch(k_topk, dim3(rows), dim3(kTopkThreads), static_cast<size_t>(ta.smem_cap) * 4, stream, ta);
+}
+
+template <int D, typename T>
+gsa_status launch_unfold_t(const UnfoldArgs &ua, int B, void *stream) {
+  const int chunk_bytes = ua.chunk * D * static_cast<int>(sizeof(T));
+  const int stages = std::min(8, std::max(2, (96 * 1024) / (2 * chunk_bytes)));
+  return launch(k_unfold<D, T>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads),
+                static_cast<size_t>(stages) * 2 * chunk_bytes, stream, ua);
+}
+
+gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const void *raw_v, const void *gist_v,
+                      const int32_t *n_gists, const int32_t *own_len, const int32_t *sel_idx, const float *sel_score,
+                      const float *prior, int n_prior, void *out, float *lse, const Layout &L, void *ws,
+                      void *stream) {
+  UnfoldArgs ua;
+  ua.q = q;
+  ua.raw_k = raw_k;
+  ua.raw_v = raw_v;
+  ua.gist_v = gist_v;
+  ua.n_gists = n_gists;
+  ua.own_len = own_len;
+  ua.sel_idx = sel_idx;
+  ua.sel_score = sel_score;
+  ua.k = d->topk;
+  ua.chunk = d->chunk;
+  ua.t_max = d->t_max;
+  ua.n_max = d->n_max;
+  ua.hq = d->hq;
+  ua.hkv = d->hkv;
+  ua.group = d->hq / d->hkv;
+  ua.exclude = d->exclude_unselected;
+  ua.scale_log2 = resolve_scale(d) * kLog2e;
+  ua.part = reinterpret_cast<float *>(at(ws, L.part_u));
+  ua.n_split = unfold_splits(d);
+  ua.prior = prior;
+  ua.n_prior = prior ? n_prior : 0;
+  ua.counters = reinterpret_cast<uint32_t *>(at(ws, L.counters));
+  ua.status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  ua.out = out;
+  ua.out_bf16 = d->out_dtype == GSA_BF16;
+  ua.lse = lse;
+  if (d->dtype == GSA_BF16)
+    return d->d == 64 ? launch_unfold_t<64, __nv_bfloat16>(ua, d->batch, stream)
+                      : launch_unfold_t<128, __nv_bfloat16>(ua, d->batch, stream);
+  return d->d == 64 ? launch_unfold_t<64, float>(ua, d->batch, stream) : launch_unfold_t<128, float>(ua, d->batch, stream);
+}
+
+// Number of partial records per row the scoring pass writes for these shapes.
+int gist_prior_count(const gsa_desc *d) {
+  const int group = d->hq / d->hkv;
+  const bool mma = d->dtype == GSA_BF16;
+  const int GH = group <= 4 ? 4 : 8;
+  return score_splits(d, mma ? cdiv(group, GH) : 1, d->n_max);
+}
+
+}  // namespace
+}  // namespace gsa
+
+using namespace gsa;
+
+extern "C" {
+
+const char *gsa_status_string(int32_t s) {
+  switch (s) {
+    case GSA_OK: return "GSA_OK";
+    case GSA_ERR_INVALID_ARG: return "GSA_ERR_INVALID_ARG: invalid argument";
+    case GSA_ERR_UNSUPPORTED: return "GSA_ERR_UNSUPPORTED: configuration not supported";
+    case GSA_ERR_WORKSPACE: return "GSA_ERR_WORKSPACE: workspace too small";
+    case GSA_ERR_CUDA: return "GSA_ERR_CUDA: CUDA runtime error";
+    case GSA_ERR_TIMEOUT: return "GSA_ERR_TIMEOUT: a bounded device wait expired";
+    default: return "unknown gsa_status";
+  }
+}
+
+int32_t gsa_version(void) { return 100; }
+
+size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc) {
+  if (check_desc(desc) != GSA_OK) return 0;
+  if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL) return 0;
+  if (op == GSA_OP_HGSA && check_hdesc(desc, hdesc) != GSA_OK) return 0;
+  return layout(desc, op, hdesc).total;
+}
+
+gsa_status gsa_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!ws || !ws_bytes) return GSA_ERR_INVALID_ARG;
+  return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_workspace_status(void *ws, size_t ws_bytes, void *stream, uint32_t *flags_out) {
+  if (!ws || ws_bytes < 256 || !flags_out) return GSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return GSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return GSA_ERR_CUDA;
+  *flags_out = v;
+  return (v & GSA_DEVERR_TIMEOUT) ? GSA_ERR_TIMEOUT : GSA_OK;
+}
+
+gsa_status gsa_score_gists(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                           const int32_t *n_gists, float *scores, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(scores));
+  GSA_TRY(need_ptr(ws));
+  if (!desc->exclude_unselected) GSA_TRY(need_ptr(gist_v));
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
+  return run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, nullptr,
+                   reinterpret_cast<uint32_t *>(at(ws, L.status)), stream);
+}
+
+gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, int32_t *sel_idx,
+                           float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(need_ptr(scores));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(need_ptr(ws));
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  if (desc->topk == 0) return GSA_OK;
+  return run_topk(desc->batch * desc->hq, desc->hq, scores, desc->n_max, n_gists, 1, nullptr, desc->topk, nullptr,
+                  sel_idx, sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+}
+
+gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *raw_k, const void *raw_v,
+                             const void *gist_v, const int32_t *n_gists, const int32_t *own_len,
+                             const int32_t *sel_idx, const float *sel_score, int32_t prior, void *out, float *lse,
+                             void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(raw_k));
+  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(own_len));
+  GSA_TRY(need_ptr(out));
+  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(need_ptr(ws));
+  if (desc->topk > 0) GSA_TRY(need_ptr(sel_idx));
+  if (desc->exclude_unselected && desc->topk > 0) {
+    GSA_TRY(need_ptr(gist_v));
+    GSA_TRY(need_ptr(sel_score));
+  }
+  if (prior != GSA_PRIOR_NONE && prior != GSA_PRIOR_GISTS && prior != GSA_PRIOR_HGSA) return GSA_ERR_INVALID_ARG;
+  if (prior == GSA_PRIOR_NONE && !desc->exclude_unselected) return GSA_ERR_INVALID_ARG;
+  const int32_t op = prior == GSA_PRIOR_HGSA ? GSA_OP_HGSA : GSA_OP_DECODE;
+  if (op == GSA_OP_HGSA) return GSA_ERR_UNSUPPORTED;  // hgsa partials: see hgsa_select
+  const Layout L = layout(desc, op, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  // The counters must be zero; gsa_topk_select re-arms them, a standalone
+  // call re-arms them here.
+  if (cudaMemsetAsync(at(ws, L.counters), 0, static_cast<size_t>(desc->batch) * desc->hq * 4,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  const float *pr = nullptr;
+  int n_prior = 0;
+  if (prior == GSA_PRIOR_GISTS && !desc->exclude_unselected) {
+    pr = reinterpret_cast<const float *>(at(ws, L.part_g));
+    n_prior = gist_prior_count(desc);
+  }
+  return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, pr, n_prior, out, lse, L,
+                    ws, stream);
+}
+
+gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v, const void *raw_k,
+                      const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
+                      int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(gist_v));
+  GSA_TRY(need_ptr(raw_k));
+  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(own_len));
+  GSA_TRY(need_ptr(out));
+  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(opt_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(need_ptr(ws));
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  float *scores = reinterpret_cast<float *>(at(ws, L.scores));
+  int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
+  float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
+  float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
+  int n_prior = 0;
+  GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
+                    stream));
+  if (desc->topk > 0) {
+    GSA_TRY(run_topk(desc->batch * desc->hq, desc->hq, scores, desc->n_max, n_gists, 1, nullptr, desc->topk, nullptr,
+                     si, ss, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream));
+  } else if (cudaMemsetAsync(at(ws, L.counters), 0, static_cast<size_t>(desc->batch) * desc->hq * 4,
+                             static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return GSA_ERR_CUDA;
+  }
+  return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, part, part ? n_prior : 0, out, lse, L,
+                    ws, stream);
+}
+
+gsa_status hgsa_select(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,
+                       const void *meta_v, const void *gist_k, const void *gist_v, const int32_t *n_gists,
+                       int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
+                       void *stream) {
+  return GSA_ERR_UNSUPPORTED;
+}
+
+gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,
+                       const void *meta_v, const void *gist_k, const void *gist_v, const void *raw_k,
+                       const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
+                       int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
+                       void *stream) {
+  return GSA_ERR_UNSUPPORTED;
+}
+
+gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *k_gist, const void *v_gist,
+                             int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  return GSA_ERR_UNSUPPORTED;
+}
+
+gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
+                              const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,
+                              const float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes,
+                              void *stream) {
+  return GSA_ERR_UNSUPPORTED;
+}
+
+gsa_status gsa_prefill(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
+                       const void *q_gist, const void *k_gist, const void *v_gist, int32_t *sel_idx,
+                       float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes, void *stream) {
+  return GSA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+"""libgsa.so builds for sm_100a, loads, exports every entry point declared in
+include/gsa.h, and rejects bad arguments on the host before any CUDA call.
+CPU only: no kernel is launched here."""
+import ctypes as C
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_gsa_b200 import build, load
+    build.build_library()
+    return load()
+
+
+def declared_functions():
+    text = (ROOT / "include" / "gsa.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/gsa.h but not exported"
+    from long_context_gsa_b200 import EXPORTS
+    assert set(EXPORTS) == set(names)
+
+
+def test_status_strings_and_version(lib):
+    from long_context_gsa_b200 import gsa_status_string, gsa_version
+    assert gsa_status_string(0) == "GSA_OK"
+    assert "workspace" in gsa_status_string(3)
+    assert gsa_version() >= 100
+
+
+def _desc(**kw):
+    """Raw descriptor (no normalisation, so invalid field values reach the C checks)."""
+    from long_context_gsa_b200 import gsa_desc
+    base = dict(batch=2, hq=8, hkv=2, d=128, chunk=16, n_max=64, t_max=64 * 16 + 16, topk=8, exclude_unselected=0,
+                scale=0.0, dtype=1, out_dtype=0)
+    base.update(kw)
+    return gsa_desc(*[base[f] for f, _ in gsa_desc._fields_])
+
+
+def test_workspace_bytes(lib):
+    from long_context_gsa_b200 import GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL, gsa_workspace_bytes, make_hdesc
+    d = _desc()
+    n = gsa_workspace_bytes(d, GSA_OP_DECODE)
+    assert n > 2 * 8 * 64 * 4 and n % 256 == 0
+    assert gsa_workspace_bytes(_desc(d=96), GSA_OP_DECODE) == 0
+    assert gsa_workspace_bytes(_desc(hq=6, hkv=4), GSA_OP_DECODE) == 0
+    h = make_hdesc(4, 4, 16)
+    assert gsa_workspace_bytes(d, GSA_OP_HGSA, h) > n
+    assert gsa_workspace_bytes(d, GSA_OP_HGSA, None) == 0
+    assert gsa_workspace_bytes(_desc(n_max=8, t_max=128, topk=4), GSA_OP_PREFILL) > 0
+
+
+# Fake device addresses are only ever passed to calls that must reject them
+# during host-side validation, before anything is enqueued.  Should a check
+# ever let one through, the call would enqueue work on a bogus address, so
+# these tests never run where a GPU is visible.
+A = 1 << 20  # aligned, never dereferenced
+
+
+def _no_gpu():
+    import torch
+    return not torch.cuda.is_available()
+
+
+cpu_only = pytest.mark.skipif(not _no_gpu(), reason="fake-pointer validation tests run only without a GPU")
+
+
+@cpu_only
+@pytest.mark.parametrize("bad,code", [
+    (dict(d=96), 2), (dict(hq=6, hkv=4), 1), (dict(chunk=0), 2), (dict(topk=-1), 1), (dict(topk=5000), 2),
+    (dict(exclude_unselected=2), 1), (dict(dtype=7), 1), (dict(batch=0), 1), (dict(hq=64, hkv=2), 2),
+])
+def test_bad_descriptor_rejected(lib, bad, code):
+    d = _desc(**bad)
+    st = lib.gsa_decode(C.byref(d), A, A, A, A, A, A, A, A, None, None, None, A, 1 << 40, None)
+    assert st == code
+
+
+@cpu_only
+def test_null_and_misaligned_pointers_rejected(lib):
+    d = _desc()
+    assert lib.gsa_decode(C.byref(d), None, A, A, A, A, A, A, A, None, None, None, A, 1 << 40, None) == 1
+    assert lib.gsa_decode(C.byref(d), A + 4, A, A, A, A, A, A, A, None, None, None, A, 1 << 40, None) == 1
+    assert lib.gsa_score_gists(C.byref(d), A, A, None, A, A, A, 1 << 40, None) == 1  # gist_v needed by default
+    assert lib.gsa_unfold_attend(C.byref(d), A, A, A, None, A, A, A, None, 0, A, None, A, 1 << 40, None) == 1
+
+
+@cpu_only
+def test_small_workspace_rejected(lib):
+    d = _desc()
+    assert lib.gsa_decode(C.byref(d), A, A, A, A, A, A, A, A, None, None, None, A, 1024, None) == 3
+    assert lib.gsa_topk_select(C.byref(d), A, A, A, None, A, 16, None) == 3
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    from long_context_gsa_b200 import gsa_decode
+    d = _desc()
+    t = torch.zeros(4)
+    with pytest.raises((ValueError, TypeError)):
+        gsa_decode(d, t, t, t, t, t, t, t, t, ws=t)

@@ -1,0 +1,160 @@
+"""Flat GSA decode on the GPU (score -> select -> unfold) against the float64
+oracle, through the C ABI.  Needs a B200 and the built libgsa.so."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import check_rows
+
+pytestmark = pytest.mark.gpu
+
+W = None
+G = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    global W, G
+    from long_context_gsa_b200 import build
+    build.build_library()
+    import long_context_gsa_b200 as G_
+    import long_context_gsa_b200.workloads as W_
+    W, G = W_, G_
+    torch.cuda.init()
+
+
+def run_gpu(x, cfg, exclude=None, out_bf16=False, fused=True):
+    dev = x["q"].device
+    B, hq, d = x["q"].shape
+    hkv, n_max, t_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2]
+    dt = G.GSA_BF16 if x["q"].dtype == torch.bfloat16 else G.GSA_F32
+    excl = cfg.exclude if exclude is None else exclude
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, excl, 0.0, dt,
+                       G.GSA_BF16 if out_bf16 else G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=dev)
+    lse = torch.empty((B, hq), dtype=torch.float32, device=dev)
+    k = max(cfg.topk, 1)
+    sel = torch.full((B, hq, k), -7, dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, k), dtype=torch.float32, device=dev)
+    scores = None
+    if fused:
+        G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
+                     out, lse, sel if cfg.topk else None, ssc if cfg.topk else None, ws)
+    else:
+        scores = torch.full((B, hq, n_max), float("nan"), dtype=torch.float32, device=dev)
+        G.gsa_score_gists(desc, x["q"], x["gist_k"], None if excl else x["gist_v"], x["n_gists"], scores, ws)
+        if cfg.topk:
+            G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"],
+                            sel if cfg.topk else None, ssc if cfg.topk else None,
+                            G.GSA_PRIOR_NONE if excl else G.GSA_PRIOR_GISTS, out, lse, ws)
+    torch.cuda.synchronize()
+    flags = G.gsa_workspace_status(ws)
+    assert flags == 0, f"device status flags {flags:#x}"
+    return out, lse, (sel if cfg.topk else torch.full((B, hq, 0), -1, dtype=torch.int32)), ssc, scores
+
+
+def run_oracle(x, cfg, exclude=None, rows=None, sel_in=None):
+    o = oracle.get()
+    tk = W.to_oracle
+    excl = cfg.exclude if exclude is None else exclude
+    return o.decode(tk(x["q"]), tk(x["gist_k"]), tk(x["gist_v"]), tk(x["raw_k"]), tk(x["raw_v"]), tk(x["n_gists"]),
+                    tk(x["own_len"]), chunk=cfg.chunk, topk=cfg.topk, exclude=excl, rows=rows, sel_in=sel_in,
+                    want_scores=True)
+
+
+def compare(x, cfg, exclude=None, out_bf16=False, rows=None, fused=True, what=""):
+    out, lse, sel, ssc, scores = run_gpu(x, cfg, exclude, out_bf16, fused)
+    B, hq, d = x["q"].shape
+    all_rows = np.arange(B * hq) if rows is None else np.asarray(rows)
+    orc = run_oracle(x, cfg, exclude, rows=all_rows)
+    g_out = out.float().reshape(B * hq, d).cpu().numpy()[all_rows]
+    g_sel = sel.reshape(B * hq, -1).cpu().numpy()[all_rows]
+
+    def rerun(slots, forced):
+        return run_oracle(x, cfg, exclude, rows=all_rows[slots], sel_in=forced)
+
+    dtype = "bf16" if x["q"].dtype == torch.bfloat16 else "f32"
+    res = check_rows(g_out, g_sel, orc, orc["scores"], cfg.topk, dtype, out_bf16, rerun, what)
+    g_lse = lse.reshape(-1).cpu().numpy()[all_rows]
+    ok = np.isfinite(orc["lse"])
+    assert np.allclose(g_lse[ok], orc["lse"][ok], atol=1e-3 if dtype == "bf16" else 1e-5)
+    if scores is not None:
+        sc = scores.reshape(B * hq, -1).cpu().numpy()[all_rows]
+        valid = ~np.isnan(orc["scores"])
+        assert np.nanmax(np.abs(sc[valid] - orc["scores"][valid])) < (1e-3 if dtype == "bf16" else 1e-5)
+    return res, g_sel
+
+
+SMALL = [
+    # name, cfg changes, n_max extra, ragged counts, own_len
+    ("g7_d128_c16", dict(batch=2, hq=28, hkv=4, d=128, chunk=16, context=1000 * 16, topk=32), [1000, 617], 16),
+    ("g4_d64_c8", dict(batch=2, hq=32, hkv=8, d=64, chunk=8, context=700 * 8, topk=64), [700, 700], 1),
+    ("g16_d128", dict(batch=1, hq=16, hkv=1, d=128, chunk=16, context=333 * 16, topk=16), None, 5),
+    ("g1_d64", dict(batch=2, hq=4, hkv=4, d=64, chunk=8, context=200 * 8, topk=8), [200, 150], 3),
+    ("n_below_k", dict(batch=1, hq=8, hkv=2, d=128, chunk=16, context=20 * 16, topk=64), None, 7),
+    ("k0", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, context=50 * 8, topk=0), None, 2),
+    ("c32_full_own", dict(batch=1, hq=8, hkv=2, d=128, chunk=32, context=300 * 32, topk=24), None, 32),
+    ("n0", dict(batch=2, hq=4, hkv=2, d=64, chunk=8, context=40 * 8, topk=4), [0, 40], 2),
+    ("big_k", dict(batch=1, hq=4, hkv=1, d=64, chunk=4, context=3000 * 4, topk=700), None, 2),
+]
+
+
+@pytest.mark.parametrize("name,chg,ragged,own", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_small_bf16(name, chg, ragged, own, exclude):
+    cfg = W.scaled(W.QWEN_16X, kv_std=1.0, **chg)
+    x = W.decode_inputs(cfg, device="cuda", own_len=own, ragged=ragged, seed=hash(name) % 100000)
+    compare(x, cfg, exclude=exclude, what=name)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_small_f32(d):
+    cfg = W.scaled(W.PR1, batch=2, hq=4, hkv=2, d=d, chunk=16, context=300 * 16, topk=12, dtype="f32")
+    x = W.decode_inputs(cfg, device="cuda", own_len=9, ragged=[300, 211])
+    compare(x, cfg, exclude=False, what=f"f32 d={d}")
+    compare(x, cfg, exclude=True, what=f"f32 d={d} exclude")
+
+
+def test_bf16_output():
+    cfg = W.scaled(W.LLAMA_8X, batch=2, context=512 * 8)
+    x = W.decode_inputs(cfg, device="cuda", own_len=4)
+    compare(x, cfg, out_bf16=True, what="bf16 out")
+
+
+def test_separate_entry_points_match_fused():
+    cfg = W.scaled(W.QWEN_16X, batch=2, context=900 * 16, kv_std=1.0)
+    x = W.decode_inputs(cfg, device="cuda", own_len=6)
+    for excl in (False, True):
+        a = run_gpu(x, cfg, excl, fused=True)
+        b = run_gpu(x, cfg, excl, fused=False)
+        assert torch.equal(a[2], b[2])
+        assert torch.equal(a[0], b[0])
+    compare(x, cfg, fused=False, what="separate calls")
+
+
+def test_pr1_all_steps():
+    """The tiny fp32 single-head workload: every one of its 64 decode steps."""
+    static, steps = W.pr1_steps(device="cuda")
+    cfg = W.PR1
+    hits = 0
+    for s, st in enumerate(steps):
+        x = dict(static, q=st["q"], n_gists=st["n_gists"], own_len=st["own_len"])
+        _, sel = compare(x, cfg, what=f"pr1 step {s}")
+        hits += len(set(sel[0].tolist()) & set(static["planted"].tolist()))
+    assert hits / (8 * len(steps)) > 0.9
+
+
+@pytest.mark.parametrize("name", ["llama1b_8x", "qwen7b_16x", "qwen7b_16x_excl"])
+def test_full_size(name):
+    """Full-size workloads; every row is checked (the oracle needs seconds here)."""
+    cfg = W.CONFIGS[name]
+    x = W.decode_inputs(cfg, device="cuda")
+    res, sel = compare(x, cfg, what=name)
+    planted = x["planted"].reshape(-1).numpy()
+    recall = np.mean([planted[r] in set(sel[r].tolist()) for r in range(len(planted))])
+    assert recall > 0.9, recall
+    print(name, res, "planted recall", recall)
