@@ -174,6 +174,34 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
                       const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
                       int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
 
+/* Scratch-free decode step.  The paper has no counterpart: this is a
+ * deployment variant of gsa_decode for callers that cannot allocate device
+ * memory -- for instance a plugin or FFI host that hands over only input
+ * and output pointers and exposes no allocator, or a latency-critical
+ * caller that must not call cudaMalloc because it may synchronise the
+ * device.  It computes exactly what gsa_decode computes, with the same
+ * arguments except that there is no `ws`: the workspace is carved from a
+ * file-scope device array of GSA_NOALLOC_SCRATCH_BYTES bytes inside
+ * libgsa.so, which every GPU that loads the library keeps until the
+ * process exits.
+ *  * The first call on a device looks up that array's device address
+ *    (once per device, with the device current); make that first call
+ *    before any stream capture.
+ *  * Problems whose workspace (gsa_workspace_bytes(desc, GSA_OP_DECODE,
+ *    NULL)) exceeds GSA_NOALLOC_SCRATCH_BYTES are rejected with
+ *    GSA_ERR_WORKSPACE before anything is enqueued.
+ *  * No cudaMalloc/cudaFree or allocating library routine is called; the
+ *    call enqueues a small cudaMemsetAsync that clears the status word and
+ *    per-row counters, then the decode kernels.
+ *  * All calls in the process share the one array and it keeps the last
+ *    call's contents: calls whose GPU work may overlap (different streams
+ *    without ordering, or several host threads) race and corrupt each
+ *    other's results.  Order them on one stream. */
+#define GSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                              const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
+                              void *out, float *lse, int32_t *sel_idx, float *sel_score, void *stream);
+
 /* ---- H-GSA decode: one meta level ([ja] 2.2; [nl] Hierarchische
  * Uitbreiding) -------------------------------------------------------- */
 

@@ -25,7 +25,7 @@ GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
 EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select", "hgsa_decode",
-    "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
+    "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill", "gsa_decode_noalloc",
 )
 
 
@@ -76,6 +76,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_prefill_score": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_decode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
     }
     for name, (argt, rest) in sig.items():
         fn = getattr(lib, name)
@@ -255,3 +256,17 @@ def gsa_prefill(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, out_raw, out_
         _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist"),
         _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True),
         _ptr(out_raw, odt, "out_raw"), _ptr(out_gist, odt, "out_gist"), p, n, _stream(stream)))
+
+
+def gsa_decode_noalloc(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None, sel_idx=None,
+                       sel_score=None, stream=None):
+    """gsa_decode without a workspace argument (the library's built-in
+    scratch array is used; see include/gsa.h for its limit and the rule
+    that calls must not overlap on the GPU)."""
+    dt = _TORCH_DT[desc.dtype]
+    _check("gsa_decode_noalloc", load().gsa_decode_noalloc(
+        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
+        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(own_len, torch.int32, "own_len"), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
+        _ptr(lse, torch.float32, "lse", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
+        _ptr(sel_score, torch.float32, "sel_score", True), _stream(stream)))

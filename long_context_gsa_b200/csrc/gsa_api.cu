@@ -479,3 +479,66 @@ gsa_status gsa_prefill(const gsa_desc *desc, const void *q_raw, const void *k_ra
 }
 
 }  // extern "C"
+
+// ---- Scratch-free decode (gsa_decode_noalloc) ------------------------------
+// For callers that cannot allocate device memory: the workspace gsa_decode
+// needs lives in a file-scope device array instead of a caller buffer.
+#include <mutex>
+
+namespace gsa {
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[GSA_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocSlot {
+  std::once_flag once;
+  void *ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+constexpr int kNoallocMaxDevices = 64;
+NoallocSlot g_noalloc_slots[kNoallocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a stand-in; the real address is looked up once
+// per device, with that device current.
+gsa_status noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GSA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return GSA_ERR_UNSUPPORTED;
+  NoallocSlot &s = g_noalloc_slots[dev];
+  std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_noalloc_scratch); });
+  if (s.err != cudaSuccess || s.ptr == nullptr) return GSA_ERR_CUDA;
+  *out = s.ptr;
+  return GSA_OK;
+}
+
+}  // namespace
+}  // namespace gsa
+
+extern "C" gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                                         const void *raw_k, const void *raw_v, const int32_t *n_gists,
+                                         const int32_t *own_len, void *out, float *lse, int32_t *sel_idx,
+                                         float *sel_score, void *stream) {
+  GSA_TRY(check_desc(desc));
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
+  if (L.total > GSA_NOALLOC_SCRATCH_BYTES) return GSA_ERR_WORKSPACE;
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(gist_v));
+  GSA_TRY(need_ptr(raw_k));
+  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(own_len));
+  GSA_TRY(need_ptr(out));
+  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(opt_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  void *ws = nullptr;
+  GSA_TRY(noalloc_scratch(&ws));
+  // The status word and the per-row counters must start at zero; the array
+  // keeps whatever the previous call left there.
+  const size_t zero_bytes = L.counters + static_cast<size_t>(desc->batch) * desc->hq * 4;
+  if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GSA_ERR_CUDA;
+  return gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score, ws,
+                    GSA_NOALLOC_SCRATCH_BYTES, stream);
+}
