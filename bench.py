@@ -7,8 +7,9 @@ unfold + attend) for the whole batch of the workload, through the C ABI of
 libgsa.so.  The default workload is the Llama-3.2-1B-shaped decode at 8x
 compression (16 sequences x 32 query heads / 8 kv heads, d=64, 32K raw
 context, chunk 8 -> 4096 gists, top-64).  Inputs are seeded synthetic
-tensors resident in HBM; L2 is flushed (a 2x-L2 buffer is written) between
-timed steps and the flush is outside the timed events.
+tensors resident in HBM; L2 is flushed between timed steps (a 2x-L2 buffer
+is written, then another 2x-L2 buffer is read so the dirty lines are written
+back before the step) and the flush is outside the timed events.
 
 With --gpus N (launched under torch.distributed.run) every rank runs its own
 batch (different seed): decode rows are independent, so the work shards with
@@ -198,7 +199,20 @@ def run_gsa(args, world, rank, local):
     ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
     scores = torch.empty((B, hq, n_max), dtype=torch.float32, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.int32, device=dev)
+
+    class _Flush:
+        """Write a 2x-L2 buffer, then read another one so that the written
+        lines are evicted (written back) before the next timed step starts."""
+
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.amax(flush_r, dim=0, out=flush_sink)
+
+    flush = _Flush()
     stream = torch.cuda.current_stream()
     prior = G.GSA_PRIOR_NONE if cfg.exclude else G.GSA_PRIOR_GISTS
 
@@ -292,7 +306,7 @@ def run_gsa(args, world, rank, local):
             "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "batch_per_gpu": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv, "d": cfg.d,
                        "context": cfg.context, "chunk": cfg.chunk, "n_gists": cfg.n_gists, "topk": cfg.topk,
-                       "exclude_unselected": cfg.exclude, "l2": "flushed between timed steps (2x L2 buffer written)",
+                       "exclude_unselected": cfg.exclude, "l2": "flushed between timed steps (2x-L2 buffer written, then another 2x-L2 buffer read so no dirty lines remain)",
                        "parallelism": f"dp{world} (independent rows per GPU)"},
             "roofline": roof,
             "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(step_gbs, 1),

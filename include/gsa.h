@@ -39,8 +39,9 @@
  *  * Scores and logits are scale * q.k with scale = 1/sqrt(d) unless
  *    desc->scale > 0.  All accumulation is fp32.
  *  * Selection per (b, h): the min(topk, N) chunks of highest score, ties
- *    to the lower chunk index ([nl] Selectie); sel_idx rows are sorted by
- *    (score desc, index asc) and padded with -1 (sel_score with -inf).
+ *    to the lower chunk index ([nl] Selectie); sel_idx rows list the chosen
+ *    chunks in ascending chunk order, padded with -1 (sel_score, the
+ *    chunk's score, with -inf).
  *  * Attended set per (b, h) ([ja] 2.1 steps 3-4, [nl] Selectieve
  *    Ontvouwing): for each selected chunk its `chunk` raw tokens and its
  *    gist token; each unselected chunk's gist token unless
@@ -84,7 +85,7 @@ typedef enum gsa_prior {
 typedef enum gsa_op { GSA_OP_DECODE = 0, GSA_OP_HGSA = 1, GSA_OP_PREFILL = 2 } gsa_op;
 
 /* Device-side status bits (gsa_workspace_status). */
-#define GSA_DEVERR_BAD_INDEX 0x1u /* a sel_idx entry outside [0, N) or repeated was skipped */
+#define GSA_DEVERR_BAD_INDEX 0x1u /* a sel_idx entry >= N was skipped */
 #define GSA_DEVERR_TIMEOUT 0x2u   /* an mbarrier wait exceeded its iteration bound */
 #define GSA_DEVERR_CAPACITY 0x4u  /* a count exceeded a capacity and was clamped */
 
@@ -161,8 +162,9 @@ gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int3
  *                 gist's logit is its score, so gist keys are not re-read)
  *   prior         which partial result ws holds (gsa_prior)
  *   out           [B, hq, d] in out_dtype; lse [B, hq] fp32 or NULL
- * Selected entries that are -1 are skipped; entries >= N or repeated are
- * skipped and flagged (GSA_DEVERR_BAD_INDEX). */
+ * Selected entries that are negative are skipped; entries >= N are skipped
+ * and flagged (GSA_DEVERR_BAD_INDEX).  A chunk listed twice is attended
+ * twice (the selection calls never list one twice). */
 gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *raw_k, const void *raw_v,
                              const void *gist_v, const int32_t *n_gists, const int32_t *own_len,
                              const int32_t *sel_idx, const float *sel_score, int32_t prior, void *out, float *lse,

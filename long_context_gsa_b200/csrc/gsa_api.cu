@@ -11,6 +11,7 @@
 
 #include "../../include/gsa.h"
 #include "common.cuh"
+#include "k_hgsa.cuh"
 #include "k_score.cuh"
 #include "k_topk.cuh"
 #include "k_unfold.cuh"
@@ -114,14 +115,29 @@ int sm_count() {
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 inline int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
-int score_splits(const gsa_desc *d, int head_split, int rows_cap) {
-  const int units = d->batch * d->hkv * head_split;
-  return clampi(cdiv(4 * sm_count(), units), 1, std::min(kScoreSplitMax, cdiv(rows_cap, 64)));
+// Allow `smem` bytes of dynamic shared memory for `kern` (needed above 48 KB).
+template <typename Kern>
+bool prepare(Kern kern, size_t smem) {
+  return smem <= 48 * 1024 ||
+         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+             cudaSuccess;
 }
 
-int unfold_splits(const gsa_desc *d) {
-  const int rows = d->batch * d->hq;
-  return clampi(cdiv(4 * sm_count(), rows), 1, std::min(kUnfoldSplitMax, std::max(1, d->topk)));
+// CTAs of `kern` that fit on the whole GPU at once.
+template <typename Kern>
+int resident_ctas(Kern kern, int threads, size_t smem) {
+  int per_sm = 0;
+  if (!prepare(kern, smem) ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return per_sm * sm_count();
+}
+
+// Splits per unit so that all CTAs fit in one wave (at least one split).
+inline int one_wave_splits(int units, int slots, int max_splits) {
+  return clampi(slots / std::max(units, 1), 1, std::max(1, max_splits));
 }
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -129,9 +145,7 @@ int unfold_splits(const gsa_desc *d) {
 template <typename Kern, typename Arg>
 gsa_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, void *stream, const Arg &arg) {
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return GSA_OK;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return GSA_ERR_CUDA;
+  if (!prepare(kern, smem)) return GSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -167,6 +181,40 @@ gsa_status launch_score_mma_t(const ScoreArgs &sa, int splits, int B, void *stre
                 stream, sa);
 }
 
+template <int D, int GH, bool V>
+int score_mma_slots() {
+  using Cfg = ScoreMmaCfg<D, GH, V>;
+  return resident_ctas(k_score_mma<D, GH, V>, Cfg::kThreads, Cfg::kSmemBytes);
+}
+
+struct ScorePlan {
+  bool mma;
+  int GH, head_split, splits;
+};
+
+// How the scoring pass is cut: CTAs over (row slices, kv head [x head
+// half], batch), as many slices as fit the GPU in one wave.
+ScorePlan plan_score(const gsa_desc *d, int rows_cap, bool with_v) {
+  ScorePlan p;
+  const int group = d->hq / d->hkv;
+  p.mma = d->dtype == GSA_BF16;
+  p.GH = group <= 4 ? 4 : 8;
+  p.head_split = p.mma ? cdiv(group, p.GH) : 1;
+  int slots;
+  if (!p.mma) {
+    slots = 4 * sm_count();
+  } else if (d->d == 64) {
+    slots = p.GH == 4 ? (with_v ? score_mma_slots<64, 4, true>() : score_mma_slots<64, 4, false>())
+                      : (with_v ? score_mma_slots<64, 8, true>() : score_mma_slots<64, 8, false>());
+  } else {
+    slots = p.GH == 4 ? (with_v ? score_mma_slots<128, 4, true>() : score_mma_slots<128, 4, false>())
+                      : (with_v ? score_mma_slots<128, 8, true>() : score_mma_slots<128, 8, false>());
+  }
+  p.splits = one_wave_splits(d->batch * d->hkv * p.head_split, slots,
+                             std::min(kScoreSplitMax, cdiv(rows_cap, 64)));
+  return p;
+}
+
 template <int D, bool V>
 gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dtype, void *stream) {
   if (dtype == GSA_BF16)
@@ -180,10 +228,11 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
                      uint32_t *status, void *stream) {
   const int group = d->hq / d->hkv;
   const bool with_v = part != nullptr;
-  const bool mma = d->dtype == GSA_BF16;
-  const int GH = group <= 4 ? 4 : 8;
-  const int head_split = mma ? cdiv(group, GH) : 1;
-  const int splits = score_splits(d, head_split, rows_cap);
+  const ScorePlan plan = plan_score(d, rows_cap, with_v);
+  const bool mma = plan.mma;
+  const int GH = plan.GH;
+  const int head_split = plan.head_split;
+  const int splits = plan.splits;
   if (splits_out) *splits_out = splits;
   ScoreArgs sa;
   sa.q = q;
@@ -238,15 +287,26 @@ gsa_status run_topk(int rows, int hq, const float *scores, int stride, const int
   ta.sel_score = sel_score;
   ta.counters = counters;
   ta.smem_cap = std::min(stride, kTopkSmemCap);
-  return launch(k_topk, dim3(rows), dim3(kTopkThreads), static_cast<size_t>(ta.smem_cap) * 4, stream, ta);
+  const dim3 grid(rows), block(kTopkRegThreads);
+  if (stride <= 4 * kTopkRegThreads) return launch(k_topk<4>, grid, block, 0, stream, ta);
+  if (stride <= 16 * kTopkRegThreads) return launch(k_topk<16>, grid, block, 0, stream, ta);
+  if (stride <= 32 * kTopkRegThreads) return launch(k_topk<32>, grid, block, 0, stream, ta);
+  if (stride <= 64 * kTopkRegThreads) return launch(k_topk<64>, grid, block, 0, stream, ta);
+  return launch(k_topk_mem, grid, dim3(kTopkThreads), static_cast<size_t>(ta.smem_cap) * 4, stream, ta);
 }
 
 template <int D, typename T>
-gsa_status launch_unfold_t(const UnfoldArgs &ua, int B, void *stream) {
-  const int chunk_bytes = ua.chunk * D * static_cast<int>(sizeof(T));
-  const int stages = std::min(8, std::max(2, (96 * 1024) / (2 * chunk_bytes)));
-  return launch(k_unfold<D, T>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads),
-                static_cast<size_t>(stages) * 2 * chunk_bytes, stream, ua);
+size_t unfold_smem(int chunk) {
+  const int piece_bytes = unfold_piece_rows<D, T>(chunk) * D * static_cast<int>(sizeof(T));
+  return static_cast<size_t>(kUnfoldWarps) * unfold_warp_stages(2 * piece_bytes) * 2 * piece_bytes;
+}
+
+template <int D, typename T>
+gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
+  const size_t smem = unfold_smem<D, T>(ua.chunk);
+  const int slots = resident_ctas(k_unfold<D, T>, kUnfoldThreads, smem);
+  ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));
+  return launch(k_unfold<D, T>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads), smem, stream, ua);
 }
 
 gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const void *raw_v, const void *gist_v,
@@ -272,7 +332,7 @@ gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const
   ua.exclude = d->exclude_unselected;
   ua.scale_log2 = resolve_scale(d) * kLog2e;
   ua.part = reinterpret_cast<float *>(at(ws, L.part_u));
-  ua.n_split = unfold_splits(d);
+  ua.n_split = 1;  // set by launch_unfold_t
   ua.prior = prior;
   ua.n_prior = prior ? n_prior : 0;
   ua.counters = reinterpret_cast<uint32_t *>(at(ws, L.counters));
@@ -286,13 +346,76 @@ gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const
   return d->d == 64 ? launch_unfold_t<64, float>(ua, d->batch, stream) : launch_unfold_t<128, float>(ua, d->batch, stream);
 }
 
-// Number of partial records per row the scoring pass writes for these shapes.
-int gist_prior_count(const gsa_desc *d) {
-  const int group = d->hq / d->hkv;
-  const bool mma = d->dtype == GSA_BF16;
-  const int GH = group <= 4 ? 4 : 8;
-  return score_splits(d, mma ? cdiv(group, GH) : 1, d->n_max);
+// Splits per row of the H-GSA candidate pass; depends on the descriptor only
+// (gsa_unfold_attend needs it without the H-GSA parameters).
+int hgsa_splits(const gsa_desc *d) {
+  return one_wave_splits(d->batch * d->hq, 4 * sm_count(), kHgsaSplitMax);
 }
+
+template <int D, typename T>
+gsa_status launch_hgsa_children_t(const HgsaArgs &ha, int B, void *stream) {
+  const int piece_bytes = unfold_piece_rows<D, T>(ha.group) * D * static_cast<int>(sizeof(T));
+  const size_t smem = static_cast<size_t>(kHgsaWarps) * unfold_warp_stages(2 * piece_bytes) * 2 * piece_bytes;
+  return launch(k_hgsa_children<D, T>, dim3(ha.n_split, ha.hq, B), dim3(kHgsaThreads), smem, stream, ha);
+}
+
+gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q, const void *meta_k,
+                           const void *meta_v, const void *gist_k, const void *gist_v, const int32_t *n_gists,
+                           int32_t *meta_idx, int32_t *sel_idx, float *sel_score, const Layout &L, void *ws,
+                           void *stream) {
+  const int rows = d->batch * d->hq;
+  uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  float *meta_scores = reinterpret_cast<float *>(at(ws, L.meta_scores));
+  // 1. meta-gist scores; 2. top meta groups (ascending group order)
+  GSA_TRY(run_score(d, q, meta_k, nullptr, n_gists, hd->group, hd->m_max, meta_scores, hd->m_max, nullptr, nullptr,
+                    status, stream));
+  GSA_TRY(run_topk(rows, d->hq, meta_scores, hd->m_max, n_gists, hd->group, nullptr, hd->topk_meta, nullptr, meta_idx,
+                   nullptr, nullptr, stream));
+  // 3. children of the chosen groups (+ trailing gists): scores, ids, partial
+  HgsaArgs ha;
+  ha.q = q;
+  ha.gist_k = gist_k;
+  ha.gist_v = gist_v;
+  ha.meta_v = meta_v;
+  ha.meta_scores = meta_scores;
+  ha.meta_idx = meta_idx;
+  ha.n_gists = n_gists;
+  ha.group = hd->group;
+  ha.topk_meta = hd->topk_meta;
+  ha.m_max = hd->m_max;
+  ha.n_max = d->n_max;
+  ha.hq = d->hq;
+  ha.hkv = d->hkv;
+  ha.gqa = d->hq / d->hkv;
+  ha.exclude = d->exclude_unselected;
+  ha.scale_log2 = resolve_scale(d) * kLog2e;
+  ha.cand_scores = reinterpret_cast<float *>(at(ws, L.cand_scores));
+  ha.cand_ids = reinterpret_cast<int32_t *>(at(ws, L.cand_ids));
+  ha.cand_count = reinterpret_cast<int32_t *>(at(ws, L.cand_count));
+  ha.cap = hgsa_cand_cap(hd);
+  ha.part = reinterpret_cast<float *>(at(ws, L.part_g));
+  ha.n_split = hgsa_splits(d);
+  ha.status = status;
+  gsa_status st;
+  if (d->dtype == GSA_BF16)
+    st = d->d == 64 ? launch_hgsa_children_t<64, __nv_bfloat16>(ha, d->batch, stream)
+                    : launch_hgsa_children_t<128, __nv_bfloat16>(ha, d->batch, stream);
+  else
+    st = d->d == 64 ? launch_hgsa_children_t<64, float>(ha, d->batch, stream)
+                    : launch_hgsa_children_t<128, float>(ha, d->batch, stream);
+  GSA_TRY(st);
+  // 4. top gists among the candidates, reported as gist (chunk) ids
+  if (d->topk > 0)
+    return run_topk(rows, d->hq, ha.cand_scores, ha.cap, nullptr, 1, ha.cand_count, d->topk, ha.cand_ids, sel_idx,
+                    sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+  return cudaMemsetAsync(at(ws, L.counters), 0, static_cast<size_t>(rows) * 4, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GSA_OK
+             : GSA_ERR_CUDA;
+}
+
+// Number of partial records per row the scoring pass writes for these shapes.
+int gist_prior_count(const gsa_desc *d) { return plan_score(d, d->n_max, true).splits; }
 
 }  // namespace
 }  // namespace gsa
@@ -389,9 +512,7 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
   }
   if (prior != GSA_PRIOR_NONE && prior != GSA_PRIOR_GISTS && prior != GSA_PRIOR_HGSA) return GSA_ERR_INVALID_ARG;
   if (prior == GSA_PRIOR_NONE && !desc->exclude_unselected) return GSA_ERR_INVALID_ARG;
-  const int32_t op = prior == GSA_PRIOR_HGSA ? GSA_OP_HGSA : GSA_OP_DECODE;
-  if (op == GSA_OP_HGSA) return GSA_ERR_UNSUPPORTED;  // hgsa partials: see hgsa_select
-  const Layout L = layout(desc, op, nullptr);
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);  // the H-GSA layout extends this one
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
   // The counters must be zero; gsa_topk_select re-arms them, a standalone
   // call re-arms them here.
@@ -403,6 +524,9 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
   if (prior == GSA_PRIOR_GISTS && !desc->exclude_unselected) {
     pr = reinterpret_cast<const float *>(at(ws, L.part_g));
     n_prior = gist_prior_count(desc);
+  } else if (prior == GSA_PRIOR_HGSA && !desc->exclude_unselected) {
+    pr = reinterpret_cast<const float *>(at(ws, L.part_g));
+    n_prior = hgsa_splits(desc);
   }
   return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, pr, n_prior, out, lse, L,
                     ws, stream);
@@ -449,7 +573,26 @@ gsa_status hgsa_select(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
                        const void *meta_v, const void *gist_k, const void *gist_v, const int32_t *n_gists,
                        int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
                        void *stream) {
-  return GSA_ERR_UNSUPPORTED;
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(check_hdesc(desc, hdesc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(meta_k));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(meta_idx));
+  GSA_TRY(need_ptr(ws));
+  if (desc->topk > 0) {
+    GSA_TRY(need_ptr(sel_idx));
+    GSA_TRY(need_ptr(sel_score));
+  }
+  if (!desc->exclude_unselected) {
+    GSA_TRY(need_ptr(meta_v));
+    GSA_TRY(need_ptr(gist_v));
+  }
+  const Layout L = layout(desc, GSA_OP_HGSA, hdesc);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  return run_hgsa_select(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, n_gists, meta_idx, sel_idx, sel_score, L,
+                         ws, stream);
 }
 
 gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,
@@ -457,7 +600,32 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
                        const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
                        int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
                        void *stream) {
-  return GSA_ERR_UNSUPPORTED;
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(check_hdesc(desc, hdesc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(meta_k));
+  GSA_TRY(need_ptr(meta_v));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(gist_v));
+  GSA_TRY(need_ptr(raw_k));
+  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(own_len));
+  GSA_TRY(need_ptr(out));
+  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(opt_ptr(meta_idx));
+  GSA_TRY(opt_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(need_ptr(ws));
+  const Layout L = layout(desc, GSA_OP_HGSA, hdesc);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  int32_t *mi = meta_idx ? meta_idx : reinterpret_cast<int32_t *>(at(ws, L.meta_idx));
+  int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
+  float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
+  GSA_TRY(run_hgsa_select(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, n_gists, mi, si, ss, L, ws, stream));
+  const float *pr = desc->exclude_unselected ? nullptr : reinterpret_cast<const float *>(at(ws, L.part_g));
+  return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, pr, pr ? hgsa_splits(desc) : 0, out, lse,
+                    L, ws, stream);
 }
 
 gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *k_gist, const void *v_gist,

@@ -56,32 +56,53 @@ template <int D, int GH, bool WITH_V>
 struct ScoreMmaCfg {
   static constexpr int kThreads = 256;
   static constexpr int kTile = 64;
-  static constexpr int kStages = 3;
+  static constexpr int kStages = D == 64 ? 4 : 3;
   static constexpr uint32_t kTileBytes = kTile * D * 2;
   static constexpr uint32_t kStageBytes = kTileBytes * (WITH_V ? 2 : 1);
+  // stages | p tiles [2][kTile][GH] | per-warp maxima [8][GH] | reference max [GH] | query fragments
+  // [D/16][32 lanes] x uint2 | flags | barriers
   static constexpr uint32_t kSmemBytes =
-      kStages * kStageBytes + (GH * kTile + kTile * GH + 3 * GH) * 4 + kStages * 8 + 64;
+      kStages * kStageBytes + (2 * kTile * GH + 8 * GH + GH) * 4 + (D / 16) * 32 * 8 + 16 + kStages * 8 + 64;
 };
+
+// Rescaling threshold (base-2 units): the running max used for the
+// exponentials is only raised when a score exceeds it by more than this,
+// so p <= 2^8 and the rescale of the accumulators is rare.  Numerator and
+// denominator use the same reference, so the result is unchanged.
+constexpr float kRescaleSlack = 8.0f;
+
+// (acc.x, acc.y) += p * (v.x, v.y) with one packed fp32x2 FMA.
+__device__ __forceinline__ void fma2(float &ax, float &ay, float p, float vx, float vy) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rb, {%2, %3};\n\t"
+      "mov.b64 rc, {%4, %4};\n\t"
+      "fma.rn.f32x2 ra, rc, rb, ra;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(ax), "+f"(ay)
+      : "f"(vx), "f"(vy), "f"(p));
+}
 
 // bf16 inputs, D in {64, 128}, up to GH (4 or 8) query heads per CTA.
 template <int D, int GH, bool WITH_V>
-__global__ void __launch_bounds__(256, 1) k_score_mma(const ScoreArgs a) {
+__global__ void __launch_bounds__(256, 2) k_score_mma(const ScoreArgs a) {
   using Cfg = ScoreMmaCfg<D, GH, WITH_V>;
   constexpr int kTile = Cfg::kTile, kStages = Cfg::kStages;
   constexpr int kLpr = D / 8, kRpw = 32 / kLpr, kSlots = 8 * kRpw;
   extern __shared__ __align__(128) uint8_t smem[];
-  float *s_tile = reinterpret_cast<float *>(smem + kStages * Cfg::kStageBytes);
-  float *p_tile = s_tile + GH * kTile;
-  float *alpha_s = p_tile + kTile * GH;
-  float *m_s = alpha_s + GH;
-  float *l_s = m_s + GH;
-  uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(l_s + GH) + 7) & ~uintptr_t(7));
+  float *p_tile = reinterpret_cast<float *>(smem + kStages * Cfg::kStageBytes);  // [2][kTile][GH]
+  float *wmax = p_tile + 2 * kTile * GH;                                         // [8][GH]
+  float *m_sh = wmax + 8 * GH;                                                    // [GH] reference max
+  uint2 *af_sh = reinterpret_cast<uint2 *>(m_sh + GH);                            // [D/16][32]
+  int *flags = reinterpret_cast<int *>(af_sh + (D / 16) * 32);                    // [0] abort
+  uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(flags + 4) + 7) & ~uintptr_t(7));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.z;
   const int kvh = blockIdx.y / a.head_split, hpart = blockIdx.y % a.head_split;
   const int h0 = kvh * a.group + hpart * GH;
   const int nh = min(GH, a.group - hpart * GH);
+  const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates: head row g, gist pair t4
 
   pdl_wait();
   int N = a.n_gists[b] / a.count_div;
@@ -97,10 +118,21 @@ __global__ void __launch_bounds__(256, 1) k_score_mma(const ScoreArgs a) {
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     mbar_fence_init();
+    flags[0] = 0;
   }
-  if (tid < GH) {
-    m_s[tid] = neg_inf();
-    l_s[tid] = 0.f;
+  if (tid < GH) m_sh[tid] = neg_inf();
+  // Query fragments (same for every warp).  The k dimension is permuted
+  // identically in A and B: lane quad t4 reads dims [32*s2 + 8*t4, +8) as
+  // two k-steps, so one 16-byte load per row feeds two mma k-steps.
+  if (warp == 0) {
+    const uint4 *qrow = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                                        (static_cast<size_t>(b) * a.hq + h0 + min(g, nh - 1)) * D);
+#pragma unroll
+    for (int s2 = 0; s2 < D / 32; ++s2) {
+      const uint4 w = g < nh ? qrow[4 * s2 + t4] : make_uint4(0, 0, 0, 0);
+      af_sh[(2 * s2) * 32 + lane] = make_uint2(w.x, w.y);
+      af_sh[(2 * s2 + 1) * 32 + lane] = make_uint2(w.z, w.w);
+    }
   }
   __syncthreads();
 
@@ -116,36 +148,63 @@ __global__ void __launch_bounds__(256, 1) k_score_mma(const ScoreArgs a) {
   if (tid == 0)
     for (int t = 0; t < min(kStages, ntiles); ++t) issue(t);
 
-  // Query fragments.  The k dimension is permuted identically in A and B:
-  // lane quad t reads dims [32*s2 + 8*t, +8) as two k-steps, so a single
-  // 16-byte load per row feeds two mma k-steps.
-  uint32_t af[D / 16][2];
-  {
-    const int r = lane >> 2, t4 = lane & 3;
-    const uint4 *qrow = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
-                                                        (static_cast<size_t>(b) * a.hq + h0 + min(r, nh - 1)) * D);
-#pragma unroll
-    for (int s2 = 0; s2 < D / 32; ++s2) {
-      uint4 w = r < nh ? qrow[4 * s2 + t4] : make_uint4(0, 0, 0, 0);
-      af[2 * s2][0] = w.x;
-      af[2 * s2][1] = w.y;
-      af[2 * s2 + 1][0] = w.z;
-      af[2 * s2 + 1][1] = w.w;
-    }
-  }
-
   float acc[GH][8];
 #pragma unroll
   for (int j = 0; j < GH; ++j)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+  // Reference max (base 2) per head lives in m_sh, identical for every
+  // thread; mg is this lane's copy for its head g.
+  float mg = neg_inf();
+  float l_part = 0.f;  // this lane's share of the sum for head g
 
   for (int t = 0; t < ntiles; ++t) {
     const int st = t % kStages;
-    const uint32_t par = (t / kStages) & 1;
     const int rows_t = min(kTile, nrows - t * kTile);
-    const bool ok = mbar_wait(&bars[st], par);
-    if (__syncthreads_or(!ok)) {
+    if (!mbar_wait(&bars[st], (t / kStages) & 1)) flags[0] = 1;
+    const uint8_t *Ks = smem + st * Cfg::kStageBytes;
+    const uint8_t *Vs = Ks + Cfg::kTileBytes;
+    float *pt = p_tile + (t & 1) * kTile * GH;
+
+    // Scores of rows 8*warp .. 8*warp+7 for every head of the group.
+    float s0 = neg_inf(), s1 = neg_inf();
+    const int gi0 = 8 * warp + 2 * t4, gi1 = gi0 + 1;
+    if (8 * warp < rows_t) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t *krow = Ks + (8 * warp + g) * D * 2;
+#pragma unroll
+      for (int s2 = 0; s2 < D / 32; ++s2) {
+        const uint4 kb = lds_v4(krow + (32 * s2 + 8 * t4) * 2);
+        const uint2 a0 = af_sh[(2 * s2) * 32 + lane], a1 = af_sh[(2 * s2 + 1) * 32 + lane];
+        mma_16816_bf16(c, a0.x, 0u, a0.y, 0u, kb.x, kb.y);
+        mma_16816_bf16(c, a1.x, 0u, a1.y, 0u, kb.z, kb.w);
+      }
+      if (g < nh) {
+        float *srow = a.scores ? a.scores + (static_cast<size_t>(b) * a.hq + h0 + g) * a.score_stride + n0 + t * kTile
+                               : nullptr;
+        if (gi0 < rows_t) {
+          if (srow) srow[gi0] = c[0] * a.scale;
+          s0 = c[0] * a.scale_log2;
+        }
+        if (gi1 < rows_t) {
+          if (srow) srow[gi1] = c[1] * a.scale;
+          s1 = c[1] * a.scale_log2;
+        }
+      }
+    }
+    bool need = false;
+    float tl = 0.f;
+    if (WITH_V) {
+      need = s0 > mg + kRescaleSlack || s1 > mg + kRescaleSlack;
+      if (!need && g < GH) {
+        const float p0 = exp2_approx(s0 - mg), p1 = exp2_approx(s1 - mg);
+        pt[gi0 * GH + g] = p0;
+        pt[gi1 * GH + g] = p1;
+        tl = p0 + p1;
+      }
+    }
+    const bool slow = __syncthreads_or(need);
+    if (flags[0]) {
       if (tid == 0) {
         flag_error(a.status, GSA_DEVERR_TIMEOUT);
         for (int u = t; u < min(t + kStages, ntiles); ++u) mbar_wait(&bars[u % kStages], (u / kStages) & 1);
@@ -153,89 +212,76 @@ __global__ void __launch_bounds__(256, 1) k_score_mma(const ScoreArgs a) {
       __syncthreads();
       return;
     }
-    const uint8_t *Ks = smem + st * Cfg::kStageBytes;
-    const uint8_t *Vs = Ks + Cfg::kTileBytes;
+    // Every warp is past the value pass of tile t-1: its stage can refill.
+    if (tid == 0 && t >= 1 && t - 1 + kStages < ntiles) issue(t - 1 + kStages);
+    if (!WITH_V) continue;
 
-    if (8 * warp < rows_t) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      const int t4 = lane & 3;
-      const uint8_t *krow = Ks + (8 * warp + (lane >> 2)) * D * 2;
-#pragma unroll
-      for (int s2 = 0; s2 < D / 32; ++s2) {
-        const uint4 kb = lds_v4(krow + (32 * s2 + 8 * t4) * 2);
-        mma_16816_bf16(c, af[2 * s2][0], 0u, af[2 * s2][1], 0u, kb.x, kb.y);
-        mma_16816_bf16(c, af[2 * s2 + 1][0], 0u, af[2 * s2 + 1][1], 0u, kb.z, kb.w);
-      }
-      const int hr = lane >> 2;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int gi = 8 * warp + 2 * t4 + e;
-        const bool valid = gi < rows_t && hr < nh;
-        if (valid && a.scores)
-          a.scores[(static_cast<size_t>(b) * a.hq + h0 + hr) * a.score_stride + n0 + t * kTile + gi] = c[e] * a.scale;
-        if (WITH_V && hr < GH) s_tile[hr * kTile + gi] = valid ? c[e] * a.scale_log2 : neg_inf();
-      }
-    }
-
-    if (WITH_V) {
+    if (slow) {
+      // Raise the reference max to this tile's max, rescale, redo p.
+      float qm = fmaxf(s0, s1);
+      qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
+      qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));
+      if (t4 == 0 && g < GH) wmax[warp * GH + g] = qm;
       __syncthreads();
-      if (warp < GH) {
-        const int j = warp;
-        const float x0 = (lane < rows_t && j < nh) ? s_tile[j * kTile + lane] : neg_inf();
-        const float x1 = (lane + 32 < rows_t && j < nh) ? s_tile[j * kTile + lane + 32] : neg_inf();
-        const float m_old = m_s[j];
-        const float m_new = fmaxf(m_old, warp_max(fmaxf(x0, x1)));
-        float alpha = 1.f, p0 = 0.f, p1 = 0.f;
-        if (m_new != neg_inf()) {
-          alpha = exp2_approx(m_old - m_new);
-          p0 = exp2_approx(x0 - m_new);
-          p1 = exp2_approx(x1 - m_new);
-        }
-        const float psum = warp_sum(p0 + p1);
-        p_tile[lane * GH + j] = p0;
-        p_tile[(lane + 32) * GH + j] = p1;
-        __syncwarp();
-        if (lane == 0) {
-          m_s[j] = m_new;
-          l_s[j] = l_s[j] * alpha + psum;
-          alpha_s[j] = alpha;
-        }
-      }
-      __syncthreads();
-      const int slot = warp * kRpw + lane / kLpr;
-      const int dd = 8 * (lane % kLpr);
+      float m_mine = neg_inf();  // new reference of head `tid` (tid < GH)
 #pragma unroll
       for (int j = 0; j < GH; ++j) {
-        const float al = alpha_s[j];
+        float tm = neg_inf();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] *= al;
-      }
-      for (int r = slot; r < rows_t; r += kSlots) {
-        float v[8];
-        Vec16<__nv_bfloat16>::unpack(lds_v4(Vs + (r * D + dd) * 2), v);
-        float p[GH];
+        for (int w = 0; w < 8; ++w) tm = fmaxf(tm, wmax[w * GH + j]);
+        const float mo = m_sh[j];
+        const float mn = fmaxf(mo, tm);
+        const float alpha = (mn == neg_inf()) ? 1.f : exp2_approx(mo - mn);
 #pragma unroll
-        for (int j4 = 0; j4 < GH / 4; ++j4) {
-          const float4 pp = reinterpret_cast<const float4 *>(p_tile + r * GH)[j4];
-          p[4 * j4] = pp.x;
-          p[4 * j4 + 1] = pp.y;
-          p[4 * j4 + 2] = pp.z;
-          p[4 * j4 + 3] = pp.w;
+        for (int e = 0; e < 8; ++e) acc[j][e] *= alpha;
+        if (j == g) {
+          l_part *= alpha;
+          mg = mn;
         }
-#pragma unroll
-        for (int j = 0; j < GH; ++j)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(p[j], v[e], acc[j][e]);
+        if (j == tid) m_mine = mn;
       }
+      __syncthreads();  // everyone has read the old reference
+      if (tid < GH) m_sh[tid] = m_mine;
+      if (g < GH) {
+        const float p0 = exp2_approx(s0 - mg), p1 = exp2_approx(s1 - mg);
+        pt[gi0 * GH + g] = p0;
+        pt[gi1 * GH + g] = p1;
+        tl = p0 + p1;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    if (tid == 0 && t + kStages < ntiles) issue(t + kStages);
+    l_part += tl;
+
+    // Values: slot = (warp, row group); this lane owns dims dd .. dd+7.
+    const int slot = warp * kRpw + lane / kLpr;
+    const int dd = 8 * (lane % kLpr);
+    for (int r = slot; r < rows_t; r += kSlots) {
+      const uint4 vw = lds_v4(Vs + (r * D + dd) * 2);
+      float v[8];
+      Vec16<__nv_bfloat16>::unpack(vw, v);
+      float p[GH];
+#pragma unroll
+      for (int j4 = 0; j4 < GH / 4; ++j4) {
+        const float4 pp = reinterpret_cast<const float4 *>(pt + r * GH)[j4];
+        p[4 * j4] = pp.x;
+        p[4 * j4 + 1] = pp.y;
+        p[4 * j4 + 2] = pp.z;
+        p[4 * j4 + 3] = pp.w;
+      }
+#pragma unroll
+      for (int j = 0; j < GH; ++j)
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) fma2(acc[j][e], acc[j][e + 1], p[j], v[e], v[e + 1]);
+    }
   }
 
   pdl_trigger();
   if (WITH_V && a.part) {
-    // Slots of one warp that own the same dims are merged by shuffles, then
-    // the 8 warps through shared memory (the stage ring is idle now).
+    __syncthreads();  // all value passes done before the ring is reused
+    // Per-head sums: lanes of quad g across all warps.
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    if (t4 == 0 && g < GH) wmax[warp * GH + g] = l_part;
 #pragma unroll
     for (int o = kLpr; o < 32; o <<= 1)
 #pragma unroll
@@ -260,9 +306,13 @@ __global__ void __launch_bounds__(256, 1) k_score_mma(const ScoreArgs a) {
       a.part[((static_cast<size_t>(b) * a.hq + h0 + j) * a.n_split + split) * (D + kPartHeader) + kPartHeader + dim] = s;
     }
     if (tid < nh) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) l += wmax[w * GH + tid];
+      const float mt = m_sh[tid];
       float *hdr = a.part + ((static_cast<size_t>(b) * a.hq + h0 + tid) * a.n_split + split) * (D + kPartHeader);
-      hdr[0] = m_s[tid];
-      hdr[1] = l_s[tid];
+      hdr[0] = mt;
+      hdr[1] = l;
       hdr[2] = 0.f;
       hdr[3] = 0.f;
     }

@@ -4,11 +4,14 @@
 // the k most relevant gists are kept; gist.science/ja section 2.1 step 3.
 // Equal scores go to the lower chunk index (the pages leave ties open).
 //
-// One CTA per row.  Scores become order-preserving uint32 keys; an 8-bit
-// radix select (at most four histogram passes over shared memory, stopping
-// as soon as the boundary digit is fully taken) finds the k-th key; keys
-// equal to it are taken in index order; a bitonic sort orders the k
-// survivors by (key desc, index asc).
+// One CTA per row.  Scores become order-preserving uint32 keys.  An 8-bit
+// radix select finds the k-th largest key, stopping as soon as the boundary
+// digit is taken whole; keys equal to the threshold are taken in index
+// order, which is the lower-index tie rule.  The main kernel keeps the keys
+// in registers (warp-contiguous index ranges, coalesced loads), aggregates
+// the contended first-digit histogram per warp with match.any, and writes
+// the selection by ballot compaction, so the output is in ascending chunk
+// order and needs no sort.  Rows longer than 16384 use k_topk_mem.
 #pragma once
 
 #include "common.cuh"
@@ -54,10 +57,43 @@ __device__ __forceinline__ int block_exclusive_scan_512(int v, int *warp_tot) {
     if (lane < kTopkThreads / 32) warp_tot[lane] = xi - x;
   }
   __syncthreads();
-  return incl - v + warp_tot[warp];
+  const int r = incl - v + warp_tot[warp];
+  __syncthreads();  // warp_tot may be reused by the next scan
+  return r;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkArgs a) {
+// Exclusive prefix sum in reversed thread order: for thread t, the sum of v
+// over threads t+1 .. 511.
+__device__ __forceinline__ int scan_excl_512_rev(int v, int *warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;  // sum over lanes >= lane within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  if (lane == 0) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = kTopkThreads / 32;
+    int x = lane < nw ? warp_tot[lane] : 0;
+    int xi = x;  // sum over warps >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_down_sync(0xffffffffu, xi, o);
+      if (lane + o < 32) xi += t;
+    }
+    if (lane < nw) warp_tot[lane] = xi - x;  // sum over warps > lane
+  }
+  __syncthreads();
+  const int r = incl - v + warp_tot[warp];
+  __syncthreads();
+  return r;
+}
+
+// Fallback for rows longer than the register-resident kernel handles:
+// keys are re-read from shared or global memory on every pass.
+__global__ void __launch_bounds__(kTopkThreads) k_topk_mem(const TopkArgs a) {
   constexpr int T = kTopkThreads;
   extern __shared__ __align__(16) uint32_t keys_sm[];
   __shared__ uint32_t hist[256];
@@ -197,6 +233,137 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkArgs a) {
     }
     out_i[i] = id;
     if (out_s) out_s[i] = sc;
+  }
+  if (a.counters && tid == 0) a.counters[row] = 0u;
+}
+
+
+constexpr int kTopkRegThreads = 256;
+
+// Register-resident top-k.  Warp w holds indices [w*32*KPT, (w+1)*32*KPT);
+// lane l's key j is index w*32*KPT + 32*j + l, so loads are coalesced and
+// index order inside a warp is (j, lane) order.
+template <int KPT>
+__global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : (KPT <= 32 ? 2 : 1)) k_topk(const TopkArgs a) {
+  constexpr int T = kTopkRegThreads, W = T / 32;
+  __shared__ uint32_t hist[256];
+  __shared__ int info[4];
+  __shared__ int wtot[2][W];
+
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  const int b = row / a.hq;
+  int n = a.counts ? a.counts[row] : a.n_gists[b] / a.count_div;
+  n = min(max(n, 0), min(a.stride, KPT * T));
+  const float *srow = a.scores + static_cast<size_t>(row) * a.stride;
+  const int base = warp * 32 * KPT + lane;
+
+  uint32_t key[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = base + 32 * j;
+    key[j] = i < n ? float_to_key(__ldcg(srow + i)) : 0u;
+  }
+
+  const int kk = min(a.k, n);
+  uint32_t prefix = 0, pmask = 0;
+  int rem = kk;
+  bool all_eq = kk == n;
+  for (int shift = 24; shift >= 0 && !all_eq && kk > 0; shift -= 8) {
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const bool in = (base + 32 * j < n) && ((key[j] & pmask) == prefix);
+      const uint32_t bin = (key[j] >> shift) & 255u;
+      if (shift == 24) {
+        // first digit: few distinct bins, aggregate per warp
+        const unsigned peers = __match_any_sync(0xffffffffu, in ? bin : 0x100u);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+      } else if (in) {
+        atomicAdd(&hist[bin], 1u);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[lane * 8 + e];
+        tot += c[e];
+      }
+      uint32_t incl = tot;  // bins of lanes >= lane
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+      }
+      uint32_t cum = incl - tot;
+#pragma unroll
+      for (int e = 7; e >= 0; --e) {
+        if (cum < static_cast<uint32_t>(rem) && cum + c[e] >= static_cast<uint32_t>(rem)) {
+          info[0] = lane * 8 + e;
+          info[1] = static_cast<int>(cum);
+          info[2] = static_cast<int>(c[e]);
+        }
+        cum += c[e];
+      }
+    }
+    __syncthreads();
+    rem -= info[1];
+    prefix |= static_cast<uint32_t>(info[0]) << shift;
+    pmask |= 0xFFu << shift;
+    all_eq = info[2] == rem;
+  }
+
+  // Compaction in index order: ballots within the warp, one small scan
+  // across warps for the boundary ranks and the output offsets.
+  const unsigned lt = (1u << lane) - 1u;
+  int w_gt = 0, w_eq = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const bool valid = kk > 0 && base + 32 * j < n;
+    const uint32_t km = key[j] & pmask;
+    w_gt += __popc(__ballot_sync(0xffffffffu, valid && km > prefix));
+    w_eq += __popc(__ballot_sync(0xffffffffu, valid && km == prefix));
+  }
+  if (lane == 0) {
+    wtot[0][warp] = w_eq;
+  }
+  __syncthreads();
+  int eq_before = 0;  // boundary keys in lower warps
+  for (int w = 0; w < warp; ++w) eq_before += wtot[0][w];
+  const int eq_take_w = all_eq ? w_eq : max(0, min(w_eq, rem - eq_before));
+  if (lane == 0) wtot[1][warp] = w_gt + eq_take_w;
+  __syncthreads();
+  int out_base = 0;
+  for (int w = 0; w < warp; ++w) out_base += wtot[1][w];
+  pdl_trigger();
+
+  int32_t *out_i = a.sel_idx + static_cast<size_t>(row) * a.k;
+  float *out_s = a.sel_score ? a.sel_score + static_cast<size_t>(row) * a.k : nullptr;
+  int pos = out_base, eq_seen = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    // boundary keys of this j-row taken in lane order while eq_seen < eq_take_w
+    const bool valid = kk > 0 && base + 32 * j < n;
+    const uint32_t km = key[j] & pmask;
+    const unsigned eqs = __ballot_sync(0xffffffffu, valid && km == prefix);
+    const int my_eq_rank = eq_seen + __popc(eqs & lt);
+    const bool take_eq = ((eqs >> lane) & 1u) && my_eq_rank < eq_take_w;
+    const unsigned sel = __ballot_sync(0xffffffffu, (valid && km > prefix) || take_eq);
+    if ((sel >> lane) & 1u) {
+      const int o = pos + __popc(sel & lt);
+      const int idx = base + 32 * j;
+      out_i[o] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
+      if (out_s) out_s[o] = key_to_float(key[j]);
+    }
+    pos += __popc(sel);
+    eq_seen += __popc(eqs);
+  }
+  for (int i = kk + tid; i < a.k; i += T) {
+    out_i[i] = -1;
+    if (out_s) out_s[i] = neg_inf();
   }
   if (a.counters && tid == 0) a.counters[row] = 0u;
 }

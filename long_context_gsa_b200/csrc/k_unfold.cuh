@@ -9,10 +9,12 @@
 // merge per-host attention in its second phase.
 //
 // Grid: (splits, hq, B).  Split s of row (b, h) gathers its share of the
-// selected chunks (each a contiguous chunk*D span of K and of V) with bulk
-// copies into a shared-memory ring; the last split also takes the own
-// chunk.  Each group of lanes that owns one row runs an online softmax; the
-// CTA result is a partial (max, sum, acc).  The CTA that arrives last at
+// selected chunks (each a contiguous chunk*D span of K and of V, cut into
+// pieces of at most 4 KB) with bulk copies; the last split also takes the
+// own chunk.  Each of the 4 warps streams its own pieces through a private
+// mbarrier ring, so the main loop has no CTA-wide barrier.  Each group of
+// lanes that owns one row runs an online softmax; the CTA result is a
+// partial (max, sum, acc).  The CTA that arrives last at
 // the row's counter (an atomic, no waiting) merges all partials with the
 // prior partial (all gists, or the H-GSA levels) and writes out and lse.
 #pragma once
@@ -42,7 +44,7 @@ struct UnfoldArgs {
 };
 
 constexpr int kUnfoldThreads = 128;
-constexpr int kUnfoldMaxItems = 1025;
+constexpr int kUnfoldMaxItems = 1024;
 
 // Merge (m2, l2, acc2) into (m, l, acc): base-2 online-softmax combination.
 template <int E>
@@ -80,34 +82,50 @@ __device__ void combine_records(const float *const *recs, const int *counts, int
   }
 }
 
+// Rows of one bulk-copy piece: at most 4 KB of K (and of V) per piece, so
+// long chunks pipeline in several pieces.
+template <int D, typename T>
+__host__ __device__ __forceinline__ int unfold_piece_rows(int chunk) {
+  const int cap = 4096 / (D * static_cast<int>(sizeof(T)));
+  return chunk < cap ? chunk : (cap < 1 ? 1 : cap);
+}
+
+// Stages of each warp's ring (a stage holds one piece of K and of V).
+__host__ __device__ __forceinline__ int unfold_warp_stages(int stage_bytes) {
+  const int s = 8192 / stage_bytes;
+  return s < 2 ? 2 : (s > 8 ? 8 : s);
+}
+
+constexpr int kUnfoldWarps = kUnfoldThreads / 32;
+
 template <int D, typename T>
 __global__ void __launch_bounds__(kUnfoldThreads) k_unfold(const UnfoldArgs a) {
   constexpr int kE = Vec16<T>::kElems;          // elements per lane
   constexpr int kLpr = D / kE;                  // lanes per row
   constexpr int kRpw = 32 / kLpr;               // rows per warp pass
-  constexpr int kSlots = (kUnfoldThreads / 32) * kRpw;
   constexpr int kRowBytes = D * static_cast<int>(sizeof(T));
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int items[kUnfoldMaxItems];
   __shared__ int item_pos[kUnfoldMaxItems];
   __shared__ int n_items_s;
   __shared__ int is_last_s;
-  __shared__ float red[kUnfoldThreads / 32][2 + D];
-  __shared__ uint64_t bars[8];
+  __shared__ float red[kUnfoldWarps][2 + D];
+  __shared__ uint64_t bars[kUnfoldWarps][8];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / a.group;
   const size_t row = static_cast<size_t>(b) * a.hq + h;
-  const uint32_t chunk_bytes = static_cast<uint32_t>(a.chunk) * kRowBytes;
-  const int stages = min(8, max(2, (96 * 1024) / static_cast<int>(2 * chunk_bytes)));
+  const int pr = unfold_piece_rows<D, T>(a.chunk);
+  const uint32_t piece_bytes = static_cast<uint32_t>(pr) * kRowBytes;
+  const int sw = unfold_warp_stages(static_cast<int>(2 * piece_bytes));
 
   pdl_wait();
   const int N = min(min(max(a.n_gists[b], 0), a.n_max), a.t_max / a.chunk);
   int own = min(max(a.own_len[b], 0), a.chunk);
   if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
 
-  // Items of this split, in list order: selected chunks, then the own chunk.
+  // Selected chunks of this split, in list order (invalid entries dropped).
   const int per = (a.k + a.n_split - 1) / a.n_split;
   const int i0 = min(a.k, split * per), i1 = min(a.k, i0 + per);
   if (warp == 0) {
@@ -130,102 +148,121 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold(const UnfoldArgs a) {
       }
       cnt += __popc(ball);
     }
-    if (lane == 0) {
-      if (split == a.n_split - 1 && own > 0) {
-        items[cnt] = -1;  // the own chunk
-        item_pos[cnt] = -1;
-        ++cnt;
-      }
-      n_items_s = cnt;
-      for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
-      mbar_fence_init();
-    }
+    if (lane == 0) n_items_s = cnt;
+    if (lane < kUnfoldWarps)
+      for (int s = 0; s < sw; ++s) mbar_init(&bars[lane][s], 1);
+    if (lane == 0) mbar_fence_init();
   }
   __syncthreads();
-  const int n_items = n_items_s;
+
+  // Pieces: each selected chunk gives ppc pieces; the own chunk (last split)
+  // gives ceil(own / pr) pieces.  Warp w takes pieces w, w + 4, ...
+  const int ppc = (a.chunk + pr - 1) / pr;
+  const int n_sel = n_items_s;
+  const int own_pieces = (split == a.n_split - 1 && own > 0) ? (own + pr - 1) / pr : 0;
+  const int n_pieces = n_sel * ppc + own_pieces;
+  const int n_mine = n_pieces > warp ? (n_pieces - warp + kUnfoldWarps - 1) / kUnfoldWarps : 0;
 
   const size_t kv_base = (static_cast<size_t>(b) * a.hkv + kvh) * a.t_max;
   const uint8_t *rk = reinterpret_cast<const uint8_t *>(a.raw_k) + kv_base * kRowBytes;
   const uint8_t *rv = reinterpret_cast<const uint8_t *>(a.raw_v) + kv_base * kRowBytes;
-  auto item_rows = [&](int it) { return items[it] >= 0 ? a.chunk : own; };
-  auto issue = [&](int it) {
-    const int st = it % stages;
-    const int m = items[it];
-    const size_t first = m >= 0 ? static_cast<size_t>(m) * a.chunk : static_cast<size_t>(N) * a.chunk;
-    const uint32_t bytes = static_cast<uint32_t>(item_rows(it)) * kRowBytes;
-    uint8_t *dst = smem + static_cast<size_t>(st) * 2 * chunk_bytes;
-    mbar_arrive_expect_tx(&bars[st], 2 * bytes);
-    bulk_g2s(dst, rk + first * kRowBytes, bytes, &bars[st]);
-    bulk_g2s(dst + chunk_bytes, rv + first * kRowBytes, bytes, &bars[st]);
+  uint8_t *ring = smem + static_cast<size_t>(warp) * sw * 2 * piece_bytes;
+  // piece p -> first raw row and row count
+  auto piece = [&](int p, int &first, int &rows) {
+    if (p < n_sel * ppc) {
+      const int it = p / ppc, sub = p % ppc;
+      first = items[it] * a.chunk + sub * pr;
+      rows = min(pr, a.chunk - sub * pr);
+    } else {
+      const int q = p - n_sel * ppc;
+      first = N * a.chunk + q * pr;
+      rows = min(pr, own - q * pr);
+    }
   };
-  if (tid == 0)
-    for (int it = 0; it < min(stages, n_items); ++it) issue(it);
+  auto issue = [&](int li) {
+    int first, rows;
+    piece(warp + kUnfoldWarps * li, first, rows);
+    const int st = li % sw;
+    const uint32_t bytes = static_cast<uint32_t>(rows) * kRowBytes;
+    uint8_t *dst = ring + static_cast<size_t>(st) * 2 * piece_bytes;
+    mbar_arrive_expect_tx(&bars[warp][st], 2 * bytes);
+    bulk_g2s(dst, rk + static_cast<size_t>(first) * kRowBytes, bytes, &bars[warp][st]);
+    bulk_g2s(dst + piece_bytes, rv + static_cast<size_t>(first) * kRowBytes, bytes, &bars[warp][st]);
+  };
+  if (lane == 0)
+    for (int li = 0; li < min(sw, n_mine); ++li) issue(li);
 
-  // Query slice of this lane (dims dd .. dd+kE-1).
-  const int slot = warp * kRpw + lane / kLpr;
+  const int slot = lane / kLpr;
   const int dd = kE * (lane % kLpr);
   float qf[kE];
   Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(a.q) + row * D + dd), qf);
 
+  // Online softmax state of this lane's slot; the reference max m is only
+  // raised when a logit exceeds it by more than 2^8 (rare after warm-up).
   float m = neg_inf(), l = 0.f, acc[kE];
 #pragma unroll
   for (int e = 0; e < kE; ++e) acc[e] = 0.f;
-
-  for (int it = 0; it < n_items; ++it) {
-    const int st = it % stages;
-    const bool ok = mbar_wait(&bars[st], (it / stages) & 1);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) {
-        flag_error(a.status, GSA_DEVERR_TIMEOUT);
-        for (int u = it; u < min(it + stages, n_items); ++u) mbar_wait(&bars[u % stages], (u / stages) & 1);
-      }
-      __syncthreads();
-      return;
+  auto update = [&](float z, const float *vf) {
+    if (z > m + 8.0f) {
+      const float c = exp2_approx(m - z);
+      l *= c;
+#pragma unroll
+      for (int e = 0; e < kE; ++e) acc[e] *= c;
+      m = z;
     }
-    const uint8_t *Ks = smem + static_cast<size_t>(st) * 2 * chunk_bytes;
-    const uint8_t *Vs = Ks + chunk_bytes;
-    const int rows = item_rows(it);
-    for (int r0 = 0; r0 < rows; r0 += kSlots) {
+    const float p = exp2_approx(z - m);
+    l += p;
+#pragma unroll
+    for (int e = 0; e < kE; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
+  };
+
+  int stuck = -1;  // first piece whose wait expired
+  for (int li = 0; li < n_mine; ++li) {
+    const int st = li % sw;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[warp][st], (li / sw) & 1))) {
+      stuck = li;
+      break;
+    }
+    const int p = warp + kUnfoldWarps * li;
+    int first, rows;
+    piece(p, first, rows);
+    const uint8_t *Ks = ring + static_cast<size_t>(st) * 2 * piece_bytes;
+    const uint8_t *Vs = Ks + piece_bytes;
+    for (int r0 = 0; r0 < rows; r0 += kRpw) {
       const int r = r0 + slot;
       const bool valid = r < rows;
       float kf[kE], part = 0.f;
-      Vec16<T>::unpack(lds_v4(Ks + (valid ? r : 0) * kRowBytes + dd * sizeof(T)), kf);
+      Vec16<T>::unpack(lds_v4(Ks + (valid ? r : 0) * kRowBytes + dd * static_cast<int>(sizeof(T))), kf);
 #pragma unroll
       for (int e = 0; e < kE; ++e) part = fmaf(qf[e], kf[e], part);
 #pragma unroll
       for (int o = 1; o < kLpr; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
       if (valid) {
-        const float z = part * a.scale_log2;
         float vf[kE];
-        Vec16<T>::unpack(lds_v4(Vs + r * kRowBytes + dd * sizeof(T)), vf);
-        const float mn = fmaxf(m, z);
-        const float corr = exp2_approx(m - mn), p = exp2_approx(z - mn);
-        l = l * corr + p;
-#pragma unroll
-        for (int e = 0; e < kE; ++e) acc[e] = fmaf(p, vf[e], acc[e] * corr);
-        m = mn;
+        Vec16<T>::unpack(lds_v4(Vs + r * kRowBytes + dd * static_cast<int>(sizeof(T))), vf);
+        update(part * a.scale_log2, vf);
       }
     }
-    // Exclude mode: the selected chunk's gist token (logit = its score).
-    if (a.exclude && items[it] >= 0 && slot == it % kSlots) {
-      const float z = a.sel_score[row * a.k + item_pos[it]] * kLog2e;
+    // Exclude mode: the selected chunk's gist token joins with its first piece.
+    if (a.exclude && p < n_sel * ppc && p % ppc == 0 && slot == 0) {
+      const int it = p / ppc;
       float vf[kE];
       const T *gv = reinterpret_cast<const T *>(a.gist_v) +
                     ((static_cast<size_t>(b) * a.hkv + kvh) * a.n_max + items[it]) * D + dd;
       Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(gv), vf);
-      const float mn = fmaxf(m, z);
-      const float corr = exp2_approx(m - mn), p = exp2_approx(z - mn);
-      l = l * corr + p;
-#pragma unroll
-      for (int e = 0; e < kE; ++e) acc[e] = fmaf(p, vf[e], acc[e] * corr);
-      m = mn;
+      update(a.sel_score[row * a.k + item_pos[it]] * kLog2e, vf);
     }
-    __syncthreads();
-    if (tid == 0 && it + stages < n_items) issue(it + stages);
+    __syncwarp();
+    if (lane == 0 && li + sw < n_mine) issue(li + sw);
+  }
+  if (stuck >= 0 && lane == 0) {
+    // Let the copies already issued land before the CTA can exit.
+    flag_error(a.status, GSA_DEVERR_TIMEOUT);
+    for (int li = stuck; li < min(stuck + sw, n_mine); ++li) mbar_wait(&bars[warp][li % sw], (li / sw) & 1);
   }
   pdl_trigger();
 
-  // Merge the slots of a warp that own the same dims, then the warps.
+  // Merge the slots of the warp that own the same dims, then the warps.
 #pragma unroll
   for (int o = kLpr; o < 32; o <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
@@ -247,19 +284,19 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold(const UnfoldArgs a) {
   {
     float M = neg_inf();
 #pragma unroll
-    for (int w = 0; w < kUnfoldThreads / 32; ++w) M = fmaxf(M, red[w][0]);
+    for (int w = 0; w < kUnfoldWarps; ++w) M = fmaxf(M, red[w][0]);
     for (int dim = tid; dim < D; dim += kUnfoldThreads) {
       float s = 0.f;
       if (M != neg_inf())
 #pragma unroll
-        for (int w = 0; w < kUnfoldThreads / 32; ++w) s += red[w][2 + dim] * exp2_approx(red[w][0] - M);
+        for (int w = 0; w < kUnfoldWarps; ++w) s += red[w][2 + dim] * exp2_approx(red[w][0] - M);
       rec[kPartHeader + dim] = s;
     }
     if (tid == 0) {
       float L = 0.f;
       if (M != neg_inf())
 #pragma unroll
-        for (int w = 0; w < kUnfoldThreads / 32; ++w) L += red[w][1] * exp2_approx(red[w][0] - M);
+        for (int w = 0; w < kUnfoldWarps; ++w) L += red[w][1] * exp2_approx(red[w][0] - M);
       rec[0] = M;
       rec[1] = L;
       rec[2] = 0.f;
