@@ -240,15 +240,24 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
  * selection among them) and its own chunk's raw tokens m*chunk .. i.  Gist
  * position m sees its chunk's raw tokens and gists 0..m (compression mask).
  *
- * Stage 1, scoring + selection for every raw position (tensor cores):
- *   sel_idx [B, hq, L, topk] int32 out, sel_score [B, hq, L, topk] fp32
- *   out; in default mode ws also receives each row's softmax partial over
- *   its completed gists. */
-gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *k_gist, const void *v_gist,
+ * Both stages are built for bf16 inputs with d = 128 and topk <= 32
+ * (GSA_ERR_UNSUPPORTED otherwise), and need t_max = n_max * chunk.
+ *
+ * Stage 1, scoring + selection (tensor cores).  Every raw row is scored
+ * against the gists it can see and keeps the top k; every row (raw and
+ * gist) also records its maximum visible score in ws, the softmax
+ * reference stage 2 uses.
+ *   sel_idx [B, hq, L, topk] int32 out (ascending chunk order, -1 padded),
+ *   sel_score [B, hq, L, topk] fp32 out. */
+gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *q_gist, const void *k_gist,
                              int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
 
-/* Stage 2, unfolding + attention for every raw and gist position:
- *   out_raw [B, hq, L, d], out_gist [B, hq, N, d] in out_dtype. */
+/* Stage 2, unfolding + attention for every raw and gist position, given
+ * stage 1's selection and the row maxima it left in ws (same ws):
+ *   out_raw [B, hq, L, d], out_gist [B, hq, N, d] in out_dtype.
+ * The dense gist part (all visible gists of a row) runs on the tensor cores
+ * with bf16 softmax weights normalised by their own sum; the selected
+ * chunks and the own chunk run on the CUDA cores in fp32. */
 gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
                               const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,
                               const float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes,

@@ -226,11 +226,11 @@ def hgsa_decode(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_
         _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
 
 
-def gsa_prefill_score(desc, q_raw, k_gist, v_gist, sel_idx, sel_score, ws, stream=None):
+def gsa_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, ws, stream=None):
     dt = _TORCH_DT[desc.dtype]
     p, n = _ws(ws)
     _check("gsa_prefill_score", load().gsa_prefill_score(
-        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist", True),
+        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"),
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
 
 

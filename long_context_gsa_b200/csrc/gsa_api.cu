@@ -8,10 +8,12 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/gsa.h"
 #include "common.cuh"
 #include "k_hgsa.cuh"
+#include "k_prefill.cuh"
 #include "k_score.cuh"
 #include "k_topk.cuh"
 #include "k_unfold.cuh"
@@ -35,7 +37,7 @@ inline float resolve_scale(const gsa_desc *d) {
 struct Layout {
   size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
-  size_t pf_stats = 0;
+  size_t pf_stats = 0, pf_gist = 0, pf_vh = 0;
   size_t total = 0;
 };
 
@@ -83,6 +85,8 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     take(L.sel_idx, prow * d->topk * 4);
     take(L.sel_score, prow * d->topk * 4);
     take(L.pf_stats, prow * rec);
+    take(L.pf_gist, rows * static_cast<size_t>(d->n_max) * rec);
+    take(L.pf_vh, static_cast<size_t>(d->batch) * d->hkv * d->n_max * d->d * 2);
     L.total = off;
     return L;
   }
@@ -142,8 +146,8 @@ inline int one_wave_splits(int units, int slots, int max_splits) {
 
 // Launch with programmatic stream serialization: the kernel may start while
 // its predecessor drains; it calls griddepcontrol.wait before touching data.
-template <typename Kern, typename Arg>
-gsa_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, void *stream, const Arg &arg) {
+template <typename Kern, typename... Args>
+gsa_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, void *stream, const Args &...args) {
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return GSA_OK;
   if (!prepare(kern, smem)) return GSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -156,7 +160,7 @@ gsa_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, void *stream, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, arg);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GSA_ERR_CUDA;
@@ -414,6 +418,129 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
              : GSA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- prefill
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2D 16-bit view [rows, 128] with 64-column, box_rows-row boxes, 128-byte swizzle.
+bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+gsa_status check_prefill(const gsa_desc *d) {
+  GSA_TRY(check_desc(d));
+  if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
+  if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->n_max) * d->chunk != d->t_max) return GSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
+  return GSA_OK;
+}
+
+PrefillArgs prefill_args(const gsa_desc *d, int32_t *sel_idx, float *sel_score, const Layout &L, void *ws) {
+  PrefillArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  pa.bh = d->batch * d->hq;
+  pa.hq = d->hq;
+  pa.hkv = d->hkv;
+  pa.group = d->hq / d->hkv;
+  pa.chunk = d->chunk;
+  pa.n_chunks = d->n_max;
+  pa.L = d->t_max;
+  pa.topk = d->topk;
+  pa.exclude = d->exclude_unselected;
+  pa.scale = resolve_scale(d);
+  pa.scale_log2 = pa.scale * kLog2e;
+  pa.sel_idx = sel_idx;
+  pa.sel_score = sel_score;
+  pa.rec_raw = reinterpret_cast<float *>(at(ws, L.pf_stats));
+  pa.rec_gist = reinterpret_cast<float *>(at(ws, L.pf_gist));
+  pa.gist_tiles = cdiv(d->n_max, kPfRows);
+  pa.raw_tiles = cdiv(d->t_max, kPfRows);
+  pa.status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  return pa;
+}
+
+gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q_gist, const void *k_gist,
+                             int32_t *sel_idx, float *sel_score, const Layout &L, void *ws, void *stream) {
+  PrefillArgs pa = prefill_args(d, sel_idx, sel_score, L, ws);
+  const uint64_t bh = static_cast<uint64_t>(d->batch) * d->hq, bkv = static_cast<uint64_t>(d->batch) * d->hkv;
+  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, bh * d->n_max, kPfRows) ||
+      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kPfKeys))
+    return GSA_ERR_CUDA;
+  const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
+  const int grid = std::min(total, sm_count());
+  const size_t smem = PfSmem::kBytes;
+  if (d->topk <= 16) return launch(k_prefill_score<16>, dim3(grid), dim3(kPfThreads), smem, stream, pa);
+  return launch(k_prefill_score<32>, dim3(grid), dim3(kPfThreads), smem, stream, pa);
+}
+
+gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,
+                              const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,
+                              const float *sel_score, void *out_raw, void *out_gist, const Layout &L, void *ws,
+                              void *stream) {
+  PrefillArgs pa = prefill_args(d, nullptr, nullptr, L, ws);
+  const uint64_t bh = static_cast<uint64_t>(d->batch) * d->hq, bkv = static_cast<uint64_t>(d->batch) * d->hkv;
+  void *vh = at(ws, L.pf_vh);
+  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, bh * d->n_max, kPfRows) ||
+      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kGaKeys) ||
+      !map_rows(&pa.tm_vgist, vh, bkv * d->n_max, kGaKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return GSA_ERR_CUDA;
+  const size_t n8 = bkv * d->n_max * 128 / 8;
+  GSA_TRY(launch(k_bf16_to_f16, dim3(static_cast<unsigned>(std::min<size_t>((n8 + 255) / 256, 4 * sm_count()))),
+                 dim3(256), 0, stream, static_cast<const __nv_bfloat16 *>(v_gist), static_cast<__half *>(vh), n8));
+  const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
+  GSA_TRY(launch(k_prefill_gist_attn, dim3(std::min(total, sm_count())), dim3(kPfThreads), GaSmem::kBytes, stream, pa));
+  GatherArgs ga;
+  ga.q_raw = static_cast<const __nv_bfloat16 *>(q_raw);
+  ga.k_raw = static_cast<const __nv_bfloat16 *>(k_raw);
+  ga.v_raw = static_cast<const __nv_bfloat16 *>(v_raw);
+  ga.q_gist = static_cast<const __nv_bfloat16 *>(q_gist);
+  ga.v_gist = static_cast<const __nv_bfloat16 *>(v_gist);
+  ga.sel_idx = sel_idx;
+  ga.sel_score = sel_score;
+  ga.rec_raw = pa.rec_raw;
+  ga.rec_gist = pa.rec_gist;
+  ga.bh = pa.bh;
+  ga.hq = d->hq;
+  ga.group = pa.group;
+  ga.chunk = d->chunk;
+  ga.n_chunks = d->n_max;
+  ga.L = d->t_max;
+  ga.topk = d->topk;
+  ga.exclude = d->exclude_unselected;
+  ga.scale_log2 = pa.scale_log2;
+  ga.out_raw = out_raw;
+  ga.out_gist = out_gist;
+  ga.out_bf16 = d->out_dtype == GSA_BF16;
+  const int64_t rows = static_cast<int64_t>(pa.bh) * (d->t_max + d->n_max);
+  return launch(k_prefill_gather, dim3(static_cast<unsigned>((rows + kGatherWarps - 1) / kGatherWarps)),
+                dim3(kGatherWarps * 32), 0, stream, ga);
+}
+
 // Number of partial records per row the scoring pass writes for these shapes.
 int gist_prior_count(const gsa_desc *d) { return plan_score(d, d->n_max, true).splits; }
 
@@ -628,22 +755,60 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
                     L, ws, stream);
 }
 
-gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *k_gist, const void *v_gist,
+gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *q_gist, const void *k_gist,
                              int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream) {
-  return GSA_ERR_UNSUPPORTED;
+  GSA_TRY(check_prefill(desc));
+  GSA_TRY(need_ptr(q_raw));
+  GSA_TRY(need_ptr(q_gist));
+  GSA_TRY(need_ptr(k_gist));
+  GSA_TRY(need_ptr(ws));
+  if (desc->topk > 0) {
+    GSA_TRY(need_ptr(sel_idx));
+    GSA_TRY(need_ptr(sel_score));
+  }
+  const Layout L = layout(desc, GSA_OP_PREFILL, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  return run_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, L, ws, stream);
 }
 
 gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
                               const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,
                               const float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes,
                               void *stream) {
-  return GSA_ERR_UNSUPPORTED;
+  GSA_TRY(check_prefill(desc));
+  GSA_TRY(need_ptr(q_raw));
+  GSA_TRY(need_ptr(k_raw));
+  GSA_TRY(need_ptr(v_raw));
+  GSA_TRY(need_ptr(q_gist));
+  GSA_TRY(need_ptr(k_gist));
+  GSA_TRY(need_ptr(v_gist));
+  GSA_TRY(need_ptr(out_raw));
+  GSA_TRY(need_ptr(out_gist));
+  GSA_TRY(need_ptr(ws));
+  if (desc->topk > 0) {
+    GSA_TRY(need_ptr(sel_idx));
+    GSA_TRY(need_ptr(sel_score));
+  }
+  const Layout L = layout(desc, GSA_OP_PREFILL, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  return run_prefill_attend(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, sel_idx, sel_score, out_raw, out_gist,
+                            L, ws, stream);
 }
 
 gsa_status gsa_prefill(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
                        const void *q_gist, const void *k_gist, const void *v_gist, int32_t *sel_idx,
                        float *sel_score, void *out_raw, void *out_gist, void *ws, size_t ws_bytes, void *stream) {
-  return GSA_ERR_UNSUPPORTED;
+  GSA_TRY(check_prefill(desc));
+  GSA_TRY(opt_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(need_ptr(ws));
+  const Layout L = layout(desc, GSA_OP_PREFILL, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
+  float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
+  GSA_TRY(gsa_prefill_score(desc, q_raw, q_gist, k_gist, si, ss, ws, ws_bytes, stream));
+  return gsa_prefill_attend(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, si, ss, out_raw, out_gist, ws, ws_bytes,
+                            stream);
 }
 
 }  // extern "C"

@@ -1,0 +1,147 @@
+"""Causal GSA prefill on the GPU (tensor-core scoring + selection, tensor-core
+gist attention, gathered raw tokens) against the float64 oracle, through the
+C ABI.  Raw rows compare selections (tie window as in decode) and outputs;
+gist rows compare outputs."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import TOL, tie_window
+
+pytestmark = pytest.mark.gpu
+
+W = None
+G = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    global W, G
+    from long_context_gsa_b200 import build
+    build.build_library()
+    import long_context_gsa_b200 as G_
+    import long_context_gsa_b200.workloads as W_
+    W, G = W_, G_
+
+
+def run_gpu(x, cfg, exclude, split=False):
+    B, hq, L, d = x["q_raw"].shape
+    hkv, N = x["k_raw"].shape[1], x["k_gist"].shape[2]
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, N, L, cfg.topk, exclude, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_PREFILL), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+    out_raw = torch.full((B, hq, L, d), float("nan"), dtype=torch.float32, device="cuda")
+    out_gist = torch.full((B, hq, N, d), float("nan"), dtype=torch.float32, device="cuda")
+    sel = torch.full((B, hq, L, cfg.topk), -9, dtype=torch.int32, device="cuda")
+    ssc = torch.empty((B, hq, L, cfg.topk), dtype=torch.float32, device="cuda")
+    if split:
+        G.gsa_prefill_score(desc, x["q_raw"], x["q_gist"], x["k_gist"], sel, ssc, ws)
+        G.gsa_prefill_attend(desc, x["q_raw"], x["k_raw"], x["v_raw"], x["q_gist"], x["k_gist"], x["v_gist"], sel, ssc,
+                             out_raw, out_gist, ws)
+    else:
+        G.gsa_prefill(desc, x["q_raw"], x["k_raw"], x["v_raw"], x["q_gist"], x["k_gist"], x["v_gist"], out_raw, out_gist,
+                      sel, ssc, ws)
+    torch.cuda.synchronize()
+    assert G.gsa_workspace_status(ws) == 0
+    return out_raw, out_gist, sel
+
+
+def check(x, cfg, exclude, rows=None, what=""):
+    """rows: oracle row ids ((b*hq+h)*(L+N) + pos); None = all rows."""
+    out_raw, out_gist, sel = run_gpu(x, cfg, exclude)
+    B, hq, L, d = x["q_raw"].shape
+    hkv, N = x["k_raw"].shape[1], x["k_gist"].shape[2]
+    P = L + N
+    if rows is None:
+        rows = np.arange(B * hq * P)
+    rows = np.asarray(rows, dtype=np.int64)
+    tk = W.to_oracle
+    args = [tk(x[k]) for k in ("q_raw", "k_raw", "v_raw", "q_gist", "k_gist", "v_gist")]
+    orc = oracle.get().prefill(*args, chunk=cfg.chunk, topk=cfg.topk, exclude=exclude, rows=rows)
+    g_raw = out_raw.reshape(B * hq * L, d).cpu().numpy()
+    g_gist = out_gist.reshape(B * hq * N, d).cpu().numpy()
+    g_sel = sel.reshape(B * hq * L, cfg.topk).cpu().numpy()
+    qr = W.to_oracle(x["q_raw"])
+    kg = W.to_oracle(x["k_gist"])
+    as64 = (lambda a: (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)) if qr.dtype == np.uint16 else \
+        (lambda a: a.astype(np.float64))
+    scale = 1.0 / np.sqrt(d)
+    G_ = hq // hkv
+    worst, exempt, forced = 0.0, 0, []
+    for i, r in enumerate(rows):
+        bh, pos = divmod(int(r), P)
+        b, h = divmod(bh, hq)
+        if pos >= L:
+            got = g_gist[bh * N + (pos - L)]
+        else:
+            got = g_raw[bh * L + pos]
+            m = pos // cfg.chunk
+            gs = set(int(t) for t in g_sel[bh * L + pos] if t >= 0)
+            os = set(int(t) for t in orc["sel"][i] if t >= 0)
+            if gs != os:
+                s = scale * (as64(kg[b, h // G_, :m]) @ as64(qr[b, h, pos]))
+                ex, lo, hi = tie_window(s, cfg.topk)
+                assert ex and len(gs) == len(os) and all(lo <= s[t] <= hi for t in gs ^ os), \
+                    f"{what}: selection differs outside the tie window at row {r} (pos {pos})"
+                exempt += 1
+                forced.append((i, r, sorted(gs) + [-1] * (cfg.topk - len(gs))))
+                continue
+        err = float(np.abs(got - orc["out"][i]).max())
+        assert err <= TOL["bf16"], f"{what}: row {r} (pos {pos}, gist={pos >= L}) max abs err {err}"
+        worst = max(worst, err)
+    if forced:
+        fr = oracle.get().prefill(*args, chunk=cfg.chunk, topk=cfg.topk, exclude=exclude,
+                                  rows=np.array([f[1] for f in forced]), sel_in=np.array([f[2] for f in forced]))
+        for j, (i, r, _) in enumerate(forced):
+            bh, pos = divmod(int(r), P)
+            err = float(np.abs(g_raw[bh * L + pos] - fr["out"][j]).max())
+            assert err <= TOL["bf16"], f"{what}: tie-exempt row {r} max abs err {err}"
+    return {"max_abs_err": worst, "tie_exempt": exempt, "rows": len(rows)}
+
+
+SMALL = [
+    ("n40_c16_k4", dict(batch=1, hq=4, hkv=2, chunk=16, n_chunks=40, topk=4)),
+    ("n300_c8_k16", dict(batch=1, hq=8, hkv=2, chunk=8, n_chunks=300, topk=16)),
+    ("ragged_tile_n37", dict(batch=2, hq=2, hkv=1, chunk=16, n_chunks=37, topk=5)),
+    ("k32_n520_c4", dict(batch=1, hq=4, hkv=1, chunk=4, n_chunks=520, topk=32)),
+]
+
+
+@pytest.mark.parametrize("name,chg", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_small(name, chg, exclude):
+    cfg = W.scaled(W.PREFILL_32K, seed=zlib.crc32(name.encode()), **chg)
+    x = W.prefill_inputs(cfg, device="cuda")
+    print(name, check(x, cfg, exclude, what=name))
+
+
+def test_split_calls_match_fused():
+    cfg = W.scaled(W.PREFILL_32K, batch=1, hq=4, hkv=2, chunk=16, n_chunks=100, topk=8)
+    x = W.prefill_inputs(cfg, device="cuda")
+    a = run_gpu(x, cfg, False, split=False)
+    b = run_gpu(x, cfg, False, split=True)
+    assert torch.equal(a[2], b[2]) and torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_full_size_sampled():
+    """The 32K-token prefill (28/4 heads, 2048 chunks of 16, top-16): a sample of
+    rows -- the first chunks, the last chunk, every 64th chunk, random rows and
+    gist rows -- against the oracle."""
+    cfg = W.PREFILL_32K
+    x = W.prefill_inputs(cfg, device="cuda")
+    L, N, hq = cfg.length, cfg.n_chunks, cfg.hq
+    P = L + N
+    rng = np.random.default_rng(7)
+    rows = []
+    for h in (0, 13, 27):
+        base = h * P
+        rows += [base + p for p in range(0, 20 * cfg.chunk, 7)]                   # early chunks (m <= k)
+        rows += [base + p for p in range(L - cfg.chunk, L)]                       # last chunk
+        rows += [base + m * cfg.chunk + 5 for m in range(0, N, 64)]               # every 64th chunk
+        rows += [base + L + m for m in (0, 1, 2, 511, 1024, N - 1)]               # gist rows
+    rows += list(rng.integers(0, hq * P, 400))
+    res = check(x, cfg, False, rows=sorted(set(int(r) for r in rows)), what="prefill_32k")
+    print("prefill_32k", res)
