@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--impl", default="gsa", choices=["gsa", "reference"])
     p.add_argument("--workload", default="llama1b_8x")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--main-only", action="store_true", help="skip the other workloads")
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,prefill_32k",
+                   help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
 
@@ -176,6 +179,206 @@ def host_copy(x):
 
 
 # ---------------------------------------------------------------- GSA arm
+class Flusher:
+    """Write a 2x-L2 buffer, then read another one, so the written lines are
+    evicted (written back) before the next timed step starts."""
+
+    def __init__(self, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        n = max(2 * l2, 256 << 20)
+        self.w = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(n // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        torch.amax(self.r, dim=0, out=self.sink)
+
+
+def timed_steps(step, steps, flush, n_marks=1):
+    """Run `steps` steps, L2 flushed before each; step(evs) records events
+    evs[0..n_marks] on the current stream.  Returns [steps, n_marks] ms."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)] for _ in range(steps)]
+    for s in range(steps):
+        flush()
+        step(ev[s])
+    torch.cuda.synchronize()
+    return np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(n_marks)] for s in range(steps)])
+
+
+def decode_setup(G, W, cfg, dev, seed):
+    x = W.decode_inputs(cfg, device=dev, seed=seed)
+    B, hq, d = x["q"].shape
+    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
+    dt = G.GSA_BF16 if cfg.dtype == "bf16" else G.GSA_F32
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, cfg.exclude, 0.0, dt, G.GSA_F32)
+    return x, desc
+
+
+def measure_flat(G, W, cfg, dev, args, flush, seed, e2e=False, clock_index=None):
+    x, desc = decode_setup(G, W, cfg, dev, seed)
+    B, hq, d = x["q"].shape
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+    scores = torch.empty((B, hq, x["gist_k"].shape[2]), dtype=torch.float32, device=dev)
+    prior = G.GSA_PRIOR_NONE if cfg.exclude else G.GSA_PRIOR_GISTS
+
+    def fused():
+        G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
+                     out, None, sel, ssc, ws)
+
+    def step_fused(evs):
+        evs[0].record()
+        fused()
+        evs[1].record()
+
+    def step_split(evs):
+        evs[0].record()
+        G.gsa_score_gists(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores, ws)
+        evs[1].record()
+        G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
+        evs[2].record()
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
+                            prior, out, None, ws)
+        evs[3].record()
+
+    for _ in range(args.warmup):
+        flush()
+        fused()
+    torch.cuda.synchronize()
+    clk = ClockSampler(clock_index) if clock_index is not None else None
+    if clk:
+        clk.__enter__()
+    step_ms = timed_steps(step_fused, args.steps, flush)[:, 0]
+    if clk:
+        clk.__exit__()
+    kern_ms = timed_steps(step_split, args.steps, flush, 3)
+    res = {"x": x, "sel": sel, "step_ms": step_ms, "kern_ms": kern_ms, "clocks": clk.summary() if clk else None,
+           "ws": ws}
+    if e2e:
+        q_host = x["q"].cpu().pin_memory()
+        out_host = torch.empty_like(out, device="cpu").pin_memory()
+
+        def step_e2e(evs):
+            evs[0].record()
+            x["q"].copy_(q_host, non_blocking=True)
+            fused()
+            out_host.copy_(out, non_blocking=True)
+            evs[1].record()
+
+        res["e2e_ms"] = timed_steps(step_e2e, args.steps, flush)[:, 0]
+        res["h2d"] = int(x["q"].numel() * x["q"].element_size())
+        res["d2h"] = int(out.numel() * out.element_size())
+    assert G.gsa_workspace_status(ws) == 0, "device status flags set"
+    return res
+
+
+def flat_summary(cfg, m, hbm):
+    ms = float(np.mean(m["step_ms"]))
+    ab = algorithmic_bytes(cfg, m["x"], m["sel"])
+    k = m["kern_ms"].mean(0)
+    return {"metric": "GSA decode head-queries/s", "value": round(cfg.head_queries / (ms / 1e3), 1),
+            "unit": UNIT, "ms_per_step": round(ms, 5),
+            "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(ab["total"] / (ms / 1e3) / 1e9, 1),
+                         "frac": round(ab["total"] / (ms / 1e3) / 1e9 / hbm, 4)},
+            "kernels_us": {"score_gists": round(float(k[0]) * 1e3, 2), "topk_select": round(float(k[1]) * 1e3, 2),
+                           "unfold_attend": round(float(k[2]) * 1e3, 2)},
+            "score_gists_gbs": round(score_kernel_bytes(cfg) / (k[0] / 1e3) / 1e9, 1),
+            "unfold_gbs": round((ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]) / (k[2] / 1e3) / 1e9, 1)}
+
+
+def measure_hgsa(G, W, cfg, dev, args, flush, hbm):
+    x = W.decode_inputs(cfg, device=dev)
+    B, hq, d = x["q"].shape
+    hkv, n_max, t_max, m_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2], x["meta_k"].shape[2]
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, cfg.exclude, 0.0, G.GSA_BF16, G.GSA_F32)
+    hd = G.make_hdesc(cfg.group, cfg.topk_meta, m_max)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_HGSA, hd), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    mi = torch.empty((B, hq, cfg.topk_meta), dtype=torch.int32, device=dev)
+    si = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ss = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+
+    def fused(evs=None):
+        if evs:
+            evs[0].record()
+        G.hgsa_decode(desc, hd, x["q"], x["meta_k"], x["meta_v"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"],
+                      x["n_gists"], x["own_len"], out, None, mi, si, ss, ws)
+        if evs:
+            evs[1].record()
+
+    def split(evs):
+        evs[0].record()
+        G.hgsa_select(desc, hd, x["q"], x["meta_k"], x["meta_v"], x["gist_k"], x["gist_v"], x["n_gists"], mi, si, ss,
+                      ws)
+        evs[1].record()
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], si, ss,
+                            G.GSA_PRIOR_HGSA, out, None, ws)
+        evs[2].record()
+
+    for _ in range(args.warmup):
+        flush()
+        fused()
+    step_ms = timed_steps(fused, args.steps, flush)[:, 0]
+    k = timed_steps(split, args.steps, flush, 2).mean(0)
+    assert G.gsa_workspace_status(ws) == 0
+    # algorithmic bytes: meta K+V, K+V of the chosen groups' children (union per
+    # (b, kv head)), raw K/V of the chosen chunks (union), own rows, q and out
+    e, G_ = 2, hq // hkv
+    M = cfg.n_gists // cfg.group
+    meta = B * hkv * M * d * e * 2
+    mic, sic = mi.reshape(B, hkv, G_, -1).cpu(), si.reshape(B, hkv, G_, -1).cpu()
+    ug = sum(int((torch.unique(mic[b, kv]) >= 0).sum()) for b in range(B) for kv in range(hkv))
+    uc = sum(int((torch.unique(sic[b, kv]) >= 0).sum()) for b in range(B) for kv in range(hkv))
+    total = meta + ug * cfg.group * d * e * 2 + uc * cfg.chunk * d * e * 2 + B * hkv * d * e * 2 + B * hq * d * (e + 4)
+    ms = float(np.mean(step_ms))
+    return {"metric": "GSA decode head-queries/s", "value": round(cfg.head_queries / (ms / 1e3), 1), "unit": UNIT,
+            "ms_per_step": round(ms, 5),
+            "step_hbm": {"alg_bytes": total, "achieved_gbs": round(total / (ms / 1e3) / 1e9, 1),
+                         "frac": round(total / (ms / 1e3) / 1e9 / hbm, 4)},
+            "kernels_us": {"hgsa_select": round(float(k[0]) * 1e3, 2), "unfold_attend": round(float(k[1]) * 1e3, 2)}}
+
+
+def measure_prefill(G, W, cfg, dev, args, flush, bf16_peak):
+    x = W.prefill_inputs(cfg, device=dev)
+    B, hq, L, d = x["q_raw"].shape
+    hkv, N = x["k_raw"].shape[1], x["k_gist"].shape[2]
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, N, L, cfg.topk, cfg.exclude, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_PREFILL), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out_raw = torch.empty((B, hq, L, d), dtype=torch.float32, device=dev)
+    out_gist = torch.empty((B, hq, N, d), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, hq, L, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, L, cfg.topk), dtype=torch.float32, device=dev)
+
+    def split(evs):
+        evs[0].record()
+        G.gsa_prefill_score(desc, x["q_raw"], x["q_gist"], x["k_gist"], sel, ssc, ws)
+        evs[1].record()
+        G.gsa_prefill_attend(desc, x["q_raw"], x["k_raw"], x["v_raw"], x["q_gist"], x["k_gist"], x["v_gist"], sel,
+                             ssc, out_raw, out_gist, ws)
+        evs[2].record()
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(max(1, min(args.warmup, 3))):
+        flush()
+        split([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    k = timed_steps(split, steps, flush, 2).mean(0)
+    assert G.gsa_workspace_status(ws) == 0
+    # scoring FLOPs: raw position in chunk m scores m gists (2*d FLOP each)
+    flops = B * hq * 2 * d * cfg.chunk * N * (N - 1) / 2
+    tf = flops / (k[0] / 1e3) / 1e12
+    tokens = B * (L + N)
+    return {"metric": "GSA prefill scoring TFLOP/s", "value": round(tf, 1), "unit": "TFLOP/s",
+            "scoring_ms": round(float(k[0]), 4), "attend_ms": round(float(k[1]), 4),
+            "prefill_tokens_per_s": round(tokens / ((k[0] + k[1]) / 1e3), 1), "scoring_alg_flops": flops,
+            "tensor_frac": round(tf / bf16_peak, 4), "steps": steps}
+
+
 def run_gsa(args, world, rank, local):
     import long_context_gsa_b200 as G
     import long_context_gsa_b200.workloads as W
@@ -187,139 +390,70 @@ def run_gsa(args, world, rank, local):
         import datetime
         torch.distributed.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
     cfg = W.CONFIGS[args.workload]
-    x = W.decode_inputs(cfg, device=dev, seed=cfg.seed + 1000 * rank)
-    B, hq, d = x["q"].shape
-    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
-    dt = G.GSA_BF16 if cfg.dtype == "bf16" else G.GSA_F32
-    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, cfg.exclude, 0.0, dt, G.GSA_F32)
-    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
-    G.gsa_workspace_init(ws)
-    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
-    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
-    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
-    scores = torch.empty((B, hq, n_max), dtype=torch.float32, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_w = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
-    flush_r = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.int32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.int32, device=dev)
-
-    class _Flush:
-        """Write a 2x-L2 buffer, then read another one so that the written
-        lines are evicted (written back) before the next timed step starts."""
-
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            torch.amax(flush_r, dim=0, out=flush_sink)
-
-    flush = _Flush()
-    stream = torch.cuda.current_stream()
-    prior = G.GSA_PRIOR_NONE if cfg.exclude else G.GSA_PRIOR_GISTS
-
-    def step_fused():
-        G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
-                     out, None, sel, ssc, ws)
-
-    def step_split(evs):
-        evs[0].record(stream)
-        G.gsa_score_gists(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores, ws)
-        evs[1].record(stream)
-        G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
-        evs[2].record(stream)
-        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
-                            prior, out, None, ws)
-        evs[3].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step_fused()
-    torch.cuda.synchronize()
+    flush = Flusher(dev)
+    hbm, bf16, peak_kind = peaks()
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    # (A) headline: fused decode steps, each bracketed by events, L2 flushed between
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
-        barrier()
-        for s in range(args.steps):
-            flush.zero_()
-            ev[s][0].record(stream)
-            step_fused()
-            ev[s][1].record(stream)
-        barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    local_ms = sum(step_ms)
-    clocks = clk.summary()
-
-    # (B) per-kernel durations: the same steps through the three entry points
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
-    for s in range(args.steps):
-        flush.zero_()
-        step_split(kev[s])
+    main = measure_flat(G, W, cfg, dev, args, flush, cfg.seed + 1000 * rank, e2e=True, clock_index=local)
     barrier()
-    kern_ms = np.array([[kev[s][i].elapsed_time(kev[s][i + 1]) for i in range(3)] for s in range(args.steps)])
-
-    # (C) end to end through the public call with host buffers: H2D q, decode, D2H out
-    q_host = x["q"].cpu().pin_memory()
-    out_host = torch.empty_like(out, device="cpu").pin_memory()
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier()
-    for s in range(args.steps):
-        flush.zero_()
-        eev[s][0].record(stream)
-        x["q"].copy_(q_host, non_blocking=True)
-        step_fused()
-        out_host.copy_(out, non_blocking=True)
-        eev[s][1].record(stream)
-    barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
-
-    t = torch.tensor([local_ms, e2e_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([float(np.sum(main["step_ms"])), float(np.sum(main["e2e_ms"]))], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     total_ms, total_e2e_ms = float(t[0]), float(t[1])
-    ab = algorithmic_bytes(cfg, x, sel)
+
+    extra = {}
+    if rank == 0 and world == 1 and not args.main_only:
+        for name in [n for n in args.extra.split(",") if n]:
+            c = W.CONFIGS[name]
+            if name.startswith("prefill"):
+                extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)
+            elif c.group:
+                extra[name] = measure_hgsa(G, W, c, dev, args, flush, hbm)
+            else:
+                m = measure_flat(G, W, c, dev, args, flush, c.seed)
+                extra[name] = flat_summary(c, m, hbm)
+                del m
+            torch.cuda.empty_cache()
+
     result = None
     if rank == 0:
-        hbm, bf16, peak_kind = peaks()
-        hq_total = cfg.head_queries * world * args.steps
-        value = hq_total / (total_ms / 1e3)
-        ms_step = total_ms / args.steps
-        k_avg = kern_ms.mean(0)
+        s = flat_summary(cfg, main, hbm)
+        value = cfg.head_queries * world * args.steps / (total_ms / 1e3)
+        k = main["kern_ms"].mean(0)
         names = ["score_gists", "topk_select", "unfold_attend"]
-        kb = score_kernel_bytes(cfg)
-        dom = int(np.argmax(k_avg))
-        dom_bytes = [kb, None, ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]][dom]
-        roof = None
-        if dom_bytes:
-            ach = dom_bytes / (k_avg[dom] / 1e3) / 1e9
-            roof = {"bound": "hbm", "kernel": names[dom], "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(ach / hbm, 4), "traffic": None, "peak_kind": peak_kind}
-        step_gbs = ab["total"] / (ms_step / 1e3) / 1e9
+        ab = algorithmic_bytes(cfg, main["x"], main["sel"])
+        kbytes = [score_kernel_bytes(cfg), 0, ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]]
+        dom = int(np.argmax(k))
+        ach = kbytes[dom] / (k[dom] / 1e3) / 1e9 if kbytes[dom] else None
+        roof = {"bound": "hbm", "kernel": names[dom], "achieved": round(ach, 1) if ach else None, "peak": hbm,
+                "unit": "GB/s", "frac": round(ach / hbm, 4) if ach else None,
+                "traffic": recorded_traffic(names[dom], cfg.name, kbytes[dom]), "peak_kind": peak_kind}
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "batch_per_gpu": cfg.batch, "hq": cfg.hq, "hkv": cfg.hkv, "d": cfg.d,
                        "context": cfg.context, "chunk": cfg.chunk, "n_gists": cfg.n_gists, "topk": cfg.topk,
-                       "exclude_unselected": cfg.exclude, "l2": "flushed between timed steps (2x-L2 buffer written, then another 2x-L2 buffer read so no dirty lines remain)",
+                       "exclude_unselected": cfg.exclude,
+                       "l2": "flushed between timed steps (2x-L2 buffer written, then another 2x-L2 buffer read "
+                             "so no dirty lines remain)",
                        "parallelism": f"dp{world} (independent rows per GPU)"},
             "roofline": roof,
-            "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(step_gbs, 1),
-                         "frac": round(step_gbs / hbm, 4), "union_chunks": ab["union_chunks"]},
-            "kernels_us": {n: round(float(v) * 1e3, 2) for n, v in zip(names, k_avg)},
+            "step_hbm": s["step_hbm"],
+            "kernels_us": s["kernels_us"],
             "e2e": {"value": round(cfg.head_queries * world * args.steps / (total_e2e_ms / 1e3), 1), "unit": UNIT,
-                    "h2d_bytes_per_step": int(x["q"].numel() * x["q"].element_size()),
-                    "d2h_bytes_per_step": int(out.numel() * out.element_size())},
-            "clocks": clocks,
+                    "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"]},
+            "clocks": main["clocks"],
             "gpu_launches": 3 * args.steps,
+            "workloads": extra,
         }
     if not args.no_cpu_baseline and rank == 0 and world == 1:
-        xh = host_copy(x)
+        xh = host_copy(main["x"])
         rate, calls, el, cores = oracle_rate(xh, cfg, cfg.head_queries, args.cpu_seconds)
         result["cpu_baseline"] = {"value": round(rate, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
                                   "sample": f"{calls} full steps of {cfg.head_queries} head-queries ({el:.1f} s)"}
@@ -327,6 +461,25 @@ def run_gsa(args, world, rank, local):
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     return result
+
+
+def recorded_traffic(kernel, workload, alg_bytes):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of that kernel; otherwise None."""
+    f = ROOT / "profiles" / "traffic.json"
+    if not f.exists():
+        return None
+    try:
+        rec = json.loads(f.read_text()).get(f"{kernel}/{workload}")
+    except ValueError:
+        return None
+    if not rec:
+        return None
+    import hashlib
+    src = ROOT / "long_context_gsa_b200" / "csrc" / rec["source"]
+    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != rec["sha"]:
+        return None
+    return rec["bytes"]
 
 
 # ---------------------------------------------------------- reference arm

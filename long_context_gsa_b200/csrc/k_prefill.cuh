@@ -10,14 +10,21 @@
 //
 // Stage 1 (this file, k_prefill_score): the dense part -- every query row
 // against every visible gist key -- on the 5th-generation tensor cores.
-// Persistent CTAs walk query tiles of 128 rows of one head (raw tiles, then
-// gist-query tiles, heaviest first).  Warp 0 issues TMA loads (Q tile, then
-// 256-gist key tiles into a 2-stage ring), warp 1 issues tcgen05.mma into
-// two 256-column TMEM accumulators, warps 2..5 (one TMEM lane quadrant each,
-// one query row per thread) read the scores with tcgen05.ld, apply the
-// block-causal mask, keep the row maximum and, for raw rows, a running
-// top-k in registers.  Outputs: sel_idx/sel_score (ascending chunk order)
-// and the row maximum that the attention stage uses as softmax reference.
+// Persistent CTAs walk query tiles of 128 rows of one head (gist-query
+// tiles, then raw tiles, heaviest first).  Warp 0 issues TMA loads (Q tile,
+// then 128-gist key tiles into a 3-stage ring), warp 1 issues tcgen05.mma
+// into two 128-column TMEM accumulators, warps 2..5 (one TMEM lane quadrant
+// each, one query row per thread) read the scores with tcgen05.ld, apply
+// the block-causal mask and keep the row maximum.  For raw rows the top-k
+// is found without per-value sorting: a score above the row's threshold is
+// appended to the row's candidate column in shared memory (column-major,
+// so appends of different rows never share a bank), and the candidates are
+// reduced to the best k only when the column fills and at the end of the
+// row.  The threshold starts from the first fully visible key tile: the
+// smallest of k group maxima (k disjoint column groups) is a lower bound on
+// the row's final k-th score, so nothing it discards can be selected.
+// Outputs: sel_idx/sel_score (ascending chunk order) and the row maximum
+// that the attention stage uses as softmax reference.
 #pragma once
 
 #include "tc100.cuh"
@@ -41,9 +48,11 @@ struct PrefillArgs {
 };
 
 constexpr int kPfRows = 128;        // query rows per tile (TMEM lanes)
-constexpr int kPfKeys = 256;        // gist keys per MMA tile (TMEM columns)
+constexpr int kPfKeys = 128;        // gist keys per MMA tile (TMEM columns)
 constexpr int kPfThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kPfTopkMax = 32;
+constexpr int kPfTopkMax = 16;
+constexpr int kPsThreads = 320;     // scoring: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (2 per row)
+constexpr int kPsCap = 48;          // candidate slots per row half (shared memory)
 
 struct PfTile {
   int is_gist, bh, row0, n_kt;
@@ -78,20 +87,127 @@ struct PfSmem {
   static constexpr uint32_t kKBlock = kPfKeys * 128;
   static constexpr uint32_t kKBytes = 2 * kKBlock;
   static constexpr uint32_t kQOff = 0;                       // 2 Q buffers
-  static constexpr uint32_t kKOff = 2 * kQBytes;             // 2 K stages
-  static constexpr uint32_t kBarOff = kKOff + 2 * kKBytes;
-  static constexpr uint32_t kBytes = kBarOff + 256 + 1024;   // + alignment slack
+  static constexpr uint32_t kKOff = 2 * kQBytes;             // kKStages K stages
+  static constexpr int kKStages = 2;
+  static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;  // [2 halves][kPsCap][128] x (score, index)
+  static constexpr uint32_t kXOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [128] x (bound, max) of half 1
+  static constexpr uint32_t kBarOff = kXOff + kPfRows * 8;
+  static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
 };
 
+// (score, index) ranking: higher score first, then lower index.
+__device__ __forceinline__ bool pf_before(float x, int xi, float y, int yi) { return x > y || (x == y && xi < yi); }
+
+// Drop this column's candidates that fall below `lb` (order kept).
+__device__ __noinline__ void pf_filter(uint2 *col, int &cnt, float lb) {
+  int w = 0;
+  for (int s = 0; s < cnt; ++s) {
+    const uint2 e = col[s * kPfRows];
+    if (__uint_as_float(e.x) >= lb) col[(w++) * kPfRows] = e;
+  }
+  cnt = w;
+}
+
+// Keep only this column's best KTOP candidates; returns the KTOP-th score
+// (a lower bound on the row's final k-th score) or -inf if fewer remain.
 template <int KTOP>
-__global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
+__device__ __noinline__ float pf_reduce(uint2 *col, int &cnt) {
+  float best[KTOP];
+  int bidx[KTOP];
+#pragma unroll
+  for (int e = 0; e < KTOP; ++e) {
+    best[e] = neg_inf();
+    bidx[e] = 0x7fffffff;
+  }
+  for (int s = 0; s < cnt; ++s) {
+    const uint2 en = col[s * kPfRows];
+    float x = __uint_as_float(en.x);
+    int xi = static_cast<int>(en.y);
+#pragma unroll
+    for (int q = 0; q < KTOP; ++q)
+      if (pf_before(x, xi, best[q], bidx[q])) {
+        const float tv = best[q];
+        const int ti = bidx[q];
+        best[q] = x;
+        bidx[q] = xi;
+        x = tv;
+        xi = ti;
+      }
+  }
+  cnt = min(cnt, KTOP);
+  for (int e = 0; e < cnt; ++e) col[e * kPfRows] = make_uint2(__float_as_uint(best[e]), static_cast<uint32_t>(bidx[e]));
+  return cnt == KTOP ? best[KTOP - 1] : neg_inf();
+}
+
+// Final selection of one row from both halves' candidates (those >= lb):
+// the best `topk` by (score desc, index asc), written in ascending chunk
+// order with scores scaled (-1 / -inf padding).
+template <int KTOP>
+__device__ __noinline__ void pf_emit(const uint2 *c0, int n0, const uint2 *c1, int n1, float lb, int topk, float scale,
+                                     int32_t *oi, float *os) {
+  float best[KTOP];
+  int bidx[KTOP];
+#pragma unroll
+  for (int e = 0; e < KTOP; ++e) {
+    best[e] = neg_inf();
+    bidx[e] = 0x7fffffff;
+  }
+  for (int h = 0; h < 2; ++h) {
+    const uint2 *col = h ? c1 : c0;
+    const int n = h ? n1 : n0;
+    for (int s = 0; s < n; ++s) {
+      const uint2 en = col[s * kPfRows];
+      float x = __uint_as_float(en.x);
+      if (!(x >= lb)) continue;
+      int xi = static_cast<int>(en.y);
+#pragma unroll
+      for (int q = 0; q < KTOP; ++q)
+        if (pf_before(x, xi, best[q], bidx[q])) {
+          const float tv = best[q];
+          const int ti = bidx[q];
+          best[q] = x;
+          bidx[q] = xi;
+          x = tv;
+          xi = ti;
+        }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < KTOP; ++e)
+    if (e >= topk || best[e] == neg_inf()) bidx[e] = -1;
+#pragma unroll
+  for (int i = 1; i < KTOP; ++i)
+#pragma unroll
+    for (int j2 = KTOP - 1; j2 >= i; --j2) {
+      const unsigned x = static_cast<unsigned>(bidx[j2 - 1]), y = static_cast<unsigned>(bidx[j2]);
+      if (x > y) {  // -1 sorts last as unsigned
+        bidx[j2 - 1] = static_cast<int>(y);
+        bidx[j2] = static_cast<int>(x);
+        const float tv = best[j2 - 1];
+        best[j2 - 1] = best[j2];
+        best[j2] = tv;
+      }
+    }
+#pragma unroll
+  for (int e = 0; e < KTOP; ++e)
+    if (e < topk) {
+      oi[e] = bidx[e];
+      os[e] = bidx[e] >= 0 ? best[e] * scale : neg_inf();
+    }
+}
+
+template <int KTOP>
+__global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PfSmem::kBarOff);
-  uint64_t *q_full = bars, *q_empty = bars + 2, *k_full = bars + 4, *k_empty = bars + 6;
-  uint64_t *acc_full = bars + 8, *acc_empty = bars + 10;
-  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 12);
-  int *abort_s = reinterpret_cast<int *>(bars + 13);
+  uint64_t *q_full = bars, *q_empty = bars + 2, *k_full = bars + 4, *k_empty = bars + 7;
+  uint64_t *acc_full = bars + 10, *acc_empty = bars + 12;
+  uint64_t *pair_bar = bars + 14;  // [4]: the two epilogue warps of one TMEM quadrant
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 18);
+  int *abort_s = reinterpret_cast<int *>(bars + 19);
+  uint2 *cand = reinterpret_cast<uint2 *>(smem + PfSmem::kCandOff);   // [2][kPsCap][128] (score bits, index)
+  float2 *xchg = reinterpret_cast<float2 *>(smem + PfSmem::kXOff);     // [128] (bound, max) of half 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.bh * (a.gist_tiles + a.raw_tiles);
@@ -100,18 +216,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 8 * 32);
+    }
+    for (int i = 0; i < PfSmem::kKStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4 * 32);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 64);
     *abort_s = 0;
     mbar_fence_init();
     tc::prefetch_map(&a.tm_qraw);
     tc::prefetch_map(&a.tm_qgist);
     tc::prefetch_map(&a.tm_kgist);
   }
-  if (warp == 1) tc::tmem_alloc(tmem_base_s, 512);
+  if (warp == 1) tc::tmem_alloc(tmem_base_s, 256);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -144,8 +263,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
         bool ok = true;
         for (int j = 0; j < tl.n_kt; ++j, ++ki) {
-          const int ks = ki & 1;
-          if (!wait(&k_empty[ks], ((ki >> 1) & 1) ^ 1)) {
+          const int ks = ki % PfSmem::kKStages;
+          if (!wait(&k_empty[ks], ((ki / PfSmem::kKStages) & 1) ^ 1)) {
             ok = false;
             break;
           }
@@ -171,8 +290,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
         if (!wait(&q_full[qs], (qi >> 1) & 1)) break;
         bool ok = true;
         for (int j = 0; j < tl.n_kt; ++j, ++ki, ++ai) {
-          const int ks = ki & 1, as = ai & 1;
-          if (!wait(&k_full[ks], (ki >> 1) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
+          const int ks = ki % PfSmem::kKStages, as = ai & 1;
+          if (!wait(&k_full[ks], (ki / PfSmem::kKStages) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
             ok = false;
             break;
           }
@@ -194,24 +313,36 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
       }
     }
   } else {
-    // ---------------- epilogue: one query row per thread ----------------
-    const int quad = warp & 3;
+    // ---------------- epilogue: two threads per query row ----------------
+    // Warp w reads TMEM lane quadrant w % 4; half (w - 2) / 4 takes columns
+    // [64*half, 64*half + 64) of every key tile.  Per score: one fmax into
+    // one of 16 slot maxima (each slot a disjoint set of columns, so the
+    // smallest slot maximum bounds the row's k-th score from below), one
+    // compare with that bound and one predicated append of (score, index).
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
-    uint32_t ai = 0;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    uint2 *col = cand + half * kPsCap * kPfRows + r;  // slot s at col[s * 128]
+    const float nan = __int_as_float(0x7fffffff);
+    uint32_t ai = 0, pair_phase = 0;
+    // both warps of the quadrant meet here (bounded wait, like every wait)
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&pair_bar[quad]);
+      const bool okp = wait(&pair_bar[quad], pair_phase);
+      pair_phase ^= 1;
+      return okp;
+    };
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const PfTile tl = pf_tile(a, t);
       const int row = tl.row0 + r;
       const bool row_ok = row < (tl.is_gist ? a.n_chunks : a.L);
       const int limit = !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, row / a.chunk));
-      float best[KTOP];
-      int bidx[KTOP];
+      const bool want_topk = !tl.is_gist && a.topk > 0;
+      float G[16];
 #pragma unroll
-      for (int e = 0; e < KTOP; ++e) {
-        best[e] = neg_inf();
-        bidx[e] = -1;
-      }
-      float thr = neg_inf(), mx = neg_inf();
-      const bool want_topk = !tl.is_gist;
+      for (int s = 0; s < 16; ++s) G[s] = neg_inf();
+      float mx = neg_inf(), floor_lb = neg_inf();
+      int cnt = 0;
       bool ok = true;
       for (int j = 0; j < tl.n_kt; ++j, ++ai) {
         const int as = ai & 1;
@@ -220,73 +351,66 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
           break;
         }
         tc::fence_after_sync();
-        const int t0 = j * kPfKeys;
 #pragma unroll 1
-        for (int c = 0; c < kPfKeys / 32; ++c) {
+        for (int b = 0; b < 2; ++b) {
+          const int tb = j * kPfKeys + half * 64 + b * 32;
           float v[32];
           __syncwarp();  // tcgen05.ld is warp-collective
-          tc::ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + as * kPfKeys + c * 32, v);
-          const int tb = t0 + c * 32;
+          tc::ld32(lane_addr + as * kPfKeys + half * 64 + b * 32, v);
+          if (tb + 32 > limit)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float s = v[e] * a.scale;
-            if (tb + e < limit) {
-              mx = fmaxf(mx, s);
-              if (want_topk && s > thr) {
-                float cv = s;
-                int ci = tb + e;
+            for (int e = 0; e < 32; ++e)
+              if (tb + e >= limit) v[e] = nan;  // masked: fails every compare, ignored by fmax
 #pragma unroll
-                for (int q = 0; q < KTOP; ++q) {
-                  if (cv > best[q]) {
-                    const float tv = best[q];
-                    const int ti = bidx[q];
-                    best[q] = cv;
-                    bidx[q] = ci;
-                    cv = tv;
-                    ci = ti;
-                  }
-                }
-                thr = best[KTOP - 1];
-              }
-            }
+          for (int e = 0; e < 32; ++e) G[e >> 1] = fmaxf(G[e >> 1], v[e]);
+          if (!want_topk) continue;
+          float lb = G[0];
+#pragma unroll
+          for (int s = 1; s < 16; ++s) lb = fminf(lb, G[s]);
+          lb = fmaxf(lb, floor_lb);
+          if (cnt > kPsCap - 32) {  // room for a full batch of appends
+            pf_filter(col, cnt, lb);
+            if (cnt > kPsCap - 32) floor_lb = fmaxf(floor_lb, pf_reduce<KTOP>(col, cnt));
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (v[e] >= lb) {
+              col[cnt * kPfRows] = make_uint2(__float_as_uint(v[e]), static_cast<uint32_t>(tb + e));
+              ++cnt;
+            }
         }
         tc::fence_before_sync();
         mbar_arrive(&acc_empty[as]);
       }
       if (!ok) break;
-      if (!row_ok) continue;
-      const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
-      if (tl.is_gist) {
-        a.rec_gist[orow * (128 + kPartHeader)] = mx == neg_inf() ? mx : mx * kLog2e;
-        continue;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) mx = fmaxf(mx, G[s]);
+      float lb = G[0];
+#pragma unroll
+      for (int s = 1; s < 16; ++s) lb = fminf(lb, G[s]);
+      lb = fmaxf(lb, floor_lb);
+      // half 1 hands its bound and maximum to half 0, which writes the row;
+      // a NaN score marks the end of a column that is not full
+      if (half == 1) {
+        xchg[r] = make_float2(lb, mx);
+        if (cnt < kPsCap) col[cnt * kPfRows] = make_uint2(0x7fffffffu, 0u);
       }
-      a.rec_raw[orow * (128 + kPartHeader)] = mx == neg_inf() ? mx : mx * kLog2e;
-      // keep the first topk of the ranked list, report in ascending chunk order
-#pragma unroll
-      for (int e = 0; e < KTOP; ++e)
-        if (e >= a.topk) bidx[e] = -1;
-#pragma unroll
-      for (int i = 1; i < KTOP; ++i)
-#pragma unroll
-        for (int j2 = KTOP - 1; j2 >= i; --j2) {
-          const unsigned x = static_cast<unsigned>(bidx[j2 - 1]), y = static_cast<unsigned>(bidx[j2]);
-          if (x > y) {  // -1 sorts last as unsigned
-            bidx[j2 - 1] = static_cast<int>(y);
-            bidx[j2] = static_cast<int>(x);
-            const float tv = best[j2 - 1];
-            best[j2 - 1] = best[j2];
-            best[j2] = tv;
-          }
+      if (!pair_sync()) break;
+      if (half == 0 && row_ok) {
+        const float2 o = xchg[r];
+        mx = fmaxf(mx, o.y);
+        const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
+        float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
+        rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
+        if (want_topk) {
+          const uint2 *c1 = cand + kPsCap * kPfRows + r;
+          int n1 = 0;
+          while (n1 < kPsCap && c1[n1 * kPfRows].x != 0x7fffffffu) ++n1;
+          pf_emit<KTOP>(col, cnt, c1, n1, fmaxf(lb, o.x), a.topk, a.scale, a.sel_idx + orow * a.topk,
+                        a.sel_score + orow * a.topk);
         }
-      int32_t *oi = a.sel_idx + orow * a.topk;
-      float *os = a.sel_score + orow * a.topk;
-#pragma unroll
-      for (int e = 0; e < KTOP; ++e)
-        if (e < a.topk) {
-          oi[e] = bidx[e];
-          os[e] = bidx[e] >= 0 ? best[e] : neg_inf();
-        }
+      }
+      if (!pair_sync()) break;
     }
   }
 
@@ -294,7 +418,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_score(const __grid_co
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 512);
+    tc::tmem_dealloc(tmem, 256);
   }
 }
 

@@ -106,7 +106,8 @@ SMALL = [
     ("n40_c16_k4", dict(batch=1, hq=4, hkv=2, chunk=16, n_chunks=40, topk=4)),
     ("n300_c8_k16", dict(batch=1, hq=8, hkv=2, chunk=8, n_chunks=300, topk=16)),
     ("ragged_tile_n37", dict(batch=2, hq=2, hkv=1, chunk=16, n_chunks=37, topk=5)),
-    ("k32_n520_c4", dict(batch=1, hq=4, hkv=1, chunk=4, n_chunks=520, topk=32)),
+    ("k16_n520_c4", dict(batch=1, hq=4, hkv=1, chunk=4, n_chunks=520, topk=16)),
+    ("k1_n200_c8", dict(batch=1, hq=2, hkv=2, chunk=8, n_chunks=200, topk=1)),
 ]
 
 
