@@ -454,7 +454,7 @@ bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
-  if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;  // candidate columns hold 16 kept + 32 new
+  if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;  // running top-k lists hold at most 16
   if (static_cast<int64_t>(d->n_max) * d->chunk != d->t_max) return GSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
   return GSA_OK;
@@ -493,7 +493,8 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
     return GSA_ERR_CUDA;
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
   const int grid = std::min(total, sm_count());
-  return launch(k_prefill_score<16>, dim3(grid), dim3(kPsThreads), PfSmem::kBytes, stream, pa);
+  auto kern = d->topk <= 4 ? k_prefill_score<4> : d->topk <= 8 ? k_prefill_score<8> : k_prefill_score<16>;
+  return launch(kern, dim3(grid), dim3(kPsThreads), PfSmem::kBytes, stream, pa);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,

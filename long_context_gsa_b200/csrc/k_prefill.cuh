@@ -12,17 +12,18 @@
 // against every visible gist key -- on the 5th-generation tensor cores.
 // Persistent CTAs walk query tiles of 128 rows of one head (gist-query
 // tiles, then raw tiles, heaviest first).  Warp 0 issues TMA loads (Q tile,
-// then 128-gist key tiles into a 3-stage ring), warp 1 issues tcgen05.mma
-// into two 128-column TMEM accumulators, warps 2..5 (one TMEM lane quadrant
-// each, one query row per thread) read the scores with tcgen05.ld, apply
-// the block-causal mask and keep the row maximum.  For raw rows the top-k
-// is found without per-value sorting: a score above the row's threshold is
-// appended to the row's candidate column in shared memory (column-major,
-// so appends of different rows never share a bank), and the candidates are
-// reduced to the best k only when the column fills and at the end of the
-// row.  The threshold starts from the first fully visible key tile: the
-// smallest of k group maxima (k disjoint column groups) is a lower bound on
-// the row's final k-th score, so nothing it discards can be selected.
+// then 128-gist key tiles into a 2-stage ring), warp 1 issues tcgen05.mma
+// into two 128-column TMEM accumulators, and warps 2..9 (two per TMEM lane
+// quadrant, so two threads per query row, each owning half of the key
+// columns) read the scores with tcgen05.ld, apply the block-causal mask and
+// keep the row maximum.  For raw rows the top-k runs against a lower bound
+// on the row's final k-th score: each half keeps the K largest scores it
+// has appended (sorted, values only) and the partner half's K-th is read
+// once per key tile; only scores above the bound are appended as (score,
+// index) candidates to a per-row column in shared memory (column-major, so
+// appends of different rows never share a bank).  At the end of the row one
+// thread merges both halves' lists into the k-th score and walks both
+// columns in ascending index order.
 // Outputs: sel_idx/sel_score (ascending chunk order) and the row maximum
 // that the attention stage uses as softmax reference.
 #pragma once
@@ -52,7 +53,7 @@ constexpr int kPfKeys = 128;        // gist keys per MMA tile (TMEM columns)
 constexpr int kPfThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kPfTopkMax = 16;
 constexpr int kPsThreads = 320;     // scoring: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (2 per row)
-constexpr int kPsCap = 48;          // candidate slots per row half (shared memory)
+constexpr int kPsCap = 38;          // candidate slots per row half (shared memory)
 
 struct PfTile {
   int is_gist, bh, row0, n_kt;
@@ -89,42 +90,135 @@ struct PfSmem {
   static constexpr uint32_t kQOff = 0;                       // 2 Q buffers
   static constexpr uint32_t kKOff = 2 * kQBytes;             // kKStages K stages
   static constexpr int kKStages = 2;
-  static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;  // [2 halves][kPsCap][128] x (score, index)
-  static constexpr uint32_t kXOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [128] x (bound, max) of half 1
-  static constexpr uint32_t kBarOff = kXOff + kPfRows * 8;
+  static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;           // [2 halves][kPsCap][128] (score, index)
+  static constexpr uint32_t kListOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [2][kPfTopkMax][128] best values
+  static constexpr uint32_t kThrOff = kListOff + 2 * kPfTopkMax * kPfRows * 4;  // [2][128] (threshold, tile tag)
+  static constexpr uint32_t kCntOff = kThrOff + 2 * kPfRows * 8;             // [2][128] filtered candidate counts
+  static constexpr uint32_t kBarOff = kCntOff + 2 * kPfRows * 4;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
 };
+static_assert(PfSmem::kBytes <= 232448, "prefill scoring shared memory");
+
+constexpr uint32_t kPsSlot = kPfRows * 8;  // bytes between consecutive slots of one row's column
 
 // (score, index) ranking: higher score first, then lower index.
 __device__ __forceinline__ bool pf_before(float x, int xi, float y, int yi) { return x > y || (x == y && xi < yi); }
 
-// Drop this column's candidates that fall below `lb` (order kept).
-__device__ __noinline__ void pf_filter(uint2 *col, int &cnt, float lb) {
-  int w = 0;
-  for (int s = 0; s < cnt; ++s) {
-    const uint2 e = col[s * kPfRows];
-    if (__uint_as_float(e.x) >= lb) col[(w++) * kPfRows] = e;
-  }
-  cnt = w;
+__device__ __forceinline__ uint2 lds_u2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
 }
 
-// Keep only this column's best KTOP candidates; returns the KTOP-th score
-// (a lower bound on the row's final k-th score) or -inf if fewer remain.
-template <int KTOP>
-__device__ __noinline__ float pf_reduce(uint2 *col, int &cnt) {
-  float best[KTOP];
-  int bidx[KTOP];
+__device__ __forceinline__ void sts_u2(uint32_t a, uint2 v) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Append (v, idx) at the column cursor `cur` when v > thr (GE: v >= thr),
+// without a branch: the store and the cursor step are predicated.  NaN
+// (a masked score) fails both compares.
+template <bool GE>
+__device__ __forceinline__ void pf_append(uint32_t &cur, float v, float thr, uint32_t idx) {
+  if (GE)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ge.f32 p, %1, %2;\n\t"
+        "@p st.shared.v2.u32 [%0], {%3, %4};\n\t"
+        "@p add.u32 %0, %0, %5;\n\t}\n"
+        : "+r"(cur)
+        : "f"(v), "f"(thr), "r"(__float_as_uint(v)), "r"(idx), "n"(kPsSlot)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.gt.f32 p, %1, %2;\n\t"
+        "@p st.shared.v2.u32 [%0], {%3, %4};\n\t"
+        "@p add.u32 %0, %0, %5;\n\t}\n"
+        : "+r"(cur)
+        : "f"(v), "f"(thr), "r"(__float_as_uint(v)), "r"(idx), "n"(kPsSlot)
+        : "memory");
+}
+
+// Values-only insertion into a descending list (the running top K).
+template <int K>
+__device__ __forceinline__ void pf_insert(float (&b)[K], float x) {
 #pragma unroll
-  for (int e = 0; e < KTOP; ++e) {
+  for (int q = 0; q < K; ++q) {
+    const float hi = fmaxf(b[q], x);
+    x = fminf(b[q], x);
+    b[q] = hi;
+  }
+}
+
+// Descending bitonic sort of 32 values in registers (no NaN inputs).
+__device__ __forceinline__ void pf_sort32(float (&w)[32]) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const float x = w[i], y = w[l];
+          const bool desc = (i & k) == 0;
+          w[i] = desc ? fmaxf(x, y) : fminf(x, y);
+          w[l] = desc ? fminf(x, y) : fmaxf(x, y);
+        }
+      }
+}
+
+// Store v at a when p (predicated, no branch).
+__device__ __forceinline__ void sts_u2_if(bool p, uint32_t a, uint2 v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.shared.v2.u32 [%1], {%2, %3};\n\t}\n" ::"r"(
+          static_cast<uint32_t>(p)),
+      "r"(a), "r"(v.x), "r"(v.y)
+      : "memory");
+}
+
+// Keep the column's candidates with score >= lb (order kept).  Called by
+// the whole warp (one column per lane): the loop runs to the longest
+// column, four slots per step with the loads issued together; a lane's
+// slots past its cursor are read but neither kept nor counted (every
+// address read lies inside the column's kPsCap slots).  Returns the cursor.
+__device__ __forceinline__ uint32_t pf_filter(uint32_t base, uint32_t cur, float lb) {
+  const int n = static_cast<int>((cur - base) / kPsSlot);
+  const int nmax = __reduce_max_sync(0xffffffffu, n);
+  uint32_t w = base;
+  for (int s = 0; s < nmax; s += 4) {
+    uint2 e[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) e[u] = lds_u2(base + min(s + u, kPsCap - 1) * kPsSlot);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool live = s + u < n;
+      sts_u2_if(live, w, e[u]);  // w <= s + u: never overwrites an unread slot
+      w += (live && __uint_as_float(e[u].x) >= lb) ? kPsSlot : 0u;
+    }
+  }
+  return w;
+}
+
+// Rare path (many exactly equal scores): keep the column's best K
+// candidates by (score desc, index asc), left in ascending index order;
+// returns the new cursor.
+template <int K>
+__device__ __noinline__ uint32_t pf_reduce(uint32_t base, uint32_t cur) {
+  float best[K];
+  int bidx[K];
+#pragma unroll
+  for (int e = 0; e < K; ++e) {
     best[e] = neg_inf();
     bidx[e] = 0x7fffffff;
   }
-  for (int s = 0; s < cnt; ++s) {
-    const uint2 en = col[s * kPfRows];
+  int cnt = 0;
+  for (uint32_t s = base; s < cur; s += kPsSlot, ++cnt) {
+    const uint2 en = lds_u2(s);
     float x = __uint_as_float(en.x);
     int xi = static_cast<int>(en.y);
 #pragma unroll
-    for (int q = 0; q < KTOP; ++q)
+    for (int q = 0; q < K; ++q)
       if (pf_before(x, xi, best[q], bidx[q])) {
         const float tv = best[q];
         const int ti = bidx[q];
@@ -134,69 +228,32 @@ __device__ __noinline__ float pf_reduce(uint2 *col, int &cnt) {
         xi = ti;
       }
   }
-  cnt = min(cnt, KTOP);
-  for (int e = 0; e < cnt; ++e) col[e * kPfRows] = make_uint2(__float_as_uint(best[e]), static_cast<uint32_t>(bidx[e]));
-  return cnt == KTOP ? best[KTOP - 1] : neg_inf();
-}
-
-// Final selection of one row from both halves' candidates (those >= lb):
-// the best `topk` by (score desc, index asc), written in ascending chunk
-// order with scores scaled (-1 / -inf padding).
-template <int KTOP>
-__device__ __noinline__ void pf_emit(const uint2 *c0, int n0, const uint2 *c1, int n1, float lb, int topk, float scale,
-                                     int32_t *oi, float *os) {
-  float best[KTOP];
-  int bidx[KTOP];
+  const int n = min(cnt, K);
 #pragma unroll
-  for (int e = 0; e < KTOP; ++e) {
-    best[e] = neg_inf();
-    bidx[e] = 0x7fffffff;
-  }
-  for (int h = 0; h < 2; ++h) {
-    const uint2 *col = h ? c1 : c0;
-    const int n = h ? n1 : n0;
-    for (int s = 0; s < n; ++s) {
-      const uint2 en = col[s * kPfRows];
-      float x = __uint_as_float(en.x);
-      if (!(x >= lb)) continue;
-      int xi = static_cast<int>(en.y);
+  for (int i = 1; i < K; ++i)
 #pragma unroll
-      for (int q = 0; q < KTOP; ++q)
-        if (pf_before(x, xi, best[q], bidx[q])) {
-          const float tv = best[q];
-          const int ti = bidx[q];
-          best[q] = x;
-          bidx[q] = xi;
-          x = tv;
-          xi = ti;
-        }
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < KTOP; ++e)
-    if (e >= topk || best[e] == neg_inf()) bidx[e] = -1;
-#pragma unroll
-  for (int i = 1; i < KTOP; ++i)
-#pragma unroll
-    for (int j2 = KTOP - 1; j2 >= i; --j2) {
-      const unsigned x = static_cast<unsigned>(bidx[j2 - 1]), y = static_cast<unsigned>(bidx[j2]);
-      if (x > y) {  // -1 sorts last as unsigned
-        bidx[j2 - 1] = static_cast<int>(y);
-        bidx[j2] = static_cast<int>(x);
+    for (int j2 = K - 1; j2 >= i; --j2)
+      if (bidx[j2 - 1] > bidx[j2]) {  // unused slots hold INT_MAX and sort last
+        const int ti = bidx[j2 - 1];
+        bidx[j2 - 1] = bidx[j2];
+        bidx[j2] = ti;
         const float tv = best[j2 - 1];
         best[j2 - 1] = best[j2];
         best[j2] = tv;
       }
-    }
 #pragma unroll
-  for (int e = 0; e < KTOP; ++e)
-    if (e < topk) {
-      oi[e] = bidx[e];
-      os[e] = bidx[e] >= 0 ? best[e] * scale : neg_inf();
-    }
+  for (int e = 0; e < K; ++e)
+    if (e < n) sts_u2(base + e * kPsSlot, make_uint2(__float_as_uint(best[e]), static_cast<uint32_t>(bidx[e])));
+  return base + n * kPsSlot;
 }
 
-template <int KTOP>
+// A value a little below x (x itself for -inf): comparing v > below(x)
+// keeps every v >= x.
+__device__ __forceinline__ float pf_below(float x) { return fmaf(-fabsf(x), 1e-6f, x) - 1e-30f; }
+
+// Stage 1, k_prefill_score<K>: scores, row maxima and the top-k selection
+// (topk <= K) of every query row.
+template <int K>
 __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -206,8 +263,9 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
   uint64_t *pair_bar = bars + 14;  // [4]: the two epilogue warps of one TMEM quadrant
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 18);
   int *abort_s = reinterpret_cast<int *>(bars + 19);
-  uint2 *cand = reinterpret_cast<uint2 *>(smem + PfSmem::kCandOff);   // [2][kPsCap][128] (score bits, index)
-  float2 *xchg = reinterpret_cast<float2 *>(smem + PfSmem::kXOff);     // [128] (bound, max) of half 1
+  float *lists = reinterpret_cast<float *>(smem + PfSmem::kListOff);
+  float2 *thr_x = reinterpret_cast<float2 *>(smem + PfSmem::kThrOff);
+  int *cnt_x = reinterpret_cast<int *>(smem + PfSmem::kCntOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.bh * (a.gist_tiles + a.raw_tiles);
@@ -230,6 +288,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     tc::prefetch_map(&a.tm_qgist);
     tc::prefetch_map(&a.tm_kgist);
   }
+  for (int i = threadIdx.x; i < 2 * kPfRows; i += blockDim.x) thr_x[i] = make_float2(neg_inf(), __int_as_float(-1));
   if (warp == 1) tc::tmem_alloc(tmem_base_s, 256);
   tc::fence_before_sync();
   __syncthreads();
@@ -314,18 +373,24 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     }
   } else {
     // ---------------- epilogue: two threads per query row ----------------
-    // Warp w reads TMEM lane quadrant w % 4; half (w - 2) / 4 takes columns
-    // [64*half, 64*half + 64) of every key tile.  Per score: one fmax into
-    // one of 16 slot maxima (each slot a disjoint set of columns, so the
-    // smallest slot maximum bounds the row's k-th score from below), one
-    // compare with that bound and one predicated append of (score, index).
+    // Warp w reads TMEM lane quadrant w % 4; half h = (w - 2) / 4 takes
+    // columns [64h, 64h + 64) of every key tile, in ascending order.  Each
+    // half keeps the K largest scores it has appended (values only, sorted
+    // descending); its K-th is a lower bound on the row's final k-th score,
+    // and so is the partner half's, published once per key tile.  A score is
+    // appended as a (score, index) candidate only when it beats that bound,
+    // so after the first key tile few scores are appended at all; appends
+    // are predicated stores, never branches.  Equal scores: a score equal
+    // to the own bound is not appended (K earlier, lower-index scores of
+    // this half already rank ahead of it); one equal to the partner's is.
     const int quad = warp & 3, half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    uint2 *col = cand + half * kPsCap * kPfRows + r;  // slot s at col[s * 128]
+    const uint32_t base = smem_u32(smem + PfSmem::kCandOff) + (half * kPsCap * kPfRows + r) * 8u;
+    const uint32_t base1 = smem_u32(smem + PfSmem::kCandOff) + (kPsCap * kPfRows + r) * 8u;
+    const uint32_t room = base + (kPsCap - 8) * kPsSlot;  // a cursor beyond this leaves < 8 free slots
     const float nan = __int_as_float(0x7fffffff);
     uint32_t ai = 0, pair_phase = 0;
-    // both warps of the quadrant meet here (bounded wait, like every wait)
     auto pair_sync = [&]() -> bool {
       mbar_arrive(&pair_bar[quad]);
       const bool okp = wait(&pair_bar[quad], pair_phase);
@@ -338,77 +403,167 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       const bool row_ok = row < (tl.is_gist ? a.n_chunks : a.L);
       const int limit = !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, row / a.chunk));
       const bool want_topk = !tl.is_gist && a.topk > 0;
-      float G[16];
+      float bst[K];
 #pragma unroll
-      for (int s = 0; s < 16; ++s) G[s] = neg_inf();
-      float mx = neg_inf(), floor_lb = neg_inf();
-      int cnt = 0;
+      for (int q = 0; q < K; ++q) bst[q] = neg_inf();
+      float mx = neg_inf(), thr = neg_inf(), tp = neg_inf();
+      uint32_t cur = base, c0 = base;  // column cursor; entries [c0, cur) not yet in bst
+      // fold the candidates appended since the last call into bst (whole
+      // warp; -inf pads the lanes with fewer, and inserting -inf changes
+      // nothing)
+      auto absorb = [&]() {
+        const int n = static_cast<int>((cur - c0) / kPsSlot);
+        const int nmax = __reduce_max_sync(0xffffffffu, n);
+        const uint32_t last = base + (kPsCap - 1) * kPsSlot;
+        for (int s = 0; s < nmax; s += 4) {
+          float x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float y = __uint_as_float(lds_u2(min(c0 + (s + u) * kPsSlot, last)).x);
+            x[u] = s + u < n ? y : neg_inf();
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) pf_insert<K>(bst, x[u]);
+        }
+        c0 = cur;
+      };
       bool ok = true;
       for (int j = 0; j < tl.n_kt; ++j, ++ai) {
         const int as = ai & 1;
-        if (!wait(&acc_full[as], (ai >> 1) & 1)) {
+        if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai >> 1) & 1))) {  // warp-uniform outcome
           ok = false;
           break;
         }
         tc::fence_after_sync();
+        const bool edge = __any_sync(0xffffffffu, (j + 1) * kPfKeys > limit);  // some row ends in this tile
 #pragma unroll 1
         for (int b = 0; b < 2; ++b) {
           const int tb = j * kPfKeys + half * 64 + b * 32;
           float v[32];
           __syncwarp();  // tcgen05.ld is warp-collective
           tc::ld32(lane_addr + as * kPfKeys + half * 64 + b * 32, v);
-          if (tb + 32 > limit)
+          if (edge)
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (tb + e >= limit) v[e] = nan;  // masked: fails every compare, ignored by fmax
+            for (int e = 0; e < 32; ++e) v[e] = tb + e < limit ? v[e] : nan;  // masked: fails every compare
+          if (!want_topk) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) G[e >> 1] = fmaxf(G[e >> 1], v[e]);
-          if (!want_topk) continue;
-          float lb = G[0];
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+            continue;
+          }
+          if (j == 0 && b == 0) {
+            // first block: its K largest seed the list; append those >= the K-th
+            float w[32];
 #pragma unroll
-          for (int s = 1; s < 16; ++s) lb = fminf(lb, G[s]);
-          lb = fmaxf(lb, floor_lb);
-          if (cnt > kPsCap - 32) {  // room for a full batch of appends
-            pf_filter(col, cnt, lb);
-            if (cnt > kPsCap - 32) floor_lb = fmaxf(floor_lb, pf_reduce<KTOP>(col, cnt));
+            for (int e = 0; e < 32; ++e) w[e] = v[e] == v[e] ? v[e] : neg_inf();
+            pf_sort32(w);
+#pragma unroll
+            for (int q = 0; q < K; ++q) bst[q] = w[q];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pf_append<true>(cur, v[e], bst[K - 1], static_cast<uint32_t>(tb + e));
+            c0 = cur;
+            thr = bst[K - 1];
+            continue;
           }
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (v[e] >= lb) {
-              col[cnt * kPfRows] = make_uint2(__float_as_uint(v[e]), static_cast<uint32_t>(tb + e));
-              ++cnt;
+          for (int g = 0; g < 4; ++g) {
+            if (__any_sync(0xffffffffu, cur > room)) {
+              // some lane has fewer than 8 free slots: every lane drops
+              // what can no longer be selected (one pass for the warp)
+              absorb();
+              cur = pf_filter(base, cur, fmaxf(bst[K - 1], tp));
+              if (cur > room) cur = pf_reduce<K>(base, cur);  // only under many equal scores
+              c0 = cur;
+              thr = fmaxf(bst[K - 1], pf_below(tp));
             }
+#pragma unroll
+            for (int e = 8 * g; e < 8 * g + 8; ++e) pf_append<false>(cur, v[e], thr, static_cast<uint32_t>(tb + e));
+          }
         }
         tc::fence_before_sync();
         mbar_arrive(&acc_empty[as]);
+        if (want_topk) {  // update the list, publish this half's bound, take the partner's
+          absorb();
+          thr_x[half * kPfRows + r] = make_float2(bst[K - 1], __int_as_float(t));
+          const float2 p = thr_x[(half ^ 1) * kPfRows + r];
+          if (__float_as_int(p.y) == t) tp = fmaxf(tp, p.x);
+          thr = fmaxf(bst[K - 1], pf_below(tp));
+        }
       }
       if (!ok) break;
+      // Row end.  Both halves publish their lists; each computes the row's
+      // k-th score T from both and keeps the candidates >= T of its own
+      // column; half 0 merges the two (ascending index) and writes the row.
+      float *mine = lists + half * (kPfTopkMax * kPfRows) + r;
+      const float *theirs = lists + (half ^ 1) * (kPfTopkMax * kPfRows) + r;
+      if (want_topk) {
 #pragma unroll
-      for (int s = 0; s < 16; ++s) mx = fmaxf(mx, G[s]);
-      float lb = G[0];
+        for (int q = 0; q < K; ++q) mine[q * kPfRows] = bst[q];
+      } else {
+        mine[0] = mx;
+      }
+      if (!pair_sync()) break;
+      float T = neg_inf();
+      int n_gt = 0;
+      if (!want_topk) {
+        mx = fmaxf(mx, theirs[0]);
+      } else {
+        // top K of both lists: elementwise max against the reversed partner
+        // list is a bitonic sequence holding them; sort it descending
+        float c[K];
 #pragma unroll
-      for (int s = 1; s < 16; ++s) lb = fminf(lb, G[s]);
-      lb = fmaxf(lb, floor_lb);
-      // half 1 hands its bound and maximum to half 0, which writes the row;
-      // a NaN score marks the end of a column that is not full
-      if (half == 1) {
-        xchg[r] = make_float2(lb, mx);
-        if (cnt < kPsCap) col[cnt * kPfRows] = make_uint2(0x7fffffffu, 0u);
+        for (int q = 0; q < K; ++q) c[q] = fmaxf(bst[q], theirs[(K - 1 - q) * kPfRows]);
+#pragma unroll
+        for (int j2 = K >> 1; j2 > 0; j2 >>= 1)
+#pragma unroll
+          for (int i = 0; i < K; ++i)
+            if ((i & j2) == 0) {
+              const float x = c[i], y = c[i + j2];
+              c[i] = fmaxf(x, y);
+              c[i + j2] = fminf(x, y);
+            }
+        mx = c[0];
+        T = c[0];
+#pragma unroll
+        for (int q = 0; q < K; ++q)
+          if (q < a.topk) T = c[q];
+#pragma unroll
+        for (int q = 0; q < K; ++q) n_gt += (q < a.topk && c[q] > T) ? 1 : 0;
+        cur = pf_filter(base, cur, T);
+        cnt_x[half * kPfRows + r] = static_cast<int>((cur - base) / kPsSlot);
       }
       if (!pair_sync()) break;
       if (half == 0 && row_ok) {
-        const float2 o = xchg[r];
-        mx = fmaxf(mx, o.y);
         const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
         float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
-        rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
         if (want_topk) {
-          const uint2 *c1 = cand + kPsCap * kPfRows + r;
-          int n1 = 0;
-          while (n1 < kPsCap && c1[n1 * kPfRows].x != 0x7fffffffu) ++n1;
-          pf_emit<KTOP>(col, cnt, c1, n1, fmaxf(lb, o.x), a.topk, a.scale, a.sel_idx + orow * a.topk,
-                        a.sel_score + orow * a.topk);
+          // every score > T, then the lowest-index scores == T up to k
+          int quota = a.topk - n_gt, n_out = 0;
+          const uint32_t end1 = base1 + cnt_x[kPfRows + r] * kPsSlot;
+          int32_t *oi = a.sel_idx + orow * a.topk;
+          float *os = a.sel_score + orow * a.topk;
+          uint32_t p0 = base, p1 = base1;
+          while (p0 < cur || p1 < end1) {
+            const uint2 e0 = p0 < cur ? lds_u2(p0) : make_uint2(0u, 0x7fffffffu);
+            const uint2 e1 = p1 < end1 ? lds_u2(p1) : make_uint2(0u, 0x7fffffffu);
+            const bool take0 = e0.y < e1.y;
+            const uint2 e = take0 ? e0 : e1;
+            p0 += take0 ? kPsSlot : 0u;
+            p1 += take0 ? 0u : kPsSlot;
+            const float x = __uint_as_float(e.x);
+            const bool sel = x > T || (x == T && quota > 0);
+            if (sel) {
+              quota -= x > T ? 0 : 1;
+              oi[n_out] = static_cast<int32_t>(e.y);
+              os[n_out] = x * a.scale;
+              ++n_out;
+            }
+          }
+          for (int q = n_out; q < a.topk; ++q) {
+            oi[q] = -1;
+            os[q] = neg_inf();
+          }
         }
+        rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
       }
       if (!pair_sync()) break;
     }
@@ -421,7 +576,6 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     tc::tmem_dealloc(tmem, 256);
   }
 }
-
 
 // ---------------------------------------------------------------------------
 // Stage 2a, k_prefill_gist_attn: softmax partial of every row over its
