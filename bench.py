@@ -379,6 +379,25 @@ def measure_prefill(G, W, cfg, dev, args, flush, bf16_peak):
             "tensor_frac": round(tf / bf16_peak, 4), "steps": steps}
 
 
+def rank_seed(cfg, rank):
+    """Each rank draws its own batch of the workload (weak scaling: disjoint
+    rows, no data-path exchange)."""
+    return cfg.seed + 1000 * rank
+
+
+def max_over_ranks(values, world, device):
+    """Per-rank timed totals -> the maximum over ranks (the job's time)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_rate(units_per_rank_step, world, steps, total_ms):
+    """Whole-job throughput: the units all ranks processed / the max-over-ranks time."""
+    return units_per_rank_step * world * steps / (total_ms / 1e3)
+
+
 def run_gsa(args, world, rank, local):
     import long_context_gsa_b200 as G
     import long_context_gsa_b200.workloads as W
@@ -399,12 +418,9 @@ def run_gsa(args, world, rank, local):
         torch.cuda.synchronize()
 
     barrier()
-    main = measure_flat(G, W, cfg, dev, args, flush, cfg.seed + 1000 * rank, e2e=True, clock_index=local)
+    main = measure_flat(G, W, cfg, dev, args, flush, rank_seed(cfg, rank), e2e=True, clock_index=local)
     barrier()
-    t = torch.tensor([float(np.sum(main["step_ms"])), float(np.sum(main["e2e_ms"]))], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, total_e2e_ms = float(t[0]), float(t[1])
+    total_ms, total_e2e_ms = max_over_ranks([np.sum(main["step_ms"]), np.sum(main["e2e_ms"])], world, dev)
 
     extra = {}
     if rank == 0 and world == 1 and not args.main_only:
@@ -423,7 +439,7 @@ def run_gsa(args, world, rank, local):
     result = None
     if rank == 0:
         s = flat_summary(cfg, main, hbm)
-        value = cfg.head_queries * world * args.steps / (total_ms / 1e3)
+        value = job_rate(cfg.head_queries, world, args.steps, total_ms)
         k = main["kern_ms"].mean(0)
         names = ["score_gists", "topk_select", "unfold_attend"]
         ab = algorithmic_bytes(cfg, main["x"], main["sel"])
@@ -446,7 +462,7 @@ def run_gsa(args, world, rank, local):
             "roofline": roof,
             "step_hbm": s["step_hbm"],
             "kernels_us": s["kernels_us"],
-            "e2e": {"value": round(cfg.head_queries * world * args.steps / (total_e2e_ms / 1e3), 1), "unit": UNIT,
+            "e2e": {"value": round(job_rate(cfg.head_queries, world, args.steps, total_e2e_ms), 1), "unit": UNIT,
                     "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"]},
             "clocks": main["clocks"],
             "gpu_launches": 3 * args.steps,

@@ -239,16 +239,113 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_mem(const TopkArgs a) {
 
 
 constexpr int kTopkRegThreads = 256;
+constexpr int kTopkCandCap = 1024;  // candidates the bound path ranks in shared memory
 
-// Register-resident top-k.  Warp w holds indices [w*32*KPT, (w+1)*32*KPT);
-// lane l's key j is index w*32*KPT + 32*j + l, so loads are coalesced and
-// index order inside a warp is (j, lane) order.
+struct BoundSmem {
+  unsigned long long cand[kTopkCandCap];
+  uint32_t sel[kTopkCandCap];
+  uint32_t wbound[kTopkRegThreads / 32];
+  int count;
+};
+
+// Rank key of chunk i: the order-preserving score key above, the inverted
+// index below, so a larger value ranks first and equal scores go to the
+// lower index.  Every valid entry's value is distinct and nonzero.
+__device__ __forceinline__ unsigned long long rank_key(uint32_t key, int i) {
+  return (static_cast<unsigned long long>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
+}
+
+// Top-k through a lower bound (0 < kk < n, kk <= 256):
+//  1. every warp finds the r-th largest of its 32 threads' maximum keys,
+//     r = ceil(kk / 8); the smallest of these 8 values, L, is reached by at
+//     least 8 r >= kk distinct entries, so it bounds the row's kk-th score
+//     key from below;
+//  2. every entry with key >= L is a candidate (in practice about 1.8 kk);
+//  3. each candidate's rank among the candidates, by (score desc, index
+//     asc), is counted directly; ranks < kk are the selection, and a
+//     second count over the selected gives each one's output slot in
+//     ascending chunk order.
+// Returns false (nothing written) when the candidates exceed the buffer;
+// the caller then runs the radix select.  Called by the whole block.
+template <int KPT>
+__device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n, int kk, const uint32_t (&key)[KPT],
+                                              int base, BoundSmem &sm) {
+  constexpr int T = kTopkRegThreads, W = T / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t m = 0u;  // valid keys are nonzero; 0 marks "no entry"
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (base + 32 * j < n) m = max(m, key[j]);
+  // descending bitonic sort of the warp's 32 maxima (shuffles only)
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int j = size >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, m, j);
+      const bool keep_max = ((lane & size) == 0) == ((lane & j) == 0);
+      m = keep_max ? max(m, o) : min(m, o);
+    }
+  const int r = (kk + W - 1) / W;
+  if (lane == r - 1) sm.wbound[warp] = m;
+  if (tid == 0) sm.count = 0;
+  __syncthreads();
+  uint32_t L = sm.wbound[0];
+#pragma unroll
+  for (int w = 1; w < W; ++w) L = min(L, sm.wbound[w]);
+  // gather the candidates: one shared atomic per warp
+  const unsigned lt = (1u << lane) - 1u;
+  int w_cnt = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) w_cnt += __popc(__ballot_sync(0xffffffffu, base + 32 * j < n && key[j] >= L));
+  int w_base = 0;
+  if (lane == 0 && w_cnt) w_base = atomicAdd(&sm.count, w_cnt);
+  w_base = __shfl_sync(0xffffffffu, w_base, 0);
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const bool c = base + 32 * j < n && key[j] >= L;
+    const unsigned bal = __ballot_sync(0xffffffffu, c);
+    const int slot = w_base + __popc(bal & lt);
+    if (c && slot < kTopkCandCap) sm.cand[slot] = rank_key(key[j], base + 32 * j);
+    w_base += __popc(bal);
+  }
+  __syncthreads();
+  const int C = sm.count;
+  if (C > kTopkCandCap) return false;  // block-uniform
+  // rank of each candidate among all candidates (keys are distinct)
+  for (int t = tid; t < C; t += T) {
+    const unsigned long long x = sm.cand[t];
+    int rank = 0;
+    for (int u = 0; u < C; ++u) rank += sm.cand[u] > x ? 1 : 0;
+    sm.sel[t] = rank < kk ? static_cast<uint32_t>(x) : 0u;  // inverted index of a selected entry, else 0
+  }
+  __syncthreads();
+  pdl_trigger();
+  int32_t *out_i = a.sel_idx + static_cast<size_t>(row) * a.k;
+  float *out_s = a.sel_score ? a.sel_score + static_cast<size_t>(row) * a.k : nullptr;
+  for (int t = tid; t < C; t += T) {
+    const uint32_t inv = sm.sel[t];
+    if (inv == 0u) continue;
+    int pos = 0;  // selected entries with a lower chunk index (a larger inverted index)
+    for (int u = 0; u < C; ++u) pos += sm.sel[u] > inv ? 1 : 0;
+    const int idx = static_cast<int>(0xFFFFFFFFu - inv);
+    out_i[pos] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
+    if (out_s) out_s[pos] = key_to_float(static_cast<uint32_t>(sm.cand[t] >> 32));
+  }
+  for (int i = kk + tid; i < a.k; i += T) {
+    out_i[i] = -1;
+    if (out_s) out_s[i] = neg_inf();
+  }
+  if (a.counters && tid == 0) a.counters[row] = 0u;
+  return true;
+}
+
 template <int KPT>
 __global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : (KPT <= 32 ? 2 : 1)) k_topk(const TopkArgs a) {
   constexpr int T = kTopkRegThreads, W = T / 32;
   __shared__ uint32_t hist[256];
   __shared__ int info[4];
   __shared__ int wtot[2][W];
+  __shared__ BoundSmem bsm;
 
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
@@ -266,6 +363,7 @@ __global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : (KPT <= 32 ? 
   }
 
   const int kk = min(a.k, n);
+  if (kk > 0 && kk < n && kk <= T && topk_by_bound<KPT>(a, row, n, kk, key, base, bsm)) return;
   uint32_t prefix = 0, pmask = 0;
   int rem = kk;
   bool all_eq = kk == n;

@@ -1,5 +1,7 @@
 """Flat GSA decode on the GPU (score -> select -> unfold) against the float64
 oracle, through the C ABI.  Needs a B200 and the built libgsa.so."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -107,7 +109,7 @@ SMALL = [
 @pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
 def test_small_bf16(name, chg, ragged, own, exclude):
     cfg = W.scaled(W.QWEN_16X, kv_std=1.0, **chg)
-    x = W.decode_inputs(cfg, device="cuda", own_len=own, ragged=ragged, seed=hash(name) % 100000)
+    x = W.decode_inputs(cfg, device="cuda", own_len=own, ragged=ragged, seed=zlib.crc32(name.encode()) % 100000)
     compare(x, cfg, exclude=exclude, what=name)
 
 
