@@ -178,11 +178,48 @@ gsa_status need_ptr(const void *p) { return (p && aligned16(p)) ? GSA_OK : GSA_E
 gsa_status opt_ptr(const void *p) { return (!p || aligned16(p)) ? GSA_OK : GSA_ERR_INVALID_ARG; }
 
 // ---------------------------------------------------------------- scoring
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2D 16-bit view [rows, cols] with 64-column, box_rows-row boxes, 128-byte swizzle.
+bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint64_t cols = 128) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int GH, bool V>
 gsa_status launch_score_mma_t(const ScoreArgs &sa, int splits, int B, void *stream) {
   using Cfg = ScoreMmaCfg<D, GH, V>;
+  ScoreArgs ta = sa;
+  const uint64_t rows = static_cast<uint64_t>(B) * sa.hkv * sa.rows_cap;
+  if (!map_rows(&ta.tm_k, sa.gk, rows, Cfg::kTile, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D) ||
+      (V && !map_rows(&ta.tm_v, sa.gv, rows, Cfg::kTile, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D)))
+    return GSA_ERR_CUDA;
   return launch(k_score_mma<D, GH, V>, dim3(splits, sa.hkv * sa.head_split, B), dim3(Cfg::kThreads), Cfg::kSmemBytes,
-                stream, sa);
+                stream, ta);
 }
 
 template <int D, int GH, bool V>
@@ -419,38 +456,6 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
 }
 
 // ---------------------------------------------------------------- prefill
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
-// 2D 16-bit view [rows, 128] with 64-column, box_rows-row boxes, 128-byte swizzle.
-bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows,
-              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {128, rows};
-  const cuuint64_t strides[1] = {128 * 2};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t es[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;

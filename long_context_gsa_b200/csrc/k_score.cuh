@@ -10,16 +10,21 @@
 //
 // Work decomposition: one CTA per (split of the gist rows, kv head [x head
 // half], batch).  The query heads of one GQA group share every K/V load.
-// Rows are staged global->shared by bulk copies (TMA engine) into a 3-stage
-// mbarrier ring; scores come from mma.sync m16n8k16 (rows = query heads,
-// columns = gists); the value accumulation runs on the CUDA cores in fp32.
+// Rows are staged global->shared by TMA tiled loads (128-byte swizzle) into
+// a 3-stage mbarrier ring.  Each warp owns 16 rows of a stage: the scores
+// come from mma.sync m16n8k16 (rows = query heads, columns = gists), and
+// the same accumulator fragments, exponentiated and split into a bf16 high
+// and low part, are the A operand of the P.V mma (k = the 16 rows), so the
+// value accumulation also runs on the tensor cores with fp32 accumulators.
 #pragma once
 
 #include "common.cuh"
+#include "tc100.cuh"
 
 namespace gsa {
 
 struct ScoreArgs {
+  CUtensorMap tm_k, tm_v;  // bf16 tensor-core path: [B*hkv*rows_cap, D] boxes of 64 columns x kTile rows
   const void *q;          // [B, hq, D]
   const void *gk, *gv;    // [B, hkv, rows_cap, D]
   const int32_t *n_gists; // [B]
@@ -54,15 +59,22 @@ __device__ __forceinline__ void score_slice(int N, int n_split, int split, int &
 
 template <int D, int GH, bool WITH_V>
 struct ScoreMmaCfg {
-  static constexpr int kThreads = 256;
-  static constexpr int kTile = 64;
-  static constexpr int kStages = D == 64 ? 4 : 3;
-  static constexpr uint32_t kTileBytes = kTile * D * 2;
+  static constexpr int kWarps = D == 64 ? 8 : 4;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kTile = 16 * kWarps;         // rows per stage; warp w owns rows 16w .. 16w+15
+  static constexpr int kBoxes = D / 64;             // 64-column (128-byte) TMA boxes per row
+  static constexpr uint32_t kBoxBytes = kTile * 128;
+  static constexpr uint32_t kTileBytes = kBoxes * kBoxBytes;  // K (or V) of one stage
+  static constexpr int kStages = 3;
   static constexpr uint32_t kStageBytes = kTileBytes * (WITH_V ? 2 : 1);
-  // stages | p tiles [2][kTile][GH] | per-warp maxima [8][GH] | reference max [GH] | query fragments
-  // [D/16][32 lanes] x uint2 | flags | barriers
-  static constexpr uint32_t kSmemBytes =
-      kStages * kStageBytes + (2 * kTile * GH + 8 * GH + GH) * 4 + (D / 16) * 32 * 8 + 16 + kStages * 8 + 64;
+  // stages (1024-aligned) | per-warp (max, sum) [2][warps][GH] | query fragments [D/16][32] x uint2 |
+  // stage release counters, abort flag, last tile issued per stage | barriers
+  static constexpr uint32_t kStateOff = kStages * kStageBytes;
+  static constexpr uint32_t kAfOff = kStateOff + 2 * kWarps * GH * 4;
+  static constexpr uint32_t kCntOff = kAfOff + (D / 16) * 32 * 8;
+  static constexpr uint32_t kBarOff = (kCntOff + (2 * kStages + 1) * 4 + 7) & ~7u;
+  static constexpr uint32_t kSmemBytes = kBarOff + kStages * 8 + 1024;  // + alignment slack
+  static_assert(kStages * kStageBytes >= kWarps * GH * D * 4 || !WITH_V, "merge buffer fits in the ring");
 };
 
 // Rescaling threshold (base-2 units): the running max used for the
@@ -83,19 +95,44 @@ __device__ __forceinline__ void fma2(float &ax, float &ay, float p, float vx, fl
       : "f"(vx), "f"(vy), "f"(p));
 }
 
+// ldmatrix .x4 .trans: four 8x8 bf16 matrices, row addresses from lanes
+// 8i .. 8i+7 for matrix i, each thread receiving the transposed fragment.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Two floats -> bf16x2 (lo in the low half), round to nearest.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte offset of the 16-byte chunk `c` (0..7) of row `r` in a 128-byte
+// swizzled TMA box (chunk index XOR row mod 8).
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)); }
+
 // bf16 inputs, D in {64, 128}, up to GH (4 or 8) query heads per CTA.
+// Each warp owns 16 rows of every stage from scores to values, with its
+// own softmax reference per head, so no block-wide barrier is needed per
+// stage: the last warp to finish a stage refills it, and the warps' (max,
+// sum, acc) states are merged once at the end.
 template <int D, int GH, bool WITH_V>
-__global__ void __launch_bounds__(256, 2) k_score_mma(const ScoreArgs a) {
+__global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
+    k_score_mma(const __grid_constant__ ScoreArgs a) {
   using Cfg = ScoreMmaCfg<D, GH, WITH_V>;
-  constexpr int kTile = Cfg::kTile, kStages = Cfg::kStages;
-  constexpr int kLpr = D / 8, kRpw = 32 / kLpr, kSlots = 8 * kRpw;
-  extern __shared__ __align__(128) uint8_t smem[];
-  float *p_tile = reinterpret_cast<float *>(smem + kStages * Cfg::kStageBytes);  // [2][kTile][GH]
-  float *wmax = p_tile + 2 * kTile * GH;                                         // [8][GH]
-  float *m_sh = wmax + 8 * GH;                                                    // [GH] reference max
-  uint2 *af_sh = reinterpret_cast<uint2 *>(m_sh + GH);                            // [D/16][32]
-  int *flags = reinterpret_cast<int *>(af_sh + (D / 16) * 32);                    // [0] abort
-  uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(flags + 4) + 7) & ~uintptr_t(7));
+  constexpr int kTile = Cfg::kTile, kStages = Cfg::kStages, kWarps = Cfg::kWarps;
+  constexpr int kNT = D / 8;  // value n-tiles (8 dims each)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float *st_m = reinterpret_cast<float *>(smem + Cfg::kStateOff);  // [warps][GH]
+  float *st_l = st_m + kWarps * GH;                                // [warps][GH]
+  uint2 *af_sh = reinterpret_cast<uint2 *>(smem + Cfg::kAfOff);   // [D/16][32]
+  int *cnt = reinterpret_cast<int *>(smem + Cfg::kCntOff);         // [kStages] warps done, [kStages] abort
+  int *last_issued = cnt + kStages + 1;                            // [kStages]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.z;
@@ -111,16 +148,16 @@ __global__ void __launch_bounds__(256, 2) k_score_mma(const ScoreArgs a) {
   score_slice(N, a.n_split, split, n0, n1);
   const int nrows = n1 - n0;
   const int ntiles = (nrows + kTile - 1) / kTile;
-  const size_t row_base = (static_cast<size_t>(b) * a.hkv + kvh) * a.rows_cap + n0;
-  const uint8_t *gk = reinterpret_cast<const uint8_t *>(a.gk) + row_base * D * 2;
-  const uint8_t *gv = WITH_V ? reinterpret_cast<const uint8_t *>(a.gv) + row_base * D * 2 : nullptr;
+  const int row0 = (b * a.hkv + kvh) * a.rows_cap + n0;  // first tensor-map row of this slice
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s <= kStages; ++s) cnt[s] = 0;
+    for (int s = 0; s < kStages; ++s) last_issued[s] = -1;
     mbar_fence_init();
-    flags[0] = 0;
+    tc::prefetch_map(&a.tm_k);
+    if (WITH_V) tc::prefetch_map(&a.tm_v);
   }
-  if (tid < GH) m_sh[tid] = neg_inf();
   // Query fragments (same for every warp).  The k dimension is permuted
   // identically in A and B: lane quad t4 reads dims [32*s2 + 8*t4, +8) as
   // two k-steps, so one 16-byte load per row feeds two mma k-steps.
@@ -135,183 +172,191 @@ __global__ void __launch_bounds__(256, 2) k_score_mma(const ScoreArgs a) {
     }
   }
   __syncthreads();
+  uint2 afr[D / 16];
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) afr[i] = af_sh[i * 32 + lane];
 
   auto issue = [&](int t) {
     const int st = t % kStages;
-    const int rows = min(kTile, nrows - t * kTile);
-    const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
     uint8_t *dst = smem + st * Cfg::kStageBytes;
-    mbar_arrive_expect_tx(&bars[st], bytes * (WITH_V ? 2u : 1u));
-    bulk_g2s(dst, gk + static_cast<size_t>(t) * Cfg::kTileBytes, bytes, &bars[st]);
-    if (WITH_V) bulk_g2s(dst + Cfg::kTileBytes, gv + static_cast<size_t>(t) * Cfg::kTileBytes, bytes, &bars[st]);
+    *reinterpret_cast<volatile int *>(&last_issued[st]) = t;
+    mbar_arrive_expect_tx(&bars[st], Cfg::kStageBytes);
+#pragma unroll
+    for (int x = 0; x < Cfg::kBoxes; ++x) {
+      tc::tma_load_2d(dst + x * Cfg::kBoxBytes, &a.tm_k, 64 * x, row0 + t * kTile, &bars[st]);
+      if (WITH_V)
+        tc::tma_load_2d(dst + Cfg::kTileBytes + x * Cfg::kBoxBytes, &a.tm_v, 64 * x, row0 + t * kTile, &bars[st]);
+    }
   };
   if (tid == 0)
     for (int t = 0; t < min(kStages, ntiles); ++t) issue(t);
 
-  float acc[GH][8];
+  float acc[kNT][4];  // P.V accumulators: rows g (head g) and g+8 (unused), dims 8*nt + 2*t4 (+1)
 #pragma unroll
-  for (int j = 0; j < GH; ++j)
+  for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
-  // Reference max (base 2) per head lives in m_sh, identical for every
-  // thread; mg is this lane's copy for its head g.
-  float mg = neg_inf();
-  float l_part = 0.f;  // this lane's share of the sum for head g
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  float mg = neg_inf();  // this warp's reference max (base 2) for head g
+  float lg = 0.f;        // this lane's share of the sum for head g
+  const int rw = 16 * warp;
+  const uint32_t sbase = smem_u32(smem);
+  bool aborted = false;
 
   for (int t = 0; t < ntiles; ++t) {
     const int st = t % kStages;
     const int rows_t = min(kTile, nrows - t * kTile);
-    if (!mbar_wait(&bars[st], (t / kStages) & 1)) flags[0] = 1;
-    const uint8_t *Ks = smem + st * Cfg::kStageBytes;
-    const uint8_t *Vs = Ks + Cfg::kTileBytes;
-    float *pt = p_tile + (t & 1) * kTile * GH;
-
-    // Scores of rows 8*warp .. 8*warp+7 for every head of the group.
-    float s0 = neg_inf(), s1 = neg_inf();
-    const int gi0 = 8 * warp + 2 * t4, gi1 = gi0 + 1;
-    if (8 * warp < rows_t) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint8_t *krow = Ks + (8 * warp + g) * D * 2;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (t / kStages) & 1))) {
+      aborted = true;
+      break;
+    }
+    const uint32_t ks = sbase + st * Cfg::kStageBytes, vs = ks + Cfg::kTileBytes;
+    if (rw < rows_t) {
+      // scores of rows rw .. rw+15 (two n-tiles of 8) for every head
+      float c[2][4];
 #pragma unroll
-      for (int s2 = 0; s2 < D / 32; ++s2) {
-        const uint4 kb = lds_v4(krow + (32 * s2 + 8 * t4) * 2);
-        const uint2 a0 = af_sh[(2 * s2) * 32 + lane], a1 = af_sh[(2 * s2 + 1) * 32 + lane];
-        mma_16816_bf16(c, a0.x, 0u, a0.y, 0u, kb.x, kb.y);
-        mma_16816_bf16(c, a1.x, 0u, a1.y, 0u, kb.z, kb.w);
-      }
-      if (g < nh) {
-        float *srow = a.scores ? a.scores + (static_cast<size_t>(b) * a.hq + h0 + g) * a.score_stride + n0 + t * kTile
-                               : nullptr;
-        if (gi0 < rows_t) {
-          if (srow) srow[gi0] = c[0] * a.scale;
-          s0 = c[0] * a.scale_log2;
-        }
-        if (gi1 < rows_t) {
-          if (srow) srow[gi1] = c[1] * a.scale;
-          s1 = c[1] * a.scale_log2;
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+        const int r = rw + 8 * nt + g;
+#pragma unroll
+        for (int s2 = 0; s2 < D / 32; ++s2) {
+          uint4 kb;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(kb.x), "=r"(kb.y), "=r"(kb.z), "=r"(kb.w)
+                       : "r"(ks + (s2 >> 1) * Cfg::kBoxBytes + sw128(r, (s2 & 1) * 4 + t4)));
+          mma_16816_bf16(c[nt], afr[2 * s2].x, 0u, afr[2 * s2].y, 0u, kb.x, kb.y);
+          mma_16816_bf16(c[nt], afr[2 * s2 + 1].x, 0u, afr[2 * s2 + 1].y, 0u, kb.z, kb.w);
         }
       }
-    }
-    bool need = false;
-    float tl = 0.f;
-    if (WITH_V) {
-      need = s0 > mg + kRescaleSlack || s1 > mg + kRescaleSlack;
-      if (!need && g < GH) {
-        const float p0 = exp2_approx(s0 - mg), p1 = exp2_approx(s1 - mg);
-        pt[gi0 * GH + g] = p0;
-        pt[gi1 * GH + g] = p1;
-        tl = p0 + p1;
-      }
-    }
-    const bool slow = __syncthreads_or(need);
-    if (flags[0]) {
-      if (tid == 0) {
-        flag_error(a.status, GSA_DEVERR_TIMEOUT);
-        for (int u = t; u < min(t + kStages, ntiles); ++u) mbar_wait(&bars[u % kStages], (u / kStages) & 1);
-      }
-      __syncthreads();
-      return;
-    }
-    // Every warp is past the value pass of tile t-1: its stage can refill.
-    if (tid == 0 && t >= 1 && t - 1 + kStages < ntiles) issue(t - 1 + kStages);
-    if (!WITH_V) continue;
-
-    if (slow) {
-      // Raise the reference max to this tile's max, rescale, redo p.
-      float qm = fmaxf(s0, s1);
-      qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
-      qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));
-      if (t4 == 0 && g < GH) wmax[warp * GH + g] = qm;
-      __syncthreads();
-      float m_mine = neg_inf();  // new reference of head `tid` (tid < GH)
+      float s[2][2];
 #pragma unroll
-      for (int j = 0; j < GH; ++j) {
-        float tm = neg_inf();
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int w = 0; w < 8; ++w) tm = fmaxf(tm, wmax[w * GH + j]);
-        const float mo = m_sh[j];
-        const float mn = fmaxf(mo, tm);
-        const float alpha = (mn == neg_inf()) ? 1.f : exp2_approx(mo - mn);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] *= alpha;
-        if (j == g) {
-          l_part *= alpha;
+        for (int e = 0; e < 2; ++e) {
+          const int gi = rw + 8 * nt + 2 * t4 + e;
+          s[nt][e] = neg_inf();
+          if (g < nh && gi < rows_t) {
+            if (a.scores)
+              a.scores[(static_cast<size_t>(b) * a.hq + h0 + g) * a.score_stride + n0 + t * kTile + gi] = c[nt][e] * a.scale;
+            s[nt][e] = c[nt][e] * a.scale_log2;
+          }
+        }
+      if (WITH_V) {
+        // lazy reference: raised only when this warp's rows exceed it by
+        // more than kRescaleSlack; the head's accumulators then rescale
+        float qm = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
+        qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));
+        const bool need = qm > mg + kRescaleSlack;
+        if (__any_sync(0xffffffffu, need)) {
+          const float mn = need ? qm : mg;
+          const float alpha = (mg == neg_inf() || mn == mg) ? 1.f : exp2_approx(mg - mn);
+          lg *= alpha;
           mg = mn;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            acc[nt][0] *= alpha;
+            acc[nt][1] *= alpha;
+          }
         }
-        if (j == tid) m_mine = mn;
+        float p[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) p[nt][e] = s[nt][e] > neg_inf() ? exp2_approx(s[nt][e] - mg) : 0.f;
+        lg += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        // A operand of P.V (k = the warp's 16 rows): bf16 high part and the
+        // bf16 rounding of the remainder, so the weights keep ~16 bits
+        const uint32_t h0p = pack_bf16(p[0][0], p[0][1]), h1p = pack_bf16(p[1][0], p[1][1]);
+        const uint32_t l0p = pack_bf16(p[0][0] - bf16_lo(h0p), p[0][1] - bf16_hi(h0p));
+        const uint32_t l1p = pack_bf16(p[1][0] - bf16_lo(h1p), p[1][1] - bf16_hi(h1p));
+        if (rows_t - rw < 16) {
+          // rows past the slice end enter the product with weight 0; clear
+          // their values so that whatever the buffer holds there (the next
+          // slice, or unwritten memory) cannot turn 0 * v into NaN
+          for (int i = lane; i < (rw + 16 - max(rw, rows_t)) * 8 * Cfg::kBoxes; i += 32) {
+            const int r = max(rw, rows_t) + i / (8 * Cfg::kBoxes), x = (i / 8) % Cfg::kBoxes, ch = i % 8;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs + x * Cfg::kBoxBytes + sw128(r, ch)),
+                         "r"(0u)
+                         : "memory");
+          }
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+        }
+        const int mi = lane >> 3;               // ldmatrix: matrix fed by this lane's address
+        const int vr = rw + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int dp = 0; dp < kNT / 2; ++dp) {
+          const int dim0 = 8 * (2 * dp + (mi >> 1));
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_trans(vs + (dim0 >> 6) * Cfg::kBoxBytes + sw128(vr, (dim0 & 63) >> 3), b0, b1, b2, b3);
+          mma_16816_bf16(acc[2 * dp], h0p, 0u, h1p, 0u, b0, b1);
+          mma_16816_bf16(acc[2 * dp], l0p, 0u, l1p, 0u, b0, b1);
+          mma_16816_bf16(acc[2 * dp + 1], h0p, 0u, h1p, 0u, b2, b3);
+          mma_16816_bf16(acc[2 * dp + 1], l0p, 0u, l1p, 0u, b2, b3);
+        }
       }
-      __syncthreads();  // everyone has read the old reference
-      if (tid < GH) m_sh[tid] = m_mine;
-      if (g < GH) {
-        const float p0 = exp2_approx(s0 - mg), p1 = exp2_approx(s1 - mg);
-        pt[gi0 * GH + g] = p0;
-        pt[gi1 * GH + g] = p1;
-        tl = p0 + p1;
-      }
-      __syncthreads();
     }
-    l_part += tl;
-
-    // Values: slot = (warp, row group); this lane owns dims dd .. dd+7.
-    const int slot = warp * kRpw + lane / kLpr;
-    const int dd = 8 * (lane % kLpr);
-    for (int r = slot; r < rows_t; r += kSlots) {
-      const uint4 vw = lds_v4(Vs + (r * D + dd) * 2);
-      float v[8];
-      Vec16<__nv_bfloat16>::unpack(vw, v);
-      float p[GH];
-#pragma unroll
-      for (int j4 = 0; j4 < GH / 4; ++j4) {
-        const float4 pp = reinterpret_cast<const float4 *>(pt + r * GH)[j4];
-        p[4 * j4] = pp.x;
-        p[4 * j4 + 1] = pp.y;
-        p[4 * j4 + 2] = pp.z;
-        p[4 * j4 + 3] = pp.w;
-      }
-#pragma unroll
-      for (int j = 0; j < GH; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) fma2(acc[j][e], acc[j][e + 1], p[j], v[e], v[e + 1]);
-    }
+    // release the stage; the last of the warps to finish it refills it
+    __syncwarp();
+    if (lane == 0 && atomicAdd(&cnt[st], 1) == (t / kStages + 1) * kWarps - 1 && t + kStages < ntiles)
+      issue(t + kStages);
   }
-
+  if (aborted && lane == 0) atomicExch(&cnt[kStages], 1);
+  __syncthreads();
+  if (cnt[kStages]) {
+    // a wait expired: let every copy that may be in flight land, then leave
+    if (tid == 0) {
+      flag_error(a.status, GSA_DEVERR_TIMEOUT);
+      for (int s = 0; s < kStages; ++s) {
+        const int tl = *reinterpret_cast<volatile int *>(&last_issued[s]);
+        if (tl >= 0) mbar_wait(&bars[s], (tl / kStages) & 1);
+      }
+    }
+    __syncthreads();
+    return;
+  }
   pdl_trigger();
   if (WITH_V && a.part) {
-    __syncthreads();  // all value passes done before the ring is reused
-    // Per-head sums: lanes of quad g across all warps.
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-    if (t4 == 0 && g < GH) wmax[warp * GH + g] = l_part;
-#pragma unroll
-    for (int o = kLpr; o < 32; o <<= 1)
-#pragma unroll
-      for (int j = 0; j < GH; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], o);
-    float *red = reinterpret_cast<float *>(smem);  // [8][GH][D]
-    if (lane < kLpr) {
-#pragma unroll
-      for (int j = 0; j < GH; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; e += 4)
-          *reinterpret_cast<float4 *>(red + (warp * GH + j) * D + 8 * lane + e) =
-              make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
+    // Per-warp states -> shared memory (the ring is free now), then merge.
+    lg += __shfl_xor_sync(0xffffffffu, lg, 1);
+    lg += __shfl_xor_sync(0xffffffffu, lg, 2);
+    if (t4 == 0 && g < GH) {
+      st_m[warp * GH + g] = mg;
+      st_l[warp * GH + g] = lg;
     }
+    float *red = reinterpret_cast<float *>(smem);  // [warps][GH][D]
+    if (g < GH)
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+        *reinterpret_cast<float2 *>(red + (warp * GH + g) * D + 8 * nt + 2 * t4) = make_float2(acc[nt][0], acc[nt][1]);
     __syncthreads();
     for (int i = tid; i < nh * D; i += Cfg::kThreads) {
       const int j = i / D, dim = i % D;
-      float s = 0.f;
+      float M = neg_inf();
 #pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[(w * GH + j) * D + dim];
-      a.part[((static_cast<size_t>(b) * a.hq + h0 + j) * a.n_split + split) * (D + kPartHeader) + kPartHeader + dim] = s;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, st_m[w * GH + j]);
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = st_m[w * GH + j];
+        if (mw > neg_inf()) sum += red[(w * GH + j) * D + dim] * exp2_approx(mw - M);
+      }
+      a.part[((static_cast<size_t>(b) * a.hq + h0 + j) * a.n_split + split) * (D + kPartHeader) + kPartHeader + dim] =
+          sum;
     }
     if (tid < nh) {
+      float M = neg_inf();
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, st_m[w * GH + tid]);
       float l = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) l += wmax[w * GH + tid];
-      const float mt = m_sh[tid];
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = st_m[w * GH + tid];
+        if (mw > neg_inf()) l += st_l[w * GH + tid] * exp2_approx(mw - M);
+      }
       float *hdr = a.part + ((static_cast<size_t>(b) * a.hq + h0 + tid) * a.n_split + split) * (D + kPartHeader);
-      hdr[0] = mt;
+      hdr[0] = M;
       hdr[1] = l;
       hdr[2] = 0.f;
       hdr[3] = 0.f;
