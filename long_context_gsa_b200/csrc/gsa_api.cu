@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/gsa.h"
 #include "common.cuh"
@@ -344,6 +345,17 @@ size_t unfold_smem(int chunk) {
 
 template <int D, typename T>
 gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
+  if (std::is_same<T, __nv_bfloat16>::value) {
+    // tensor-core kernel: raw K/V as 2D maps with 8-row boxes
+    const size_t smem = UnfoldTcCfg<D>::kSmemBytes;
+    const int slots = resident_ctas(k_unfold_tc<D>, kUnfoldThreads, smem);
+    ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));
+    const uint64_t rows = static_cast<uint64_t>(B) * ua.hkv * ua.t_max;
+    if (!map_rows(&ua.tm_k, ua.raw_k, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D) ||
+        !map_rows(&ua.tm_v, ua.raw_v, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D))
+      return GSA_ERR_CUDA;
+    return launch(k_unfold_tc<D>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads), smem, stream, ua);
+  }
   const size_t smem = unfold_smem<D, T>(ua.chunk);
   const int slots = resident_ctas(k_unfold<D, T>, kUnfoldThreads, smem);
   ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));

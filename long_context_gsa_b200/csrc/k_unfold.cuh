@@ -20,10 +20,13 @@
 #pragma once
 
 #include "common.cuh"
+#include "k_score.cuh"  // mma.sync, ldmatrix and swizzle helpers
+#include "tc100.cuh"
 
 namespace gsa {
 
 struct UnfoldArgs {
+  CUtensorMap tm_k, tm_v;    // bf16 tensor-core path: raw K/V as [B*hkv*t_max, D], boxes of 64 columns x 8 rows
   const void *q;             // [B, hq, D]
   const void *raw_k, *raw_v; // [B, hkv, t_max, D]
   const void *gist_v;        // [B, hkv, n_max, D] (exclude mode)
@@ -97,6 +100,59 @@ __host__ __device__ __forceinline__ int unfold_warp_stages(int stage_bytes) {
 }
 
 constexpr int kUnfoldWarps = kUnfoldThreads / 32;
+
+// The CTA's partial (the warps' states in red) goes to the row's split slot;
+// the CTA that arrives last at the row's counter merges all splits with the
+// prior partials and writes the output row.  Called by the whole block.
+template <int NW, int D>
+__device__ void unfold_finish(const UnfoldArgs &a, size_t row, int split, const float (*red)[2 + D], int &is_last_s) {
+  const int tid = threadIdx.x;
+  constexpr int kUnfoldWarps = NW;
+  __syncthreads();
+  float *rec = a.part + (row * a.n_split + split) * (D + kPartHeader);
+  {
+    float M = neg_inf();
+#pragma unroll
+    for (int w = 0; w < kUnfoldWarps; ++w) M = fmaxf(M, red[w][0]);
+    for (int dim = tid; dim < D; dim += kUnfoldThreads) {
+      float s = 0.f;
+      if (M != neg_inf())
+#pragma unroll
+        for (int w = 0; w < kUnfoldWarps; ++w) s += red[w][2 + dim] * exp2_approx(red[w][0] - M);
+      rec[kPartHeader + dim] = s;
+    }
+    if (tid == 0) {
+      float L = 0.f;
+      if (M != neg_inf())
+#pragma unroll
+        for (int w = 0; w < kUnfoldWarps; ++w) L += red[w][1] * exp2_approx(red[w][0] - M);
+      rec[0] = M;
+      rec[1] = L;
+      rec[2] = 0.f;
+      rec[3] = 0.f;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int last = 1;
+    if (a.n_split > 1) {
+      __threadfence();
+      const uint32_t prev = atomicAdd(&a.counters[row], 1u);
+      last = prev == static_cast<uint32_t>(a.n_split - 1);
+      if (last) {
+        __threadfence();
+        a.counters[row] = 0u;
+      }
+    }
+    is_last_s = last;
+  }
+  __syncthreads();
+  if (!is_last_s) return;
+  const float *recs[2] = {a.part + row * a.n_split * (D + kPartHeader),
+                          a.prior ? a.prior + row * a.n_prior * (D + kPartHeader) : nullptr};
+  const int counts[2] = {a.n_split, a.prior ? a.n_prior : 0};
+  combine_records<D>(recs, counts, 2, a.out, row, a.out_bf16, a.lse);
+}
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kUnfoldThreads) k_unfold(const UnfoldArgs a) {
@@ -279,50 +335,271 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold(const UnfoldArgs a) {
       red[warp][1] = l;
     }
   }
-  __syncthreads();
-  float *rec = a.part + (row * a.n_split + split) * (D + kPartHeader);
-  {
-    float M = neg_inf();
-#pragma unroll
-    for (int w = 0; w < kUnfoldWarps; ++w) M = fmaxf(M, red[w][0]);
-    for (int dim = tid; dim < D; dim += kUnfoldThreads) {
-      float s = 0.f;
-      if (M != neg_inf())
-#pragma unroll
-        for (int w = 0; w < kUnfoldWarps; ++w) s += red[w][2 + dim] * exp2_approx(red[w][0] - M);
-      rec[kPartHeader + dim] = s;
+  unfold_finish<kUnfoldWarps, D>(a, row, split, red, is_last_s);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 inputs, D in {64, 128}: the same split and combine, with the rows on
+// the tensor cores.  The attended raw rows are cut into half-steps of 8 rows
+// (one TMA box of 8 rows x 64 columns per 64 dims, 128-byte swizzle; a chunk
+// of c rows gives ceil(c/8) half-steps, the own chunk ceil(own/8)); warp w
+// takes steps w, w+4, ... of two half-steps (16 rows) through its own ring.
+// Per step: s = q.K^T with mma.sync (the query is row 0 of the A operand), a
+// lazy online softmax on lanes 0..3 (the lanes holding row 0), and P.V as
+// mma.sync with P split into bf16 high and low parts and V read by
+// ldmatrix.trans.  Rows past a half-step's valid count get weight 0 and
+// their values are cleared in shared memory first.
+template <int D>
+struct UnfoldTcCfg {
+  static constexpr int kBoxes = D / 64;
+  static constexpr uint32_t kHalf = kBoxes * 1024;        // K (or V) of one 8-row half-step
+  static constexpr uint32_t kStage = 4 * kHalf;           // K and V of two half-steps
+  static constexpr int kStages = 2;  // two steps in flight per warp; more stages cost residency
+  static constexpr uint32_t kSmemBytes = kUnfoldWarps * kStages * kStage + 1024;  // + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_constant__ UnfoldArgs a) {
+  using Cfg = UnfoldTcCfg<D>;
+  constexpr int kNT = D / 8, S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ int items[kUnfoldMaxItems];
+  __shared__ int item_pos[kUnfoldMaxItems];
+  __shared__ int n_items_s;
+  __shared__ int is_last_s;
+  __shared__ float red[kUnfoldWarps][2 + D];
+  __shared__ uint64_t bars[kUnfoldWarps][4];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / a.group;
+  const size_t row = static_cast<size_t>(b) * a.hq + h;
+  const int g = lane >> 2, t4 = lane & 3;
+
+  pdl_wait();
+  const int N = min(min(max(a.n_gists[b], 0), a.n_max), a.t_max / a.chunk);
+  int own = min(max(a.own_len[b], 0), a.chunk);
+  if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
+
+  // Selected chunks of this split, in list order (invalid entries dropped).
+  const int per = (a.k + a.n_split - 1) / a.n_split;
+  const int i0 = min(a.k, split * per), i1 = min(a.k, i0 + per);
+  if (warp == 0) {
+    int cnt = 0;
+    for (int base = i0; base < i1; base += 32) {
+      const int i = base + lane;
+      int m = -1;
+      if (i < i1) {
+        m = a.sel_idx[row * a.k + i];
+        if (m >= N) {
+          flag_error(a.status, GSA_DEVERR_BAD_INDEX);
+          m = -1;
+        }
+      }
+      const unsigned ball = __ballot_sync(0xffffffffu, m >= 0);
+      if (m >= 0) {
+        const int slot = cnt + __popc(ball & ((1u << lane) - 1u));
+        items[slot] = m;
+        item_pos[slot] = i;
+      }
+      cnt += __popc(ball);
     }
-    if (tid == 0) {
-      float L = 0.f;
-      if (M != neg_inf())
-#pragma unroll
-        for (int w = 0; w < kUnfoldWarps; ++w) L += red[w][1] * exp2_approx(red[w][0] - M);
-      rec[0] = M;
-      rec[1] = L;
-      rec[2] = 0.f;
-      rec[3] = 0.f;
+    if (lane == 0) n_items_s = cnt;
+    if (lane < kUnfoldWarps)
+      for (int s = 0; s < S; ++s) mbar_init(&bars[lane][s], 1);
+    if (lane == 0) {
+      mbar_fence_init();
+      tc::prefetch_map(&a.tm_k);
+      tc::prefetch_map(&a.tm_v);
     }
   }
   __syncthreads();
-  if (tid == 0) {
-    int last = 1;
-    if (a.n_split > 1) {
-      __threadfence();
-      const uint32_t prev = atomicAdd(&a.counters[row], 1u);
-      last = prev == static_cast<uint32_t>(a.n_split - 1);
-      if (last) {
-        __threadfence();
-        a.counters[row] = 0u;
+
+  // half-step j -> (first raw row, valid rows, chunk item or -1 for own rows)
+  const int hpc = (a.chunk + 7) >> 3;  // half-steps per chunk
+  const int n_sel = n_items_s;
+  const int own_half = (split == a.n_split - 1 && own > 0) ? (own + 7) >> 3 : 0;
+  const int n_half = n_sel * hpc + own_half;
+  const int n_steps = (n_half + 1) >> 1;
+  const int n_mine = n_steps > warp ? (n_steps - warp + kUnfoldWarps - 1) / kUnfoldWarps : 0;
+  auto half = [&](int j, int &first, int &valid, int &item) {
+    if (j >= n_half) {
+      first = 0;
+      valid = 0;
+      item = -1;
+    } else if (j < n_sel * hpc) {
+      const int it = j / hpc, sub = j % hpc;
+      first = items[it] * a.chunk + 8 * sub;
+      valid = min(8, a.chunk - 8 * sub);
+      item = sub == 0 ? it : -1;  // the chunk's gist joins with its first half-step
+    } else {
+      const int q = j - n_sel * hpc;
+      first = N * a.chunk + 8 * q;
+      valid = min(8, own - 8 * q);
+      item = -1;
+    }
+  };
+  const int kv_row0 = (b * a.hkv + kvh) * a.t_max;  // tensor-map row of this kv head's first raw row
+  uint8_t *ring = smem + static_cast<size_t>(warp) * S * Cfg::kStage;
+  auto issue = [&](int li) {
+    const int step = warp + kUnfoldWarps * li, st = li % S;
+    uint8_t *dst = ring + st * Cfg::kStage;
+    mbar_arrive_expect_tx(&bars[warp][st], Cfg::kStage);
+#pragma unroll
+    for (int hs = 0; hs < 2; ++hs) {
+      int first, valid, item;
+      half(2 * step + hs, first, valid, item);
+#pragma unroll
+      for (int x = 0; x < Cfg::kBoxes; ++x) {
+        tc::tma_load_2d(dst + (hs * Cfg::kBoxes + x) * 1024, &a.tm_k, 64 * x, kv_row0 + first, &bars[warp][st]);
+        tc::tma_load_2d(dst + 2 * Cfg::kHalf + (hs * Cfg::kBoxes + x) * 1024, &a.tm_v, 64 * x, kv_row0 + first,
+                        &bars[warp][st]);
       }
     }
-    is_last_s = last;
+  };
+  if (lane == 0)
+    for (int li = 0; li < min(S, n_mine); ++li) issue(li);
+
+  // the query as row 0 of the A operand (k permuted as in the scoring pass)
+  uint2 afr[D / 16];
+  {
+    const uint4 *qrow = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) + row * D);
+#pragma unroll
+    for (int s2 = 0; s2 < D / 32; ++s2) {
+      const uint4 w = g == 0 ? qrow[4 * s2 + t4] : make_uint4(0, 0, 0, 0);
+      afr[2 * s2] = make_uint2(w.x, w.y);
+      afr[2 * s2 + 1] = make_uint2(w.z, w.w);
+    }
   }
-  __syncthreads();
-  if (!is_last_s) return;
-  const float *recs[2] = {a.part + row * a.n_split * (D + kPartHeader),
-                          a.prior ? a.prior + row * a.n_prior * (D + kPartHeader) : nullptr};
-  const int counts[2] = {a.n_split, a.prior ? a.n_prior : 0};
-  combine_records<D>(recs, counts, 2, a.out, row, a.out_bf16, a.lse);
+  float acc[kNT][4];  // row 0 (lanes 0..3): dims 8*nt + 2*t4 (+1); other rows unused
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  float mg = neg_inf(), lg = 0.f;  // reference max (base 2, same in every lane) and this lane's sum
+  const uint32_t ring_u = smem_u32(ring);
+  const __nv_bfloat16 *gv_base =
+      reinterpret_cast<const __nv_bfloat16 *>(a.gist_v) + (static_cast<size_t>(b) * a.hkv + kvh) * a.n_max * D;
+  int stuck = -1;
+  for (int li = 0; li < n_mine; ++li) {
+    const int st = li % S, step = warp + kUnfoldWarps * li;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[warp][st], (li / S) & 1))) {
+      stuck = li;
+      break;
+    }
+    const uint32_t kst = ring_u + st * Cfg::kStage, vst = kst + 2 * Cfg::kHalf;
+    int valid[2], item[2], first;
+    half(2 * step, first, valid[0], item[0]);
+    half(2 * step + 1, first, valid[1], item[1]);
+    if (valid[0] < 8 || valid[1] < 8) {
+      // clear the values of rows past the valid ones (they get weight 0)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs)
+        for (int i = lane; i < (8 - valid[hs]) * Cfg::kBoxes * 8; i += 32) {
+          const int r = valid[hs] + i / (8 * Cfg::kBoxes), x = (i / 8) % Cfg::kBoxes, ch = i % 8;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vst + (hs * Cfg::kBoxes + x) * 1024 +
+                                                                        sw128(r, ch)),
+                       "r"(0u)
+                       : "memory");
+        }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+    }
+    float s[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s2 = 0; s2 < D / 32; ++s2) {
+        uint4 kb;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(kb.x), "=r"(kb.y), "=r"(kb.z), "=r"(kb.w)
+                     : "r"(kst + (nt * Cfg::kBoxes + (s2 >> 1)) * 1024 + sw128(g, (s2 & 1) * 4 + t4)));
+        mma_16816_bf16(c, afr[2 * s2].x, 0u, afr[2 * s2].y, 0u, kb.x, kb.y);
+        mma_16816_bf16(c, afr[2 * s2 + 1].x, 0u, afr[2 * s2 + 1].y, 0u, kb.z, kb.w);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) s[nt][e] = (g == 0 && 2 * t4 + e < valid[nt]) ? c[e] * a.scale_log2 : neg_inf();
+    }
+    // exclude mode: a selected chunk's gist token joins with its first half-step
+    float z[2] = {neg_inf(), neg_inf()};
+    if (a.exclude)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs)
+        if (item[hs] >= 0) z[hs] = a.sel_score[row * a.k + item_pos[item[hs]]] * kLog2e;
+    float qm = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+    qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
+    qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));
+    qm = fmaxf(__shfl_sync(0xffffffffu, qm, 0), fmaxf(z[0], z[1]));
+    if (qm > mg + kRescaleSlack) {  // warp-uniform: raise the reference, rescale
+      const float alpha = mg == neg_inf() ? 1.f : exp2_approx(mg - qm);
+      lg *= alpha;
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        acc[nt][0] *= alpha;
+        acc[nt][1] *= alpha;
+      }
+      mg = qm;
+    }
+    float p[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) p[nt][e] = s[nt][e] > neg_inf() ? exp2_approx(s[nt][e] - mg) : 0.f;
+    lg += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+    const uint32_t h0p = pack_bf16(p[0][0], p[0][1]), h1p = pack_bf16(p[1][0], p[1][1]);
+    const uint32_t l0p = pack_bf16(p[0][0] - bf16_lo(h0p), p[0][1] - bf16_hi(h0p));
+    const uint32_t l1p = pack_bf16(p[1][0] - bf16_lo(h1p), p[1][1] - bf16_hi(h1p));
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int dp = 0; dp < kNT / 2; ++dp) {
+      const int dim0 = 8 * (2 * dp + (mi >> 1));
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(vst + ((mi & 1) * Cfg::kBoxes + (dim0 >> 6)) * 1024 + sw128(lane & 7, (dim0 & 63) >> 3), b0, b1,
+                    b2, b3);
+      mma_16816_bf16(acc[2 * dp], h0p, 0u, h1p, 0u, b0, b1);
+      mma_16816_bf16(acc[2 * dp], l0p, 0u, l1p, 0u, b0, b1);
+      mma_16816_bf16(acc[2 * dp + 1], h0p, 0u, h1p, 0u, b2, b3);
+      mma_16816_bf16(acc[2 * dp + 1], l0p, 0u, l1p, 0u, b2, b3);
+    }
+    if (a.exclude)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs)
+        if (item[hs] >= 0 && g == 0) {
+          const float pz = exp2_approx(z[hs] - mg);
+          if (t4 == 0) lg += pz;
+          const __nv_bfloat16 *gv = gv_base + static_cast<size_t>(items[item[hs]]) * D + 2 * t4;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(gv + 8 * nt);
+            acc[nt][0] = fmaf(pz, bf16_lo(w), acc[nt][0]);
+            acc[nt][1] = fmaf(pz, bf16_hi(w), acc[nt][1]);
+          }
+        }
+    __syncwarp();
+    if (lane == 0 && li + S < n_mine) issue(li + S);
+  }
+  if (stuck >= 0 && lane == 0) {
+    // Let the copies already issued land before the CTA can exit.
+    flag_error(a.status, GSA_DEVERR_TIMEOUT);
+    for (int li = stuck; li < min(stuck + S, n_mine); ++li) mbar_wait(&bars[warp][li % S], (li / S) & 1);
+  }
+  pdl_trigger();
+  lg += __shfl_xor_sync(0xffffffffu, lg, 1);
+  lg += __shfl_xor_sync(0xffffffffu, lg, 2);
+  if (lane < 4) {
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      red[warp][2 + 8 * nt + 2 * t4] = acc[nt][0];
+      red[warp][2 + 8 * nt + 2 * t4 + 1] = acc[nt][1];
+    }
+    if (lane == 0) {
+      red[warp][0] = mg;
+      red[warp][1] = lg;
+    }
+  }
+  unfold_finish<kUnfoldWarps, D>(a, row, split, red, is_last_s);
 }
 
 }  // namespace gsa
