@@ -38,7 +38,7 @@ inline float resolve_scale(const gsa_desc *d) {
 struct Layout {
   size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
-  size_t pf_stats = 0, pf_gist = 0, pf_vh = 0;
+  size_t pf_stats = 0, pf_gist = 0, pf_vh = 0, pf_ovf = 0;
   size_t total = 0;
 };
 
@@ -88,6 +88,7 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     take(L.pf_stats, prow * rec);
     take(L.pf_gist, rows * static_cast<size_t>(d->n_max) * rec);
     take(L.pf_vh, static_cast<size_t>(d->batch) * d->hkv * d->n_max * d->d * 2);
+    take(L.pf_ovf, prow * 4);
     L.total = off;
     return L;
   }
@@ -468,6 +469,10 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
 }
 
 // ---------------------------------------------------------------- prefill
+// Words of the 256-byte status block used by the prefill overflow list
+// (word 0 is the device status; all are zeroed by gsa_workspace_init).
+constexpr int kPfOvfCountWord = 16, kPfOvfDoneWord = 17;
+
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
@@ -498,6 +503,8 @@ PrefillArgs prefill_args(const gsa_desc *d, int32_t *sel_idx, float *sel_score, 
   pa.gist_tiles = cdiv(d->n_max, kPfRows);
   pa.raw_tiles = cdiv(d->t_max, kPfRows);
   pa.status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  pa.ovf_rows = reinterpret_cast<int32_t *>(at(ws, L.pf_ovf));
+  pa.ovf_count = pa.status + kPfOvfCountWord;
   return pa;
 }
 
@@ -510,8 +517,26 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
     return GSA_ERR_CUDA;
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
   const int grid = std::min(total, sm_count());
-  auto kern = d->topk <= 4 ? k_prefill_score<4> : d->topk <= 8 ? k_prefill_score<8> : k_prefill_score<16>;
-  return launch(kern, dim3(grid), dim3(kPsThreads), PfSmem::kBytes, stream, pa);
+  GSA_TRY(launch(k_prefill_score<kPfTopkMax>, dim3(grid), dim3(kPsThreads), PfSmem::kBytes, stream, pa));
+  if (d->topk <= 0) return GSA_OK;
+  // rows whose candidates overflowed: exact per-row selection (usually none)
+  SelectRowsArgs sr;
+  sr.q_raw = static_cast<const __nv_bfloat16 *>(q_raw);
+  sr.k_gist = static_cast<const __nv_bfloat16 *>(k_gist);
+  sr.rows = pa.ovf_rows;
+  sr.count = pa.ovf_count;
+  sr.done = pa.status + kPfOvfDoneWord;
+  sr.group = pa.group;
+  sr.chunk = d->chunk;
+  sr.n_chunks = d->n_max;
+  sr.L = d->t_max;
+  sr.topk = d->topk;
+  sr.scale = pa.scale;
+  sr.sel_idx = sel_idx;
+  sr.sel_score = sel_score;
+  const int nw = clampi(static_cast<int>((160u << 10) / (static_cast<size_t>(d->n_max) * 4)), 1, 8);
+  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(32 * nw), static_cast<size_t>(nw) * d->n_max * 4, stream,
+                sr);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,

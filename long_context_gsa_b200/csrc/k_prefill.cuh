@@ -14,16 +14,12 @@
 // tiles, then raw tiles, heaviest first).  Warp 0 issues TMA loads (Q tile,
 // then 128-gist key tiles into a 2-stage ring), warp 1 issues tcgen05.mma
 // into two 128-column TMEM accumulators, and warps 2..9 (two per TMEM lane
-// quadrant, so two threads per query row, each owning half of the key
-// columns) read the scores with tcgen05.ld, apply the block-causal mask and
-// keep the row maximum.  For raw rows the top-k runs against a lower bound
-// on the row's final k-th score: each half keeps the K largest scores it
-// has appended (sorted, values only) and the partner half's K-th is read
-// once per key tile; only scores above the bound are appended as (score,
-// index) candidates to a per-row column in shared memory (column-major, so
-// appends of different rows never share a bank).  At the end of the row one
-// thread merges both halves' lists into the k-th score and walks both
-// columns in ascending index order.
+// quadrant, so two threads per query row, each owning a 64-column half of
+// every key tile) read the scores with tcgen05.ld and apply the
+// block-causal mask.  Raw rows take the key tiles twice: a first pass of
+// slot maxima gives the row maximum and a lower bound on its k-th score,
+// a second pass appends the few scores above the bound to shared-memory
+// candidate columns, from which the exact selection is read off.
 // Outputs: sel_idx/sel_score (ascending chunk order) and the row maximum
 // that the attention stage uses as softmax reference.
 #pragma once
@@ -46,14 +42,14 @@ struct PrefillArgs {
   int32_t gist_tiles;    // query tiles per head over the gist rows
   int32_t raw_tiles;     // query tiles per head over the raw rows
   uint32_t *status;
+  int32_t *ovf_rows;     // rows whose candidates overflowed (exact pass in k_prefill_select_rows)
+  uint32_t *ovf_count;
 };
 
 constexpr int kPfRows = 128;        // query rows per tile (TMEM lanes)
 constexpr int kPfKeys = 128;        // gist keys per MMA tile (TMEM columns)
 constexpr int kPfThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kPfTopkMax = 16;
-constexpr int kPsThreads = 320;     // scoring: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (2 per row)
-constexpr int kPsCap = 38;          // candidate slots per row half (shared memory)
 
 struct PfTile {
   int is_gist, bh, row0, n_kt;
@@ -82,6 +78,13 @@ __device__ __forceinline__ PfTile pf_tile(const PrefillArgs &a, int t) {
   return r;
 }
 
+// Scoring-stage layout: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue; warp
+// w reads TMEM lane quadrant w % 4 and owns the 64-column half
+// (w - 2) / 4 of every key tile, so two threads share a query row.
+constexpr int kPsEpiWarps = 8;
+constexpr int kPsThreads = 64 + 32 * kPsEpiWarps;
+constexpr int kPsCap = 48;  // candidate slots per row half
+
 struct PfSmem {
   static constexpr uint32_t kQBlock = kPfRows * 128;         // 128 rows x 64 bf16
   static constexpr uint32_t kQBytes = 2 * kQBlock;           // d = 128
@@ -90,19 +93,17 @@ struct PfSmem {
   static constexpr uint32_t kQOff = 0;                       // 2 Q buffers
   static constexpr uint32_t kKOff = 2 * kQBytes;             // kKStages K stages
   static constexpr int kKStages = 2;
-  static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;           // [2 halves][kPsCap][128] (score, index)
-  static constexpr uint32_t kListOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [2][kPfTopkMax][128] best values
-  static constexpr uint32_t kThrOff = kListOff + 2 * kPfTopkMax * kPfRows * 4;  // [2][128] (threshold, tile tag)
-  static constexpr uint32_t kCntOff = kThrOff + 2 * kPfRows * 8;             // [2][128] filtered candidate counts
-  static constexpr uint32_t kBarOff = kCntOff + 2 * kPfRows * 4;
+  // [2 halves][kPsCap][128 rows] (score, index); pass A first uses a row
+  // half's first 8 slots for its 16 sorted slot maxima
+  static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;
+  static constexpr uint32_t kCntOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [2][128] candidate counts (bytes)
+  static constexpr uint32_t kBarOff = kCntOff + 2 * kPfRows;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
 };
 static_assert(PfSmem::kBytes <= 232448, "prefill scoring shared memory");
+static_assert(kPsCap >= 8, "a column holds the 16 slot maxima");
 
 constexpr uint32_t kPsSlot = kPfRows * 8;  // bytes between consecutive slots of one row's column
-
-// (score, index) ranking: higher score first, then lower index.
-__device__ __forceinline__ bool pf_before(float x, int xi, float y, int yi) { return x > y || (x == y && xi < yi); }
 
 __device__ __forceinline__ uint2 lds_u2(uint32_t a) {
   uint2 v;
@@ -114,50 +115,31 @@ __device__ __forceinline__ void sts_u2(uint32_t a, uint2 v) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
 
-// Append (v, idx) at the column cursor `cur` when v > thr (GE: v >= thr),
-// without a branch: the store and the cursor step are predicated.  NaN
-// (a masked score) fails both compares.
-template <bool GE>
-__device__ __forceinline__ void pf_append(uint32_t &cur, float v, float thr, uint32_t idx) {
-  if (GE)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ge.f32 p, %1, %2;\n\t"
-        "@p st.shared.v2.u32 [%0], {%3, %4};\n\t"
-        "@p add.u32 %0, %0, %5;\n\t}\n"
-        : "+r"(cur)
-        : "f"(v), "f"(thr), "r"(__float_as_uint(v)), "r"(idx), "n"(kPsSlot)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.gt.f32 p, %1, %2;\n\t"
-        "@p st.shared.v2.u32 [%0], {%3, %4};\n\t"
-        "@p add.u32 %0, %0, %5;\n\t}\n"
-        : "+r"(cur)
-        : "f"(v), "f"(thr), "r"(__float_as_uint(v)), "r"(idx), "n"(kPsSlot)
-        : "memory");
+// Append (v, idx) to a row quarter's column when v >= bound: the store and
+// the count are predicated (no branch); past kPsCap the last slot is
+// overwritten and only the count grows, which the row end reports as an
+// overflow.  NaN (a masked score) fails the compare.
+__device__ __forceinline__ void ps_append(uint32_t base, uint32_t &cnt, float v, float bound, uint32_t idx) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .u32 s, ad;\n\t"
+      "setp.ge.f32 p, %1, %2;\n\t"
+      "min.u32 s, %0, %5;\n\t"
+      "mad.lo.u32 ad, s, %6, %3;\n\t"
+      "@p st.shared.v2.u32 [ad], {%4, %7};\n\t"
+      "@p add.u32 %0, %0, 1;\n\t}\n"
+      : "+r"(cnt)
+      : "f"(v), "f"(bound), "r"(base), "r"(__float_as_uint(v)), "r"(kPsCap - 1), "r"(kPsSlot), "r"(idx)
+      : "memory");
 }
 
-// Values-only insertion into a descending list (the running top K).
-template <int K>
-__device__ __forceinline__ void pf_insert(float (&b)[K], float x) {
+// Descending bitonic sort of 16 values in registers (no NaN inputs).
+__device__ __forceinline__ void ps_sort16(float (&w)[16]) {
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
-    const float hi = fmaxf(b[q], x);
-    x = fminf(b[q], x);
-    b[q] = hi;
-  }
-}
-
-// Descending bitonic sort of 32 values in registers (no NaN inputs).
-__device__ __forceinline__ void pf_sort32(float (&w)[32]) {
-#pragma unroll
-  for (int k = 2; k <= 32; k <<= 1)
+  for (int k = 2; k <= 16; k <<= 1)
 #pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1)
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const int l = i ^ j;
         if (l > i) {
           const float x = w[i], y = w[l];
@@ -168,128 +150,80 @@ __device__ __forceinline__ void pf_sort32(float (&w)[32]) {
       }
 }
 
-// Store v at a when p (predicated, no branch).
-__device__ __forceinline__ void sts_u2_if(bool p, uint32_t a, uint2 v) {
-  asm volatile(
-      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.shared.v2.u32 [%1], {%2, %3};\n\t}\n" ::"r"(
-          static_cast<uint32_t>(p)),
-      "r"(a), "r"(v.x), "r"(v.y)
-      : "memory");
+// Values-only insertion into a descending list of 16.
+__device__ __forceinline__ void ps_insert16(float (&b)[16], float x) {
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float hi = fmaxf(b[q], x);
+    x = fminf(b[q], x);
+    b[q] = hi;
+  }
 }
 
-// Keep the column's candidates with score >= lb (order kept).  Called by
-// the whole warp (one column per lane): the loop runs to the longest
-// column, four slots per step with the loads issued together; a lane's
-// slots past its cursor are read but neither kept nor counted (every
-// address read lies inside the column's kPsCap slots).  Returns the cursor.
-__device__ __forceinline__ uint32_t pf_filter(uint32_t base, uint32_t cur, float lb) {
-  const int n = static_cast<int>((cur - base) / kPsSlot);
-  const int nmax = __reduce_max_sync(0xffffffffu, n);
-  uint32_t w = base;
-  for (int s = 0; s < nmax; s += 4) {
-    uint2 e[4];
+// a <- the 16 largest of a (sorted descending) and b (sorted descending):
+// the elementwise max against b reversed is bitonic; half-cleaners sort it.
+__device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16]) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) e[u] = lds_u2(base + min(s + u, kPsCap - 1) * kPsSlot);
+  for (int i = 0; i < 16; ++i) a[i] = fmaxf(a[i], b[15 - i]);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool live = s + u < n;
-      sts_u2_if(live, w, e[u]);  // w <= s + u: never overwrites an unread slot
-      w += (live && __uint_as_float(e[u].x) >= lb) ? kPsSlot : 0u;
-    }
-  }
-  return w;
-}
-
-// Rare path (many exactly equal scores): keep the column's best K
-// candidates by (score desc, index asc), left in ascending index order;
-// returns the new cursor.
-template <int K>
-__device__ __noinline__ uint32_t pf_reduce(uint32_t base, uint32_t cur) {
-  float best[K];
-  int bidx[K];
+  for (int j = 8; j > 0; j >>= 1)
 #pragma unroll
-  for (int e = 0; e < K; ++e) {
-    best[e] = neg_inf();
-    bidx[e] = 0x7fffffff;
-  }
-  int cnt = 0;
-  for (uint32_t s = base; s < cur; s += kPsSlot, ++cnt) {
-    const uint2 en = lds_u2(s);
-    float x = __uint_as_float(en.x);
-    int xi = static_cast<int>(en.y);
-#pragma unroll
-    for (int q = 0; q < K; ++q)
-      if (pf_before(x, xi, best[q], bidx[q])) {
-        const float tv = best[q];
-        const int ti = bidx[q];
-        best[q] = x;
-        bidx[q] = xi;
-        x = tv;
-        xi = ti;
+    for (int i = 0; i < 16; ++i)
+      if ((i & j) == 0) {
+        const float x = a[i], y = a[i + j];
+        a[i] = fmaxf(x, y);
+        a[i + j] = fminf(x, y);
       }
-  }
-  const int n = min(cnt, K);
-#pragma unroll
-  for (int i = 1; i < K; ++i)
-#pragma unroll
-    for (int j2 = K - 1; j2 >= i; --j2)
-      if (bidx[j2 - 1] > bidx[j2]) {  // unused slots hold INT_MAX and sort last
-        const int ti = bidx[j2 - 1];
-        bidx[j2 - 1] = bidx[j2];
-        bidx[j2] = ti;
-        const float tv = best[j2 - 1];
-        best[j2 - 1] = best[j2];
-        best[j2] = tv;
-      }
-#pragma unroll
-  for (int e = 0; e < K; ++e)
-    if (e < n) sts_u2(base + e * kPsSlot, make_uint2(__float_as_uint(best[e]), static_cast<uint32_t>(bidx[e])));
-  return base + n * kPsSlot;
 }
 
-// A value a little below x (x itself for -inf): comparing v > below(x)
-// keeps every v >= x.
-__device__ __forceinline__ float pf_below(float x) { return fmaf(-fabsf(x), 1e-6f, x) - 1e-30f; }
-
-// Stage 1, k_prefill_score<K>: scores, row maxima and the top-k selection
-// (topk <= K) of every query row.
+// Stage 1, k_prefill_score: row maxima and the top-k selection (k <= 16)
+// of every query row, in two passes over the visible key tiles of a query
+// tile (the key tiles stream twice; Q stays in shared memory):
+//  A. each thread keeps 16 slot maxima over its half of the columns
+//     (slot = column mod 16); the 16 largest of the row's 32 slot maxima
+//     are distinct scores, so the k-th largest of them bounds the row's
+//     k-th score from below;
+//  B. every score >= that bound is appended as a (score, index) candidate
+//     (about k + 5 per row) by predicated stores; at the row end the
+//     candidates' exact ranks by (score desc, index asc) give the selection
+//     and their output slots in ascending chunk order.
+// A row whose candidates overflow a half's kPsCap slots is listed for
+// k_prefill_select_rows, which recomputes it exactly.
 template <int K>
 __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PfSmem::kBarOff);
-  uint64_t *q_full = bars, *q_empty = bars + 2, *k_full = bars + 4, *k_empty = bars + 7;
-  uint64_t *acc_full = bars + 10, *acc_empty = bars + 12;
-  uint64_t *pair_bar = bars + 14;  // [4]: the two epilogue warps of one TMEM quadrant
-  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 18);
-  int *abort_s = reinterpret_cast<int *>(bars + 19);
-  float *lists = reinterpret_cast<float *>(smem + PfSmem::kListOff);
-  float2 *thr_x = reinterpret_cast<float2 *>(smem + PfSmem::kThrOff);
-  int *cnt_x = reinterpret_cast<int *>(smem + PfSmem::kCntOff);
+  uint64_t *q_full = bars, *q_empty = bars + 2, *k_full = bars + 4, *k_empty = bars + 6;
+  uint64_t *acc_full = bars + 8, *acc_empty = bars + 10;
+  uint64_t *quad_bar = bars + 12;  // [4]: the two epilogue warps of one TMEM quadrant
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 16);
+  int *abort_s = reinterpret_cast<int *>(bars + 17);
+  uint8_t *cnt_x = smem + PfSmem::kCntOff;                               // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.bh * (a.gist_tiles + a.raw_tiles);
+  const bool raw_topk = a.topk > 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 8 * 32);
+      mbar_init(&acc_empty[i], kPsEpiWarps * 32);
     }
     for (int i = 0; i < PfSmem::kKStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 64);
+    for (int i = 0; i < 4; ++i) mbar_init(&quad_bar[i], 2 * 32);
     *abort_s = 0;
     mbar_fence_init();
     tc::prefetch_map(&a.tm_qraw);
     tc::prefetch_map(&a.tm_qgist);
     tc::prefetch_map(&a.tm_kgist);
   }
-  for (int i = threadIdx.x; i < 2 * kPfRows; i += blockDim.x) thr_x[i] = make_float2(neg_inf(), __int_as_float(-1));
-  if (warp == 1) tc::tmem_alloc(tmem_base_s, 256);
+  if (warp == 1) tc::tmem_alloc(tmem_base_s, 512);  // two accumulators + the row-end exchange
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -303,12 +237,15 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     flag_error(a.status, GSA_DEVERR_TIMEOUT);
     return false;
   };
+  // key-tile passes of a query tile: raw rows with a selection take two
+  auto passes = [&](const PfTile &tl) { return (!tl.is_gist && raw_topk) ? 2 : 1; };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       uint32_t qi = 0, ki = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const PfTile tl = pf_tile(a, t);
         if (tl.n_kt == 0) continue;
         const int qs = qi & 1;
@@ -320,9 +257,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         tc::tma_load_2d(qdst, qm, 0, qrow, &q_full[qs]);
         tc::tma_load_2d(qdst + PfSmem::kQBlock, qm, 64, qrow, &q_full[qs]);
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
-        bool ok = true;
-        for (int j = 0; j < tl.n_kt; ++j, ++ki) {
-          const int ks = ki % PfSmem::kKStages;
+        for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki) {
+          const int j = jj % tl.n_kt, ks = ki % PfSmem::kKStages;
           if (!wait(&k_empty[ks], ((ki / PfSmem::kKStages) & 1) ^ 1)) {
             ok = false;
             break;
@@ -332,7 +268,6 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
           tc::tma_load_2d(kdst, &a.tm_kgist, 0, krow0 + j * kPfKeys, &k_full[ks]);
           tc::tma_load_2d(kdst + PfSmem::kKBlock, &a.tm_kgist, 64, krow0 + j * kPfKeys, &k_full[ks]);
         }
-        if (!ok) break;
         ++qi;
       }
     }
@@ -342,13 +277,13 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       constexpr uint32_t idesc = tc::idesc_bf16(kPfRows, kPfKeys, false, false);
       uint32_t qi = 0, ki = 0, ai = 0;
       const uint32_t sbase = smem_u32(smem);
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const PfTile tl = pf_tile(a, t);
         if (tl.n_kt == 0) continue;
         const int qs = qi & 1;
         if (!wait(&q_full[qs], (qi >> 1) & 1)) break;
-        bool ok = true;
-        for (int j = 0; j < tl.n_kt; ++j, ++ki, ++ai) {
+        for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki, ++ai) {
           const int ks = ki % PfSmem::kKStages, as = ai & 1;
           if (!wait(&k_full[ks], (ki / PfSmem::kKStages) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
             ok = false;
@@ -373,199 +308,187 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     }
   } else {
     // ---------------- epilogue: two threads per query row ----------------
-    // Warp w reads TMEM lane quadrant w % 4; half h = (w - 2) / 4 takes
-    // columns [64h, 64h + 64) of every key tile, in ascending order.  Each
-    // half keeps the K largest scores it has appended (values only, sorted
-    // descending); its K-th is a lower bound on the row's final k-th score,
-    // and so is the partner half's, published once per key tile.  A score is
-    // appended as a (score, index) candidate only when it beats that bound,
-    // so after the first key tile few scores are appended at all; appends
-    // are predicated stores, never branches.  Equal scores: a score equal
-    // to the own bound is not appended (K earlier, lower-index scores of
-    // this half already rank ahead of it); one equal to the partner's is.
-    const int quad = warp & 3, half = (warp - 2) >> 2;
+    const int quad = warp & 3, h = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t base = smem_u32(smem + PfSmem::kCandOff) + (half * kPsCap * kPfRows + r) * 8u;
-    const uint32_t base1 = smem_u32(smem + PfSmem::kCandOff) + (kPsCap * kPfRows + r) * 8u;
-    const uint32_t room = base + (kPsCap - 8) * kPsSlot;  // a cursor beyond this leaves < 8 free slots
+    const uint32_t cand_u = smem_u32(smem + PfSmem::kCandOff);
+    const uint32_t base = cand_u + (h * kPsCap * kPfRows + r) * 8u;          // slot s at base + s * kPsSlot
+    const uint32_t pbase = cand_u + ((h ^ 1) * kPsCap * kPfRows + r) * 8u;  // the partner half's column
     const float nan = __int_as_float(0x7fffffff);
     uint32_t ai = 0, pair_phase = 0;
     auto pair_sync = [&]() -> bool {
-      mbar_arrive(&pair_bar[quad]);
-      const bool okp = wait(&pair_bar[quad], pair_phase);
+      mbar_arrive(&quad_bar[quad]);
+      const bool okq = wait(&quad_bar[quad], pair_phase);
       pair_phase ^= 1;
-      return okp;
+      return okq;
     };
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const PfTile tl = pf_tile(a, t);
+    // one accumulator: this thread's 64 scores, masked past `limit`,
+    // handed to f(v, first column)
+    auto take = [&](int j, int limit, auto &&f) -> bool {
+      const int as = ai & 1;
+      if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai >> 1) & 1))) return false;
+      tc::fence_after_sync();
+      const bool edge = __any_sync(0xffffffffu, (j + 1) * kPfKeys > limit);
+      float v[64];
+      __syncwarp();  // tcgen05.ld is warp-collective
+      tc::ld64(lane_addr + as * kPfKeys + 64 * h, v);
+      const int tb = j * kPfKeys + 64 * h;
+      if (edge)
+#pragma unroll
+        for (int e = 0; e < 64; ++e) v[e] = tb + e < limit ? v[e] : nan;  // masked: fails every compare
+      f(v, tb);
+      tc::fence_before_sync();
+      mbar_arrive(&acc_empty[as]);
+      ++ai;
+      return true;
+    };
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const PfTile tl = pf_tile(a, t);  // (no key tile: every row sees nothing; still written)
       const int row = tl.row0 + r;
       const bool row_ok = row < (tl.is_gist ? a.n_chunks : a.L);
       const int limit = !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, row / a.chunk));
-      const bool want_topk = !tl.is_gist && a.topk > 0;
-      float bst[K];
+      const bool sel_rows = !tl.is_gist && raw_topk;
+      const int ksel = min(a.topk, limit);  // entries this row selects
+      // ---- pass A: slot maxima ----
+      float G[16];
 #pragma unroll
-      for (int q = 0; q < K; ++q) bst[q] = neg_inf();
-      float mx = neg_inf(), thr = neg_inf(), tp = neg_inf();
-      uint32_t cur = base, c0 = base;  // column cursor; entries [c0, cur) not yet in bst
-      // fold the candidates appended since the last call into bst (whole
-      // warp; -inf pads the lanes with fewer, and inserting -inf changes
-      // nothing)
-      auto absorb = [&]() {
-        const int n = static_cast<int>((cur - c0) / kPsSlot);
-        const int nmax = __reduce_max_sync(0xffffffffu, n);
-        const uint32_t last = base + (kPsCap - 1) * kPsSlot;
-        for (int s = 0; s < nmax; s += 4) {
-          float x[4];
+      for (int q = 0; q < 16; ++q) G[q] = neg_inf();
+      for (int j = 0; j < tl.n_kt && ok; ++j)
+        ok = take(j, limit, [&](const float(&v)[64], int) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float y = __uint_as_float(lds_u2(min(c0 + (s + u) * kPsSlot, last)).x);
-            x[u] = s + u < n ? y : neg_inf();
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) pf_insert<K>(bst, x[u]);
-        }
-        c0 = cur;
-      };
-      bool ok = true;
-      for (int j = 0; j < tl.n_kt; ++j, ++ai) {
-        const int as = ai & 1;
-        if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai >> 1) & 1))) {  // warp-uniform outcome
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        const bool edge = __any_sync(0xffffffffu, (j + 1) * kPfKeys > limit);  // some row ends in this tile
-#pragma unroll 1
-        for (int b = 0; b < 2; ++b) {
-          const int tb = j * kPfKeys + half * 64 + b * 32;
-          float v[32];
-          __syncwarp();  // tcgen05.ld is warp-collective
-          tc::ld32(lane_addr + as * kPfKeys + half * 64 + b * 32, v);
-          if (edge)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = tb + e < limit ? v[e] : nan;  // masked: fails every compare
-          if (!want_topk) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
-            continue;
-          }
-          if (j == 0 && b == 0) {
-            // first block: its K largest seed the list; append those >= the K-th
-            float w[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = v[e] == v[e] ? v[e] : neg_inf();
-            pf_sort32(w);
-#pragma unroll
-            for (int q = 0; q < K; ++q) bst[q] = w[q];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pf_append<true>(cur, v[e], bst[K - 1], static_cast<uint32_t>(tb + e));
-            c0 = cur;
-            thr = bst[K - 1];
-            continue;
-          }
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (__any_sync(0xffffffffu, cur > room)) {
-              // some lane has fewer than 8 free slots: every lane drops
-              // what can no longer be selected (one pass for the warp)
-              absorb();
-              cur = pf_filter(base, cur, fmaxf(bst[K - 1], tp));
-              if (cur > room) cur = pf_reduce<K>(base, cur);  // only under many equal scores
-              c0 = cur;
-              thr = fmaxf(bst[K - 1], pf_below(tp));
-            }
-#pragma unroll
-            for (int e = 8 * g; e < 8 * g + 8; ++e) pf_append<false>(cur, v[e], thr, static_cast<uint32_t>(tb + e));
-          }
-        }
-        tc::fence_before_sync();
-        mbar_arrive(&acc_empty[as]);
-        if (want_topk) {  // update the list, publish this half's bound, take the partner's
-          absorb();
-          thr_x[half * kPfRows + r] = make_float2(bst[K - 1], __int_as_float(t));
-          const float2 p = thr_x[(half ^ 1) * kPfRows + r];
-          if (__float_as_int(p.y) == t) tp = fmaxf(tp, p.x);
-          thr = fmaxf(bst[K - 1], pf_below(tp));
-        }
-      }
+          for (int e = 0; e < 64; ++e) G[e & 15] = fmaxf(G[e & 15], v[e]);
+        });
       if (!ok) break;
-      // Row end.  Both halves publish their lists; each computes the row's
-      // k-th score T from both and keeps the candidates >= T of its own
-      // column; half 0 merges the two (ascending index) and writes the row.
-      float *mine = lists + half * (kPfTopkMax * kPfRows) + r;
-      const float *theirs = lists + (half ^ 1) * (kPfTopkMax * kPfRows) + r;
-      if (want_topk) {
+      ps_sort16(G);
+      // the sorted slot maxima go to this row half's own candidate column
+      // (two per slot); rows of other quadrants, which run ahead or behind,
+      // never touch them
 #pragma unroll
-        for (int q = 0; q < K; ++q) mine[q * kPfRows] = bst[q];
-      } else {
-        mine[0] = mx;
-      }
+      for (int q = 0; q < 16; q += 2)
+        sts_u2(base + (q >> 1) * kPsSlot, make_uint2(__float_as_uint(G[q]), __float_as_uint(G[q + 1])));
       if (!pair_sync()) break;
-      float T = neg_inf();
-      int n_gt = 0;
-      if (!want_topk) {
-        mx = fmaxf(mx, theirs[0]);
-      } else {
-        // top K of both lists: elementwise max against the reversed partner
-        // list is a bitonic sequence holding them; sort it descending
-        float c[K];
+      {
+        float o[16];
 #pragma unroll
-        for (int q = 0; q < K; ++q) c[q] = fmaxf(bst[q], theirs[(K - 1 - q) * kPfRows]);
-#pragma unroll
-        for (int j2 = K >> 1; j2 > 0; j2 >>= 1)
-#pragma unroll
-          for (int i = 0; i < K; ++i)
-            if ((i & j2) == 0) {
-              const float x = c[i], y = c[i + j2];
-              c[i] = fmaxf(x, y);
-              c[i + j2] = fminf(x, y);
-            }
-        mx = c[0];
-        T = c[0];
-#pragma unroll
-        for (int q = 0; q < K; ++q)
-          if (q < a.topk) T = c[q];
-#pragma unroll
-        for (int q = 0; q < K; ++q) n_gt += (q < a.topk && c[q] > T) ? 1 : 0;
-        cur = pf_filter(base, cur, T);
-        cnt_x[half * kPfRows + r] = static_cast<int>((cur - base) / kPsSlot);
-      }
-      if (!pair_sync()) break;
-      if (half == 0 && row_ok) {
-        const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
-        float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
-        if (want_topk) {
-          // every score > T, then the lowest-index scores == T up to k
-          int quota = a.topk - n_gt, n_out = 0;
-          const uint32_t end1 = base1 + cnt_x[kPfRows + r] * kPsSlot;
-          int32_t *oi = a.sel_idx + orow * a.topk;
-          float *os = a.sel_score + orow * a.topk;
-          uint32_t p0 = base, p1 = base1;
-          while (p0 < cur || p1 < end1) {
-            const uint2 e0 = p0 < cur ? lds_u2(p0) : make_uint2(0u, 0x7fffffffu);
-            const uint2 e1 = p1 < end1 ? lds_u2(p1) : make_uint2(0u, 0x7fffffffu);
-            const bool take0 = e0.y < e1.y;
-            const uint2 e = take0 ? e0 : e1;
-            p0 += take0 ? kPsSlot : 0u;
-            p1 += take0 ? 0u : kPsSlot;
-            const float x = __uint_as_float(e.x);
-            const bool sel = x > T || (x == T && quota > 0);
-            if (sel) {
-              quota -= x > T ? 0 : 1;
-              oi[n_out] = static_cast<int32_t>(e.y);
-              os[n_out] = x * a.scale;
-              ++n_out;
-            }
-          }
-          for (int q = n_out; q < a.topk; ++q) {
-            oi[q] = -1;
-            os[q] = neg_inf();
-          }
+        for (int q = 0; q < 16; q += 2) {
+          const uint2 w = lds_u2(pbase + (q >> 1) * kPsSlot);
+          o[q] = __uint_as_float(w.x);
+          o[q + 1] = __uint_as_float(w.y);
         }
-        rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
+        ps_merge16(G, o);  // top 16 of the row's 32 slot maxima
       }
+      const float mx = G[0];
+      float bound = G[0];
+#pragma unroll
+      for (int q = 1; q < 16; ++q)
+        if (q < ksel) bound = G[q];
+      if (!pair_sync()) break;  // the slot maxima area becomes the candidate columns
+      const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
+      float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
+      if (h == 0 && row_ok) rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
+      if (!sel_rows) continue;
+      // ---- pass B: candidates >= bound ----
+      uint32_t cnt = 0;
+      for (int j = 0; j < tl.n_kt && ok; ++j)
+        ok = take(j, limit, [&](const float(&v)[64], int tb) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) ps_append(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e));
+        });
+      if (!ok) break;
+      cnt_x[h * kPfRows + r] = static_cast<uint8_t>(min(cnt, 255u));
+      // The row's k-th candidate score T: each half's 16 largest (values
+      // only) meet through TMEM columns 256.. (lane = row), merged by both.
+      const int mine = min(static_cast<int>(cnt), kPsCap);
+      float top[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) top[q] = neg_inf();
+      for (int s0 = 0; s0 < mine; s0 += 4) {
+        float x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(lds_u2(base + min(s0 + i, kPsCap - 1) * kPsSlot).x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (s0 + i < mine) ps_insert16(top, x[i]);
+      }
+      tc::st16(tmem + lane_addr + 256 + 16 * h, top);
+      tc::fence_before_sync();
       if (!pair_sync()) break;
+      tc::fence_after_sync();
+      {
+        float o[16];
+        tc::ld16(tmem + lane_addr + 256 + 16 * (h ^ 1), o);
+        ps_merge16(top, o);
+      }
+      float T = top[0];
+#pragma unroll
+      for (int q = 1; q < 16; ++q)
+        if (q < ksel) T = top[q];
+      const int theirs_raw = cnt_x[(h ^ 1) * kPfRows + r];
+      const int theirs = min(theirs_raw, kPsCap);
+      bool ovf = static_cast<int>(cnt) > kPsCap || theirs_raw > kPsCap;
+      // every candidate >= T is selected unless T is shared past the k-th
+      // place (then the index rule decides: the exact per-row pass)
+      int n_sel = 0;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t qb = q ? pbase : base;
+        const int cq = q ? theirs : mine;
+        for (int u0 = 0; u0 < cq; u0 += 8) {
+          uint32_t y[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) y[k] = lds_u2(qb + min(u0 + k, kPsCap - 1) * kPsSlot).x;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) n_sel += (u0 + k < cq && __uint_as_float(y[k]) >= T) ? 1 : 0;
+        }
+      }
+      ovf |= n_sel != ksel;
+      if (row_ok) {
+        int32_t *oi = a.sel_idx + orow * a.topk;
+        float *os = a.sel_score + orow * a.topk;
+        if (ovf) {
+          if (h == 0) {  // listed for the exact per-row pass
+            const uint32_t slot = atomicAdd(a.ovf_count, 1u);
+            a.ovf_rows[slot] = static_cast<int32_t>(orow);
+          }
+        } else {
+          // both columns are in ascending chunk order: a selected own entry's
+          // slot is the number of selected own entries before it plus the
+          // selected partner entries with a lower index (four own entries at
+          // a time against eight loaded partner entries)
+          int own_before = 0;
+          for (int s0 = 0; s0 < mine; s0 += 4) {
+            uint2 x[4];
+            int pc[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[i] = lds_u2(base + min(s0 + i, kPsCap - 1) * kPsSlot);
+            for (int u0 = 0; u0 < theirs; u0 += 8) {
+              uint2 y[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) y[k] = lds_u2(pbase + min(u0 + k, kPsCap - 1) * kPsSlot);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const bool ys = u0 + k < theirs && __uint_as_float(y[k].x) >= T;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pc[i] += (ys && y[k].y < x[i].y) ? 1 : 0;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (s0 + i < mine && __uint_as_float(x[i].x) >= T) {
+                oi[own_before + pc[i]] = static_cast<int32_t>(x[i].y);
+                os[own_before + pc[i]] = __uint_as_float(x[i].x) * a.scale;
+                ++own_before;
+              }
+          }
+          if (h == 0)
+            for (int q = ksel; q < a.topk; ++q) {
+              oi[q] = -1;
+              os[q] = neg_inf();
+            }
+        }
+      }
+      if (!pair_sync()) break;  // the columns are free for the next tile
     }
   }
 
@@ -573,7 +496,103 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Stage 1b, k_prefill_select_rows: the exact selection of the rows whose
+// candidates overflowed a column in k_prefill_score (short rows with many
+// scores near the bound; none for most inputs).  One warp per listed row:
+// its visible gist scores go to shared memory (lanes split the 128 dims,
+// one warp reduction per key), then k rounds of a warp argmax by (score
+// desc, index asc) pick the row's top k, written in ascending chunk order.
+// The last CTA re-arms the list counter for the next call.
+struct SelectRowsArgs {
+  const __nv_bfloat16 *q_raw, *k_gist;  // [B*hq*L, 128], [B*hkv*N, 128]
+  const int32_t *rows;                  // listed output rows (b*hq + h)*L + pos
+  uint32_t *count, *done;               // list length; CTAs finished
+  int32_t group, chunk, n_chunks, L, topk;
+  float scale;
+  int32_t *sel_idx;
+  float *sel_score;
+};
+
+__global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArgs a) {
+  extern __shared__ float sc_all[];  // [warps][n_chunks]
+  pdl_wait();
+  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t n = *reinterpret_cast<volatile uint32_t *>(a.count);
+  float *sc = sc_all + static_cast<size_t>(warp) * a.n_chunks;
+  for (uint32_t i = blockIdx.x * nw + warp; i < n; i += gridDim.x * nw) {
+    const int orow = a.rows[i];
+    const int bh = orow / a.L, pos = orow % a.L;
+    const int limit = min(a.n_chunks, pos / a.chunk);
+    const int ksel = min(a.topk, limit);
+    const uint2 qw = *reinterpret_cast<const uint2 *>(a.q_raw + static_cast<size_t>(orow) * 128 + 4 * lane);
+    const float q0 = bf16_lo(qw.x), q1 = bf16_hi(qw.x), q2 = bf16_lo(qw.y), q3 = bf16_hi(qw.y);
+    const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128 + 4 * lane;
+    for (int t = 0; t < limit; ++t) {
+      const uint2 kw = *reinterpret_cast<const uint2 *>(kb + static_cast<size_t>(t) * 128);
+      float s = q0 * bf16_lo(kw.x);
+      s = fmaf(q1, bf16_hi(kw.x), s);
+      s = fmaf(q2, bf16_lo(kw.y), s);
+      s = fmaf(q3, bf16_hi(kw.y), s);
+      s = warp_sum(s);
+      if (lane == 0) sc[t] = s;
+    }
+    __syncwarp();
+    int mine = 0x7fffffff;  // lane r < ksel keeps the r-th pick
+    float mine_s = 0.f;
+    for (int it = 0; it < ksel; ++it) {
+      float bv = neg_inf();
+      int bi = 0x7fffffff;
+      for (int t = lane; t < limit; t += 32) {
+        const float v = sc[t];
+        if (v > bv) {  // t increases: equal scores keep the lower index
+          bv = v;
+          bi = t;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == it) {
+        mine = bi;
+        mine_s = bv;
+      }
+      if (lane == 0) sc[bi] = neg_inf();  // taken (scores are finite)
+      __syncwarp();
+    }
+    // ascending chunk order: a pick's slot is the number of picks below it
+    int slot = 0;
+#pragma unroll
+    for (int o = 0; o < 32; ++o) slot += __shfl_sync(0xffffffffu, mine, o) < mine ? 1 : 0;
+    int32_t *oi = a.sel_idx + static_cast<size_t>(orow) * a.topk;
+    float *os = a.sel_score + static_cast<size_t>(orow) * a.topk;
+    if (lane < ksel) {
+      oi[slot] = mine;
+      os[slot] = mine_s * a.scale;
+    } else if (lane < a.topk) {
+      oi[lane] = -1;
+      os[lane] = neg_inf();
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(a.done, 1u) == gridDim.x - 1) {
+      *a.count = 0u;
+      *a.done = 0u;
+      __threadfence();
+    }
   }
 }
 
