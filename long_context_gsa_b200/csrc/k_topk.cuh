@@ -256,10 +256,10 @@ __device__ __forceinline__ unsigned long long rank_key(uint32_t key, int i) {
 }
 
 // Top-k through a lower bound (0 < kk < n, kk <= 256):
-//  1. every warp finds the r-th largest of its 32 threads' maximum keys,
-//     r = ceil(kk / 8); the smallest of these 8 values, L, is reached by at
-//     least 8 r >= kk distinct entries, so it bounds the row's kk-th score
-//     key from below;
+//  1. every warp whose 32 lanes all hold entries finds the r-th largest of
+//     its threads' maximum keys, r = ceil(kk / those warps); the smallest of
+//     these values, L, is reached by at least kk distinct entries, so it
+//     bounds the row's kk-th score key from below;
 //  2. every entry with key >= L is a candidate (in practice about 1.8 kk);
 //  3. each candidate's rank among the candidates, by (score desc, index
 //     asc), is counted directly; ranks < kk are the selection, and a
@@ -285,13 +285,17 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
       const bool keep_max = ((lane & size) == 0) == ((lane & j) == 0);
       m = keep_max ? max(m, o) : min(m, o);
     }
-  const int r = (kk + W - 1) / W;
+  // only warps whose 32 lanes all hold entries take part: each gives r
+  // distinct entries >= its value, and the ones taking part give >= kk
+  const int w_full = n >= 32 ? min(W, (n - 32) / (32 * KPT) + 1) : 0;  // warps w with w*32*KPT + 31 < n
+  if (w_full == 0) return false;  // block-uniform
+  const int r = (kk + w_full - 1) / w_full;
+  if (r > 32) return false;
   if (lane == r - 1) sm.wbound[warp] = m;
   if (tid == 0) sm.count = 0;
   __syncthreads();
   uint32_t L = sm.wbound[0];
-#pragma unroll
-  for (int w = 1; w < W; ++w) L = min(L, sm.wbound[w]);
+  for (int w = 1; w < w_full; ++w) L = min(L, sm.wbound[w]);
   // gather the candidates: one shared atomic per warp
   const unsigned lt = (1u << lane) - 1u;
   int w_cnt = 0;
