@@ -534,9 +534,9 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.scale = pa.scale;
   sr.sel_idx = sel_idx;
   sr.sel_score = sel_score;
-  const int nw = clampi(static_cast<int>((160u << 10) / (static_cast<size_t>(d->n_max) * 4)), 1, 8);
-  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(32 * nw), static_cast<size_t>(nw) * d->n_max * 4, stream,
-                sr);
+  const int nw = clampi(static_cast<int>((160u << 10) / ((static_cast<size_t>(d->n_max) + 128) * 4)), 1, 8);
+  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(32 * nw), static_cast<size_t>(nw) * (d->n_max + 128) * 4,
+                stream, sr);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,

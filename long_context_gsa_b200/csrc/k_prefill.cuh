@@ -79,8 +79,9 @@ __device__ __forceinline__ PfTile pf_tile(const PrefillArgs &a, int t) {
 }
 
 // Scoring-stage layout: warp 0 TMA, warp 1 MMA, warps 2..9 epilogue; warp
-// w reads TMEM lane quadrant w % 4 and owns the 64-column half
-// (w - 2) / 4 of every key tile, so two threads share a query row.
+// w reads TMEM lane quadrant w % 4 and owns half h = (w - 2) / 4 of every
+// key tile (columns 32h .. 32h+31 and 64+32h .. 95+32h, so short rows still
+// spread over both halves); two threads share a query row.
 constexpr int kPsEpiWarps = 8;
 constexpr int kPsThreads = 64 + 32 * kPsEpiWarps;
 constexpr int kPsCap = 48;  // candidate slots per row half
@@ -322,8 +323,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       pair_phase ^= 1;
       return okq;
     };
-    // one accumulator: this thread's 64 scores, masked past `limit`,
-    // handed to f(v, first column)
+    // one accumulator: this thread's 64 scores (columns 32h .. 32h+31 and
+    // 64+32h .. 95+32h of the key tile), masked past `limit`, handed to f
     auto take = [&](int j, int limit, auto &&f) -> bool {
       const int as = ai & 1;
       if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai >> 1) & 1))) return false;
@@ -331,11 +332,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       const bool edge = __any_sync(0xffffffffu, (j + 1) * kPfKeys > limit);
       float v[64];
       __syncwarp();  // tcgen05.ld is warp-collective
-      tc::ld64(lane_addr + as * kPfKeys + 64 * h, v);
-      const int tb = j * kPfKeys + 64 * h;
+      tc::ld32x2(lane_addr + as * kPfKeys + 32 * h, lane_addr + as * kPfKeys + 64 + 32 * h, v);
+      const int tb = j * kPfKeys + 32 * h;  // v[e] is column tb + e (e < 32) or tb + 32 + e (e >= 32)
       if (edge)
 #pragma unroll
-        for (int e = 0; e < 64; ++e) v[e] = tb + e < limit ? v[e] : nan;  // masked: fails every compare
+        for (int e = 0; e < 64; ++e) v[e] = tb + e + (e >> 5) * 32 < limit ? v[e] : nan;  // masked: fails every compare
       f(v, tb);
       tc::fence_before_sync();
       mbar_arrive(&acc_empty[as]);
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       for (int j = 0; j < tl.n_kt && ok; ++j)
         ok = take(j, limit, [&](const float(&v)[64], int tb) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) ps_append(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e));
+          for (int e = 0; e < 64; ++e) ps_append(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
         });
       if (!ok) break;
       cnt_x[h * kPfRows + r] = static_cast<uint8_t>(min(cnt, 255u));
@@ -519,27 +520,41 @@ struct SelectRowsArgs {
 };
 
 __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArgs a) {
-  extern __shared__ float sc_all[];  // [warps][n_chunks]
+  extern __shared__ float sc_all[];  // [warps][n_chunks] scores, then [warps][128] query
   pdl_wait();
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t n = *reinterpret_cast<volatile uint32_t *>(a.count);
   float *sc = sc_all + static_cast<size_t>(warp) * a.n_chunks;
+  float *qs = sc_all + static_cast<size_t>(nw) * a.n_chunks + warp * 128;
   for (uint32_t i = blockIdx.x * nw + warp; i < n; i += gridDim.x * nw) {
     const int orow = a.rows[i];
     const int bh = orow / a.L, pos = orow % a.L;
     const int limit = min(a.n_chunks, pos / a.chunk);
     const int ksel = min(a.topk, limit);
-    const uint2 qw = *reinterpret_cast<const uint2 *>(a.q_raw + static_cast<size_t>(orow) * 128 + 4 * lane);
-    const float q0 = bf16_lo(qw.x), q1 = bf16_hi(qw.x), q2 = bf16_lo(qw.y), q3 = bf16_hi(qw.y);
-    const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128 + 4 * lane;
-    for (int t = 0; t < limit; ++t) {
-      const uint2 kw = *reinterpret_cast<const uint2 *>(kb + static_cast<size_t>(t) * 128);
-      float s = q0 * bf16_lo(kw.x);
-      s = fmaf(q1, bf16_hi(kw.x), s);
-      s = fmaf(q2, bf16_lo(kw.y), s);
-      s = fmaf(q3, bf16_hi(kw.y), s);
-      s = warp_sum(s);
-      if (lane == 0) sc[t] = s;
+    {
+      const uint2 qw = *reinterpret_cast<const uint2 *>(a.q_raw + static_cast<size_t>(orow) * 128 + 4 * lane);
+      qs[4 * lane] = bf16_lo(qw.x);
+      qs[4 * lane + 1] = bf16_hi(qw.x);
+      qs[4 * lane + 2] = bf16_lo(qw.y);
+      qs[4 * lane + 3] = bf16_hi(qw.y);
+    }
+    __syncwarp();
+    // lane t scores keys t, t + 32, ...: whole dot products, 16 independent loads each
+    const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128;
+    for (int t = lane; t < limit; t += 32) {
+      const uint4 *kr = reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(t) * 128);
+      uint4 w[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) w[c] = kr[c];
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(w[c], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s = fmaf(qs[8 * c + e], f[e], s);
+      }
+      sc[t] = s;
     }
     __syncwarp();
     int mine = 0x7fffffff;  // lane r < ksel keeps the r-th pick
