@@ -348,9 +348,11 @@ template <int D, typename T>
 gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
   if (std::is_same<T, __nv_bfloat16>::value) {
     // tensor-core kernel: raw K/V as 2D maps with 8-row boxes
-    const size_t smem = UnfoldTcCfg<D>::kSmemBytes;
-    const int slots = resident_ctas(k_unfold_tc<D>, kUnfoldThreads, smem);
+    // residency with the largest list share (one split), then the share of the chosen split count
+    const int slots =
+        resident_ctas(k_unfold_tc<D>, kUnfoldThreads, UnfoldTcCfg<D>::smem_bytes(std::max(1, ua.k), ua.chunk));
     ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));
+    const size_t smem = UnfoldTcCfg<D>::smem_bytes((std::max(1, ua.k) + ua.n_split - 1) / ua.n_split, ua.chunk);
     const uint64_t rows = static_cast<uint64_t>(B) * ua.hkv * ua.t_max;
     if (!map_rows(&ua.tm_k, ua.raw_k, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D) ||
         !map_rows(&ua.tm_v, ua.raw_v, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D))

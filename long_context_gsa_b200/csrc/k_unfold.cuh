@@ -354,8 +354,15 @@ struct UnfoldTcCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr uint32_t kHalf = kBoxes * 1024;        // K (or V) of one 8-row half-step
   static constexpr uint32_t kStage = 4 * kHalf;           // K and V of two half-steps
-  static constexpr int kStages = 2;  // two steps in flight per warp; more stages cost residency
-  static constexpr uint32_t kSmemBytes = kUnfoldWarps * kStages * kStage + 1024;  // + alignment slack
+  static constexpr int kStages = D == 64 ? 3 : 2;
+  static constexpr uint32_t kRingBytes = kUnfoldWarps * kStages * kStage;
+  // ring (1024-aligned) | selected chunks and their list positions [2][per] |
+  // half-steps (first raw row, valid rows << 16 | item + 1) [(per + 1) * ceil(chunk / 8) + 1]
+  // (the own chunk adds up to ceil(chunk / 8), the last step's pad one)
+  static size_t smem_bytes(int per, int chunk) {
+    const size_t hpc = static_cast<size_t>((chunk + 7) / 8);
+    return kRingBytes + 1024 + 2 * static_cast<size_t>(per) * 4 + ((static_cast<size_t>(per) + 1) * hpc + 1) * 8;
+  }
 };
 
 template <int D>
@@ -364,8 +371,9 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   constexpr int kNT = D / 8, S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ int items[kUnfoldMaxItems];
-  __shared__ int item_pos[kUnfoldMaxItems];
+  const int per = (a.k + a.n_split - 1) / a.n_split;  // list entries of one split
+  int *items = reinterpret_cast<int *>(smem + Cfg::kRingBytes);
+  int *item_pos = items + per;
   __shared__ int n_items_s;
   __shared__ int is_last_s;
   __shared__ float red[kUnfoldWarps][2 + D];
@@ -383,7 +391,6 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
 
   // Selected chunks of this split, in list order (invalid entries dropped).
-  const int per = (a.k + a.n_split - 1) / a.n_split;
   const int i0 = min(a.k, split * per), i1 = min(a.k, i0 + per);
   if (warp == 0) {
     int cnt = 0;
@@ -416,29 +423,35 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   }
   __syncthreads();
 
-  // half-step j -> (first raw row, valid rows, chunk item or -1 for own rows)
+  // half-step j -> (first raw row, valid rows, chunk item or -1 for own
+  // rows), tabulated once so the per-step issue and compute only look up
   const int hpc = (a.chunk + 7) >> 3;  // half-steps per chunk
   const int n_sel = n_items_s;
   const int own_half = (split == a.n_split - 1 && own > 0) ? (own + 7) >> 3 : 0;
   const int n_half = n_sel * hpc + own_half;
   const int n_steps = (n_half + 1) >> 1;
   const int n_mine = n_steps > warp ? (n_steps - warp + kUnfoldWarps - 1) / kUnfoldWarps : 0;
-  auto half = [&](int j, int &first, int &valid, int &item) {
-    if (j >= n_half) {
-      first = 0;
-      valid = 0;
-      item = -1;
-    } else if (j < n_sel * hpc) {
-      const int it = j / hpc, sub = j % hpc;
+  int2 *htab = reinterpret_cast<int2 *>(item_pos + per);
+  for (int j = tid; j < 2 * n_steps; j += kUnfoldThreads) {
+    int first = 0, valid = 0, item = -1;
+    if (j < n_sel * hpc) {
+      const int it = j / hpc, sub = j - it * hpc;
       first = items[it] * a.chunk + 8 * sub;
       valid = min(8, a.chunk - 8 * sub);
       item = sub == 0 ? it : -1;  // the chunk's gist joins with its first half-step
-    } else {
+    } else if (j < n_half) {
       const int q = j - n_sel * hpc;
       first = N * a.chunk + 8 * q;
       valid = min(8, own - 8 * q);
-      item = -1;
     }
+    htab[j] = make_int2(first, (valid << 16) | (item + 1));
+  }
+  __syncthreads();
+  auto half = [&](int j, int &first, int &valid, int &item) {
+    const int2 e = htab[j];
+    first = e.x;
+    valid = e.y >> 16;
+    item = (e.y & 0xffff) - 1;
   };
   const int kv_row0 = (b * a.hkv + kvh) * a.t_max;  // tensor-map row of this kv head's first raw row
   uint8_t *ring = smem + static_cast<size_t>(warp) * S * Cfg::kStage;
