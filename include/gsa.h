@@ -240,8 +240,9 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
  * selection among them) and its own chunk's raw tokens m*chunk .. i.  Gist
  * position m sees its chunk's raw tokens and gists 0..m (compression mask).
  *
- * Both stages are built for bf16 inputs with d = 128 and topk <= 16
- * (GSA_ERR_UNSUPPORTED otherwise), and need t_max = n_max * chunk.
+ * Both stages are built for bf16 inputs with d = 128, topk <= 16 and
+ * n_max <= 57968 chunks (GSA_ERR_UNSUPPORTED otherwise), and need
+ * t_max = n_max * chunk.
  *
  * Stage 1, scoring + selection (tensor cores).  Every raw row is scored
  * against the gists it can see and keeps the top k; every row (raw and

@@ -474,11 +474,14 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
 // Words of the 256-byte status block used by the prefill overflow list
 // (word 0 is the device status; all are zeroed by gsa_workspace_init).
 constexpr int kPfOvfCountWord = 16, kPfOvfDoneWord = 17;
+constexpr int kPfSelectMaxChunks = (227 << 10) / 4 - 128 - kPfTopkMax;
 
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
   if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;  // running top-k lists hold at most 16
+  // the exact re-selection of listed rows holds one row's gist scores in shared memory
+  if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->n_max) * d->chunk != d->t_max) return GSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
   return GSA_OK;
@@ -536,9 +539,8 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.scale = pa.scale;
   sr.sel_idx = sel_idx;
   sr.sel_score = sel_score;
-  const int nw = clampi(static_cast<int>((160u << 10) / ((static_cast<size_t>(d->n_max) + 128) * 4)), 1, 8);
-  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(32 * nw), static_cast<size_t>(nw) * (d->n_max + 128) * 4,
-                stream, sr);
+  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(256),
+                (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4, stream, sr);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,

@@ -502,11 +502,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
-// Stage 1b, k_prefill_select_rows: the exact selection of the rows whose
-// candidates overflowed a column in k_prefill_score (short rows with many
-// scores near the bound; none for most inputs).  One warp per listed row:
-// its visible gist scores go to shared memory (lanes split the 128 dims,
-// one warp reduction per key), then k rounds of a warp argmax by (score
+// Stage 1b, k_prefill_select_rows: the exact selection of the rows that
+// k_prefill_score listed (a full candidate column, or scores equal to the
+// k-th at the boundary; a handful of rows for most inputs).  One CTA per
+// listed row: its visible gist scores go to shared memory (each thread a
+// whole dot product per key), then k rounds of a block argmax by (score
 // desc, index asc) pick the row's top k, written in ascending chunk order.
 // The last CTA re-arms the list counter for the next call.
 struct SelectRowsArgs {
@@ -520,28 +520,24 @@ struct SelectRowsArgs {
 };
 
 __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArgs a) {
-  extern __shared__ float sc_all[];  // [warps][n_chunks] scores, then [warps][128] query
+  extern __shared__ float sc[];  // [n_chunks] scores, then [128] query
+  __shared__ float rv[8];
+  __shared__ int ri[8];
+  __shared__ int picks[32];
   pdl_wait();
-  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t n = *reinterpret_cast<volatile uint32_t *>(a.count);
-  float *sc = sc_all + static_cast<size_t>(warp) * a.n_chunks;
-  float *qs = sc_all + static_cast<size_t>(nw) * a.n_chunks + warp * 128;
-  for (uint32_t i = blockIdx.x * nw + warp; i < n; i += gridDim.x * nw) {
+  float *qs = sc + a.n_chunks;
+  for (uint32_t i = blockIdx.x; i < n; i += gridDim.x) {  // one listed row per CTA
     const int orow = a.rows[i];
     const int bh = orow / a.L, pos = orow % a.L;
     const int limit = min(a.n_chunks, pos / a.chunk);
     const int ksel = min(a.topk, limit);
-    {
-      const uint2 qw = *reinterpret_cast<const uint2 *>(a.q_raw + static_cast<size_t>(orow) * 128 + 4 * lane);
-      qs[4 * lane] = bf16_lo(qw.x);
-      qs[4 * lane + 1] = bf16_hi(qw.x);
-      qs[4 * lane + 2] = bf16_lo(qw.y);
-      qs[4 * lane + 3] = bf16_hi(qw.y);
-    }
-    __syncwarp();
-    // lane t scores keys t, t + 32, ...: whole dot products, 16 independent loads each
+    if (tid < 128) qs[tid] = __bfloat162float(a.q_raw[static_cast<size_t>(orow) * 128 + tid]);
+    __syncthreads();
+    // thread t scores keys t, t + 256, ...: whole dot products, 16 independent loads each
     const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128;
-    for (int t = lane; t < limit; t += 32) {
+    for (int t = tid; t < limit; t += 256) {
       const uint4 *kr = reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(t) * 128);
       uint4 w[16];
 #pragma unroll
@@ -556,13 +552,12 @@ __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArg
       }
       sc[t] = s;
     }
-    __syncwarp();
-    int mine = 0x7fffffff;  // lane r < ksel keeps the r-th pick
-    float mine_s = 0.f;
+    __syncthreads();
+    // k rounds of a block argmax by (score desc, index asc)
     for (int it = 0; it < ksel; ++it) {
       float bv = neg_inf();
       int bi = 0x7fffffff;
-      for (int t = lane; t < limit; t += 32) {
+      for (int t = tid; t < limit; t += 256) {
         const float v = sc[t];
         if (v > bv) {  // t increases: equal scores keep the lower index
           bv = v;
@@ -578,30 +573,41 @@ __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArg
           bi = oi;
         }
       }
-      if (lane == it) {
-        mine = bi;
-        mine_s = bv;
+      if (lane == 0) {
+        rv[warp] = bv;
+        ri[warp] = bi;
       }
-      if (lane == 0) sc[bi] = neg_inf();  // taken (scores are finite)
-      __syncwarp();
+      __syncthreads();
+      if (tid == 0) {
+        for (int w = 1; w < 8; ++w)
+          if (rv[w] > bv || (rv[w] == bv && ri[w] < bi)) {
+            bv = rv[w];
+            bi = ri[w];
+          }
+        const bool ok = bi < limit;  // false only for non-finite scores
+        picks[it] = ok ? bi : 0x7fffffff;
+        if (ok) sc[bi] = neg_inf();  // taken
+        qs[128 + it] = bv;           // pick scores follow the query
+      }
+      __syncthreads();
     }
     // ascending chunk order: a pick's slot is the number of picks below it
-    int slot = 0;
-#pragma unroll
-    for (int o = 0; o < 32; ++o) slot += __shfl_sync(0xffffffffu, mine, o) < mine ? 1 : 0;
     int32_t *oi = a.sel_idx + static_cast<size_t>(orow) * a.topk;
     float *os = a.sel_score + static_cast<size_t>(orow) * a.topk;
-    if (lane < ksel) {
-      oi[slot] = mine;
-      os[slot] = mine_s * a.scale;
-    } else if (lane < a.topk) {
-      oi[lane] = -1;
-      os[lane] = neg_inf();
+    if (tid < ksel) {
+      int slot = 0;
+      for (int u = 0; u < ksel; ++u) slot += (picks[u] < picks[tid] || (picks[u] == picks[tid] && u < tid)) ? 1 : 0;
+      const bool ok = picks[tid] != 0x7fffffff;
+      oi[slot] = ok ? picks[tid] : -1;
+      os[slot] = ok ? qs[128 + tid] * a.scale : neg_inf();
+    } else if (tid < a.topk) {
+      oi[tid] = -1;
+      os[tid] = neg_inf();
     }
-    __syncwarp();
+    __syncthreads();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     __threadfence();
     if (atomicAdd(a.done, 1u) == gridDim.x - 1) {
       *a.count = 0u;

@@ -319,7 +319,13 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
   for (int t = tid; t < C; t += T) {
     const unsigned long long x = sm.cand[t];
     int rank = 0;
-    for (int u = 0; u < C; ++u) rank += sm.cand[u] > x ? 1 : 0;
+    for (int u0 = 0; u0 < C; u0 += 8) {  // eight loads in flight per step
+      unsigned long long y[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = sm.cand[min(u0 + k, C - 1)];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) rank += (u0 + k < C && y[k] > x) ? 1 : 0;
+    }
     sm.sel[t] = rank < kk ? static_cast<uint32_t>(x) : 0u;  // inverted index of a selected entry, else 0
   }
   __syncthreads();
@@ -330,7 +336,13 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
     const uint32_t inv = sm.sel[t];
     if (inv == 0u) continue;
     int pos = 0;  // selected entries with a lower chunk index (a larger inverted index)
-    for (int u = 0; u < C; ++u) pos += sm.sel[u] > inv ? 1 : 0;
+    for (int u0 = 0; u0 < C; u0 += 8) {
+      uint32_t y[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = sm.sel[min(u0 + k, C - 1)];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) pos += (u0 + k < C && y[k] > inv) ? 1 : 0;
+    }
     const int idx = static_cast<int>(0xFFFFFFFFu - inv);
     out_i[pos] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
     if (out_s) out_s[pos] = key_to_float(static_cast<uint32_t>(sm.cand[t] >> 32));
