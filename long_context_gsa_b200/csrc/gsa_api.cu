@@ -331,10 +331,11 @@ gsa_status run_topk(int rows, int hq, const float *scores, int stride, const int
   ta.counters = counters;
   ta.smem_cap = std::min(stride, kTopkSmemCap);
   const dim3 grid(rows), block(kTopkRegThreads);
-  if (stride <= 4 * kTopkRegThreads) return launch(k_topk<4>, grid, block, 0, stream, ta);
-  if (stride <= 16 * kTopkRegThreads) return launch(k_topk<16>, grid, block, 0, stream, ta);
-  if (stride <= 32 * kTopkRegThreads) return launch(k_topk<32>, grid, block, 0, stream, ta);
-  if (stride <= 64 * kTopkRegThreads) return launch(k_topk<64>, grid, block, 0, stream, ta);
+  constexpr size_t kRowBytes = kTopkRegThreads * 4;  // staged row bytes per key a thread holds
+  if (stride <= 4 * kTopkRegThreads) return launch(k_topk<4>, grid, block, 4 * kRowBytes, stream, ta);
+  if (stride <= 16 * kTopkRegThreads) return launch(k_topk<16>, grid, block, 16 * kRowBytes, stream, ta);
+  if (stride <= 32 * kTopkRegThreads) return launch(k_topk<32>, grid, block, 32 * kRowBytes, stream, ta);
+  if (stride <= 64 * kTopkRegThreads) return launch(k_topk<64>, grid, block, 64 * kRowBytes, stream, ta);
   return launch(k_topk_mem, grid, dim3(kTopkThreads), static_cast<size_t>(ta.smem_cap) * 4, stream, ta);
 }
 

@@ -200,6 +200,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_mem(const TopkArgs a) {
   }
   __syncthreads();
 
+  // the kk selected entries, sorted to ascending chunk order (descending
+  // inverted index; the zero padding sorts last)
   int P = 1;
   while (P < kk) P <<= 1;
   for (int i = kk + tid; i < P; i += T) cand[i] = 0ull;
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_mem(const TopkArgs a) {
         const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
         const bool desc = (lo & size) == 0;
         const unsigned long long x = cand[lo], y = cand[hi];
-        if (desc ? (x < y) : (x > y)) {
+        const uint32_t xi = static_cast<uint32_t>(x), yi = static_cast<uint32_t>(y);  // inverted indices
+        if (desc ? (xi < yi) : (xi > yi)) {
           cand[lo] = y;
           cand[hi] = x;
         }
@@ -239,12 +242,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_mem(const TopkArgs a) {
 
 
 constexpr int kTopkRegThreads = 256;
-constexpr int kTopkCandCap = 1024;  // candidates the bound path ranks in shared memory
 
 struct BoundSmem {
-  unsigned long long cand[kTopkCandCap];
-  uint32_t sel[kTopkCandCap];
-  uint32_t wbound[kTopkRegThreads / 32];
+  unsigned long long cand[1024];
+  uint32_t wtop[kTopkRegThreads];       // the full warps' sorted thread maxima
+  uint32_t wcnt[kTopkRegThreads / 32];  // per-warp counts of selected entries
+  unsigned long long kth;               // the kk-th largest rank key
+  uint32_t bound;
   int count;
 };
 
@@ -255,18 +259,52 @@ __device__ __forceinline__ unsigned long long rank_key(uint32_t key, int i) {
   return (static_cast<unsigned long long>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
 }
 
+// Descending bitonic sort of 32*E values by one warp, E per lane (element
+// i = lane*E + e): pairs closer than E meet in registers, the rest through
+// shuffles.
+template <int E, typename K>
+__device__ __forceinline__ void warp_sort_desc(K (&v)[E], int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32 * E; size <<= 1)
+#pragma unroll
+    for (int j = size >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          if ((e & j) == 0) {
+            const bool desc = ((lane * E + e) & size) == 0;
+            const K x = v[e], y = v[e | j];
+            v[e] = desc ? max(x, y) : min(x, y);
+            v[e | j] = desc ? min(x, y) : max(x, y);
+          }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = lane * E + e;
+          const K o = __shfl_xor_sync(0xffffffffu, v[e], j / E);
+          const bool keep_max = ((i & size) == 0) == ((i & j) == 0);
+          v[e] = keep_max ? max(v[e], o) : min(v[e], o);
+        }
+      }
+    }
+}
+
+constexpr int kTopkCandCap = 1024;  // candidates the bound path ranks in shared memory
+
 // Top-k through a lower bound (0 < kk < n, kk <= 256):
-//  1. every warp whose 32 lanes all hold entries finds the r-th largest of
-//     its threads' maximum keys, r = ceil(kk / those warps); the smallest of
-//     these values, L, is reached by at least kk distinct entries, so it
-//     bounds the row's kk-th score key from below;
-//  2. every entry with key >= L is a candidate (in practice about 1.8 kk);
-//  3. each candidate's rank among the candidates, by (score desc, index
-//     asc), is counted directly; ranks < kk are the selection, and a
-//     second count over the selected gives each one's output slot in
-//     ascending chunk order.
-// Returns false (nothing written) when the candidates exceed the buffer;
-// the caller then runs the radix select.  Called by the whole block.
+//  1. the warps whose 32 lanes all hold entries sort their threads' maximum
+//     keys (shuffles); one warp sorts their top R (R = 16, or 32 for
+//     kk > 64) and takes the kk-th largest, L: kk distinct entries reach L,
+//     so it bounds the row's kk-th score key from below;
+//  2. every entry with key >= L is a candidate (in practice under 1.2 kk);
+//  3. the candidate of rank kk - 1 among the candidates, by (score desc,
+//     index asc), is the row's kk-th rank key: one warp sorts up to 128
+//     candidates, more are ranked by counting (each against all);
+//  4. the entries reaching that key (exactly kk: rank keys are distinct)
+//     are written in ascending chunk order straight from the registers.
+// Returns false (nothing written) when no bound can be taken or the
+// candidates exceed the buffer; the caller then runs the radix select.
+// Called by the whole block.
 template <int KPT>
 __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n, int kk, const uint32_t (&key)[KPT],
                                               int base, BoundSmem &sm) {
@@ -276,26 +314,38 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
 #pragma unroll
   for (int j = 0; j < KPT; ++j)
     if (base + 32 * j < n) m = max(m, key[j]);
-  // descending bitonic sort of the warp's 32 maxima (shuffles only)
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1)
-#pragma unroll
-    for (int j = size >> 1; j > 0; j >>= 1) {
-      const uint32_t o = __shfl_xor_sync(0xffffffffu, m, j);
-      const bool keep_max = ((lane & size) == 0) == ((lane & j) == 0);
-      m = keep_max ? max(m, o) : min(m, o);
-    }
-  // only warps whose 32 lanes all hold entries take part: each gives r
-  // distinct entries >= its value, and the ones taking part give >= kk
+  {
+    uint32_t v[1] = {m};
+    warp_sort_desc<1>(v, lane);
+    m = v[0];
+  }
   const int w_full = n >= 32 ? min(W, (n - 32) / (32 * KPT) + 1) : 0;  // warps w with w*32*KPT + 31 < n
-  if (w_full == 0) return false;  // block-uniform
-  const int r = (kk + w_full - 1) / w_full;
-  if (r > 32) return false;
-  if (lane == r - 1) sm.wbound[warp] = m;
+  const int R = kk > 64 ? 32 : 16;
+  if (w_full * R < kk) return false;  // block-uniform
+  if (lane < R) sm.wtop[warp * R + lane] = warp < w_full ? m : 0u;
   if (tid == 0) sm.count = 0;
   __syncthreads();
-  uint32_t L = sm.wbound[0];
-  for (int w = 1; w < w_full; ++w) L = min(L, sm.wbound[w]);
+  if (warp == 0) {
+    if (R == 16) {
+      uint32_t v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = sm.wtop[lane * 4 + e];
+      warp_sort_desc<4>(v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (lane * 4 + e == kk - 1) sm.bound = v[e];
+    } else {
+      uint32_t v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = sm.wtop[lane * 8 + e];
+      warp_sort_desc<8>(v, lane);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (lane * 8 + e == kk - 1) sm.bound = v[e];
+    }
+  }
+  __syncthreads();
+  const uint32_t L = sm.bound;  // nonzero: at least kk nonzero values were sorted
   // gather the candidates: one shared atomic per warp
   const unsigned lt = (1u << lane) - 1u;
   int w_cnt = 0;
@@ -315,37 +365,54 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
   __syncthreads();
   const int C = sm.count;
   if (C > kTopkCandCap) return false;  // block-uniform
-  // rank of each candidate among all candidates (keys are distinct)
-  for (int t = tid; t < C; t += T) {
-    const unsigned long long x = sm.cand[t];
-    int rank = 0;
-    for (int u0 = 0; u0 < C; u0 += 8) {  // eight loads in flight per step
-      unsigned long long y[8];
+  if (C <= 128) {  // one warp sorts the candidates
+    if (warp == 0) {
+      unsigned long long v[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = sm.cand[min(u0 + k, C - 1)];
+      for (int e = 0; e < 4; ++e) v[e] = lane * 4 + e < C ? sm.cand[lane * 4 + e] : 0ull;
+      warp_sort_desc<4>(v, lane);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) rank += (u0 + k < C && y[k] > x) ? 1 : 0;
+      for (int e = 0; e < 4; ++e)
+        if (lane * 4 + e == kk - 1) sm.kth = v[e];
     }
-    sm.sel[t] = rank < kk ? static_cast<uint32_t>(x) : 0u;  // inverted index of a selected entry, else 0
+  } else {  // each candidate's rank is counted against all
+    for (int t = tid; t < C; t += T) {
+      const unsigned long long x = sm.cand[t];
+      int rank = 0;
+      for (int u0 = 0; u0 < C; u0 += 8) {  // eight loads in flight per step
+        unsigned long long y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[k] = sm.cand[min(u0 + k, C - 1)];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rank += (u0 + k < C && y[k] > x) ? 1 : 0;
+      }
+      if (rank == kk - 1) sm.kth = x;
+    }
   }
   __syncthreads();
+  const unsigned long long kth = sm.kth;
+  int w_sel = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    w_sel += __popc(__ballot_sync(0xffffffffu, base + 32 * j < n && key[j] >= L && rank_key(key[j], base + 32 * j) >= kth));
+  if (lane == 0) sm.wcnt[warp] = w_sel;
+  __syncthreads();
+  int pos = 0;
+  for (int w = 0; w < warp; ++w) pos += sm.wcnt[w];
   pdl_trigger();
   int32_t *out_i = a.sel_idx + static_cast<size_t>(row) * a.k;
   float *out_s = a.sel_score ? a.sel_score + static_cast<size_t>(row) * a.k : nullptr;
-  for (int t = tid; t < C; t += T) {
-    const uint32_t inv = sm.sel[t];
-    if (inv == 0u) continue;
-    int pos = 0;  // selected entries with a lower chunk index (a larger inverted index)
-    for (int u0 = 0; u0 < C; u0 += 8) {
-      uint32_t y[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = sm.sel[min(u0 + k, C - 1)];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) pos += (u0 + k < C && y[k] > inv) ? 1 : 0;
+  for (int j = 0; j < KPT; ++j) {
+    const int idx = base + 32 * j;
+    const bool c = idx < n && key[j] >= L && rank_key(key[j], idx) >= kth;
+    const unsigned bal = __ballot_sync(0xffffffffu, c);
+    if (c) {
+      const int o = pos + __popc(bal & lt);
+      out_i[o] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
+      if (out_s) out_s[o] = key_to_float(key[j]);
     }
-    const int idx = static_cast<int>(0xFFFFFFFFu - inv);
-    out_i[pos] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
-    if (out_s) out_s[pos] = key_to_float(static_cast<uint32_t>(sm.cand[t] >> 32));
+    pos += __popc(bal);
   }
   for (int i = kk + tid; i < a.k; i += T) {
     out_i[i] = -1;
@@ -356,14 +423,22 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
 }
 
 template <int KPT>
-__global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : (KPT <= 32 ? 2 : 1)) k_topk(const TopkArgs a) {
+__global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : 1) k_topk(const TopkArgs a) {
   constexpr int T = kTopkRegThreads, W = T / 32;
   __shared__ uint32_t hist[256];
   __shared__ int info[4];
   __shared__ int wtot[2][W];
   __shared__ BoundSmem bsm;
 
+  extern __shared__ __align__(16) float srow_s[];  // [KPT * T]: the row, staged by one bulk copy
+  __shared__ uint64_t load_bar;
+
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    mbar_init(&load_bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
   pdl_wait();
   const int b = row / a.hq;
   int n = a.counts ? a.counts[row] : a.n_gists[b] / a.count_div;
@@ -371,11 +446,20 @@ __global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : (KPT <= 32 ? 
   const float *srow = a.scores + static_cast<size_t>(row) * a.stride;
   const int base = warp * 32 * KPT + lane;
 
+  // the row's first n & ~3 scores arrive in one bulk copy when the row
+  // starts on a 16-byte boundary; the rest (and a timed-out copy) are read
+  // from global memory directly
+  const int n4 = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0 ? (n & ~3) : 0;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&load_bar, static_cast<uint32_t>(n4) * 4u);
+    if (n4 > 0) bulk_g2s(srow_s, srow, static_cast<uint32_t>(n4) * 4u, &load_bar);
+  }
+  const int staged = mbar_wait(&load_bar, 0) ? n4 : 0;
   uint32_t key[KPT];
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
     const int i = base + 32 * j;
-    key[j] = i < n ? float_to_key(__ldcg(srow + i)) : 0u;
+    key[j] = i < staged ? float_to_key(srow_s[i]) : (i < n ? float_to_key(__ldcg(srow + i)) : 0u);
   }
 
   const int kk = min(a.k, n);

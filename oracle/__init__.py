@@ -112,6 +112,8 @@ class Oracle:
             fn.argtypes = [C.POINTER(argt)]
             fn.restype = C.c_int
         self.lib.gsa_oracle_default_threads.restype = C.c_int
+        self.lib.gsa_oracle_topk.argtypes = [_dp, _ip, C.c_int64, C.c_int32, C.c_int32, _ip, _dp]
+        self.lib.gsa_oracle_topk.restype = C.c_int
 
     def default_threads(self) -> int:
         return int(self.lib.gsa_oracle_default_threads())
@@ -138,6 +140,20 @@ class Oracle:
                         _ip_(res.get("set_idx")), _dp_(res.get("set_w")), n_threads)
         _ok(self.lib.gsa_oracle_decode(C.byref(a)), "decode")
         return res
+
+    # -------------------------------------------------------------------- topk
+    def topk(self, scores, n_valid, k):
+        """Selection step alone on given scores [rows, stride] (float64 compare):
+        (sel [rows, k] ascending index, -1 padded; sel_score, -inf padded)."""
+        s = np.ascontiguousarray(scores, dtype=np.float64)
+        rows, stride = s.shape
+        n = _i32(n_valid)
+        if n.shape != (rows,):
+            raise ValueError("n_valid shape")
+        sel = np.full((rows, k), -1, np.int32)
+        ssc = np.zeros((rows, k))
+        _ok(self.lib.gsa_oracle_topk(s.ctypes.data_as(_dp), _ip_(n), rows, stride, k, _ip_(sel), _dp_(ssc)), "topk")
+        return sel, ssc
 
     # -------------------------------------------------------------------- hgsa
     def hgsa(self, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, *, chunk, group,

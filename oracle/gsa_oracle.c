@@ -254,6 +254,50 @@ static int32_t forced_selection(const int32_t *in, int32_t k, int32_t n_valid, s
   return n;
 }
 
+/* Step 2 alone, on given scores ([nl] Selectie, [ja] 2.1 step 3): for each
+ * row, the min(k, n_valid[row]) highest of scores[row][0 .. n_valid), equal
+ * scores to the lower index, written in ascending index order to sel_idx
+ * [rows][k] (-1 padded) with their scores in sel_score (NULL allowed; -inf
+ * padded).  Scores are compared as given (no rescaling).  Returns ORC_EINVAL
+ * for a negative count or one above `stride`. */
+int gsa_oracle_topk(const double *scores, const int32_t *n_valid, int64_t rows, int32_t stride, int32_t k,
+                    int32_t *sel_idx, double *sel_score) {
+  if (rows < 0 || stride < 0 || k < 0) return ORC_EINVAL;
+  scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)(stride > 0 ? stride : 1));
+  if (!cand) return ORC_ENOMEM;
+  for (int64_t r = 0; r < rows; ++r) {
+    const int32_t n = n_valid[r];
+    if (n < 0 || n > stride) {
+      free(cand);
+      return ORC_EINVAL;
+    }
+    for (int32_t m = 0; m < n; ++m) {
+      cand[m].s = scores[r * stride + m];
+      cand[m].m = m;
+    }
+    const int32_t ns = select_topk(cand, n, k);
+    /* ascending index order: mark, then sweep the indices */
+    int32_t *out = sel_idx + r * k;
+    double *outs = sel_score ? sel_score + r * k : NULL;
+    for (int32_t i = 0; i < k; ++i) {
+      out[i] = -1;
+      if (outs) outs[i] = -INFINITY;
+    }
+    for (int32_t i = 0; i < ns; ++i) { /* insertion by index among the chosen */
+      int32_t j = i;
+      while (j > 0 && out[j - 1] > cand[i].m) {
+        out[j] = out[j - 1];
+        if (outs) outs[j] = outs[j - 1];
+        --j;
+      }
+      out[j] = cand[i].m;
+      if (outs) outs[j] = cand[i].s;
+    }
+  }
+  free(cand);
+  return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Thread pool over output rows.                                             */
 /* ------------------------------------------------------------------------ */

@@ -467,9 +467,45 @@ def _check_golden(orc, G):
         assert abs(res["lse"][row] - lse) < 1e-13, case["name"]
 
 
+# ------------------------------------------------------------ selection alone
+def pin_topk_selection(orc):
+    """Selection on given scores: the chosen set is the brute-force best
+    subset on tiny rows; on larger tie-heavy rows every chosen entry
+    outranks every other by (score desc, index asc); output in ascending
+    index order, -1 / -inf padded; k >= n keeps all, k = 0 keeps none."""
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        n = int(rng.integers(0, 8))
+        k = int(rng.integers(0, 6))
+        sc = rng.integers(0, 4, size=(1, 8)).astype(np.float64) * 0.5  # many exact ties
+        sel, ssc = orc.topk(sc, [n], k)
+        want = brute_topk(list(sc[0, :n]), k)
+        got = [int(x) for x in sel[0] if x >= 0]
+        assert set(got) == want, (trial, got, want)
+        assert got == sorted(got) and len(got) == min(k, n)
+        assert all(int(x) == -1 for x in sel[0][len(got):])
+        assert all(ssc[0, i] == sc[0, got[i]] for i in range(len(got)))
+        assert all(ssc[0, i] == -np.inf for i in range(len(got), k))
+    for n, k, levels in ((300, 17, 5), (1000, 64, 1000), (50, 50, 3), (64, 80, 2)):
+        sc = rng.integers(0, levels, size=(3, n)).astype(np.float64)
+        nv = [n, n // 2, 0]
+        sel, _ = orc.topk(sc, nv, k)
+        for r in range(3):
+            got = [int(x) for x in sel[r] if x >= 0]
+            assert got == sorted(got) and len(got) == min(k, nv[r])
+            chosen = set(got)
+            rest = [m for m in range(nv[r]) if m not in chosen]
+            if got and rest:
+                worst = min(got, key=lambda m: (sc[r, m], -m))     # lowest-ranked chosen
+                best = max(rest, key=lambda m: (sc[r, m], -m))     # highest-ranked other
+                assert (sc[r, worst], -worst) > (sc[r, best], -best)
+    sel, _ = orc.topk(np.zeros((1, 10)), [10], 4)
+    assert [int(x) for x in sel[0]] == [0, 1, 2, 3]  # all equal: the lowest indices
+
+
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
                pin_decode_golden]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]
-ALL_PINS = DECODE_PINS + HGSA_PINS + PREFILL_PINS
+ALL_PINS = [pin_topk_selection] + DECODE_PINS + HGSA_PINS + PREFILL_PINS
