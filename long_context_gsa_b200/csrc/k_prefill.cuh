@@ -91,14 +91,16 @@ struct PfSmem {
   static constexpr uint32_t kQBytes = 2 * kQBlock;           // d = 128
   static constexpr uint32_t kKBlock = kPfKeys * 128;
   static constexpr uint32_t kKBytes = 2 * kKBlock;
-  static constexpr uint32_t kQOff = 0;                       // 2 Q buffers
-  static constexpr uint32_t kKOff = 2 * kQBytes;             // kKStages K stages
-  static constexpr int kKStages = 2;
+  static constexpr int kQStages = 1;  // the next tile's Q lands during the row end
+  static constexpr int kKStages = 3;
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKOff = kQStages * kQBytes;
   // [2 halves][kPsCap][128 rows] (score, index); pass A first uses a row
   // half's first 8 slots for its 16 sorted slot maxima
   static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;
   static constexpr uint32_t kCntOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [2][128] candidate counts (bytes)
-  static constexpr uint32_t kBarOff = kCntOff + 2 * kPfRows;
+  static constexpr uint32_t kSelOff = kCntOff + 2 * kPfRows;                 // [2][128] selected counts (bytes)
+  static constexpr uint32_t kBarOff = kSelOff + 2 * kPfRows;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
 };
 static_assert(PfSmem::kBytes <= 232448, "prefill scoring shared memory");
@@ -116,7 +118,7 @@ __device__ __forceinline__ void sts_u2(uint32_t a, uint2 v) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
 
-// Append (v, idx) to a row quarter's column when v >= bound: the store and
+// Append (v, idx) to a row half's column when v >= bound: the store and
 // the count are predicated (no branch); past kPsCap the last slot is
 // overwritten and only the count grows, which the row end reports as an
 // overflow.  NaN (a masked score) fails the compare.
@@ -131,6 +133,12 @@ __device__ __forceinline__ void ps_append(uint32_t base, uint32_t &cnt, float v,
       : "+r"(cnt)
       : "f"(v), "f"(bound), "r"(base), "r"(__float_as_uint(v)), "r"(kPsCap - 1), "r"(kPsSlot), "r"(idx)
       : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
 }
 
 // Descending bitonic sort of 16 values in registers (no NaN inputs).
@@ -179,41 +187,50 @@ __device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16])
 
 // Stage 1, k_prefill_score: row maxima and the top-k selection (k <= 16)
 // of every query row, in two passes over the visible key tiles of a query
-// tile (the key tiles stream twice; Q stays in shared memory):
+// tile (the key tiles stream twice through a 3-stage ring; Q stays in
+// shared memory):
 //  A. each thread keeps 16 slot maxima over its half of the columns
 //     (slot = column mod 16); the 16 largest of the row's 32 slot maxima
 //     are distinct scores, so the k-th largest of them bounds the row's
 //     k-th score from below;
 //  B. every score >= that bound is appended as a (score, index) candidate
-//     (about k + 5 per row) by predicated stores; at the row end the
-//     candidates' exact ranks by (score desc, index asc) give the selection
-//     and their output slots in ascending chunk order.
-// A row whose candidates overflow a half's kPsCap slots is listed for
-// k_prefill_select_rows, which recomputes it exactly.
+//     (about k + 5 per row) by predicated stores, in ascending index order;
+//     at the row end each half sorts its 16 largest candidate values, the
+//     halves exchange them through TMEM and merge them into the row's k-th
+//     candidate score T, keep (compact) their entries >= T, and write the
+//     two ascending lists merged by index, eight output slots per half.
+// A row whose candidates overflow a half's kPsCap slots, or whose k-th
+// score is shared by a (k+1)-th (the index rule then decides), is listed
+// for k_prefill_select_rows, which recomputes it exactly.
 template <int K>
 __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PfSmem::kBarOff);
-  uint64_t *q_full = bars, *q_empty = bars + 2, *k_full = bars + 4, *k_empty = bars + 6;
-  uint64_t *acc_full = bars + 8, *acc_empty = bars + 10;
-  uint64_t *quad_bar = bars + 12;  // [4]: the two epilogue warps of one TMEM quadrant
+  constexpr int kQS = PfSmem::kQStages, kKS = PfSmem::kKStages;
+  uint64_t *q_full = bars, *q_empty = bars + kQS, *k_full = bars + 2 * kQS, *k_empty = k_full + kKS;
+  uint64_t *acc_full = k_empty + kKS, *acc_empty = acc_full + 2;
+  uint64_t *quad_bar = acc_empty + 2;  // [4]: the two epilogue warps of one TMEM quadrant
+  static_assert(2 * kQS + 2 * kKS + 8 <= 16, "barrier block");
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 16);
   int *abort_s = reinterpret_cast<int *>(bars + 17);
   uint8_t *cnt_x = smem + PfSmem::kCntOff;                               // [2][128]
+  uint8_t *sel_x = smem + PfSmem::kSelOff;                               // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.bh * (a.gist_tiles + a.raw_tiles);
   const bool raw_topk = a.topk > 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQS; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kPsEpiWarps * 32);
     }
-    for (int i = 0; i < PfSmem::kKStages; ++i) {
+    for (int i = 0; i < kKS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
@@ -249,8 +266,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const PfTile tl = pf_tile(a, t);
         if (tl.n_kt == 0) continue;
-        const int qs = qi & 1;
-        if (!wait(&q_empty[qs], ((qi >> 1) & 1) ^ 1)) break;
+        const int qs = qi % kQS;
+        if (!wait(&q_empty[qs], ((qi / kQS) & 1) ^ 1)) break;
         uint8_t *qdst = smem + PfSmem::kQOff + qs * PfSmem::kQBytes;
         const CUtensorMap *qm = tl.is_gist ? &a.tm_qgist : &a.tm_qraw;
         const int qrow = tl.bh * (tl.is_gist ? a.n_chunks : a.L) + tl.row0;
@@ -259,8 +276,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         tc::tma_load_2d(qdst + PfSmem::kQBlock, qm, 64, qrow, &q_full[qs]);
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
         for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki) {
-          const int j = jj % tl.n_kt, ks = ki % PfSmem::kKStages;
-          if (!wait(&k_empty[ks], ((ki / PfSmem::kKStages) & 1) ^ 1)) {
+          const int j = jj % tl.n_kt, ks = ki % kKS;
+          if (!wait(&k_empty[ks], ((ki / kKS) & 1) ^ 1)) {
             ok = false;
             break;
           }
@@ -282,11 +299,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const PfTile tl = pf_tile(a, t);
         if (tl.n_kt == 0) continue;
-        const int qs = qi & 1;
-        if (!wait(&q_full[qs], (qi >> 1) & 1)) break;
+        const int qs = qi % kQS;
+        if (!wait(&q_full[qs], (qi / kQS) & 1)) break;
         for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki, ++ai) {
-          const int ks = ki % PfSmem::kKStages, as = ai & 1;
-          if (!wait(&k_full[ks], (ki / PfSmem::kKStages) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
+          const int ks = ki % kKS, as = ai & 1;
+          if (!wait(&k_full[ks], (ki / kKS) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
             ok = false;
             break;
           }
@@ -397,20 +414,25 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
           for (int e = 0; e < 64; ++e) ps_append(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
         });
       if (!ok) break;
-      cnt_x[h * kPfRows + r] = static_cast<uint8_t>(min(cnt, 255u));
-      // The row's k-th candidate score T: each half's 16 largest (values
-      // only) meet through TMEM columns 256.. (lane = row), merged by both.
+      bool ovf = cnt > static_cast<uint32_t>(kPsCap);  // the row goes to the exact per-row pass
       const int mine = min(static_cast<int>(cnt), kPsCap);
+      cnt_x[h * kPfRows + r] = static_cast<uint8_t>(ovf ? 255 : mine);
+      // The row's k-th candidate score T: each half's 16 largest (values
+      // only, sorted 16 at a time) meet through TMEM columns 256.. (lane =
+      // row) and are merged by both.
       float top[16];
+      {
 #pragma unroll
-      for (int q = 0; q < 16; ++q) top[q] = neg_inf();
-      for (int s0 = 0; s0 < mine; s0 += 4) {
-        float x[4];
+        for (int q = 0; q < 16; ++q) top[q] = q < mine ? __uint_as_float(lds_u32(base + q * kPsSlot)) : neg_inf();
+        ps_sort16(top);
+        for (int s0 = 16; s0 < mine; s0 += 16) {
+          float x[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(lds_u2(base + min(s0 + i, kPsCap - 1) * kPsSlot).x);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (s0 + i < mine) ps_insert16(top, x[i]);
+          for (int q = 0; q < 16; ++q)
+            x[q] = s0 + q < mine ? __uint_as_float(lds_u32(base + (s0 + q) * kPsSlot)) : neg_inf();
+          ps_sort16(x);
+          ps_merge16(top, x);
+        }
       }
       tc::st16(tmem + lane_addr + 256 + 16 * h, top);
       tc::fence_before_sync();
@@ -425,68 +447,72 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
 #pragma unroll
       for (int q = 1; q < 16; ++q)
         if (q < ksel) T = top[q];
-      const int theirs_raw = cnt_x[(h ^ 1) * kPfRows + r];
-      const int theirs = min(theirs_raw, kPsCap);
-      bool ovf = static_cast<int>(cnt) > kPsCap || theirs_raw > kPsCap;
-      // every candidate >= T is selected unless T is shared past the k-th
-      // place (then the index rule decides: the exact per-row pass)
-      int n_sel = 0;
+      ovf |= cnt_x[(h ^ 1) * kPfRows + r] == 255;
+      // this half's entries >= T, compacted in order to the column's front
+      uint32_t w = base;
+      for (int s0 = 0; s0 < mine; s0 += 8) {
+        uint2 x[8];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const uint32_t qb = q ? pbase : base;
-        const int cq = q ? theirs : mine;
-        for (int u0 = 0; u0 < cq; u0 += 8) {
-          uint32_t y[8];
+        for (int k = 0; k < 8; ++k) x[k] = lds_u2(base + min(s0 + k, kPsCap - 1) * kPsSlot);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) y[k] = lds_u2(qb + min(u0 + k, kPsCap - 1) * kPsSlot).x;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) n_sel += (u0 + k < cq && __uint_as_float(y[k]) >= T) ? 1 : 0;
-        }
+        for (int k = 0; k < 8; ++k)
+          if (s0 + k < mine && __uint_as_float(x[k].x) >= T) {
+            sts_u2(w, x[k]);
+            w += kPsSlot;
+          }
       }
-      ovf |= n_sel != ksel;
+      const int n_own = static_cast<int>((w - base) / kPsSlot);
+      sel_x[h * kPfRows + r] = static_cast<uint8_t>(n_own);
+      if (!pair_sync()) break;
+      const int n_their = sel_x[(h ^ 1) * kPfRows + r];
+      // every entry >= T is selected unless T is shared past the k-th place
+      // (then the index rule decides: the exact per-row pass)
+      ovf |= n_own + n_their != ksel;
       if (row_ok) {
-        int32_t *oi = a.sel_idx + orow * a.topk;
-        float *os = a.sel_score + orow * a.topk;
         if (ovf) {
           if (h == 0) {  // listed for the exact per-row pass
             const uint32_t slot = atomicAdd(a.ovf_count, 1u);
             a.ovf_rows[slot] = static_cast<int32_t>(orow);
           }
         } else {
-          // both columns are in ascending chunk order: a selected own entry's
-          // slot is the number of selected own entries before it plus the
-          // selected partner entries with a lower index (four own entries at
-          // a time against eight loaded partner entries)
-          int own_before = 0;
-          for (int s0 = 0; s0 < mine; s0 += 4) {
-            uint2 x[4];
-            int pc[4] = {0, 0, 0, 0};
+          // the merged selection in ascending chunk index order; this half
+          // writes output slots 8h .. 8h+7 (both lists are ascending)
+          int ia = 0, ib = 0;
+          for (int q = 0; q < 8 * h; ++q) {
+            const uint32_t xa = ia < n_own ? lds_u32(base + ia * kPsSlot + 4) : 0xffffffffu;
+            const uint32_t xb = ib < n_their ? lds_u32(pbase + ib * kPsSlot + 4) : 0xffffffffu;
+            if (xa < xb) ++ia;
+            else ++ib;
+          }
+          int32_t oid[8];
+          float osc[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) x[i] = lds_u2(base + min(s0 + i, kPsCap - 1) * kPsSlot);
-            for (int u0 = 0; u0 < theirs; u0 += 8) {
-              uint2 y[8];
+          for (int q = 0; q < 8; ++q) {
+            const uint2 xa = ia < n_own ? lds_u2(base + ia * kPsSlot) : make_uint2(0u, 0xffffffffu);
+            const uint2 xb = ib < n_their ? lds_u2(pbase + ib * kPsSlot) : make_uint2(0u, 0xffffffffu);
+            const bool ta = xa.y < xb.y;
+            const uint2 x = ta ? xa : xb;
+            ia += ta ? 1 : 0;
+            ib += ta ? 0 : 1;
+            const bool valid = x.y != 0xffffffffu;
+            oid[q] = valid ? static_cast<int32_t>(x.y) : -1;
+            osc[q] = valid ? __uint_as_float(x.x) * a.scale : neg_inf();
+          }
+          int32_t *oi = a.sel_idx + orow * a.topk + 8 * h;
+          float *os = a.sel_score + orow * a.topk + 8 * h;
+          if (a.topk == 16) {
+            reinterpret_cast<int4 *>(oi)[0] = make_int4(oid[0], oid[1], oid[2], oid[3]);
+            reinterpret_cast<int4 *>(oi)[1] = make_int4(oid[4], oid[5], oid[6], oid[7]);
+            reinterpret_cast<float4 *>(os)[0] = make_float4(osc[0], osc[1], osc[2], osc[3]);
+            reinterpret_cast<float4 *>(os)[1] = make_float4(osc[4], osc[5], osc[6], osc[7]);
+          } else {
 #pragma unroll
-              for (int k = 0; k < 8; ++k) y[k] = lds_u2(pbase + min(u0 + k, kPsCap - 1) * kPsSlot);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const bool ys = u0 + k < theirs && __uint_as_float(y[k].x) >= T;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) pc[i] += (ys && y[k].y < x[i].y) ? 1 : 0;
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (s0 + i < mine && __uint_as_float(x[i].x) >= T) {
-                oi[own_before + pc[i]] = static_cast<int32_t>(x[i].y);
-                os[own_before + pc[i]] = __uint_as_float(x[i].x) * a.scale;
-                ++own_before;
+            for (int q = 0; q < 8; ++q)
+              if (8 * h + q < a.topk) {
+                oi[q] = oid[q];
+                os[q] = osc[q];
               }
           }
-          if (h == 0)
-            for (int q = ksel; q < a.topk; ++q) {
-              oi[q] = -1;
-              os[q] = neg_inf();
-            }
         }
       }
       if (!pair_sync()) break;  // the columns are free for the next tile
