@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--workload", default="llama1b_8x")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
+    p.add_argument("--extra-only", action="store_true",
+                   help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
     p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,prefill_32k",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
@@ -398,6 +400,23 @@ def job_rate(units_per_rank_step, world, steps, total_ms):
     return units_per_rank_step * world * steps / (total_ms / 1e3)
 
 
+def measure_extra(G, W, args, dev, flush, hbm, bf16):
+    """The --extra workloads, each against its own roofline (rank 0, one GPU)."""
+    extra = {}
+    for name in [n for n in args.extra.split(",") if n]:
+        c = W.CONFIGS[name]
+        if name.startswith("prefill"):
+            extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)
+        elif c.group:
+            extra[name] = measure_hgsa(G, W, c, dev, args, flush, hbm)
+        else:
+            m = measure_flat(G, W, c, dev, args, flush, c.seed)
+            extra[name] = flat_summary(c, m, hbm)
+            del m
+        torch.cuda.empty_cache()
+    return extra
+
+
 def run_gsa(args, world, rank, local):
     import long_context_gsa_b200 as G
     import long_context_gsa_b200.workloads as W
@@ -418,23 +437,17 @@ def run_gsa(args, world, rank, local):
         torch.cuda.synchronize()
 
     barrier()
+    if getattr(args, "extra_only", False) and world == 1:
+        if rank == 0:
+            print(json.dumps({"note": "extra workloads only", "workloads": measure_extra(G, W, args, dev, flush, hbm, bf16)}))
+        return None
     main = measure_flat(G, W, cfg, dev, args, flush, rank_seed(cfg, rank), e2e=True, clock_index=local)
     barrier()
     total_ms, total_e2e_ms = max_over_ranks([np.sum(main["step_ms"]), np.sum(main["e2e_ms"])], world, dev)
 
     extra = {}
     if rank == 0 and world == 1 and not args.main_only:
-        for name in [n for n in args.extra.split(",") if n]:
-            c = W.CONFIGS[name]
-            if name.startswith("prefill"):
-                extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)
-            elif c.group:
-                extra[name] = measure_hgsa(G, W, c, dev, args, flush, hbm)
-            else:
-                m = measure_flat(G, W, c, dev, args, flush, c.seed)
-                extra[name] = flat_summary(c, m, hbm)
-                del m
-            torch.cuda.empty_cache()
+        extra = measure_extra(G, W, args, dev, flush, hbm, bf16)
 
     result = None
     if rank == 0:

@@ -85,6 +85,11 @@ __device__ __forceinline__ PfTile pf_tile(const PrefillArgs &a, int t) {
 constexpr int kPsEpiWarps = 8;
 constexpr int kPsThreads = 64 + 32 * kPsEpiWarps;
 constexpr int kPsCap = 48;  // candidate slots per row half
+// TMEM columns: kPsAcc accumulators of 128 (the MMA runs that many key
+// tiles ahead of the epilogue), then the row-end exchange (2 x 16)
+constexpr int kPsAcc = 3;
+constexpr int kPsXchgCol = kPsAcc * kPfKeys;
+static_assert(kPsXchgCol + 32 <= 512, "TMEM columns");
 
 struct PfSmem {
   static constexpr uint32_t kQBlock = kPfRows * 128;         // 128 rows x 64 bf16
@@ -209,11 +214,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PfSmem::kBarOff);
   constexpr int kQS = PfSmem::kQStages, kKS = PfSmem::kKStages;
   uint64_t *q_full = bars, *q_empty = bars + kQS, *k_full = bars + 2 * kQS, *k_empty = k_full + kKS;
-  uint64_t *acc_full = k_empty + kKS, *acc_empty = acc_full + 2;
-  uint64_t *quad_bar = acc_empty + 2;  // [4]: the two epilogue warps of one TMEM quadrant
-  static_assert(2 * kQS + 2 * kKS + 8 <= 16, "barrier block");
-  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 16);
-  int *abort_s = reinterpret_cast<int *>(bars + 17);
+  uint64_t *acc_full = k_empty + kKS, *acc_empty = acc_full + kPsAcc;
+  uint64_t *quad_bar = acc_empty + kPsAcc;  // [4]: the two epilogue warps of one TMEM quadrant
+  static_assert(2 * kQS + 2 * kKS + 2 * kPsAcc + 4 <= 24, "barrier block");
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 24);
+  int *abort_s = reinterpret_cast<int *>(bars + 25);
   uint8_t *cnt_x = smem + PfSmem::kCntOff;                               // [2][128]
   uint8_t *sel_x = smem + PfSmem::kSelOff;                               // [2][128]
 
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPsAcc; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kPsEpiWarps * 32);
     }
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     tc::prefetch_map(&a.tm_qgist);
     tc::prefetch_map(&a.tm_kgist);
   }
-  if (warp == 1) tc::tmem_alloc(tmem_base_s, 512);  // two accumulators + the row-end exchange
+  if (warp == 1) tc::tmem_alloc(tmem_base_s, 512);  // accumulators + the row-end exchange
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -302,8 +307,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         const int qs = qi % kQS;
         if (!wait(&q_full[qs], (qi / kQS) & 1)) break;
         for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki, ++ai) {
-          const int ks = ki % kKS, as = ai & 1;
-          if (!wait(&k_full[ks], (ki / kKS) & 1) || !wait(&acc_empty[as], ((ai >> 1) & 1) ^ 1)) {
+          const int ks = ki % kKS, as = ai % kPsAcc;
+          if (!wait(&k_full[ks], (ki / kKS) & 1) || !wait(&acc_empty[as], ((ai / kPsAcc) & 1) ^ 1)) {
             ok = false;
             break;
           }
@@ -343,8 +348,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     // one accumulator: this thread's 64 scores (columns 32h .. 32h+31 and
     // 64+32h .. 95+32h of the key tile), masked past `limit`, handed to f
     auto take = [&](int j, int limit, auto &&f) -> bool {
-      const int as = ai & 1;
-      if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai >> 1) & 1))) return false;
+      const int as = ai % kPsAcc;
+      if (!__all_sync(0xffffffffu, wait(&acc_full[as], (ai / kPsAcc) & 1))) return false;
       tc::fence_after_sync();
       const bool edge = __any_sync(0xffffffffu, (j + 1) * kPfKeys > limit);
       float v[64];
@@ -434,13 +439,13 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
           ps_merge16(top, x);
         }
       }
-      tc::st16(tmem + lane_addr + 256 + 16 * h, top);
+      tc::st16(tmem + lane_addr + kPsXchgCol + 16 * h, top);
       tc::fence_before_sync();
       if (!pair_sync()) break;
       tc::fence_after_sync();
       {
         float o[16];
-        tc::ld16(tmem + lane_addr + 256 + 16 * (h ^ 1), o);
+        tc::ld16(tmem + lane_addr + kPsXchgCol + 16 * (h ^ 1), o);
         ps_merge16(top, o);
       }
       float T = top[0];
