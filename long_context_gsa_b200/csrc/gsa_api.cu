@@ -406,7 +406,8 @@ gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const
 // Splits per row of the H-GSA candidate pass; depends on the descriptor only
 // (gsa_unfold_attend needs it without the H-GSA parameters).
 int hgsa_splits(const gsa_desc *d) {
-  return one_wave_splits(d->batch * d->hq, 4 * sm_count(), kHgsaSplitMax);
+  // the children kernel's rings take at most 64 KB per CTA: 3 CTAs per SM
+  return one_wave_splits(d->batch * d->hq, 3 * sm_count(), kHgsaSplitMax);
 }
 
 template <int D, typename T>

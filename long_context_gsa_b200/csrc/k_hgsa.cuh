@@ -211,22 +211,39 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
   const int j0 = min(M, split * per_m), j1 = min(M, j0 + per_m);
   const T *mv = reinterpret_cast<const T *>(a.meta_v) + (static_cast<size_t>(b) * a.hkv + kvh) * a.m_max * D;
   const float *ms = a.meta_scores + row * a.m_max;
-  for (int j = j0 + warp * kRpw + slot; j - slot < j1; j += kHgsaWarps * kRpw) {
-    const bool valid = j < j1;
-    bool chosen = false;
-    if (valid) {
-      int lo = 0, hi = n_sel_meta;  // sel_meta ascending
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (sel_meta[mid] < j) lo = mid + 1; else hi = mid;
+  constexpr int kU = 8;                          // meta rows in flight per lane group
+  constexpr int kStride = kHgsaWarps * kRpw;     // rows between a lane group's consecutive rows
+  // a lane group's rows ascend, so one pointer walks the ascending sel_meta
+  int sp = 0;
+  {
+    const int jfirst = j0 + warp * kRpw + slot;
+    int hi = n_sel_meta;
+    while (sp < hi) {
+      const int mid = (sp + hi) >> 1;
+      if (sel_meta[mid] < jfirst) sp = mid + 1; else hi = mid;
+    }
+  }
+  for (int jb = j0 + warp * kRpw + slot; jb - slot < j1; jb += kStride * kU) {
+    uint4 w[kU];
+    float z[kU];
+    bool use[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int j = jb + u * kStride;
+      while (sp < n_sel_meta && sel_meta[sp] < j) ++sp;
+      const bool chosen = sp < n_sel_meta && sel_meta[sp] == j;
+      use[u] = j < j1 && !chosen;
+      // every load of the batch is issued before the first is used
+      w[u] = use[u] ? *reinterpret_cast<const uint4 *>(mv + static_cast<size_t>(j) * D + dd) : make_uint4(0, 0, 0, 0);
+      z[u] = use[u] ? __ldcg(ms + j) * kLog2e : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (use[u]) {
+        float vf[kE];
+        Vec16<T>::unpack(w[u], vf);
+        update(z[u], vf);
       }
-      chosen = lo < n_sel_meta && sel_meta[lo] == j;
-    }
-    if (valid && !chosen) {
-      float vf[kE];
-      Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(mv + static_cast<size_t>(j) * D + dd), vf);
-      update(__ldcg(ms + j) * kLog2e, vf);
-    }
   }
   pdl_trigger();
 
