@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
 #pragma unroll
   for (int i = 0; i < D / 16; ++i) afr[i] = af_sh[i * 32 + lane];
 
+  const uint64_t stream_policy = tc::policy_evict_first();  // every gist row is read once
   auto issue = [&](int t) {
     const int st = t % kStages;
     uint8_t *dst = smem + st * Cfg::kStageBytes;
@@ -183,9 +184,10 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
     mbar_arrive_expect_tx(&bars[st], Cfg::kStageBytes);
 #pragma unroll
     for (int x = 0; x < Cfg::kBoxes; ++x) {
-      tc::tma_load_2d(dst + x * Cfg::kBoxBytes, &a.tm_k, 64 * x, row0 + t * kTile, &bars[st]);
+      tc::tma_load_2d_hint(dst + x * Cfg::kBoxBytes, &a.tm_k, 64 * x, row0 + t * kTile, &bars[st], stream_policy);
       if (WITH_V)
-        tc::tma_load_2d(dst + Cfg::kTileBytes + x * Cfg::kBoxBytes, &a.tm_v, 64 * x, row0 + t * kTile, &bars[st]);
+        tc::tma_load_2d_hint(dst + Cfg::kTileBytes + x * Cfg::kBoxBytes, &a.tm_v, 64 * x, row0 + t * kTile, &bars[st],
+                             stream_policy);
     }
   };
   if (tid == 0)

@@ -293,39 +293,49 @@ constexpr int kTopkCandCap = 1024;  // candidates the bound path ranks in shared
 
 // Top-k through a lower bound (0 < kk < n, kk <= 256):
 //  1. the warps whose 32 lanes all hold entries sort their threads' maximum
-//     keys (shuffles); one warp sorts their top R (R = 16, or 32 for
-//     kk > 64) and takes the kk-th largest, L: kk distinct entries reach L,
-//     so it bounds the row's kk-th score key from below;
+//     keys (shuffles); one warp sorts their top R (16, or 32 when fewer
+//     than 2 kk maxima would be sorted) and takes the kk-th largest, L: kk
+//     distinct entries reach L, so it bounds the row's kk-th score key from
+//     below;
 //  2. every entry with key >= L is a candidate (in practice under 1.2 kk);
 //  3. the candidate of rank kk - 1 among the candidates, by (score desc,
-//     index asc), is the row's kk-th rank key: one warp sorts up to 128
-//     candidates, more are ranked by counting (each against all);
+//     index asc), is the row's kk-th rank key: up to 256 candidates are
+//     sorted by two warps (128 each) and the kk-th of the two lists found by
+//     a binary search; more are ranked by counting (each against all);
 //  4. the entries reaching that key (exactly kk: rank keys are distinct)
 //     are written in ascending chunk order straight from the registers.
 // Returns false (nothing written) when no bound can be taken or the
 // candidates exceed the buffer; the caller then runs the radix select.
 // Called by the whole block.
 template <int KPT>
-__device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n, int kk, const uint32_t (&key)[KPT],
-                                              int base, BoundSmem &sm) {
+__device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n, int kk, const float *rs, int base,
+                                              BoundSmem &sm) {
   constexpr int T = kTopkRegThreads, W = T / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t m = 0u;  // valid keys are nonzero; 0 marks "no entry"
-#pragma unroll
-  for (int j = 0; j < KPT; ++j)
-    if (base + 32 * j < n) m = max(m, key[j]);
+  // The loops over this thread's KPT entries (element base + 32 j of the
+  // staged row) are only partly unrolled: each phase runs once per block,
+  // so its instructions are fetched cold whenever an earlier kernel has
+  // streamed through L2, and a fully unrolled body costs more in fetch
+  // stalls than the loop does in issue.
+  auto key_at = [&](int j) -> uint32_t {
+    const int i = base + 32 * j;
+    return i < n ? float_to_key(rs[i]) : 0u;  // valid keys are nonzero; 0 marks "no entry"
+  };
+  uint32_t m = 0u;
+#pragma unroll 4
+  for (int j = 0; j < KPT; ++j) m = max(m, key_at(j));
   {
     uint32_t v[1] = {m};
     warp_sort_desc<1>(v, lane);
     m = v[0];
   }
   const int w_full = n >= 32 ? min(W, (n - 32) / (32 * KPT) + 1) : 0;  // warps w with w*32*KPT + 31 < n
-  const int R = kk > 64 ? 32 : 16;
-  if (w_full * R < kk) return false;  // block-uniform
+  const int R = w_full * 16 >= 2 * kk ? 16 : 32;  // sort at least 2 kk maxima when there are enough
+  if (w_full * R < kk) return false;              // block-uniform
   if (lane < R) sm.wtop[warp * R + lane] = warp < w_full ? m : 0u;
   if (tid == 0) sm.count = 0;
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0) {  // one warp sorts them
     if (R == 16) {
       uint32_t v[4];
 #pragma unroll
@@ -349,31 +359,48 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
   // gather the candidates: one shared atomic per warp
   const unsigned lt = (1u << lane) - 1u;
   int w_cnt = 0;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) w_cnt += __popc(__ballot_sync(0xffffffffu, base + 32 * j < n && key[j] >= L));
+#pragma unroll 4
+  for (int j = 0; j < KPT; ++j) w_cnt += __popc(__ballot_sync(0xffffffffu, key_at(j) >= L));
   int w_base = 0;
   if (lane == 0 && w_cnt) w_base = atomicAdd(&sm.count, w_cnt);
   w_base = __shfl_sync(0xffffffffu, w_base, 0);
-#pragma unroll
+#pragma unroll 4
   for (int j = 0; j < KPT; ++j) {
-    const bool c = base + 32 * j < n && key[j] >= L;
+    const uint32_t kj = key_at(j);
+    const bool c = kj >= L;
     const unsigned bal = __ballot_sync(0xffffffffu, c);
     const int slot = w_base + __popc(bal & lt);
-    if (c && slot < kTopkCandCap) sm.cand[slot] = rank_key(key[j], base + 32 * j);
+    if (c && slot < kTopkCandCap) sm.cand[slot] = rank_key(kj, base + 32 * j);
     w_base += __popc(bal);
   }
   __syncthreads();
   const int C = sm.count;
   if (C > kTopkCandCap) return false;  // block-uniform
-  if (C <= 128) {  // one warp sorts the candidates
-    if (warp == 0) {
+  if (C <= 256) {  // warps 0 and 1 sort 128 candidates each; the kk-th of the two lists
+    if (warp < 2 && 128 * warp < C) {
       unsigned long long v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = lane * 4 + e < C ? sm.cand[lane * 4 + e] : 0ull;
+      for (int e = 0; e < 4; ++e) {
+        const int i = 128 * warp + lane * 4 + e;
+        v[e] = i < C ? sm.cand[i] : 0ull;
+      }
       warp_sort_desc<4>(v, lane);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (lane * 4 + e == kk - 1) sm.kth = v[e];
+      for (int e = 0; e < 4; ++e) sm.cand[128 * warp + lane * 4 + e] = v[e];
+    }
+    __syncthreads();
+    if (tid == 0) {  // i entries from the first list and kk - i from the second (keys are distinct)
+      const unsigned long long *A = sm.cand, *Bl = sm.cand + 128;
+      const int nA = min(C, 128), nB = C - nA;
+      int lo = max(0, kk - nB), hi = min(kk, nA);
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (A[mid] > Bl[kk - mid - 1]) lo = mid + 1;
+        else hi = mid;
+      }
+      const int j = kk - lo;
+      const unsigned long long a_last = lo > 0 ? A[lo - 1] : ~0ull, b_last = j > 0 ? Bl[j - 1] : ~0ull;
+      sm.kth = min(a_last, b_last);
     }
   } else {  // each candidate's rank is counted against all
     for (int t = tid; t < C; t += T) {
@@ -390,11 +417,13 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
     }
   }
   __syncthreads();
-  const unsigned long long kth = sm.kth;
+  // selected: key > the k-th's, or equal with an index at or below its index
+  const uint32_t kth_key = static_cast<uint32_t>(sm.kth >> 32);
+  const int kth_idx = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(sm.kth));
+  auto selected = [&](uint32_t kj, int idx) { return kj > kth_key || (kj == kth_key && idx <= kth_idx); };
   int w_sel = 0;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j)
-    w_sel += __popc(__ballot_sync(0xffffffffu, base + 32 * j < n && key[j] >= L && rank_key(key[j], base + 32 * j) >= kth));
+#pragma unroll 4
+  for (int j = 0; j < KPT; ++j) w_sel += __popc(__ballot_sync(0xffffffffu, selected(key_at(j), base + 32 * j)));
   if (lane == 0) sm.wcnt[warp] = w_sel;
   __syncthreads();
   int pos = 0;
@@ -402,15 +431,16 @@ __device__ __forceinline__ bool topk_by_bound(const TopkArgs &a, int row, int n,
   pdl_trigger();
   int32_t *out_i = a.sel_idx + static_cast<size_t>(row) * a.k;
   float *out_s = a.sel_score ? a.sel_score + static_cast<size_t>(row) * a.k : nullptr;
-#pragma unroll
+#pragma unroll 4
   for (int j = 0; j < KPT; ++j) {
     const int idx = base + 32 * j;
-    const bool c = idx < n && key[j] >= L && rank_key(key[j], idx) >= kth;
+    const uint32_t kj = key_at(j);
+    const bool c = selected(kj, idx);
     const unsigned bal = __ballot_sync(0xffffffffu, c);
     if (c) {
       const int o = pos + __popc(bal & lt);
       out_i[o] = a.id_map ? a.id_map[static_cast<size_t>(row) * a.stride + idx] : idx;
-      if (out_s) out_s[o] = key_to_float(key[j]);
+      if (out_s) out_s[o] = key_to_float(kj);
     }
     pos += __popc(bal);
   }
@@ -455,15 +485,18 @@ __global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : 1) k_topk(con
     if (n4 > 0) bulk_g2s(srow_s, srow, static_cast<uint32_t>(n4) * 4u, &load_bar);
   }
   const int staged = mbar_wait(&load_bar, 0) ? n4 : 0;
+  for (int i = staged + tid; i < n; i += T) srow_s[i] = __ldcg(srow + i);  // the tail (and a timed-out copy)
+  __syncthreads();
+
+  const int kk = min(a.k, n);
+  if (kk > 0 && kk < n && kk <= T && topk_by_bound<KPT>(a, row, n, kk, srow_s, base, bsm)) return;
   uint32_t key[KPT];
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
     const int i = base + 32 * j;
-    key[j] = i < staged ? float_to_key(srow_s[i]) : (i < n ? float_to_key(__ldcg(srow + i)) : 0u);
+    key[j] = i < n ? float_to_key(srow_s[i]) : 0u;
   }
 
-  const int kk = min(a.k, n);
-  if (kk > 0 && kk < n && kk <= T && topk_by_bound<KPT>(a, row, n, kk, key, base, bsm)) return;
   uint32_t prefix = 0, pmask = 0;
   int rem = kk;
   bool all_eq = kk == n;
