@@ -541,6 +541,8 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.scale = pa.scale;
   sr.sel_idx = sel_idx;
   sr.sel_score = sel_score;
+  sr.rec_raw = pa.rec_raw;
+  sr.scale_log2 = pa.scale_log2;
   return launch(k_prefill_select_rows, dim3(sm_count()), dim3(256),
                 (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4, stream, sr);
 }

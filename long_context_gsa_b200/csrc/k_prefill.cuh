@@ -192,14 +192,18 @@ __device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16])
 
 // Stage 1, k_prefill_score: row maxima and the top-k selection (k <= 16)
 // of every query row, in two passes over the visible key tiles of a query
-// tile (the key tiles stream twice through a 3-stage ring; Q stays in
-// shared memory):
-//  A. each thread keeps 16 slot maxima over its half of the columns
-//     (slot = column mod 16); the 16 largest of the row's 32 slot maxima
-//     are distinct scores, so the k-th largest of them bounds the row's
-//     k-th score from below;
-//  B. every score >= that bound is appended as a (score, index) candidate
-//     (about k + 5 per row) by predicated stores, in ascending index order;
+// tile (the key tiles stream through a 3-stage ring; Q stays in shared
+// memory):
+//  A. over every other key tile (0, 2, 4, ...), each thread keeps 16 slot
+//     maxima over its half of the columns (slot = column mod 16); the 16
+//     largest of the row's 32 slot maxima are distinct scores, so the k-th
+//     largest of them bounds the row's k-th score from below (sampling half
+//     the tiles loosens the bound, doubling the candidates, and halves the
+//     pass's tensor work);
+//  B. over all key tiles, every score >= that bound is appended as a
+//     (score, index) candidate (about 2k + 10 per row) by predicated
+//     stores, in ascending index order; the largest candidate is the row
+//     maximum;
 //     at the row end each half sorts its 16 largest candidate values, the
 //     halves exchange them through TMEM and merge them into the row's k-th
 //     candidate score T, keep (compact) their entries >= T, and write the
@@ -261,7 +265,17 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     return false;
   };
   // key-tile passes of a query tile: raw rows with a selection take two
-  auto passes = [&](const PfTile &tl) { return (!tl.is_gist && raw_topk) ? 2 : 1; };
+  // Key tiles of a query tile, in MMA order.  Rows with a selection take
+  // pass A over every other key tile (0, 2, 4, ...; the bound it gives
+  // stays exact, only looser) and then pass B over all of them; other rows
+  // take pass A over all key tiles (their exact row maximum).
+  auto n_pass_a = [&](const PfTile &tl) { return (!tl.is_gist && raw_topk) ? (tl.n_kt + 1) / 2 : tl.n_kt; };
+  auto n_steps = [&](const PfTile &tl) { return n_pass_a(tl) + ((!tl.is_gist && raw_topk) ? tl.n_kt : 0); };
+  auto step_tile = [&](const PfTile &tl, int jj) {
+    const bool sel = !tl.is_gist && raw_topk;
+    const int na = n_pass_a(tl);
+    return jj < na ? (sel ? 2 * jj : jj) : jj - na;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -280,8 +294,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         tc::tma_load_2d(qdst, qm, 0, qrow, &q_full[qs]);
         tc::tma_load_2d(qdst + PfSmem::kQBlock, qm, 64, qrow, &q_full[qs]);
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
-        for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki) {
-          const int j = jj % tl.n_kt, ks = ki % kKS;
+        for (int jj = 0; jj < n_steps(tl); ++jj, ++ki) {
+          const int j = step_tile(tl, jj), ks = ki % kKS;
           if (!wait(&k_empty[ks], ((ki / kKS) & 1) ^ 1)) {
             ok = false;
             break;
@@ -306,7 +320,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         if (tl.n_kt == 0) continue;
         const int qs = qi % kQS;
         if (!wait(&q_full[qs], (qi / kQS) & 1)) break;
-        for (int jj = 0; jj < passes(tl) * tl.n_kt; ++jj, ++ki, ++ai) {
+        for (int jj = 0; jj < n_steps(tl); ++jj, ++ki, ++ai) {
           const int ks = ki % kKS, as = ai % kPsAcc;
           if (!wait(&k_full[ks], (ki / kKS) & 1) || !wait(&acc_empty[as], ((ai / kPsAcc) & 1) ^ 1)) {
             ok = false;
@@ -377,8 +391,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       float G[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) G[q] = neg_inf();
-      for (int j = 0; j < tl.n_kt && ok; ++j)
-        ok = take(j, limit, [&](const float(&v)[64], int) {
+      for (int jj = 0; jj < n_pass_a(tl) && ok; ++jj)
+        ok = take(step_tile(tl, jj), limit, [&](const float(&v)[64], int) {
 #pragma unroll
           for (int e = 0; e < 64; ++e) G[e & 15] = fmaxf(G[e & 15], v[e]);
         });
@@ -409,8 +423,10 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       if (!pair_sync()) break;  // the slot maxima area becomes the candidate columns
       const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
       float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
-      if (h == 0 && row_ok) rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
-      if (!sel_rows) continue;
+      if (!sel_rows) {  // pass A saw every key tile: its maximum is the row's
+        if (h == 0 && row_ok) rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
+        continue;
+      }
       // ---- pass B: candidates >= bound ----
       uint32_t cnt = 0;
       for (int j = 0; j < tl.n_kt && ok; ++j)
@@ -452,6 +468,9 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
 #pragma unroll
       for (int q = 1; q < 16; ++q)
         if (q < ksel) T = top[q];
+      // the row maximum: the largest candidate (every score at or above the
+      // bound is one); a listed row gets it from the exact per-row pass
+      if (h == 0 && row_ok) rec[0] = top[0] == neg_inf() ? top[0] : top[0] * a.scale_log2;
       ovf |= cnt_x[(h ^ 1) * kPfRows + r] == 255;
       // this half's entries >= T, compacted in order to the column's front
       uint32_t w = base;
@@ -548,6 +567,8 @@ struct SelectRowsArgs {
   float scale;
   int32_t *sel_idx;
   float *sel_score;
+  float *rec_raw;     // [rows, 128 + 4]: [0] gets the row maximum (base 2)
+  float scale_log2;
 };
 
 __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArgs a) {
@@ -622,6 +643,9 @@ __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArg
       }
       __syncthreads();
     }
+    // the first pick is the row maximum
+    if (tid == 0)
+      a.rec_raw[static_cast<size_t>(orow) * (128 + kPartHeader)] = ksel > 0 ? qs[128] * a.scale_log2 : neg_inf();
     // ascending chunk order: a pick's slot is the number of picks below it
     int32_t *oi = a.sel_idx + static_cast<size_t>(orow) * a.topk;
     float *os = a.sel_score + static_cast<size_t>(orow) * a.topk;
