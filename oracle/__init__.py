@@ -114,6 +114,9 @@ class Oracle:
         self.lib.gsa_oracle_default_threads.restype = C.c_int
         self.lib.gsa_oracle_topk.argtypes = [_dp, _ip, C.c_int64, C.c_int32, C.c_int32, _ip, _dp]
         self.lib.gsa_oracle_topk.restype = C.c_int
+        self.lib.gsa_oracle_topp.argtypes = [_dp, _ip, C.c_int64, C.c_int32, C.c_int32, C.c_double, _ip, _dp, _ip,
+                                             _dp, _dp]
+        self.lib.gsa_oracle_topp.restype = C.c_int
 
     def default_threads(self) -> int:
         return int(self.lib.gsa_oracle_default_threads())
@@ -154,6 +157,22 @@ class Oracle:
         ssc = np.zeros((rows, k))
         _ok(self.lib.gsa_oracle_topk(s.ctypes.data_as(_dp), _ip_(n), rows, stride, k, _ip_(sel), _dp_(ssc)), "topk")
         return sel, ssc
+
+    def topp(self, scores, n_valid, k, top_p):
+        """Top-p (nucleus) selection on given scores [rows, stride]: the shortest
+        rank-order prefix with softmax mass >= top_p, 1..k entries.  Returns
+        dict(sel, sel_score, count, mass_lo, mass_hi)."""
+        s = np.ascontiguousarray(scores, dtype=np.float64)
+        rows, stride = s.shape
+        n = _i32(n_valid)
+        if n.shape != (rows,):
+            raise ValueError("n_valid shape")
+        res = {"sel": np.full((rows, k), -1, np.int32), "sel_score": np.zeros((rows, k)),
+               "count": np.zeros(rows, np.int32), "mass_lo": np.zeros(rows), "mass_hi": np.zeros(rows)}
+        _ok(self.lib.gsa_oracle_topp(s.ctypes.data_as(_dp), _ip_(n), rows, stride, k, float(top_p), _ip_(res["sel"]),
+                                     _dp_(res["sel_score"]), _ip_(res["count"]), _dp_(res["mass_lo"]),
+                                     _dp_(res["mass_hi"])), "topp")
+        return res
 
     # -------------------------------------------------------------------- hgsa
     def hgsa(self, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, *, chunk, group,

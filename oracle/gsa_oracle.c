@@ -157,6 +157,12 @@ static int cmp_rank(const void *x, const void *y) {
   return (a->m < b->m) ? -1 : (a->m > b->m);
 }
 
+/* Index order (ascending), for writing a selection out. */
+static int cmp_index(const void *x, const void *y) {
+  const scored_t *a = (const scored_t *)x, *b = (const scored_t *)y;
+  return (a->m > b->m) - (a->m < b->m);
+}
+
 /* ------------------------------------------------------------------------ */
 /* The attended set and exact softmax attention over it.                    */
 /* ------------------------------------------------------------------------ */
@@ -292,6 +298,63 @@ int gsa_oracle_topk(const double *scores, const int32_t *n_valid, int64_t rows, 
       }
       out[j] = cand[i].m;
       if (outs) outs[j] = cand[i].s;
+    }
+  }
+  free(cand);
+  return ORC_OK;
+}
+
+/* Top-p (nucleus) selection on given scores, the variant the pages compare
+ * with top-k ([ja] section 4, "Top-k vs Top-p"; [nl] "Stabiliteit": a fixed
+ * probability threshold instead of a fixed chunk budget).  For each row the
+ * chunk probabilities are the softmax of scores[row][0 .. n_valid), and the
+ * selection is the shortest prefix of the ranking above (score desc, index
+ * asc) whose probability mass reaches top_p, at least one chunk when
+ * n_valid >= 1 and at most k.  Output as for gsa_oracle_topk, plus the count
+ * per row in sel_count and the prefix masses before and at the last chosen
+ * entry in mass_lo / mass_hi (NULL allowed), which bound how far top_p is
+ * from a boundary. */
+int gsa_oracle_topp(const double *scores, const int32_t *n_valid, int64_t rows, int32_t stride, int32_t k,
+                    double top_p, int32_t *sel_idx, double *sel_score, int32_t *sel_count, double *mass_lo,
+                    double *mass_hi) {
+  if (rows < 0 || stride < 0 || k < 0) return ORC_EINVAL;
+  scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)(stride > 0 ? stride : 1));
+  if (!cand) return ORC_ENOMEM;
+  for (int64_t r = 0; r < rows; ++r) {
+    const int32_t n = n_valid[r];
+    if (n < 0 || n > stride) {
+      free(cand);
+      return ORC_EINVAL;
+    }
+    for (int32_t m = 0; m < n; ++m) {
+      cand[m].s = scores[r * stride + m];
+      cand[m].m = m;
+    }
+    qsort(cand, (size_t)n, sizeof(scored_t), cmp_rank);
+    double z = 0.0;
+    for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s - cand[0].s);
+    int32_t ns = 0;
+    double before = 0.0, mass = 0.0;
+    while (ns < n && ns < k) {
+      before = mass;
+      mass += exp(cand[ns].s - cand[0].s) / z;
+      ++ns;
+      if (mass >= top_p) break;
+    }
+    if (sel_count) sel_count[r] = ns;
+    if (mass_lo) mass_lo[r] = before;
+    if (mass_hi) mass_hi[r] = mass;
+    int32_t *out = sel_idx + r * k;
+    double *outs = sel_score ? sel_score + r * k : NULL;
+    for (int32_t i = 0; i < k; ++i) {
+      out[i] = -1;
+      if (outs) outs[i] = -INFINITY;
+    }
+    /* ascending index order: the chosen entries sorted by index */
+    qsort(cand, (size_t)ns, sizeof(scored_t), cmp_index);
+    for (int32_t i = 0; i < ns; ++i) {
+      out[i] = cand[i].m;
+      if (outs) outs[i] = cand[i].s;
     }
   }
   free(cand);

@@ -503,9 +503,52 @@ def pin_topk_selection(orc):
     assert [int(x) for x in sel[0]] == [0, 1, 2, 3]  # all equal: the lowest indices
 
 
+def pin_topp_selection(orc):
+    """Top-p against closed forms: uniform scores need ceil(p*n) chunks (the
+    lowest indices); scores -i*ln2 give masses 2^-i, so the count has a closed
+    form; p >= 1 keeps min(k, n); a dominant chunk alone covers p below its
+    mass; a constant shift of the scores changes nothing; the set is always
+    the rank-order prefix of that length (the top-k set of the same size)."""
+    rng = np.random.default_rng(9)
+    # uniform: p = 0.5 of n = 4 is exactly two chunks (masses 1/4 are exact)
+    r = orc.topp(np.zeros((1, 4)), [4], 4, 0.5)
+    assert r["count"][0] == 2 and [int(x) for x in r["sel"][0][:2]] == [0, 1]
+    for n, pp in ((10, 0.35), (64, 0.26), (7, 0.99)):
+        r = orc.topp(np.zeros((1, n)), [n], n, pp)
+        want = math.ceil(pp * n)
+        assert r["count"][0] == want and [int(x) for x in r["sel"][0][:want]] == list(range(want)), (n, pp, r["count"])
+    # geometric: mass of the first m chunks = (1 - 2^-m) / (1 - 2^-n)
+    n = 20
+    sc = -np.arange(n) * math.log(2.0)
+    perm = rng.permutation(n)
+    for pp in (0.3, 0.6, 0.9, 0.999):
+        want = next(m for m in range(1, n + 1) if (1 - 2.0 ** -m) / (1 - 2.0 ** -n) >= pp)
+        r = orc.topp(sc[perm][None, :], [n], n, pp)
+        assert r["count"][0] == want, (pp, r["count"][0], want)
+        assert sorted(int(x) for x in r["sel"][0][:want]) == sorted(int(np.where(perm == i)[0][0]) for i in range(want))
+        assert r["mass_lo"][0] < pp <= r["mass_hi"][0]
+    # p >= 1, the cap k, and a dominant chunk
+    r = orc.topp(rng.standard_normal((2, 30)), [30, 12], 16, 1.0)
+    assert list(r["count"]) == [16, 12]
+    sc = rng.standard_normal((1, 50))
+    sc[0, 17] = 40.0
+    r = orc.topp(sc, [50], 8, 0.9)
+    assert r["count"][0] == 1 and r["sel"][0][0] == 17
+    # shift invariance (also keeps large scores finite) and the prefix property
+    sc = rng.standard_normal((3, 200)) * 3
+    a = orc.topp(sc, [200, 150, 1], 64, 0.7)
+    b = orc.topp(sc + 1000.0, [200, 150, 1], 64, 0.7)
+    assert np.array_equal(a["sel"], b["sel"]) and np.array_equal(a["count"], b["count"])
+    assert a["count"][2] == 1
+    for r_ in range(2):
+        c = int(a["count"][r_])
+        t, _ = orc.topk(sc[r_:r_ + 1], [[200, 150][r_]], c)
+        assert [int(x) for x in a["sel"][r_][:c]] == [int(x) for x in t[0]]
+
+
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
                pin_decode_golden]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]
-ALL_PINS = [pin_topk_selection] + DECODE_PINS + HGSA_PINS + PREFILL_PINS
+ALL_PINS = [pin_topk_selection, pin_topp_selection] + DECODE_PINS + HGSA_PINS + PREFILL_PINS

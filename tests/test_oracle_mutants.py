@@ -39,6 +39,10 @@ MUTANTS = [
     ("prefill_gist_query_excludes_itself", "for (int32_t t = 0; t <= m && !st; ++t)", "for (int32_t t = 0; t < m && !st; ++t)"),
     ("prefill_chunk_of_position_off_by_one", "const int32_t m = (int32_t)(pos / c), j = (int32_t)(pos % c);",
      "const int32_t m = (int32_t)((pos + 1) / c), j = (int32_t)((pos + 1) % c);"),
+    ("topp_output_descending", "return (a->m > b->m) - (a->m < b->m);", "return (a->m < b->m) - (a->m > b->m);"),
+    ("topp_strict_mass_test", "if (mass >= top_p) break;", "if (mass > top_p) break;"),
+    ("topp_unshifted_exponent", "for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s - cand[0].s);",
+     "for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s);"),
     ("topk_output_in_rank_order", "while (j > 0 && out[j - 1] > cand[i].m) {", "while (0) {"),
     ("prefill_ignores_exclude", "} else if (!a->exclude) {\n        st = push(&S, a->k_gist", "} else {\n        st = push(&S, a->k_gist"),
 ]
