@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,prefill_32k",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,prefill_32k,llama1b_8x_topp",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
@@ -381,6 +381,49 @@ def measure_prefill(G, W, cfg, dev, args, flush, bf16_peak):
             "tensor_frac": round(tf / bf16_peak, 4), "steps": steps}
 
 
+def measure_topp(G, W, cfg, dev, args, flush, hbm, top_p):
+    """A decode step with top-p selection (score -> top-p -> unfold): the
+    selection is variable-length, so the step's bytes follow the actual
+    union of chosen chunks."""
+    x, desc = decode_setup(G, W, cfg, dev, cfg.seed)
+    B, hq, d = x["q"].shape
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+    cnt = torch.empty((B, hq), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, hq, x["gist_k"].shape[2]), dtype=torch.float32, device=dev)
+
+    def step(evs):
+        evs[0].record()
+        G.gsa_score_gists(desc, x["q"], x["gist_k"], x["gist_v"], x["n_gists"], scores, ws)
+        evs[1].record()
+        G.gsa_topp_select(desc, scores, x["n_gists"], top_p, sel, ssc, cnt, ws)
+        evs[2].record()
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
+                            G.GSA_PRIOR_GISTS, out, None, ws)
+        evs[3].record()
+
+    for _ in range(args.warmup):
+        flush()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    k = timed_steps(step, args.steps, flush, 3)
+    assert G.gsa_workspace_status(ws) == 0, "device status flags set"
+    ms = float(k.sum(1).mean())
+    ab = algorithmic_bytes(cfg, x, sel)
+    c = cnt.float()
+    return {"metric": "GSA decode head-queries/s", "value": round(cfg.head_queries / (ms / 1e3), 1), "unit": UNIT,
+            "top_p": top_p, "ms_per_step": round(ms, 5),
+            "chunks_selected": {"mean": round(float(c.mean()), 2), "min": int(c.min()), "max": int(c.max()),
+                                "cap": cfg.topk},
+            "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(ab["total"] / (ms / 1e3) / 1e9, 1),
+                         "frac": round(ab["total"] / (ms / 1e3) / 1e9 / hbm, 4)},
+            "kernels_us": {"score_gists": round(float(k[:, 0].mean()) * 1e3, 2),
+                           "topp_select": round(float(k[:, 1].mean()) * 1e3, 2),
+                           "unfold_attend": round(float(k[:, 2].mean()) * 1e3, 2)}}
+
+
 def rank_seed(cfg, rank):
     """Each rank draws its own batch of the workload (weak scaling: disjoint
     rows, no data-path exchange)."""
@@ -404,6 +447,12 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
     """The --extra workloads, each against its own roofline (rank 0, one GPU)."""
     extra = {}
     for name in [n for n in args.extra.split(",") if n]:
+        if name.endswith("_topp"):  # <decode workload>_topp: the same step with top-p selection, p = 0.1
+            # (the softmax over thousands of gists is flat: p = 0.1 keeps from a few chunks up to the cap)
+            c = W.CONFIGS[name[:-len("_topp")]]
+            extra[name] = measure_topp(G, W, c, dev, args, flush, hbm, 0.1)
+            torch.cuda.empty_cache()
+            continue
         c = W.CONFIGS[name]
         if name.startswith("prefill"):
             extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)

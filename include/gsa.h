@@ -152,6 +152,24 @@ gsa_status gsa_score_gists(const gsa_desc *desc, const void *q, const void *gist
 gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, int32_t *sel_idx,
                            float *sel_score, void *ws, size_t ws_bytes, void *stream);
 
+/* Step 2, top-p variant: the probability-threshold selection the pages
+ * compare with top-k ([ja] section 4 "Top-k vs Top-p"; [nl] Stabiliteit).
+ * The chunk probabilities of row (b,h) are the softmax of its first
+ * n_gists[b] scores; the selection is the shortest prefix of the ranking
+ * (score desc, ties to the lower chunk index) whose probability mass reaches
+ * top_p -- at least one chunk (when n_gists[b] >= 1) and at most topk.
+ *   scores    [B, hq, n_max] fp32 (as gsa_score_gists writes them)
+ *   sel_idx   [B, hq, topk] int32 out, ascending chunk order, -1 padded;
+ *   sel_score [B, hq, topk] fp32 out (may be NULL), -inf padded;
+ *   sel_count [B, hq] int32 out (may be NULL): chunks selected per row.
+ * topk must be 1..256 and n_max <= 16384 (GSA_ERR_UNSUPPORTED otherwise);
+ * a NaN top_p is GSA_ERR_INVALID_ARG; top_p >= 1 keeps min(topk, N).  The
+ * output feeds gsa_unfold_attend like gsa_topk_select's, and the per-row
+ * counters in ws are re-armed the same way. */
+gsa_status gsa_topp_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, float top_p,
+                           int32_t *sel_idx, float *sel_score, int32_t *sel_count, void *ws, size_t ws_bytes,
+                           void *stream);
+
 /* Step 3, selective unfolding + exact attention ([nl] Selectieve
  * Ontvouwing; [ja] 2.1 steps 3-4).
  *   raw_k, raw_v  [B, hkv, t_max, d]  chunk m occupies rows m*chunk ..

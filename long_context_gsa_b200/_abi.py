@@ -24,8 +24,8 @@ GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
-    "gsa_score_gists", "gsa_topk_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select", "hgsa_decode",
-    "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill", "gsa_decode_noalloc",
+    "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
+    "hgsa_decode", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill", "gsa_decode_noalloc",
 )
 
 
@@ -69,6 +69,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_workspace_status": ([vp, sz, vp, C.POINTER(C.c_uint32)], i32),
         "gsa_score_gists": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_topk_select": ([D, vp, vp, vp, vp, vp, sz, vp], i32),
+        "gsa_topp_select": ([D, vp, vp, C.c_float, vp, vp, vp, vp, sz, vp], i32),
         "gsa_unfold_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
         "gsa_decode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "hgsa_select": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
@@ -175,6 +176,15 @@ def gsa_topk_select(desc, scores, n_gists, sel_idx, sel_score, ws, stream=None):
     _check("gsa_topk_select", load().gsa_topk_select(
         C.byref(desc), _ptr(scores, torch.float32, "scores"), _ptr(n_gists, torch.int32, "n_gists"),
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
+        _stream(stream)))
+
+
+def gsa_topp_select(desc, scores, n_gists, top_p, sel_idx, sel_score, sel_count, ws, stream=None):
+    p, n = _ws(ws)
+    _check("gsa_topp_select", load().gsa_topp_select(
+        C.byref(desc), _ptr(scores, torch.float32, "scores"), _ptr(n_gists, torch.int32, "n_gists"),
+        C.c_float(float(top_p)), _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_score, torch.float32, "sel_score", True), _ptr(sel_count, torch.int32, "sel_count", True), p, n,
         _stream(stream)))
 
 

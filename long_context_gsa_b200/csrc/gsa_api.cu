@@ -17,6 +17,7 @@
 #include "k_prefill.cuh"
 #include "k_score.cuh"
 #include "k_topk.cuh"
+#include "k_topp.cuh"
 #include "k_unfold.cuh"
 
 namespace gsa {
@@ -666,6 +667,42 @@ gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int3
   if (desc->topk == 0) return GSA_OK;
   return run_topk(desc->batch * desc->hq, desc->hq, scores, desc->n_max, n_gists, 1, nullptr, desc->topk, nullptr,
                   sel_idx, sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+}
+
+gsa_status gsa_topp_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, float top_p,
+                           int32_t *sel_idx, float *sel_score, int32_t *sel_count, void *ws, size_t ws_bytes,
+                           void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(need_ptr(scores));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(opt_ptr(sel_count));
+  GSA_TRY(need_ptr(ws));
+  if (!(top_p == top_p)) return GSA_ERR_INVALID_ARG;  // NaN
+  if (desc->topk < 1) return GSA_ERR_INVALID_ARG;
+  if (desc->topk > kToppMaxK || desc->n_max > 64 * kTopkRegThreads) return GSA_ERR_UNSUPPORTED;
+  const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  ToppArgs ta;
+  ta.scores = scores;
+  ta.stride = desc->n_max;
+  ta.n_gists = n_gists;
+  ta.hq = desc->hq;
+  ta.k = desc->topk;
+  ta.top_p = top_p;
+  ta.sel_idx = sel_idx;
+  ta.sel_score = sel_score;
+  ta.sel_count = sel_count;
+  ta.counters = reinterpret_cast<uint32_t *>(at(ws, L.counters));
+  const dim3 grid(desc->batch * desc->hq), block(kTopkRegThreads);
+  // the staged row, then one bit per entry for the exact tie path
+  auto smem = [](int kpt) { return static_cast<size_t>(kpt) * kTopkRegThreads * 4 + kpt * kTopkRegThreads / 8; };
+  const int stride = desc->n_max;
+  if (stride <= 4 * kTopkRegThreads) return launch(k_topp<4>, grid, block, smem(4), stream, ta);
+  if (stride <= 16 * kTopkRegThreads) return launch(k_topp<16>, grid, block, smem(16), stream, ta);
+  if (stride <= 32 * kTopkRegThreads) return launch(k_topp<32>, grid, block, smem(32), stream, ta);
+  return launch(k_topp<64>, grid, block, smem(64), stream, ta);
 }
 
 gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *raw_k, const void *raw_v,
