@@ -71,6 +71,22 @@ class _HgsaArgs(C.Structure):
     ]
 
 
+class _Hgsa2Args(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
+        ("n_max", C.c_int32), ("t_max", C.c_int32), ("m1_max", C.c_int32), ("m2_max", C.c_int32),
+        ("group1", C.c_int32), ("group2", C.c_int32), ("topk2", C.c_int32), ("topk1", C.c_int32),
+        ("topk", C.c_int32), ("exclude", C.c_int32), ("dtype", C.c_int32), ("scale", C.c_double),
+        ("q", _vp), ("meta2_k", _vp), ("meta2_v", _vp), ("meta_k", _vp), ("meta_v", _vp), ("gist_k", _vp),
+        ("gist_v", _vp), ("raw_k", _vp), ("raw_v", _vp), ("n_gists", _ip), ("own_len", _ip),
+        ("n_rows", C.c_int32), ("rows", _ip), ("meta2_sel_in", _ip), ("meta_sel_in", _ip), ("sel_in", _ip),
+        ("out", _dp), ("lse", _dp), ("meta2_sel_out", _ip), ("meta_sel_out", _ip), ("sel_out", _ip),
+        ("meta2_scores", _dp), ("meta_cand_scores", _dp), ("cand_scores", _dp),
+        ("set_cap", C.c_int32), ("set_n", _ip), ("set_kind", _ip), ("set_idx", _ip), ("set_w", _dp),
+        ("n_threads", C.c_int32),
+    ]
+
+
 class _PrefillArgs(C.Structure):
     _fields_ = [
         ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
@@ -107,6 +123,7 @@ class Oracle:
         self.path = path
         self.lib = C.CDLL(str(path))
         for name, argt in (("gsa_oracle_decode", _DecodeArgs), ("gsa_oracle_hgsa", _HgsaArgs),
+                           ("gsa_oracle_hgsa2", _Hgsa2Args),
                            ("gsa_oracle_prefill", _PrefillArgs)):
             fn = getattr(self.lib, name)
             fn.argtypes = [C.POINTER(argt)]
@@ -204,6 +221,43 @@ class Oracle:
                       _ip_(res.get("set_n")), _ip_(res.get("set_kind")), _ip_(res.get("set_idx")),
                       _dp_(res.get("set_w")), n_threads)
         _ok(self.lib.gsa_oracle_hgsa(C.byref(a)), "hgsa")
+        return res
+
+    def hgsa2(self, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, *,
+              chunk, group1, group2, topk2, topk1, topk, exclude=False, scale=0.0, rows=None, meta2_sel_in=None,
+              meta_sel_in=None, sel_in=None, want_scores=False, set_cap=0, n_threads=0):
+        """H-GSA decode with two meta levels for the given rows."""
+        dtype, arrs = _storage(q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v)
+        q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v = arrs
+        B, Hq, d = q.shape
+        _, Hkv, n_max, _ = gist_k.shape
+        m1_max, m2_max, t_max = meta_k.shape[2], meta2_k.shape[2], raw_k.shape[2]
+        _check_shapes(gist_k, (B, Hkv, n_max, d), gist_v, raw_k, raw_v, t_max)
+        if meta_k.shape != (B, Hkv, m1_max, d) or meta_v.shape != meta_k.shape:
+            raise ValueError("meta_k/meta_v shape")
+        if meta2_k.shape != (B, Hkv, m2_max, d) or meta2_v.shape != meta2_k.shape:
+            raise ValueError("meta2_k/meta2_v shape")
+        n_gists, own_len = _i32(n_gists), _i32(own_len)
+        rows_a, n_rows = _rows32(rows, B * Hq)
+        m2s = None if meta2_sel_in is None else _i32(meta2_sel_in).reshape(n_rows, topk2)
+        m1s = None if meta_sel_in is None else _i32(meta_sel_in).reshape(n_rows, topk1)
+        sel = None if sel_in is None else _i32(sel_in).reshape(n_rows, topk)
+        res = _alloc(n_rows, d, topk, set_cap)
+        res["meta2_sel"] = np.full((n_rows, topk2), -1, np.int32)
+        res["meta_sel"] = np.full((n_rows, topk1), -1, np.int32)
+        if want_scores:
+            res["meta2_scores"] = np.zeros((n_rows, m2_max))
+            res["meta_cand_scores"] = np.zeros((n_rows, m1_max))
+            res["cand_scores"] = np.zeros((n_rows, n_max))
+        a = _Hgsa2Args(B, Hq, Hkv, d, chunk, n_max, t_max, m1_max, m2_max, group1, group2, topk2, topk1, topk,
+                       int(bool(exclude)), dtype, float(scale), _ptr(q), _ptr(meta2_k), _ptr(meta2_v), _ptr(meta_k),
+                       _ptr(meta_v), _ptr(gist_k), _ptr(gist_v), _ptr(raw_k), _ptr(raw_v), _ip_(n_gists),
+                       _ip_(own_len), n_rows, _ip_(rows_a), _ip_(m2s), _ip_(m1s), _ip_(sel), _dp_(res["out"]),
+                       _dp_(res["lse"]), _ip_(res["meta2_sel"]), _ip_(res["meta_sel"]), _ip_(res["sel"]),
+                       _dp_(res.get("meta2_scores")), _dp_(res.get("meta_cand_scores")), _dp_(res.get("cand_scores")),
+                       set_cap, _ip_(res.get("set_n")), _ip_(res.get("set_kind")), _ip_(res.get("set_idx")),
+                       _dp_(res.get("set_w")), n_threads)
+        _ok(self.lib.gsa_oracle_hgsa2(C.byref(a)), "hgsa2")
         return res
 
     # ----------------------------------------------------------------- prefill

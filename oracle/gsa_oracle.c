@@ -60,6 +60,7 @@
 #define TOK_RAW 0
 #define TOK_GIST 1
 #define TOK_META 2
+#define TOK_META2 3
 
 /* ------------------------------------------------------------------------ */
 /* Argument blocks (mirrored by ctypes in oracle/__init__.py).               */
@@ -106,6 +107,28 @@ typedef struct {
   double *set_w;
   int32_t n_threads;
 } orc_hgsa_args;
+
+/* H-GSA with two meta levels: level-1 meta-gist j summarises gists
+ * j*group1 .. +group1-1; level-2 meta-gist i summarises level-1 meta-gists
+ * i*group2 .. +group2-1. */
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk;
+  int32_t n_max, t_max, m1_max, m2_max;
+  int32_t group1, group2, topk2, topk1, topk, exclude, dtype;
+  double scale;
+  const void *q, *meta2_k, *meta2_v, *meta_k, *meta_v, *gist_k, *gist_v, *raw_k, *raw_v;
+  const int32_t *n_gists, *own_len;
+  int32_t n_rows;
+  const int32_t *rows;
+  const int32_t *meta2_sel_in, *meta_sel_in, *sel_in; /* optional forced selections per level */
+  double *out, *lse;
+  int32_t *meta2_sel_out, *meta_sel_out, *sel_out;     /* [n_rows][topk2], [topk1], [topk] */
+  double *meta2_scores, *meta_cand_scores, *cand_scores;/* [n_rows][m2_max], [m1_max], [n_max]; NaN = not scored */
+  int32_t set_cap;
+  int32_t *set_n, *set_kind, *set_idx;
+  double *set_w;
+  int32_t n_threads;
+} orc_hgsa2_args;
 
 typedef struct {
   int32_t batch, hq, hkv, d, chunk;
@@ -632,6 +655,169 @@ static int hgsa_row(const void *pa, int64_t slot) {
   free(is_cand);
   free(chosen);
   return st;
+}
+
+/* One level of the coarse-to-fine selection: the candidates are the
+ * children of the chosen parents plus the entries of an incomplete trailing
+ * group (no parent summarises them); they are scored and the top k (or a
+ * forced list) chosen.  `chosen_parent` has `n_parents` entries (complete
+ * groups); `cand`, `score`, `is_cand`, `chosen` have `n` entries.  Returns
+ * the number chosen, or -1 for an invalid forced list. */
+static int32_t select_level(const void *q, size_t qo, const void *keys, size_t kbase, int d, int dt, double scale,
+                            int32_t n, int32_t group, int32_t n_parents, const char *chosen_parent, int32_t k,
+                            const int32_t *forced, scored_t *cand, double *score, char *is_cand, char *chosen) {
+  int32_t nc = 0;
+  for (int32_t m = 0; m < n; ++m) {
+    const int32_t grp = m / group;
+    is_cand[m] = 0;
+    chosen[m] = 0;
+    if (grp >= n_parents || chosen_parent[grp]) {
+      is_cand[m] = 1;
+      score[m] = scale * dot(q, qo, keys, (kbase + m) * d, d, dt);
+      cand[nc].s = score[m];
+      cand[nc].m = m;
+      ++nc;
+    }
+  }
+  int32_t ns;
+  if (forced) {
+    ns = forced_selection(forced, k, n, cand, score);
+    if (ns < 0) return -1;
+    for (int32_t i = 0; i < ns; ++i)
+      if (!is_cand[cand[i].m]) return -1;
+  } else {
+    ns = select_topk(cand, nc, k);
+  }
+  for (int32_t i = 0; i < ns; ++i) chosen[cand[i].m] = 1;
+  return ns;
+}
+
+static int hgsa2_row(const void *pa, int64_t slot) {
+  const orc_hgsa2_args *a = (const orc_hgsa2_args *)pa;
+  const int32_t row = a->rows ? a->rows[slot] : (int32_t)slot;
+  const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);
+  const int d = a->d, c = a->chunk, dt = a->dtype;
+  const double scale = resolve_scale(a->scale, d);
+  const int32_t N = a->n_gists[b], own = a->own_len[b];
+  const int32_t M1 = N / a->group1, M2 = M1 / a->group2; /* complete groups at each level */
+  const size_t qo = ((size_t)b * a->hq + h) * d;
+  const size_t gbase = ((size_t)b * a->hkv + kvh) * a->n_max;
+  const size_t m1base = ((size_t)b * a->hkv + kvh) * a->m1_max;
+  const size_t m2base = ((size_t)b * a->hkv + kvh) * a->m2_max;
+  const size_t rbase = ((size_t)b * a->hkv + kvh) * a->t_max;
+  int st = ORC_OK;
+  const int32_t cap = (N > 0 ? N : 1);
+  scored_t *cand = (scored_t *)malloc((size_t)cap * sizeof(scored_t));
+  double *score2 = (double *)malloc((size_t)(M2 > 0 ? M2 : 1) * sizeof(double));
+  double *score1 = (double *)malloc((size_t)(M1 > 0 ? M1 : 1) * sizeof(double));
+  double *score0 = (double *)malloc((size_t)cap * sizeof(double));
+  char *all2 = (char *)calloc(1, 1);
+  char *cand2 = (char *)calloc((size_t)(M2 > 0 ? M2 : 1), 1), *chosen2 = (char *)calloc((size_t)(M2 > 0 ? M2 : 1), 1);
+  char *cand1 = (char *)calloc((size_t)(M1 > 0 ? M1 : 1), 1), *chosen1 = (char *)calloc((size_t)(M1 > 0 ? M1 : 1), 1);
+  char *cand0 = (char *)calloc((size_t)cap, 1), *chosen0 = (char *)calloc((size_t)cap, 1);
+  if (!cand || !score2 || !score1 || !score0 || !all2 || !cand2 || !chosen2 || !cand1 || !chosen1 || !cand0 || !chosen0)
+    return ORC_ENOMEM;
+
+  /* level 2: every level-2 meta-gist is a candidate (one group with no parent) */
+  const int32_t n2 = select_level(a->q, qo, a->meta2_k, m2base, d, dt, scale, M2, M2 > 0 ? M2 : 1, 0, all2,
+                                  a->topk2, a->meta2_sel_in ? a->meta2_sel_in + (size_t)slot * a->topk2 : NULL,
+                                  cand, score2, cand2, chosen2);
+  if (n2 < 0) return ORC_EINVAL;
+  if (a->meta2_sel_out) {
+    int32_t *o = a->meta2_sel_out + (size_t)slot * a->topk2;
+    for (int32_t i = 0; i < a->topk2; ++i) o[i] = i < n2 ? cand[i].m : -1;
+  }
+  if (a->meta2_scores) {
+    double *o = a->meta2_scores + (size_t)slot * a->m2_max;
+    for (int32_t j = 0; j < a->m2_max; ++j) o[j] = j < M2 ? score2[j] : NAN;
+  }
+  /* level 1: children of the chosen level-2 groups + the trailing level-1 meta-gists */
+  const int32_t n1 = select_level(a->q, qo, a->meta_k, m1base, d, dt, scale, M1, a->group2, M2, chosen2, a->topk1,
+                                  a->meta_sel_in ? a->meta_sel_in + (size_t)slot * a->topk1 : NULL, cand, score1,
+                                  cand1, chosen1);
+  if (n1 < 0) return ORC_EINVAL;
+  if (a->meta_sel_out) {
+    int32_t *o = a->meta_sel_out + (size_t)slot * a->topk1;
+    for (int32_t i = 0; i < a->topk1; ++i) o[i] = i < n1 ? cand[i].m : -1;
+  }
+  if (a->meta_cand_scores) {
+    double *o = a->meta_cand_scores + (size_t)slot * a->m1_max;
+    for (int32_t j = 0; j < a->m1_max; ++j) o[j] = (j < M1 && cand1[j]) ? score1[j] : NAN;
+  }
+  /* level 0: children of the chosen level-1 meta-gists + the trailing gists */
+  const int32_t n0 = select_level(a->q, qo, a->gist_k, gbase, d, dt, scale, N, a->group1, M1, chosen1, a->topk,
+                                  a->sel_in ? a->sel_in + (size_t)slot * a->topk : NULL, cand, score0, cand0,
+                                  chosen0);
+  if (n0 < 0) return ORC_EINVAL;
+  if (a->sel_out) {
+    int32_t *o = a->sel_out + (size_t)slot * a->topk;
+    for (int32_t i = 0; i < a->topk; ++i) o[i] = i < n0 ? cand[i].m : -1;
+  }
+  if (a->cand_scores) {
+    double *o = a->cand_scores + (size_t)slot * a->n_max;
+    for (int32_t m = 0; m < a->n_max; ++m) o[m] = (m < N && cand0[m]) ? score0[m] : NAN;
+  }
+
+  /* the attended set at every resolution: unselected level-2 meta-gists,
+   * unselected level-1 candidates, unselected gist candidates, the chosen
+   * chunks (raw + gist) and the own raw rows */
+  tokset_t S = {0};
+  if (!a->exclude) {
+    for (int32_t i = 0; i < M2 && !st; ++i)
+      if (!chosen2[i]) st = push(&S, a->meta2_k, a->meta2_v, (m2base + i) * d, TOK_META2, i);
+    for (int32_t j = 0; j < M1 && !st; ++j)
+      if (cand1[j] && !chosen1[j]) st = push(&S, a->meta_k, a->meta_v, (m1base + j) * d, TOK_META, j);
+  }
+  for (int32_t m = 0; m < N && !st; ++m) {
+    if (chosen0[m]) {
+      for (int j = 0; j < c && !st; ++j)
+        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    } else if (cand0[m] && !a->exclude) {
+      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    }
+  }
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  if (!st) {
+    const size_t so = (size_t)slot;
+    st = attend(a->q, qo, &S, d, dt, scale, a->out + so * d, a->lse ? a->lse + so : NULL, a->set_cap,
+                a->set_n ? a->set_n + so : NULL, a->set_kind ? a->set_kind + so * a->set_cap : NULL,
+                a->set_idx ? a->set_idx + so * a->set_cap : NULL, a->set_w ? a->set_w + so * a->set_cap : NULL);
+  }
+  free(S.tok);
+  free(cand);
+  free(score2);
+  free(score1);
+  free(score0);
+  free(all2);
+  free(cand2);
+  free(chosen2);
+  free(cand1);
+  free(chosen1);
+  free(cand0);
+  free(chosen0);
+  return st;
+}
+
+int gsa_oracle_hgsa2(const orc_hgsa2_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (a->group1 <= 0 || a->group2 <= 0 || a->topk < 0 || a->topk1 < 0 || a->topk2 < 0) return ORC_EINVAL;
+  if (!a->q || !a->meta2_k || !a->meta2_v || !a->meta_k || !a->meta_v || !a->gist_k || !a->gist_v || !a->raw_k ||
+      !a->raw_v || !a->out)
+    return ORC_EINVAL;
+  if (!a->n_gists || !a->own_len) return ORC_EINVAL;
+  for (int b = 0; b < a->batch; ++b) {
+    int32_t N = a->n_gists[b], own = a->own_len[b];
+    if (N < 0 || N > a->n_max || own < 0 || own > a->chunk) return ORC_EINVAL;
+    if (N / a->group1 > a->m1_max || N / a->group1 / a->group2 > a->m2_max) return ORC_EINVAL;
+    if ((int64_t)N * a->chunk + own > a->t_max) return ORC_EINVAL;
+  }
+  int64_t n = a->rows ? a->n_rows : (int64_t)a->batch * a->hq;
+  if (a->rows)
+    for (int64_t i = 0; i < n; ++i)
+      if (a->rows[i] < 0 || a->rows[i] >= a->batch * a->hq) return ORC_EINVAL;
+  return run_pool(hgsa2_row, a, n, a->n_threads);
 }
 
 int gsa_oracle_hgsa(const orc_hgsa_args *a) {

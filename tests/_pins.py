@@ -350,6 +350,95 @@ def pin_hgsa_reduces_to_flat(orc):
         np.testing.assert_allclose(res1["out"], flat["out"], rtol=1e-12, atol=1e-12)
 
 
+def rand_hgsa2(rng, B, Hq, Hkv, d, c, N, g1, g2, own):
+    arr = rand_hgsa(rng, B, Hq, Hkv, d, c, N, g1, own)
+    M2 = max(1, (N // g1) // g2)
+    arr["meta2_k"] = rng.standard_normal((B, Hkv, M2 + 1, d)).astype(np.float32)
+    arr["meta2_v"] = rng.standard_normal((B, Hkv, M2 + 1, d)).astype(np.float32)
+    return arr
+
+
+def run_hgsa2(orc, arr, c, g1, g2, k2, k1, k, exclude, **kw):
+    return orc.hgsa2(arr["q"], arr["meta2_k"], arr["meta2_v"], arr["meta_k"], arr["meta_v"], arr["gist_k"],
+                     arr["gist_v"], arr["raw_k"], arr["raw_v"], arr["n_gists"], arr["own_len"], chunk=c, group1=g1,
+                     group2=g2, topk2=k2, topk1=k1, topk=k, exclude=exclude, **kw)
+
+
+def pin_hgsa2_bruteforce(orc):
+    """Two meta levels: subsets by enumeration at each level (level-2 groups,
+    then level-1 children, then gist children); dense mask over raw, gist,
+    level-1 and level-2 tokens."""
+    rng = np.random.default_rng(23)
+    for trial in range(24):
+        c = int(rng.integers(1, 3))
+        g1, g2 = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+        N = int(rng.integers(0, 16))
+        k2, k1, k = int(rng.integers(0, 3)), int(rng.integers(0, 4)), int(rng.integers(0, 4))
+        own = int(rng.integers(1, c + 1))
+        d = 3
+        arr = rand_hgsa2(rng, 1, 2, 1, d, c, N, g1, g2, own)
+        M1 = N // g1
+        M2 = M1 // g2
+        for exclude in (False, True):
+            res = run_hgsa2(orc, arr, c, g1, g2, k2, k1, k, exclude)
+            for h in range(2):
+                q = arr["q"][0, h].astype(np.float64)
+                sc = 1 / math.sqrt(d)
+                m2k, m2v = arr["meta2_k"][0, 0].astype(np.float64), arr["meta2_v"][0, 0].astype(np.float64)
+                mk, mv = arr["meta_k"][0, 0].astype(np.float64), arr["meta_v"][0, 0].astype(np.float64)
+                gk, gv = arr["gist_k"][0, 0].astype(np.float64), arr["gist_v"][0, 0].astype(np.float64)
+                rk, rv = arr["raw_k"][0, 0].astype(np.float64), arr["raw_v"][0, 0].astype(np.float64)
+                S2 = brute_topk(list(sc * (m2k[:M2] @ q)), k2)
+                cand1 = [j for j in range(M1) if j // g2 >= M2 or j // g2 in S2]
+                s1 = sc * (mk[cand1] @ q) if cand1 else np.zeros(0)
+                S1 = {cand1[i] for i in brute_topk(list(s1), k1)}
+                cand0 = [m for m in range(N) if m // g1 >= M1 or m // g1 in S1]
+                s0 = sc * (gk[cand0] @ q) if cand0 else np.zeros(0)
+                S0 = {cand0[i] for i in brute_topk(list(s0), k)}
+                K, V, lab = interleaved(rk, rv, gk, gv, N, c, own)
+                if M1:
+                    K, V = np.concatenate([K, mk[:M1]]), np.concatenate([V, mv[:M1]])
+                    lab = lab + [("meta", j) for j in range(M1)]
+                if M2:
+                    K, V = np.concatenate([K, m2k[:M2]]), np.concatenate([V, m2v[:M2]])
+                    lab = lab + [("meta2", i) for i in range(M2)]
+                mask = np.array([(kind == "raw" and m in S0)
+                                 or (kind == "gist" and m in cand0 and (m in S0 or not exclude))
+                                 or kind == "own"
+                                 or (kind == "meta" and m in cand1 and m not in S1 and not exclude)
+                                 or (kind == "meta2" and m not in S2 and not exclude) for kind, m in lab])
+                out, lse, _ = softmax_attend(q, K, V, mask, sc)
+                assert {int(x) for x in res["meta2_sel"][h] if x >= 0} == S2
+                assert {int(x) for x in res["meta_sel"][h] if x >= 0} == S1
+                assert {int(x) for x in res["sel"][h] if x >= 0} == S0
+                np.testing.assert_allclose(res["out"][h], out, rtol=1e-12, atol=1e-12)
+                assert abs(res["lse"][h] - lse) < 1e-12
+
+
+def pin_hgsa2_reduces_to_one_level(orc):
+    """Every level-2 group chosen -> the one-level H-GSA (a separate routine)
+    with the same level-1 budget; one level-1 meta per level-2 meta with the
+    same keys and values behaves like one level with the budget of level 2."""
+    rng = np.random.default_rng(24)
+    B, Hq, Hkv, d, c, N, g1, g2, own, k1, k = 1, 4, 2, 6, 2, 24, 3, 2, 2, 3, 4
+    arr = rand_hgsa2(rng, B, Hq, Hkv, d, c, N, g1, g2, own)
+    M2 = (N // g1) // g2
+    for exclude in (False, True):
+        one = run_hgsa(orc, arr, c, g1, k1, k, exclude)
+        two = run_hgsa2(orc, arr, c, g1, g2, M2, k1, k, exclude)
+        np.testing.assert_allclose(two["out"], one["out"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(two["lse"], one["lse"], rtol=1e-12, atol=1e-12)
+        assert (two["sel"] == one["sel"]).all() and (two["meta_sel"] == one["meta_sel"]).all()
+        # g2 = 1 and level-2 rows equal to the level-1 rows: level 2 picks the
+        # same groups the one-level H-GSA picks, and every level-1 candidate
+        # is chosen (k1 = its budget), so the sets coincide
+        arr1 = dict(arr)
+        arr1["meta2_k"], arr1["meta2_v"] = arr["meta_k"], arr["meta_v"]
+        two1 = run_hgsa2(orc, arr1, c, g1, 1, k1, k1, k, exclude)
+        np.testing.assert_allclose(two1["out"], one["out"], rtol=1e-12, atol=1e-12)
+        assert (two1["sel"] == one["sel"]).all()
+
+
 def pin_hgsa_golden(orc):
     """Hand-derived example (tests/golden/hgsa_hand.json)."""
     _check_golden(orc, json.loads((GOLDEN / "hgsa_hand.json").read_text()))
@@ -549,6 +638,7 @@ def pin_topp_selection(orc):
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
                pin_decode_golden]
-HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden]
+HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden, pin_hgsa2_bruteforce,
+             pin_hgsa2_reduces_to_one_level]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]
 ALL_PINS = [pin_topk_selection, pin_topp_selection] + DECODE_PINS + HGSA_PINS + PREFILL_PINS

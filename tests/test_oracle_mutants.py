@@ -39,6 +39,11 @@ MUTANTS = [
     ("prefill_gist_query_excludes_itself", "for (int32_t t = 0; t <= m && !st; ++t)", "for (int32_t t = 0; t < m && !st; ++t)"),
     ("prefill_chunk_of_position_off_by_one", "const int32_t m = (int32_t)(pos / c), j = (int32_t)(pos % c);",
      "const int32_t m = (int32_t)((pos + 1) / c), j = (int32_t)((pos + 1) % c);"),
+    ("hgsa2_noncandidate_level1_attended", "if (cand1[j] && !chosen1[j]) st = push(&S, a->meta_k",
+     "if (!chosen1[j]) st = push(&S, a->meta_k"),
+    ("hgsa2_chosen_level2_attended", "if (!chosen2[i]) st = push(&S, a->meta2_k", "if (1) st = push(&S, a->meta2_k"),
+    ("hgsa2_level0_under_level2_groups", "const int32_t n0 = select_level(a->q, qo, a->gist_k, gbase, d, dt, scale, N, a->group1, M1, chosen1,",
+     "const int32_t n0 = select_level(a->q, qo, a->gist_k, gbase, d, dt, scale, N, a->group1 * a->group2, M2, chosen2,"),
     ("topp_output_descending", "return (a->m > b->m) - (a->m < b->m);", "return (a->m < b->m) - (a->m > b->m);"),
     ("topp_strict_mass_test", "if (mass >= top_p) break;", "if (mass > top_p) break;"),
     ("topp_unshifted_exponent", "for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s - cand[0].s);",
