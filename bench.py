@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,prefill_32k,llama1b_8x_topp",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
@@ -345,6 +345,75 @@ def measure_hgsa(G, W, cfg, dev, args, flush, hbm):
             "kernels_us": {"hgsa_select": round(float(k[0]) * 1e3, 2), "unfold_attend": round(float(k[1]) * 1e3, 2)}}
 
 
+def measure_hgsa2(G, W, cfg, dev, args, flush, hbm):
+    """H-GSA with two meta levels: the fused step (hgsa2_decode), the select
+    and unfold halves, and the step's algorithmic bytes (all level-2
+    meta-gists, the level-1 candidates under the chosen level-2 groups, the
+    gist candidates under the chosen level-1 meta-gists -- unions per (b, kv
+    head) -- the chosen chunks' raw rows, own rows, q and out)."""
+    x = W.decode_inputs(cfg, device=dev)
+    B, hq, d = x["q"].shape
+    hkv, n_max, t_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2]
+    m1_max, m2_max = x["meta_k"].shape[2], x["meta2_k"].shape[2]
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, cfg.exclude, 0.0, G.GSA_BF16, G.GSA_F32)
+    h2 = G.make_h2desc(G.make_hdesc(cfg.group, cfg.topk_meta, m1_max), G.make_hdesc(cfg.group2, cfg.topk_meta2, m2_max))
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_HGSA2, h2), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    m2 = torch.empty((B, hq, cfg.topk_meta2), dtype=torch.int32, device=dev)
+    m1 = torch.empty((B, hq, cfg.topk_meta), dtype=torch.int32, device=dev)
+    si = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ss = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+    args_ = (x["q"], x["meta2_k"], x["meta2_v"], x["meta_k"], x["meta_v"], x["gist_k"], x["gist_v"])
+
+    def fused(evs=None):
+        if evs:
+            evs[0].record()
+        G.hgsa2_decode(desc, h2, *args_, x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"], out, None, m2, m1, si,
+                       ss, ws)
+        if evs:
+            evs[1].record()
+
+    def split(evs):
+        evs[0].record()
+        G.hgsa2_select(desc, h2, *args_, x["n_gists"], m2, m1, si, ss, ws)
+        evs[1].record()
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], si, ss,
+                            G.GSA_PRIOR_HGSA2, out, None, ws)
+        evs[2].record()
+
+    for _ in range(args.warmup):
+        flush()
+        fused()
+    step_ms = timed_steps(fused, args.steps, flush)[:, 0]
+    k = timed_steps(split, args.steps, flush, 2).mean(0)
+    assert G.gsa_workspace_status(ws) == 0
+    e, G_ = 2, hq // hkv
+    M1 = cfg.n_gists // cfg.group
+    M2 = M1 // cfg.group2
+
+    def union(t):
+        t = t.reshape(B, hkv, G_, -1).cpu()
+        return sum(int((torch.unique(t[b, kv]) >= 0).sum()) for b in range(B) for kv in range(hkv))
+
+    meta2 = B * hkv * M2 * d * e * 2
+    u2, u1, u0 = union(m2), union(m1), union(si)
+    trail1 = B * hkv * (M1 - M2 * cfg.group2)  # level-1 meta-gists of an incomplete level-2 group
+    trail0 = B * hkv * (cfg.n_gists - M1 * cfg.group)
+    total = (meta2 + (u2 * cfg.group2 + trail1) * d * e * 2 + (u1 * cfg.group + trail0) * d * e * 2
+             + u0 * cfg.chunk * d * e * 2 + B * hkv * d * e * 2 + B * hq * d * (e + 4))
+    one_level_meta = B * hkv * M1 * d * e * 2  # what scoring every level-1 meta-gist would read
+    ms = float(np.mean(step_ms))
+    return {"metric": "GSA decode head-queries/s", "value": round(cfg.head_queries / (ms / 1e3), 1), "unit": UNIT,
+            "ms_per_step": round(ms, 5),
+            "step_hbm": {"alg_bytes": total, "achieved_gbs": round(total / (ms / 1e3) / 1e9, 1),
+                         "frac": round(total / (ms / 1e3) / 1e9 / hbm, 4)},
+            "level_bytes": {"level2_meta": meta2, "level1_candidates": (u2 * cfg.group2 + trail1) * d * e * 2,
+                            "gist_candidates": (u1 * cfg.group + trail0) * d * e * 2,
+                            "one_level_meta_read_instead": one_level_meta},
+            "kernels_us": {"hgsa2_select": round(float(k[0]) * 1e3, 2), "unfold_attend": round(float(k[1]) * 1e3, 2)}}
+
+
 def measure_prefill(G, W, cfg, dev, args, flush, bf16_peak):
     x = W.prefill_inputs(cfg, device=dev)
     B, hq, L, d = x["q_raw"].shape
@@ -456,6 +525,8 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
         c = W.CONFIGS[name]
         if name.startswith("prefill"):
             extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)
+        elif c.group2:
+            extra[name] = measure_hgsa2(G, W, c, dev, args, flush, hbm)
         elif c.group:
             extra[name] = measure_hgsa(G, W, c, dev, args, flush, hbm)
         else:

@@ -78,11 +78,12 @@ typedef enum gsa_dtype { GSA_F32 = 0, GSA_BF16 = 1 } gsa_dtype;
 typedef enum gsa_prior {
   GSA_PRIOR_NONE = 0,  /* nothing: only valid with exclude_unselected = 1 */
   GSA_PRIOR_GISTS = 1, /* gsa_score_gists in default mode: all completed gists */
-  GSA_PRIOR_HGSA = 2   /* hgsa_select: unselected meta-gists + unselected candidate gists */
+  GSA_PRIOR_HGSA = 2,  /* hgsa_select: unselected meta-gists + unselected candidate gists */
+  GSA_PRIOR_HGSA2 = 3  /* hgsa2_select: the same over two meta levels */
 } gsa_prior;
 
 /* Workspace sizing: which call sequence the workspace serves. */
-typedef enum gsa_op { GSA_OP_DECODE = 0, GSA_OP_HGSA = 1, GSA_OP_PREFILL = 2 } gsa_op;
+typedef enum gsa_op { GSA_OP_DECODE = 0, GSA_OP_HGSA = 1, GSA_OP_PREFILL = 2, GSA_OP_HGSA2 = 3 } gsa_op;
 
 /* Device-side status bits (gsa_workspace_status). */
 #define GSA_DEVERR_BAD_INDEX 0x1u /* a sel_idx entry >= N was skipped */
@@ -109,6 +110,15 @@ typedef struct gsa_hdesc {
   int32_t m_max;     /* meta capacity per (b, kv head), >= n_max / group */
 } gsa_hdesc;
 
+/* H-GSA with two meta levels: level1 groups gists into meta-gists (as
+ * gsa_hdesc for hgsa_select); level2 groups level-1 meta-gists into
+ * level-2 meta-gists (group = level-1 meta-gists per level-2 meta-gist,
+ * topk_meta = level-2 groups kept, m_max = level-2 capacity). */
+typedef struct gsa_h2desc {
+  gsa_hdesc level1;
+  gsa_hdesc level2;
+} gsa_h2desc;
+
 /* Human-readable name of a status code (static string). */
 const char *gsa_status_string(int32_t status);
 
@@ -116,8 +126,9 @@ const char *gsa_status_string(int32_t status);
 int32_t gsa_version(void);
 
 /* Bytes of workspace the call sequence `op` needs for these shapes
- * (hdesc only for GSA_OP_HGSA, may be NULL otherwise).  Returns 0 if the
- * shapes are invalid. */
+ * (hdesc only for GSA_OP_HGSA, may be NULL otherwise; for GSA_OP_HGSA2 it
+ * points at the two descriptors of a gsa_h2desc, level1 first).  Returns 0
+ * if the shapes are invalid. */
 size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc);
 
 /* Zero the workspace on `stream` (cudaMemsetAsync).  Needed once after
@@ -247,6 +258,37 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
                        const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
                        int32_t *meta_idx, int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes,
                        void *stream);
+
+/* ---- H-GSA decode: two meta levels (the recursive gist-of-gist form of
+ * [ja] 2.2 / [nl] Hierarchische Uitbreiding) ------------------------------ */
+
+/* Coarse-to-fine over three levels.  With N = n_gists[b], M1 = N / g1
+ * level-1 meta-gists and M2 = M1 / g2 level-2 meta-gists (g1 =
+ * level1.group, g2 = level2.group): the top level2.topk_meta level-2
+ * groups are kept; their level-1 children plus the level-1 meta-gists of an
+ * incomplete trailing level-2 group are scored and the top level1.topk_meta
+ * kept; their gist children plus the gists of an incomplete trailing
+ * level-1 group are scored and the top desc->topk chosen.
+ *   meta2_k, meta2_v [B, hkv, level2.m_max, d]; meta_k, meta_v [B, hkv,
+ *   level1.m_max, d]; gist and raw arrays as for hgsa_select.
+ *   meta2_idx [B, hq, level2.topk_meta], meta_idx [B, hq, level1.topk_meta]
+ *   int32 out (ascending, -1 padded); sel_idx / sel_score as hgsa_select.
+ * In default mode ws receives the softmax partial over the unselected
+ * level-2 meta-gists, the unselected level-1 candidates and all gist
+ * candidates, consumed with prior = GSA_PRIOR_HGSA2.  Workspace:
+ * gsa_workspace_bytes(desc, GSA_OP_HGSA2, &h2desc.level1). */
+gsa_status hgsa2_select(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,
+                        const void *meta2_v, const void *meta_k, const void *meta_v, const void *gist_k,
+                        const void *gist_v, const int32_t *n_gists, int32_t *meta2_idx, int32_t *meta_idx,
+                        int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
+
+/* One two-level H-GSA decode step = hgsa2_select -> gsa_unfold_attend; the
+ * index and score outputs may be NULL (ws holds them). */
+gsa_status hgsa2_decode(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,
+                        const void *meta2_v, const void *meta_k, const void *meta_v, const void *gist_k,
+                        const void *gist_v, const void *raw_k, const void *raw_v, const int32_t *n_gists,
+                        const int32_t *own_len, void *out, float *lse, int32_t *meta2_idx, int32_t *meta_idx,
+                        int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
 
 /* ---- Causal prefill with interleaved gists ([nl] Compressie + the
  * decode steps applied at every position) ------------------------------ */

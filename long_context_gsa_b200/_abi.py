@@ -18,14 +18,15 @@ from .build import LIB
 
 GSA_OK, GSA_ERR_INVALID_ARG, GSA_ERR_UNSUPPORTED, GSA_ERR_WORKSPACE, GSA_ERR_CUDA, GSA_ERR_TIMEOUT = range(6)
 GSA_F32, GSA_BF16 = 0, 1
-GSA_PRIOR_NONE, GSA_PRIOR_GISTS, GSA_PRIOR_HGSA = 0, 1, 2
-GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL = 0, 1, 2
+GSA_PRIOR_NONE, GSA_PRIOR_GISTS, GSA_PRIOR_HGSA, GSA_PRIOR_HGSA2 = 0, 1, 2, 3
+GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL, GSA_OP_HGSA2 = 0, 1, 2, 3
 GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
-    "hgsa_decode", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill", "gsa_decode_noalloc",
+    "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
+    "gsa_decode_noalloc",
 )
 
 
@@ -44,6 +45,10 @@ class gsa_desc(C.Structure):
 
 class gsa_hdesc(C.Structure):
     _fields_ = [("group", C.c_int32), ("topk_meta", C.c_int32), ("m_max", C.c_int32)]
+
+
+class gsa_h2desc(C.Structure):
+    _fields_ = [("level1", gsa_hdesc), ("level2", gsa_hdesc)]
 
 
 _lib = None
@@ -74,6 +79,8 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_decode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "hgsa_select": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "hgsa_decode": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "hgsa2_select": ([D, C.POINTER(gsa_h2desc)] + [vp] * 13 + [sz, vp], i32),
+        "hgsa2_decode": ([D, C.POINTER(gsa_h2desc)] + [vp] * 18 + [sz, vp], i32),
         "gsa_prefill_score": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
@@ -100,6 +107,10 @@ def make_desc(batch, hq, hkv, d, chunk, n_max, t_max, topk, exclude_unselected=F
 
 def make_hdesc(group, topk_meta, m_max) -> gsa_hdesc:
     return gsa_hdesc(group, topk_meta, m_max)
+
+
+def make_h2desc(level1: gsa_hdesc, level2: gsa_hdesc) -> gsa_h2desc:
+    return gsa_h2desc(level1, level2)
 
 
 def _ptr(t, dtype=None, name="tensor", optional=False):
@@ -145,8 +156,13 @@ def gsa_version() -> int:
     return int(load().gsa_version())
 
 
-def gsa_workspace_bytes(desc: gsa_desc, op: int = GSA_OP_DECODE, hdesc: gsa_hdesc | None = None) -> int:
-    return int(load().gsa_workspace_bytes(C.byref(desc), op, C.byref(hdesc) if hdesc is not None else None))
+def gsa_workspace_bytes(desc: gsa_desc, op: int = GSA_OP_DECODE, hdesc=None) -> int:
+    """hdesc: a gsa_hdesc for GSA_OP_HGSA, a gsa_h2desc for GSA_OP_HGSA2 (its level1 is passed)."""
+    if isinstance(hdesc, gsa_h2desc):
+        ref = C.cast(C.byref(hdesc), C.POINTER(gsa_hdesc))
+    else:
+        ref = C.byref(hdesc) if hdesc is not None else None
+    return int(load().gsa_workspace_bytes(C.byref(desc), op, ref))
 
 
 def gsa_workspace_init(ws, stream=None):
@@ -234,6 +250,33 @@ def hgsa_decode(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_
         _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True),
         _ptr(meta_idx, torch.int32, "meta_idx", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
         _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
+
+
+def hgsa2_select(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, n_gists, meta2_idx, meta_idx,
+                 sel_idx, sel_score, ws, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("hgsa2_select", load().hgsa2_select(
+        C.byref(desc), C.byref(h2desc), _ptr(q, dt, "q"), _ptr(meta2_k, dt, "meta2_k"),
+        _ptr(meta2_v, dt, "meta2_v", True), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v", True),
+        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(meta2_idx, torch.int32, "meta2_idx"), _ptr(meta_idx, torch.int32, "meta_idx"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+
+
+def hgsa2_decode(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len,
+                 out, lse=None, meta2_idx=None, meta_idx=None, sel_idx=None, sel_score=None, ws=None, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    p, n = _ws(ws)
+    _check("hgsa2_decode", load().hgsa2_decode(
+        C.byref(desc), C.byref(h2desc), _ptr(q, dt, "q"), _ptr(meta2_k, dt, "meta2_k"), _ptr(meta2_v, dt, "meta2_v"),
+        _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v"), _ptr(gist_k, dt, "gist_k"),
+        _ptr(gist_v, dt, "gist_v"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
+        _ptr(n_gists, torch.int32, "n_gists"), _ptr(own_len, torch.int32, "own_len"),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True),
+        _ptr(meta2_idx, torch.int32, "meta2_idx", True), _ptr(meta_idx, torch.int32, "meta_idx", True),
+        _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
+        _stream(stream)))
 
 
 def gsa_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, ws, stream=None):

@@ -39,6 +39,7 @@ inline float resolve_scale(const gsa_desc *d) {
 struct Layout {
   size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
+  size_t meta2_scores = 0, meta2_idx = 0, cand1_scores = 0, cand1_ids = 0, cand1_count = 0;
   size_t pf_stats = 0, pf_gist = 0, pf_vh = 0, pf_ovf = 0;
   size_t total = 0;
 };
@@ -71,6 +72,21 @@ gsa_status check_hdesc(const gsa_desc *d, const gsa_hdesc *h) {
 
 inline int hgsa_cand_cap(const gsa_hdesc *h) { return h->topk_meta * h->group + h->group - 1; }
 
+// Two meta levels: level1 groups gists into meta-gists, level2 groups
+// level-1 meta-gists into level-2 meta-gists.
+gsa_status check_h2desc(const gsa_desc *d, const gsa_h2desc *h) {
+  if (!h) return GSA_ERR_INVALID_ARG;
+  const gsa_status s1 = check_hdesc(d, &h->level1);
+  if (s1 != GSA_OK) return s1;
+  const gsa_hdesc &l2 = h->level2;
+  if (l2.group < 1 || l2.topk_meta < 1 || l2.m_max < 1) return GSA_ERR_INVALID_ARG;
+  if (l2.topk_meta > 64 || static_cast<int64_t>(l2.topk_meta) * l2.group > 4096 || l2.group > 4096)
+    return GSA_ERR_UNSUPPORTED;
+  if (l2.m_max < h->level1.m_max / l2.group) return GSA_ERR_INVALID_ARG;
+  if (h->level1.topk_meta > hgsa_cand_cap(&l2)) return GSA_ERR_INVALID_ARG;
+  return GSA_OK;
+}
+
 Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   Layout L;
   const size_t rows = static_cast<size_t>(d->batch) * d->hq;
@@ -98,7 +114,7 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   take(L.sel_score, rows * d->topk * 4);
   take(L.part_g, rows * kScoreSplitMax * rec);
   take(L.part_u, rows * kUnfoldSplitMax * rec);
-  if (op == GSA_OP_HGSA && h) {
+  if ((op == GSA_OP_HGSA || op == GSA_OP_HGSA2) && h) {
     const size_t cap = hgsa_cand_cap(h);
     take(L.meta_scores, rows * h->m_max * 4);
     take(L.meta_idx, rows * h->topk_meta * 4);
@@ -106,6 +122,15 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     take(L.cand_ids, rows * cap * 4);
     take(L.cand_count, rows * 4);
     take(L.part_h, rows * kHgsaSplitMax * rec);
+  }
+  if (op == GSA_OP_HGSA2 && h) {  // h points at a gsa_h2desc: level1, then level2
+    const gsa_hdesc *l2 = h + 1;
+    const size_t cap1 = hgsa_cand_cap(l2);
+    take(L.meta2_scores, rows * l2->m_max * 4);
+    take(L.meta2_idx, rows * l2->topk_meta * 4);
+    take(L.cand1_scores, rows * cap1 * 4);
+    take(L.cand1_ids, rows * cap1 * 4);
+    take(L.cand1_count, rows * 4);
   }
   L.total = off;
   return L;
@@ -418,6 +443,14 @@ gsa_status launch_hgsa_children_t(const HgsaArgs &ha, int B, void *stream) {
   return launch(k_hgsa_children<D, T>, dim3(ha.n_split, ha.hq, B), dim3(kHgsaThreads), smem, stream, ha);
 }
 
+gsa_status launch_children(const gsa_desc *d, const HgsaArgs &ha, void *stream) {
+  if (d->dtype == GSA_BF16)
+    return d->d == 64 ? launch_hgsa_children_t<64, __nv_bfloat16>(ha, d->batch, stream)
+                      : launch_hgsa_children_t<128, __nv_bfloat16>(ha, d->batch, stream);
+  return d->d == 64 ? launch_hgsa_children_t<64, float>(ha, d->batch, stream)
+                    : launch_hgsa_children_t<128, float>(ha, d->batch, stream);
+}
+
 gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q, const void *meta_k,
                            const void *meta_v, const void *gist_k, const void *gist_v, const int32_t *n_gists,
                            int32_t *meta_idx, int32_t *sel_idx, float *sel_score, const Layout &L, void *ws,
@@ -455,15 +488,106 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
   ha.part = reinterpret_cast<float *>(at(ws, L.part_g));
   ha.n_split = hgsa_splits(d);
   ha.status = status;
-  gsa_status st;
-  if (d->dtype == GSA_BF16)
-    st = d->d == 64 ? launch_hgsa_children_t<64, __nv_bfloat16>(ha, d->batch, stream)
-                    : launch_hgsa_children_t<128, __nv_bfloat16>(ha, d->batch, stream);
-  else
-    st = d->d == 64 ? launch_hgsa_children_t<64, float>(ha, d->batch, stream)
-                    : launch_hgsa_children_t<128, float>(ha, d->batch, stream);
-  GSA_TRY(st);
+  ha.count_div = 1;
+  ha.fold_children = 1;
+  ha.parent_ids = nullptr;
+  ha.parent_scores = nullptr;
+  ha.parent_count = nullptr;
+  ha.parent_cap = 0;
+  ha.part_stride = ha.n_split;
+  ha.part_off = 0;
+  GSA_TRY(launch_children(d, ha, stream));
   // 4. top gists among the candidates, reported as gist (chunk) ids
+  if (d->topk > 0)
+    return run_topk(rows, d->hq, ha.cand_scores, ha.cap, nullptr, 1, ha.cand_count, d->topk, ha.cand_ids, sel_idx,
+                    sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+  return cudaMemsetAsync(at(ws, L.counters), 0, static_cast<size_t>(rows) * 4, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GSA_OK
+             : GSA_ERR_CUDA;
+}
+
+// Two meta levels: level-2 scores -> top level-2 groups -> level-1
+// candidates (children pass, partial of the unselected level-2 meta-gists)
+// -> top level-1 meta-gists -> gist candidates (children pass, partial of
+// the unselected level-1 candidates and all gist candidates) -> top gists.
+// The two passes' partials share one prior array: [rows][2 * splits].
+gsa_status run_hgsa2_select(const gsa_desc *d, const gsa_h2desc *h2, const void *q, const void *meta2_k,
+                            const void *meta2_v, const void *meta_k, const void *meta_v, const void *gist_k,
+                            const void *gist_v, const int32_t *n_gists, int32_t *meta2_idx, int32_t *meta_idx,
+                            int32_t *sel_idx, float *sel_score, const Layout &L, void *ws, void *stream) {
+  const gsa_hdesc &l1 = h2->level1, &l2 = h2->level2;
+  const int rows = d->batch * d->hq;
+  uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  float *meta2_scores = reinterpret_cast<float *>(at(ws, L.meta2_scores));
+  const int g12 = l1.group * l2.group;
+  GSA_TRY(run_score(d, q, meta2_k, nullptr, n_gists, g12, l2.m_max, meta2_scores, l2.m_max, nullptr, nullptr, status,
+                    stream));
+  GSA_TRY(run_topk(rows, d->hq, meta2_scores, l2.m_max, n_gists, g12, nullptr, l2.topk_meta, nullptr, meta2_idx,
+                   nullptr, nullptr, stream));
+  const int splits = hgsa_splits(d);
+  HgsaArgs ha;
+  ha.q = q;
+  ha.n_gists = n_gists;
+  ha.hq = d->hq;
+  ha.hkv = d->hkv;
+  ha.gqa = d->hq / d->hkv;
+  ha.exclude = d->exclude_unselected;
+  ha.scale_log2 = resolve_scale(d) * kLog2e;
+  ha.part = reinterpret_cast<float *>(at(ws, L.part_g));
+  ha.n_split = splits;
+  ha.status = status;
+  ha.part_stride = 2 * splits;
+  // level-1 candidates: children of the chosen level-2 groups
+  ha.gist_k = meta_k;
+  ha.gist_v = meta_v;
+  ha.meta_v = meta2_v;
+  ha.meta_scores = meta2_scores;
+  ha.meta_idx = meta2_idx;
+  ha.group = l2.group;
+  ha.topk_meta = l2.topk_meta;
+  ha.m_max = l2.m_max;
+  ha.n_max = l1.m_max;
+  ha.count_div = l1.group;
+  ha.fold_children = 0;  // the unselected level-1 candidates enter in the next pass
+  ha.parent_ids = nullptr;
+  ha.parent_scores = nullptr;
+  ha.parent_count = nullptr;
+  ha.parent_cap = 0;
+  ha.cand_scores = reinterpret_cast<float *>(at(ws, L.cand1_scores));
+  ha.cand_ids = reinterpret_cast<int32_t *>(at(ws, L.cand1_ids));
+  ha.cand_count = reinterpret_cast<int32_t *>(at(ws, L.cand1_count));
+  ha.cap = hgsa_cand_cap(&l2);
+  ha.part_off = 0;
+  GSA_TRY(launch_children(d, ha, stream));
+  GSA_TRY(run_topk(rows, d->hq, ha.cand_scores, ha.cap, nullptr, 1, ha.cand_count, l1.topk_meta, ha.cand_ids,
+                   meta_idx, nullptr, nullptr, stream));
+  // gist candidates: children of the chosen level-1 meta-gists; the
+  // unselected level-1 candidates are the listed parents of this pass
+  const float *c1_scores = ha.cand_scores;
+  const int32_t *c1_ids = ha.cand_ids, *c1_count = ha.cand_count;
+  const int cap1 = ha.cap;
+  ha.gist_k = gist_k;
+  ha.gist_v = gist_v;
+  ha.meta_v = meta_v;
+  ha.meta_scores = c1_scores;  // (unused with listed parents)
+  ha.meta_idx = meta_idx;
+  ha.group = l1.group;
+  ha.topk_meta = l1.topk_meta;
+  ha.m_max = l1.m_max;
+  ha.n_max = d->n_max;
+  ha.count_div = 1;
+  ha.fold_children = 1;
+  ha.parent_ids = c1_ids;
+  ha.parent_scores = c1_scores;
+  ha.parent_count = c1_count;
+  ha.parent_cap = cap1;
+  ha.cand_scores = reinterpret_cast<float *>(at(ws, L.cand_scores));
+  ha.cand_ids = reinterpret_cast<int32_t *>(at(ws, L.cand_ids));
+  ha.cand_count = reinterpret_cast<int32_t *>(at(ws, L.cand_count));
+  ha.cap = hgsa_cand_cap(&l1);
+  ha.part_off = splits;
+  GSA_TRY(launch_children(d, ha, stream));
   if (d->topk > 0)
     return run_topk(rows, d->hq, ha.cand_scores, ha.cap, nullptr, 1, ha.cand_count, d->topk, ha.cand_ids, sel_idx,
                     sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
@@ -617,8 +741,10 @@ int32_t gsa_version(void) { return 100; }
 
 size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc) {
   if (check_desc(desc) != GSA_OK) return 0;
-  if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL) return 0;
+  if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL && op != GSA_OP_HGSA2) return 0;
   if (op == GSA_OP_HGSA && check_hdesc(desc, hdesc) != GSA_OK) return 0;
+  if (op == GSA_OP_HGSA2 && (!hdesc || check_h2desc(desc, reinterpret_cast<const gsa_h2desc *>(hdesc)) != GSA_OK))
+    return 0;
   return layout(desc, op, hdesc).total;
 }
 
@@ -723,7 +849,8 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
     GSA_TRY(need_ptr(gist_v));
     GSA_TRY(need_ptr(sel_score));
   }
-  if (prior != GSA_PRIOR_NONE && prior != GSA_PRIOR_GISTS && prior != GSA_PRIOR_HGSA) return GSA_ERR_INVALID_ARG;
+  if (prior != GSA_PRIOR_NONE && prior != GSA_PRIOR_GISTS && prior != GSA_PRIOR_HGSA && prior != GSA_PRIOR_HGSA2)
+    return GSA_ERR_INVALID_ARG;
   if (prior == GSA_PRIOR_NONE && !desc->exclude_unselected) return GSA_ERR_INVALID_ARG;
   const Layout L = layout(desc, GSA_OP_DECODE, nullptr);  // the H-GSA layout extends this one
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
@@ -740,6 +867,9 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
   } else if (prior == GSA_PRIOR_HGSA && !desc->exclude_unselected) {
     pr = reinterpret_cast<const float *>(at(ws, L.part_g));
     n_prior = hgsa_splits(desc);
+  } else if (prior == GSA_PRIOR_HGSA2 && !desc->exclude_unselected) {
+    pr = reinterpret_cast<const float *>(at(ws, L.part_g));
+    n_prior = 2 * hgsa_splits(desc);
   }
   return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, pr, n_prior, out, lse, L,
                     ws, stream);
@@ -839,6 +969,73 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
   const float *pr = desc->exclude_unselected ? nullptr : reinterpret_cast<const float *>(at(ws, L.part_g));
   return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, pr, pr ? hgsa_splits(desc) : 0, out, lse,
                     L, ws, stream);
+}
+
+gsa_status hgsa2_select(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,
+                        const void *meta2_v, const void *meta_k, const void *meta_v, const void *gist_k,
+                        const void *gist_v, const int32_t *n_gists, int32_t *meta2_idx, int32_t *meta_idx,
+                        int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(check_h2desc(desc, h2desc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(meta2_k));
+  GSA_TRY(need_ptr(meta_k));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(meta2_idx));
+  GSA_TRY(need_ptr(meta_idx));
+  GSA_TRY(need_ptr(ws));
+  if (desc->topk > 0) {
+    GSA_TRY(need_ptr(sel_idx));
+    GSA_TRY(need_ptr(sel_score));
+  }
+  if (!desc->exclude_unselected) {
+    GSA_TRY(need_ptr(meta2_v));
+    GSA_TRY(need_ptr(meta_v));
+    GSA_TRY(need_ptr(gist_v));
+  }
+  const Layout L = layout(desc, GSA_OP_HGSA2, &h2desc->level1);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  return run_hgsa2_select(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, n_gists, meta2_idx,
+                          meta_idx, sel_idx, sel_score, L, ws, stream);
+}
+
+gsa_status hgsa2_decode(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,
+                        const void *meta2_v, const void *meta_k, const void *meta_v, const void *gist_k,
+                        const void *gist_v, const void *raw_k, const void *raw_v, const int32_t *n_gists,
+                        const int32_t *own_len, void *out, float *lse, int32_t *meta2_idx, int32_t *meta_idx,
+                        int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  GSA_TRY(check_h2desc(desc, h2desc));
+  GSA_TRY(need_ptr(q));
+  GSA_TRY(need_ptr(meta2_k));
+  GSA_TRY(need_ptr(meta2_v));
+  GSA_TRY(need_ptr(meta_k));
+  GSA_TRY(need_ptr(meta_v));
+  GSA_TRY(need_ptr(gist_k));
+  GSA_TRY(need_ptr(gist_v));
+  GSA_TRY(need_ptr(raw_k));
+  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(n_gists));
+  GSA_TRY(need_ptr(own_len));
+  GSA_TRY(need_ptr(out));
+  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(opt_ptr(meta2_idx));
+  GSA_TRY(opt_ptr(meta_idx));
+  GSA_TRY(opt_ptr(sel_idx));
+  GSA_TRY(opt_ptr(sel_score));
+  GSA_TRY(need_ptr(ws));
+  const Layout L = layout(desc, GSA_OP_HGSA2, &h2desc->level1);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  int32_t *m2 = meta2_idx ? meta2_idx : reinterpret_cast<int32_t *>(at(ws, L.meta2_idx));
+  int32_t *mi = meta_idx ? meta_idx : reinterpret_cast<int32_t *>(at(ws, L.meta_idx));
+  int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
+  float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
+  GSA_TRY(run_hgsa2_select(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, n_gists, m2, mi, si,
+                           ss, L, ws, stream));
+  const float *pr = desc->exclude_unselected ? nullptr : reinterpret_cast<const float *>(at(ws, L.part_g));
+  return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, pr, pr ? 2 * hgsa_splits(desc) : 0,
+                    out, lse, L, ws, stream);
 }
 
 gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *q_gist, const void *k_gist,

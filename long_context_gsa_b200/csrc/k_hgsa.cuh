@@ -37,9 +37,17 @@ struct HgsaArgs {
   int32_t *cand_ids;              // [B*hq, cap]
   int32_t *cand_count;            // [B*hq]
   int32_t cap;
-  float *part;                    // [B*hq, n_split, D+4] (default mode)
+  float *part;                    // [B*hq, part_stride, D+4] (default mode); this pass: slots part_off ..
   int32_t n_split;
   uint32_t *status;
+  // generalisations for a second meta level (zero / null: one level)
+  int32_t count_div;              // entries at this level = n_gists[b] / count_div
+  int32_t fold_children;          // fold the candidates' values into the partial (the gist level)
+  const int32_t *parent_ids;      // parents to attend, as a list [B*hq, parent_cap] (null: all of [0, M))
+  const float *parent_scores;     //   their scores (natural units), same layout
+  const int32_t *parent_count;    //   list length per row
+  int32_t parent_cap;
+  int32_t part_stride, part_off;
 };
 
 constexpr int kHgsaThreads = 128;
@@ -70,7 +78,7 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
   const int sw = unfold_warp_stages(static_cast<int>(2 * piece_bytes));
 
   pdl_wait();
-  const int N = min(max(a.n_gists[b], 0), a.n_max);
+  const int N = min(max(a.n_gists[b] / a.count_div, 0), a.n_max);
   const int M = min(N / g, a.m_max);
   if (warp == 0) {
     // chosen groups, ascending (the meta top-k writes them in ascending order)
@@ -120,7 +128,7 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
   const uint8_t *gk = reinterpret_cast<const uint8_t *>(a.gist_k) + gbase * kRowBytes;
   const uint8_t *gv = reinterpret_cast<const uint8_t *>(a.gist_v) + gbase * kRowBytes;
   uint8_t *ring = smem + static_cast<size_t>(warp) * sw * 2 * piece_bytes;
-  const bool with_v = !a.exclude;
+  const bool with_v = !a.exclude && a.fold_children;  // candidate values go into the partial
   auto piece = [&](int p, int &first, int &rows, int &slot0) {
     const int gi = p / ppg, sub = p % ppg;
     first = groups[gi] + sub * pr;
@@ -203,24 +211,30 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
     flag_error(a.status, GSA_DEVERR_TIMEOUT);
     for (int li = stuck; li < min(stuck + sw, n_mine); ++li) mbar_wait(&bars[warp][li % sw], (li / sw) & 1);
   }
-  if (!with_v) return;
+  if (a.exclude) return;
 
-  // Unselected meta-gists of this split's share of [0, M): logit from the
-  // meta scores, value from meta_v.
-  const int per_m = (M + a.n_split - 1) / a.n_split;
-  const int j0 = min(M, split * per_m), j1 = min(M, j0 + per_m);
+  // Unselected parents of this split's share: all of [0, M) with logits
+  // from the meta scores, or the listed parents (positions of the list)
+  // with their own scores; values from meta_v.
+  const bool listed = a.parent_ids != nullptr;
+  const int P = listed ? min(max(a.parent_count[row], 0), a.parent_cap) : M;
+  const int per_m = (P + a.n_split - 1) / a.n_split;
+  const int j0 = min(P, split * per_m), j1 = min(P, j0 + per_m);
+  auto parent_id = [&](int j) { return listed ? a.parent_ids[row * a.parent_cap + j] : j; };
   const T *mv = reinterpret_cast<const T *>(a.meta_v) + (static_cast<size_t>(b) * a.hkv + kvh) * a.m_max * D;
   const float *ms = a.meta_scores + row * a.m_max;
   constexpr int kU = 8;                          // meta rows in flight per lane group
   constexpr int kStride = kHgsaWarps * kRpw;     // rows between a lane group's consecutive rows
-  // a lane group's rows ascend, so one pointer walks the ascending sel_meta
+  // a lane group's rows ascend (listed parents are in ascending id order
+  // too), so one pointer walks the ascending sel_meta
   int sp = 0;
   {
     const int jfirst = j0 + warp * kRpw + slot;
+    const int idfirst = jfirst < j1 ? parent_id(jfirst) : 0x7fffffff;
     int hi = n_sel_meta;
     while (sp < hi) {
       const int mid = (sp + hi) >> 1;
-      if (sel_meta[mid] < jfirst) sp = mid + 1; else hi = mid;
+      if (sel_meta[mid] < idfirst) sp = mid + 1; else hi = mid;
     }
   }
   for (int jb = j0 + warp * kRpw + slot; jb - slot < j1; jb += kStride * kU) {
@@ -230,12 +244,13 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int j = jb + u * kStride;
-      while (sp < n_sel_meta && sel_meta[sp] < j) ++sp;
-      const bool chosen = sp < n_sel_meta && sel_meta[sp] == j;
+      const int id = j < j1 ? parent_id(j) : 0x7fffffff;
+      while (sp < n_sel_meta && sel_meta[sp] < id) ++sp;
+      const bool chosen = sp < n_sel_meta && sel_meta[sp] == id;
       use[u] = j < j1 && !chosen;
       // every load of the batch is issued before the first is used
-      w[u] = use[u] ? *reinterpret_cast<const uint4 *>(mv + static_cast<size_t>(j) * D + dd) : make_uint4(0, 0, 0, 0);
-      z[u] = use[u] ? __ldcg(ms + j) * kLog2e : 0.f;
+      w[u] = use[u] ? *reinterpret_cast<const uint4 *>(mv + static_cast<size_t>(id) * D + dd) : make_uint4(0, 0, 0, 0);
+      z[u] = use[u] ? (listed ? __ldcg(a.parent_scores + row * a.parent_cap + j) : __ldcg(ms + id)) * kLog2e : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u)
@@ -264,7 +279,7 @@ __global__ void __launch_bounds__(kHgsaThreads) k_hgsa_children(const HgsaArgs a
     }
   }
   __syncthreads();
-  float *rec = a.part + (row * a.n_split + split) * (D + kPartHeader);
+  float *rec = a.part + (row * a.part_stride + a.part_off + split) * (D + kPartHeader);
   float M2 = neg_inf();
 #pragma unroll
   for (int w = 0; w < kHgsaWarps; ++w) M2 = fmaxf(M2, red[w][0]);

@@ -43,6 +43,8 @@ class DecodeConfig:
     # H-GSA
     group: int = 0          # gists per meta-gist; 0 = flat GSA
     topk_meta: int = 0
+    group2: int = 0         # meta-gists per level-2 meta-gist; 0 = one meta level
+    topk_meta2: int = 0
     seed: int = 0
     extra: dict = field(default_factory=dict)
 
@@ -84,9 +86,14 @@ QWEN_16X = DecodeConfig("qwen7b_16x", 4, 28, 4, 128, 16, 131072, 128, "bf16", kv
 QWEN_16X_EXCL = DecodeConfig("qwen7b_16x_excl", 4, 28, 4, 128, 16, 131072, 128, "bf16", kv_std=1 / math.sqrt(128),
                              exclude=True, seed=20260003)
 HGSA_32X = DecodeConfig("hgsa_32x", 2, 32, 8, 128, 32, 524288, 64, "bf16", group=16, topk_meta=32, seed=20260004)
+# H-GSA with a second meta level over the same 512K context: 16 level-1
+# meta-gists per level-2 meta-gist (64 of them); keep 8 level-2 groups, then
+# 32 of their 128 level-1 children, then 64 of those 512 gists.
+HGSA2_32X = DecodeConfig("hgsa2_32x", 2, 32, 8, 128, 32, 524288, 64, "bf16", group=16, topk_meta=32, group2=16,
+                         topk_meta2=8, seed=20260006)
 PREFILL_32K = PrefillConfig("prefill_32k", 1, 28, 4, 128, 16, 2048, 16, "bf16", seed=20260005)
 
-CONFIGS = {c.name: c for c in (PR1, LLAMA_8X, QWEN_16X, QWEN_16X_EXCL, HGSA_32X, PREFILL_32K)}
+CONFIGS = {c.name: c for c in (PR1, LLAMA_8X, QWEN_16X, QWEN_16X_EXCL, HGSA_32X, HGSA2_32X, PREFILL_32K)}
 
 
 def _gen(device, seed):
@@ -123,7 +130,8 @@ def decode_inputs(cfg: DecodeConfig, device="cpu", seed=None, own_len=1, n_max=N
     t_max = t_max or (N + 1) * c
     g = _gen(device, cfg.seed if seed is None else seed)
     dt = DTYPES[cfg.dtype]
-    out = {k: [] for k in ("q", "gist_k", "gist_v", "raw_k", "raw_v", "meta_k", "meta_v", "planted")}
+    out = {k: [] for k in ("q", "gist_k", "gist_v", "raw_k", "raw_v", "meta_k", "meta_v", "meta2_k", "meta2_v",
+                           "planted")}
     counts = list(ragged) if ragged is not None else [N] * B
     for b in range(B):
         raw_k = _randn((hkv, t_max, d), g, device, cfg.kv_std)
@@ -169,6 +177,23 @@ def decode_inputs(cfg: DecodeConfig, device="cpu", seed=None, own_len=1, n_max=N
                         if m // cfg.group < M:
                             meta_k[kv, m // cfg.group] = 0.8 * qdir[kv * G + j] * math.sqrt(d) + 0.1 * _randn(
                                 (d,), g, device)
+            if cfg.group2:
+                # level 2 from level 1 as level 1 from the gists; planted at every level
+                M2_cap, M2 = max(M_cap // cfg.group2, 1), M // cfg.group2
+                meta2_k = torch.zeros((hkv, M2_cap, d), device=device)
+                meta2_v = torch.zeros((hkv, M2_cap, d), device=device)
+                meta2_k[:, :M2] = meta_k[:, : M2 * cfg.group2].reshape(hkv, M2, cfg.group2, d).mean(2) + _randn(
+                    (hkv, M2, d), g, device, 0.5)
+                meta2_v[:, :M2] = meta_v[:, : M2 * cfg.group2].reshape(hkv, M2, cfg.group2, d).mean(2) + _randn(
+                    (hkv, M2, d), g, device, 0.5)
+                if plant and nb > 0:
+                    for kv in range(hkv):
+                        for j in range(G):
+                            m2 = int(out["planted"][-1][kv * G + j]) // cfg.group // cfg.group2
+                            if m2 < M2:
+                                meta2_k[kv, m2] = 0.8 * qdir[kv * G + j] * math.sqrt(d) + 0.1 * _randn((d,), g, device)
+                out["meta2_k"].append(meta2_k.to(dt))
+                out["meta2_v"].append(meta2_v.to(dt))
             out["meta_k"].append(meta_k.to(dt))
             out["meta_v"].append(meta_v.to(dt))
         out["q"].append(q.to(dt))

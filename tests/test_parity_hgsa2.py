@@ -1,0 +1,146 @@
+"""H-GSA with two meta levels (level-2 -> level-1 -> gist -> unfold) on the
+GPU against the float64 oracle, through the C ABI.  Near-ties are resolved
+level by level as for one meta level: where the GPU's choice at a level
+differs from the oracle's only inside the tie window, the oracle is re-run
+with the GPU's choices up to that level (the conditional oracle) before the
+next level and the output are compared."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import TOL, selection_ok
+
+pytestmark = pytest.mark.gpu
+
+W = None
+G = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    global W, G
+    from long_context_gsa_b200 import build
+    build.build_library()
+    import long_context_gsa_b200 as G_
+    import long_context_gsa_b200.workloads as W_
+    W, G = W_, G_
+
+
+def run_gpu(x, cfg, exclude, fused=True):
+    B, hq, d = x["q"].shape
+    hkv, n_max, t_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2]
+    m1_max, m2_max = x["meta_k"].shape[2], x["meta2_k"].shape[2]
+    dt = G.GSA_BF16 if x["q"].dtype == torch.bfloat16 else G.GSA_F32
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, exclude, 0.0, dt, G.GSA_F32)
+    h2 = G.make_h2desc(G.make_hdesc(cfg.group, cfg.topk_meta, m1_max), G.make_hdesc(cfg.group2, cfg.topk_meta2, m2_max))
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_HGSA2, h2), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, hq), dtype=torch.float32, device="cuda")
+    m2 = torch.full((B, hq, cfg.topk_meta2), -9, dtype=torch.int32, device="cuda")
+    m1 = torch.full((B, hq, cfg.topk_meta), -9, dtype=torch.int32, device="cuda")
+    si = torch.full((B, hq, max(cfg.topk, 1)), -9, dtype=torch.int32, device="cuda")
+    ss = torch.empty((B, hq, max(cfg.topk, 1)), dtype=torch.float32, device="cuda")
+    args = (x["q"], x["meta2_k"], x["meta2_v"], x["meta_k"], x["meta_v"], x["gist_k"], x["gist_v"])
+    if fused:
+        G.hgsa2_decode(desc, h2, *args, x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"], out, lse, m2, m1, si, ss,
+                       ws)
+    else:
+        G.hgsa2_select(desc, h2, *args, x["n_gists"], m2, m1, si, ss, ws)
+        G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], si, ss,
+                            G.GSA_PRIOR_NONE if exclude else G.GSA_PRIOR_HGSA2, out, lse, ws)
+    torch.cuda.synchronize()
+    assert G.gsa_workspace_status(ws) == 0
+    return out, lse, m2, m1, si
+
+
+def run_oracle(x, cfg, exclude, rows=None, meta2_sel_in=None, meta_sel_in=None, sel_in=None):
+    tk = W.to_oracle
+    return oracle.get().hgsa2(tk(x["q"]), tk(x["meta2_k"]), tk(x["meta2_v"]), tk(x["meta_k"]), tk(x["meta_v"]),
+                              tk(x["gist_k"]), tk(x["gist_v"]), tk(x["raw_k"]), tk(x["raw_v"]), tk(x["n_gists"]),
+                              tk(x["own_len"]), chunk=cfg.chunk, group1=cfg.group, group2=cfg.group2,
+                              topk2=cfg.topk_meta2, topk1=cfg.topk_meta, topk=cfg.topk, exclude=exclude, rows=rows,
+                              meta2_sel_in=meta2_sel_in, meta_sel_in=meta_sel_in, sel_in=sel_in, want_scores=True)
+
+
+def compare(x, cfg, exclude, fused=True, what=""):
+    out, lse, m2, m1, si = run_gpu(x, cfg, exclude, fused)
+    B, hq, d = x["q"].shape
+    orc = run_oracle(x, cfg, exclude, rows=np.arange(B * hq))
+    g_out = out.reshape(B * hq, d).cpu().numpy()
+    g_m2 = m2.reshape(B * hq, -1).cpu().numpy()
+    g_m1 = m1.reshape(B * hq, -1).cpu().numpy()
+    g_si = si.reshape(B * hq, -1).cpu().numpy()[:, : cfg.topk]
+    dtype = "bf16" if x["q"].dtype == torch.bfloat16 else "f32"
+    worst, exempt = 0.0, 0
+    for r in range(B * hq):
+        ref = {k: v[r:r + 1] for k, v in orc.items()}
+        forced = {}
+        for level, got, key, sc_key, k in (("meta2", g_m2, "meta2_sel", "meta2_scores", cfg.topk_meta2),
+                                           ("meta", g_m1, "meta_sel", "meta_cand_scores", cfg.topk_meta),
+                                           ("gist", g_si, "sel", "cand_scores", cfg.topk)):
+            ok, ex = selection_ok(got[r], ref[key][0], ref[sc_key][0], k)
+            assert ok, f"{what}: {level} selection differs outside the tie window in row {r}"
+            if ex:
+                exempt += 1
+                forced[{"meta2": "meta2_sel_in", "meta": "meta_sel_in", "gist": "sel_in"}[level]] = got[r:r + 1]
+                ref = run_oracle(x, cfg, exclude, rows=[r], **forced)
+            else:
+                forced[{"meta2": "meta2_sel_in", "meta": "meta_sel_in", "gist": "sel_in"}[level]] = None
+        err = np.abs(g_out[r] - ref["out"][0]).max()
+        assert err <= TOL[dtype], f"{what}: row {r} max abs err {err}"
+        worst = max(worst, float(err))
+    return {"max_abs_err": worst, "tie_exempt": exempt}, g_si
+
+
+SMALL = [
+    ("g4_trailing", dict(batch=2, hq=8, hkv=2, d=64, chunk=4, context=4 * (4 * 4 * 6 + 7), group=4, group2=4,
+                         topk_meta=3, topk_meta2=2, topk=5), [103, 70]),
+    ("g16_c32", dict(batch=1, hq=8, hkv=2, d=128, chunk=32, context=32 * (16 * 8 * 10 + 37), group=16, group2=8,
+                     topk_meta=8, topk_meta2=3, topk=16), None),
+    ("g2_1", dict(batch=1, hq=4, hkv=1, d=128, chunk=8, context=8 * 100, group=2, group2=1, topk_meta=6,
+                  topk_meta2=6, topk=6), None),
+    ("k2_ge_M2", dict(batch=1, hq=4, hkv=2, d=64, chunk=8, context=8 * 60, group=4, group2=3, topk_meta=4,
+                      topk_meta2=9, topk=7), None),
+    ("few_gists", dict(batch=2, hq=4, hkv=2, d=128, chunk=16, context=16 * 9, group=4, group2=4, topk_meta=2,
+                       topk_meta2=1, topk=3), [9, 0]),
+]
+
+
+@pytest.mark.parametrize("name,chg,ragged", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_small_bf16(name, chg, ragged, exclude):
+    cfg = W.scaled(W.HGSA2_32X, **chg)
+    x = W.decode_inputs(cfg, device="cuda", own_len=3, ragged=ragged, seed=zlib.crc32(name.encode()))
+    compare(x, cfg, exclude, what=name)
+
+
+def test_small_f32():
+    cfg = W.scaled(W.HGSA2_32X, batch=1, hq=4, hkv=2, d=64, chunk=8, context=8 * (8 * 4 * 5 + 11), group=8, group2=4,
+                   topk_meta=4, topk_meta2=2, topk=9, dtype="f32")
+    x = W.decode_inputs(cfg, device="cuda", own_len=5)
+    compare(x, cfg, False, what="f32")
+    compare(x, cfg, True, what="f32 exclude")
+
+
+def test_select_then_unfold_matches_fused():
+    cfg = W.scaled(W.HGSA2_32X, batch=1, hq=8, hkv=2, context=32 * 16 * 16 * 3)
+    x = W.decode_inputs(cfg, device="cuda", own_len=2)
+    for excl in (False, True):
+        a = run_gpu(x, cfg, excl, fused=True)
+        b = run_gpu(x, cfg, excl, fused=False)
+        assert torch.equal(a[4], b[4]) and torch.equal(a[0], b[0])
+
+
+def test_full_size():
+    """The 512K-context workload with two meta levels; every row is checked."""
+    cfg = W.HGSA2_32X
+    x = W.decode_inputs(cfg, device="cuda")
+    res, sel = compare(x, cfg, False, what="hgsa2_32x")
+    planted = x["planted"].reshape(-1).numpy()
+    recall = np.mean([planted[r] in set(sel[r].tolist()) for r in range(len(planted))])
+    assert recall > 0.9, recall
+    print("hgsa2_32x", res, "planted recall", recall)
