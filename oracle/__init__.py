@@ -71,6 +71,17 @@ class _HgsaArgs(C.Structure):
     ]
 
 
+class _DecodeBwdArgs(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
+        ("n_max", C.c_int32), ("t_max", C.c_int32), ("topk", C.c_int32), ("exclude", C.c_int32),
+        ("dtype", C.c_int32), ("scale", C.c_double),
+        ("q", _vp), ("gist_k", _vp), ("gist_v", _vp), ("raw_k", _vp), ("raw_v", _vp),
+        ("n_gists", _ip), ("own_len", _ip), ("sel_in", _ip), ("d_out", _dp), ("d_q", _dp),
+        ("d_gist_k", _dp), ("d_gist_v", _dp), ("d_raw_k", _dp), ("d_raw_v", _dp),
+    ]
+
+
 class _Hgsa2Args(C.Structure):
     _fields_ = [
         ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
@@ -123,7 +134,7 @@ class Oracle:
         self.path = path
         self.lib = C.CDLL(str(path))
         for name, argt in (("gsa_oracle_decode", _DecodeArgs), ("gsa_oracle_hgsa", _HgsaArgs),
-                           ("gsa_oracle_hgsa2", _Hgsa2Args),
+                           ("gsa_oracle_hgsa2", _Hgsa2Args), ("gsa_oracle_decode_backward", _DecodeBwdArgs),
                            ("gsa_oracle_prefill", _PrefillArgs)):
             fn = getattr(self.lib, name)
             fn.argtypes = [C.POINTER(argt)]
@@ -159,6 +170,30 @@ class Oracle:
                         _dp_(res.get("scores")), set_cap, _ip_(res.get("set_n")), _ip_(res.get("set_kind")),
                         _ip_(res.get("set_idx")), _dp_(res.get("set_w")), n_threads)
         _ok(self.lib.gsa_oracle_decode(C.byref(a)), "decode")
+        return res
+
+    def decode_backward(self, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, sel_in, d_out, *, chunk, topk,
+                        exclude=False, scale=0.0):
+        """Gradients of sum(d_out * out) of a decode step with the given
+        (fixed) selection: d_q [B, Hq, d]; d_gist_k/v, d_raw_k/v shaped like
+        their inputs (float64)."""
+        dtype, arrs = _storage(q, gist_k, gist_v, raw_k, raw_v)
+        q, gist_k, gist_v, raw_k, raw_v = arrs
+        B, Hq, d = q.shape
+        _, Hkv, n_max, _ = gist_k.shape
+        t_max = raw_k.shape[2]
+        _check_shapes(gist_k, (B, Hkv, n_max, d), gist_v, raw_k, raw_v, t_max)
+        sel = _i32(sel_in).reshape(B * Hq, topk) if topk else None
+        g = np.ascontiguousarray(d_out, dtype=np.float64).reshape(B * Hq, d)
+        res = {"d_q": np.zeros((B, Hq, d)), "d_gist_k": np.zeros((B, Hkv, n_max, d)),
+               "d_gist_v": np.zeros((B, Hkv, n_max, d)), "d_raw_k": np.zeros((B, Hkv, t_max, d)),
+               "d_raw_v": np.zeros((B, Hkv, t_max, d))}
+        n_gists, own_len = _i32(n_gists), _i32(own_len)
+        a = _DecodeBwdArgs(B, Hq, Hkv, d, chunk, n_max, t_max, topk, int(bool(exclude)), dtype, float(scale),
+                           _ptr(q), _ptr(gist_k), _ptr(gist_v), _ptr(raw_k), _ptr(raw_v), _ip_(n_gists),
+                           _ip_(own_len), _ip_(sel), g.ctypes.data_as(_dp), _dp_(res["d_q"]), _dp_(res["d_gist_k"]),
+                           _dp_(res["d_gist_v"]), _dp_(res["d_raw_k"]), _dp_(res["d_raw_v"]))
+        _ok(self.lib.gsa_oracle_decode_backward(C.byref(a)), "decode_backward")
         return res
 
     # -------------------------------------------------------------------- topk

@@ -108,6 +108,21 @@ typedef struct {
   int32_t n_threads;
 } orc_hgsa_args;
 
+/* Backward of the decode attention for a fixed selection (the top-k choice
+ * is piecewise constant, so no gradient flows through the scores). */
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk;
+  int32_t n_max, t_max, topk, exclude, dtype;
+  double scale;
+  const void *q, *gist_k, *gist_v, *raw_k, *raw_v;
+  const int32_t *n_gists, *own_len;
+  const int32_t *sel_in;              /* [B*hq][topk] the selection (-1 entries skipped) */
+  const double *d_out;                /* [B*hq][d] */
+  double *d_q;                        /* [B*hq][d] written */
+  double *d_gist_k, *d_gist_v;        /* [B][hkv][n_max][d] accumulated */
+  double *d_raw_k, *d_raw_v;          /* [B][hkv][t_max][d] accumulated */
+} orc_decode_bwd_args;
+
 /* H-GSA with two meta levels: level-1 meta-gist j summarises gists
  * j*group1 .. +group1-1; level-2 meta-gist i summarises level-1 meta-gists
  * i*group2 .. +group2-1. */
@@ -521,6 +536,101 @@ static int check_common(int32_t B, int32_t hq, int32_t hkv, int32_t d, int32_t c
   if (B <= 0 || hq <= 0 || hkv <= 0 || d <= 0 || c <= 0) return ORC_EINVAL;
   if (hq % hkv) return ORC_EINVAL;
   if (dtype != ORC_F32 && dtype != ORC_BF16) return ORC_EINVAL;
+  return ORC_OK;
+}
+
+/* Gradients of one decode row.  With w = softmax(z), z_u = scale q.k_u over
+ * the attended set, o = sum w_u v_u and g = dL/do:
+ *   dL/dv_u = w_u g,  dL/dz_u = w_u (g.v_u - g.o),
+ *   dL/dq = scale sum_u dL/dz_u k_u,  dL/dk_u = scale dL/dz_u q. */
+static int decode_bwd_row(const orc_decode_bwd_args *a, int32_t row) {
+  const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);
+  const int d = a->d, c = a->chunk, dt = a->dtype;
+  const double scale = resolve_scale(a->scale, d);
+  const int32_t N = a->n_gists[b], own = a->own_len[b];
+  const size_t qo = ((size_t)b * a->hq + h) * d;
+  const size_t gbase = ((size_t)b * a->hkv + kvh) * a->n_max;
+  const size_t rbase = ((size_t)b * a->hkv + kvh) * a->t_max;
+  char *chosen = (char *)calloc((size_t)(N > 0 ? N : 1), 1);
+  if (!chosen) return ORC_ENOMEM;
+  for (int32_t i = 0; i < a->topk; ++i) {
+    const int32_t m = a->sel_in[(size_t)row * a->topk + i];
+    if (m >= 0 && m < N) chosen[m] = 1;
+  }
+  tokset_t S = {0};
+  int st = ORC_OK;
+  for (int32_t m = 0; m < N && !st; ++m) {
+    if (chosen[m]) {
+      for (int j = 0; j < c && !st; ++j)
+        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    } else if (!a->exclude) {
+      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+    }
+  }
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  double *dq = a->d_q + (size_t)row * d;
+  for (int i = 0; i < d; ++i) dq[i] = 0.0;
+  if (!st && S.n > 0) {
+    const double *g = a->d_out + (size_t)row * d;
+    double *w = (double *)malloc((size_t)S.n * sizeof(double));
+    double *gv = (double *)malloc((size_t)S.n * sizeof(double));
+    if (!w || !gv) return ORC_ENOMEM;
+    double Z = -INFINITY, denom = 0.0;
+    for (int u = 0; u < S.n; ++u) {
+      w[u] = scale * dot(a->q, qo, S.tok[u].kb, S.tok[u].off, d, dt);
+      if (w[u] > Z) Z = w[u];
+    }
+    for (int u = 0; u < S.n; ++u) {
+      w[u] = exp(w[u] - Z);
+      denom += w[u];
+    }
+    double go = 0.0; /* g.o = sum_u w_u g.v_u */
+    for (int u = 0; u < S.n; ++u) {
+      w[u] /= denom;
+      double x = 0.0;
+      for (int i = 0; i < d; ++i) x += g[i] * elem(S.tok[u].vb, S.tok[u].off + i, dt);
+      gv[u] = x;
+      go += w[u] * x;
+    }
+    for (int u = 0; u < S.n; ++u) {
+      const double dz = w[u] * (gv[u] - go);
+      const int gist = S.tok[u].kind == TOK_GIST;
+      double *dk = (gist ? a->d_gist_k : a->d_raw_k) + S.tok[u].off;
+      double *dv = (gist ? a->d_gist_v : a->d_raw_v) + S.tok[u].off;
+      for (int i = 0; i < d; ++i) {
+        dq[i] += scale * dz * elem(S.tok[u].kb, S.tok[u].off + i, dt);
+        dk[i] += scale * dz * elem(a->q, qo + i, dt);
+        dv[i] += w[u] * g[i];
+      }
+    }
+    free(w);
+    free(gv);
+  }
+  free(S.tok);
+  free(chosen);
+  return st;
+}
+
+/* Rows run one after another: every row adds into the shared key / value
+ * gradients. */
+int gsa_oracle_decode_backward(const orc_decode_bwd_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (a->topk < 0 || !a->q || !a->gist_k || !a->gist_v || !a->raw_k || !a->raw_v || !a->n_gists || !a->own_len)
+    return ORC_EINVAL;
+  if ((a->topk > 0 && !a->sel_in) || !a->d_out || !a->d_q || !a->d_gist_k || !a->d_gist_v || !a->d_raw_k ||
+      !a->d_raw_v)
+    return ORC_EINVAL;
+  for (int b = 0; b < a->batch; ++b) {
+    int32_t N = a->n_gists[b], own = a->own_len[b];
+    if (N < 0 || N > a->n_max || own < 0 || own > a->chunk) return ORC_EINVAL;
+    if ((int64_t)N * a->chunk + own > a->t_max) return ORC_EINVAL;
+  }
+  for (int32_t r = 0; r < a->batch * a->hq; ++r) {
+    const int st = decode_bwd_row(a, r);
+    if (st) return st;
+  }
   return ORC_OK;
 }
 

@@ -635,9 +635,56 @@ def pin_topp_selection(orc):
         assert [int(x) for x in a["sel"][r_][:c]] == [int(x) for x in t[0]]
 
 
+def pin_decode_backward(orc):
+    """Gradients of L = sum(g * out) for a fixed selection: central finite
+    differences of the forward oracle in every input; a single attended
+    token gives d_q = 0, d_v = g, d_k = 0; the value gradients sum to g."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, d, c, N, own, k = 1, 2, 1, 4, 2, 6, 2, 2
+    for exclude in (False, True):
+        arr = rand_decode(rng, B, Hq, Hkv, d, c, N, own)
+        sel = np.array([[1, 4], [3, -1]], np.int32)
+        g = rng.standard_normal((B, Hq, d))
+        grads = orc.decode_backward(arr["q"], arr["gist_k"], arr["gist_v"], arr["raw_k"], arr["raw_v"],
+                                    arr["n_gists"], arr["own_len"], sel, g, chunk=c, topk=k, exclude=exclude)
+
+        def loss(a2):
+            r = run_decode(orc, a2, c, k, exclude, sel_in=sel)
+            return float((r["out"] * g.reshape(B * Hq, d)).sum())
+
+        eps = 1e-2
+        for key, gkey in (("q", "d_q"), ("gist_k", "d_gist_k"), ("gist_v", "d_gist_v"), ("raw_k", "d_raw_k"),
+                          ("raw_v", "d_raw_v")):
+            flat = arr[key].reshape(-1)
+            for _ in range(6):
+                i = int(rng.integers(0, flat.size))
+                a_p, a_m = dict(arr), dict(arr)
+                a_p[key] = flat.copy()
+                a_p[key][i] += eps
+                a_p[key] = a_p[key].reshape(arr[key].shape)
+                a_m[key] = flat.copy()
+                a_m[key][i] -= eps
+                a_m[key] = a_m[key].reshape(arr[key].shape)
+                # the inputs are float32: use the perturbation actually stored
+                h = float(a_p[key].reshape(-1)[i]) - float(a_m[key].reshape(-1)[i])
+                fd = (loss(a_p) - loss(a_m)) / h
+                an = grads[gkey].reshape(-1)[i]
+                assert abs(fd - an) <= 1e-4 + 2e-3 * abs(an), (exclude, key, i, fd, an)
+        # the value gradients of a row sum to its g (softmax weights sum to 1); one kv head here
+        total_v = grads["d_gist_v"].sum(axis=(0, 1, 2)) + grads["d_raw_v"].sum(axis=(0, 1, 2))
+        np.testing.assert_allclose(total_v, g.sum(axis=(0, 1)), rtol=1e-12, atol=1e-12)
+    # a single attended token: the own row alone
+    arr = rand_decode(rng, 1, 1, 1, 3, 2, 0, 1)
+    g = rng.standard_normal((1, 1, 3))
+    gr = orc.decode_backward(arr["q"], arr["gist_k"], arr["gist_v"], arr["raw_k"], arr["raw_v"], arr["n_gists"],
+                             arr["own_len"], np.zeros((1, 0), np.int32), g, chunk=2, topk=0)
+    assert np.abs(gr["d_q"]).max() < 1e-15 and np.abs(gr["d_raw_k"]).max() < 1e-15
+    np.testing.assert_allclose(gr["d_raw_v"][0, 0, 0], g[0, 0], rtol=0, atol=1e-15)
+
+
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
-               pin_decode_golden]
+               pin_decode_golden, pin_decode_backward]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden, pin_hgsa2_bruteforce,
              pin_hgsa2_reduces_to_one_level]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]

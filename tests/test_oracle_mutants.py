@@ -39,6 +39,9 @@ MUTANTS = [
     ("prefill_gist_query_excludes_itself", "for (int32_t t = 0; t <= m && !st; ++t)", "for (int32_t t = 0; t < m && !st; ++t)"),
     ("prefill_chunk_of_position_off_by_one", "const int32_t m = (int32_t)(pos / c), j = (int32_t)(pos % c);",
      "const int32_t m = (int32_t)((pos + 1) / c), j = (int32_t)((pos + 1) % c);"),
+    ("backward_drops_mean_term", "const double dz = w[u] * (gv[u] - go);", "const double dz = w[u] * gv[u];"),
+    ("backward_key_grad_from_key", "dk[i] += scale * dz * elem(a->q, qo + i, dt);",
+     "dk[i] += scale * dz * elem(S.tok[u].kb, S.tok[u].off + i, dt);"),
     ("hgsa2_noncandidate_level1_attended", "if (cand1[j] && !chosen1[j]) st = push(&S, a->meta_k",
      "if (!chosen1[j]) st = push(&S, a->meta_k"),
     ("hgsa2_chosen_level2_attended", "if (!chosen2[i]) st = push(&S, a->meta2_k", "if (1) st = push(&S, a->meta2_k"),
