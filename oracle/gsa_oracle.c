@@ -544,7 +544,8 @@ static int check_common(int32_t B, int32_t hq, int32_t hkv, int32_t d, int32_t c
  *   dL/dv_u = w_u g,  dL/dz_u = w_u (g.v_u - g.o),
  *   dL/dq = scale sum_u dL/dz_u k_u,  dL/dk_u = scale dL/dz_u q. */
 static int decode_bwd_row(const orc_decode_bwd_args *a, int32_t row) {
-  const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);
+  const int b = row / a->hq, h = row % a->hq;
+  const int kvh = h / (a->hq / a->hkv); /* contiguous GQA grouping */
   const int d = a->d, c = a->chunk, dt = a->dtype;
   const double scale = resolve_scale(a->scale, d);
   const int32_t N = a->n_gists[b], own = a->own_len[b];
