@@ -459,6 +459,28 @@ static double resolve_scale(double scale, int d) { return scale > 0.0 ? scale : 
 /* Flat GSA decode, one (b, h) row.                                          */
 /* ------------------------------------------------------------------------ */
 
+/* The attended set of a flat decode row, in interleaved-sequence order:
+ * for each selected chunk its raw rows and its gist, the gist of every
+ * unselected chunk unless `exclude`, then the own raw rows ([ja] 2.1 steps
+ * 3-4, the SG+SR rule). */
+static int decode_set(tokset_t *S, const void *raw_k, const void *raw_v, const void *gist_k, const void *gist_v,
+                      size_t rbase, size_t gbase, int d, int c, int32_t N, int32_t own, int exclude,
+                      const char *chosen) {
+  int st = ORC_OK;
+  for (int32_t m = 0; m < N && !st; ++m) {
+    if (chosen[m]) {
+      for (int j = 0; j < c && !st; ++j)
+        st = push(S, raw_k, raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
+      if (!st) st = push(S, gist_k, gist_v, (gbase + m) * d, TOK_GIST, m);
+    } else if (!exclude) {
+      st = push(S, gist_k, gist_v, (gbase + m) * d, TOK_GIST, m);
+    }
+  }
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(S, raw_k, raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  return st;
+}
+
 static int decode_row(const void *pa, int64_t slot) {
   const orc_decode_args *a = (const orc_decode_args *)pa;
   const int32_t row = a->rows ? a->rows[slot] : (int32_t)slot;
@@ -505,18 +527,7 @@ static int decode_row(const void *pa, int64_t slot) {
 
   /* 3. the attended set, in interleaved-sequence order */
   tokset_t S = {0};
-  int st = ORC_OK;
-  for (int32_t m = 0; m < N && !st; ++m) {
-    if (chosen[m]) {
-      for (int j = 0; j < c && !st; ++j)
-        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
-      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
-    } else if (!a->exclude) {
-      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
-    }
-  }
-  for (int32_t j = 0; j < own && !st; ++j)
-    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  int st = decode_set(&S, a->raw_k, a->raw_v, a->gist_k, a->gist_v, rbase, gbase, d, c, N, own, a->exclude, chosen);
 
   /* 4. exact softmax attention over the set */
   if (!st) {
@@ -559,18 +570,7 @@ static int decode_bwd_row(const orc_decode_bwd_args *a, int32_t row) {
     if (m >= 0 && m < N) chosen[m] = 1;
   }
   tokset_t S = {0};
-  int st = ORC_OK;
-  for (int32_t m = 0; m < N && !st; ++m) {
-    if (chosen[m]) {
-      for (int j = 0; j < c && !st; ++j)
-        st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);
-      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
-    } else if (!a->exclude) {
-      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
-    }
-  }
-  for (int32_t j = 0; j < own && !st; ++j)
-    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  int st = decode_set(&S, a->raw_k, a->raw_v, a->gist_k, a->gist_v, rbase, gbase, d, c, N, own, a->exclude, chosen);
   double *dq = a->d_q + (size_t)row * d;
   for (int i = 0; i < d; ++i) dq[i] = 0.0;
   if (!st && S.n > 0) {

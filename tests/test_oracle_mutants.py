@@ -24,14 +24,14 @@ MUTANTS = [
     ("value_reads_key", "out[i] += w * elem(S->tok[u].vb,", "out[i] += w * elem(S->tok[u].kb,"),
     ("gqa_modulo_mapping", "const int b = row / a->hq, h = row % a->hq, kvh = h / (a->hq / a->hkv);\n  const int d = a->d, c = a->chunk, dt = a->dtype;\n  const double scale = resolve_scale(a->scale, d);\n  const int32_t N = a->n_gists[b], own = a->own_len[b];\n  const size_t qo",
      "const int b = row / a->hq, h = row % a->hq, kvh = h % a->hkv;\n  const int d = a->d, c = a->chunk, dt = a->dtype;\n  const double scale = resolve_scale(a->scale, d);\n  const int32_t N = a->n_gists[b], own = a->own_len[b];\n  const size_t qo"),
-    ("decode_raw_row_off_by_one", "st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);\n      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    } else if (!a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own",
-     "st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)m * c + j + 1) * d, TOK_RAW, m * c + j);\n      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    } else if (!a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own"),
-    ("decode_selected_gist_dropped", "      if (!st) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    } else if (!a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own",
-     "    } else if (!a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own"),
-    ("decode_unselected_gists_dropped", "    } else if (!a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own",
-     "    } else if (a->exclude) {\n      st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);\n    }\n  }\n  for (int32_t j = 0; j < own"),
-    ("decode_first_own_row_dropped", "for (int32_t j = 0; j < own && !st; ++j)\n    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);\n\n  /* 4.",
-     "for (int32_t j = 1; j < own && !st; ++j)\n    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);\n\n  /* 4."),
+    ("decode_raw_row_off_by_one", "st = push(S, raw_k, raw_v, (rbase + (size_t)m * c + j) * d, TOK_RAW, m * c + j);",
+     "st = push(S, raw_k, raw_v, (rbase + (size_t)m * c + j + 1) * d, TOK_RAW, m * c + j);"),
+    ("decode_selected_gist_dropped", "      if (!st) st = push(S, gist_k, gist_v, (gbase + m) * d, TOK_GIST, m);\n    } else if (!exclude) {",
+     "    } else if (!exclude) {"),
+    ("decode_unselected_gists_dropped", "    } else if (!exclude) {\n      st = push(S, gist_k, gist_v,",
+     "    } else if (exclude) {\n      st = push(S, gist_k, gist_v,"),
+    ("decode_first_own_row_dropped", "for (int32_t j = 0; j < own && !st; ++j)\n    st = push(S, raw_k, raw_v,",
+     "for (int32_t j = 1; j < own && !st; ++j)\n    st = push(S, raw_k, raw_v,"),
     ("hgsa_trailing_group_ignored", "if (grp >= M || meta_chosen[grp])", "if (grp < M && meta_chosen[grp])"),
     ("hgsa_unselected_meta_dropped", "if (!meta_chosen[j]) st = push(&S, a->meta_k", "if (meta_chosen[j]) st = push(&S, a->meta_k"),
     ("hgsa_meta_uses_gist_keys", "ms[j] = scale * dot(a->q, qo, a->meta_k,", "ms[j] = scale * dot(a->q, qo, a->gist_k,"),
