@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
@@ -493,6 +493,62 @@ def measure_topp(G, W, cfg, dev, args, flush, hbm, top_p):
                            "unfold_attend": round(float(k[:, 2].mean()) * 1e3, 2)}}
 
 
+def backward_bytes(cfg, x, sel):
+    """Bytes the decode backward must move: every attended key / value row
+    read once (bf16 or fp32) and its fp32 key / value gradient rows read and
+    written once (the gradients accumulate), plus q, out, d_out, lse and the
+    d_q read-modify-write per query head.  The attended rows per (b, kv head)
+    are the gists (all, or the union of the selected ones with exclude), the
+    union of the selected chunks' raw rows and the own rows."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    B, hq, hkv, d, c = cfg.batch, cfg.hq, cfg.hkv, cfg.d, cfg.chunk
+    s = sel.reshape(B, hkv, hq // hkv, -1).cpu()
+    union = sum(int((torch.unique(s[b, kv]) >= 0).sum()) for b in range(B) for kv in range(hkv))
+    own = int(x["own_len"].sum()) * hkv
+    rows = (union if cfg.exclude else B * hkv * cfg.n_gists) + union * c + own
+    return rows * d * (2 * e + 2 * 4 * 2) + B * hq * d * (e + 4 + 4 + 2 * 4) + B * hq * 4
+
+
+def measure_backward(G, W, cfg, dev, args, flush, hbm):
+    """The backward of a decode step for the forward's selection
+    (gsa_decode_backward alone; the forward runs once, untimed, to give the
+    selection, output and lse).  The fp32 gradient buffers accumulate over
+    the timed calls, as in gradient accumulation."""
+    x, desc = decode_setup(G, W, cfg, dev, cfg.seed)
+    B, hq, d = x["q"].shape
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, hq), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device=dev)
+    G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"], out, lse,
+                 sel, ssc, ws)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed + 7)
+    d_out = torch.randn((B, hq, d), generator=gen, dtype=torch.float32, device=dev)
+    grads = [torch.zeros((B, hq, d), dtype=torch.float32, device=dev)] + \
+        [torch.zeros(x[k].shape, dtype=torch.float32, device=dev) for k in ("gist_k", "gist_v", "raw_k", "raw_v")]
+
+    def step(evs):
+        evs[0].record()
+        G.gsa_decode_backward(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"],
+                              x["own_len"], sel, out, lse, d_out, *grads)
+        evs[1].record()
+
+    for _ in range(args.warmup):
+        flush()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    k = timed_steps(step, args.steps, flush, 1)
+    assert G.gsa_workspace_status(ws) == 0, "device status flags set"
+    ms = float(k[:, 0].mean())
+    ab = backward_bytes(cfg, x, sel)
+    del grads
+    return {"metric": "GSA decode backward head-queries/s", "value": round(cfg.head_queries / (ms / 1e3), 1),
+            "unit": UNIT, "ms_per_step": round(ms, 5),
+            "roofline": {"bound": "hbm", "alg_bytes": ab, "achieved_gbs": round(ab / (ms / 1e3) / 1e9, 1),
+                         "peak_gbs": hbm, "frac": round(ab / (ms / 1e3) / 1e9 / hbm, 4)}}
+
+
 def rank_seed(cfg, rank):
     """Each rank draws its own batch of the workload (weak scaling: disjoint
     rows, no data-path exchange)."""
@@ -516,6 +572,10 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
     """The --extra workloads, each against its own roofline (rank 0, one GPU)."""
     extra = {}
     for name in [n for n in args.extra.split(",") if n]:
+        if name.endswith("_bwd"):  # <decode workload>_bwd: the backward of that decode step
+            extra[name] = measure_backward(G, W, W.CONFIGS[name[:-len("_bwd")]], dev, args, flush, hbm)
+            torch.cuda.empty_cache()
+            continue
         if name.endswith("_topp"):  # <decode workload>_topp: the same step with top-p selection, p = 0.1
             # (the softmax over thousands of gists is flat: p = 0.1 keeps from a few chunks up to the cap)
             c = W.CONFIGS[name[:-len("_topp")]]

@@ -233,6 +233,26 @@ gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, const void *g
                               const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
                               void *out, float *lse, int32_t *sel_idx, float *sel_score, void *stream);
 
+/* Backward of a decode step for a fixed selection (selective finetuning
+ * trains through the path; the top-k choice is piecewise constant, so the
+ * gradient flows through the attention over the attended set only).
+ * With w = softmax(z), z_u = scale q.k_u over the set, o = sum w_u v_u and
+ * g = d_out:  dv_u += w_u g;  dk_u += scale w_u (g.v_u - g.o) q;
+ *             d_q += scale sum_u w_u (g.v_u - g.o) k_u.
+ *   sel_idx   [B, hq, topk] the forward's selection (negative entries and
+ *             entries >= N skipped; no chunk listed twice)
+ *   out, lse  the forward's fp32 output [B, hq, d] and lse [B, hq]
+ *   d_out     [B, hq, d] fp32
+ *   d_q [B, hq, d], d_gist_k / d_gist_v [B, hkv, n_max, d], d_raw_k /
+ *   d_raw_v [B, hkv, t_max, d]: fp32, ACCUMULATED (the caller zeroes them;
+ *   the heads of a GQA group add into the same key / value rows).
+ * Needs no workspace. */
+gsa_status gsa_decode_backward(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                               const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
+                               const int32_t *sel_idx, const float *out, const float *lse, const float *d_out,
+                               float *d_q, float *d_gist_k, float *d_gist_v, float *d_raw_k, float *d_raw_v,
+                               void *stream);
+
 /* ---- H-GSA decode: one meta level ([ja] 2.2; [nl] Hierarchische
  * Uitbreiding) -------------------------------------------------------- */
 

@@ -25,7 +25,7 @@ GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
 EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
-    "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
+    "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_decode_backward", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
     "gsa_decode_noalloc",
 )
 
@@ -80,6 +80,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "hgsa_select": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "hgsa_decode": ([D, H, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "hgsa2_select": ([D, C.POINTER(gsa_h2desc)] + [vp] * 13 + [sz, vp], i32),
+        "gsa_decode_backward": ([D] + [vp] * 17, i32),
         "hgsa2_decode": ([D, C.POINTER(gsa_h2desc)] + [vp] * 18 + [sz, vp], i32),
         "gsa_prefill_score": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
@@ -277,6 +278,18 @@ def hgsa2_decode(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist
         _ptr(meta2_idx, torch.int32, "meta2_idx", True), _ptr(meta_idx, torch.int32, "meta_idx", True),
         _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
         _stream(stream)))
+
+
+def gsa_decode_backward(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, sel_idx, out, lse, d_out, d_q,
+                        d_gist_k, d_gist_v, d_raw_k, d_raw_v, stream=None):
+    dt = _TORCH_DT[desc.dtype]
+    f = torch.float32
+    _check("gsa_decode_backward", load().gsa_decode_backward(
+        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
+        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
+        _ptr(own_len, torch.int32, "own_len"), _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(out, f, "out"),
+        _ptr(lse, f, "lse"), _ptr(d_out, f, "d_out"), _ptr(d_q, f, "d_q"), _ptr(d_gist_k, f, "d_gist_k"),
+        _ptr(d_gist_v, f, "d_gist_v"), _ptr(d_raw_k, f, "d_raw_k"), _ptr(d_raw_v, f, "d_raw_v"), _stream(stream)))
 
 
 def gsa_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, ws, stream=None):

@@ -13,6 +13,7 @@
 
 #include "../../include/gsa.h"
 #include "common.cuh"
+#include "k_backward.cuh"
 #include "k_hgsa.cuh"
 #include "k_prefill.cuh"
 #include "k_score.cuh"
@@ -969,6 +970,65 @@ gsa_status hgsa_decode(const gsa_desc *desc, const gsa_hdesc *hdesc, const void 
   const float *pr = desc->exclude_unselected ? nullptr : reinterpret_cast<const float *>(at(ws, L.part_g));
   return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, pr, pr ? hgsa_splits(desc) : 0, out, lse,
                     L, ws, stream);
+}
+
+gsa_status gsa_decode_backward(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                               const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
+                               const int32_t *sel_idx, const float *out, const float *lse, const float *d_out,
+                               float *d_q, float *d_gist_k, float *d_gist_v, float *d_raw_k, float *d_raw_v,
+                               void *stream) {
+  GSA_TRY(check_desc(desc));
+  for (const void *p : {q, gist_k, gist_v, raw_k, raw_v, static_cast<const void *>(n_gists),
+                        static_cast<const void *>(own_len), static_cast<const void *>(out),
+                        static_cast<const void *>(lse), static_cast<const void *>(d_out), static_cast<const void *>(d_q),
+                        static_cast<const void *>(d_gist_k), static_cast<const void *>(d_gist_v),
+                        static_cast<const void *>(d_raw_k), static_cast<const void *>(d_raw_v)})
+    GSA_TRY(need_ptr(p));
+  if (desc->topk > 0) GSA_TRY(need_ptr(sel_idx));
+  BackwardArgs ba;
+  ba.q = q;
+  ba.gist_k = gist_k;
+  ba.gist_v = gist_v;
+  ba.raw_k = raw_k;
+  ba.raw_v = raw_v;
+  ba.n_gists = n_gists;
+  ba.own_len = own_len;
+  ba.sel_idx = sel_idx;
+  ba.k = desc->topk;
+  ba.out = out;
+  ba.lse = lse;
+  ba.d_out = d_out;
+  ba.d_q = d_q;
+  ba.d_gist_k = d_gist_k;
+  ba.d_gist_v = d_gist_v;
+  ba.d_raw_k = d_raw_k;
+  ba.d_raw_v = d_raw_v;
+  ba.hq = desc->hq;
+  ba.hkv = desc->hkv;
+  ba.group = desc->hq / desc->hkv;
+  ba.chunk = desc->chunk;
+  ba.n_max = desc->n_max;
+  ba.t_max = desc->t_max;
+  ba.exclude = desc->exclude_unselected;
+  ba.scale = resolve_scale(desc);
+  // (batch, kv head) pairs, each split into about 4 waves' worth of CTAs in all
+  const int pairs = desc->batch * desc->hkv;
+  const int splits = clampi(cdiv(4 * sm_count(), pairs), 1, 128);
+  const dim3 grid(splits, desc->hkv, desc->batch), block(kBwdWarps * 32);
+  const size_t smem = bwd_smem_bytes(ba.group, desc->d, ba.k);
+  const bool bf = desc->dtype == GSA_BF16;
+  const int gm = ba.group <= 4 ? 4 : (ba.group <= 8 ? 8 : 16);
+#define GSA_BWD_LAUNCH(D_, T_)                                                                         \
+  return gm == 4   ? launch(k_decode_bwd<D_, T_, 4>, grid, block, smem, stream, ba)                   \
+         : gm == 8 ? launch(k_decode_bwd<D_, T_, 8>, grid, block, smem, stream, ba)                   \
+                   : launch(k_decode_bwd<D_, T_, 16>, grid, block, smem, stream, ba)
+  if (desc->d == 64) {
+    if (bf) GSA_BWD_LAUNCH(64, __nv_bfloat16);
+    GSA_BWD_LAUNCH(64, float);
+  }
+  if (bf) GSA_BWD_LAUNCH(128, __nv_bfloat16);
+  GSA_BWD_LAUNCH(128, float);
+#undef GSA_BWD_LAUNCH
 }
 
 gsa_status hgsa2_select(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,
