@@ -719,6 +719,15 @@ gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *
 // Number of partial records per row the scoring pass writes for these shapes.
 int gist_prior_count(const gsa_desc *d) { return plan_score(d, d->n_max, true).splits; }
 
+// Each (batch, kv head) pair is split into the same number of CTAs, chosen
+// so the launch is about kBwdWaves full waves of resident CTAs.
+template <int D, typename T, int GM>
+gsa_status launch_bwd(const BackwardArgs &ba, int B, int hkv, size_t smem, void *stream) {
+  const int slots = resident_ctas(k_decode_bwd<D, T, GM>, kBwdWarps * 32, smem);
+  const int splits = clampi(kBwdWaves * slots / std::max(1, B * hkv), 1, 256);
+  return launch(k_decode_bwd<D, T, GM>, dim3(splits, hkv, B), dim3(kBwdWarps * 32), smem, stream, ba);
+}
+
 }  // namespace
 }  // namespace gsa
 
@@ -1011,17 +1020,14 @@ gsa_status gsa_decode_backward(const gsa_desc *desc, const void *q, const void *
   ba.t_max = desc->t_max;
   ba.exclude = desc->exclude_unselected;
   ba.scale = resolve_scale(desc);
-  // (batch, kv head) pairs, each split into about 4 waves' worth of CTAs in all
-  const int pairs = desc->batch * desc->hkv;
-  const int splits = clampi(cdiv(4 * sm_count(), pairs), 1, 128);
-  const dim3 grid(splits, desc->hkv, desc->batch), block(kBwdWarps * 32);
   const size_t smem = bwd_smem_bytes(ba.group, desc->d, ba.k);
   const bool bf = desc->dtype == GSA_BF16;
   const int gm = ba.group <= 4 ? 4 : (ba.group <= 8 ? 8 : 16);
-#define GSA_BWD_LAUNCH(D_, T_)                                                                         \
-  return gm == 4   ? launch(k_decode_bwd<D_, T_, 4>, grid, block, smem, stream, ba)                   \
-         : gm == 8 ? launch(k_decode_bwd<D_, T_, 8>, grid, block, smem, stream, ba)                   \
-                   : launch(k_decode_bwd<D_, T_, 16>, grid, block, smem, stream, ba)
+  const int B = desc->batch, hkv = desc->hkv;
+#define GSA_BWD_LAUNCH(D_, T_)                                                    \
+  return gm == 4   ? launch_bwd<D_, T_, 4>(ba, B, hkv, smem, stream)              \
+         : gm == 8 ? launch_bwd<D_, T_, 8>(ba, B, hkv, smem, stream)              \
+                   : launch_bwd<D_, T_, 16>(ba, B, hkv, smem, stream)
   if (desc->d == 64) {
     if (bf) GSA_BWD_LAUNCH(64, __nv_bfloat16);
     GSA_BWD_LAUNCH(64, float);

@@ -50,6 +50,12 @@ struct BackwardArgs {
 };
 
 constexpr int kBwdWarps = 4;
+constexpr int kBwdWaves = 4;  // CTAs per launch: about this many full waves
+// Shared-list tokens per lane group per pass: two for groups of up to 4
+// heads; larger groups hold more per-head dq registers, and two tokens would
+// cost a resident CTA per SM (measured slower on the 7-head Qwen shape).
+template <int GM>
+constexpr int bwd_unroll() { return GM <= 4 ? 2 : 1; }
 
 // Dynamic shared memory of k_decode_bwd for a group of G heads, D wide, k
 // selections per head.
@@ -144,18 +150,35 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_decode_bwd(const BackwardArg
   for (int h = 0; h < GM; ++h)
 #pragma unroll
     for (int e = 0; e < kE; ++e) dq[h][e] = 0.f;
-  for (int tb = s0 + warp * kRpw; tb < s1; tb += kBwdWarps * kRpw) {
-    const int t = tb + slot;
-    const bool valid = t < s1;
-    const bool gist = t < n_gs;
-    const size_t r = gist ? gbase + t : rbase + static_cast<size_t>(N) * a.chunk + (t - n_gs);
-    const T *kp = reinterpret_cast<const T *>(gist ? a.gist_k : a.raw_k) + r * D + dd;
-    const T *vp = reinterpret_cast<const T *>(gist ? a.gist_v : a.raw_v) + r * D + dd;
-    float kf[kE], vf[kE], dk[kE], dv[kE];
-    Vec16<T>::unpack(valid ? ldg_nc_v4(kp) : make_uint4(0, 0, 0, 0), kf);
-    Vec16<T>::unpack(valid ? ldg_nc_v4(vp) : make_uint4(0, 0, 0, 0), vf);
+  // kBwdU tokens per lane group per pass: their loads are all in flight
+  // together and each head's q / g slice is read from shared memory once.
+  constexpr int kBwdU = bwd_unroll<GM>();
+  for (int tb = s0 + warp * kRpw * kBwdU; tb < s1; tb += kBwdWarps * kRpw * kBwdU) {
+    float kf[kBwdU][kE], vf[kBwdU][kE], dk[kBwdU][kE], dv[kBwdU][kE];
+    float *dkp[kBwdU], *dvp[kBwdU];
+    bool valid[kBwdU];
 #pragma unroll
-    for (int e = 0; e < kE; ++e) dk[e] = dv[e] = 0.f;
+    for (int u = 0; u < kBwdU; ++u) {
+      const int t = tb + u * kRpw + slot;
+      valid[u] = t < s1;
+      const bool gist = t < n_gs;
+      const size_t r = gist ? gbase + t : rbase + static_cast<size_t>(N) * a.chunk + (t - n_gs);
+      const T *kp = reinterpret_cast<const T *>(gist ? a.gist_k : a.raw_k) + r * D + dd;
+      const T *vp = reinterpret_cast<const T *>(gist ? a.gist_v : a.raw_v) + r * D + dd;
+      dkp[u] = (gist ? a.d_gist_k : a.d_raw_k) + r * D + dd;
+      dvp[u] = (gist ? a.d_gist_v : a.d_raw_v) + r * D + dd;
+      Vec16<T>::unpack(valid[u] ? ldg_nc_v4(kp) : make_uint4(0, 0, 0, 0), kf[u]);
+      Vec16<T>::unpack(valid[u] ? ldg_nc_v4(vp) : make_uint4(0, 0, 0, 0), vf[u]);
+      // the gradient rows' current values, fetched with the keys / values
+      // so that the loads overlap instead of following the arithmetic
+#pragma unroll
+      for (int e = 0; e < kE; e += 4) {
+        const float4 x = valid[u] ? *reinterpret_cast<const float4 *>(dkp[u] + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 y = valid[u] ? *reinterpret_cast<const float4 *>(dvp[u] + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        dk[u][e] = x.x; dk[u][e + 1] = x.y; dk[u][e + 2] = x.z; dk[u][e + 3] = x.w;
+        dv[u][e] = y.x; dv[u][e + 1] = y.y; dv[u][e + 2] = y.z; dv[u][e + 3] = y.w;
+      }
+    }
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
@@ -167,37 +190,39 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_decode_bwd(const BackwardArg
           qh[e] = qv.x; qh[e + 1] = qv.y; qh[e + 2] = qv.z; qh[e + 3] = qv.w;
           gh[e] = gw.x; gh[e + 1] = gw.y; gh[e + 2] = gw.z; gh[e + 3] = gw.w;
         }
-        float qk = 0.f, gv = 0.f;
+        const float lh = lse_s[h], goh = go_s[h];
 #pragma unroll
-        for (int e = 0; e < kE; ++e) {
-          qk = fmaf(qh[e], kf[e], qk);
-          gv = fmaf(gh[e], vf[e], gv);
-        }
+        for (int u = 0; u < kBwdU; ++u) {
+          float qk = 0.f, gv = 0.f;
 #pragma unroll
-        for (int o = 1; o < kLpr; o <<= 1) {
-          qk += __shfl_xor_sync(0xffffffffu, qk, o);
-          gv += __shfl_xor_sync(0xffffffffu, gv, o);
-        }
-        const float w = valid ? exp2f(qk * sl2 - lse_s[h]) : 0.f;
-        const float sdz = a.scale * w * (gv - go_s[h]);
+          for (int e = 0; e < kE; ++e) {
+            qk = fmaf(qh[e], kf[u][e], qk);
+            gv = fmaf(gh[e], vf[u][e], gv);
+          }
 #pragma unroll
-        for (int e = 0; e < kE; ++e) {
-          dq[h][e] = fmaf(sdz, kf[e], dq[h][e]);
-          dk[e] = fmaf(sdz, qh[e], dk[e]);
-          dv[e] = fmaf(w, gh[e], dv[e]);
+          for (int o = 1; o < kLpr; o <<= 1) {
+            qk += __shfl_xor_sync(0xffffffffu, qk, o);
+            gv += __shfl_xor_sync(0xffffffffu, gv, o);
+          }
+          const float w = valid[u] ? exp2f(qk * sl2 - lh) : 0.f;
+          const float sdz = a.scale * w * (gv - goh);
+#pragma unroll
+          for (int e = 0; e < kE; ++e) {
+            dq[h][e] = fmaf(sdz, kf[u][e], dq[h][e]);
+            dk[u][e] = fmaf(sdz, qh[e], dk[u][e]);
+            dv[u][e] = fmaf(w, gh[e], dv[u][e]);
+          }
         }
       }
     }
-    if (valid) {
-      float *dkp = (gist ? a.d_gist_k : a.d_raw_k) + r * D + dd;
-      float *dvp = (gist ? a.d_gist_v : a.d_raw_v) + r * D + dd;
 #pragma unroll
-      for (int e = 0; e < kE; e += 4) {
-        float4 x = *reinterpret_cast<float4 *>(dkp + e), y = *reinterpret_cast<float4 *>(dvp + e);
-        x.x += dk[e]; x.y += dk[e + 1]; x.z += dk[e + 2]; x.w += dk[e + 3];
-        y.x += dv[e]; y.y += dv[e + 1]; y.z += dv[e + 2]; y.w += dv[e + 3];
-        *reinterpret_cast<float4 *>(dkp + e) = x;
-        *reinterpret_cast<float4 *>(dvp + e) = y;
+    for (int u = 0; u < kBwdU; ++u) {
+      if (valid[u]) {
+#pragma unroll
+        for (int e = 0; e < kE; e += 4) {
+          *reinterpret_cast<float4 *>(dkp[u] + e) = make_float4(dk[u][e], dk[u][e + 1], dk[u][e + 2], dk[u][e + 3]);
+          *reinterpret_cast<float4 *>(dvp[u] + e) = make_float4(dv[u][e], dv[u][e + 1], dv[u][e + 2], dv[u][e + 3]);
+        }
       }
     }
   }
