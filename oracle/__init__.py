@@ -82,6 +82,15 @@ class _DecodeBwdArgs(C.Structure):
     ]
 
 
+class _GistStepArgs(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
+        ("n_max", C.c_int32), ("t_max", C.c_int32), ("dtype", C.c_int32), ("scale", C.c_double),
+        ("q", _vp), ("k_new", _vp), ("v_new", _vp), ("gist_k", _vp), ("gist_v", _vp), ("raw_k", _vp),
+        ("raw_v", _vp), ("n_gists", _ip), ("own_len", _ip), ("out", _dp), ("lse", _dp), ("n_threads", C.c_int32),
+    ]
+
+
 class _Hgsa2Args(C.Structure):
     _fields_ = [
         ("batch", C.c_int32), ("hq", C.c_int32), ("hkv", C.c_int32), ("d", C.c_int32), ("chunk", C.c_int32),
@@ -135,6 +144,7 @@ class Oracle:
         self.lib = C.CDLL(str(path))
         for name, argt in (("gsa_oracle_decode", _DecodeArgs), ("gsa_oracle_hgsa", _HgsaArgs),
                            ("gsa_oracle_hgsa2", _Hgsa2Args), ("gsa_oracle_decode_backward", _DecodeBwdArgs),
+                           ("gsa_oracle_gist_step", _GistStepArgs),
                            ("gsa_oracle_prefill", _PrefillArgs)):
             fn = getattr(self.lib, name)
             fn.argtypes = [C.POINTER(argt)]
@@ -194,6 +204,27 @@ class Oracle:
                            _ip_(own_len), _ip_(sel), g.ctypes.data_as(_dp), _dp_(res["d_q"]), _dp_(res["d_gist_k"]),
                            _dp_(res["d_gist_v"]), _dp_(res["d_raw_k"]), _dp_(res["d_raw_v"]))
         _ok(self.lib.gsa_oracle_decode_backward(C.byref(a)), "decode_backward")
+        return res
+
+    def gist_step(self, q, k_new, v_new, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, *, chunk, scale=0.0,
+                  n_threads=0):
+        """Gist-position step at chunk completion: q [B, Hq, d] attends the
+        gists 0..N-1, the own chunk's raw rows and itself (k_new / v_new
+        [B, Hkv, d]).  Returns {"out": [B*Hq, d], "lse": [B*Hq]}."""
+        dtype, arrs = _storage(q, k_new, v_new, gist_k, gist_v, raw_k, raw_v)
+        q, k_new, v_new, gist_k, gist_v, raw_k, raw_v = arrs
+        B, Hq, d = q.shape
+        _, Hkv, n_max, _ = gist_k.shape
+        t_max = raw_k.shape[2]
+        _check_shapes(gist_k, (B, Hkv, n_max, d), gist_v, raw_k, raw_v, t_max)
+        if k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d):
+            raise ValueError("k_new / v_new shape")
+        res = {"out": np.zeros((B * Hq, d)), "lse": np.zeros(B * Hq)}
+        n_gists, own_len = _i32(n_gists), _i32(own_len)
+        a = _GistStepArgs(B, Hq, Hkv, d, chunk, n_max, t_max, dtype, float(scale), _ptr(q), _ptr(k_new), _ptr(v_new),
+                          _ptr(gist_k), _ptr(gist_v), _ptr(raw_k), _ptr(raw_v), _ip_(n_gists), _ip_(own_len),
+                          _dp_(res["out"]), _dp_(res["lse"]), n_threads)
+        _ok(self.lib.gsa_oracle_gist_step(C.byref(a)), "gist_step")
         return res
 
     # -------------------------------------------------------------------- topk

@@ -108,6 +108,22 @@ typedef struct {
   int32_t n_threads;
 } orc_hgsa_args;
 
+/* Gist-position step at chunk completion.  Once the raw tokens of chunk N
+ * are complete, its gist token is decoded under the compression mask ([nl]
+ * Compressie): the gist query sees the raw tokens of its own chunk and the
+ * gists 0..N, the last of which is itself (key / value k_new, v_new, given
+ * per kv head).  Afterwards it is the (N+1)-th completed gist. */
+typedef struct {
+  int32_t batch, hq, hkv, d, chunk, n_max, t_max, dtype;
+  double scale;
+  const void *q;                      /* [batch][hq][d] gist-position queries */
+  const void *k_new, *v_new;          /* [batch][hkv][d] */
+  const void *gist_k, *gist_v, *raw_k, *raw_v;
+  const int32_t *n_gists, *own_len;   /* [batch] */
+  double *out, *lse;                  /* [batch*hq][d], [batch*hq] or NULL */
+  int32_t n_threads;
+} orc_gist_step_args;
+
 /* Backward of the decode attention for a fixed selection (the top-k choice
  * is piecewise constant, so no gradient flows through the scores). */
 typedef struct {
@@ -633,6 +649,46 @@ int gsa_oracle_decode_backward(const orc_decode_bwd_args *a) {
     if (st) return st;
   }
   return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gist-position step, one (b, h) row.                                       */
+/* ------------------------------------------------------------------------ */
+
+/* The set in interleaved-sequence order: the completed gists 0..N-1, the raw
+ * tokens of chunk N (own_len of them; c once the chunk is complete), then
+ * the gist token itself. */
+static int gist_step_row(const void *pa, int64_t row) {
+  const orc_gist_step_args *a = (const orc_gist_step_args *)pa;
+  const int b = (int)(row / a->hq), h = (int)(row % a->hq), kvh = h / (a->hq / a->hkv);
+  const int d = a->d, c = a->chunk, dt = a->dtype;
+  const int32_t N = a->n_gists[b], own = a->own_len[b];
+  const size_t gbase = ((size_t)b * a->hkv + kvh) * a->n_max;
+  const size_t rbase = ((size_t)b * a->hkv + kvh) * a->t_max;
+  tokset_t S = {0};
+  int st = ORC_OK;
+  for (int32_t m = 0; m < N && !st; ++m) st = push(&S, a->gist_k, a->gist_v, (gbase + m) * d, TOK_GIST, m);
+  for (int32_t j = 0; j < own && !st; ++j)
+    st = push(&S, a->raw_k, a->raw_v, (rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);
+  if (!st) st = push(&S, a->k_new, a->v_new, ((size_t)b * a->hkv + kvh) * d, TOK_GIST, N);
+  if (!st)
+    st = attend(a->q, (size_t)row * d, &S, d, dt, resolve_scale(a->scale, d), a->out + (size_t)row * d,
+                a->lse ? a->lse + row : NULL, 0, NULL, NULL, NULL, NULL);
+  free(S.tok);
+  return st;
+}
+
+int gsa_oracle_gist_step(const orc_gist_step_args *a) {
+  if (!a || check_common(a->batch, a->hq, a->hkv, a->d, a->chunk, a->dtype)) return ORC_EINVAL;
+  if (!a->q || !a->k_new || !a->v_new || !a->gist_k || !a->gist_v || !a->raw_k || !a->raw_v || !a->out)
+    return ORC_EINVAL;
+  if (!a->n_gists || !a->own_len) return ORC_EINVAL;
+  for (int b = 0; b < a->batch; ++b) {
+    int32_t N = a->n_gists[b], own = a->own_len[b];
+    if (N < 0 || N >= a->n_max || own < 0 || own > a->chunk) return ORC_EINVAL; /* room for the new gist */
+    if ((int64_t)N * a->chunk + own > a->t_max) return ORC_EINVAL;
+  }
+  return run_pool(gist_step_row, a, (int64_t)a->batch * a->hq, a->n_threads);
 }
 
 int gsa_oracle_decode(const orc_decode_args *a) {

@@ -682,9 +682,64 @@ def pin_decode_backward(orc):
     np.testing.assert_allclose(gr["d_raw_v"][0, 0, 0], g[0, 0], rtol=0, atol=1e-15)
 
 
+def pin_gist_step_is_prefill_gist_row(orc):
+    """The gist-position step at chunk completion equals the prefill oracle's
+    gist row N of the same sequence: chunk N's raw tokens plus gists 0..N,
+    the new gist (k_new, v_new) being gist N ([nl] Compressie)."""
+    rng = np.random.default_rng(41)
+    Hq, Hkv, d, c = 4, 2, 5, 3
+    for N in (0, 1, 4):
+        arr = rand_decode(rng, 1, Hq, Hkv, d, c, N, c)
+        k_new = rng.standard_normal((1, Hkv, d)).astype(np.float32)
+        v_new = rng.standard_normal((1, Hkv, d)).astype(np.float32)
+        res = orc.gist_step(arr["q"], k_new, v_new, arr["gist_k"], arr["gist_v"], arr["raw_k"], arr["raw_v"],
+                            arr["n_gists"], arr["own_len"], chunk=c)
+        Np, L = N + 1, (N + 1) * c
+        q_raw = rng.standard_normal((1, Hq, L, d)).astype(np.float32)
+        q_gist = rng.standard_normal((1, Hq, Np, d)).astype(np.float32)
+        q_gist[:, :, N] = arr["q"]
+        k_gist = np.concatenate([arr["gist_k"][:, :, :N], k_new[:, :, None]], axis=2)
+        v_gist = np.concatenate([arr["gist_v"][:, :, :N], v_new[:, :, None]], axis=2)
+        rows = [h * (L + Np) + L + N for h in range(Hq)]
+        pf = orc.prefill(q_raw, arr["raw_k"][:, :, :L].copy(), arr["raw_v"][:, :, :L].copy(), q_gist, k_gist, v_gist,
+                         chunk=c, topk=1, rows=rows)
+        np.testing.assert_allclose(res["out"], pf["out"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(res["lse"], pf["lse"], rtol=1e-12, atol=1e-12)
+
+
+def pin_gist_step_closed_form(orc):
+    """Dense softmax over the written-out set, including a partial own chunk
+    and GQA heads sharing a kv head; the weights of the set sum to one, so a
+    constant value row is returned unchanged."""
+    rng = np.random.default_rng(42)
+    Hq, Hkv, d, c = 4, 2, 3, 4
+    for N, own in ((0, 4), (2, 1), (3, 4)):
+        arr = rand_decode(rng, 2, Hq, Hkv, d, c, N, own)
+        k_new = rng.standard_normal((2, Hkv, d)).astype(np.float32)
+        v_new = rng.standard_normal((2, Hkv, d)).astype(np.float32)
+        res = orc.gist_step(arr["q"], k_new, v_new, arr["gist_k"], arr["gist_v"], arr["raw_k"], arr["raw_v"],
+                            arr["n_gists"], arr["own_len"], chunk=c)
+        for b in range(2):
+            for h in range(Hq):
+                kv = h // (Hq // Hkv)
+                K = np.concatenate([arr["gist_k"][b, kv, :N], arr["raw_k"][b, kv, N * c:N * c + own],
+                                    k_new[b, kv][None]]).astype(np.float64)
+                V = np.concatenate([arr["gist_v"][b, kv, :N], arr["raw_v"][b, kv, N * c:N * c + own],
+                                    v_new[b, kv][None]]).astype(np.float64)
+                z = (K @ arr["q"][b, h].astype(np.float64)) / math.sqrt(d)
+                w = np.exp(z - z.max())
+                np.testing.assert_allclose(res["out"][b * Hq + h], (w / w.sum()) @ V, rtol=1e-12, atol=1e-12)
+                assert abs(res["lse"][b * Hq + h] - (z.max() + math.log(w.sum()))) < 1e-12
+        const = {k: np.full_like(v, 0.75) for k, v in arr.items() if k in ("gist_v", "raw_v")}
+        r2 = orc.gist_step(arr["q"], k_new, np.full_like(v_new, 0.75), arr["gist_k"], const["gist_v"], arr["raw_k"],
+                           const["raw_v"], arr["n_gists"], arr["own_len"], chunk=c)
+        np.testing.assert_allclose(r2["out"], 0.75, rtol=0, atol=1e-14)
+
+
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
-               pin_decode_golden, pin_decode_backward]
+               pin_decode_golden, pin_decode_backward, pin_gist_step_is_prefill_gist_row,
+               pin_gist_step_closed_form]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden, pin_hgsa2_bruteforce,
              pin_hgsa2_reduces_to_one_level]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]

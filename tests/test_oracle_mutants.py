@@ -52,6 +52,12 @@ MUTANTS = [
     ("topp_unshifted_exponent", "for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s - cand[0].s);",
      "for (int32_t m = 0; m < n; ++m) z += exp(cand[m].s);"),
     ("topk_output_in_rank_order", "while (j > 0 && out[j - 1] > cand[i].m) {", "while (0) {"),
+    ("gist_step_self_dropped", "if (!st) st = push(&S, a->k_new, a->v_new,", "if (0) st = push(&S, a->k_new, a->v_new,"),
+    ("gist_step_own_rows_of_previous_chunk",
+     "(rbase + (size_t)N * c + j) * d, TOK_RAW, N * c + j);\n  if (!st) st = push(&S, a->k_new",
+     "(rbase + (size_t)(N > 0 ? N - 1 : 0) * c + j) * d, TOK_RAW, N * c + j);\n  if (!st) st = push(&S, a->k_new"),
+    ("gist_step_last_gist_dropped", "for (int32_t m = 0; m < N && !st; ++m) st = push(&S, a->gist_k,",
+     "for (int32_t m = 0; m + 1 < N && !st; ++m) st = push(&S, a->gist_k,"),
     ("prefill_ignores_exclude", "} else if (!a->exclude) {\n        st = push(&S, a->k_gist", "} else {\n        st = push(&S, a->k_gist"),
 ]
 
