@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
@@ -549,6 +549,46 @@ def measure_backward(G, W, cfg, dev, args, flush, hbm):
                          "peak_gbs": hbm, "frac": round(ab / (ms / 1e3) / 1e9 / hbm, 4)}}
 
 
+def measure_gist_step(G, W, cfg, dev, args, flush, hbm):
+    """The gist-position step at chunk completion (gsa_gist_step) for every
+    sequence of the workload: append the new gist, attend gists 0..N and the
+    completed chunk's raw rows, advance the counts.  The counts are put back
+    before each step, outside the timed region."""
+    x = W.gist_step_inputs(cfg, device=dev)
+    B, hq, d = x["q"].shape
+    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
+    dt = G.GSA_BF16 if cfg.dtype == "bf16" else G.GSA_F32
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, 0, False, 0.0, dt, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_GIST_STEP), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+    n0, o0 = x["n_gists"].clone(), x["own_len"].clone()
+
+    def step(evs):
+        x["n_gists"].copy_(n0)
+        x["own_len"].copy_(o0)
+        evs[0].record()
+        G.gsa_gist_step(desc, x["q"], x["k_new"], x["v_new"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"],
+                        x["n_gists"], x["own_len"], out, None, ws)
+        evs[1].record()
+
+    for _ in range(args.warmup):
+        flush()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    k = timed_steps(step, args.steps, flush, 1)
+    assert G.gsa_workspace_status(ws) == 0, "device status flags set"
+    ms = float(k[:, 0].mean())
+    e = 2 if cfg.dtype == "bf16" else 4
+    # gists 0..N and the chunk's raw rows (key + value), the new gist read and
+    # written, q in and fp32 out
+    rows = int(n0.sum()) * cfg.hkv + B * cfg.hkv + int(o0.sum()) * cfg.hkv
+    ab = rows * d * e * 2 + B * cfg.hkv * d * e * 2 * 2 + B * hq * d * (e + 4)
+    return {"metric": "GSA gist-position steps (head-queries)/s", "value": round(cfg.head_queries / (ms / 1e3), 1),
+            "unit": UNIT, "ms_per_step": round(ms, 5),
+            "roofline": {"bound": "hbm", "alg_bytes": ab, "achieved_gbs": round(ab / (ms / 1e3) / 1e9, 1),
+                         "peak_gbs": hbm, "frac": round(ab / (ms / 1e3) / 1e9 / hbm, 4)}}
+
+
 def rank_seed(cfg, rank):
     """Each rank draws its own batch of the workload (weak scaling: disjoint
     rows, no data-path exchange)."""
@@ -572,6 +612,10 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
     """The --extra workloads, each against its own roofline (rank 0, one GPU)."""
     extra = {}
     for name in [n for n in args.extra.split(",") if n]:
+        if name.endswith("_giststep"):  # <decode workload>_giststep: chunk completion for every sequence
+            extra[name] = measure_gist_step(G, W, W.CONFIGS[name[:-len("_giststep")]], dev, args, flush, hbm)
+            torch.cuda.empty_cache()
+            continue
         if name.endswith("_bwd"):  # <decode workload>_bwd: the backward of that decode step
             extra[name] = measure_backward(G, W, W.CONFIGS[name[:-len("_bwd")]], dev, args, flush, hbm)
             torch.cuda.empty_cache()

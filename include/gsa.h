@@ -83,7 +83,13 @@ typedef enum gsa_prior {
 } gsa_prior;
 
 /* Workspace sizing: which call sequence the workspace serves. */
-typedef enum gsa_op { GSA_OP_DECODE = 0, GSA_OP_HGSA = 1, GSA_OP_PREFILL = 2, GSA_OP_HGSA2 = 3 } gsa_op;
+typedef enum gsa_op {
+  GSA_OP_DECODE = 0,
+  GSA_OP_HGSA = 1,
+  GSA_OP_PREFILL = 2,
+  GSA_OP_HGSA2 = 3,
+  GSA_OP_GIST_STEP = 4
+} gsa_op;
 
 /* Device-side status bits (gsa_workspace_status). */
 #define GSA_DEVERR_BAD_INDEX 0x1u /* a sel_idx entry >= N was skipped */
@@ -232,6 +238,26 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
 gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
                               const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
                               void *out, float *lse, int32_t *sel_idx, float *sel_score, void *stream);
+
+/* Gist-position step at chunk completion (gist.science/nl/paper/2604.20920,
+ * "Het Proces", Compressie: a gist token sees only its own block and the
+ * gists before it).  For each sequence b with N = n_gists[b] completed
+ * gists and own = own_len[b] raw tokens in chunk N (own = chunk once the
+ * chunk is complete):
+ *   1. the new gist's key / value (k_new, v_new [B, hkv, d], desc->dtype)
+ *      are written at gist row N of gist_k / gist_v;
+ *   2. the gist-position query q [B, hq, d] attends the gists 0..N (the
+ *      last is itself) and raw rows N*chunk .. N*chunk+own-1 with an exact
+ *      softmax: out [B, hq, d] in desc->out_dtype, lse [B, hq] fp32 or NULL;
+ *   3. n_gists[b] becomes N+1 and own_len[b] becomes 0 (device-side).
+ * desc->topk and desc->exclude_unselected are ignored (the mask has no
+ * selection).  Needs N < n_max: a full sequence is flagged
+ * (GSA_DEVERR_CAPACITY), attends gists 0..N-1 and the raw rows, and keeps
+ * its counts.  Workspace: gsa_workspace_bytes(desc, GSA_OP_GIST_STEP, NULL).
+ * gist_k / gist_v / n_gists / own_len are written in place on `stream`. */
+gsa_status gsa_gist_step(const gsa_desc *desc, const void *q, const void *k_new, const void *v_new, void *gist_k,
+                         void *gist_v, const void *raw_k, const void *raw_v, int32_t *n_gists, int32_t *own_len,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /* Backward of a decode step for a fixed selection (selective finetuning
  * trains through the path; the top-k choice is piecewise constant, so the

@@ -14,6 +14,7 @@
 #include "../../include/gsa.h"
 #include "common.cuh"
 #include "k_backward.cuh"
+#include "k_gist_step.cuh"
 #include "k_hgsa.cuh"
 #include "k_prefill.cuh"
 #include "k_score.cuh"
@@ -42,6 +43,7 @@ struct Layout {
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
   size_t meta2_scores = 0, meta2_idx = 0, cand1_scores = 0, cand1_ids = 0, cand1_count = 0;
   size_t pf_stats = 0, pf_gist = 0, pf_vh = 0, pf_ovf = 0;
+  size_t gs_cur = 0, gs_plus = 0;
   size_t total = 0;
 };
 
@@ -123,6 +125,10 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     take(L.cand_ids, rows * cap * 4);
     take(L.cand_count, rows * 4);
     take(L.part_h, rows * kHgsaSplitMax * rec);
+  }
+  if (op == GSA_OP_GIST_STEP) {
+    take(L.gs_cur, static_cast<size_t>(d->batch) * 4);
+    take(L.gs_plus, static_cast<size_t>(d->batch) * 4);
   }
   if (op == GSA_OP_HGSA2 && h) {  // h points at a gsa_h2desc: level1, then level2
     const gsa_hdesc *l2 = h + 1;
@@ -719,6 +725,15 @@ gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *
 // Number of partial records per row the scoring pass writes for these shapes.
 int gist_prior_count(const gsa_desc *d) { return plan_score(d, d->n_max, true).splits; }
 
+// The gist-position step runs the decode path with no selection over the
+// full gist set (the compression mask has no unselected-gist choice).
+gsa_desc gist_step_desc(const gsa_desc *d) {
+  gsa_desc g = *d;
+  g.topk = 0;
+  g.exclude_unselected = 0;
+  return g;
+}
+
 // Each (batch, kv head) pair is split into the same number of CTAs, chosen
 // so the launch is about kBwdWaves full waves of resident CTAs.
 template <int D, typename T, int GM>
@@ -751,7 +766,13 @@ int32_t gsa_version(void) { return 100; }
 
 size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc) {
   if (check_desc(desc) != GSA_OK) return 0;
-  if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL && op != GSA_OP_HGSA2) return 0;
+  if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL && op != GSA_OP_HGSA2 &&
+      op != GSA_OP_GIST_STEP)
+    return 0;
+  if (op == GSA_OP_GIST_STEP) {
+    const gsa_desc g = gist_step_desc(desc);
+    return layout(&g, op, nullptr).total;
+  }
   if (op == GSA_OP_HGSA && check_hdesc(desc, hdesc) != GSA_OK) return 0;
   if (op == GSA_OP_HGSA2 && (!hdesc || check_h2desc(desc, reinterpret_cast<const gsa_h2desc *>(hdesc)) != GSA_OK))
     return 0;
@@ -1035,6 +1056,51 @@ gsa_status gsa_decode_backward(const gsa_desc *desc, const void *q, const void *
   if (bf) GSA_BWD_LAUNCH(128, __nv_bfloat16);
   GSA_BWD_LAUNCH(128, float);
 #undef GSA_BWD_LAUNCH
+}
+
+gsa_status gsa_gist_step(const gsa_desc *desc, const void *q, const void *k_new, const void *v_new, void *gist_k,
+                         void *gist_v, const void *raw_k, const void *raw_v, int32_t *n_gists, int32_t *own_len,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_desc(desc));
+  for (const void *p : {q, k_new, v_new, static_cast<const void *>(gist_k), static_cast<const void *>(gist_v), raw_k,
+                        raw_v, static_cast<const void *>(n_gists), static_cast<const void *>(own_len),
+                        static_cast<const void *>(out), static_cast<const void *>(ws)})
+    GSA_TRY(need_ptr(p));
+  GSA_TRY(opt_ptr(lse));
+  const gsa_desc g = gist_step_desc(desc);
+  const Layout L = layout(&g, GSA_OP_GIST_STEP, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  int32_t *n_cur = reinterpret_cast<int32_t *>(at(ws, L.gs_cur));
+  int32_t *n_plus = reinterpret_cast<int32_t *>(at(ws, L.gs_plus));
+  GistAppendArgs ga;
+  ga.k_new = static_cast<const uint4 *>(k_new);
+  ga.v_new = static_cast<const uint4 *>(v_new);
+  ga.gist_k = static_cast<uint4 *>(gist_k);
+  ga.gist_v = static_cast<uint4 *>(gist_v);
+  ga.n_gists = n_gists;
+  ga.n_cur = n_cur;
+  ga.n_plus = n_plus;
+  ga.hkv = g.hkv;
+  ga.n_max = g.n_max;
+  ga.row_vecs = static_cast<int32_t>(static_cast<size_t>(g.d) * elem_size(g.dtype) / 16);
+  ga.status = status;
+  // 1. the new gist joins the gist arrays at row N (counted as N+1 by the scoring pass)
+  GSA_TRY(launch(k_gist_append, dim3(g.hkv, g.batch), dim3(32), 0, stream, ga));
+  // 2. the compression-mask attention: gists 0..N through the scoring pass's
+  //    partial, chunk N's raw rows through the unfold (no selected chunk)
+  float *scores = reinterpret_cast<float *>(at(ws, L.scores));
+  float *part = reinterpret_cast<float *>(at(ws, L.part_g));
+  int n_prior = 0;
+  GSA_TRY(run_score(&g, q, gist_k, gist_v, n_plus, 1, g.n_max, scores, g.n_max, part, &n_prior, status, stream));
+  if (cudaMemsetAsync(at(ws, L.counters), 0, static_cast<size_t>(g.batch) * g.hq * 4,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  GSA_TRY(run_unfold(&g, q, raw_k, raw_v, gist_v, n_cur, own_len, reinterpret_cast<int32_t *>(at(ws, L.sel_idx)),
+                     reinterpret_cast<float *>(at(ws, L.sel_score)), part, n_prior, out, lse, L, ws, stream));
+  // 3. chunk completion: n_gists = N+1, own_len = 0
+  return launch(k_gist_commit, dim3(cdiv(g.batch, 128)), dim3(128), 0, stream, static_cast<const int32_t *>(n_cur),
+                static_cast<const int32_t *>(n_plus), n_gists, own_len, static_cast<int>(g.batch));
 }
 
 gsa_status hgsa2_select(const gsa_desc *desc, const gsa_h2desc *h2desc, const void *q, const void *meta2_k,

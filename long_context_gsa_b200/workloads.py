@@ -208,6 +208,28 @@ def decode_inputs(cfg: DecodeConfig, device="cpu", seed=None, own_len=1, n_max=N
     return res
 
 
+def gist_step_inputs(cfg: DecodeConfig, device="cpu", seed=None, ragged=None, own_len=None):
+    """Inputs of a gist-position step at chunk completion: the decode inputs
+    with room for one more gist (n_max = N + 1) and a full own chunk
+    (own_len = chunk unless given), plus the new gist's key / value
+    k_new / v_new [B, hkv, d] drawn like the other gists (mean of the
+    chunk's raw rows + N(0, 0.5)).  q is the gist-position query."""
+    c = cfg.chunk
+    x = decode_inputs(cfg, device=device, seed=seed, own_len=c if own_len is None else own_len,
+                      n_max=cfg.n_gists + 1, t_max=(cfg.n_gists + 1) * c, ragged=ragged, plant=False)
+    g = _gen(device, (cfg.seed if seed is None else seed) + 17)
+    dt = DTYPES[cfg.dtype]
+    B, hkv, d = cfg.batch, cfg.hkv, cfg.d
+    k_new = torch.empty((B, hkv, d), device=device)
+    v_new = torch.empty((B, hkv, d), device=device)
+    for b in range(B):
+        N = int(x["n_gists"][b])
+        k_new[b] = x["raw_k"][b, :, N * c:(N + 1) * c].float().mean(1) + _randn((hkv, d), g, device, 0.5)
+        v_new[b] = x["raw_v"][b, :, N * c:(N + 1) * c].float().mean(1) + _randn((hkv, d), g, device, 0.5)
+    x["k_new"], x["v_new"] = k_new.to(dt), v_new.to(dt)
+    return x
+
+
 def pr1_steps(cfg: DecodeConfig = PR1, device="cpu", seed=None):
     """The tiny single-head workload stepped through its decode steps.
 
