@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep,kvreuse_qwen7b",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     return p.parse_args()
@@ -589,6 +589,36 @@ def measure_gist_step(G, W, cfg, dev, args, flush, hbm):
                          "peak_gbs": hbm, "frac": round(ab / (ms / 1e3) / 1e9 / hbm, 4)}}
 
 
+def measure_multiquery(G, W, cfg, dev, args, flush, bf16):
+    """Multi-query scoring against one shared gist cache (KV reuse): every
+    query row of every head scores all N gists on the tensor cores and
+    keeps its top k (gsa_multiquery_select)."""
+    x = W.multiquery_inputs(cfg, device=dev)
+    B, hq, Q, d = x["q"].shape
+    desc = G.make_desc(B, hq, cfg.hkv, d, 1, cfg.n_gists, Q, cfg.topk, False, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_MULTIQUERY), dtype=torch.uint8, device=dev)
+    G.gsa_workspace_init(ws)
+    sel = torch.empty((B, hq, Q, cfg.topk), dtype=torch.int32, device=dev)
+    ssc = torch.empty((B, hq, Q, cfg.topk), dtype=torch.float32, device=dev)
+
+    def step(evs):
+        evs[0].record()
+        G.gsa_multiquery_select(desc, x["q"], x["gist_k"], sel, ssc, ws)
+        evs[1].record()
+
+    for _ in range(args.warmup):
+        flush()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    k = timed_steps(step, args.steps, flush, 1)
+    assert G.gsa_workspace_status(ws) == 0, "device status flags set"
+    ms = float(k[:, 0].mean())
+    tf = cfg.flops / (ms / 1e3) / 1e12
+    return {"metric": "GSA multi-query routing queries/s", "value": round(B * hq * Q / (ms / 1e3), 1),
+            "unit": "query-rows/s", "ms_per_step": round(ms, 5),
+            "roofline": {"bound": "tensor", "flops": cfg.flops, "achieved_tflops": round(tf, 1), "peak_tflops": bf16,
+                         "frac": round(tf / bf16, 4)}}
+
+
 def rank_seed(cfg, rank):
     """Each rank draws its own batch of the workload (weak scaling: disjoint
     rows, no data-path exchange)."""
@@ -627,6 +657,10 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
             torch.cuda.empty_cache()
             continue
         c = W.CONFIGS[name]
+        if name.startswith("kvreuse"):
+            extra[name] = measure_multiquery(G, W, c, dev, args, flush, bf16)
+            torch.cuda.empty_cache()
+            continue
         if name.startswith("prefill"):
             extra[name] = measure_prefill(G, W, c, dev, args, flush, bf16)
         elif c.group2:

@@ -88,7 +88,8 @@ typedef enum gsa_op {
   GSA_OP_HGSA = 1,
   GSA_OP_PREFILL = 2,
   GSA_OP_HGSA2 = 3,
-  GSA_OP_GIST_STEP = 4
+  GSA_OP_GIST_STEP = 4,
+  GSA_OP_MULTIQUERY = 5
 } gsa_op;
 
 /* Device-side status bits (gsa_workspace_status). */
@@ -358,6 +359,24 @@ gsa_status hgsa2_decode(const gsa_desc *desc, const gsa_h2desc *h2desc, const vo
  *   sel_score [B, hq, L, topk] fp32 out. */
 gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void *q_gist, const void *k_gist,
                              int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
+
+
+/* Multi-query scoring against one shared gist cache (KV reuse: several
+ * queries routed over the same document's gists, [ja] section 3 and the
+ * KV-cache reuse experiment).  Every query sees all N = desc->n_max gists
+ * of its document (the cache is complete), scores them with scale * q.k on
+ * the tensor cores (the prefill scoring kernel with the queries placed
+ * after the cache) and keeps the top k.
+ *   desc: batch = documents; t_max = Q, the queries per (document, query
+ *         head); bf16, d = 128, topk 1..16, n_max <= 57968
+ *         (GSA_ERR_UNSUPPORTED otherwise); chunk is ignored.
+ *   q       [B, hq, Q, d]; query head h reads kv head h / (hq / hkv)
+ *   gist_k  [B, hkv, N, d]
+ *   sel_idx [B, hq, Q, topk] int32 out (ascending chunk order),
+ *   sel_score [B, hq, Q, topk] fp32 out.
+ * Workspace: gsa_workspace_bytes(desc, GSA_OP_MULTIQUERY, NULL). */
+gsa_status gsa_multiquery_select(const gsa_desc *desc, const void *q, const void *gist_k, int32_t *sel_idx,
+                                 float *sel_score, void *ws, size_t ws_bytes, void *stream);
 
 /* Stage 2, unfolding + attention for every raw and gist position, given
  * stage 1's selection and the row maxima it left in ws (same ws):

@@ -19,13 +19,13 @@ from .build import LIB
 GSA_OK, GSA_ERR_INVALID_ARG, GSA_ERR_UNSUPPORTED, GSA_ERR_WORKSPACE, GSA_ERR_CUDA, GSA_ERR_TIMEOUT = range(6)
 GSA_F32, GSA_BF16 = 0, 1
 GSA_PRIOR_NONE, GSA_PRIOR_GISTS, GSA_PRIOR_HGSA, GSA_PRIOR_HGSA2 = 0, 1, 2, 3
-GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL, GSA_OP_HGSA2, GSA_OP_GIST_STEP = 0, 1, 2, 3, 4
+GSA_OP_DECODE, GSA_OP_HGSA, GSA_OP_PREFILL, GSA_OP_HGSA2, GSA_OP_GIST_STEP, GSA_OP_MULTIQUERY = 0, 1, 2, 3, 4, 5
 GSA_DEVERR_BAD_INDEX, GSA_DEVERR_TIMEOUT, GSA_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
-    "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_decode_backward", "gsa_gist_step", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
+    "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_decode_backward", "gsa_gist_step", "gsa_multiquery_select", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
     "gsa_decode_noalloc",
 )
 
@@ -82,6 +82,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "hgsa2_select": ([D, C.POINTER(gsa_h2desc)] + [vp] * 13 + [sz, vp], i32),
         "gsa_decode_backward": ([D] + [vp] * 17, i32),
         "gsa_gist_step": ([D] + [vp] * 12 + [sz, vp], i32),
+        "gsa_multiquery_select": ([D] + [vp] * 5 + [sz, vp], i32),
         "hgsa2_decode": ([D, C.POINTER(gsa_h2desc)] + [vp] * 18 + [sz, vp], i32),
         "gsa_prefill_score": ([D, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
@@ -279,6 +280,13 @@ def hgsa2_decode(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist
         _ptr(meta2_idx, torch.int32, "meta2_idx", True), _ptr(meta_idx, torch.int32, "meta_idx", True),
         _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
         _stream(stream)))
+
+
+def gsa_multiquery_select(desc, q, gist_k, sel_idx, sel_score, ws, stream=None):
+    _check("gsa_multiquery_select", load().gsa_multiquery_select(
+        C.byref(desc), _ptr(q, torch.bfloat16, "q"), _ptr(gist_k, torch.bfloat16, "gist_k"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
 
 
 def gsa_gist_step(desc, q, k_new, v_new, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, ws, stream=None):

@@ -101,6 +101,13 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   };
   take(L.status, 256);
   take(L.counters, rows * 4);
+  if (op == GSA_OP_MULTIQUERY) {  // t_max = queries per (document, head)
+    const size_t prow = rows * static_cast<size_t>(d->t_max);
+    take(L.pf_stats, prow * rec);
+    take(L.pf_ovf, prow * 4);
+    L.total = off;
+    return L;
+  }
   if (op == GSA_OP_PREFILL) {
     const size_t prow = rows * static_cast<size_t>(d->t_max);
     take(L.sel_idx, prow * d->topk * 4);
@@ -621,6 +628,17 @@ gsa_status check_prefill(const gsa_desc *d) {
   return GSA_OK;
 }
 
+// Multi-query scoring runs the prefill scoring kernel: bf16, d = 128,
+// topk 1..16, one row of gist scores in shared memory for the exact re-pass.
+gsa_status check_multiquery(const gsa_desc *d) {
+  GSA_TRY(check_desc(d));
+  if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
+  if (d->topk < 1 || d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;
+  if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
+  return GSA_OK;
+}
+
 PrefillArgs prefill_args(const gsa_desc *d, int32_t *sel_idx, float *sel_score, const Layout &L, void *ws) {
   PrefillArgs pa;
   std::memset(&pa, 0, sizeof(pa));
@@ -647,11 +665,19 @@ PrefillArgs prefill_args(const gsa_desc *d, int32_t *sel_idx, float *sel_score, 
   return pa;
 }
 
+// pos0 > 0 (multi-query scoring): the raw rows are queries placed after
+// the whole gist cache, and there are no gist-position rows.
 gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q_gist, const void *k_gist,
-                             int32_t *sel_idx, float *sel_score, const Layout &L, void *ws, void *stream) {
+                             int32_t *sel_idx, float *sel_score, const Layout &L, void *ws, void *stream,
+                             int pos0 = 0) {
   PrefillArgs pa = prefill_args(d, sel_idx, sel_score, L, ws);
+  if (pos0 > 0) {
+    pa.pos0 = pos0;
+    pa.gist_tiles = 0;
+  }
   const uint64_t bh = static_cast<uint64_t>(d->batch) * d->hq, bkv = static_cast<uint64_t>(d->batch) * d->hkv;
-  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, bh * d->n_max, kPfRows) ||
+  const uint64_t qgist_rows = pos0 > 0 ? bh * d->t_max : bh * d->n_max;  // (not read when there are no gist rows)
+  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, qgist_rows, kPfRows) ||
       !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kPfKeys))
     return GSA_ERR_CUDA;
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
@@ -669,6 +695,7 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.chunk = d->chunk;
   sr.n_chunks = d->n_max;
   sr.L = d->t_max;
+  sr.pos0 = pa.pos0;
   sr.topk = d->topk;
   sr.scale = pa.scale;
   sr.sel_idx = sel_idx;
@@ -767,8 +794,9 @@ int32_t gsa_version(void) { return 100; }
 size_t gsa_workspace_bytes(const gsa_desc *desc, int32_t op, const gsa_hdesc *hdesc) {
   if (check_desc(desc) != GSA_OK) return 0;
   if (op != GSA_OP_DECODE && op != GSA_OP_HGSA && op != GSA_OP_PREFILL && op != GSA_OP_HGSA2 &&
-      op != GSA_OP_GIST_STEP)
+      op != GSA_OP_GIST_STEP && op != GSA_OP_MULTIQUERY)
     return 0;
+  if (op == GSA_OP_MULTIQUERY && check_multiquery(desc) != GSA_OK) return 0;
   if (op == GSA_OP_GIST_STEP) {
     const gsa_desc g = gist_step_desc(desc);
     return layout(&g, op, nullptr).total;
@@ -1184,6 +1212,21 @@ gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void
   const Layout L = layout(desc, GSA_OP_PREFILL, nullptr);
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
   return run_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, L, ws, stream);
+}
+
+gsa_status gsa_multiquery_select(const gsa_desc *desc, const void *q, const void *gist_k, int32_t *sel_idx,
+                                 float *sel_score, void *ws, size_t ws_bytes, void *stream) {
+  GSA_TRY(check_multiquery(desc));
+  for (const void *p : {q, gist_k, static_cast<const void *>(sel_idx), static_cast<const void *>(sel_score),
+                        static_cast<const void *>(ws)})
+    GSA_TRY(need_ptr(p));
+  const Layout L = layout(desc, GSA_OP_MULTIQUERY, nullptr);
+  if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
+  // the queries are raw rows of a one-token-per-chunk stream placed after
+  // the N gists, so each sees all of them: chunk = 1, causal offset N
+  gsa_desc m = *desc;
+  m.chunk = 1;
+  return run_prefill_score(&m, q, q, gist_k, sel_idx, sel_score, L, ws, stream, m.n_max);
 }
 
 gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,

@@ -34,6 +34,7 @@ struct PrefillArgs {
   CUtensorMap tm_kgist;  // [B*hkv*N, d], box 256 x 64
   CUtensorMap tm_vgist;  // [B*hkv*N, d] fp16 copy of the gist values, box 128 x 64 (attention stage)
   int32_t bh, hq, hkv, group, chunk, n_chunks, L, topk, exclude;
+  int32_t pos0;          // causal position of raw row 0 (0 in prefill; multi-query rows sit after the cache)
   float scale, scale_log2;
   int32_t *sel_idx;      // [B*hq*L, topk]
   float *sel_score;      // [B*hq*L, topk]
@@ -72,7 +73,7 @@ __device__ __forceinline__ PfTile pf_tile(const PrefillArgs &a, int t) {
     r.bh = u % a.bh;
     r.row0 = (a.raw_tiles - 1 - u / a.bh) * kPfRows;
     const int last = min(a.L - 1, r.row0 + kPfRows - 1);
-    const int visible = min(a.n_chunks, last / a.chunk);    // raw i sees 0..i/c-1
+    const int visible = min(a.n_chunks, (a.pos0 + last) / a.chunk);  // raw i sees 0..i/c-1
     r.n_kt = (visible + kPfKeys - 1) / kPfKeys;
   }
   return r;
@@ -384,7 +385,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       const PfTile tl = pf_tile(a, t);  // (no key tile: every row sees nothing; still written)
       const int row = tl.row0 + r;
       const bool row_ok = row < (tl.is_gist ? a.n_chunks : a.L);
-      const int limit = !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, row / a.chunk));
+      const int limit =
+          !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, (a.pos0 + row) / a.chunk));
       const bool sel_rows = !tl.is_gist && raw_topk;
       const int ksel = min(a.topk, limit);  // entries this row selects
       // ---- pass A: slot maxima ----
@@ -563,7 +565,7 @@ struct SelectRowsArgs {
   const __nv_bfloat16 *q_raw, *k_gist;  // [B*hq*L, 128], [B*hkv*N, 128]
   const int32_t *rows;                  // listed output rows (b*hq + h)*L + pos
   uint32_t *count, *done;               // list length; CTAs finished
-  int32_t group, chunk, n_chunks, L, topk;
+  int32_t group, chunk, n_chunks, L, topk, pos0;
   float scale;
   int32_t *sel_idx;
   float *sel_score;
@@ -583,7 +585,7 @@ __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArg
   for (uint32_t i = blockIdx.x; i < n; i += gridDim.x) {  // one listed row per CTA
     const int orow = a.rows[i];
     const int bh = orow / a.L, pos = orow % a.L;
-    const int limit = min(a.n_chunks, pos / a.chunk);
+    const int limit = min(a.n_chunks, (a.pos0 + pos) / a.chunk);
     const int ksel = min(a.topk, limit);
     if (tid < 128) qs[tid] = __bfloat162float(a.q_raw[static_cast<size_t>(orow) * 128 + tid]);
     __syncthreads();

@@ -76,6 +76,26 @@ class PrefillConfig:
         return self.n_chunks * self.chunk
 
 
+@dataclass(frozen=True)
+class MultiQueryConfig:
+    """Several queries routed over one document's complete gist cache (KV
+    reuse): `queries` query rows per (document, query head)."""
+    name: str
+    batch: int
+    hq: int
+    hkv: int
+    d: int
+    n_gists: int
+    queries: int
+    topk: int
+    dtype: str = "bf16"
+    seed: int = 0
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.batch * self.hq * self.queries * self.n_gists * self.d
+
+
 # The five workloads: a tiny fp32 single-head decode stepped 64 times, two
 # flat decodes at 8x / 16x compression, an H-GSA decode at 32x and a causal
 # prefill.  Seeds are fixed per workload.
@@ -92,8 +112,12 @@ HGSA_32X = DecodeConfig("hgsa_32x", 2, 32, 8, 128, 32, 524288, 64, "bf16", group
 HGSA2_32X = DecodeConfig("hgsa2_32x", 2, 32, 8, 128, 32, 524288, 64, "bf16", group=16, topk_meta=32, group2=16,
                          topk_meta2=8, seed=20260006)
 PREFILL_32K = PrefillConfig("prefill_32k", 1, 28, 4, 128, 16, 2048, 16, "bf16", seed=20260005)
+# KV reuse: a 128K-token document compressed 16x (8192 gists) shared by 4096
+# query rows per head (Qwen2-7B head layout), top-16 routing per query.
+KVREUSE_QWEN = MultiQueryConfig("kvreuse_qwen7b", 1, 28, 4, 128, 8192, 4096, 16, seed=20260007)
 
-CONFIGS = {c.name: c for c in (PR1, LLAMA_8X, QWEN_16X, QWEN_16X_EXCL, HGSA_32X, HGSA2_32X, PREFILL_32K)}
+CONFIGS = {c.name: c for c in (PR1, LLAMA_8X, QWEN_16X, QWEN_16X_EXCL, HGSA_32X, HGSA2_32X, PREFILL_32K,
+                               KVREUSE_QWEN)}
 
 
 def _gen(device, seed):
@@ -264,6 +288,30 @@ def pr1_steps(cfg: DecodeConfig = PR1, device="cpu", seed=None):
                          "own_len": torch.tensor([pos % c + 1], dtype=torch.int32, device=device)})
     static = {"gist_k": gist_k, "gist_v": gist_v, "raw_k": raw_k, "raw_v": raw_v, "planted": planted.cpu()}
     return static, per_step
+
+
+def multiquery_inputs(cfg: MultiQueryConfig, device="cpu", seed=None):
+    """q [B,hq,Q,d] and gist_k [B,hkv,N,d], N(0,1); for each (document, kv
+    head) every query row of its group has one planted gist (drawn among
+    all N) whose key is 0.8*sqrt(d)*qhat + N(0, 0.1^2), as in the decode
+    workloads, so routing has something to find."""
+    B, hq, hkv, d, N, Q = cfg.batch, cfg.hq, cfg.hkv, cfg.d, cfg.n_gists, cfg.queries
+    g = _gen(device, cfg.seed if seed is None else seed)
+    dt = DTYPES[cfg.dtype]
+    q = _randn((B, hq, Q, d), g, device)
+    gk = _randn((B, hkv, N, d), g, device)
+    G = hq // hkv
+    for b in range(B):
+        for kv in range(hkv):
+            # a few planted gists per kv head, each aligned with one query row
+            n_plant = min(N, 8)
+            chunks = torch.randperm(N, generator=g, device=device)[:n_plant].tolist()
+            for j, m in enumerate(chunks):
+                h = kv * G + j % G
+                i = int(torch.randint(0, Q, (1,), generator=g, device=device))
+                qhat = q[b, h, i] / q[b, h, i].norm()
+                gk[b, kv, m] = 0.8 * qhat * math.sqrt(d) + 0.1 * _randn((d,), g, device)
+    return {"q": q.to(dt), "gist_k": gk.to(dt)}
 
 
 def prefill_inputs(cfg: PrefillConfig, device="cpu", seed=None):

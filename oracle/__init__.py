@@ -182,6 +182,24 @@ class Oracle:
         _ok(self.lib.gsa_oracle_decode(C.byref(a)), "decode")
         return res
 
+    def multiquery_select(self, q, gist_k, *, topk, scale=0.0, rows=None, n_threads=0):
+        """Top-k gists of every query against one shared, complete gist cache
+        (KV reuse).  q [B, Hq, Q, d]; query head h reads kv head h / (Hq/Hkv);
+        gist_k [B, Hkv, N, d].  These are the decode oracle's scoring and
+        selection steps with the Q queries of head h taken as query heads
+        h*Q .. h*Q+Q-1 of a group of Q*Hq/Hkv heads (so they read the same
+        kv head h / (Hq/Hkv)), N completed gists and no raw rows.  Row id
+        (b*Hq + h)*Q + i.  Returns the decode result dict (sel in rank order,
+        sel_score, scores; out / lse are those of the compression-only set)."""
+        dtype, arrs = _storage(q, gist_k)
+        q, gist_k = arrs
+        B, Hq, Q, d = q.shape
+        _, Hkv, N, _ = gist_k.shape
+        no_raw = np.zeros((B, Hkv, N, d), dtype=gist_k.dtype)
+        return self.decode(q.reshape(B, Hq * Q, d), gist_k, gist_k, no_raw, no_raw, np.full(B, N, np.int32),
+                           np.zeros(B, np.int32), chunk=1, topk=topk, scale=scale, rows=rows, want_scores=True,
+                           n_threads=n_threads)
+
     def decode_backward(self, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, sel_in, d_out, *, chunk, topk,
                         exclude=False, scale=0.0):
         """Gradients of sum(d_out * out) of a decode step with the given

@@ -736,10 +736,38 @@ def pin_gist_step_closed_form(orc):
         np.testing.assert_allclose(r2["out"], 0.75, rtol=0, atol=1e-14)
 
 
+def pin_multiquery_bruteforce(orc):
+    """Multi-query selection against a shared cache: per query, the k
+    highest scale*q.k over all N gists by (score desc, index asc), found by
+    sorting in numpy; GQA heads read their group's kv head; exact ties go
+    to the lower index."""
+    rng = np.random.default_rng(43)
+    B, Hq, Hkv, Q, N, d, k = 2, 4, 2, 3, 9, 4, 3
+    q = rng.standard_normal((B, Hq, Q, d)).astype(np.float32)
+    gk = rng.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    gk[1, 0, 2] = 10.0 * gk[1, 0, 2] / np.linalg.norm(gk[1, 0, 2])
+    gk[1, 0, 5] = gk[1, 0, 2]  # an exact tie between two gists of one kv head
+    res = orc.multiquery_select(q, gk, topk=k)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // (Hq // Hkv)
+            for i in range(Q):
+                s = (gk[b, kv].astype(np.float64) @ q[b, h, i].astype(np.float64)) / math.sqrt(d)
+                order = np.lexsort((np.arange(N), -s))[:k]
+                r = (b * Hq + h) * Q + i
+                assert list(res["sel"][r]) == order.tolist(), (b, h, i)  # rank order
+                np.testing.assert_allclose(res["scores"][r], s, rtol=1e-12, atol=1e-12)
+    # the tie (the top score of a query along the tied key): the lower index wins when only one fits
+    q1 = np.zeros((1, 1, 1, d), np.float32)
+    q1[0, 0, 0] = gk[1, 0, 2]
+    r1 = orc.multiquery_select(q1, gk[1:2, :1], topk=1)
+    assert list(r1["sel"][0]) == [2]
+
+
 DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_compression_only,
                pin_decode_zero_query, pin_decode_invariants, pin_decode_exact_ties, pin_decode_gqa_mapping,
                pin_decode_golden, pin_decode_backward, pin_gist_step_is_prefill_gist_row,
-               pin_gist_step_closed_form]
+               pin_gist_step_closed_form, pin_multiquery_bruteforce]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden, pin_hgsa2_bruteforce,
              pin_hgsa2_reduces_to_one_level]
 PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]

@@ -1,0 +1,108 @@
+"""Multi-query scoring against one shared gist cache (KV reuse:
+gsa_multiquery_select, the tensor-core scoring kernel with the queries
+placed after the cache) on the GPU against the float64 oracle.
+
+Selections are compared as sets (the GPU lists them in ascending chunk
+order), exactly except inside the oracle's near-tie window; the GPU's fp32
+scores of the chosen gists must match the oracle's to fp32 accumulation
+error.  With exactly representable inputs the tie rule (lower index first)
+is checked exactly."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import selection_ok
+
+pytestmark = pytest.mark.gpu
+
+W = None
+G = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    global W, G
+    from long_context_gsa_b200 import build
+    build.build_library()
+    import long_context_gsa_b200 as G_
+    import long_context_gsa_b200.workloads as W_
+    W, G = W_, G_
+
+
+def run_gpu(q, gk, k):
+    B, hq, Q, d = q.shape
+    hkv, N = gk.shape[1], gk.shape[2]
+    desc = G.make_desc(B, hq, hkv, d, 1, N, Q, k, False, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_MULTIQUERY), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+    sel = torch.full((B, hq, Q, k), -7, dtype=torch.int32, device="cuda")
+    ssc = torch.full((B, hq, Q, k), float("nan"), dtype=torch.float32, device="cuda")
+    G.gsa_multiquery_select(desc, q, gk, sel, ssc, ws)
+    torch.cuda.synchronize()
+    assert G.gsa_workspace_status(ws) == 0
+    return sel.reshape(B * hq * Q, k).cpu().numpy(), ssc.reshape(B * hq * Q, k).cpu().numpy()
+
+
+def compare(q, gk, k, rows=None, exact_ties=False, what=""):
+    sel, ssc = run_gpu(q, gk, k)
+    tk = W.to_oracle
+    n = sel.shape[0]
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    ref = oracle.get().multiquery_select(tk(q), tk(gk), topk=k, rows=rows)
+    N = gk.shape[2]
+    exempt = 0
+    for j, r in enumerate(rows):
+        got = sel[r]
+        assert list(got) == sorted(got[got >= 0].tolist()) + [-1] * int((got < 0).sum()), (what, r, got)
+        if exact_ties:
+            assert {int(x) for x in got if x >= 0} == {int(x) for x in ref["sel"][j] if x >= 0}, (what, r)
+        else:
+            ok, ex = selection_ok(got, ref["sel"][j], ref["scores"][j], k)
+            assert ok, f"{what}: row {r} selection differs outside the tie window"
+            exempt += ex
+        valid = got >= 0
+        assert valid.sum() == min(k, N)
+        np.testing.assert_allclose(ssc[r][valid], ref["scores"][j][got[valid]], rtol=1e-4, atol=1e-4)
+    return exempt
+
+
+CASES = [
+    # name, B, hq, hkv, Q, N, k
+    ("one_head_ragged", 1, 1, 1, 100, 300, 16),
+    ("gqa4_tiles", 2, 8, 2, 256, 1000, 16),
+    ("gqa7_ragged_keys", 1, 28, 4, 200, 128 * 5 + 3, 8),
+    ("k_above_n", 1, 4, 2, 130, 5, 16),
+    ("k1", 1, 4, 4, 64, 700, 1),
+]
+
+
+@pytest.mark.parametrize("name,B,hq,hkv,Q,N,k", CASES, ids=[c[0] for c in CASES])
+def test_random(name, B, hq, hkv, Q, N, k):
+    gen = torch.Generator(device="cuda").manual_seed(zlib.crc32(name.encode()))
+    q = torch.randn((B, hq, Q, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    gk = torch.randn((B, hkv, N, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    compare(q, gk, k, what=name)
+
+
+def test_exact_ties_go_to_lower_index():
+    """Small-integer inputs make every score exact in fp32 and fp64 and
+    produce many equal scores; the set must be the oracle's exactly."""
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    q = torch.randint(-2, 3, (1, 8, 160, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    gk = torch.randint(-1, 2, (1, 2, 900, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    gk[:, :, 600:] = gk[:, :, :300]  # repeated keys: exact ties at every score level
+    compare(q, gk, 16, exact_ties=True, what="ties")
+
+
+def test_full_size_sampled():
+    """The 8192-gist, 4096-query-per-head workload; 600 sampled rows (and
+    every row's ascending order) against the oracle."""
+    cfg = W.KVREUSE_QWEN
+    x = W.multiquery_inputs(cfg, device="cuda")
+    n = cfg.batch * cfg.hq * cfg.queries
+    rows = np.random.default_rng(5).choice(n, size=600, replace=False)
+    exempt = compare(x["q"], x["gist_k"], cfg.topk, rows=np.sort(rows), what=cfg.name)
+    print(cfg.name, "tie-exempt rows", exempt)
