@@ -99,6 +99,10 @@ SMALL = [
     ("k_above_n", dict(batch=2, hq=4, hkv=1, d=128, chunk=8, context=8 * 40, topk=64), [40, 7], 2),
     ("no_gists", dict(batch=2, hq=4, hkv=2, d=64, chunk=8, context=8 * 30, topk=8), [0, 30], 4),
     ("topk0", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, context=8 * 50, topk=0), None, 2),
+    # a 16-head group with 200 selections each: many heads adding into the same rows
+    ("g16_k200", dict(batch=1, hq=32, hkv=2, d=64, chunk=4, context=4 * 400, topk=200), [400], 2),
+    # heads of a group choosing overlapping chunks (few gists, many heads)
+    ("overlap_g7", dict(batch=1, hq=28, hkv=4, d=128, chunk=16, context=16 * 40, topk=16), None, 5),
 ]
 
 
