@@ -110,3 +110,45 @@ def test_binding_refuses_cpu_tensors(lib):
     t = torch.zeros(4)
     with pytest.raises((ValueError, TypeError)):
         gsa_decode(d, t, t, t, t, t, t, t, t, ws=t)
+
+
+def test_workspace_bytes_new_ops(lib):
+    from long_context_gsa_b200 import GSA_OP_DECODE, GSA_OP_GIST_STEP, GSA_OP_MULTIQUERY, gsa_workspace_bytes
+    d = _desc()
+    assert gsa_workspace_bytes(d, GSA_OP_GIST_STEP) > 0
+    # the gist step ignores topk: its workspace does not grow with it
+    assert gsa_workspace_bytes(_desc(topk=512), GSA_OP_GIST_STEP) == gsa_workspace_bytes(_desc(topk=0), GSA_OP_GIST_STEP)
+    mq = _desc(topk=16, t_max=300)
+    assert gsa_workspace_bytes(mq, GSA_OP_MULTIQUERY) > 2 * 8 * 300 * 4
+    assert gsa_workspace_bytes(_desc(topk=16, dtype=0), GSA_OP_MULTIQUERY) == 0  # fp32 inputs: not built
+    assert gsa_workspace_bytes(_desc(topk=17), GSA_OP_MULTIQUERY) == 0
+    assert gsa_workspace_bytes(_desc(topk=0), GSA_OP_MULTIQUERY) == 0
+    assert gsa_workspace_bytes(d, 99) == 0
+    assert gsa_workspace_bytes(d, GSA_OP_DECODE) > 0
+
+
+@cpu_only
+def test_new_entry_points_reject_bad_arguments(lib):
+    d = _desc()
+    f = C.c_float
+    # top-p: NaN threshold, k beyond 256
+    assert lib.gsa_topp_select(C.byref(d), A, A, f(float("nan")), A, A, A, A, 1 << 40, None) == 1
+    assert lib.gsa_topp_select(C.byref(_desc(topk=300)), A, A, f(0.5), A, A, A, A, 1 << 40, None) == 2
+    # backward: a missing gradient buffer, a misaligned one, a bad descriptor
+    args = [A] * 16
+    bad = list(args)
+    bad[13] = None  # d_gist_k
+    assert lib.gsa_decode_backward(C.byref(d), *bad, None) == 1
+    bad = list(args)
+    bad[12] = A + 4  # d_q
+    assert lib.gsa_decode_backward(C.byref(d), *bad, None) == 1
+    assert lib.gsa_decode_backward(C.byref(_desc(d=96)), *args, None) == 2
+    # gist step: a missing count array, a workspace too small
+    assert lib.gsa_gist_step(C.byref(d), A, A, A, A, A, A, A, None, A, A, None, A, 1 << 40, None) == 1
+    assert lib.gsa_gist_step(C.byref(d), A, A, A, A, A, A, A, A, A, A, None, A, 256, None) == 3
+    # multi-query: unsupported head size / k, missing output, small workspace
+    mq = _desc(topk=16, t_max=300)
+    assert lib.gsa_multiquery_select(C.byref(_desc(d=64, topk=16)), A, A, A, A, A, 1 << 40, None) == 2
+    assert lib.gsa_multiquery_select(C.byref(_desc(topk=20)), A, A, A, A, A, 1 << 40, None) == 2
+    assert lib.gsa_multiquery_select(C.byref(mq), A, A, None, A, A, 1 << 40, None) == 1
+    assert lib.gsa_multiquery_select(C.byref(mq), A, A, A, A, A, 1024, None) == 3
