@@ -615,7 +615,9 @@ gsa_status run_hgsa2_select(const gsa_desc *d, const gsa_h2desc *h2, const void 
 // Words of the 256-byte status block used by the prefill overflow list
 // (word 0 is the device status; all are zeroed by gsa_workspace_init).
 constexpr int kPfOvfCountWord = 16, kPfOvfDoneWord = 17;
-constexpr int kPfSelectMaxChunks = (227 << 10) / 4 - 128 - kPfTopkMax;
+// the exact per-row pass holds a row's scores, the query and its picks in
+// dynamic shared memory next to the warps' pick lists (static)
+constexpr int kPfSelectMaxChunks = (227 << 10) / 4 - 128 - kPfTopkMax - (2 * kSelWarps * kPfTopkMax + 32);
 
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
@@ -702,7 +704,7 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.sel_score = sel_score;
   sr.rec_raw = pa.rec_raw;
   sr.scale_log2 = pa.scale_log2;
-  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(256),
+  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(kSelThreads),
                 (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4, stream, sr);
 }
 

@@ -573,10 +573,13 @@ struct SelectRowsArgs {
   float scale_log2;
 };
 
-__global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArgs a) {
+constexpr int kSelThreads = 1024;  // k_prefill_select_rows: a whole block per listed row
+constexpr int kSelWarps = kSelThreads / 32;
+
+__global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const SelectRowsArgs a) {
   extern __shared__ float sc[];  // [n_chunks] scores, then [128] query
-  __shared__ float rv[8];
-  __shared__ int ri[8];
+  __shared__ float wl_v[kSelWarps * kPfTopkMax];  // each warp's best ksel (score, index)
+  __shared__ int wl_i[kSelWarps * kPfTopkMax];
   __shared__ int picks[32];
   pdl_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -589,62 +592,127 @@ __global__ void __launch_bounds__(256) k_prefill_select_rows(const SelectRowsArg
     const int ksel = min(a.topk, limit);
     if (tid < 128) qs[tid] = __bfloat162float(a.q_raw[static_cast<size_t>(orow) * 128 + tid]);
     __syncthreads();
-    // thread t scores keys t, t + 256, ...: whole dot products, 16 independent loads each
+    // Scores: 16 lanes per key (8 elements each, the query slice in
+    // registers), so a warp reads two whole keys (512 contiguous bytes) per
+    // load; eight such loads are issued before the arithmetic.
     const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128;
-    for (int t = tid; t < limit; t += 256) {
-      const uint4 *kr = reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(t) * 128);
-      uint4 w[16];
+    {
+      const int sub = lane & 15, half = lane >> 4;
+      float qv[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) w[c] = kr[c];
-      float s = 0.f;
+      for (int e = 0; e < 8; ++e) qv[e] = qs[8 * sub + e];
+      constexpr int kU = 8;
+      for (int j0 = 0; j0 * 2 * kSelWarps < limit; j0 += kU) {
+        uint4 w[kU];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float f[8];
-        Vec16<__nv_bfloat16>::unpack(w[c], f);
+        for (int u = 0; u < kU; ++u) {
+          const int t = ((j0 + u) * kSelWarps + warp) * 2 + half;
+          w[u] = t < limit ? ldg_nc_v4(kb + static_cast<size_t>(t) * 128 + 8 * sub) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(qs[8 * c + e], f[e], s);
+        for (int u = 0; u < kU; ++u) {
+          const int t = ((j0 + u) * kSelWarps + warp) * 2 + half;
+          float f[8];
+          Vec16<__nv_bfloat16>::unpack(w[u], f);
+          float s = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s = fmaf(qv[e], f[e], s);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (sub == 0 && t < limit) sc[t] = s;
+        }
       }
-      sc[t] = s;
     }
     __syncthreads();
-    // k rounds of a block argmax by (score desc, index asc)
-    for (int it = 0; it < ksel; ++it) {
-      float bv = neg_inf();
-      int bi = 0x7fffffff;
-      for (int t = tid; t < limit; t += 256) {
+    // Top ksel by (score desc, index asc), in two levels of argmax rounds
+    // that stay inside a warp: warp w takes keys w*32 + lane + kSelThreads j
+    // (each lane keeps its best untaken key and rescans after losing it)
+    // and lists its ksel best; warp 0 then picks the row's ksel from the
+    // warps' lists.  Equal scores keep the lower index at every step.
+    auto better = [](float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); };
+    auto lane_best = [&](float &bv, int &bi) {
+      bv = neg_inf();
+      bi = 0x7fffffff;
+      for (int t = warp * 32 + lane; t < limit; t += kSelThreads) {
         const float v = sc[t];
         if (v > bv) {  // t increases: equal scores keep the lower index
           bv = v;
           bi = t;
         }
       }
+    };
+    {
+      float bv;
+      int bi;
+      lane_best(bv, bi);
+      for (int it = 0; it < ksel; ++it) {
+        float wv = bv;
+        int wi = bi;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
+          if (better(ov, oi, wv, wi)) {
+            wv = ov;
+            wi = oi;
+          }
+        }
+        if (lane == 0) {
+          wl_v[warp * kPfTopkMax + it] = wv;
+          wl_i[warp * kPfTopkMax + it] = wi;
+        }
+        if (wi == bi && wi != 0x7fffffff) {  // this lane's key was taken: its next best
+          sc[bi] = neg_inf();
+          lane_best(bv, bi);
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds list entries l, l + 32, ... of the kSelWarps x 16 slots
+      constexpr int kPer = kSelWarps * kPfTopkMax / 32;
+      float cv[kPer];
+      int ci[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int e = lane + 32 * u, it = e % kPfTopkMax;
+        const bool in = it < ksel;
+        cv[u] = in ? wl_v[e] : neg_inf();
+        ci[u] = in ? wl_i[e] : 0x7fffffff;
+      }
+      for (int it = 0; it < ksel; ++it) {
+        float wv = cv[0];
+        int wi = ci[0];
+#pragma unroll
+        for (int u = 1; u < kPer; ++u)
+          if (better(cv[u], ci[u], wv, wi)) {
+            wv = cv[u];
+            wi = ci[u];
+          }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
+          if (better(ov, oi, wv, wi)) {
+            wv = ov;
+            wi = oi;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u)
+          if (ci[u] == wi) {  // taken (indices are distinct)
+            cv[u] = neg_inf();
+            ci[u] = 0x7fffffff;
+          }
+        if (lane == 0) {
+          const bool ok = wi < limit;  // false only for non-finite scores
+          picks[it] = ok ? wi : 0x7fffffff;
+          qs[128 + it] = wv;  // pick scores follow the query
         }
       }
-      if (lane == 0) {
-        rv[warp] = bv;
-        ri[warp] = bi;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        for (int w = 1; w < 8; ++w)
-          if (rv[w] > bv || (rv[w] == bv && ri[w] < bi)) {
-            bv = rv[w];
-            bi = ri[w];
-          }
-        const bool ok = bi < limit;  // false only for non-finite scores
-        picks[it] = ok ? bi : 0x7fffffff;
-        if (ok) sc[bi] = neg_inf();  // taken
-        qs[128 + it] = bv;           // pick scores follow the query
-      }
-      __syncthreads();
     }
+    __syncthreads();
     // the first pick is the row maximum
     if (tid == 0)
       a.rec_raw[static_cast<size_t>(orow) * (128 + kPartHeader)] = ksel > 0 ? qs[128] * a.scale_log2 : neg_inf();
