@@ -556,11 +556,12 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
 // ---------------------------------------------------------------------------
 // Stage 1b, k_prefill_select_rows: the exact selection of the rows that
 // k_prefill_score listed (a full candidate column, or scores equal to the
-// k-th at the boundary; a handful of rows for most inputs).  One CTA per
-// listed row: its visible gist scores go to shared memory (each thread a
-// whole dot product per key), then k rounds of a block argmax by (score
-// desc, index asc) pick the row's top k, written in ascending chunk order.
-// The last CTA re-arms the list counter for the next call.
+// k-th at the boundary; a handful of rows for most inputs).  One CTA of
+// 1024 threads per listed row: its visible gist scores go to shared memory
+// (16 lanes per key), each warp picks its k best of its keys by rounds of
+// a warp argmax by (score desc, index asc), warp 0 picks the row's k from
+// the warps' lists, and they are written in ascending chunk order.  The
+// last CTA re-arms the list counter for the next call.
 struct SelectRowsArgs {
   const __nv_bfloat16 *q_raw, *k_gist;  // [B*hq*L, 128], [B*hkv*N, 128]
   const int32_t *rows;                  // listed output rows (b*hq + h)*L + pos
