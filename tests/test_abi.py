@@ -152,3 +152,19 @@ def test_new_entry_points_reject_bad_arguments(lib):
     assert lib.gsa_multiquery_select(C.byref(_desc(topk=20)), A, A, A, A, A, 1 << 40, None) == 2
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, None, A, A, 1 << 40, None) == 1
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, A, A, A, 1024, None) == 3
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """The binding has no fallback: a missing libgsa.so is an error naming the build step."""
+    from long_context_gsa_b200 import _abi
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _abi.load(tmp_path / "libgsa.so")
+
+
+def test_product_path_does_not_import_the_oracle():
+    """Only tests, smoke() and the benchmark's CPU leg may touch oracle/: the
+    package's sources never import it."""
+    pkg = ROOT / "long_context_gsa_b200"
+    for f in list(pkg.glob("*.py")) + list((pkg / "csrc").glob("*")):
+        text = f.read_text(errors="ignore")
+        assert "import oracle" not in text and "from oracle" not in text and "gsa_oracle" not in text, f
