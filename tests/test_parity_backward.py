@@ -170,3 +170,16 @@ def test_full_size_sampled_batches(excl):
         ref = run_oracle(x, cfg, excl, sel, d_out, batches=bsel)
         res = compare(got, ref, "bf16", f"llama1b_8x batch {bsel}", batches=bsel)
     print("llama1b_8x backward", "exclude" if excl else "default", res)
+
+
+def test_full_size_qwen_one_batch():
+    """The 128K-context Qwen-shaped workload (7 query heads per kv head, d = 128,
+    top-128 of 8192 chunks of 16) on the GPU; the oracle recomputes batch 0's
+    gradients, every element of which is compared."""
+    cfg = W.QWEN_16X
+    x = W.decode_inputs(cfg, device="cuda")
+    d_out = d_out_for(x, 123)
+    got, sel = run_gpu(x, cfg, False, d_out)
+    ref = run_oracle(x, cfg, False, sel, d_out, batches=[0])
+    res = compare(got, ref, "bf16", "qwen7b_16x batch 0", batches=[0])
+    print("qwen7b_16x backward", res)
