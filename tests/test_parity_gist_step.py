@@ -165,9 +165,12 @@ def test_chunk_completion_loop():
         assert x["n_gists"].cpu().tolist() == [41 + step, 8 + step]
 
 
-def test_full_size_llama_shape():
-    """Chunk completion for every sequence of the 32K-context, batch-16
-    Llama-shaped workload; every row is compared."""
-    x = W.gist_step_inputs(W.LLAMA_8X, device="cuda")
-    err = check(x, W.LLAMA_8X, "llama1b_8x gist step")
-    print("llama1b_8x gist step max abs err", err)
+@pytest.mark.parametrize("name", ["llama1b_8x", "qwen7b_16x"])
+def test_full_size(name):
+    """Chunk completion for every sequence of the full-size decode workloads
+    (32K context, batch 16, GQA 4; 128K context, batch 4, GQA 7); every row
+    is compared."""
+    cfg = W.CONFIGS[name]
+    x = W.gist_step_inputs(cfg, device="cuda")
+    err = check(x, cfg, name + " gist step")
+    print(name, "gist step max abs err", err)
