@@ -134,3 +134,39 @@ def test_topp_decode_step():
                               sel_in=sel.cpu().numpy().reshape(B * hq, cfg.topk))
     err = np.abs(out.cpu().numpy().reshape(B * hq, d) - orc["out"]).max()
     assert err <= TOL["bf16"], err
+
+
+def test_topp_full_size_decode():
+    """The full-size 32K-context, batch-16 decode with top-p (p = 0.1, at
+    most 64 chunks): every row's selection against the oracle's top-p step
+    on the GPU's scores, and every row's output against the oracle run with
+    the GPU's selection."""
+    from _parity import TOL
+    cfg = W.LLAMA_8X
+    x = W.decode_inputs(cfg, device="cuda")
+    B, hq, d = x["q"].shape
+    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, False, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+    scores = torch.empty((B, hq, n_max), dtype=torch.float32, device="cuda")
+    sel = torch.empty((B, hq, cfg.topk), dtype=torch.int32, device="cuda")
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device="cuda")
+    cnt = torch.empty((B, hq), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
+    G.gsa_score_gists(desc, x["q"], x["gist_k"], x["gist_v"], x["n_gists"], scores, ws)
+    G.gsa_topp_select(desc, scores, x["n_gists"], 0.1, sel, ssc, cnt, ws)
+    G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
+                        G.GSA_PRIOR_GISTS, out, None, ws)
+    torch.cuda.synchronize()
+    assert G.gsa_workspace_status(ws) == 0
+    ng = x["n_gists"].cpu().tolist()
+    _check(scores.cpu().numpy(), ng, hq, cfg.topk, 0.1, sel.cpu().numpy().reshape(B * hq, -1),
+           ssc.cpu().numpy().reshape(B * hq, -1), cnt.cpu().numpy().reshape(-1))
+    tk = W.to_oracle
+    orc = oracle.get().decode(tk(x["q"]), tk(x["gist_k"]), tk(x["gist_v"]), tk(x["raw_k"]), tk(x["raw_v"]),
+                              tk(x["n_gists"]), tk(x["own_len"]), chunk=cfg.chunk, topk=cfg.topk,
+                              sel_in=sel.cpu().numpy().reshape(B * hq, cfg.topk))
+    err = np.abs(out.cpu().numpy().reshape(B * hq, d) - orc["out"]).max()
+    assert err <= TOL["bf16"], err
+    print("llama1b_8x top-p decode: max abs err", err, "chunks mean", float(cnt.float().mean()))
