@@ -125,11 +125,12 @@ def test_select_then_unfold_matches_fused():
         assert torch.equal(a[3], b[3]) and torch.equal(a[0], b[0])
 
 
-def test_full_size():
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_full_size(exclude):
     """The 512K-context, 32x-compression H-GSA workload; every row is checked."""
     cfg = W.HGSA_32X
     x = W.decode_inputs(cfg, device="cuda")
-    res, sel = compare(x, cfg, False, what="hgsa_32x")
+    res, sel = compare(x, cfg, exclude, what="hgsa_32x exclude" if exclude else "hgsa_32x")
     planted = x["planted"].reshape(-1).numpy()
     recall = np.mean([planted[r] in set(sel[r].tolist()) for r in range(len(planted))])
     assert recall > 0.9, recall

@@ -135,11 +135,12 @@ def test_select_then_unfold_matches_fused():
         assert torch.equal(a[4], b[4]) and torch.equal(a[0], b[0])
 
 
-def test_full_size():
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_full_size(exclude):
     """The 512K-context workload with two meta levels; every row is checked."""
     cfg = W.HGSA2_32X
     x = W.decode_inputs(cfg, device="cuda")
-    res, sel = compare(x, cfg, False, what="hgsa2_32x")
+    res, sel = compare(x, cfg, exclude, what="hgsa2_32x exclude" if exclude else "hgsa2_32x")
     planted = x["planted"].reshape(-1).numpy()
     recall = np.mean([planted[r] in set(sel[r].tolist()) for r in range(len(planted))])
     assert recall > 0.9, recall
