@@ -104,7 +104,8 @@ def test_topp_matches_oracle(name, B, hq, n_max, k, ng, dist, top_p):
     _check(s, ng, hq, k, top_p, got, got_s, got_c)
 
 
-def test_topp_decode_step():
+@pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
+def test_topp_decode_step(exclude):
     """score -> top-p -> unfold on a small bf16 decode problem; the output
     is compared with the oracle run on the GPU's (variable-length) selection."""
     from _parity import TOL
@@ -112,7 +113,7 @@ def test_topp_decode_step():
     x = W.decode_inputs(cfg, device="cuda", seed=zlib.crc32(b"topp_decode"))
     B, hq, d = x["q"].shape
     n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
-    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, False, 0.0, G.GSA_BF16, G.GSA_F32)
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, exclude, 0.0, G.GSA_BF16, G.GSA_F32)
     ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device="cuda")
     G.gsa_workspace_init(ws)
     scores = torch.empty((B, hq, n_max), dtype=torch.float32, device="cuda")
@@ -123,14 +124,14 @@ def test_topp_decode_step():
     G.gsa_score_gists(desc, x["q"], x["gist_k"], x["gist_v"], x["n_gists"], scores, ws)
     G.gsa_topp_select(desc, scores, x["n_gists"], 0.8, sel, ssc, cnt, ws)
     G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
-                        G.GSA_PRIOR_GISTS, out, None, ws)
+                        G.GSA_PRIOR_NONE if exclude else G.GSA_PRIOR_GISTS, out, None, ws)
     torch.cuda.synchronize()
     assert G.gsa_workspace_status(ws) == 0
     c = cnt.cpu().numpy().reshape(-1)
     assert (c >= 1).all() and (c <= cfg.topk).all()
     tk = W.to_oracle
     orc = oracle.get().decode(tk(x["q"]), tk(x["gist_k"]), tk(x["gist_v"]), tk(x["raw_k"]), tk(x["raw_v"]),
-                              tk(x["n_gists"]), tk(x["own_len"]), chunk=cfg.chunk, topk=cfg.topk,
+                              tk(x["n_gists"]), tk(x["own_len"]), chunk=cfg.chunk, topk=cfg.topk, exclude=exclude,
                               sel_in=sel.cpu().numpy().reshape(B * hq, cfg.topk))
     err = np.abs(out.cpu().numpy().reshape(B * hq, d) - orc["out"]).max()
     assert err <= TOL["bf16"], err
