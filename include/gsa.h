@@ -239,6 +239,17 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
 gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
                               const void *raw_k, const void *raw_v, const int32_t *n_gists, const int32_t *own_len,
                               void *out, float *lse, int32_t *sel_idx, float *sel_score, void *stream);
+/* Device-side status of the last gsa_decode_noalloc call(s) on the current
+ * device: synchronises `stream`, copies the GSA_DEVERR_* bits the kernels
+ * left in the built-in scratch array to *flags_out and clears them, as
+ * gsa_workspace_status does for a caller's workspace (which a scratch-free
+ * caller does not have).  Returns GSA_ERR_TIMEOUT when the TIMEOUT bit is
+ * set.  Each gsa_decode_noalloc call clears the bits when it starts, so
+ * read them after the call whose result you want to check.  Allocates
+ * nothing.  The scratch address is looked up once per device; after a
+ * device reset (cudaDeviceReset, or a destroyed primary context) it is
+ * stale, so neither call may be used across one. */
+gsa_status gsa_noalloc_status(void *stream, uint32_t *flags_out);
 
 /* Gist-position step at chunk completion (gist.science/nl/paper/2604.20920,
  * "Het Proces", Compressie: a gist token sees only its own block and the
@@ -382,7 +393,7 @@ gsa_status gsa_multiquery_select(const gsa_desc *desc, const void *q, const void
  * stage 1's selection and the row maxima it left in ws (same ws):
  *   out_raw [B, hq, L, d], out_gist [B, hq, N, d] in out_dtype.
  * The dense gist part (all visible gists of a row) runs on the tensor cores
- * with bf16 softmax weights normalised by their own sum; the selected
+ * with fp16 softmax weights normalised by their own sum; the selected
  * chunks and the own chunk run on the CUDA cores in fp32. */
 gsa_status gsa_prefill_attend(const gsa_desc *desc, const void *q_raw, const void *k_raw, const void *v_raw,
                               const void *q_gist, const void *k_gist, const void *v_gist, const int32_t *sel_idx,

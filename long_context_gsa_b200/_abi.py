@@ -26,7 +26,7 @@ EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
     "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_decode_backward", "gsa_gist_step", "gsa_multiquery_select", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
-    "gsa_decode_noalloc",
+    "gsa_decode_noalloc", "gsa_noalloc_status",
 )
 
 
@@ -88,6 +88,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_prefill_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_decode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
+        "gsa_noalloc_status": ([vp, C.POINTER(C.c_uint32)], i32),
     }
     for name, (argt, rest) in sig.items():
         fn = getattr(lib, name)
@@ -116,13 +117,39 @@ def make_h2desc(level1: gsa_hdesc, level2: gsa_hdesc) -> gsa_h2desc:
     return gsa_h2desc(level1, level2)
 
 
-def _ptr(t, dtype=None, name="tensor", optional=False):
+def _n(desc, what, m_max=0, k=None):
+    """Element count of one C ABI buffer for `desc` (layouts of include/gsa.h)."""
+    B, hq, hkv, d = desc.batch, desc.hq, desc.hkv, desc.d
+    k = desc.topk if k is None else k
+    return {
+        "q": B * hq * d,                        # q, out, d_q, k_new-per-head rows
+        "kv_new": B * hkv * d,                  # k_new, v_new
+        "gists": B * hkv * desc.n_max * d,      # gist_k, gist_v and their gradients
+        "raw": B * hkv * desc.t_max * d,        # raw_k, raw_v and their gradients
+        "meta": B * hkv * m_max * d,            # meta_k, meta_v (m_max rows)
+        "batch": B,                             # n_gists, own_len
+        "heads": B * hq,                        # lse, sel_count
+        "scores": B * hq * desc.n_max,
+        "sel": B * hq * k,                      # sel_idx, sel_score, meta_idx
+        "rows_q": B * hq * desc.t_max * d,      # prefill q_raw / out_raw, multi-query q
+        "rows_gq": B * hq * desc.n_max * d,     # prefill q_gist / out_gist
+        "rows_sel": B * hq * desc.t_max * k,    # prefill / multi-query selections
+    }[what]
+
+
+def _ptr(t, dtype=None, name="tensor", optional=False, numel=None):
+    """Data pointer of `t` after the checks the C ABI relies on: a contiguous
+    CUDA tensor of `dtype` holding at least `numel` elements (the size its
+    layout in include/gsa.h implies for the descriptor).  A short buffer is
+    rejected here, before the library could read or write past its end."""
     if t is None:
         if optional:
             return None
         raise ValueError(f"{name} is required")
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the descriptor needs at least {numel}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (the GSA path has no CPU implementation)")
     if dtype is not None and t.dtype != dtype:
@@ -184,163 +211,205 @@ def gsa_workspace_status(ws, stream=None) -> int:
 
 def gsa_score_gists(desc, q, gist_k, gist_v, n_gists, scores, ws, stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("gsa_score_gists", load().gsa_score_gists(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True),
-        _ptr(n_gists, torch.int32, "n_gists"), _ptr(scores, torch.float32, "scores"), p, n, _stream(stream)))
+        C.byref(desc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+        _ptr(gist_v, dt, "gist_v", True, _n(desc, "gists")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(scores, torch.float32, "scores", numel=_n(desc, "scores")), *_ws(ws), _stream(stream)))
 
 
 def gsa_topk_select(desc, scores, n_gists, sel_idx, sel_score, ws, stream=None):
-    p, n = _ws(ws)
     _check("gsa_topk_select", load().gsa_topk_select(
-        C.byref(desc), _ptr(scores, torch.float32, "scores"), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
-        _stream(stream)))
+        C.byref(desc), _ptr(scores, torch.float32, "scores", numel=_n(desc, "scores")),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")), *_ws(ws), _stream(stream)))
 
 
 def gsa_topp_select(desc, scores, n_gists, top_p, sel_idx, sel_score, sel_count, ws, stream=None):
-    p, n = _ws(ws)
     _check("gsa_topp_select", load().gsa_topp_select(
-        C.byref(desc), _ptr(scores, torch.float32, "scores"), _ptr(n_gists, torch.int32, "n_gists"),
-        C.c_float(float(top_p)), _ptr(sel_idx, torch.int32, "sel_idx"),
-        _ptr(sel_score, torch.float32, "sel_score", True), _ptr(sel_count, torch.int32, "sel_count", True), p, n,
-        _stream(stream)))
+        C.byref(desc), _ptr(scores, torch.float32, "scores", numel=_n(desc, "scores")),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch), C.c_float(float(top_p)),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")),
+        _ptr(sel_count, torch.int32, "sel_count", True, _n(desc, "heads")), *_ws(ws), _stream(stream)))
 
 
 def gsa_unfold_attend(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, prior, out, lse, ws,
                       stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("gsa_unfold_attend", load().gsa_unfold_attend(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
-        _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(own_len, torch.int32, "own_len"), _ptr(sel_idx, torch.int32, "sel_idx", True),
-        _ptr(sel_score, torch.float32, "sel_score", True), int(prior), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
-        _ptr(lse, torch.float32, "lse", True), p, n, _stream(stream)))
+        C.byref(desc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")),
+        _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")), _ptr(gist_v, dt, "gist_v", True, _n(desc, "gists")),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+        _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")), int(prior),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
+        _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")), *_ws(ws), _stream(stream)))
+
+
+def _decode_ptrs(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score):
+    """The pointer arguments shared by gsa_decode and gsa_decode_noalloc."""
+    dt = _TORCH_DT[desc.dtype]
+    return (_ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+            _ptr(gist_v, dt, "gist_v", numel=_n(desc, "gists")), _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")),
+            _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+            _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+            _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
+            _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")),
+            _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")),
+            _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")))
 
 
 def gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None, sel_idx=None,
                sel_score=None, ws=None, stream=None):
-    dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("gsa_decode", load().gsa_decode(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
-        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(own_len, torch.int32, "own_len"), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
-        _ptr(lse, torch.float32, "lse", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
-        _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
+        C.byref(desc), *_decode_ptrs(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx,
+                                     sel_score), *_ws(ws), _stream(stream)))
 
 
 def hgsa_select(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, n_gists, meta_idx, sel_idx, sel_score, ws,
                 stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
+    nm = _n(desc, "meta", m_max=hdesc.m_max)
     _check("hgsa_select", load().hgsa_select(
-        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q"), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v", True),
-        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(meta_idx, torch.int32, "meta_idx"), _ptr(sel_idx, torch.int32, "sel_idx"),
-        _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(meta_k, dt, "meta_k", numel=nm),
+        _ptr(meta_v, dt, "meta_v", True, nm), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+        _ptr(gist_v, dt, "gist_v", True, _n(desc, "gists")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(meta_idx, torch.int32, "meta_idx", numel=_n(desc, "sel", k=hdesc.topk_meta)),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", numel=_n(desc, "sel")), *_ws(ws), _stream(stream)))
 
 
 def hgsa_decode(desc, hdesc, q, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None,
                 meta_idx=None, sel_idx=None, sel_score=None, ws=None, stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
+    nm = _n(desc, "meta", m_max=hdesc.m_max)
     _check("hgsa_decode", load().hgsa_decode(
-        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q"), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v"),
-        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
-        _ptr(n_gists, torch.int32, "n_gists"), _ptr(own_len, torch.int32, "own_len"),
-        _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True),
-        _ptr(meta_idx, torch.int32, "meta_idx", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
-        _ptr(sel_score, torch.float32, "sel_score", True), p, n, _stream(stream)))
+        C.byref(desc), C.byref(hdesc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(meta_k, dt, "meta_k", numel=nm),
+        _ptr(meta_v, dt, "meta_v", numel=nm), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+        _ptr(gist_v, dt, "gist_v", numel=_n(desc, "gists")), _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")),
+        _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
+        _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")),
+        _ptr(meta_idx, torch.int32, "meta_idx", True, _n(desc, "sel", k=hdesc.topk_meta)),
+        _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")), *_ws(ws), _stream(stream)))
+
+
+def _hgsa2_ptrs(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, v_optional):
+    dt = _TORCH_DT[desc.dtype]
+    n2 = _n(desc, "meta", m_max=h2desc.level2.m_max)
+    n1 = _n(desc, "meta", m_max=h2desc.level1.m_max)
+    return (_ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(meta2_k, dt, "meta2_k", numel=n2),
+            _ptr(meta2_v, dt, "meta2_v", v_optional, n2), _ptr(meta_k, dt, "meta_k", numel=n1),
+            _ptr(meta_v, dt, "meta_v", v_optional, n1), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+            _ptr(gist_v, dt, "gist_v", v_optional, _n(desc, "gists")))
 
 
 def hgsa2_select(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, n_gists, meta2_idx, meta_idx,
                  sel_idx, sel_score, ws, stream=None):
-    dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("hgsa2_select", load().hgsa2_select(
-        C.byref(desc), C.byref(h2desc), _ptr(q, dt, "q"), _ptr(meta2_k, dt, "meta2_k"),
-        _ptr(meta2_v, dt, "meta2_v", True), _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v", True),
-        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v", True), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(meta2_idx, torch.int32, "meta2_idx"), _ptr(meta_idx, torch.int32, "meta_idx"),
-        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+        C.byref(desc), C.byref(h2desc),
+        *_hgsa2_ptrs(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, True),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(meta2_idx, torch.int32, "meta2_idx", numel=_n(desc, "sel", k=h2desc.level2.topk_meta)),
+        _ptr(meta_idx, torch.int32, "meta_idx", numel=_n(desc, "sel", k=h2desc.level1.topk_meta)),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", numel=_n(desc, "sel")), *_ws(ws), _stream(stream)))
 
 
 def hgsa2_decode(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, raw_k, raw_v, n_gists, own_len,
                  out, lse=None, meta2_idx=None, meta_idx=None, sel_idx=None, sel_score=None, ws=None, stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("hgsa2_decode", load().hgsa2_decode(
-        C.byref(desc), C.byref(h2desc), _ptr(q, dt, "q"), _ptr(meta2_k, dt, "meta2_k"), _ptr(meta2_v, dt, "meta2_v"),
-        _ptr(meta_k, dt, "meta_k"), _ptr(meta_v, dt, "meta_v"), _ptr(gist_k, dt, "gist_k"),
-        _ptr(gist_v, dt, "gist_v"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
-        _ptr(n_gists, torch.int32, "n_gists"), _ptr(own_len, torch.int32, "own_len"),
-        _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True),
-        _ptr(meta2_idx, torch.int32, "meta2_idx", True), _ptr(meta_idx, torch.int32, "meta_idx", True),
-        _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True), p, n,
-        _stream(stream)))
+        C.byref(desc), C.byref(h2desc),
+        *_hgsa2_ptrs(desc, h2desc, q, meta2_k, meta2_v, meta_k, meta_v, gist_k, gist_v, False),
+        _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")), _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
+        _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")),
+        _ptr(meta2_idx, torch.int32, "meta2_idx", True, _n(desc, "sel", k=h2desc.level2.topk_meta)),
+        _ptr(meta_idx, torch.int32, "meta_idx", True, _n(desc, "sel", k=h2desc.level1.topk_meta)),
+        _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")), *_ws(ws), _stream(stream)))
 
 
 def gsa_multiquery_select(desc, q, gist_k, sel_idx, sel_score, ws, stream=None):
     _check("gsa_multiquery_select", load().gsa_multiquery_select(
-        C.byref(desc), _ptr(q, torch.bfloat16, "q"), _ptr(gist_k, torch.bfloat16, "gist_k"),
-        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"),
-        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+        C.byref(desc), _ptr(q, torch.bfloat16, "q", numel=_n(desc, "rows_q")),
+        _ptr(gist_k, torch.bfloat16, "gist_k", numel=_n(desc, "gists")),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "rows_sel")),
+        _ptr(sel_score, torch.float32, "sel_score", numel=_n(desc, "rows_sel")), *_ws(ws), _stream(stream)))
 
 
 def gsa_gist_step(desc, q, k_new, v_new, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, ws, stream=None):
     dt = _TORCH_DT[desc.dtype]
     _check("gsa_gist_step", load().gsa_gist_step(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(k_new, dt, "k_new"), _ptr(v_new, dt, "v_new"),
-        _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"), _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"),
-        _ptr(n_gists, torch.int32, "n_gists"), _ptr(own_len, torch.int32, "own_len"),
-        _ptr(out, _TORCH_DT[desc.out_dtype], "out"), _ptr(lse, torch.float32, "lse", True), _ptr(ws, torch.uint8, "ws"),
-        ws.numel(), _stream(stream)))
+        C.byref(desc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(k_new, dt, "k_new", numel=_n(desc, "kv_new")),
+        _ptr(v_new, dt, "v_new", numel=_n(desc, "kv_new")), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+        _ptr(gist_v, dt, "gist_v", numel=_n(desc, "gists")), _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")),
+        _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+        _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
+        _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")), *_ws(ws), _stream(stream)))
 
 
 def gsa_decode_backward(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, sel_idx, out, lse, d_out, d_q,
                         d_gist_k, d_gist_v, d_raw_k, d_raw_v, stream=None):
     dt = _TORCH_DT[desc.dtype]
     f = torch.float32
+    nq, ng, nr = _n(desc, "q"), _n(desc, "gists"), _n(desc, "raw")
     _check("gsa_decode_backward", load().gsa_decode_backward(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
-        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(own_len, torch.int32, "own_len"), _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(out, f, "out"),
-        _ptr(lse, f, "lse"), _ptr(d_out, f, "d_out"), _ptr(d_q, f, "d_q"), _ptr(d_gist_k, f, "d_gist_k"),
-        _ptr(d_gist_v, f, "d_gist_v"), _ptr(d_raw_k, f, "d_raw_k"), _ptr(d_raw_v, f, "d_raw_v"), _stream(stream)))
+        C.byref(desc), _ptr(q, dt, "q", numel=nq), _ptr(gist_k, dt, "gist_k", numel=ng),
+        _ptr(gist_v, dt, "gist_v", numel=ng), _ptr(raw_k, dt, "raw_k", numel=nr), _ptr(raw_v, dt, "raw_v", numel=nr),
+        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+        _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")), _ptr(out, f, "out", numel=nq),
+        _ptr(lse, f, "lse", numel=_n(desc, "heads")), _ptr(d_out, f, "d_out", numel=nq),
+        _ptr(d_q, f, "d_q", numel=nq), _ptr(d_gist_k, f, "d_gist_k", numel=ng),
+        _ptr(d_gist_v, f, "d_gist_v", numel=ng), _ptr(d_raw_k, f, "d_raw_k", numel=nr),
+        _ptr(d_raw_v, f, "d_raw_v", numel=nr), _stream(stream)))
 
 
 def gsa_prefill_score(desc, q_raw, q_gist, k_gist, sel_idx, sel_score, ws, stream=None):
     dt = _TORCH_DT[desc.dtype]
-    p, n = _ws(ws)
     _check("gsa_prefill_score", load().gsa_prefill_score(
-        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"),
-        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"), p, n, _stream(stream)))
+        C.byref(desc), _ptr(q_raw, dt, "q_raw", numel=_n(desc, "rows_q")),
+        _ptr(q_gist, dt, "q_gist", numel=_n(desc, "rows_gq")), _ptr(k_gist, dt, "k_gist", numel=_n(desc, "gists")),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "rows_sel")),
+        _ptr(sel_score, torch.float32, "sel_score", numel=_n(desc, "rows_sel")), *_ws(ws), _stream(stream)))
+
+
+def _prefill_inputs(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist):
+    dt = _TORCH_DT[desc.dtype]
+    return (_ptr(q_raw, dt, "q_raw", numel=_n(desc, "rows_q")), _ptr(k_raw, dt, "k_raw", numel=_n(desc, "raw")),
+            _ptr(v_raw, dt, "v_raw", numel=_n(desc, "raw")), _ptr(q_gist, dt, "q_gist", numel=_n(desc, "rows_gq")),
+            _ptr(k_gist, dt, "k_gist", numel=_n(desc, "gists")), _ptr(v_gist, dt, "v_gist", numel=_n(desc, "gists")))
 
 
 def gsa_prefill_attend(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, sel_idx, sel_score, out_raw, out_gist, ws,
                        stream=None):
-    dt = _TORCH_DT[desc.dtype]
     odt = _TORCH_DT[desc.out_dtype]
-    p, n = _ws(ws)
     _check("gsa_prefill_attend", load().gsa_prefill_attend(
-        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_raw, dt, "k_raw"), _ptr(v_raw, dt, "v_raw"),
-        _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist"),
-        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_score, torch.float32, "sel_score"),
-        _ptr(out_raw, odt, "out_raw"), _ptr(out_gist, odt, "out_gist"), p, n, _stream(stream)))
+        C.byref(desc), *_prefill_inputs(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist),
+        _ptr(sel_idx, torch.int32, "sel_idx", numel=_n(desc, "rows_sel")),
+        _ptr(sel_score, torch.float32, "sel_score", numel=_n(desc, "rows_sel")),
+        _ptr(out_raw, odt, "out_raw", numel=_n(desc, "rows_q")),
+        _ptr(out_gist, odt, "out_gist", numel=_n(desc, "rows_gq")), *_ws(ws), _stream(stream)))
 
 
 def gsa_prefill(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist, out_raw, out_gist, sel_idx=None, sel_score=None,
                 ws=None, stream=None):
-    dt = _TORCH_DT[desc.dtype]
     odt = _TORCH_DT[desc.out_dtype]
-    p, n = _ws(ws)
     _check("gsa_prefill", load().gsa_prefill(
-        C.byref(desc), _ptr(q_raw, dt, "q_raw"), _ptr(k_raw, dt, "k_raw"), _ptr(v_raw, dt, "v_raw"),
-        _ptr(q_gist, dt, "q_gist"), _ptr(k_gist, dt, "k_gist"), _ptr(v_gist, dt, "v_gist"),
-        _ptr(sel_idx, torch.int32, "sel_idx", True), _ptr(sel_score, torch.float32, "sel_score", True),
-        _ptr(out_raw, odt, "out_raw"), _ptr(out_gist, odt, "out_gist"), p, n, _stream(stream)))
+        C.byref(desc), *_prefill_inputs(desc, q_raw, k_raw, v_raw, q_gist, k_gist, v_gist),
+        _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "rows_sel")),
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "rows_sel")),
+        _ptr(out_raw, odt, "out_raw", numel=_n(desc, "rows_q")),
+        _ptr(out_gist, odt, "out_gist", numel=_n(desc, "rows_gq")), *_ws(ws), _stream(stream)))
 
 
 def gsa_decode_noalloc(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse=None, sel_idx=None,
@@ -348,10 +417,16 @@ def gsa_decode_noalloc(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, 
     """gsa_decode without a workspace argument (the library's built-in
     scratch array is used; see include/gsa.h for its limit and the rule
     that calls must not overlap on the GPU)."""
-    dt = _TORCH_DT[desc.dtype]
     _check("gsa_decode_noalloc", load().gsa_decode_noalloc(
-        C.byref(desc), _ptr(q, dt, "q"), _ptr(gist_k, dt, "gist_k"), _ptr(gist_v, dt, "gist_v"),
-        _ptr(raw_k, dt, "raw_k"), _ptr(raw_v, dt, "raw_v"), _ptr(n_gists, torch.int32, "n_gists"),
-        _ptr(own_len, torch.int32, "own_len"), _ptr(out, _TORCH_DT[desc.out_dtype], "out"),
-        _ptr(lse, torch.float32, "lse", True), _ptr(sel_idx, torch.int32, "sel_idx", True),
-        _ptr(sel_score, torch.float32, "sel_score", True), _stream(stream)))
+        C.byref(desc), *_decode_ptrs(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx,
+                                     sel_score), _stream(stream)))
+
+
+def gsa_noalloc_status(stream=None) -> int:
+    """GSA_DEVERR_* bits left by gsa_decode_noalloc on the current device
+    (read and cleared; synchronises the stream)."""
+    flags = C.c_uint32(0)
+    st = load().gsa_noalloc_status(_stream(stream), C.byref(flags))
+    if st not in (GSA_OK, GSA_ERR_TIMEOUT):
+        _check("gsa_noalloc_status", st)
+    return int(flags.value)

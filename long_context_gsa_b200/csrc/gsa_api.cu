@@ -1335,3 +1335,12 @@ extern "C" gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, co
   return gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score, ws,
                     GSA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" gsa_status gsa_noalloc_status(void *stream, uint32_t *flags_out) {
+  if (!flags_out) return GSA_ERR_INVALID_ARG;
+  void *ws = nullptr;
+  GSA_TRY(noalloc_scratch(&ws));
+  // The status word is word 0 of the array (the decode layout starts there);
+  // reading it needs no allocation, only a copy into the caller's variable.
+  return gsa_workspace_status(ws, GSA_NOALLOC_SCRATCH_BYTES, stream, flags_out);
+}

@@ -168,3 +168,51 @@ def test_product_path_does_not_import_the_oracle():
     for f in list(pkg.glob("*.py")) + list((pkg / "csrc").glob("*")):
         text = f.read_text(errors="ignore")
         assert "import oracle" not in text and "from oracle" not in text and "gsa_oracle" not in text, f
+
+
+def test_binding_sizes_follow_the_header_layouts():
+    """The element counts the binding requires are the layouts of include/gsa.h."""
+    from long_context_gsa_b200._abi import _n
+    d = _desc(batch=3, hq=8, hkv=2, d=64, n_max=50, t_max=816, topk=7)
+    assert _n(d, "q") == 3 * 8 * 64
+    assert _n(d, "gists") == 3 * 2 * 50 * 64
+    assert _n(d, "raw") == 3 * 2 * 816 * 64
+    assert _n(d, "meta", m_max=5) == 3 * 2 * 5 * 64
+    assert _n(d, "scores") == 3 * 8 * 50
+    assert _n(d, "sel") == 3 * 8 * 7 and _n(d, "sel", k=4) == 3 * 8 * 4
+    assert _n(d, "heads") == 24 and _n(d, "batch") == 3 and _n(d, "kv_new") == 3 * 2 * 64
+    assert _n(d, "rows_q") == 3 * 8 * 816 * 64 and _n(d, "rows_gq") == 3 * 8 * 50 * 64
+    assert _n(d, "rows_sel") == 3 * 8 * 816 * 7
+
+
+def test_binding_rejects_short_buffers_before_any_call(lib):
+    """A buffer shorter than its layout needs is refused by the binding (the
+    library would otherwise read or write past its end); a longer one is
+    accepted by the size check."""
+    import torch
+    from long_context_gsa_b200 import _abi
+    d = _desc(batch=2, hq=4, hkv=2, d=64, n_max=16, t_max=16 * 8 + 8, topk=4)
+    short = torch.zeros(2 * 4 * 64 - 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="holds 511 elements"):
+        _abi._ptr(short, torch.bfloat16, "q", numel=_abi._n(d, "q"))
+    long_ = torch.zeros(2 * 4 * 64 + 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):  # size passes; the device check comes next
+        _abi._ptr(long_, torch.bfloat16, "q", numel=_abi._n(d, "q"))
+    t = torch.zeros(4)
+    # the first pointer of each entry point is checked first, before the workspace
+    calls = [
+        lambda: _abi.gsa_decode(d, short, t, t, t, t, t, t, t, ws=t),
+        lambda: _abi.gsa_decode_noalloc(d, short, t, t, t, t, t, t, t),
+        lambda: _abi.gsa_score_gists(d, short, t, t, t, t, t),
+        lambda: _abi.gsa_unfold_attend(d, short, t, t, t, t, t, t, t, 1, t, None, t),
+        lambda: _abi.gsa_topk_select(d, torch.zeros(2 * 4 * 16 - 1), t, t, None, t),
+        lambda: _abi.gsa_gist_step(d, short, t, t, t, t, t, t, t, t, t, None, t),
+        lambda: _abi.gsa_decode_backward(d, short, *([t] * 16)),
+        lambda: _abi.hgsa_select(d, _abi.make_hdesc(4, 2, 4), short, t, t, t, t, t, t, t, t, t),
+        lambda: _abi.gsa_prefill_score(d, short, t, t, t, t, t),
+        lambda: _abi.gsa_prefill(d, short, t, t, t, t, t, t, t, ws=t),
+        lambda: _abi.gsa_multiquery_select(d, short, t, t, t, t),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(ValueError, match="holds"):
+            call()
