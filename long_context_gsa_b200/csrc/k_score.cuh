@@ -34,6 +34,9 @@ struct ScoreArgs {
   int32_t score_stride;
   float *part;            // [B*hq, n_split, D+4] or null
   int32_t n_split;
+  float *gmax;            // [B*hq, gmax_stride] or null: max score of gists 16i .. 16i+15 (tensor-core path)
+  int32_t gmax_stride;
+  uint32_t *zero_rows;    // [B*hq] or null: zeroed for this kernel's heads (re-arms the unfold's counters)
   uint32_t *status;
   int32_t hq, hkv, group;
   int32_t head_split;     // CTAs per kv head along the query heads
@@ -49,9 +52,10 @@ __device__ __forceinline__ void mma_16816_bf16(float c[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Slice of rows [n0, n1) handled by `split`; slices are multiples of 8.
+// Slice of rows [n0, n1) handled by `split`; slices are multiples of 16,
+// so every group of 16 consecutive rows (a group maximum) lies in one slice.
 __device__ __forceinline__ void score_slice(int N, int n_split, int split, int &n0, int &n1) {
-  const int per = ((N + n_split - 1) / n_split + 7) & ~7;
+  const int per = ((N + n_split - 1) / n_split + 15) & ~15;
   n0 = split * per;
   n1 = min(N, n0 + per);
   if (n1 < n0) n1 = n0;
@@ -150,6 +154,7 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
   const int ntiles = (nrows + kTile - 1) / kTile;
   const int row0 = (b * a.hkv + kvh) * a.rows_cap + n0;  // first tensor-map row of this slice
 
+  if (a.zero_rows && split == 0 && tid < nh) a.zero_rows[static_cast<size_t>(b) * a.hq + h0 + tid] = 0u;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     for (int s = 0; s <= kStages; ++s) cnt[s] = 0;
@@ -243,6 +248,20 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
             s[nt][e] = c[nt][e] * a.scale_log2;
           }
         }
+      if (a.gmax) {
+        // the maximum of this warp's 16 rows per head (lanes 4g .. 4g+3 hold
+        // head g's scores), in the same units as the stored scores
+        float gm = neg_inf();
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (s[nt][e] > neg_inf()) gm = fmaxf(gm, c[nt][e] * a.scale);
+        gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 1));
+        gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 2));
+        if (t4 == 0 && g < nh)
+          a.gmax[(static_cast<size_t>(b) * a.hq + h0 + g) * a.gmax_stride + (n0 + t * kTile + rw) / 16] = gm;
+      }
       if (WITH_V) {
         // lazy reference: raised only when this warp's rows exceed it by
         // more than kRescaleSlack; the head's accumulators then rescale

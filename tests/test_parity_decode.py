@@ -128,14 +128,96 @@ def test_bf16_output():
 
 
 def test_separate_entry_points_match_fused():
+    """gsa_decode (selection in the unfold prologue) against the three
+    separate calls (gsa_topk_select's own kernel): the same selection, and
+    outputs equal up to fp32 summation order (the two launches may cut a
+    row's unfold into different splits)."""
     cfg = W.scaled(W.QWEN_16X, batch=2, context=900 * 16, kv_std=1.0)
     x = W.decode_inputs(cfg, device="cuda", own_len=6)
     for excl in (False, True):
         a = run_gpu(x, cfg, excl, fused=True)
         b = run_gpu(x, cfg, excl, fused=False)
         assert torch.equal(a[2], b[2])
-        assert torch.equal(a[0], b[0])
+        assert torch.equal(a[3], b[3])  # selected scores
+        assert (a[0] - b[0]).abs().max().item() <= 1e-5
     compare(x, cfg, fused=False, what="separate calls")
+
+
+def _select_attend(x, cfg, excl):
+    """gsa_score_gists, then gsa_select_attend (selection + unfold in one launch)."""
+    B, hq, d = x["q"].shape
+    hkv, n_max, t_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2]
+    desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, excl, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+    scores = torch.empty((B, hq, n_max), dtype=torch.float32, device="cuda")
+    out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, hq), dtype=torch.float32, device="cuda")
+    sel = torch.full((B, hq, cfg.topk), -7, dtype=torch.int32, device="cuda")
+    ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device="cuda")
+    G.gsa_score_gists(desc, x["q"], x["gist_k"], None if excl else x["gist_v"], x["n_gists"], scores, ws)
+    G.gsa_select_attend(desc, scores, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel,
+                        ssc, out, lse, ws)
+    torch.cuda.synchronize()
+    assert G.gsa_workspace_status(ws) == 0
+    return out, lse, sel, ssc
+
+
+@pytest.mark.parametrize("excl", [False, True], ids=["default", "exclude"])
+def test_select_attend_entry_point(excl):
+    """gsa_score_gists followed by gsa_select_attend computes the fused step."""
+    cfg = W.scaled(W.LLAMA_8X, batch=3, context=1500 * 8)
+    x = W.decode_inputs(cfg, device="cuda", own_len=5, ragged=[1500, 999, 64])
+    a = run_gpu(x, cfg, excl, fused=True)
+    out, lse, sel, ssc = _select_attend(x, cfg, excl)
+    assert torch.equal(a[2], sel) and torch.equal(a[3], ssc)
+    assert (a[0] - out).abs().max().item() <= 1e-5 and (a[1] - lse).abs().max().item() <= 1e-5
+
+
+TIE_CASES = [
+    # gist keys repeated in runs of three: most rows' k-th place falls inside a run of equal scores
+    ("runs_of_3", dict(batch=2, hq=32, hkv=8, d=64, chunk=8, context=2000 * 8, topk=64), 3),
+    ("runs_of_3_d128", dict(batch=1, hq=28, hkv=4, d=128, chunk=16, context=3000 * 16, topk=128), 3),
+    # every gist key equal: all scores of a row tie (the exact radix fallback)
+    ("all_equal", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, context=3000 * 8, topk=64), 0),
+    # fewer groups of 16 than k: the scores themselves are the bound's values
+    ("few_groups", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, context=300 * 8, topk=64), 3),
+    # a row longer than the group list (more than 16384 gists): the radix path
+    ("long_row", dict(batch=1, hq=4, hkv=1, d=64, chunk=8, context=20000 * 8, topk=32), 3),
+]
+
+
+@pytest.mark.parametrize("name,chg,run", TIE_CASES, ids=[c[0] for c in TIE_CASES])
+def test_exact_ties_go_to_lower_index(name, chg, run):
+    """Bit-equal scores on both sides of the k-th place: the selection takes
+    the lower chunk indices ([nl] Selectie; ties to the lower index), in the
+    fused step as in gsa_topk_select, and matches the oracle."""
+    cfg = W.scaled(W.QWEN_16X, kv_std=1.0, **chg)
+    x = W.decode_inputs(cfg, device="cuda", own_len=3, seed=zlib.crc32(name.encode()) % 100000)
+    N = cfg.n_gists
+    src = torch.arange(N, device="cuda")
+    src = src // run * run if run else torch.zeros_like(src)
+    x["gist_k"] = x["gist_k"][:, :, src].contiguous()
+    a = run_gpu(x, cfg, False, fused=True)
+    b = run_gpu(x, cfg, False, fused=False)
+    assert torch.equal(a[2], b[2]), f"{name}: fused and separate selections differ"
+    B, hq, d = x["q"].shape
+    rows = np.arange(B * hq)
+    orc = run_oracle(x, cfg, rows=rows)
+    g_sel = np.sort(a[2].reshape(B * hq, -1).cpu().numpy(), -1)
+    o_sel = np.sort(orc["sel"], -1)
+    exact_tie_rows = 0
+    for r in rows:
+        s = orc["scores"][r]
+        srt = np.sort(s[~np.isnan(s)])[::-1]
+        if len(srt) > cfg.topk and srt[cfg.topk - 1] == srt[cfg.topk]:
+            exact_tie_rows += 1
+        if not np.array_equal(g_sel[r], o_sel[r]):
+            gs, os_ = set(g_sel[r].tolist()) - {-1}, set(o_sel[r].tolist()) - {-1}
+            lost = {s[t] for t in os_ - gs}
+            assert not any(s[t] in lost for t in gs - os_), f"{name}: row {r}: exact tie went to a higher index"
+    assert exact_tie_rows > len(rows) // 2, (name, exact_tie_rows)
+    compare(x, cfg, what=name)
 
 
 def test_pr1_all_steps():
