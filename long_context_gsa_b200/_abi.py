@@ -89,7 +89,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_decode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
         "gsa_noalloc_status": ([vp, C.POINTER(C.c_uint32)], i32),
-        "gsa_select_attend": ([D] + [vp] * 11 + [sz, vp], i32),
+        "gsa_select_attend": ([D] + [vp] * 12 + [sz, vp], i32),
     }
     for name, (argt, rest) in sig.items():
         fn = getattr(lib, name)

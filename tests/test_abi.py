@@ -216,3 +216,15 @@ def test_binding_rejects_short_buffers_before_any_call(lib):
     for i, call in enumerate(calls):
         with pytest.raises(ValueError, match="holds"):
             call()
+
+
+def test_binding_arities_match_the_header(lib):
+    """Every ctypes signature has as many arguments as its declaration in
+    include/gsa.h."""
+    text = re.sub(r"/\*.*?\*/", "", (ROOT / "include" / "gsa.h").read_text(), flags=re.S)
+    decls = dict(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(([^)]*)\)\s*;", text, flags=re.M))
+    assert len(decls) >= 20, sorted(decls)
+    for name, params in decls.items():
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(lib, name).argtypes) == n, f"{name}: binding has {len(getattr(lib, name).argtypes)}, header {n}"
