@@ -238,10 +238,19 @@ def measure_flat(G, W, cfg, dev, args, flush, seed, e2e=False, clock_index=None)
         evs[1].record()
 
     def step_split(evs):
+        """The fused step's kernels one call at a time: (bf16) scoring with
+        the selection in its tail, then the unfold; (fp32) scoring,
+        selection, unfold."""
         evs[0].record()
-        G.gsa_score_gists(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores, ws)
-        evs[1].record()
-        G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
+        if cfg.dtype == "bf16":
+            G.gsa_score_select(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores,
+                               sel, ssc, ws)
+            evs[1].record()
+        else:
+            G.gsa_score_gists(desc, x["q"], x["gist_k"], None if cfg.exclude else x["gist_v"], x["n_gists"], scores,
+                              ws)
+            evs[1].record()
+            G.gsa_topk_select(desc, scores, x["n_gists"], sel, ssc, ws)
         evs[2].record()
         G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
                             prior, out, None, ws)
@@ -286,10 +295,18 @@ def flat_summary(cfg, m, hbm):
             "unit": UNIT, "ms_per_step": round(ms, 5),
             "step_hbm": {"alg_bytes": ab["total"], "achieved_gbs": round(ab["total"] / (ms / 1e3) / 1e9, 1),
                          "frac": round(ab["total"] / (ms / 1e3) / 1e9 / hbm, 4)},
-            "kernels_us": {"score_gists": round(float(k[0]) * 1e3, 2), "topk_select": round(float(k[1]) * 1e3, 2),
-                           "unfold_attend": round(float(k[2]) * 1e3, 2)},
+            "kernels_us": kernel_times(cfg, k),
             "score_gists_gbs": round(score_kernel_bytes(cfg) / (k[0] / 1e3) / 1e9, 1),
             "unfold_gbs": round((ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]) / (k[2] / 1e3) / 1e9, 1)}
+
+
+def kernel_times(cfg, k):
+    """Per-call event times (us) of the split step: bf16 runs two kernels
+    (scoring + selection; unfold), fp32 three."""
+    if cfg.dtype == "bf16":
+        return {"score_select": round(float(k[0]) * 1e3, 2), "unfold_attend": round(float(k[2]) * 1e3, 2)}
+    return {"score_gists": round(float(k[0]) * 1e3, 2), "topk_select": round(float(k[1]) * 1e3, 2),
+            "unfold_attend": round(float(k[2]) * 1e3, 2)}
 
 
 def measure_hgsa(G, W, cfg, dev, args, flush, hbm):
@@ -712,9 +729,14 @@ def run_gsa(args, world, rank, local):
         s = flat_summary(cfg, main, hbm)
         value = job_rate(cfg.head_queries, world, args.steps, total_ms)
         k = main["kern_ms"].mean(0)
-        names = ["score_gists", "topk_select", "unfold_attend"]
         ab = algorithmic_bytes(cfg, main["x"], main["sel"])
-        kbytes = [score_kernel_bytes(cfg), 0, ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]]
+        if cfg.dtype == "bf16":  # two kernels: scoring + selection; unfold
+            names = ["score_select", "unfold_attend"]
+            k = np.array([k[0], k[2]])
+            kbytes = [score_kernel_bytes(cfg), ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]]
+        else:
+            names = ["score_gists", "topk_select", "unfold_attend"]
+            kbytes = [score_kernel_bytes(cfg), 0, ab["raw_union"] + ab["gist_sel"] + ab["own"] + ab["q_out"]]
         dom = int(np.argmax(k))
         ach = kbytes[dom] / (k[dom] / 1e3) / 1e9 if kbytes[dom] else None
         rec = recorded_kernel(names[dom], cfg.name)
@@ -775,7 +797,10 @@ def recorded_kernel(kernel, workload):
 
 
 def launches_per_step(cfg):
-    """Kernels of this library one fused decode step launches."""
+    """Kernels of this library one fused decode step launches (bf16: scoring,
+    then selection + unfold; fp32: scoring, selection, unfold)."""
+    if cfg.dtype == "bf16":
+        return 2
     return 3 if cfg.topk > 0 else 2
 
 

@@ -206,26 +206,21 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
                              const int32_t *sel_idx, const float *sel_score, int32_t prior, void *out, float *lse,
                              void *ws, size_t ws_bytes, void *stream);
 
-/* Steps 2 and 3 in one launch ([nl] Selectie + Selectieve Ontvouwing;
- * [ja] 2.1 steps 3-4), bf16 inputs only (GSA_ERR_UNSUPPORTED otherwise):
- * every CTA of a row selects the row's top k itself, in the prologue of the
- * unfold kernel, from
- *   scores  [B, hq, n_max] fp32, as gsa_score_gists wrote them, and
- *   the group maxima (max of every 16 consecutive scores) that the same
- *   gsa_score_gists call left in ws (same ws),
- * then unfolds and attends exactly as gsa_unfold_attend with the gist prior
- * of that scoring call (default mode).  The selection is the one
- * gsa_topk_select would write (ties to the lower chunk index) and is
- * written to sel_idx / sel_score ([B, hq, topk], may be NULL).
- *   raw_k, raw_v, gist_v, n_gists, own_len, out, lse: as gsa_unfold_attend
- *   (gist_v needed only with exclude_unselected = 1).
- * The per-row counters the unfold uses are re-armed by gsa_score_gists. */
-gsa_status gsa_select_attend(const gsa_desc *desc, const float *scores, const void *q, const void *raw_k,
-                             const void *raw_v, const void *gist_v, const int32_t *n_gists, const int32_t *own_len,
-                             int32_t *sel_idx, float *sel_score, void *out, float *lse, void *ws, size_t ws_bytes,
-                             void *stream);
+/* Steps 1 and 2 in one launch ([nl] Scoring + Selectie; [ja] 2.1 steps
+ * 2-3), bf16 inputs only (GSA_ERR_UNSUPPORTED otherwise): gsa_score_gists,
+ * and in the same kernel the top-k selection of every row -- the CTA that
+ * finishes a (b, kv head) group last selects for the group's query heads
+ * while other groups are still being scored.  The selection is the one
+ * gsa_topk_select writes (ties to the lower chunk index).
+ *   scores    [B, hq, n_max] fp32 out, or NULL (ws holds them)
+ *   sel_idx, sel_score  [B, hq, topk] out, or NULL (ws holds them)
+ * In default mode ws also receives the gist partial for gsa_unfold_attend
+ * with prior = GSA_PRIOR_GISTS. */
+gsa_status gsa_score_select(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                            const int32_t *n_gists, float *scores, int32_t *sel_idx, float *sel_score, void *ws,
+                            size_t ws_bytes, void *stream);
 /* One decode step = score -> select -> unfold on `stream` (bf16: two
- * launches, gsa_score_gists then gsa_select_attend; fp32: three).  sel_idx /
+ * launches, gsa_score_select then the unfold; fp32: three).  sel_idx /
  * sel_score ([B, hq, topk]) may be NULL, in which case ws holds them. */
 gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v, const void *raw_k,
                       const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,

@@ -10,7 +10,7 @@ from ._abi import (  # noqa: F401
     GSA_ERR_INVALID_ARG, GSA_ERR_TIMEOUT, GSA_ERR_UNSUPPORTED, GSA_ERR_WORKSPACE, GSA_F32, GSA_OK, GSA_OP_DECODE,
     GSA_OP_GIST_STEP, GSA_OP_HGSA, GSA_OP_HGSA2, GSA_OP_MULTIQUERY, GSA_OP_PREFILL, GSA_PRIOR_GISTS, GSA_PRIOR_HGSA, GSA_PRIOR_HGSA2,
     GSA_PRIOR_NONE, GsaError, gsa_decode, gsa_decode_backward, gsa_decode_noalloc, gsa_desc, gsa_gist_step,
-    gsa_noalloc_status, gsa_select_attend,
+    gsa_noalloc_status, gsa_score_select,
     gsa_h2desc, gsa_hdesc, gsa_multiquery_select, gsa_prefill, gsa_prefill_attend, gsa_prefill_score, gsa_score_gists, gsa_status_string,
     gsa_topk_select, gsa_topp_select, gsa_unfold_attend, gsa_version, gsa_workspace_bytes, gsa_workspace_init,
     gsa_workspace_status,

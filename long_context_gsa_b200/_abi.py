@@ -26,7 +26,7 @@ EXPORTS = (
     "gsa_status_string", "gsa_version", "gsa_workspace_bytes", "gsa_workspace_init", "gsa_workspace_status",
     "gsa_score_gists", "gsa_topk_select", "gsa_topp_select", "gsa_unfold_attend", "gsa_decode", "hgsa_select",
     "hgsa_decode", "hgsa2_select", "hgsa2_decode", "gsa_decode_backward", "gsa_gist_step", "gsa_multiquery_select", "gsa_prefill_score", "gsa_prefill_attend", "gsa_prefill",
-    "gsa_decode_noalloc", "gsa_noalloc_status", "gsa_select_attend",
+    "gsa_decode_noalloc", "gsa_noalloc_status", "gsa_score_select",
 )
 
 
@@ -89,7 +89,7 @@ def load(path: Path | None = None) -> C.CDLL:
         "gsa_prefill": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "gsa_decode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
         "gsa_noalloc_status": ([vp, C.POINTER(C.c_uint32)], i32),
-        "gsa_select_attend": ([D] + [vp] * 12 + [sz, vp], i32),
+        "gsa_score_select": ([D] + [vp] * 8 + [sz, vp], i32),
     }
     for name, (argt, rest) in sig.items():
         fn = getattr(lib, name)
@@ -249,19 +249,14 @@ def gsa_unfold_attend(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, 
         _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")), *_ws(ws), _stream(stream)))
 
 
-def gsa_select_attend(desc, scores, q, raw_k, raw_v, gist_v, n_gists, own_len, sel_idx, sel_score, out, lse, ws,
-                      stream=None):
+def gsa_score_select(desc, q, gist_k, gist_v, n_gists, scores, sel_idx, sel_score, ws, stream=None):
     dt = _TORCH_DT[desc.dtype]
-    _check("gsa_select_attend", load().gsa_select_attend(
-        C.byref(desc), _ptr(scores, torch.float32, "scores", numel=_n(desc, "scores")),
-        _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(raw_k, dt, "raw_k", numel=_n(desc, "raw")),
-        _ptr(raw_v, dt, "raw_v", numel=_n(desc, "raw")), _ptr(gist_v, dt, "gist_v", True, _n(desc, "gists")),
-        _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
-        _ptr(own_len, torch.int32, "own_len", numel=desc.batch),
+    _check("gsa_score_select", load().gsa_score_select(
+        C.byref(desc), _ptr(q, dt, "q", numel=_n(desc, "q")), _ptr(gist_k, dt, "gist_k", numel=_n(desc, "gists")),
+        _ptr(gist_v, dt, "gist_v", True, _n(desc, "gists")), _ptr(n_gists, torch.int32, "n_gists", numel=desc.batch),
+        _ptr(scores, torch.float32, "scores", True, _n(desc, "scores")),
         _ptr(sel_idx, torch.int32, "sel_idx", True, _n(desc, "sel")),
-        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")),
-        _ptr(out, _TORCH_DT[desc.out_dtype], "out", numel=_n(desc, "q")),
-        _ptr(lse, torch.float32, "lse", True, _n(desc, "heads")), *_ws(ws), _stream(stream)))
+        _ptr(sel_score, torch.float32, "sel_score", True, _n(desc, "sel")), *_ws(ws), _stream(stream)))
 
 
 def _decode_ptrs(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score):

@@ -41,6 +41,7 @@ inline float resolve_scale(const gsa_desc *d) {
 
 struct Layout {
   size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0, gmax = 0;
+  size_t unit_counters = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
   size_t meta2_scores = 0, meta2_idx = 0, cand1_scores = 0, cand1_ids = 0, cand1_count = 0;
   size_t pf_stats = 0, pf_gist = 0, pf_vh = 0, pf_ovf = 0;
@@ -125,6 +126,7 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   }
   take(L.scores, rows * d->n_max * 4);
   take(L.gmax, rows * gmax_stride(d) * 4);
+  take(L.unit_counters, rows * 4);
   take(L.sel_idx, rows * d->topk * 4);
   take(L.sel_score, rows * d->topk * 4);
   take(L.part_g, rows * kScoreSplitMax * rec);
@@ -314,7 +316,8 @@ gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dt
 gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const void *vals, const int32_t *n_gists,
                      int count_div, int rows_cap, float *scores, int score_stride, float *part, int *splits_out,
                      uint32_t *status, void *stream, float *gmax = nullptr, int gmax_stride = 0,
-                     uint32_t *zero_rows = nullptr) {
+                     uint32_t *zero_rows = nullptr, uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr,
+                     float *sel_score = nullptr) {
   const int group = d->hq / d->hkv;
   const bool with_v = part != nullptr;
   const ScorePlan plan = plan_score(d, rows_cap, with_v);
@@ -337,6 +340,10 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
   sa.gmax = mma ? gmax : nullptr;
   sa.gmax_stride = gmax_stride;
   sa.zero_rows = mma ? zero_rows : nullptr;
+  sa.unit_counters = mma && gmax && scores ? unit_counters : nullptr;
+  sa.topk = d->topk;
+  sa.sel_idx = sel_idx;
+  sa.sel_score = sel_score;
   sa.status = status;
   sa.hq = d->hq;
   sa.hkv = d->hkv;
@@ -399,12 +406,10 @@ gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
   if (std::is_same<T, __nv_bfloat16>::value) {
     // tensor-core kernel: raw K/V as 2D maps with 8-row boxes
     // residency with the largest list share (one split), then the share of the chosen split count
-    const int ksel = ua.select ? ua.k : 0;
-    const int slots = resident_ctas(k_unfold_tc<D>, kUnfoldThreads,
-                                    UnfoldTcCfg<D>::smem_bytes(std::max(1, ua.k), ua.chunk, ksel));
+    const int slots =
+        resident_ctas(k_unfold_tc<D>, kUnfoldThreads, UnfoldTcCfg<D>::smem_bytes(std::max(1, ua.k), ua.chunk));
     ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));
-    const size_t smem =
-        UnfoldTcCfg<D>::smem_bytes((std::max(1, ua.k) + ua.n_split - 1) / ua.n_split, ua.chunk, ksel);
+    const size_t smem = UnfoldTcCfg<D>::smem_bytes((std::max(1, ua.k) + ua.n_split - 1) / ua.n_split, ua.chunk);
     const uint64_t rows = static_cast<uint64_t>(B) * ua.hkv * ua.t_max;
     if (!map_rows(&ua.tm_k, ua.raw_k, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D) ||
         !map_rows(&ua.tm_v, ua.raw_v, rows, 8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D))
@@ -417,29 +422,11 @@ gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
   return launch(k_unfold<D, T>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads), smem, stream, ua);
 }
 
-// Selection in the unfold prologue: the scoring pass's scores and group
-// maxima in, the selection out (outputs may be null).
-struct SelectIn {
-  const float *scores = nullptr;
-  int score_stride = 0;
-  const float *gmax = nullptr;
-  int gmax_stride = 0;
-  int32_t *sel_idx_out = nullptr;
-  float *sel_score_out = nullptr;
-};
-
 gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const void *raw_v, const void *gist_v,
                       const int32_t *n_gists, const int32_t *own_len, const int32_t *sel_idx, const float *sel_score,
                       const float *prior, int n_prior, void *out, float *lse, const Layout &L, void *ws,
-                      void *stream, const SelectIn *sel_in = nullptr) {
+                      void *stream) {
   UnfoldArgs ua;
-  ua.select = sel_in != nullptr;
-  ua.row_scores = sel_in ? sel_in->scores : nullptr;
-  ua.score_stride = sel_in ? sel_in->score_stride : 0;
-  ua.gmax = sel_in ? sel_in->gmax : nullptr;
-  ua.gmax_stride = sel_in ? sel_in->gmax_stride : 0;
-  ua.sel_idx_out = sel_in ? sel_in->sel_idx_out : nullptr;
-  ua.sel_score_out = sel_in ? sel_in->sel_score_out : nullptr;
   ua.q = q;
   ua.raw_k = raw_k;
   ua.raw_v = raw_v;
@@ -867,9 +854,7 @@ gsa_status gsa_score_gists(const gsa_desc *desc, const void *q, const void *gist
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
   float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
   return run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, nullptr,
-                   reinterpret_cast<uint32_t *>(at(ws, L.status)), stream,
-                   reinterpret_cast<float *>(at(ws, L.gmax)), gmax_stride(desc),
-                   reinterpret_cast<uint32_t *>(at(ws, L.counters)));
+                   reinterpret_cast<uint32_t *>(at(ws, L.status)), stream);
 }
 
 gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, int32_t *sel_idx,
@@ -992,20 +977,14 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
   float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
   int n_prior = 0;
   if (desc->dtype == GSA_BF16) {
-    // Two launches: scoring (with group maxima; it re-arms the unfold's
-    // counters), then selection in the unfold's prologue and the unfold.
-    float *gmax = reinterpret_cast<float *>(at(ws, L.gmax));
+    // Two launches: scoring with the selection in its tail (it also re-arms
+    // the unfold's counters), then the unfold.
     GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
-                      stream, gmax, gmax_stride(desc), reinterpret_cast<uint32_t *>(at(ws, L.counters))));
-    SelectIn sel;
-    sel.scores = scores;
-    sel.score_stride = desc->n_max;
-    sel.gmax = gmax;
-    sel.gmax_stride = gmax_stride(desc);
-    sel.sel_idx_out = sel_idx;
-    sel.sel_score_out = sel_score;
-    return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, nullptr, nullptr, part, part ? n_prior : 0,
-                      out, lse, L, ws, stream, &sel);
+                      stream, reinterpret_cast<float *>(at(ws, L.gmax)), gmax_stride(desc),
+                      reinterpret_cast<uint32_t *>(at(ws, L.counters)),
+                      reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss));
+    return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, part, part ? n_prior : 0, out, lse, L,
+                      ws, stream);
   }
   GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
                     stream));
@@ -1020,36 +999,29 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
                     ws, stream);
 }
 
-gsa_status gsa_select_attend(const gsa_desc *desc, const float *scores, const void *q, const void *raw_k,
-                             const void *raw_v, const void *gist_v, const int32_t *n_gists, const int32_t *own_len,
-                             int32_t *sel_idx, float *sel_score, void *out, float *lse, void *ws, size_t ws_bytes,
-                             void *stream) {
+gsa_status gsa_score_select(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v,
+                            const int32_t *n_gists, float *scores, int32_t *sel_idx, float *sel_score, void *ws,
+                            size_t ws_bytes, void *stream) {
   GSA_TRY(check_desc(desc));
   if (desc->dtype != GSA_BF16) return GSA_ERR_UNSUPPORTED;
-  GSA_TRY(need_ptr(scores));
   GSA_TRY(need_ptr(q));
-  GSA_TRY(need_ptr(raw_k));
-  GSA_TRY(need_ptr(raw_v));
+  GSA_TRY(need_ptr(gist_k));
   GSA_TRY(need_ptr(n_gists));
-  GSA_TRY(need_ptr(own_len));
-  GSA_TRY(need_ptr(out));
-  GSA_TRY(opt_ptr(lse));
+  GSA_TRY(opt_ptr(scores));
   GSA_TRY(opt_ptr(sel_idx));
   GSA_TRY(opt_ptr(sel_score));
   GSA_TRY(need_ptr(ws));
-  if (desc->exclude_unselected) GSA_TRY(need_ptr(gist_v));
+  if (!desc->exclude_unselected) GSA_TRY(need_ptr(gist_v));
   const Layout L = layout(desc, GSA_OP_DECODE, nullptr);
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
-  SelectIn sel;
-  sel.scores = scores;
-  sel.score_stride = desc->n_max;
-  sel.gmax = reinterpret_cast<const float *>(at(ws, L.gmax));
-  sel.gmax_stride = gmax_stride(desc);
-  sel.sel_idx_out = sel_idx;
-  sel.sel_score_out = sel_score;
-  const float *pr = desc->exclude_unselected ? nullptr : reinterpret_cast<const float *>(at(ws, L.part_g));
-  return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, nullptr, nullptr, pr,
-                    pr ? gist_prior_count(desc) : 0, out, lse, L, ws, stream, &sel);
+  float *sc = scores ? scores : reinterpret_cast<float *>(at(ws, L.scores));
+  int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
+  float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
+  float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
+  return run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, sc, desc->n_max, part, nullptr,
+                   reinterpret_cast<uint32_t *>(at(ws, L.status)), stream, reinterpret_cast<float *>(at(ws, L.gmax)),
+                   gmax_stride(desc), reinterpret_cast<uint32_t *>(at(ws, L.counters)),
+                   reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss);
 }
 
 gsa_status hgsa_select(const gsa_desc *desc, const gsa_hdesc *hdesc, const void *q, const void *meta_k,

@@ -19,6 +19,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "k_select.cuh"
 #include "tc100.cuh"
 
 namespace gsa {
@@ -37,6 +38,13 @@ struct ScoreArgs {
   float *gmax;            // [B*hq, gmax_stride] or null: max score of gists 16i .. 16i+15 (tensor-core path)
   int32_t gmax_stride;
   uint32_t *zero_rows;    // [B*hq] or null: zeroed for this kernel's heads (re-arms the unfold's counters)
+  // Selection in the tail (tensor-core path, needs scores and gmax): the
+  // CTA that arrives last at its group's counter selects the top k of each
+  // of the group's query heads, one warp per head.
+  uint32_t *unit_counters;  // [B*hkv*head_split] or null; re-armed to 0 by the last CTA
+  int32_t topk;
+  int32_t *sel_idx;       // [B*hq, topk]
+  float *sel_score;       // [B*hq, topk] or null
   uint32_t *status;
   int32_t hq, hkv, group;
   int32_t head_split;     // CTAs per kv head along the query heads
@@ -79,6 +87,11 @@ struct ScoreMmaCfg {
   static constexpr uint32_t kBarOff = (kCntOff + (2 * kStages + 1) * 4 + 7) & ~7u;
   static constexpr uint32_t kSmemBytes = kBarOff + kStages * 8 + 1024;  // + alignment slack
   static_assert(kStages * kStageBytes >= kWarps * GH * D * 4 || !WITH_V, "merge buffer fits in the ring");
+  // warps selecting at once in the tail (their scratch lives in the ring)
+  static constexpr int kSelWarps = (kStages * kStageBytes) / sizeof(WarpSelSmem) < kWarps
+                                       ? static_cast<int>((kStages * kStageBytes) / sizeof(WarpSelSmem))
+                                       : kWarps;
+  static_assert(kSelWarps >= 1, "one selection scratch fits in the ring");
 };
 
 // Rescaling threshold (base-2 units): the running max used for the
@@ -325,14 +338,17 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
   }
   if (aborted && lane == 0) atomicExch(&cnt[kStages], 1);
   __syncthreads();
+  const int unit = blockIdx.z * gridDim.y + blockIdx.y;  // (b, kv head [x head half])
   if (cnt[kStages]) {
     // a wait expired: let every copy that may be in flight land, then leave
+    // (still counted at the group's counter, which the last CTA re-arms)
     if (tid == 0) {
       flag_error(a.status, GSA_DEVERR_TIMEOUT);
       for (int s = 0; s < kStages; ++s) {
         const int tl = *reinterpret_cast<volatile int *>(&last_issued[s]);
         if (tl >= 0) mbar_wait(&bars[s], (tl / kStages) & 1);
       }
+      if (a.unit_counters && atomicAdd(&a.unit_counters[unit], 1u) == gridDim.x - 1) a.unit_counters[unit] = 0u;
     }
     __syncthreads();
     return;
@@ -381,6 +397,31 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
       hdr[1] = l;
       hdr[2] = 0.f;
       hdr[3] = 0.f;
+    }
+  }
+  if (a.unit_counters) {
+    // The group's last CTA selects: every CTA's scores and group maxima are
+    // visible to it once it has seen the others' arrivals (fence, counter,
+    // fence).  The ring is free, and holds the warps' selection scratch.
+    __shared__ int last_s;
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      const bool last = atomicAdd(&a.unit_counters[unit], 1u) == gridDim.x - 1;
+      if (last) {
+        a.unit_counters[unit] = 0u;
+        __threadfence();
+      }
+      last_s = last;
+    }
+    __syncthreads();
+    if (last_s && warp < Cfg::kSelWarps) {
+      WarpSelSmem &wsm = reinterpret_cast<WarpSelSmem *>(smem)[warp];
+      for (int j = warp; j < nh; j += Cfg::kSelWarps) {
+        const size_t row = static_cast<size_t>(b) * a.hq + h0 + j;
+        warp_select(a.scores + row * a.score_stride, a.gmax + row * a.gmax_stride, N, a.topk, wsm,
+                    a.sel_idx + row * a.topk, a.sel_score ? a.sel_score + row * a.topk : nullptr);
+      }
     }
   }
 }

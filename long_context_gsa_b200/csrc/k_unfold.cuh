@@ -21,7 +21,6 @@
 
 #include "common.cuh"
 #include "k_score.cuh"  // mma.sync, ldmatrix and swizzle helpers
-#include "k_select.cuh"
 #include "tc100.cuh"
 
 namespace gsa {
@@ -45,16 +44,6 @@ struct UnfoldArgs {
   void *out;                 // [B*hq, D]
   int32_t out_bf16;
   float *lse;                // [B*hq] or null
-  // Selection in the prologue (bf16 kernel): instead of reading sel_idx /
-  // sel_score, every CTA of a row selects the row's top k from the scoring
-  // pass's scores and group maxima; split 0 writes the selection out.
-  int32_t select;
-  const float *row_scores;   // [B*hq, score_stride]
-  int32_t score_stride;
-  const float *gmax;         // [B*hq, gmax_stride]: max of every kSelGroup consecutive scores
-  int32_t gmax_stride;
-  int32_t *sel_idx_out;      // [B*hq, k] or null
-  float *sel_score_out;      // [B*hq, k] or null
 };
 
 constexpr int kUnfoldThreads = 128;
@@ -367,17 +356,13 @@ struct UnfoldTcCfg {
   static constexpr uint32_t kStage = 4 * kHalf;           // K and V of two half-steps
   static constexpr int kStages = D == 64 ? 3 : 2;
   static constexpr uint32_t kRingBytes = kUnfoldWarps * kStages * kStage;
-  // ring (1024-aligned; the selection scratch aliases it before the first
-  // copy) | the row's selection and scores [2][ksel] (select mode) |
-  // selected chunks and their list positions [2][per] |
+  // ring (1024-aligned) | selected chunks and their list positions [2][per] |
   // half-steps (first raw row, valid rows << 16 | item + 1) [(per + 1) * ceil(chunk / 8) + 1]
   // (the own chunk adds up to ceil(chunk / 8), the last step's pad one)
-  static size_t smem_bytes(int per, int chunk, int ksel = 0) {
+  static size_t smem_bytes(int per, int chunk) {
     const size_t hpc = static_cast<size_t>((chunk + 7) / 8);
-    return kRingBytes + 1024 + 2 * static_cast<size_t>(ksel) * 4 + 2 * static_cast<size_t>(per) * 4 +
-           ((static_cast<size_t>(per) + 1) * hpc + 1) * 8;
+    return kRingBytes + 1024 + 2 * static_cast<size_t>(per) * 4 + ((static_cast<size_t>(per) + 1) * hpc + 1) * 8;
   }
-  static_assert(kRingBytes >= sizeof(SelectSmem), "the selection scratch fits in the ring");
 };
 
 template <int D>
@@ -387,10 +372,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int per = (a.k + a.n_split - 1) / a.n_split;  // list entries of one split
-  const int ksel = a.select ? a.k : 0;
-  int *sel_all = reinterpret_cast<int *>(smem + Cfg::kRingBytes);  // [ksel]
-  float *sel_sc = reinterpret_cast<float *>(sel_all + ksel);        // [ksel]
-  int *items = reinterpret_cast<int *>(sel_sc + ksel);
+  int *items = reinterpret_cast<int *>(smem + Cfg::kRingBytes);
   int *item_pos = items + per;
   __shared__ int n_items_s;
   __shared__ int is_last_s;
@@ -408,27 +390,6 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   int own = min(max(a.own_len[b], 0), a.chunk);
   if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
 
-  const int kk = min(a.k, N);  // chunks selected in select mode
-  if (a.select) {
-    const float *srow = a.row_scores + row * a.score_stride;
-    if (kk >= N) {
-      for (int i = tid; i < N; i += kUnfoldThreads) {
-        sel_all[i] = i;
-        sel_sc[i] = __ldcg(srow + i);
-      }
-    } else if (kk > 0) {
-      select_row(srow, a.gmax + row * a.gmax_stride, N, kk, *reinterpret_cast<SelectSmem *>(smem), sel_all,
-                 sel_sc);
-    }
-    tc::fence_proxy_async_smem();  // the scratch in the ring is rewritten by TMA copies next
-    __syncthreads();
-    if (split == 0)
-      for (int i = tid; i < a.k; i += kUnfoldThreads) {
-        if (a.sel_idx_out) a.sel_idx_out[row * a.k + i] = i < kk ? sel_all[i] : -1;
-        if (a.sel_score_out) a.sel_score_out[row * a.k + i] = i < kk ? sel_sc[i] : neg_inf();
-      }
-  }
-
   // Selected chunks of this split, in list order (invalid entries dropped).
   const int i0 = min(a.k, split * per), i1 = min(a.k, i0 + per);
   if (warp == 0) {
@@ -437,7 +398,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
       const int i = base + lane;
       int m = -1;
       if (i < i1) {
-        m = a.select ? (i < kk ? sel_all[i] : -1) : a.sel_idx[row * a.k + i];
+        m = a.sel_idx[row * a.k + i];
         if (m >= N) {
           flag_error(a.status, GSA_DEVERR_BAD_INDEX);
           m = -1;
@@ -579,8 +540,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
     if (a.exclude)
 #pragma unroll
       for (int hs = 0; hs < 2; ++hs)
-        if (item[hs] >= 0)
-          z[hs] = (a.select ? sel_sc[item_pos[item[hs]]] : a.sel_score[row * a.k + item_pos[item[hs]]]) * kLog2e;
+        if (item[hs] >= 0) z[hs] = a.sel_score[row * a.k + item_pos[item[hs]]] * kLog2e;
     float qm = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
     qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
     qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));

@@ -143,35 +143,34 @@ def test_separate_entry_points_match_fused():
     compare(x, cfg, fused=False, what="separate calls")
 
 
-def _select_attend(x, cfg, excl):
-    """gsa_score_gists, then gsa_select_attend (selection + unfold in one launch)."""
+@pytest.mark.parametrize("excl", [False, True], ids=["default", "exclude"])
+def test_score_select_entry_point(excl):
+    """gsa_score_select (scoring with the selection in its tail) then
+    gsa_unfold_attend computes the fused step, and its scores are
+    gsa_score_gists's."""
+    cfg = W.scaled(W.LLAMA_8X, batch=3, context=1500 * 8)
+    x = W.decode_inputs(cfg, device="cuda", own_len=5, ragged=[1500, 999, 64])
     B, hq, d = x["q"].shape
     hkv, n_max, t_max = x["gist_k"].shape[1], x["gist_k"].shape[2], x["raw_k"].shape[2]
     desc = G.make_desc(B, hq, hkv, d, cfg.chunk, n_max, t_max, cfg.topk, excl, 0.0, G.GSA_BF16, G.GSA_F32)
     ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device="cuda")
     G.gsa_workspace_init(ws)
-    scores = torch.empty((B, hq, n_max), dtype=torch.float32, device="cuda")
+    scores = torch.full((B, hq, n_max), float("nan"), dtype=torch.float32, device="cuda")
     out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
     lse = torch.empty((B, hq), dtype=torch.float32, device="cuda")
     sel = torch.full((B, hq, cfg.topk), -7, dtype=torch.int32, device="cuda")
     ssc = torch.empty((B, hq, cfg.topk), dtype=torch.float32, device="cuda")
-    G.gsa_score_gists(desc, x["q"], x["gist_k"], None if excl else x["gist_v"], x["n_gists"], scores, ws)
-    G.gsa_select_attend(desc, scores, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel,
-                        ssc, out, lse, ws)
+    G.gsa_score_select(desc, x["q"], x["gist_k"], None if excl else x["gist_v"], x["n_gists"], scores, sel, ssc, ws)
+    G.gsa_unfold_attend(desc, x["q"], x["raw_k"], x["raw_v"], x["gist_v"], x["n_gists"], x["own_len"], sel, ssc,
+                        G.GSA_PRIOR_NONE if excl else G.GSA_PRIOR_GISTS, out, lse, ws)
     torch.cuda.synchronize()
     assert G.gsa_workspace_status(ws) == 0
-    return out, lse, sel, ssc
-
-
-@pytest.mark.parametrize("excl", [False, True], ids=["default", "exclude"])
-def test_select_attend_entry_point(excl):
-    """gsa_score_gists followed by gsa_select_attend computes the fused step."""
-    cfg = W.scaled(W.LLAMA_8X, batch=3, context=1500 * 8)
-    x = W.decode_inputs(cfg, device="cuda", own_len=5, ragged=[1500, 999, 64])
     a = run_gpu(x, cfg, excl, fused=True)
-    out, lse, sel, ssc = _select_attend(x, cfg, excl)
+    b = run_gpu(x, cfg, excl, fused=False)
     assert torch.equal(a[2], sel) and torch.equal(a[3], ssc)
     assert (a[0] - out).abs().max().item() <= 1e-5 and (a[1] - lse).abs().max().item() <= 1e-5
+    valid = torch.isfinite(b[4])
+    assert torch.equal(scores[valid], b[4][valid])
 
 
 TIE_CASES = [
