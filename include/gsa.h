@@ -206,12 +206,14 @@ gsa_status gsa_unfold_attend(const gsa_desc *desc, const void *q, const void *ra
                              const int32_t *sel_idx, const float *sel_score, int32_t prior, void *out, float *lse,
                              void *ws, size_t ws_bytes, void *stream);
 
-/* Steps 1 and 2 in one launch ([nl] Scoring + Selectie; [ja] 2.1 steps
- * 2-3), bf16 inputs only (GSA_ERR_UNSUPPORTED otherwise): gsa_score_gists,
- * and in the same kernel the top-k selection of every row -- the CTA that
- * finishes a (b, kv head) group last selects for the group's query heads
- * while other groups are still being scored.  The selection is the one
- * gsa_topk_select writes (ties to the lower chunk index).
+/* Steps 1 and 2 ([nl] Scoring + Selectie; [ja] 2.1 steps 2-3), bf16
+ * inputs only (GSA_ERR_UNSUPPORTED otherwise): gsa_score_gists and, in the
+ * same kernel, the top-k selection of every row -- the last CTAs to finish
+ * a (b, kv head) group select for the group's query heads while other
+ * groups are still being scored.  Rows longer than 4096 gists (d = 64) or
+ * 8192 (d = 128) take gsa_topk_select's kernel after the scoring instead.
+ * The selection is the one gsa_topk_select writes (ties to the lower chunk
+ * index).
  *   scores    [B, hq, n_max] fp32 out, or NULL (ws holds them)
  *   sel_idx, sel_score  [B, hq, topk] out, or NULL (ws holds them)
  * In default mode ws also receives the gist partial for gsa_unfold_attend
@@ -244,7 +246,7 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
  *    GSA_ERR_WORKSPACE before anything is enqueued.
  *  * No cudaMalloc/cudaFree or allocating library routine is called; the
  *    call enqueues a small cudaMemsetAsync that clears the status word and
- *    per-row counters, then the decode kernels.
+ *    the per-row and per-group counters, then the decode kernels.
  *  * All calls in the process share the one array and it keeps the last
  *    call's contents: calls whose GPU work may overlap (different streams
  *    without ordering, or several host threads) race and corrupt each

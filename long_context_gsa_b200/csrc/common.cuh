@@ -38,6 +38,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Acquire load of a flag or counter another CTA updates (gpu scope).
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void flag_error(uint32_t *status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }

@@ -40,7 +40,7 @@ inline float resolve_scale(const gsa_desc *d) {
 }
 
 struct Layout {
-  size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0, gmax = 0;
+  size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
   size_t unit_counters = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
   size_t meta2_scores = 0, meta2_idx = 0, cand1_scores = 0, cand1_ids = 0, cand1_count = 0;
@@ -92,8 +92,11 @@ gsa_status check_h2desc(const gsa_desc *d, const gsa_h2desc *h) {
   return GSA_OK;
 }
 
-// Group maxima per row of scores: one per kSelGroup gists.
-inline int gmax_stride(const gsa_desc *d) { return (d->n_max + kSelGroup - 1) / kSelGroup; }
+// Whether the scoring kernel can select in its tail: bf16 (tensor-core
+// scorer) and rows short enough for the selecting threads' registers.
+inline bool tail_select_ok(const gsa_desc *d) {
+  return d->dtype == GSA_BF16 && d->n_max <= kRowSelThreads * (d->d == 64 ? 32 : 64);
+}
 
 Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   Layout L;
@@ -124,9 +127,8 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     L.total = off;
     return L;
   }
+  take(L.unit_counters, rows * 8);  // with the status and counters: the prefix a scratch-free call clears
   take(L.scores, rows * d->n_max * 4);
-  take(L.gmax, rows * gmax_stride(d) * 4);
-  take(L.unit_counters, rows * 4);
   take(L.sel_idx, rows * d->topk * 4);
   take(L.sel_score, rows * d->topk * 4);
   take(L.part_g, rows * kScoreSplitMax * rec);
@@ -315,9 +317,8 @@ gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dt
 // Score rows of `keys` (gists or meta-gists) against q; optional partial.
 gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const void *vals, const int32_t *n_gists,
                      int count_div, int rows_cap, float *scores, int score_stride, float *part, int *splits_out,
-                     uint32_t *status, void *stream, float *gmax = nullptr, int gmax_stride = 0,
-                     uint32_t *zero_rows = nullptr, uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr,
-                     float *sel_score = nullptr) {
+                     uint32_t *status, void *stream, uint32_t *zero_rows = nullptr,
+                     uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr, float *sel_score = nullptr) {
   const int group = d->hq / d->hkv;
   const bool with_v = part != nullptr;
   const ScorePlan plan = plan_score(d, rows_cap, with_v);
@@ -337,10 +338,8 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
   sa.score_stride = score_stride;
   sa.part = part;
   sa.n_split = splits;
-  sa.gmax = mma ? gmax : nullptr;
-  sa.gmax_stride = gmax_stride;
   sa.zero_rows = mma ? zero_rows : nullptr;
-  sa.unit_counters = mma && gmax && scores ? unit_counters : nullptr;
+  sa.unit_counters = mma && scores && sel_idx ? unit_counters : nullptr;
   sa.topk = d->topk;
   sa.sel_idx = sel_idx;
   sa.sel_score = sel_score;
@@ -976,12 +975,11 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
   float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
   float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
   int n_prior = 0;
-  if (desc->dtype == GSA_BF16) {
+  if (tail_select_ok(desc)) {
     // Two launches: scoring with the selection in its tail (it also re-arms
     // the unfold's counters), then the unfold.
     GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
-                      stream, reinterpret_cast<float *>(at(ws, L.gmax)), gmax_stride(desc),
-                      reinterpret_cast<uint32_t *>(at(ws, L.counters)),
+                      stream, reinterpret_cast<uint32_t *>(at(ws, L.counters)),
                       reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss));
     return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, part, part ? n_prior : 0, out, lse, L,
                       ws, stream);
@@ -1018,9 +1016,16 @@ gsa_status gsa_score_select(const gsa_desc *desc, const void *q, const void *gis
   int32_t *si = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(at(ws, L.sel_idx));
   float *ss = sel_score ? sel_score : reinterpret_cast<float *>(at(ws, L.sel_score));
   float *part = desc->exclude_unselected ? nullptr : reinterpret_cast<float *>(at(ws, L.part_g));
-  return run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, sc, desc->n_max, part, nullptr,
-                   reinterpret_cast<uint32_t *>(at(ws, L.status)), stream, reinterpret_cast<float *>(at(ws, L.gmax)),
-                   gmax_stride(desc), reinterpret_cast<uint32_t *>(at(ws, L.counters)),
+  uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
+  if (!tail_select_ok(desc)) {  // rows too long for the tail: the separate selection kernel
+    GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, sc, desc->n_max, part, nullptr, status,
+                      stream));
+    if (desc->topk == 0) return GSA_OK;
+    return run_topk(desc->batch * desc->hq, desc->hq, sc, desc->n_max, n_gists, 1, nullptr, desc->topk, nullptr, si,
+                    ss, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+  }
+  return run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, sc, desc->n_max, part, nullptr, status, stream,
+                   reinterpret_cast<uint32_t *>(at(ws, L.counters)),
                    reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss);
 }
 
@@ -1379,9 +1384,9 @@ extern "C" gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, co
   GSA_TRY(opt_ptr(sel_score));
   void *ws = nullptr;
   GSA_TRY(noalloc_scratch(&ws));
-  // The status word and the per-row counters must start at zero; the array
-  // keeps whatever the previous call left there.
-  const size_t zero_bytes = L.counters + static_cast<size_t>(desc->batch) * desc->hq * 4;
+  // The status word and the per-row and per-group counters must start at
+  // zero; the array keeps whatever the previous call (of any shape) left.
+  const size_t zero_bytes = L.unit_counters + static_cast<size_t>(desc->batch) * desc->hq * 8;
   if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GSA_ERR_CUDA;
   return gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score, ws,
                     GSA_NOALLOC_SCRATCH_BYTES, stream);

@@ -35,13 +35,11 @@ struct ScoreArgs {
   int32_t score_stride;
   float *part;            // [B*hq, n_split, D+4] or null
   int32_t n_split;
-  float *gmax;            // [B*hq, gmax_stride] or null: max score of gists 16i .. 16i+15 (tensor-core path)
-  int32_t gmax_stride;
   uint32_t *zero_rows;    // [B*hq] or null: zeroed for this kernel's heads (re-arms the unfold's counters)
-  // Selection in the tail (tensor-core path, needs scores and gmax): the
-  // CTA that arrives last at its group's counter selects the top k of each
-  // of the group's query heads, one warp per head.
-  uint32_t *unit_counters;  // [B*hkv*head_split] or null; re-armed to 0 by the last CTA
+  // Selection in the tail (tensor-core path, needs scores): the last CTAs
+  // to finish a (b, kv head) group select the top k of the group's query
+  // heads, 128 threads per head.
+  uint32_t *unit_counters;  // [2 * B*hkv*head_split] (arrivals, selectors done) or null; re-armed to 0
   int32_t topk;
   int32_t *sel_idx;       // [B*hq, topk]
   float *sel_score;       // [B*hq, topk] or null
@@ -60,10 +58,9 @@ __device__ __forceinline__ void mma_16816_bf16(float c[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Slice of rows [n0, n1) handled by `split`; slices are multiples of 16,
-// so every group of 16 consecutive rows (a group maximum) lies in one slice.
+// Slice of rows [n0, n1) handled by `split`; slices are multiples of 8.
 __device__ __forceinline__ void score_slice(int N, int n_split, int split, int &n0, int &n1) {
-  const int per = ((N + n_split - 1) / n_split + 15) & ~15;
+  const int per = ((N + n_split - 1) / n_split + 7) & ~7;
   n0 = split * per;
   n1 = min(N, n0 + per);
   if (n1 < n0) n1 = n0;
@@ -87,12 +84,26 @@ struct ScoreMmaCfg {
   static constexpr uint32_t kBarOff = (kCntOff + (2 * kStages + 1) * 4 + 7) & ~7u;
   static constexpr uint32_t kSmemBytes = kBarOff + kStages * 8 + 1024;  // + alignment slack
   static_assert(kStages * kStageBytes >= kWarps * GH * D * 4 || !WITH_V, "merge buffer fits in the ring");
-  // warps selecting at once in the tail (their scratch lives in the ring)
-  static constexpr int kSelWarps = (kStages * kStageBytes) / sizeof(WarpSelSmem) < kWarps
-                                       ? static_cast<int>((kStages * kStageBytes) / sizeof(WarpSelSmem))
-                                       : kWarps;
-  static_assert(kSelWarps >= 1, "one selection scratch fits in the ring");
+  // thread groups selecting at once in the tail (their scratch lives in the ring)
+  static constexpr int kSelGroups = kThreads / kRowSelThreads;
+  // longest row the tail selects (its scratch holds the row)
+  static constexpr int kSelMaxN = D == 64 ? 4096 : 8192;
+  static_assert(kSelGroups >= 1 && kSelGroups * sizeof(SelSmem<kSelMaxN>) <= kStages * kStageBytes,
+                "selection scratch fits in the ring");
 };
+
+// The tail's selector CTAs of a group: the last `selectors` to arrive.
+__device__ __forceinline__ int score_tail_selectors(int n_split, int nh, int groups) {
+  return min(n_split, (nh + groups - 1) / groups);
+}
+
+// A selector CTA is done: the last one re-arms the group's two counters.
+__device__ __forceinline__ void score_tail_done(uint32_t *cnt, int selectors) {
+  if (atomicAdd(&cnt[1], 1u) == static_cast<uint32_t>(selectors - 1)) {
+    cnt[0] = 0u;
+    cnt[1] = 0u;
+  }
+}
 
 // Rescaling threshold (base-2 units): the running max used for the
 // exponentials is only raised when a score exceeds it by more than this,
@@ -261,20 +272,6 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
             s[nt][e] = c[nt][e] * a.scale_log2;
           }
         }
-      if (a.gmax) {
-        // the maximum of this warp's 16 rows per head (lanes 4g .. 4g+3 hold
-        // head g's scores), in the same units as the stored scores
-        float gm = neg_inf();
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-            if (s[nt][e] > neg_inf()) gm = fmaxf(gm, c[nt][e] * a.scale);
-        gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 1));
-        gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 2));
-        if (t4 == 0 && g < nh)
-          a.gmax[(static_cast<size_t>(b) * a.hq + h0 + g) * a.gmax_stride + (n0 + t * kTile + rw) / 16] = gm;
-      }
       if (WITH_V) {
         // lazy reference: raised only when this warp's rows exceed it by
         // more than kRescaleSlack; the head's accumulators then rescale
@@ -348,7 +345,11 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
         const int tl = *reinterpret_cast<volatile int *>(&last_issued[s]);
         if (tl >= 0) mbar_wait(&bars[s], (tl / kStages) & 1);
       }
-      if (a.unit_counters && atomicAdd(&a.unit_counters[unit], 1u) == gridDim.x - 1) a.unit_counters[unit] = 0u;
+      if (a.unit_counters) {  // arrive; a selector that cannot select still counts as done
+        const int S = score_tail_selectors(gridDim.x, nh, Cfg::kSelGroups);
+        if (static_cast<int>(atomicAdd(&a.unit_counters[2 * unit], 1u)) >= static_cast<int>(gridDim.x) - S)
+          score_tail_done(a.unit_counters + 2 * unit, S);
+      }
     }
     __syncthreads();
     return;
@@ -400,28 +401,53 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
     }
   }
   if (a.unit_counters) {
-    // The group's last CTA selects: every CTA's scores and group maxima are
-    // visible to it once it has seen the others' arrivals (fence, counter,
-    // fence).  The ring is free, and holds the warps' selection scratch.
-    __shared__ int last_s;
+    // The last S CTAs to arrive at the group's counter select, one query
+    // head per 128-thread group: each waits (bounded) until every CTA of
+    // the group has arrived, after which all scores are visible to it
+    // (writers: fence, then arrive; readers: acquire the count).  The ring
+    // is free and holds the groups' selection scratch.
+    __shared__ int arrive_s, ok_s;
+    uint32_t *cnt2 = a.unit_counters + 2 * unit;
+    const int n_split = static_cast<int>(gridDim.x);
+    const int S = score_tail_selectors(n_split, nh, Cfg::kSelGroups);
     __syncthreads();
     if (tid == 0) {
       __threadfence();
-      const bool last = atomicAdd(&a.unit_counters[unit], 1u) == gridDim.x - 1;
-      if (last) {
-        a.unit_counters[unit] = 0u;
-        __threadfence();
-      }
-      last_s = last;
+      arrive_s = static_cast<int>(atomicAdd(&cnt2[0], 1u));
     }
     __syncthreads();
-    if (last_s && warp < Cfg::kSelWarps) {
-      WarpSelSmem &wsm = reinterpret_cast<WarpSelSmem *>(smem)[warp];
-      for (int j = warp; j < nh; j += Cfg::kSelWarps) {
-        const size_t row = static_cast<size_t>(b) * a.hq + h0 + j;
-        warp_select(a.scores + row * a.score_stride, a.gmax + row * a.gmax_stride, N, a.topk, wsm,
-                    a.sel_idx + row * a.topk, a.sel_score ? a.sel_score + row * a.topk : nullptr);
+    const int si = arrive_s - (n_split - S);  // selector index; negative: not a selector
+    if (si >= 0) {
+      if (tid == 0) {
+        int ok = 1;
+        uint64_t t0 = 0;
+        for (uint32_t it = 0; ld_acquire_u32(&cnt2[0]) < static_cast<uint32_t>(n_split); ++it) {
+          if ((it & 15u) == 0) {
+            const uint64_t now = global_timer_ns();
+            if (!t0) t0 = now;
+            else if (now - t0 > kWaitLimitNs) {
+              ok = 0;
+              flag_error(a.status, GSA_DEVERR_TIMEOUT);
+              break;
+            }
+          }
+          __nanosleep(100);
+        }
+        ok_s = ok;
       }
+      __syncthreads();
+      if (ok_s) {
+        const int grp = tid / kRowSelThreads;
+        SelSmem<Cfg::kSelMaxN> &ssm = reinterpret_cast<SelSmem<Cfg::kSelMaxN> *>(smem)[grp];
+        for (int j = si * Cfg::kSelGroups + grp; j < nh; j += S * Cfg::kSelGroups) {
+          const size_t row = static_cast<size_t>(b) * a.hq + h0 + j;
+          group_select<Cfg::kSelMaxN>(a.scores + row * a.score_stride, N, a.topk, tid % kRowSelThreads, ssm, 1 + grp,
+                                      a.status, a.sel_idx + row * a.topk,
+                                      a.sel_score ? a.sel_score + row * a.topk : nullptr);
+        }
+      }
+      __syncthreads();
+      if (tid == 0) score_tail_done(cnt2, S);
     }
   }
 }
