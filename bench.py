@@ -55,6 +55,9 @@ def parse():
     p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep,kvreuse_qwen7b",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    p.add_argument("--sweep", action="store_true",
+                   help="context-length sweep of flat, one-level and two-level H-GSA decode (bytes and time per "
+                        "step); one JSON line per point, then a summary line")
     return p.parse_args()
 
 
@@ -692,6 +695,62 @@ def measure_extra(G, W, args, dev, flush, hbm, bf16):
     return extra
 
 
+SWEEP_CONTEXTS = (131072, 524288, 2097152)
+
+
+def sweep_config(context, levels):
+    """The H-GSA workload shape (32 query / 8 kv heads, d = 128, chunks of 32,
+    top-64) at one context length and batch 1: flat (levels 0), one meta
+    level (16 gists per meta-gist, keep 32) or two (16 meta-gists per level-2
+    meta-gist, keep 8)."""
+    import long_context_gsa_b200.workloads as W
+    kw = dict(group=16, topk_meta=32) if levels >= 1 else {}
+    if levels == 2:
+        kw.update(group2=16, topk_meta2=8)
+    return W.DecodeConfig(f"hgsa_sweep_{context // 1024}k_l{levels}", 1, 32, 8, 128, 32, context, 64, "bf16",
+                          seed=20260100 + levels, **kw)
+
+
+def run_sweep(args):
+    """How bytes and time per decode step grow with the context (the pages'
+    O(log n) claim for H-GSA): flat GSA reads every gist key and value; one
+    meta level reads every meta-gist and the chosen groups' children; two
+    levels read every level-2 meta-gist, the chosen level-1 candidates and
+    their gist children."""
+    import long_context_gsa_b200 as G
+    import long_context_gsa_b200.workloads as W
+    G.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = Flusher(dev)
+    hbm, _, _ = peaks()
+    points = []
+    for ctx in SWEEP_CONTEXTS:
+        for levels in (0, 1, 2):
+            cfg = sweep_config(ctx, levels)
+            if levels == 0:
+                m = measure_flat(G, W, cfg, dev, args, flush, cfg.seed)
+                r = flat_summary(cfg, m, hbm)
+                del m
+            elif levels == 1:
+                r = measure_hgsa(G, W, cfg, dev, args, flush, hbm)
+            else:
+                r = measure_hgsa2(G, W, cfg, dev, args, flush, hbm)
+            torch.cuda.empty_cache()
+            pt = {"sweep": "hgsa_levels", "context": ctx, "n_gists": cfg.n_gists, "meta_levels": levels,
+                  "ms_per_step": r["ms_per_step"], "alg_bytes": r["step_hbm"]["alg_bytes"],
+                  "hbm_frac": r["step_hbm"]["frac"], "head_queries_per_s": r["value"]}
+            points.append(pt)
+            print(json.dumps(pt), flush=True)
+    summary = {"sweep": "hgsa_levels", "contexts": list(SWEEP_CONTEXTS), "points": len(points)}
+    for levels in (0, 1, 2):
+        ps = [p for p in points if p["meta_levels"] == levels]
+        # growth per 4x context: bytes and time ratio between consecutive contexts
+        summary[f"l{levels}_bytes_x4"] = [round(b["alg_bytes"] / a["alg_bytes"], 3) for a, b in zip(ps, ps[1:])]
+        summary[f"l{levels}_time_x4"] = [round(b["ms_per_step"] / a["ms_per_step"], 3) for a, b in zip(ps, ps[1:])]
+    print(json.dumps(summary), flush=True)
+
+
 def run_gsa(args, world, rank, local):
     import long_context_gsa_b200 as G
     import long_context_gsa_b200.workloads as W
@@ -845,6 +904,9 @@ def run_reference(args, world, rank):
 def main():
     args = parse()
     world, rank, local = dist_env()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         res = run_reference(args, world, rank)
     else:

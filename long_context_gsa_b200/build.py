@@ -60,5 +60,22 @@ def build_library(force: bool = False, verbose: bool = False) -> Path:
     return LIB
 
 
+def build_variant(out: Path, defines: dict) -> Path:
+    """Build a copy of the library with extra preprocessor definitions (for
+    tests that need a shortened wait limit, say) at `out`; rebuilt when any
+    source is newer than it."""
+    out = Path(out)
+    if out.exists() and not any(s.stat().st_mtime > out.stat().st_mtime for s in _sources()):
+        return out
+    tmp = out.with_suffix(f".so.{os.getpid()}.tmp")
+    flags = [f"-D{k}={v}" for k, v in defines.items()]
+    res = subprocess.run([nvcc(), *NVCC_FLAGS, *flags, str(CSRC / "gsa_api.cu"), "-o", str(tmp)], capture_output=True,
+                         text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr[-8000:]}")
+    os.replace(tmp, out)
+    return out
+
+
 if __name__ == "__main__":
     print(build_library(force="--force" in sys.argv, verbose="-v" in sys.argv))

@@ -17,9 +17,21 @@ namespace gsa {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Longest time a thread waits on an mbarrier before it gives up and flags
-// GSA_DEVERR_TIMEOUT (nanoseconds of %globaltimer).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Longest time a thread waits on an mbarrier (or a counter another CTA
+// advances) before it gives up and flags GSA_DEVERR_TIMEOUT (nanoseconds of
+// %globaltimer).  A test build may shorten it with -DGSA_WAIT_LIMIT_NS.
+#ifndef GSA_WAIT_LIMIT_NS
+#define GSA_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = GSA_WAIT_LIMIT_NS;
+
+// Extra transaction bytes that some copy barriers expect: 0 in the library.
+// The failure-detection test builds a variant with 16, so those barriers
+// never complete (their copies land, the count stays short) and the bounded
+// waits must expire, flag GSA_DEVERR_TIMEOUT and let the kernel return.
+#ifndef GSA_TEST_STALL_BYTES
+#define GSA_TEST_STALL_BYTES 0u
+#endif
 
 // Partial softmax record: base-2 max, sum, then `d` accumulator floats.
 // Stored as float[d + 4] (the two pad floats keep the accumulator 16-byte

@@ -371,7 +371,7 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
 
 gsa_status run_topk(int rows, int hq, const float *scores, int stride, const int32_t *n_gists, int count_div,
                     const int32_t *counts, int k, const int32_t *id_map, int32_t *sel_idx, float *sel_score,
-                    uint32_t *counters, void *stream) {
+                    uint32_t *counters, void *stream, uint32_t *status = nullptr) {
   TopkArgs ta;
   ta.scores = scores;
   ta.stride = stride;
@@ -384,6 +384,7 @@ gsa_status run_topk(int rows, int hq, const float *scores, int stride, const int
   ta.sel_idx = sel_idx;
   ta.sel_score = sel_score;
   ta.counters = counters;
+  ta.status = status;
   ta.smem_cap = std::min(stride, kTopkSmemCap);
   const dim3 grid(rows), block(kTopkRegThreads);
   constexpr size_t kRowBytes = kTopkRegThreads * 4;  // staged row bytes per key a thread holds
@@ -868,7 +869,8 @@ gsa_status gsa_topk_select(const gsa_desc *desc, const float *scores, const int3
   if (ws_bytes < L.total) return GSA_ERR_WORKSPACE;
   if (desc->topk == 0) return GSA_OK;
   return run_topk(desc->batch * desc->hq, desc->hq, scores, desc->n_max, n_gists, 1, nullptr, desc->topk, nullptr,
-                  sel_idx, sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream);
+                  sel_idx, sel_score, reinterpret_cast<uint32_t *>(at(ws, L.counters)), stream,
+                  reinterpret_cast<uint32_t *>(at(ws, L.status)));
 }
 
 gsa_status gsa_topp_select(const gsa_desc *desc, const float *scores, const int32_t *n_gists, float top_p,

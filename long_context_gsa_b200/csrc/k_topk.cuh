@@ -31,6 +31,7 @@ struct TopkArgs {
   float *sel_score;       // [rows, k] or null
   uint32_t *counters;     // optional: counters[row] is re-armed to 0
   int32_t smem_cap;       // keys kept in shared memory when n <= smem_cap
+  uint32_t *status;       // optional: device status word (GSA_DEVERR_* bits)
 };
 
 constexpr int kTopkThreads = 512;
@@ -481,10 +482,14 @@ __global__ void __launch_bounds__(kTopkRegThreads, KPT <= 16 ? 4 : 1) k_topk(con
   // from global memory directly
   const int n4 = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0 ? (n & ~3) : 0;
   if (tid == 0) {
-    mbar_arrive_expect_tx(&load_bar, static_cast<uint32_t>(n4) * 4u);
+    mbar_arrive_expect_tx(&load_bar, static_cast<uint32_t>(n4) * 4u + GSA_TEST_STALL_BYTES);
     if (n4 > 0) bulk_g2s(srow_s, srow, static_cast<uint32_t>(n4) * 4u, &load_bar);
   }
-  const int staged = mbar_wait(&load_bar, 0) ? n4 : 0;
+  const bool landed = mbar_wait(&load_bar, 0);
+  if (!landed && tid == 0) flag_error(a.status, GSA_DEVERR_TIMEOUT);
+  // after a timeout the copy has had kWaitLimitNs to land; the row is read
+  // from global memory either way, so a late copy rewrites the same values
+  const int staged = landed ? n4 : 0;
   for (int i = staged + tid; i < n; i += T) srow_s[i] = __ldcg(srow + i);  // the tail (and a timed-out copy)
   __syncthreads();
 

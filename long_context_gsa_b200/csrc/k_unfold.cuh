@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   auto issue = [&](int li) {
     const int step = warp + kUnfoldWarps * li, st = li % S;
     uint8_t *dst = ring + st * Cfg::kStage;
-    mbar_arrive_expect_tx(&bars[warp][st], Cfg::kStage);
+    mbar_arrive_expect_tx(&bars[warp][st], Cfg::kStage + GSA_TEST_STALL_BYTES);
 #pragma unroll
     for (int hs = 0; hs < 2; ++hs) {
       int first, valid, item;
