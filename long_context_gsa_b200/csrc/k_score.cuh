@@ -40,7 +40,6 @@ struct ScoreArgs {
   // to finish a (b, kv head) group select the top k of the group's query
   // heads, 128 threads per head.
   uint32_t *unit_counters;  // [2 * B*hkv*head_split] (arrivals, selectors done) or null; re-armed to 0
-  uint32_t *ready;        // [B*hkv] or null: +1 when a (b, kv head [x head half]) group's selection is written
   int32_t topk;
   int32_t *sel_idx;       // [B*hq, topk]
   float *sel_score;       // [B*hq, topk] or null
@@ -98,18 +97,11 @@ __device__ __forceinline__ int score_tail_selectors(int n_split, int nh, int gro
   return min(n_split, (nh + groups - 1) / groups);
 }
 
-// A selector CTA is done (its selection written and fenced): the last one
-// re-arms the group's two counters and announces the group's selection to
-// the unfold (release: fence, then the flag).
-__device__ __forceinline__ void score_tail_done(uint32_t *cnt, int selectors, uint32_t *ready) {
-  __threadfence();
+// A selector CTA is done: the last one re-arms the group's two counters.
+__device__ __forceinline__ void score_tail_done(uint32_t *cnt, int selectors) {
   if (atomicAdd(&cnt[1], 1u) == static_cast<uint32_t>(selectors - 1)) {
     cnt[0] = 0u;
     cnt[1] = 0u;
-    if (ready) {
-      __threadfence();
-      atomicAdd(ready, 1u);
-    }
   }
 }
 
@@ -356,7 +348,7 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
       if (a.unit_counters) {  // arrive; a selector that cannot select still counts as done
         const int S = score_tail_selectors(gridDim.x, nh, Cfg::kSelGroups);
         if (static_cast<int>(atomicAdd(&a.unit_counters[2 * unit], 1u)) >= static_cast<int>(gridDim.x) - S)
-          score_tail_done(a.unit_counters + 2 * unit, S, a.ready ? a.ready + b * a.hkv + kvh : nullptr);
+          score_tail_done(a.unit_counters + 2 * unit, S);
       }
     }
     __syncthreads();
@@ -455,7 +447,7 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
         }
       }
       __syncthreads();
-      if (tid == 0) score_tail_done(cnt2, S, a.ready ? a.ready + b * a.hkv + kvh : nullptr);
+      if (tid == 0) score_tail_done(cnt2, S);
     }
   }
 }

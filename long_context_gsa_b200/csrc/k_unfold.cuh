@@ -44,13 +44,6 @@ struct UnfoldArgs {
   void *out;                 // [B*hq, D]
   int32_t out_bf16;
   float *lse;                // [B*hq] or null
-  // With the scoring kernel's tail selection (bf16 decode): instead of
-  // waiting for the whole scoring grid, a CTA waits until its (b, kv head)
-  // group's flag reaches ready_target (the group's head halves); the last
-  // row of the group to finish re-arms the flag.
-  uint32_t *ready;           // [B*hkv] or null
-  uint32_t *ready_done;      // [B*hkv]
-  int32_t ready_target;
 };
 
 constexpr int kUnfoldThreads = 128;
@@ -159,14 +152,6 @@ __device__ void unfold_finish(const UnfoldArgs &a, size_t row, int split, const 
                           a.prior ? a.prior + row * a.n_prior * (D + kPartHeader) : nullptr};
   const int counts[2] = {a.n_split, a.prior ? a.n_prior : 0};
   combine_records<D>(recs, counts, 2, a.out, row, a.out_bf16, a.lse);
-  if (a.ready && tid == 0) {
-    // every CTA of this row has passed its wait; the group's last row re-arms its flag
-    const size_t bk = (row / a.hq) * a.hkv + (row % a.hq) / a.group;
-    if (atomicAdd(&a.ready_done[bk], 1u) == static_cast<uint32_t>(a.group - 1)) {
-      a.ready_done[bk] = 0u;
-      a.ready[bk] = 0u;
-    }
-  }
 }
 
 template <int D, typename T>
@@ -400,33 +385,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   const size_t row = static_cast<size_t>(b) * a.hq + h;
   const int g = lane >> 2, t4 = lane & 3;
 
-  if (a.ready) {
-    // this row's group selection (bounded wait); everything else this
-    // kernel reads from the scoring pass is written before it
-    __shared__ int ready_ok_s;
-    if (tid == 0) {
-      const uint32_t *flag = a.ready + static_cast<size_t>(b) * a.hkv + kvh;
-      int ok = 1;
-      uint64_t t0 = 0;
-      for (uint32_t it = 0; ld_acquire_u32(flag) < static_cast<uint32_t>(a.ready_target); ++it) {
-        if ((it & 15u) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (!t0) t0 = now;
-          else if (now - t0 > kWaitLimitNs) {
-            ok = 0;
-            break;
-          }
-        }
-        __nanosleep(128);
-      }
-      if (!ok) flag_error(a.status, GSA_DEVERR_TIMEOUT);  // carry on: the results are void, the counts stay whole
-      ready_ok_s = ok;
-    }
-    __syncthreads();
-    (void)ready_ok_s;
-  } else {
-    pdl_wait();
-  }
+  pdl_wait();
   const int N = min(min(max(a.n_gists[b], 0), a.n_max), a.t_max / a.chunk);
   int own = min(max(a.own_len[b], 0), a.chunk);
   if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
