@@ -194,17 +194,19 @@ __device__ __forceinline__ int sel_scan_minmax(int v, uint32_t &lo, uint32_t &hi
 }
 
 
-// Monotone bin of a key: 0 .. 255 for keys >= base, -1 below.
+// Monotone bin of a key: 0 .. 255 for keys >= base, -1 below.  The bins
+// are equal power-of-two key ranges (shift chosen so that hi lands in bin
+// 255 or below): integer subtract and shift, no conversions.
 struct SelBins {
   uint32_t base;
-  float scale;
+  int shift;
   __device__ __forceinline__ void init(uint32_t lo, uint32_t hi) {
     base = lo;
-    const uint32_t span = hi - lo + 1u;
-    scale = 256.0f / (span ? __uint2float_ru(span) : 4294967296.0f);
+    const uint32_t span = hi - lo;
+    shift = span < 256u ? 0 : 24 - __clz(span);  // (span >> shift) < 256
   }
   __device__ __forceinline__ int operator()(uint32_t key) const {
-    return key < base ? -1 : min(255, static_cast<int>(__uint2float_rz(key - base) * scale));
+    return key < base ? -1 : static_cast<int>((key - base) >> shift);
   }
 };
 
