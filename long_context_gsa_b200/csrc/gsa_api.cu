@@ -94,10 +94,9 @@ gsa_status check_h2desc(const gsa_desc *d, const gsa_h2desc *h) {
 
 // Whether the scoring kernel can select in its tail: bf16 (tensor-core
 // scorer) and rows short enough for the selecting threads' registers.
-inline bool tail_select_ok(const gsa_desc *d, int rows_cap) {
-  return d->dtype == GSA_BF16 && rows_cap <= kRowSelThreads * (d->d == 64 ? 32 : 64);
+inline bool tail_select_ok(const gsa_desc *d) {
+  return d->dtype == GSA_BF16 && d->n_max <= kRowSelThreads * (d->d == 64 ? 32 : 64);
 }
-inline bool tail_select_ok(const gsa_desc *d) { return tail_select_ok(d, d->n_max); }
 
 Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
   Layout L;
@@ -319,8 +318,7 @@ gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dt
 gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const void *vals, const int32_t *n_gists,
                      int count_div, int rows_cap, float *scores, int score_stride, float *part, int *splits_out,
                      uint32_t *status, void *stream, uint32_t *zero_rows = nullptr,
-                     uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr, float *sel_score = nullptr,
-                     int topk = -1) {
+                     uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr, float *sel_score = nullptr) {
   const int group = d->hq / d->hkv;
   const bool with_v = part != nullptr;
   const ScorePlan plan = plan_score(d, rows_cap, with_v);
@@ -342,7 +340,7 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
   sa.n_split = splits;
   sa.zero_rows = mma ? zero_rows : nullptr;
   sa.unit_counters = mma && scores && sel_idx ? unit_counters : nullptr;
-  sa.topk = topk >= 0 ? topk : d->topk;
+  sa.topk = d->topk;
   sa.sel_idx = sel_idx;
   sa.sel_score = sel_score;
   sa.status = status;
@@ -490,18 +488,11 @@ gsa_status run_hgsa_select(const gsa_desc *d, const gsa_hdesc *hd, const void *q
   const int rows = d->batch * d->hq;
   uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
   float *meta_scores = reinterpret_cast<float *>(at(ws, L.meta_scores));
-  // 1. meta-gist scores; 2. top meta groups (ascending group order), in
-  // the scoring kernel's tail when the meta rows are short enough
-  if (tail_select_ok(d, hd->m_max)) {
-    GSA_TRY(run_score(d, q, meta_k, nullptr, n_gists, hd->group, hd->m_max, meta_scores, hd->m_max, nullptr, nullptr,
-                      status, stream, nullptr, reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), meta_idx,
-                      nullptr, hd->topk_meta));
-  } else {
-    GSA_TRY(run_score(d, q, meta_k, nullptr, n_gists, hd->group, hd->m_max, meta_scores, hd->m_max, nullptr, nullptr,
-                      status, stream));
-    GSA_TRY(run_topk(rows, d->hq, meta_scores, hd->m_max, n_gists, hd->group, nullptr, hd->topk_meta, nullptr,
-                     meta_idx, nullptr, nullptr, stream));
-  }
+  // 1. meta-gist scores; 2. top meta groups (ascending group order)
+  GSA_TRY(run_score(d, q, meta_k, nullptr, n_gists, hd->group, hd->m_max, meta_scores, hd->m_max, nullptr, nullptr,
+                    status, stream));
+  GSA_TRY(run_topk(rows, d->hq, meta_scores, hd->m_max, n_gists, hd->group, nullptr, hd->topk_meta, nullptr, meta_idx,
+                   nullptr, nullptr, stream));
   // 3. children of the chosen groups (+ trailing gists): scores, ids, partial
   HgsaArgs ha;
   ha.q = q;
@@ -560,16 +551,10 @@ gsa_status run_hgsa2_select(const gsa_desc *d, const gsa_h2desc *h2, const void 
   uint32_t *status = reinterpret_cast<uint32_t *>(at(ws, L.status));
   float *meta2_scores = reinterpret_cast<float *>(at(ws, L.meta2_scores));
   const int g12 = l1.group * l2.group;
-  if (tail_select_ok(d, l2.m_max)) {  // level-2 scores with the top level-2 groups in the kernel's tail
-    GSA_TRY(run_score(d, q, meta2_k, nullptr, n_gists, g12, l2.m_max, meta2_scores, l2.m_max, nullptr, nullptr,
-                      status, stream, nullptr, reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), meta2_idx,
-                      nullptr, l2.topk_meta));
-  } else {
-    GSA_TRY(run_score(d, q, meta2_k, nullptr, n_gists, g12, l2.m_max, meta2_scores, l2.m_max, nullptr, nullptr,
-                      status, stream));
-    GSA_TRY(run_topk(rows, d->hq, meta2_scores, l2.m_max, n_gists, g12, nullptr, l2.topk_meta, nullptr, meta2_idx,
-                     nullptr, nullptr, stream));
-  }
+  GSA_TRY(run_score(d, q, meta2_k, nullptr, n_gists, g12, l2.m_max, meta2_scores, l2.m_max, nullptr, nullptr, status,
+                    stream));
+  GSA_TRY(run_topk(rows, d->hq, meta2_scores, l2.m_max, n_gists, g12, nullptr, l2.topk_meta, nullptr, meta2_idx,
+                   nullptr, nullptr, stream));
   const int splits = hgsa_splits(d);
   HgsaArgs ha;
   ha.q = q;
