@@ -849,8 +849,14 @@ def recorded_kernel(kernel, workload):
     if not rec:
         return {}
     import hashlib
-    src = ROOT / "long_context_gsa_b200" / "csrc" / rec["source"]
-    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != rec["sha"]:
+    sources = rec["source"] if isinstance(rec["source"], list) else [rec["source"]]
+    h = hashlib.sha256()
+    for name in sources:  # every source file the kernel is built from
+        src = ROOT / "long_context_gsa_b200" / "csrc" / name
+        if not src.exists():
+            return {}
+        h.update(src.read_bytes())
+    if h.hexdigest()[:16] != rec["sha"]:
         return {}
     return rec
 

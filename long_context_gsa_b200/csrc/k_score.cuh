@@ -439,10 +439,11 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
       if (ok_s) {
         const int grp = tid / kRowSelThreads;
         SelSmem<Cfg::kSelMaxN> &ssm = reinterpret_cast<SelSmem<Cfg::kSelMaxN> *>(smem)[grp];
+        int use = 0;
         for (int j = si * Cfg::kSelGroups + grp; j < nh; j += S * Cfg::kSelGroups) {
           const size_t row = static_cast<size_t>(b) * a.hq + h0 + j;
           group_select<Cfg::kSelMaxN>(a.scores + row * a.score_stride, N, a.topk, tid % kRowSelThreads, ssm, 1 + grp,
-                                      a.status, a.sel_idx + row * a.topk,
+                                      use, a.status, a.sel_idx + row * a.topk,
                                       a.sel_score ? a.sel_score + row * a.topk : nullptr);
         }
       }

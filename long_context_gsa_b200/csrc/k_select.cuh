@@ -276,7 +276,7 @@ __device__ __noinline__ int sel_exact(SelSmem<NMAX> &sm, int n, int kk, int gtid
 // group (gtid 0 .. 127), which synchronise on named barrier bar_id.
 template <int NMAX>
 __device__ void group_select_row(const float *srow, int n, int kk, int gtid, SelSmem<NMAX> &sm, int bar_id,
-                                 uint32_t *status, int32_t *out_idx, float *out_score) {
+                                 int use, uint32_t *status, int32_t *out_idx, float *out_score) {
   // 0. the row into shared memory (one bulk copy), bitmaps and counts
   // cleared, once every thread is done with the group's previous row
   group_bar(bar_id);
@@ -286,24 +286,27 @@ __device__ void group_select_row(const float *srow, int n, int kk, int gtid, Sel
   const int n4 = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0 ? (n & ~3) : 0;
   if (gtid == 0) {
     sm.nmem = 0;
-    mbar_init(&sm.bar, 1);
-    mbar_fence_init();
+    if (use == 0) {  // the scratch's copy barrier is set up once; each row is one phase of it
+      mbar_init(&sm.bar, 1);
+      mbar_fence_init();
+    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the buffer was last written by this CTA's threads
     mbar_arrive_expect_tx(&sm.bar, static_cast<uint32_t>(n4) * 4u);
     if (n4 > 0) bulk_g2s(sm.row, srow, static_cast<uint32_t>(n4) * 4u, &sm.bar);
   }
   for (int i = n4 + gtid; i < n; i += kRowSelThreads) sm.row[i] = __ldcg(srow + i);
+  const uint32_t parity = static_cast<uint32_t>(use) & 1u;
   if (gtid == 0) {
-    int ok = mbar_wait(&sm.bar, 0);
+    int ok = mbar_wait(&sm.bar, parity);
     if (!ok) {  // flag it; wait once more so that no copy is left in flight
       flag_error(status, GSA_DEVERR_TIMEOUT);
-      mbar_wait(&sm.bar, 0);
+      mbar_wait(&sm.bar, parity);
     }
     sm.info[3] = ok;
   }
   group_bar(bar_id);
-  if (!sm.info[3]) return;   // group-uniform
-  mbar_wait(&sm.bar, 0);     // complete already: makes the copied row visible to this thread
+  if (!sm.info[3]) return;     // group-uniform
+  mbar_wait(&sm.bar, parity);  // complete already: makes the copied row visible to this thread
   // 1. group maxima (four 16-byte loads per group), the bound
   const int n_groups = (n + kSelGroup - 1) / kSelGroup;
   const bool by_group = n_groups >= kk;
@@ -453,8 +456,9 @@ __device__ void group_select_row(const float *srow, int n, int kk, int gtid, Sel
 // The selection of one row: kk = min(k, n) chunks in ascending order, then
 // -1 / -inf padding up to k (n <= NMAX).  Called by the 128 threads of one
 // group.
+// `use` counts the rows this group has selected with this scratch before.
 template <int NMAX>
-__device__ void group_select(const float *srow, int n, int k, int gtid, SelSmem<NMAX> &sm, int bar_id,
+__device__ void group_select(const float *srow, int n, int k, int gtid, SelSmem<NMAX> &sm, int bar_id, int &use,
                              uint32_t *status, int32_t *out_idx, float *out_score) {
   const int kk = min(k, n);
   if (kk >= n) {
@@ -463,7 +467,8 @@ __device__ void group_select(const float *srow, int n, int k, int gtid, SelSmem<
       if (out_score) out_score[i] = __ldcg(srow + i);
     }
   } else if (kk > 0) {
-    group_select_row<NMAX>(srow, n, kk, gtid, sm, bar_id, status, out_idx, out_score);
+    group_select_row<NMAX>(srow, n, kk, gtid, sm, bar_id, use, status, out_idx, out_score);
+    ++use;
   }
   for (int i = kk + gtid; i < k; i += kRowSelThreads) {
     out_idx[i] = -1;

@@ -102,6 +102,9 @@ SMALL = [
     ("c32_full_own", dict(batch=1, hq=8, hkv=2, d=128, chunk=32, context=300 * 32, topk=24), None, 32),
     ("n0", dict(batch=2, hq=4, hkv=2, d=64, chunk=8, context=40 * 8, topk=4), [0, 40], 2),
     ("big_k", dict(batch=1, hq=4, hkv=1, d=64, chunk=4, context=3000 * 4, topk=700), None, 2),
+    # one scoring CTA per (b, kv head): its thread groups select several rows each in turn
+    ("one_split_many_rows_d64", dict(batch=2, hq=16, hkv=2, d=64, chunk=8, context=60 * 8, topk=8), [60, 41], 3),
+    ("one_split_many_rows_d128", dict(batch=2, hq=28, hkv=4, d=128, chunk=16, context=60 * 16, topk=8), [60, 33], 5),
 ]
 
 
