@@ -82,7 +82,7 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,clocks.mem,clocks.max.mem")
 
     def __init__(self, index):
         self.index = index
@@ -117,16 +117,25 @@ class ClockSampler:
             if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                mem = (float(parts[9]), float(parts[10])) if len(parts) >= 11 else None
+            except ValueError:
+                mem = None
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], mem))
             except ValueError:
                 continue
         os.unlink(self.file.name)
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for _, _, flags, _ in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        out = {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+               "reasons": reasons, "samples": len(rows)}
+        mem = [r[3] for r in rows if r[3] is not None]
+        if mem:  # a memory clock below its maximum caps HBM bandwidth
+            out["mem_mhz"] = statistics.median(m[0] for m in mem)
+            out["mem_max_mhz"] = max(m[1] for m in mem)
+        return out
 
 
 def algorithmic_bytes(cfg, x, sel):
