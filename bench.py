@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--main-only", action="store_true", help="skip the other workloads")
     p.add_argument("--extra-only", action="store_true",
                    help="run only the --extra workloads (no headline line; for profiler captures of one workload)")
-    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep,kvreuse_qwen7b",
+    p.add_argument("--extra", default="qwen7b_16x,qwen7b_16x_excl,hgsa_32x,hgsa2_32x,prefill_32k,prefill_llama1b_32k,llama1b_8x_topp,llama1b_8x_bwd,qwen7b_16x_bwd,llama1b_8x_giststep,kvreuse_qwen7b",
                    help="comma-separated other workloads to measure after the headline one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     p.add_argument("--sweep", action="store_true",

@@ -637,7 +637,7 @@ constexpr int kPfSelectMaxChunks = (227 << 10) / 4 - 128 - kPfTopkMax - (2 * kSe
 
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
-  if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
+  if (d->dtype != GSA_BF16 || (d->d != 64 && d->d != 128)) return GSA_ERR_UNSUPPORTED;
   if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;  // running top-k lists hold at most 16
   // the exact re-selection of listed rows holds one row's gist scores in shared memory
   if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
@@ -646,11 +646,11 @@ gsa_status check_prefill(const gsa_desc *d) {
   return GSA_OK;
 }
 
-// Multi-query scoring runs the prefill scoring kernel: bf16, d = 128,
+// Multi-query scoring runs the prefill scoring kernel: bf16, d = 64 or 128,
 // topk 1..16, one row of gist scores in shared memory for the exact re-pass.
 gsa_status check_multiquery(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
-  if (d->dtype != GSA_BF16 || d->d != 128) return GSA_ERR_UNSUPPORTED;
+  if (d->dtype != GSA_BF16 || (d->d != 64 && d->d != 128)) return GSA_ERR_UNSUPPORTED;
   if (d->topk < 1 || d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;
   if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
@@ -695,12 +695,17 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   }
   const uint64_t bh = static_cast<uint64_t>(d->batch) * d->hq, bkv = static_cast<uint64_t>(d->batch) * d->hkv;
   const uint64_t qgist_rows = pos0 > 0 ? bh * d->t_max : bh * d->n_max;  // (not read when there are no gist rows)
-  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, qgist_rows, kPfRows) ||
-      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kPfKeys))
+  const auto bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t D = static_cast<uint64_t>(d->d);
+  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows, bf16, D) ||
+      !map_rows(&pa.tm_qgist, q_gist, qgist_rows, kPfRows, bf16, D) ||
+      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kPfKeys, bf16, D))
     return GSA_ERR_CUDA;
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
   const int grid = std::min(total, sm_count());
-  GSA_TRY(launch(k_prefill_score<kPfTopkMax>, dim3(grid), dim3(kPsThreads), PfSmem::kBytes, stream, pa));
+  GSA_TRY(d->d == 64 ? launch(k_prefill_score<kPfTopkMax, 64>, dim3(grid), dim3(kPsThreads), PfSmem<64>::kBytes, stream, pa)
+                     : launch(k_prefill_score<kPfTopkMax, 128>, dim3(grid), dim3(kPsThreads), PfSmem<128>::kBytes,
+                              stream, pa));
   if (d->topk <= 0) return GSA_OK;
   // rows whose candidates overflowed: exact per-row selection (usually none)
   SelectRowsArgs sr;
@@ -720,8 +725,9 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.sel_score = sel_score;
   sr.rec_raw = pa.rec_raw;
   sr.scale_log2 = pa.scale_log2;
-  return launch(k_prefill_select_rows, dim3(sm_count()), dim3(kSelThreads),
-                (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4, stream, sr);
+  const size_t sel_smem = (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4;  // scores, query (<= 128), picks
+  return d->d == 64 ? launch(k_prefill_select_rows<64>, dim3(sm_count()), dim3(kSelThreads), sel_smem, stream, sr)
+                    : launch(k_prefill_select_rows<128>, dim3(sm_count()), dim3(kSelThreads), sel_smem, stream, sr);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,
@@ -731,15 +737,20 @@ gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *
   PrefillArgs pa = prefill_args(d, nullptr, nullptr, L, ws);
   const uint64_t bh = static_cast<uint64_t>(d->batch) * d->hq, bkv = static_cast<uint64_t>(d->batch) * d->hkv;
   void *vh = at(ws, L.pf_vh);
-  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows) || !map_rows(&pa.tm_qgist, q_gist, bh * d->n_max, kPfRows) ||
-      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kGaKeys) ||
-      !map_rows(&pa.tm_vgist, vh, bkv * d->n_max, kGaKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+  const auto bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t D = static_cast<uint64_t>(d->d);
+  if (!map_rows(&pa.tm_qraw, q_raw, bh * d->t_max, kPfRows, bf16, D) ||
+      !map_rows(&pa.tm_qgist, q_gist, bh * d->n_max, kPfRows, bf16, D) ||
+      !map_rows(&pa.tm_kgist, k_gist, bkv * d->n_max, kGaKeys, bf16, D) ||
+      !map_rows(&pa.tm_vgist, vh, bkv * d->n_max, kGaKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, D))
     return GSA_ERR_CUDA;
-  const size_t n8 = bkv * d->n_max * 128 / 8;
+  const size_t n8 = bkv * d->n_max * D / 8;
   GSA_TRY(launch(k_bf16_to_f16, dim3(static_cast<unsigned>(std::min<size_t>((n8 + 255) / 256, 4 * sm_count()))),
                  dim3(256), 0, stream, static_cast<const __nv_bfloat16 *>(v_gist), static_cast<__half *>(vh), n8));
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
-  GSA_TRY(launch(k_prefill_gist_attn, dim3(std::min(total, sm_count())), dim3(kPfThreads), GaSmem::kBytes, stream, pa));
+  const dim3 ga_grid(std::min(total, sm_count()));
+  GSA_TRY(d->d == 64 ? launch(k_prefill_gist_attn<64>, ga_grid, dim3(kPfThreads), GaSmem<64>::kBytes, stream, pa)
+                     : launch(k_prefill_gist_attn<128>, ga_grid, dim3(kPfThreads), GaSmem<128>::kBytes, stream, pa));
   GatherArgs ga;
   ga.q_raw = static_cast<const __nv_bfloat16 *>(q_raw);
   ga.k_raw = static_cast<const __nv_bfloat16 *>(k_raw);
@@ -763,8 +774,9 @@ gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *
   ga.out_gist = out_gist;
   ga.out_bf16 = d->out_dtype == GSA_BF16;
   const int64_t rows = static_cast<int64_t>(pa.bh) * (d->t_max + d->n_max);
-  return launch(k_prefill_gather, dim3(static_cast<unsigned>((rows + kGatherWarps - 1) / kGatherWarps)),
-                dim3(kGatherWarps * 32), 0, stream, ga);
+  const dim3 g_grid(static_cast<unsigned>((rows + kGatherWarps - 1) / kGatherWarps));
+  return d->d == 64 ? launch(k_prefill_gather<64>, g_grid, dim3(kGatherWarps * 32), 0, stream, ga)
+                    : launch(k_prefill_gather<128>, g_grid, dim3(kGatherWarps * 32), 0, stream, ga);
 }
 
 // Number of partial records per row the scoring pass writes for these shapes.

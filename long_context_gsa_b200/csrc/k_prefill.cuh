@@ -92,11 +92,14 @@ constexpr int kPsAcc = 3;
 constexpr int kPsXchgCol = kPsAcc * kPfKeys;
 static_assert(kPsXchgCol + 32 <= 512, "TMEM columns");
 
+// D = 64 or 128: a row is D/64 boxes of 64 bf16 (128 bytes, swizzled).
+template <int D>
 struct PfSmem {
+  static_assert(D == 64 || D == 128, "head dim");
   static constexpr uint32_t kQBlock = kPfRows * 128;         // 128 rows x 64 bf16
-  static constexpr uint32_t kQBytes = 2 * kQBlock;           // d = 128
+  static constexpr uint32_t kQBytes = (D / 64) * kQBlock;
   static constexpr uint32_t kKBlock = kPfKeys * 128;
-  static constexpr uint32_t kKBytes = 2 * kKBlock;
+  static constexpr uint32_t kKBytes = (D / 64) * kKBlock;
   static constexpr int kQStages = 1;  // the next tile's Q lands during the row end
   static constexpr int kKStages = 3;
   static constexpr uint32_t kQOff = 0;
@@ -109,7 +112,7 @@ struct PfSmem {
   static constexpr uint32_t kBarOff = kSelOff + 2 * kPfRows;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
 };
-static_assert(PfSmem::kBytes <= 232448, "prefill scoring shared memory");
+static_assert(PfSmem<128>::kBytes <= 232448, "prefill scoring shared memory");
 static_assert(kPsCap >= 8, "a column holds the 16 slot maxima");
 
 constexpr uint32_t kPsSlot = kPfRows * 8;  // bytes between consecutive slots of one row's column
@@ -212,20 +215,21 @@ __device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16])
 // A row whose candidates overflow a half's kPsCap slots, or whose k-th
 // score is shared by a (k+1)-th (the index rule then decides), is listed
 // for k_prefill_select_rows, which recomputes it exactly.
-template <int K>
+template <int K, int D>
 __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
+  using Sm = PfSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PfSmem::kBarOff);
-  constexpr int kQS = PfSmem::kQStages, kKS = PfSmem::kKStages;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::kBarOff);
+  constexpr int kQS = Sm::kQStages, kKS = Sm::kKStages;
   uint64_t *q_full = bars, *q_empty = bars + kQS, *k_full = bars + 2 * kQS, *k_empty = k_full + kKS;
   uint64_t *acc_full = k_empty + kKS, *acc_empty = acc_full + kPsAcc;
   uint64_t *quad_bar = acc_empty + kPsAcc;  // [4]: the two epilogue warps of one TMEM quadrant
   static_assert(2 * kQS + 2 * kKS + 2 * kPsAcc + 4 <= 24, "barrier block");
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(bars + 24);
   int *abort_s = reinterpret_cast<int *>(bars + 25);
-  uint8_t *cnt_x = smem + PfSmem::kCntOff;                               // [2][128]
-  uint8_t *sel_x = smem + PfSmem::kSelOff;                               // [2][128]
+  uint8_t *cnt_x = smem + Sm::kCntOff;                               // [2][128]
+  uint8_t *sel_x = smem + Sm::kSelOff;                               // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.bh * (a.gist_tiles + a.raw_tiles);
@@ -288,12 +292,12 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         if (tl.n_kt == 0) continue;
         const int qs = qi % kQS;
         if (!wait(&q_empty[qs], ((qi / kQS) & 1) ^ 1)) break;
-        uint8_t *qdst = smem + PfSmem::kQOff + qs * PfSmem::kQBytes;
+        uint8_t *qdst = smem + Sm::kQOff + qs * Sm::kQBytes;
         const CUtensorMap *qm = tl.is_gist ? &a.tm_qgist : &a.tm_qraw;
         const int qrow = tl.bh * (tl.is_gist ? a.n_chunks : a.L) + tl.row0;
-        mbar_arrive_expect_tx(&q_full[qs], PfSmem::kQBytes);
-        tc::tma_load_2d(qdst, qm, 0, qrow, &q_full[qs]);
-        tc::tma_load_2d(qdst + PfSmem::kQBlock, qm, 64, qrow, &q_full[qs]);
+        mbar_arrive_expect_tx(&q_full[qs], Sm::kQBytes);
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x) tc::tma_load_2d(qdst + x * Sm::kQBlock, qm, 64 * x, qrow, &q_full[qs]);
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
         for (int jj = 0; jj < n_steps(tl); ++jj, ++ki) {
           const int j = step_tile(tl, jj), ks = ki % kKS;
@@ -301,10 +305,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
             ok = false;
             break;
           }
-          uint8_t *kdst = smem + PfSmem::kKOff + ks * PfSmem::kKBytes;
-          mbar_arrive_expect_tx(&k_full[ks], PfSmem::kKBytes);
-          tc::tma_load_2d(kdst, &a.tm_kgist, 0, krow0 + j * kPfKeys, &k_full[ks]);
-          tc::tma_load_2d(kdst + PfSmem::kKBlock, &a.tm_kgist, 64, krow0 + j * kPfKeys, &k_full[ks]);
+          uint8_t *kdst = smem + Sm::kKOff + ks * Sm::kKBytes;
+          mbar_arrive_expect_tx(&k_full[ks], Sm::kKBytes);
+#pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tc::tma_load_2d(kdst + x * Sm::kKBlock, &a.tm_kgist, 64 * x, krow0 + j * kPfKeys, &k_full[ks]);
         }
         ++qi;
       }
@@ -328,12 +333,12 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
             break;
           }
           tc::fence_after_sync();
-          const uint32_t qa = sbase + PfSmem::kQOff + qs * PfSmem::kQBytes;
-          const uint32_t ka = sbase + PfSmem::kKOff + ks * PfSmem::kKBytes;
+          const uint32_t qa = sbase + Sm::kQOff + qs * Sm::kQBytes;
+          const uint32_t ka = sbase + Sm::kKOff + ks * Sm::kKBytes;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // d = 128 = 8 x 16
-            const uint64_t ad = tc::sw128_desc(qa + (k >> 2) * PfSmem::kQBlock + (k & 3) * 32, 16);
-            const uint64_t bd = tc::sw128_desc(ka + (k >> 2) * PfSmem::kKBlock + (k & 3) * 32, 16);
+          for (int k = 0; k < D / 16; ++k) {  // 16 dims per MMA
+            const uint64_t ad = tc::sw128_desc(qa + (k >> 2) * Sm::kQBlock + (k & 3) * 32, 16);
+            const uint64_t bd = tc::sw128_desc(ka + (k >> 2) * Sm::kKBlock + (k & 3) * 32, 16);
             tc::mma_bf16(tmem + as * kPfKeys, ad, bd, idesc, k > 0);
           }
           tc::commit(&k_empty[ks]);
@@ -349,7 +354,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     const int quad = warp & 3, h = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t cand_u = smem_u32(smem + PfSmem::kCandOff);
+    const uint32_t cand_u = smem_u32(smem + Sm::kCandOff);
     const uint32_t base = cand_u + (h * kPsCap * kPfRows + r) * 8u;          // slot s at base + s * kPsSlot
     const uint32_t pbase = cand_u + ((h ^ 1) * kPsCap * kPfRows + r) * 8u;  // the partner half's column
     const float nan = __int_as_float(0x7fffffff);
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         if (q < ksel) bound = G[q];
       if (!pair_sync()) break;  // the slot maxima area becomes the candidate columns
       const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
-      float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
+      float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (D + kPartHeader);
       if (!sel_rows) {  // pass A saw every key tile: its maximum is the row's
         if (h == 0 && row_ok) rec[0] = mx == neg_inf() ? mx : mx * a.scale_log2;
         continue;
@@ -563,22 +568,25 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
 // the warps' lists, and they are written in ascending chunk order.  The
 // last CTA re-arms the list counter for the next call.
 struct SelectRowsArgs {
-  const __nv_bfloat16 *q_raw, *k_gist;  // [B*hq*L, 128], [B*hkv*N, 128]
+  const __nv_bfloat16 *q_raw, *k_gist;  // [B*hq*L, D], [B*hkv*N, D]
   const int32_t *rows;                  // listed output rows (b*hq + h)*L + pos
   uint32_t *count, *done;               // list length; CTAs finished
   int32_t group, chunk, n_chunks, L, topk, pos0;
   float scale;
   int32_t *sel_idx;
   float *sel_score;
-  float *rec_raw;     // [rows, 128 + 4]: [0] gets the row maximum (base 2)
+  float *rec_raw;     // [rows, D + 4]: [0] gets the row maximum (base 2)
   float scale_log2;
 };
 
 constexpr int kSelThreads = 1024;  // k_prefill_select_rows: a whole block per listed row
 constexpr int kSelWarps = kSelThreads / 32;
 
+template <int D>
 __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const SelectRowsArgs a) {
-  extern __shared__ float sc[];  // [n_chunks] scores, then [128] query
+  constexpr int kLpk = D / 8;      // lanes per key (8 dims each)
+  constexpr int kKpl = 32 / kLpk;  // keys per warp load
+  extern __shared__ float sc[];  // [n_chunks] scores, then [D] query, then the picks' scores
   __shared__ float wl_v[kSelWarps * kPfTopkMax];  // each warp's best ksel (score, index)
   __shared__ int wl_i[kSelWarps * kPfTopkMax];
   __shared__ int picks[32];
@@ -591,35 +599,35 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
     const int bh = orow / a.L, pos = orow % a.L;
     const int limit = min(a.n_chunks, (a.pos0 + pos) / a.chunk);
     const int ksel = min(a.topk, limit);
-    if (tid < 128) qs[tid] = __bfloat162float(a.q_raw[static_cast<size_t>(orow) * 128 + tid]);
+    if (tid < D) qs[tid] = __bfloat162float(a.q_raw[static_cast<size_t>(orow) * D + tid]);
     __syncthreads();
-    // Scores: 16 lanes per key (8 elements each, the query slice in
-    // registers), so a warp reads two whole keys (512 contiguous bytes) per
-    // load; eight such loads are issued before the arithmetic.
-    const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * 128;
+    // Scores: D/8 lanes per key (8 elements each, the query slice in
+    // registers), so a warp reads 32/(D/8) whole keys (512 contiguous
+    // bytes) per load; eight such loads are issued before the arithmetic.
+    const __nv_bfloat16 *kb = a.k_gist + static_cast<size_t>(bh / a.group) * a.n_chunks * D;
     {
-      const int sub = lane & 15, half = lane >> 4;
+      const int sub = lane % kLpk, half = lane / kLpk;
       float qv[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) qv[e] = qs[8 * sub + e];
       constexpr int kU = 8;
-      for (int j0 = 0; j0 * 2 * kSelWarps < limit; j0 += kU) {
+      for (int j0 = 0; j0 * kKpl * kSelWarps < limit; j0 += kU) {
         uint4 w[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-          const int t = ((j0 + u) * kSelWarps + warp) * 2 + half;
-          w[u] = t < limit ? ldg_nc_v4(kb + static_cast<size_t>(t) * 128 + 8 * sub) : make_uint4(0, 0, 0, 0);
+          const int t = ((j0 + u) * kSelWarps + warp) * kKpl + half;
+          w[u] = t < limit ? ldg_nc_v4(kb + static_cast<size_t>(t) * D + 8 * sub) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-          const int t = ((j0 + u) * kSelWarps + warp) * 2 + half;
+          const int t = ((j0 + u) * kSelWarps + warp) * kKpl + half;
           float f[8];
           Vec16<__nv_bfloat16>::unpack(w[u], f);
           float s = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) s = fmaf(qv[e], f[e], s);
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          for (int o = kLpk / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
           if (sub == 0 && t < limit) sc[t] = s;
         }
       }
@@ -709,14 +717,14 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
         if (lane == 0) {
           const bool ok = wi < limit;  // false only for non-finite scores
           picks[it] = ok ? wi : 0x7fffffff;
-          qs[128 + it] = wv;  // pick scores follow the query
+          qs[D + it] = wv;  // pick scores follow the query
         }
       }
     }
     __syncthreads();
     // the first pick is the row maximum
     if (tid == 0)
-      a.rec_raw[static_cast<size_t>(orow) * (128 + kPartHeader)] = ksel > 0 ? qs[128] * a.scale_log2 : neg_inf();
+      a.rec_raw[static_cast<size_t>(orow) * (D + kPartHeader)] = ksel > 0 ? qs[D] * a.scale_log2 : neg_inf();
     // ascending chunk order: a pick's slot is the number of picks below it
     int32_t *oi = a.sel_idx + static_cast<size_t>(orow) * a.topk;
     float *os = a.sel_score + static_cast<size_t>(orow) * a.topk;
@@ -725,7 +733,7 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
       for (int u = 0; u < ksel; ++u) slot += (picks[u] < picks[tid] || (picks[u] == picks[tid] && u < tid)) ? 1 : 0;
       const bool ok = picks[tid] != 0x7fffffff;
       oi[slot] = ok ? picks[tid] : -1;
-      os[slot] = ok ? qs[128 + tid] * a.scale : neg_inf();
+      os[slot] = ok ? qs[D + tid] * a.scale : neg_inf();
     } else if (tid < a.topk) {
       oi[tid] = -1;
       os[tid] = neg_inf();
@@ -757,14 +765,16 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
 // convex combination of the values it weights.
 constexpr int kGaKeys = 128;  // gist keys per tile (S is 128 x 128 in TMEM)
 
+template <int D>
 struct GaSmem {
-  static constexpr uint32_t kBlock = 128 * 128;                 // 128 rows x 64 bf16
-  static constexpr uint32_t kTile = 2 * kBlock;                 // 128 x 128 bf16
+  static constexpr uint32_t kBlock = 128 * 128;                 // 128 rows x 64 16-bit values
+  static constexpr uint32_t kTile = (D / 64) * kBlock;          // 128 rows x D (Q, K or V)
+  static constexpr uint32_t kPTile = 2 * kBlock;                // 128 rows x 128 keys (P)
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kTile;                      // 2 stages
   static constexpr uint32_t kVOff = kKOff + 2 * kTile;          // 2 stages
   static constexpr uint32_t kPOff = kVOff + 2 * kTile;          // 2 buffers
-  static constexpr uint32_t kBarOff = kPOff + 2 * kTile;
+  static constexpr uint32_t kBarOff = kPOff + 2 * kPTile;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1024;
 };
 
@@ -777,10 +787,12 @@ __device__ __forceinline__ PfTile ga_tile(const PrefillArgs &a, int t) {
   return r;
 }
 
+template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __grid_constant__ PrefillArgs a) {
+  using Sm = GaSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + GaSmem::kBarOff);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::kBarOff);
   uint64_t *q_full = bars, *q_empty = bars + 1, *k_full = bars + 2, *k_empty = bars + 4;
   uint64_t *v_full = bars + 6, *v_empty = bars + 8, *s_full = bars + 10, *s_empty = bars + 12;
   uint64_t *p_full = bars + 14, *p_empty = bars + 16, *o_full = bars + 18, *o_empty = bars + 19;
@@ -834,12 +846,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
         const PfTile tl = ga_tile(a, t);
         if (tl.n_kt == 0) continue;
         if (!wait(q_empty, (qi & 1) ^ 1)) break;
-        uint8_t *qdst = smem + GaSmem::kQOff;
+        uint8_t *qdst = smem + Sm::kQOff;
         const CUtensorMap *qm = tl.is_gist ? &a.tm_qgist : &a.tm_qraw;
         const int qrow = tl.bh * (tl.is_gist ? a.n_chunks : a.L) + tl.row0;
-        mbar_arrive_expect_tx(q_full, GaSmem::kTile);
-        tc::tma_load_2d(qdst, qm, 0, qrow, q_full);
-        tc::tma_load_2d(qdst + GaSmem::kBlock, qm, 64, qrow, q_full);
+        mbar_arrive_expect_tx(q_full, Sm::kTile);
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x) tc::tma_load_2d(qdst + x * Sm::kBlock, qm, 64 * x, qrow, q_full);
         const int krow0 = (tl.bh / a.group) * a.n_chunks;
         for (int j = 0; j < tl.n_kt; ++j, ++ki) {
           const int s = ki & 1;
@@ -848,14 +860,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
             ok = false;
             break;
           }
-          uint8_t *kdst = smem + GaSmem::kKOff + s * GaSmem::kTile;
-          uint8_t *vdst = smem + GaSmem::kVOff + s * GaSmem::kTile;
-          mbar_arrive_expect_tx(&k_full[s], GaSmem::kTile);
-          tc::tma_load_2d(kdst, &a.tm_kgist, 0, krow0 + j * kGaKeys, &k_full[s]);
-          tc::tma_load_2d(kdst + GaSmem::kBlock, &a.tm_kgist, 64, krow0 + j * kGaKeys, &k_full[s]);
-          mbar_arrive_expect_tx(&v_full[s], GaSmem::kTile);
-          tc::tma_load_2d(vdst, &a.tm_vgist, 0, krow0 + j * kGaKeys, &v_full[s]);
-          tc::tma_load_2d(vdst + GaSmem::kBlock, &a.tm_vgist, 64, krow0 + j * kGaKeys, &v_full[s]);
+          uint8_t *kdst = smem + Sm::kKOff + s * Sm::kTile;
+          uint8_t *vdst = smem + Sm::kVOff + s * Sm::kTile;
+          mbar_arrive_expect_tx(&k_full[s], Sm::kTile);
+#pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tc::tma_load_2d(kdst + x * Sm::kBlock, &a.tm_kgist, 64 * x, krow0 + j * kGaKeys, &k_full[s]);
+          mbar_arrive_expect_tx(&v_full[s], Sm::kTile);
+#pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tc::tma_load_2d(vdst + x * Sm::kBlock, &a.tm_vgist, 64 * x, krow0 + j * kGaKeys, &v_full[s]);
         }
         ++qi;
       }
@@ -863,7 +877,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16(kPfRows, kGaKeys, false, false);
-      constexpr uint32_t idesc_o = tc::idesc_f16kind(kPfRows, 128, false, true, false);  // fp16; B = V, MN-major
+      constexpr uint32_t idesc_o = tc::idesc_f16kind(kPfRows, D, false, true, false);  // fp16; B = V, MN-major
       const uint32_t sbase = smem_u32(smem);
       uint32_t qi = 0, ki = 0, si = 0, pi = 0, oi = 0;
       bool ok = true;
@@ -872,11 +886,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
         const int s = ki & 1, sb = si & 1;
         if (!wait(&k_full[s], (ki >> 1) & 1) || !wait(&s_empty[sb], ((si >> 1) & 1) ^ 1)) return false;
         tc::fence_after_sync();
-        const uint32_t qa = sbase + GaSmem::kQOff, ka = sbase + GaSmem::kKOff + s * GaSmem::kTile;
+        const uint32_t qa = sbase + Sm::kQOff, ka = sbase + Sm::kKOff + s * Sm::kTile;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t ad = tc::sw128_desc(qa + (k >> 2) * GaSmem::kBlock + (k & 3) * 32, 16);
-          const uint64_t bd = tc::sw128_desc(ka + (k >> 2) * GaSmem::kBlock + (k & 3) * 32, 16);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = tc::sw128_desc(qa + (k >> 2) * Sm::kBlock + (k & 3) * 32, 16);
+          const uint64_t bd = tc::sw128_desc(ka + (k >> 2) * Sm::kBlock + (k & 3) * 32, 16);
           tc::mma_bf16(tmem + sb * kGaKeys, ad, bd, idesc_s, k > 0);
         }
         tc::commit(&k_empty[s]);
@@ -890,11 +904,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
         const int s = vi & 1, pb = pi & 1;
         if (!wait(&v_full[s], (vi >> 1) & 1) || !wait(&p_full[pb], (pi >> 1) & 1)) return false;
         tc::fence_after_sync();
-        const uint32_t pa = sbase + GaSmem::kPOff + pb * GaSmem::kTile, va = sbase + GaSmem::kVOff + s * GaSmem::kTile;
+        const uint32_t pa = sbase + Sm::kPOff + pb * Sm::kPTile, va = sbase + Sm::kVOff + s * Sm::kTile;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // 128 keys = 8 x 16
-          const uint64_t ad = tc::sw128_desc(pa + (k >> 2) * GaSmem::kBlock + (k & 3) * 32, 16);
-          const uint64_t bd = tc::sw128_desc(va + k * 16 * 128, GaSmem::kBlock);
+          const uint64_t ad = tc::sw128_desc(pa + (k >> 2) * Sm::kBlock + (k & 3) * 32, 16);
+          const uint64_t bd = tc::sw128_desc(va + k * 16 * 128, Sm::kBlock);
           tc::mma_bf16(tmem + 2 * kGaKeys, ad, bd, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
         }
         tc::commit(&v_empty[s]);
@@ -932,7 +946,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
       const bool row_ok = row < (tl.is_gist ? a.n_chunks : a.L);
       const int limit = !row_ok ? 0 : (tl.is_gist ? min(a.n_chunks, row + 1) : min(a.n_chunks, row / a.chunk));
       const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + (row_ok ? row : 0);
-      float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (128 + kPartHeader);
+      float *rec = (tl.is_gist ? a.rec_gist : a.rec_raw) + orow * (D + kPartHeader);
       const float ref = (row_ok && limit > 0) ? rec[0] : 0.f;
       float l = 0.f;
       bool ok = true;
@@ -967,11 +981,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
           break;
         }
         // P row r into the swizzled K-major tile: block kb holds keys 64*kb..
-        uint8_t *pbase = smem + GaSmem::kPOff + pb * GaSmem::kTile;
+        uint8_t *pbase = smem + Sm::kPOff + pb * Sm::kPTile;
 #pragma unroll
         for (int u = 0; u < 16; ++u) {  // 16-byte units along the 128 keys
           const int kb = u >> 3, uu = u & 7;
-          uint8_t *dst = pbase + kb * GaSmem::kBlock + (prow >> 3) * 1024 + (prow & 7) * 128 + ((uu ^ (prow & 7)) * 16);
+          uint8_t *dst = pbase + kb * Sm::kBlock + (prow >> 3) * 1024 + (prow & 7) * 128 + ((uu ^ (prow & 7)) * 16);
           *reinterpret_cast<uint4 *>(dst) =
               make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
         }
@@ -983,7 +997,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
       if (!wait(o_full, oi & 1)) break;
       tc::fence_after_sync();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         float v[32];
         __syncwarp();
         tc::ld32(tmem + lane_addr + 2 * kGaKeys + c * 32, v);
@@ -1014,7 +1028,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
 // stages do not cover -- the selected chunks (with their gist in exclude
 // mode) and the own-chunk prefix for raw rows, chunk m's raw tokens for gist
 // row m -- merged with the row's gist partial.  One warp per row; a group of
-// 16 lanes owns one key row (8 dims per lane), two rows per step.
+// D/8 lanes owns one key row (8 dims per lane), 32/(D/8) rows per step.
 struct GatherArgs {
   const __nv_bfloat16 *q_raw, *k_raw, *v_raw, *q_gist, *v_gist;
   const int32_t *sel_idx;
@@ -1028,8 +1042,9 @@ struct GatherArgs {
 
 constexpr int kGatherWarps = 8;
 
+template <int D>
 __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const GatherArgs a) {
-  constexpr int D = 128, kE = 8, kLpr = 16;
+  constexpr int kE = 8, kLpr = D / kE, kSlots = 32 / kLpr;  // lanes per key row, rows per step
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rows_raw = static_cast<int64_t>(a.bh) * a.L;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kGatherWarps + warp;
@@ -1065,18 +1080,18 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
   };
   // attend raw rows [first, first + n) of this kv head, 4 rows per lane group in flight
   auto span = [&](int first, int n) {
-    for (int r0 = 0; r0 < n; r0 += 8) {
+    for (int r0 = 0; r0 < n; r0 += 4 * kSlots) {
       uint4 kw[4], vw[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int r = r0 + 2 * u + slot;
+        const int r = r0 + kSlots * u + slot;
         const size_t off = (kv0 + first + min(r, n - 1)) * D + dd;
         kw[u] = ldg_nc_v4(a.k_raw + off);
         vw[u] = ldg_nc_v4(a.v_raw + off);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int r = r0 + 2 * u + slot;
+        const int r = r0 + kSlots * u + slot;
         float kf[kE], part = 0.f;
         Vec16<__nv_bfloat16>::unpack(kw[u], kf);
 #pragma unroll
@@ -1108,12 +1123,13 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
     }
     span(mc * a.chunk, pos - mc * a.chunk + 1);
   }
-  // merge the two row slots, then the gist partial of the row
-  {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, kLpr), l2 = __shfl_xor_sync(0xffffffffu, l, kLpr);
+  // merge the row slots, then the gist partial of the row
+#pragma unroll
+  for (int o = kLpr; o < 32; o <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
     float acc2[kE];
 #pragma unroll
-    for (int e = 0; e < kE; ++e) acc2[e] = __shfl_xor_sync(0xffffffffu, acc[e], kLpr);
+    for (int e = 0; e < kE; ++e) acc2[e] = __shfl_xor_sync(0xffffffffu, acc[e], o);
     merge_state<kE>(m, l, acc, m2, l2, acc2);
   }
   const bool has_prior = is_gist || !a.exclude;

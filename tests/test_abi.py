@@ -148,7 +148,8 @@ def test_new_entry_points_reject_bad_arguments(lib):
     assert lib.gsa_gist_step(C.byref(d), A, A, A, A, A, A, A, A, A, A, None, A, 256, None) == 3
     # multi-query: unsupported head size / k, missing output, small workspace
     mq = _desc(topk=16, t_max=300)
-    assert lib.gsa_multiquery_select(C.byref(_desc(d=64, topk=16)), A, A, A, A, A, 1 << 40, None) == 2
+    assert lib.gsa_multiquery_select(C.byref(_desc(d=96, topk=16)), A, A, A, A, A, 1 << 40, None) == 2
+    assert lib.gsa_multiquery_select(C.byref(_desc(dtype=0, topk=16)), A, A, A, A, A, 1 << 40, None) == 2  # fp32
     assert lib.gsa_multiquery_select(C.byref(_desc(topk=20)), A, A, A, A, A, 1 << 40, None) == 2
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, None, A, A, 1 << 40, None) == 1
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, A, A, A, 1024, None) == 3

@@ -70,20 +70,22 @@ def compare(q, gk, k, rows=None, exact_ties=False, what=""):
 
 
 CASES = [
-    # name, B, hq, hkv, Q, N, k
-    ("one_head_ragged", 1, 1, 1, 100, 300, 16),
-    ("gqa4_tiles", 2, 8, 2, 256, 1000, 16),
-    ("gqa7_ragged_keys", 1, 28, 4, 200, 128 * 5 + 3, 8),
-    ("k_above_n", 1, 4, 2, 130, 5, 16),
-    ("k1", 1, 4, 4, 64, 700, 1),
+    # name, B, hq, hkv, Q, N, k, d
+    ("one_head_ragged", 1, 1, 1, 100, 300, 16, 128),
+    ("gqa4_tiles", 2, 8, 2, 256, 1000, 16, 128),
+    ("gqa7_ragged_keys", 1, 28, 4, 200, 128 * 5 + 3, 8, 128),
+    ("k_above_n", 1, 4, 2, 130, 5, 16, 128),
+    ("k1", 1, 4, 4, 64, 700, 1, 128),
+    ("d64_gqa4_ragged", 2, 8, 2, 200, 128 * 7 + 5, 16, 64),
+    ("d64_k3", 1, 4, 1, 130, 300, 3, 64),
 ]
 
 
-@pytest.mark.parametrize("name,B,hq,hkv,Q,N,k", CASES, ids=[c[0] for c in CASES])
-def test_random(name, B, hq, hkv, Q, N, k):
+@pytest.mark.parametrize("name,B,hq,hkv,Q,N,k,d", CASES, ids=[c[0] for c in CASES])
+def test_random(name, B, hq, hkv, Q, N, k, d):
     gen = torch.Generator(device="cuda").manual_seed(zlib.crc32(name.encode()))
-    q = torch.randn((B, hq, Q, 128), generator=gen, device="cuda").to(torch.bfloat16)
-    gk = torch.randn((B, hkv, N, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    q = torch.randn((B, hq, Q, d), generator=gen, device="cuda").to(torch.bfloat16)
+    gk = torch.randn((B, hkv, N, d), generator=gen, device="cuda").to(torch.bfloat16)
     compare(q, gk, k, what=name)
 
 

@@ -108,6 +108,10 @@ SMALL = [
     ("ragged_tile_n37", dict(batch=2, hq=2, hkv=1, chunk=16, n_chunks=37, topk=5)),
     ("k16_n520_c4", dict(batch=1, hq=4, hkv=1, chunk=4, n_chunks=520, topk=16)),
     ("k1_n200_c8", dict(batch=1, hq=2, hkv=2, chunk=8, n_chunks=200, topk=1)),
+    # d = 64 (the Llama-3.2-1B head size)
+    ("d64_n300_c8_k16", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, n_chunks=300, topk=16)),
+    ("d64_ragged_n37", dict(batch=2, hq=4, hkv=1, d=64, chunk=16, n_chunks=37, topk=5)),
+    ("d64_k1_n150_c4", dict(batch=1, hq=4, hkv=4, d=64, chunk=4, n_chunks=150, topk=1)),
 ]
 
 
@@ -217,6 +221,20 @@ def test_full_size_every_row_exclude():
     print("prefill_32k exclude, 4 heads:", res)
 
 
+def test_full_size_llama_heads():
+    """The Llama-3.2-1B-shaped 32K prefill (32/8 heads, d = 64, 4096 chunks
+    of 8, top-16): every row of four whole heads (two kv heads, first and
+    last query head of each) against the oracle in default mode, and two
+    heads in exclude mode."""
+    cfg = W.PREFILL_LLAMA_32K
+    x = W.prefill_inputs(cfg, device="cuda")
+    res = check_heads(x, cfg, False, (0, 3, 28, 31), what="prefill_llama1b_32k")
+    assert res["rows"] == 4 * (cfg.length + cfg.n_chunks)
+    print("prefill_llama1b_32k default, 4 heads:", res)
+    res = check_heads(x, cfg, True, (5, 18), what="prefill_llama1b_32k exclude")
+    print("prefill_llama1b_32k exclude, 2 heads:", res)
+
+
 @pytest.mark.parametrize("exclude", [False, True], ids=["default", "exclude"])
 def test_exact_ties_through_prefill(exclude):
     """Gist keys repeated in runs of three (chunks 3j, 3j+1, 3j+2 share one
@@ -232,3 +250,15 @@ def test_exact_ties_through_prefill(exclude):
     res = check_heads(x, cfg, exclude, range(cfg.batch * cfg.hq), what="prefill ties", exact_ties=True)
     assert res["exact_tie_rows"] > cfg.hq * 100, res  # the boundary really sits inside a run in most rows
     print("prefill exact ties:", res)
+
+
+def test_exact_ties_through_prefill_d64():
+    """The tie case of test_exact_ties_through_prefill at d = 64."""
+    cfg = W.scaled(W.PREFILL_LLAMA_32K, seed=zlib.crc32(b"prefill_ties_d64"), batch=1, hq=4, hkv=2, chunk=8,
+                   n_chunks=200, topk=8)
+    x = W.prefill_inputs(cfg, device="cuda")
+    src = torch.arange(cfg.n_chunks, device="cuda") // 3 * 3
+    x["k_gist"] = x["k_gist"][:, :, src].contiguous()
+    res = check_heads(x, cfg, False, range(cfg.batch * cfg.hq), what="prefill ties d64", exact_ties=True)
+    assert res["exact_tie_rows"] > cfg.hq * 100, res
+    print("prefill exact ties d64:", res)
