@@ -374,9 +374,9 @@ gsa_status hgsa2_decode(const gsa_desc *desc, const gsa_h2desc *h2desc, const vo
  * selection among them) and its own chunk's raw tokens m*chunk .. i.  Gist
  * position m sees its chunk's raw tokens and gists 0..m (compression mask).
  *
- * Both stages are built for bf16 inputs with d = 64 or 128, topk <= 16
- * and n_max <= 56912 chunks (GSA_ERR_UNSUPPORTED otherwise), and need
- * t_max = n_max * chunk.
+ * Both stages are built for bf16 inputs with d = 64 or 128, topk <= 64
+ * and n_max <= 56912 chunks (53760 when topk > 16; GSA_ERR_UNSUPPORTED
+ * otherwise), and need t_max = n_max * chunk.
  *
  * Stage 1, scoring + selection (tensor cores).  Every raw row is scored
  * against the gists it can see and keeps the top k; every row (raw and
@@ -395,7 +395,8 @@ gsa_status gsa_prefill_score(const gsa_desc *desc, const void *q_raw, const void
  * the tensor cores (the prefill scoring kernel with the queries placed
  * after the cache) and keeps the top k.
  *   desc: batch = documents; t_max = Q, the queries per (document, query
- *         head); bf16, d = 64 or 128, topk 1..16, n_max <= 56912
+ *         head); bf16, d = 64 or 128, topk 1..64, n_max <= 56912
+ *         (53760 when topk > 16)
  *         (GSA_ERR_UNSUPPORTED otherwise); chunk is ignored.
  *   q       [B, hq, Q, d]; query head h reads kv head h / (hq / hkv)
  *   gist_k  [B, hkv, N, d]

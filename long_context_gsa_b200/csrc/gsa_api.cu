@@ -633,26 +633,34 @@ gsa_status run_hgsa2_select(const gsa_desc *d, const gsa_h2desc *h2, const void 
 constexpr int kPfOvfCountWord = 16, kPfOvfDoneWord = 17;
 // the exact per-row pass holds a row's scores, the query and its picks in
 // dynamic shared memory next to the warps' pick lists (static)
-constexpr int kPfSelectMaxChunks = (227 << 10) / 4 - 128 - kPfTopkMax - (2 * kSelWarps * kPfTopkMax + 32);
+// (k <= K): the static lists are 2 x kSelWarps x K words plus K picks.
+constexpr int pf_select_max_chunks(int K) { return (227 << 10) / 4 - 128 - K - (2 * kSelWarps * K + (K > 32 ? K : 32)); }
+constexpr int kPfSelectMaxChunks = pf_select_max_chunks(kPfTopkMax);        // 56912
+constexpr int kPfSelectMaxChunksWide = pf_select_max_chunks(kPfTopkWide);   // 53760
+static_assert(kPfSelectMaxChunks == 56912 && kPfSelectMaxChunksWide == 53760, "documented limits");
+
+// The scorer variant a selection of k entries runs on.
+inline bool pf_wide(const gsa_desc *d) { return d->topk > kPfTopkMax; }
+inline int pf_max_chunks(const gsa_desc *d) { return pf_wide(d) ? kPfSelectMaxChunksWide : kPfSelectMaxChunks; }
 
 gsa_status check_prefill(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || (d->d != 64 && d->d != 128)) return GSA_ERR_UNSUPPORTED;
-  if (d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;  // running top-k lists hold at most 16
+  if (d->topk > kPfTopkWide) return GSA_ERR_UNSUPPORTED;  // the wide scorer's lists hold at most 64
   // the exact re-selection of listed rows holds one row's gist scores in shared memory
-  if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
+  if (d->n_max > pf_max_chunks(d)) return GSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->n_max) * d->chunk != d->t_max) return GSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
   return GSA_OK;
 }
 
 // Multi-query scoring runs the prefill scoring kernel: bf16, d = 64 or 128,
-// topk 1..16, one row of gist scores in shared memory for the exact re-pass.
+// topk 1..64, one row of gist scores in shared memory for the exact re-pass.
 gsa_status check_multiquery(const gsa_desc *d) {
   GSA_TRY(check_desc(d));
   if (d->dtype != GSA_BF16 || (d->d != 64 && d->d != 128)) return GSA_ERR_UNSUPPORTED;
-  if (d->topk < 1 || d->topk > kPfTopkMax) return GSA_ERR_UNSUPPORTED;
-  if (d->n_max > kPfSelectMaxChunks) return GSA_ERR_UNSUPPORTED;
+  if (d->topk < 1 || d->topk > kPfTopkWide) return GSA_ERR_UNSUPPORTED;
+  if (d->n_max > pf_max_chunks(d)) return GSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->batch) * d->hq * d->t_max >= (int64_t(1) << 31)) return GSA_ERR_UNSUPPORTED;
   return GSA_OK;
 }
@@ -703,9 +711,14 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
     return GSA_ERR_CUDA;
   const int total = pa.bh * (pa.gist_tiles + pa.raw_tiles);
   const int grid = std::min(total, sm_count());
-  GSA_TRY(d->d == 64 ? launch(k_prefill_score<kPfTopkMax, 64>, dim3(grid), dim3(kPsThreads), PfSmem<64>::kBytes, stream, pa)
-                     : launch(k_prefill_score<kPfTopkMax, 128>, dim3(grid), dim3(kPsThreads), PfSmem<128>::kBytes,
-                              stream, pa));
+  const dim3 ps_grid(grid), ps_block(kPsThreads);
+  constexpr int kN = kPfTopkMax, kW = kPfTopkWide;
+  if (!pf_wide(d))
+    GSA_TRY(d->d == 64 ? launch(k_prefill_score<kN, 64>, ps_grid, ps_block, PfSmem<64, kN>::kBytes, stream, pa)
+                       : launch(k_prefill_score<kN, 128>, ps_grid, ps_block, PfSmem<128, kN>::kBytes, stream, pa));
+  else
+    GSA_TRY(d->d == 64 ? launch(k_prefill_score<kW, 64>, ps_grid, ps_block, PfSmem<64, kW>::kBytes, stream, pa)
+                       : launch(k_prefill_score<kW, 128>, ps_grid, ps_block, PfSmem<128, kW>::kBytes, stream, pa));
   if (d->topk <= 0) return GSA_OK;
   // rows whose candidates overflowed: exact per-row selection (usually none)
   SelectRowsArgs sr;
@@ -725,9 +738,14 @@ gsa_status run_prefill_score(const gsa_desc *d, const void *q_raw, const void *q
   sr.sel_score = sel_score;
   sr.rec_raw = pa.rec_raw;
   sr.scale_log2 = pa.scale_log2;
-  const size_t sel_smem = (static_cast<size_t>(d->n_max) + 128 + kPfTopkMax) * 4;  // scores, query (<= 128), picks
-  return d->d == 64 ? launch(k_prefill_select_rows<64>, dim3(sm_count()), dim3(kSelThreads), sel_smem, stream, sr)
-                    : launch(k_prefill_select_rows<128>, dim3(sm_count()), dim3(kSelThreads), sel_smem, stream, sr);
+  const int kmax = pf_wide(d) ? kW : kN;
+  const size_t sel_smem = (static_cast<size_t>(d->n_max) + 128 + kmax) * 4;  // scores, query (<= 128), pick scores
+  const dim3 sr_grid(sm_count()), sr_block(kSelThreads);
+  if (!pf_wide(d))
+    return d->d == 64 ? launch(k_prefill_select_rows<64, kN>, sr_grid, sr_block, sel_smem, stream, sr)
+                      : launch(k_prefill_select_rows<128, kN>, sr_grid, sr_block, sel_smem, stream, sr);
+  return d->d == 64 ? launch(k_prefill_select_rows<64, kW>, sr_grid, sr_block, sel_smem, stream, sr)
+                    : launch(k_prefill_select_rows<128, kW>, sr_grid, sr_block, sel_smem, stream, sr);
 }
 
 gsa_status run_prefill_attend(const gsa_desc *d, const void *q_raw, const void *k_raw, const void *v_raw,

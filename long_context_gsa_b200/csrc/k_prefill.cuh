@@ -50,7 +50,8 @@ struct PrefillArgs {
 constexpr int kPfRows = 128;        // query rows per tile (TMEM lanes)
 constexpr int kPfKeys = 128;        // gist keys per MMA tile (TMEM columns)
 constexpr int kPfThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kPfTopkMax = 16;
+constexpr int kPfTopkMax = 16;   // the narrow scorer: k <= 16
+constexpr int kPfTopkWide = 64;  // the wide scorer: 16 < k <= 64
 
 struct PfTile {
   int is_gist, bh, row0, n_kt;
@@ -85,35 +86,41 @@ __device__ __forceinline__ PfTile pf_tile(const PrefillArgs &a, int t) {
 // spread over both halves); two threads share a query row.
 constexpr int kPsEpiWarps = 8;
 constexpr int kPsThreads = 64 + 32 * kPsEpiWarps;
-constexpr int kPsCap = 48;  // candidate slots per row half
 // TMEM columns: kPsAcc accumulators of 128 (the MMA runs that many key
-// tiles ahead of the epilogue), then the row-end exchange (2 x 16)
+// tiles ahead of the epilogue), then the row-end exchange (2 x the sorted
+// list length: 16 for the narrow scorer, 64 for the wide one)
 constexpr int kPsAcc = 3;
 constexpr int kPsXchgCol = kPsAcc * kPfKeys;
-static_assert(kPsXchgCol + 32 <= 512, "TMEM columns");
+static_assert(kPsXchgCol + 2 * 64 <= 512, "TMEM columns");
 
-// D = 64 or 128: a row is D/64 boxes of 64 bf16 (128 bytes, swizzled).
-template <int D>
+// Scoring-stage shared memory.  D = 64 or 128: a row is D/64 boxes of 64
+// bf16 (128 bytes, swizzled).  K = the largest k the variant selects: the
+// narrow scorer (K = 16) keeps 48 candidate slots per row half, the wide
+// one (K = 64) 64, and with d = 128 it gives up a key stage to fit them.
+template <int D, int K>
 struct PfSmem {
   static_assert(D == 64 || D == 128, "head dim");
+  static_assert(K == kPfTopkMax || K == kPfTopkWide, "scorer variant");
+  static constexpr int kCap = K > 16 ? 64 : 48;  // candidate slots per row half
   static constexpr uint32_t kQBlock = kPfRows * 128;         // 128 rows x 64 bf16
   static constexpr uint32_t kQBytes = (D / 64) * kQBlock;
   static constexpr uint32_t kKBlock = kPfKeys * 128;
   static constexpr uint32_t kKBytes = (D / 64) * kKBlock;
   static constexpr int kQStages = 1;  // the next tile's Q lands during the row end
-  static constexpr int kKStages = 3;
+  static constexpr int kKStages = (K > 16 && D == 128) ? 2 : 3;
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kQStages * kQBytes;
-  // [2 halves][kPsCap][128 rows] (score, index); pass A first uses a row
-  // half's first 8 slots for its 16 sorted slot maxima
+  // [2 halves][kCap][128 rows] (score, index); pass A first uses a row
+  // half's first slots for its sorted slot maxima (two per slot)
   static constexpr uint32_t kCandOff = kKOff + kKStages * kKBytes;
-  static constexpr uint32_t kCntOff = kCandOff + 2 * kPsCap * kPfRows * 8;  // [2][128] candidate counts (bytes)
-  static constexpr uint32_t kSelOff = kCntOff + 2 * kPfRows;                 // [2][128] selected counts (bytes)
+  static constexpr uint32_t kCntOff = kCandOff + 2 * kCap * kPfRows * 8;  // [2][128] candidate counts (bytes)
+  static constexpr uint32_t kSelOff = kCntOff + 2 * kPfRows;               // [2][128] selected counts (bytes)
   static constexpr uint32_t kBarOff = kSelOff + 2 * kPfRows;
   static constexpr uint32_t kBytes = kBarOff + 256 + 1008;   // + alignment slack (base is 16-byte aligned)
+  static_assert(kBytes <= 232448, "prefill scoring shared memory");
+  static_assert(2 * kCap >= (K > 16 ? 64 : 16), "a column holds the half's sorted slot maxima");
+  static_assert(kCap <= 255, "counts are bytes");
 };
-static_assert(PfSmem<128>::kBytes <= 232448, "prefill scoring shared memory");
-static_assert(kPsCap >= 8, "a column holds the 16 slot maxima");
 
 constexpr uint32_t kPsSlot = kPfRows * 8;  // bytes between consecutive slots of one row's column
 
@@ -128,9 +135,10 @@ __device__ __forceinline__ void sts_u2(uint32_t a, uint2 v) {
 }
 
 // Append (v, idx) to a row half's column when v >= bound: the store and
-// the count are predicated (no branch); past kPsCap the last slot is
+// the count are predicated (no branch); past CAP the last slot is
 // overwritten and only the count grows, which the row end reports as an
 // overflow.  NaN (a masked score) fails the compare.
+template <int CAP>
 __device__ __forceinline__ void ps_append(uint32_t base, uint32_t &cnt, float v, float bound, uint32_t idx) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t.reg .u32 s, ad;\n\t"
@@ -140,7 +148,7 @@ __device__ __forceinline__ void ps_append(uint32_t base, uint32_t &cnt, float v,
       "@p st.shared.v2.u32 [ad], {%4, %7};\n\t"
       "@p add.u32 %0, %0, 1;\n\t}\n"
       : "+r"(cnt)
-      : "f"(v), "f"(bound), "r"(base), "r"(__float_as_uint(v)), "r"(kPsCap - 1), "r"(kPsSlot), "r"(idx)
+      : "f"(v), "f"(bound), "r"(base), "r"(__float_as_uint(v)), "r"(CAP - 1), "r"(kPsSlot), "r"(idx)
       : "memory");
 }
 
@@ -150,14 +158,16 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
   return v;
 }
 
-// Descending bitonic sort of 16 values in registers (no NaN inputs).
-__device__ __forceinline__ void ps_sort16(float (&w)[16]) {
+// Descending bitonic sort of N (a power of two) values in registers (no
+// NaN inputs).
+template <int N>
+__device__ __forceinline__ void ps_sort(float (&w)[N]) {
 #pragma unroll
-  for (int k = 2; k <= 16; k <<= 1)
+  for (int k = 2; k <= N; k <<= 1)
 #pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < N; ++i) {
         const int l = i ^ j;
         if (l > i) {
           const float x = w[i], y = w[l];
@@ -168,25 +178,16 @@ __device__ __forceinline__ void ps_sort16(float (&w)[16]) {
       }
 }
 
-// Values-only insertion into a descending list of 16.
-__device__ __forceinline__ void ps_insert16(float (&b)[16], float x) {
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const float hi = fmaxf(b[q], x);
-    x = fminf(b[q], x);
-    b[q] = hi;
-  }
-}
-
-// a <- the 16 largest of a (sorted descending) and b (sorted descending):
+// a <- the N largest of a (sorted descending) and b (sorted descending):
 // the elementwise max against b reversed is bitonic; half-cleaners sort it.
-__device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16]) {
+template <int N>
+__device__ __forceinline__ void ps_merge(float (&a)[N], const float (&b)[N]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) a[i] = fmaxf(a[i], b[15 - i]);
+  for (int i = 0; i < N; ++i) a[i] = fmaxf(a[i], b[N - 1 - i]);
 #pragma unroll
-  for (int j = 8; j > 0; j >>= 1)
+  for (int j = N / 2; j > 0; j >>= 1)
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < N; ++i)
       if ((i & j) == 0) {
         const float x = a[i], y = a[i + j];
         a[i] = fmaxf(x, y);
@@ -194,30 +195,36 @@ __device__ __forceinline__ void ps_merge16(float (&a)[16], const float (&b)[16])
       }
 }
 
-// Stage 1, k_prefill_score: row maxima and the top-k selection (k <= 16)
-// of every query row, in two passes over the visible key tiles of a query
-// tile (the key tiles stream through a 3-stage ring; Q stays in shared
-// memory):
-//  A. over every other key tile (0, 2, 4, ...), each thread keeps 16 slot
-//     maxima over its half of the columns (slot = column mod 16); the 16
-//     largest of the row's 32 slot maxima are distinct scores, so the k-th
-//     largest of them bounds the row's k-th score from below (sampling half
-//     the tiles loosens the bound, doubling the candidates, and halves the
-//     pass's tensor work);
+// Stage 1, k_prefill_score: row maxima and the top-k selection of every
+// query row, in two passes over the visible key tiles of a query tile (the
+// key tiles stream through a ring; Q stays in shared memory).  K = 16 (the
+// narrow scorer, k <= 16) or 64 (the wide one, 16 < k <= 64); S = 16 or 64
+// slots per row half:
+//  A. each thread keeps S slot maxima over its half of the columns (slot =
+//     column mod S); the largest of the row's 2S slot maxima are distinct
+//     scores, so the k-th largest of them bounds the row's k-th score from
+//     below.  The narrow scorer samples every other key tile (0, 2, 4, ...;
+//     the bound stays valid, only looser, and the pass's tensor work
+//     halves); the wide one takes every tile, which keeps the bound tight
+//     at k = 64;
 //  B. over all key tiles, every score >= that bound is appended as a
-//     (score, index) candidate (about 2k + 10 per row) by predicated
-//     stores, in ascending index order; the largest candidate is the row
-//     maximum;
-//     at the row end each half sorts its 16 largest candidate values, the
+//     (score, index) candidate (about 2k + 10 per row for the narrow
+//     scorer, 1.4k for the wide one) by predicated stores, in ascending
+//     index order; the largest candidate is the row maximum;
+//     at the row end each half sorts its S largest candidate values, the
 //     halves exchange them through TMEM and merge them into the row's k-th
 //     candidate score T, keep (compact) their entries >= T, and write the
-//     two ascending lists merged by index, eight output slots per half.
-// A row whose candidates overflow a half's kPsCap slots, or whose k-th
-// score is shared by a (k+1)-th (the index rule then decides), is listed
-// for k_prefill_select_rows, which recomputes it exactly.
+//     two ascending lists merged by index, K/2 output slots per half.
+// A row whose candidates overflow a half's slots, or whose k-th score is
+// shared by a (k+1)-th (the index rule then decides), is listed for
+// k_prefill_select_rows, which recomputes it exactly.
 template <int K, int D>
 __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_constant__ PrefillArgs a) {
-  using Sm = PfSmem<D>;
+  using Sm = PfSmem<D, K>;
+  constexpr bool kWide = K > 16;
+  constexpr int kSl = kWide ? 64 : 16;  // slot maxima (and sorted candidate values) per row half
+  constexpr int kCap = Sm::kCap;
+  constexpr int kHalfOut = K / 2;       // output slots written by each half
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::kBarOff);
@@ -269,17 +276,19 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     flag_error(a.status, GSA_DEVERR_TIMEOUT);
     return false;
   };
-  // key-tile passes of a query tile: raw rows with a selection take two
   // Key tiles of a query tile, in MMA order.  Rows with a selection take
-  // pass A over every other key tile (0, 2, 4, ...; the bound it gives
-  // stays exact, only looser) and then pass B over all of them; other rows
-  // take pass A over all key tiles (their exact row maximum).
-  auto n_pass_a = [&](const PfTile &tl) { return (!tl.is_gist && raw_topk) ? (tl.n_kt + 1) / 2 : tl.n_kt; };
+  // pass A (the narrow scorer: over every other key tile, 0, 2, 4, ...; the
+  // bound it gives stays exact, only looser) and then pass B over all of
+  // them; other rows take pass A over all key tiles (their exact row
+  // maximum).
+  auto n_pass_a = [&](const PfTile &tl) {
+    return (!tl.is_gist && raw_topk && !kWide) ? (tl.n_kt + 1) / 2 : tl.n_kt;
+  };
   auto n_steps = [&](const PfTile &tl) { return n_pass_a(tl) + ((!tl.is_gist && raw_topk) ? tl.n_kt : 0); };
   auto step_tile = [&](const PfTile &tl, int jj) {
-    const bool sel = !tl.is_gist && raw_topk;
+    const bool sampled = !tl.is_gist && raw_topk && !kWide;
     const int na = n_pass_a(tl);
-    return jj < na ? (sel ? 2 * jj : jj) : jj - na;
+    return jj < na ? (sampled ? 2 * jj : jj) : jj - na;
   };
 
   if (warp == 0) {
@@ -355,8 +364,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t cand_u = smem_u32(smem + Sm::kCandOff);
-    const uint32_t base = cand_u + (h * kPsCap * kPfRows + r) * 8u;          // slot s at base + s * kPsSlot
-    const uint32_t pbase = cand_u + ((h ^ 1) * kPsCap * kPfRows + r) * 8u;  // the partner half's column
+    const uint32_t base = cand_u + (h * kCap * kPfRows + r) * 8u;          // slot s at base + s * kPsSlot
+    const uint32_t pbase = cand_u + ((h ^ 1) * kCap * kPfRows + r) * 8u;  // the partner half's column
     const float nan = __int_as_float(0x7fffffff);
     uint32_t ai = 0, pair_phase = 0;
     auto pair_sync = [&]() -> bool {
@@ -395,37 +404,37 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       const bool sel_rows = !tl.is_gist && raw_topk;
       const int ksel = min(a.topk, limit);  // entries this row selects
       // ---- pass A: slot maxima ----
-      float G[16];
+      float G[kSl];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) G[q] = neg_inf();
+      for (int q = 0; q < kSl; ++q) G[q] = neg_inf();
       for (int jj = 0; jj < n_pass_a(tl) && ok; ++jj)
         ok = take(step_tile(tl, jj), limit, [&](const float(&v)[64], int) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) G[e & 15] = fmaxf(G[e & 15], v[e]);
+          for (int e = 0; e < 64; ++e) G[e & (kSl - 1)] = fmaxf(G[e & (kSl - 1)], v[e]);
         });
       if (!ok) break;
-      ps_sort16(G);
+      ps_sort<kSl>(G);
       // the sorted slot maxima go to this row half's own candidate column
       // (two per slot); rows of other quadrants, which run ahead or behind,
       // never touch them
 #pragma unroll
-      for (int q = 0; q < 16; q += 2)
+      for (int q = 0; q < kSl; q += 2)
         sts_u2(base + (q >> 1) * kPsSlot, make_uint2(__float_as_uint(G[q]), __float_as_uint(G[q + 1])));
       if (!pair_sync()) break;
       {
-        float o[16];
+        float o[kSl];
 #pragma unroll
-        for (int q = 0; q < 16; q += 2) {
+        for (int q = 0; q < kSl; q += 2) {
           const uint2 w = lds_u2(pbase + (q >> 1) * kPsSlot);
           o[q] = __uint_as_float(w.x);
           o[q + 1] = __uint_as_float(w.y);
         }
-        ps_merge16(G, o);  // top 16 of the row's 32 slot maxima
+        ps_merge<kSl>(G, o);  // top kSl of the row's 2 kSl slot maxima
       }
       const float mx = G[0];
       float bound = G[0];
 #pragma unroll
-      for (int q = 1; q < 16; ++q)
+      for (int q = 1; q < kSl; ++q)
         if (q < ksel) bound = G[q];
       if (!pair_sync()) break;  // the slot maxima area becomes the candidate columns
       const size_t orow = static_cast<size_t>(tl.bh) * (tl.is_gist ? a.n_chunks : a.L) + row;
@@ -439,41 +448,44 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       for (int j = 0; j < tl.n_kt && ok; ++j)
         ok = take(j, limit, [&](const float(&v)[64], int tb) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) ps_append(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
+          for (int e = 0; e < 64; ++e)
+            ps_append<kCap>(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
         });
       if (!ok) break;
-      bool ovf = cnt > static_cast<uint32_t>(kPsCap);  // the row goes to the exact per-row pass
-      const int mine = min(static_cast<int>(cnt), kPsCap);
+      bool ovf = cnt > static_cast<uint32_t>(kCap);  // the row goes to the exact per-row pass
+      const int mine = min(static_cast<int>(cnt), kCap);
       cnt_x[h * kPfRows + r] = static_cast<uint8_t>(ovf ? 255 : mine);
-      // The row's k-th candidate score T: each half's 16 largest (values
-      // only, sorted 16 at a time) meet through TMEM columns 256.. (lane =
-      // row) and are merged by both.
-      float top[16];
+      // The row's k-th candidate score T: each half's kSl largest (values
+      // only, sorted kSl at a time) meet through the TMEM exchange columns
+      // (lane = row) and are merged by both.
+      float top[kSl];
       {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) top[q] = q < mine ? __uint_as_float(lds_u32(base + q * kPsSlot)) : neg_inf();
-        ps_sort16(top);
-        for (int s0 = 16; s0 < mine; s0 += 16) {
-          float x[16];
+        for (int q = 0; q < kSl; ++q) top[q] = q < mine ? __uint_as_float(lds_u32(base + q * kPsSlot)) : neg_inf();
+        ps_sort<kSl>(top);
+        for (int s0 = kSl; s0 < mine; s0 += kSl) {
+          float x[kSl];
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
+          for (int q = 0; q < kSl; ++q)
             x[q] = s0 + q < mine ? __uint_as_float(lds_u32(base + (s0 + q) * kPsSlot)) : neg_inf();
-          ps_sort16(x);
-          ps_merge16(top, x);
+          ps_sort<kSl>(x);
+          ps_merge<kSl>(top, x);
         }
       }
-      tc::st16(tmem + lane_addr + kPsXchgCol + 16 * h, top);
+#pragma unroll
+      for (int c = 0; c < kSl / 16; ++c) tc::st16(tmem + lane_addr + kPsXchgCol + kSl * h + 16 * c, top + 16 * c);
       tc::fence_before_sync();
       if (!pair_sync()) break;
       tc::fence_after_sync();
       {
-        float o[16];
-        tc::ld16(tmem + lane_addr + kPsXchgCol + 16 * (h ^ 1), o);
-        ps_merge16(top, o);
+        float o[kSl];
+#pragma unroll
+        for (int c = 0; c < kSl / 16; ++c) tc::ld16(tmem + lane_addr + kPsXchgCol + kSl * (h ^ 1) + 16 * c, o + 16 * c);
+        ps_merge<kSl>(top, o);
       }
       float T = top[0];
 #pragma unroll
-      for (int q = 1; q < 16; ++q)
+      for (int q = 1; q < kSl; ++q)
         if (q < ksel) T = top[q];
       // the row maximum: the largest candidate (every score at or above the
       // bound is one); a listed row gets it from the exact per-row pass
@@ -484,7 +496,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
       for (int s0 = 0; s0 < mine; s0 += 8) {
         uint2 x[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = lds_u2(base + min(s0 + k, kPsCap - 1) * kPsSlot);
+        for (int k = 0; k < 8; ++k) x[k] = lds_u2(base + min(s0 + k, kCap - 1) * kPsSlot);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           if (s0 + k < mine && __uint_as_float(x[k].x) >= T) {
@@ -507,18 +519,19 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
           }
         } else {
           // the merged selection in ascending chunk index order; this half
-          // writes output slots 8h .. 8h+7 (both lists are ascending)
+          // writes output slots (K/2) h .. (K/2) h + K/2 - 1 (both lists are
+          // ascending)
           int ia = 0, ib = 0;
-          for (int q = 0; q < 8 * h; ++q) {
+          for (int q = 0; q < kHalfOut * h; ++q) {
             const uint32_t xa = ia < n_own ? lds_u32(base + ia * kPsSlot + 4) : 0xffffffffu;
             const uint32_t xb = ib < n_their ? lds_u32(pbase + ib * kPsSlot + 4) : 0xffffffffu;
             if (xa < xb) ++ia;
             else ++ib;
           }
-          int32_t oid[8];
-          float osc[8];
+          int32_t oid[kHalfOut];
+          float osc[kHalfOut];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < kHalfOut; ++q) {
             const uint2 xa = ia < n_own ? lds_u2(base + ia * kPsSlot) : make_uint2(0u, 0xffffffffu);
             const uint2 xb = ib < n_their ? lds_u2(pbase + ib * kPsSlot) : make_uint2(0u, 0xffffffffu);
             const bool ta = xa.y < xb.y;
@@ -529,17 +542,18 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
             oid[q] = valid ? static_cast<int32_t>(x.y) : -1;
             osc[q] = valid ? __uint_as_float(x.x) * a.scale : neg_inf();
           }
-          int32_t *oi = a.sel_idx + orow * a.topk + 8 * h;
-          float *os = a.sel_score + orow * a.topk + 8 * h;
-          if (a.topk == 16) {
-            reinterpret_cast<int4 *>(oi)[0] = make_int4(oid[0], oid[1], oid[2], oid[3]);
-            reinterpret_cast<int4 *>(oi)[1] = make_int4(oid[4], oid[5], oid[6], oid[7]);
-            reinterpret_cast<float4 *>(os)[0] = make_float4(osc[0], osc[1], osc[2], osc[3]);
-            reinterpret_cast<float4 *>(os)[1] = make_float4(osc[4], osc[5], osc[6], osc[7]);
+          int32_t *oi = a.sel_idx + orow * a.topk + kHalfOut * h;
+          float *os = a.sel_score + orow * a.topk + kHalfOut * h;
+          if (a.topk == K) {  // rows of K entries: 16-byte aligned stores
+#pragma unroll
+            for (int q = 0; q < kHalfOut; q += 4) {
+              reinterpret_cast<int4 *>(oi)[q / 4] = make_int4(oid[q], oid[q + 1], oid[q + 2], oid[q + 3]);
+              reinterpret_cast<float4 *>(os)[q / 4] = make_float4(osc[q], osc[q + 1], osc[q + 2], osc[q + 3]);
+            }
           } else {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (8 * h + q < a.topk) {
+            for (int q = 0; q < kHalfOut; ++q)
+              if (kHalfOut * h + q < a.topk) {
                 oi[q] = oid[q];
                 os[q] = osc[q];
               }
@@ -582,14 +596,14 @@ struct SelectRowsArgs {
 constexpr int kSelThreads = 1024;  // k_prefill_select_rows: a whole block per listed row
 constexpr int kSelWarps = kSelThreads / 32;
 
-template <int D>
+template <int D, int K>
 __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const SelectRowsArgs a) {
   constexpr int kLpk = D / 8;      // lanes per key (8 dims each)
   constexpr int kKpl = 32 / kLpk;  // keys per warp load
   extern __shared__ float sc[];  // [n_chunks] scores, then [D] query, then the picks' scores
-  __shared__ float wl_v[kSelWarps * kPfTopkMax];  // each warp's best ksel (score, index)
-  __shared__ int wl_i[kSelWarps * kPfTopkMax];
-  __shared__ int picks[32];
+  __shared__ float wl_v[kSelWarps * K];  // each warp's best ksel (score, index), best first
+  __shared__ int wl_i[kSelWarps * K];
+  __shared__ int picks[K];
   pdl_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t n = *reinterpret_cast<volatile uint32_t *>(a.count);
@@ -636,8 +650,9 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
     // Top ksel by (score desc, index asc), in two levels of argmax rounds
     // that stay inside a warp: warp w takes keys w*32 + lane + kSelThreads j
     // (each lane keeps its best untaken key and rescans after losing it)
-    // and lists its ksel best; warp 0 then picks the row's ksel from the
-    // warps' lists.  Equal scores keep the lower index at every step.
+    // and lists its ksel best in order; warp 0 then merges the 32 ordered
+    // lists (lane l holds the head of warp l's list) into the row's ksel.
+    // Equal scores keep the lower index at every step.
     auto better = [](float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); };
     auto lane_best = [&](float &bv, int &bi) {
       bv = neg_inf();
@@ -667,8 +682,8 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
           }
         }
         if (lane == 0) {
-          wl_v[warp * kPfTopkMax + it] = wv;
-          wl_i[warp * kPfTopkMax + it] = wi;
+          wl_v[warp * K + it] = wv;
+          wl_i[warp * K + it] = wi;
         }
         if (wi == bi && wi != 0x7fffffff) {  // this lane's key was taken: its next best
           sc[bi] = neg_inf();
@@ -679,26 +694,13 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
     }
     __syncthreads();
     if (warp == 0) {
-      // lane l holds list entries l, l + 32, ... of the kSelWarps x 16 slots
-      constexpr int kPer = kSelWarps * kPfTopkMax / 32;
-      float cv[kPer];
-      int ci[kPer];
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int e = lane + 32 * u, it = e % kPfTopkMax;
-        const bool in = it < ksel;
-        cv[u] = in ? wl_v[e] : neg_inf();
-        ci[u] = in ? wl_i[e] : 0x7fffffff;
-      }
+      static_assert(kSelWarps == 32, "one list per lane");
+      int p = 0;  // this lane's position in warp `lane`'s list
       for (int it = 0; it < ksel; ++it) {
-        float wv = cv[0];
-        int wi = ci[0];
-#pragma unroll
-        for (int u = 1; u < kPer; ++u)
-          if (better(cv[u], ci[u], wv, wi)) {
-            wv = cv[u];
-            wi = ci[u];
-          }
+        const float hv = p < ksel ? wl_v[lane * K + p] : neg_inf();
+        const int hi = p < ksel ? wl_i[lane * K + p] : 0x7fffffff;
+        float wv = hv;
+        int wi = hi;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
@@ -708,12 +710,7 @@ __global__ void __launch_bounds__(kSelThreads) k_prefill_select_rows(const Selec
             wi = oi;
           }
         }
-#pragma unroll
-        for (int u = 0; u < kPer; ++u)
-          if (ci[u] == wi) {  // taken (indices are distinct)
-            cv[u] = neg_inf();
-            ci[u] = 0x7fffffff;
-          }
+        if (p < ksel && hi == wi && hv == wv) ++p;  // this list's head was taken (indices are distinct)
         if (lane == 0) {
           const bool ok = wi < limit;  // false only for non-finite scores
           picks[it] = ok ? wi : 0x7fffffff;

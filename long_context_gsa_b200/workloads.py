@@ -113,8 +113,9 @@ HGSA2_32X = DecodeConfig("hgsa2_32x", 2, 32, 8, 128, 32, 524288, 64, "bf16", gro
                          topk_meta2=8, seed=20260006)
 PREFILL_32K = PrefillConfig("prefill_32k", 1, 28, 4, 128, 16, 2048, 16, "bf16", seed=20260005)
 # The same causal prefill with the Llama-3.2-1B head layout (32 query / 8 kv
-# heads, d = 64) at 8x compression: 4096 chunks of 8 over 32K tokens, top-16.
-PREFILL_LLAMA_32K = PrefillConfig("prefill_llama1b_32k", 1, 32, 8, 64, 8, 4096, 16, "bf16", seed=20260008)
+# heads, d = 64) at 8x compression, with the decode workload's top-64: 4096
+# chunks of 8 over 32K tokens.
+PREFILL_LLAMA_32K = PrefillConfig("prefill_llama1b_32k", 1, 32, 8, 64, 8, 4096, 64, "bf16", seed=20260008)
 # KV reuse: a 128K-token document compressed 16x (8192 gists) shared by 4096
 # query rows per head (Qwen2-7B head layout), top-16 routing per query.
 KVREUSE_QWEN = MultiQueryConfig("kvreuse_qwen7b", 1, 28, 4, 128, 8192, 4096, 16, seed=20260007)

@@ -121,7 +121,7 @@ def test_workspace_bytes_new_ops(lib):
     mq = _desc(topk=16, t_max=300)
     assert gsa_workspace_bytes(mq, GSA_OP_MULTIQUERY) > 2 * 8 * 300 * 4
     assert gsa_workspace_bytes(_desc(topk=16, dtype=0), GSA_OP_MULTIQUERY) == 0  # fp32 inputs: not built
-    assert gsa_workspace_bytes(_desc(topk=17), GSA_OP_MULTIQUERY) == 0
+    assert gsa_workspace_bytes(_desc(topk=65), GSA_OP_MULTIQUERY) == 0
     assert gsa_workspace_bytes(_desc(topk=0), GSA_OP_MULTIQUERY) == 0
     assert gsa_workspace_bytes(d, 99) == 0
     assert gsa_workspace_bytes(d, GSA_OP_DECODE) > 0
@@ -150,7 +150,7 @@ def test_new_entry_points_reject_bad_arguments(lib):
     mq = _desc(topk=16, t_max=300)
     assert lib.gsa_multiquery_select(C.byref(_desc(d=96, topk=16)), A, A, A, A, A, 1 << 40, None) == 2
     assert lib.gsa_multiquery_select(C.byref(_desc(dtype=0, topk=16)), A, A, A, A, A, 1 << 40, None) == 2  # fp32
-    assert lib.gsa_multiquery_select(C.byref(_desc(topk=20)), A, A, A, A, A, 1 << 40, None) == 2
+    assert lib.gsa_multiquery_select(C.byref(_desc(topk=65)), A, A, A, A, A, 1 << 40, None) == 2
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, None, A, A, 1 << 40, None) == 1
     assert lib.gsa_multiquery_select(C.byref(mq), A, A, A, A, A, 1024, None) == 3
 

@@ -78,6 +78,8 @@ CASES = [
     ("k1", 1, 4, 4, 64, 700, 1, 128),
     ("d64_gqa4_ragged", 2, 8, 2, 200, 128 * 7 + 5, 16, 64),
     ("d64_k3", 1, 4, 1, 130, 300, 3, 64),
+    ("d64_k64_wide", 1, 8, 2, 200, 1000, 64, 64),
+    ("d128_k40_wide", 1, 4, 2, 150, 128 * 5 + 7, 40, 128),
 ]
 
 

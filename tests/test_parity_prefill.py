@@ -112,6 +112,11 @@ SMALL = [
     ("d64_n300_c8_k16", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, n_chunks=300, topk=16)),
     ("d64_ragged_n37", dict(batch=2, hq=4, hkv=1, d=64, chunk=16, n_chunks=37, topk=5)),
     ("d64_k1_n150_c4", dict(batch=1, hq=4, hkv=4, d=64, chunk=4, n_chunks=150, topk=1)),
+    # k > 16 (the wide scorer)
+    ("k64_n300_c8_d64", dict(batch=1, hq=8, hkv=2, d=64, chunk=8, n_chunks=300, topk=64)),
+    ("k32_n200_c16_d128", dict(batch=1, hq=4, hkv=2, d=128, chunk=16, n_chunks=200, topk=32)),
+    ("k17_ragged_n45_d64", dict(batch=2, hq=2, hkv=1, d=64, chunk=16, n_chunks=45, topk=17)),
+    ("k64_n140_c4_d128", dict(batch=1, hq=4, hkv=1, d=128, chunk=4, n_chunks=140, topk=64)),
 ]
 
 
@@ -223,7 +228,7 @@ def test_full_size_every_row_exclude():
 
 def test_full_size_llama_heads():
     """The Llama-3.2-1B-shaped 32K prefill (32/8 heads, d = 64, 4096 chunks
-    of 8, top-16): every row of four whole heads (two kv heads, first and
+    of 8, top-64): every row of four whole heads (two kv heads, first and
     last query head of each) against the oracle in default mode, and two
     heads in exclude mode."""
     cfg = W.PREFILL_LLAMA_32K
@@ -252,10 +257,12 @@ def test_exact_ties_through_prefill(exclude):
     print("prefill exact ties:", res)
 
 
-def test_exact_ties_through_prefill_d64():
-    """The tie case of test_exact_ties_through_prefill at d = 64."""
+@pytest.mark.parametrize("topk", [8, 40], ids=["k8", "k40"])
+def test_exact_ties_through_prefill_d64(topk):
+    """The tie case of test_exact_ties_through_prefill at d = 64, with the
+    narrow (k <= 16) and the wide scorer."""
     cfg = W.scaled(W.PREFILL_LLAMA_32K, seed=zlib.crc32(b"prefill_ties_d64"), batch=1, hq=4, hkv=2, chunk=8,
-                   n_chunks=200, topk=8)
+                   n_chunks=200, topk=topk)
     x = W.prefill_inputs(cfg, device="cuda")
     src = torch.arange(cfg.n_chunks, device="cuda") // 3 * 3
     x["k_gist"] = x["k_gist"][:, :, src].contiguous()
