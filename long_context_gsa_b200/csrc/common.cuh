@@ -57,6 +57,32 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
   return v;
 }
 
+// Release store of a flag another CTA acquires (gpu scope).
+__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// The ready list of the fused decode step: the scoring kernel's tail
+// publishes each selected row (row + 1, in completion order) and the unfold
+// CTAs take them in that order.  Words [rows .. rows + 2] are the
+// publisher's slot counter, the unfold's ticket counter and its done
+// counter; the unfold's last CTA clears the whole list.
+struct ReadyList {
+  uint32_t *w;  // [rows + 4] or null
+  int32_t rows;
+};
+
+__device__ __forceinline__ void flag_error(uint32_t *status, uint32_t bits);
+
+// Publish `row` (its outputs written and fenced by every writer).
+__device__ __forceinline__ void ready_publish(const ReadyList &r, int row, uint32_t *status) {
+  const uint32_t pos = atomicAdd(&r.w[r.rows], 1u);
+  if (pos < static_cast<uint32_t>(r.rows))
+    st_release_u32(&r.w[pos], static_cast<uint32_t>(row) + 1u);
+  else
+    flag_error(status, GSA_DEVERR_CAPACITY);  // a list left over from a failed call
+}
+
 __device__ __forceinline__ void flag_error(uint32_t *status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }

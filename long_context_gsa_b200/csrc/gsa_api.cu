@@ -41,7 +41,7 @@ inline float resolve_scale(const gsa_desc *d) {
 
 struct Layout {
   size_t status = 0, counters = 0, scores = 0, sel_idx = 0, sel_score = 0, part_g = 0, part_u = 0;
-  size_t unit_counters = 0;
+  size_t unit_counters = 0, ready = 0;
   size_t meta_scores = 0, meta_idx = 0, cand_scores = 0, cand_ids = 0, cand_count = 0, part_h = 0;
   size_t meta2_scores = 0, meta2_idx = 0, cand1_scores = 0, cand1_ids = 0, cand1_count = 0;
   size_t pf_stats = 0, pf_gist = 0, pf_vh = 0, pf_ovf = 0;
@@ -127,7 +127,8 @@ Layout layout(const gsa_desc *d, int32_t op, const gsa_hdesc *h) {
     L.total = off;
     return L;
   }
-  take(L.unit_counters, rows * 8);  // with the status and counters: the prefix a scratch-free call clears
+  take(L.unit_counters, rows * 8);
+  take(L.ready, (rows + 4) * 4);  // with the status and counters: the prefix a scratch-free call clears
   take(L.scores, rows * d->n_max * 4);
   take(L.sel_idx, rows * d->topk * 4);
   take(L.sel_score, rows * d->topk * 4);
@@ -318,7 +319,8 @@ gsa_status launch_score_generic_t(const ScoreArgs &sa, int splits, int B, int dt
 gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const void *vals, const int32_t *n_gists,
                      int count_div, int rows_cap, float *scores, int score_stride, float *part, int *splits_out,
                      uint32_t *status, void *stream, uint32_t *zero_rows = nullptr,
-                     uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr, float *sel_score = nullptr) {
+                     uint32_t *unit_counters = nullptr, int32_t *sel_idx = nullptr, float *sel_score = nullptr,
+                     uint32_t *ready = nullptr) {
   const int group = d->hq / d->hkv;
   const bool with_v = part != nullptr;
   const ScorePlan plan = plan_score(d, rows_cap, with_v);
@@ -343,6 +345,8 @@ gsa_status run_score(const gsa_desc *d, const void *q, const void *keys, const v
   sa.topk = d->topk;
   sa.sel_idx = sel_idx;
   sa.sel_score = sel_score;
+  sa.ready.w = sa.unit_counters ? ready : nullptr;
+  sa.ready.rows = d->batch * d->hq;
   sa.status = status;
   sa.hq = d->hq;
   sa.hkv = d->hkv;
@@ -416,6 +420,7 @@ gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
       return GSA_ERR_CUDA;
     return launch(k_unfold_tc<D>, dim3(ua.n_split, ua.hq, B), dim3(kUnfoldThreads), smem, stream, ua);
   }
+  ua.ready.w = nullptr;  // the CUDA-core kernel always follows the whole previous kernel
   const size_t smem = unfold_smem<D, T>(ua.chunk);
   const int slots = resident_ctas(k_unfold<D, T>, kUnfoldThreads, smem);
   ua.n_split = one_wave_splits(B * ua.hq, slots, std::min(kUnfoldSplitMax, std::max(1, ua.k)));
@@ -425,7 +430,7 @@ gsa_status launch_unfold_t(UnfoldArgs ua, int B, void *stream) {
 gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const void *raw_v, const void *gist_v,
                       const int32_t *n_gists, const int32_t *own_len, const int32_t *sel_idx, const float *sel_score,
                       const float *prior, int n_prior, void *out, float *lse, const Layout &L, void *ws,
-                      void *stream) {
+                      void *stream, uint32_t *ready = nullptr) {
   UnfoldArgs ua;
   ua.q = q;
   ua.raw_k = raw_k;
@@ -449,6 +454,8 @@ gsa_status run_unfold(const gsa_desc *d, const void *q, const void *raw_k, const
   ua.prior = prior;
   ua.n_prior = prior ? n_prior : 0;
   ua.counters = reinterpret_cast<uint32_t *>(at(ws, L.counters));
+  ua.ready.w = ready;
+  ua.ready.rows = d->batch * d->hq;
   ua.status = reinterpret_cast<uint32_t *>(at(ws, L.status));
   ua.out = out;
   ua.out_bf16 = d->out_dtype == GSA_BF16;
@@ -1009,12 +1016,14 @@ gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, c
   int n_prior = 0;
   if (tail_select_ok(desc)) {
     // Two launches: scoring with the selection in its tail (it also re-arms
-    // the unfold's counters), then the unfold.
+    // the unfold's counters), then the unfold, whose CTAs take the rows as
+    // the tail publishes them in the ready list.
+    uint32_t *ready = reinterpret_cast<uint32_t *>(at(ws, L.ready));
     GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
                       stream, reinterpret_cast<uint32_t *>(at(ws, L.counters)),
-                      reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss));
+                      reinterpret_cast<uint32_t *>(at(ws, L.unit_counters)), si, ss, ready));
     return run_unfold(desc, q, raw_k, raw_v, gist_v, n_gists, own_len, si, ss, part, part ? n_prior : 0, out, lse, L,
-                      ws, stream);
+                      ws, stream, ready);
   }
   GSA_TRY(run_score(desc, q, gist_k, gist_v, n_gists, 1, desc->n_max, scores, desc->n_max, part, &n_prior, status,
                     stream));
@@ -1418,7 +1427,7 @@ extern "C" gsa_status gsa_decode_noalloc(const gsa_desc *desc, const void *q, co
   GSA_TRY(noalloc_scratch(&ws));
   // The status word and the per-row and per-group counters must start at
   // zero; the array keeps whatever the previous call (of any shape) left.
-  const size_t zero_bytes = L.unit_counters + static_cast<size_t>(desc->batch) * desc->hq * 8;
+  const size_t zero_bytes = L.ready + (static_cast<size_t>(desc->batch) * desc->hq + 4) * 4;
   if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GSA_ERR_CUDA;
   return gsa_decode(desc, q, gist_k, gist_v, raw_k, raw_v, n_gists, own_len, out, lse, sel_idx, sel_score, ws,
                     GSA_NOALLOC_SCRATCH_BYTES, stream);

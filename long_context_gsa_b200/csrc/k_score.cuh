@@ -43,6 +43,7 @@ struct ScoreArgs {
   int32_t topk;
   int32_t *sel_idx;       // [B*hq, topk]
   float *sel_score;       // [B*hq, topk] or null
+  ReadyList ready;        // w null, or each selected row is published there for the unfold
   uint32_t *status;
   int32_t hq, hkv, group;
   int32_t head_split;     // CTAs per kv head along the query heads
@@ -96,6 +97,10 @@ struct ScoreMmaCfg {
 __device__ __forceinline__ int score_tail_selectors(int n_split, int nh, int groups) {
   return min(n_split, (nh + groups - 1) / groups);
 }
+
+// The rows (query heads j of the group) selector si of S selects: head j
+// goes to selector (j / groups) mod S, thread group j mod groups.
+__device__ __forceinline__ bool score_tail_mine(int j, int si, int S, int groups) { return (j / groups) % S == si; }
 
 // A selector CTA is done: the last one re-arms the group's two counters.
 __device__ __forceinline__ void score_tail_done(uint32_t *cnt, int selectors) {
@@ -347,8 +352,13 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
       }
       if (a.unit_counters) {  // arrive; a selector that cannot select still counts as done
         const int S = score_tail_selectors(gridDim.x, nh, Cfg::kSelGroups);
-        if (static_cast<int>(atomicAdd(&a.unit_counters[2 * unit], 1u)) >= static_cast<int>(gridDim.x) - S)
+        const int si = static_cast<int>(atomicAdd(&a.unit_counters[2 * unit], 1u)) - (static_cast<int>(gridDim.x) - S);
+        if (si >= 0) {
+          if (a.ready.w)  // its rows are published unselected, so the unfold does not wait for them
+            for (int j = 0; j < nh; ++j)
+              if (score_tail_mine(j, si, S, Cfg::kSelGroups)) ready_publish(a.ready, b * a.hq + h0 + j, a.status);
           score_tail_done(a.unit_counters + 2 * unit, S);
+        }
       }
     }
     __syncthreads();
@@ -436,8 +446,8 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
         ok_s = ok;
       }
       __syncthreads();
+      const int grp = tid / kRowSelThreads;
       if (ok_s) {
-        const int grp = tid / kRowSelThreads;
         SelSmem<Cfg::kSelMaxN> &ssm = reinterpret_cast<SelSmem<Cfg::kSelMaxN> *>(smem)[grp];
         int use = 0;
         for (int j = si * Cfg::kSelGroups + grp; j < nh; j += S * Cfg::kSelGroups) {
@@ -445,7 +455,16 @@ __global__ void __launch_bounds__(ScoreMmaCfg<D, GH, WITH_V>::kThreads, 2)
           group_select<Cfg::kSelMaxN>(a.scores + row * a.score_stride, N, a.topk, tid % kRowSelThreads, ssm, 1 + grp,
                                       use, a.status, a.sel_idx + row * a.topk,
                                       a.sel_score ? a.sel_score + row * a.topk : nullptr);
+          if (a.ready.w) {
+            // every writer fences, then the group meets; one thread publishes
+            __threadfence();
+            group_bar(1 + grp);
+            if (tid % kRowSelThreads == 0) ready_publish(a.ready, static_cast<int>(row), a.status);
+          }
         }
+      } else if (a.ready.w && tid % kRowSelThreads == 0) {
+        for (int j = si * Cfg::kSelGroups + grp; j < nh; j += S * Cfg::kSelGroups)
+          ready_publish(a.ready, b * a.hq + h0 + j, a.status);  // unselected (TIMEOUT is flagged)
       }
       __syncthreads();
       if (tid == 0) score_tail_done(cnt2, S);

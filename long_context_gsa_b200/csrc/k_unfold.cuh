@@ -40,6 +40,7 @@ struct UnfoldArgs {
   const float *prior;        // [B*hq, n_prior, D+4] or null
   int32_t n_prior;
   uint32_t *counters;        // [B*hq]
+  ReadyList ready;           // w null: CTA (split, h, b) after the previous kernel; else rows as published
   uint32_t *status;
   void *out;                 // [B*hq, D]
   int32_t out_bf16;
@@ -365,6 +366,49 @@ struct UnfoldTcCfg {
   }
 };
 
+// With a ready list (the fused decode step), CTA t takes ticket t in
+// arrival order: row = the (t / n_split)-th row published, split = t mod
+// n_split.  It waits (bounded) for that row's publication instead of the
+// whole scoring grid, so rows whose selection is done unfold while others
+// are still being selected.  The last CTA to finish clears the list.
+__device__ __forceinline__ int unfold_take_row(const UnfoldArgs &a, int &split) {
+  const uint32_t t = atomicAdd(&a.ready.w[a.ready.rows + 1], 1u);
+  const uint32_t pos = t / static_cast<uint32_t>(a.n_split);
+  split = static_cast<int>(t % static_cast<uint32_t>(a.n_split));
+  if (pos >= static_cast<uint32_t>(a.ready.rows)) {
+    flag_error(a.status, GSA_DEVERR_CAPACITY);
+    return -1;
+  }
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    const uint32_t v = ld_acquire_u32(&a.ready.w[pos]);
+    if (v != 0u) return v <= static_cast<uint32_t>(a.ready.rows) ? static_cast<int>(v) - 1 : -1;
+    if ((it & 15u) == 0) {
+      const uint64_t now = global_timer_ns();
+      if (!t0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) {
+        flag_error(a.status, GSA_DEVERR_TIMEOUT);
+        return -1;
+      }
+    }
+    __nanosleep(64);
+  }
+}
+
+__device__ __forceinline__ void unfold_ready_done(const UnfoldArgs &a) {
+  __shared__ int last_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t total = gridDim.x * gridDim.y * gridDim.z;
+    last_s = atomicAdd(&a.ready.w[a.ready.rows + 2], 1u) == total - 1;
+  }
+  __syncthreads();
+  if (last_s) {  // every CTA has read its entry: clear the list for the next step
+    for (int i = threadIdx.x; i < a.ready.rows + 4; i += blockDim.x) a.ready.w[i] = 0u;
+    __threadfence();
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_constant__ UnfoldArgs a) {
   using Cfg = UnfoldTcCfg<D>;
@@ -376,18 +420,38 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
   int *item_pos = items + per;
   __shared__ int n_items_s;
   __shared__ int is_last_s;
+  __shared__ int take_s[2];
   __shared__ float red[kUnfoldWarps][2 + D];
   __shared__ uint64_t bars[kUnfoldWarps][4];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  int split, h, b;
+  if (a.ready.w) {
+    if (tid == 0) {
+      int sp = 0;
+      take_s[0] = unfold_take_row(a, sp);
+      take_s[1] = sp;
+    }
+    __syncthreads();
+    if (take_s[0] < 0) {  // flagged: nothing to attend
+      unfold_ready_done(a);
+      return;
+    }
+    split = take_s[1];
+    h = take_s[0] % a.hq;
+    b = take_s[0] / a.hq;
+  } else {
+    pdl_wait();
+    split = blockIdx.x;
+    h = blockIdx.y;
+    b = blockIdx.z;
+  }
   const int kvh = h / a.group;
   const size_t row = static_cast<size_t>(b) * a.hq + h;
   const int g = lane >> 2, t4 = lane & 3;
 
-  pdl_wait();
-  const int N = min(min(max(a.n_gists[b], 0), a.n_max), a.t_max / a.chunk);
-  int own = min(max(a.own_len[b], 0), a.chunk);
+  const int N = min(min(max(__ldcg(a.n_gists + b), 0), a.n_max), a.t_max / a.chunk);
+  int own = min(max(__ldcg(a.own_len + b), 0), a.chunk);
   if (static_cast<int64_t>(N) * a.chunk + own > a.t_max) own = max(0, a.t_max - N * a.chunk);
 
   // Selected chunks of this split, in list order (invalid entries dropped).
@@ -398,7 +462,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
       const int i = base + lane;
       int m = -1;
       if (i < i1) {
-        m = a.sel_idx[row * a.k + i];
+        m = __ldcg(a.sel_idx + row * a.k + i);
         if (m >= N) {
           flag_error(a.status, GSA_DEVERR_BAD_INDEX);
           m = -1;
@@ -540,7 +604,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
     if (a.exclude)
 #pragma unroll
       for (int hs = 0; hs < 2; ++hs)
-        if (item[hs] >= 0) z[hs] = a.sel_score[row * a.k + item_pos[item[hs]]] * kLog2e;
+        if (item[hs] >= 0) z[hs] = __ldcg(a.sel_score + row * a.k + item_pos[item[hs]]) * kLog2e;
     float qm = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
     qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 1));
     qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, 2));
@@ -613,6 +677,7 @@ __global__ void __launch_bounds__(kUnfoldThreads) k_unfold_tc(const __grid_const
     }
   }
   unfold_finish<kUnfoldWarps, D>(a, row, split, red, is_last_s);
+  if (a.ready.w) unfold_ready_done(a);
 }
 
 }  // namespace gsa
