@@ -134,21 +134,21 @@ __device__ __forceinline__ void sts_u2(uint32_t a, uint2 v) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
 }
 
-// Append (v, idx) to a row half's column when v >= bound: the store and
-// the count are predicated (no branch); past CAP the last slot is
-// overwritten and only the count grows, which the row end reports as an
-// overflow.  NaN (a masked score) fails the compare.
-template <int CAP>
-__device__ __forceinline__ void ps_append(uint32_t base, uint32_t &cnt, float v, float bound, uint32_t idx) {
+// Append (v, idx) to a row half's column when v >= bound, at the slot
+// address `ad`, which then moves on by one slot (the count is (ad - base) /
+// kPsSlot).  The store and the step are predicated (no branch).  Past the
+// last slot the store lands in the last one while the address keeps
+// counting, which the row end reports as an overflow.  NaN (a masked
+// score) fails the compare.
+__device__ __forceinline__ void ps_append(uint32_t &ad, uint32_t last, float v, float bound, uint32_t idx) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .u32 s, ad;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .u32 a2;\n\t"
       "setp.ge.f32 p, %1, %2;\n\t"
-      "min.u32 s, %0, %5;\n\t"
-      "mad.lo.u32 ad, s, %6, %3;\n\t"
-      "@p st.shared.v2.u32 [ad], {%4, %7};\n\t"
-      "@p add.u32 %0, %0, 1;\n\t}\n"
-      : "+r"(cnt)
-      : "f"(v), "f"(bound), "r"(base), "r"(__float_as_uint(v)), "r"(CAP - 1), "r"(kPsSlot), "r"(idx)
+      "min.u32 a2, %0, %6;\n\t"
+      "@p st.shared.v2.u32 [a2], {%3, %4};\n\t"
+      "@p add.u32 %0, %0, %5;\n\t}\n"
+      : "+r"(ad)
+      : "f"(v), "f"(bound), "r"(__float_as_uint(v)), "r"(idx), "n"(kPsSlot), "r"(last)
       : "memory");
 }
 
@@ -444,14 +444,15 @@ __global__ void __launch_bounds__(kPsThreads, 1) k_prefill_score(const __grid_co
         continue;
       }
       // ---- pass B: candidates >= bound ----
-      uint32_t cnt = 0;
+      uint32_t ad = base;
+      const uint32_t last = base + (kCap - 1) * kPsSlot;
       for (int j = 0; j < tl.n_kt && ok; ++j)
         ok = take(j, limit, [&](const float(&v)[64], int tb) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            ps_append<kCap>(base, cnt, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
+          for (int e = 0; e < 64; ++e) ps_append(ad, last, v[e], bound, static_cast<uint32_t>(tb + e + (e >> 5) * 32));
         });
       if (!ok) break;
+      const uint32_t cnt = (ad - base) / kPsSlot;
       bool ovf = cnt > static_cast<uint32_t>(kCap);  // the row goes to the exact per-row pass
       const int mine = min(static_cast<int>(cnt), kCap);
       cnt_x[h * kPfRows + r] = static_cast<uint8_t>(ovf ? 255 : mine);
