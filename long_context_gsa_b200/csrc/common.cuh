@@ -33,6 +33,13 @@ constexpr uint64_t kWaitLimitNs = GSA_WAIT_LIMIT_NS;
 #define GSA_TEST_STALL_BYTES 0u
 #endif
 
+// Test builds only: with 1, the fused decode's scoring tail never publishes
+// row 0 in the ready list, so the unfold CTA that waits for the last slot
+// must run out of its wait, flag GSA_DEVERR_TIMEOUT and return.
+#ifndef GSA_TEST_SKIP_PUBLISH
+#define GSA_TEST_SKIP_PUBLISH 0
+#endif
+
 // Partial softmax record: base-2 max, sum, then `d` accumulator floats.
 // Stored as float[d + 4] (the two pad floats keep the accumulator 16-byte
 // aligned).  Logits are kept in the base-2 domain: z2 = scale*log2(e)*q.k.
@@ -76,6 +83,7 @@ __device__ __forceinline__ void flag_error(uint32_t *status, uint32_t bits);
 
 // Publish `row` (its outputs written and fenced by every writer).
 __device__ __forceinline__ void ready_publish(const ReadyList &r, int row, uint32_t *status) {
+  if (GSA_TEST_SKIP_PUBLISH && row == 0) return;
   const uint32_t pos = atomicAdd(&r.w[r.rows], 1u);
   if (pos < static_cast<uint32_t>(r.rows))
     st_release_u32(&r.w[pos], static_cast<uint32_t>(row) + 1u);

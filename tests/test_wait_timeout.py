@@ -8,7 +8,13 @@ limit and copy barriers that expect 16 bytes more than their copies bring
 unfold's per-warp ring waits must then run out; the calls return, the
 status reads TIMEOUT, the top-k result is still exact (the row is read from
 global memory after the failed wait), and the normal library keeps working
-in the same process."""
+in the same process.
+
+A second variant (50 ms limit) never publishes row 0 in the fused decode's
+ready list: the unfold CTA that waits for the last published row must run
+out of its wait and report it, every other row must come out exactly as
+the normal library computes it, and the list must be left clear for the
+next call."""
 import pytest
 import torch
 
@@ -79,3 +85,42 @@ def test_stalled_waits_time_out_and_report(libs):
     assert G.gsa_workspace_status(ws) == 0
     assert torch.equal(torch.sort(sel2, -1).values, torch.sort(ref_sel, -1).values)
     assert torch.isfinite(out2).all()
+
+
+@pytest.fixture(scope="module")
+def skip_lib():
+    from long_context_gsa_b200 import _abi, build
+    build.build_library()
+    return _abi.load(build.build_variant(build.PKG / "libgsa_skiptest.so",
+                                         {"GSA_WAIT_LIMIT_NS": "50000000ull", "GSA_TEST_SKIP_PUBLISH": "1"}))
+
+
+def test_unpublished_row_times_out(skip_lib):
+    import long_context_gsa_b200 as G
+    import long_context_gsa_b200.workloads as W
+    cfg = W.scaled(W.LLAMA_8X, batch=2, context=512 * 8)
+    x = W.decode_inputs(cfg, device="cuda", own_len=5)
+    B, hq, d = x["q"].shape
+    n_max, t_max = x["gist_k"].shape[2], x["raw_k"].shape[2]
+    desc = G.make_desc(B, hq, cfg.hkv, d, cfg.chunk, n_max, t_max, cfg.topk, False, 0.0, G.GSA_BF16, G.GSA_F32)
+    ws = torch.empty(G.gsa_workspace_bytes(desc, G.GSA_OP_DECODE), dtype=torch.uint8, device="cuda")
+    G.gsa_workspace_init(ws)
+
+    def decode():
+        out = torch.full((B, hq, d), float("nan"), dtype=torch.float32, device="cuda")
+        G.gsa_decode(desc, x["q"], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
+                     out, None, None, None, ws)
+        torch.cuda.synchronize()
+        return out
+
+    ref = decode()
+    assert G.gsa_workspace_status(ws) == 0
+    out = _call_with(skip_lib, decode)
+    flags = _call_with(skip_lib, G.gsa_workspace_status, ws)
+    assert flags & G.GSA_DEVERR_TIMEOUT, f"status {flags:#x}"
+    # every row but row 0 was published and unfolded as usual
+    assert torch.equal(out.reshape(B * hq, d)[1:], ref.reshape(B * hq, d)[1:])
+    # the last unfold CTA cleared the list: the normal library decodes cleanly
+    G.gsa_workspace_init(ws)
+    assert torch.equal(decode(), ref)
+    assert G.gsa_workspace_status(ws) == 0
