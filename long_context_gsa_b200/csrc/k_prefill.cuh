@@ -1026,7 +1026,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_prefill_gist_attn(const __gri
 // stages do not cover -- the selected chunks (with their gist in exclude
 // mode) and the own-chunk prefix for raw rows, chunk m's raw tokens for gist
 // row m -- merged with the row's gist partial.  One warp per row; a group of
-// D/8 lanes owns one key row (8 dims per lane), 32/(D/8) rows per step.
+// D/16 lanes owns one key row (16 dims per lane, packed fp32x2 FMAs), so a
+// step covers 32/(D/16) rows, and up to two steps' loads are in flight.
 struct GatherArgs {
   const __nv_bfloat16 *q_raw, *k_raw, *v_raw, *q_gist, *v_gist;
   const int32_t *sel_idx;
@@ -1038,11 +1039,23 @@ struct GatherArgs {
   int32_t out_bf16;
 };
 
-constexpr int kGatherWarps = 8;
+constexpr int kGatherWarps = 4;
+
+// (d.x, d.y) += (a.x * b.x, a.y * b.y): one packed fp32x2 FMA.
+__device__ __forceinline__ void fma2_pair(float2 &d, float ax, float ay, float bx, float by) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+}
 
 template <int D>
 __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const GatherArgs a) {
-  constexpr int kE = 8, kLpr = D / kE, kSlots = 32 / kLpr;  // lanes per key row, rows per step
+  constexpr int kE = 16, kLpr = D / kE, kSlots = 32 / kLpr, kU = 2;  // dims per lane, lanes per row, rows per step
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rows_raw = static_cast<int64_t>(a.bh) * a.L;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kGatherWarps + warp;
@@ -1060,48 +1073,66 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
                                       : a.q_raw + (static_cast<size_t>(bh) * a.L + pos) * D;
   float qf[kE];
   Vec16<__nv_bfloat16>::unpack(ldg_nc_v4(qrow + dd), qf);
-  float m = neg_inf(), l = 0.f, acc[kE];
+  Vec16<__nv_bfloat16>::unpack(ldg_nc_v4(qrow + dd + 8), qf + 8);
+  float m = neg_inf(), l = 0.f;
+  float2 acc[kE / 2];
 #pragma unroll
-  for (int e = 0; e < kE; ++e) acc[e] = 0.f;
-  auto update = [&](float z, const float *vf) {
+  for (int e = 0; e < kE / 2; ++e) acc[e] = make_float2(0.f, 0.f);
+  // acc += p * v for the 16 values of v (two 16-byte words of bf16 pairs)
+  auto add_v = [&](float p, const uint4 &v0, const uint4 &v1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) fma2_pair(acc[e], p, p, bf16_lo(w[e]), bf16_hi(w[e]));
+  };
+  auto update = [&](float z, const uint4 &v0, const uint4 &v1) {
     if (z > m + 8.0f) {
       const float c = exp2_approx(m - z);
       l *= c;
 #pragma unroll
-      for (int e = 0; e < kE; ++e) acc[e] *= c;
+      for (int e = 0; e < kE / 2; ++e) {
+        acc[e].x *= c;
+        acc[e].y *= c;
+      }
       m = z;
     }
     const float p = exp2_approx(z - m);
     l += p;
-#pragma unroll
-    for (int e = 0; e < kE; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
+    add_v(p, v0, v1);
   };
-  // attend raw rows [first, first + n) of this kv head, 4 rows per lane group in flight
+  // q . k for this lane's 16 dims (packed), summed over the row's lanes
+  auto dot = [&](const uint4 &k0, const uint4 &k1) {
+    const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) fma2_pair(s, qf[2 * e], qf[2 * e + 1], bf16_lo(w[e]), bf16_hi(w[e]));
+    float part = s.x + s.y;
+#pragma unroll
+    for (int o = 1; o < kLpr; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    return part;
+  };
+  // attend raw rows [first, first + n) of this kv head: up to kU steps of
+  // kSlots rows with their loads in flight (steps past n are skipped)
   auto span = [&](int first, int n) {
-    for (int r0 = 0; r0 < n; r0 += 4 * kSlots) {
-      uint4 kw[4], vw[4];
+    for (int r0 = 0; r0 < n; r0 += kU * kSlots) {
+      uint4 kw[kU][2], vw[kU][2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + kSlots * u + slot;
-        const size_t off = (kv0 + first + min(r, n - 1)) * D + dd;
-        kw[u] = ldg_nc_v4(a.k_raw + off);
-        vw[u] = ldg_nc_v4(a.v_raw + off);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + kSlots * u + slot;
-        float kf[kE], part = 0.f;
-        Vec16<__nv_bfloat16>::unpack(kw[u], kf);
-#pragma unroll
-        for (int e = 0; e < kE; ++e) part = fmaf(qf[e], kf[e], part);
-#pragma unroll
-        for (int o = 1; o < kLpr; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (r < n) {
-          float vf[kE];
-          Vec16<__nv_bfloat16>::unpack(vw[u], vf);
-          update(part * a.scale_log2, vf);
+      for (int u = 0; u < kU; ++u)
+        if (r0 + kSlots * u < n) {  // warp-uniform
+          const int r = r0 + kSlots * u + slot;
+          const __nv_bfloat16 *kp = a.k_raw + (kv0 + first + min(r, n - 1)) * D + dd;
+          const __nv_bfloat16 *vp = a.v_raw + (kv0 + first + min(r, n - 1)) * D + dd;
+          kw[u][0] = ldg_nc_v4(kp);
+          kw[u][1] = ldg_nc_v4(kp + 8);
+          vw[u][0] = ldg_nc_v4(vp);
+          vw[u][1] = ldg_nc_v4(vp + 8);
         }
-      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (r0 + kSlots * u < n) {
+          const int r = r0 + kSlots * u + slot;
+          const float part = dot(kw[u][0], kw[u][1]);
+          if (r < n) update(part * a.scale_log2, vw[u][0], vw[u][1]);
+        }
     }
   };
   if (is_gist) {
@@ -1114,21 +1145,26 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
       if (t < 0 || t >= mc) continue;
       span(t * a.chunk, a.chunk);
       if (a.exclude && slot == 0) {
-        float vf[kE];
-        Vec16<__nv_bfloat16>::unpack(ldg_nc_v4(a.v_gist + (static_cast<size_t>(kvh) * a.n_chunks + t) * D + dd), vf);
-        update(a.sel_score[ridx * a.topk + e] * kLog2e, vf);
+        const __nv_bfloat16 *gv = a.v_gist + (static_cast<size_t>(kvh) * a.n_chunks + t) * D + dd;
+        update(a.sel_score[ridx * a.topk + e] * kLog2e, ldg_nc_v4(gv), ldg_nc_v4(gv + 8));
       }
     }
     span(mc * a.chunk, pos - mc * a.chunk + 1);
   }
   // merge the row slots, then the gist partial of the row
+  float accf[kE];
+#pragma unroll
+  for (int e = 0; e < kE / 2; ++e) {
+    accf[2 * e] = acc[e].x;
+    accf[2 * e + 1] = acc[e].y;
+  }
 #pragma unroll
   for (int o = kLpr; o < 32; o <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
     float acc2[kE];
 #pragma unroll
-    for (int e = 0; e < kE; ++e) acc2[e] = __shfl_xor_sync(0xffffffffu, acc[e], o);
-    merge_state<kE>(m, l, acc, m2, l2, acc2);
+    for (int e = 0; e < kE; ++e) acc2[e] = __shfl_xor_sync(0xffffffffu, accf[e], o);
+    merge_state<kE>(m, l, accf, m2, l2, acc2);
   }
   const bool has_prior = is_gist || !a.exclude;
   if (has_prior) {
@@ -1136,18 +1172,22 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
     const float pm = rec[0], pl = rec[1];
     if (pm != neg_inf() && pl > 0.f) {
       float pacc[kE];
-      const float4 x = *reinterpret_cast<const float4 *>(rec + kPartHeader + dd);
-      const float4 y = *reinterpret_cast<const float4 *>(rec + kPartHeader + dd + 4);
-      pacc[0] = x.x; pacc[1] = x.y; pacc[2] = x.z; pacc[3] = x.w;
-      pacc[4] = y.x; pacc[5] = y.y; pacc[6] = y.z; pacc[7] = y.w;
-      merge_state<kE>(m, l, acc, pm, pl, pacc);
+#pragma unroll
+      for (int e = 0; e < kE; e += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(rec + kPartHeader + dd + e);
+        pacc[e] = x.x;
+        pacc[e + 1] = x.y;
+        pacc[e + 2] = x.z;
+        pacc[e + 3] = x.w;
+      }
+      merge_state<kE>(m, l, accf, pm, pl, pacc);
     }
   }
   if (lane < kLpr) {
     void *out = is_gist ? a.out_gist : a.out_raw;
     const size_t base = static_cast<size_t>(ridx) * D + dd;
 #pragma unroll
-    for (int e = 0; e < kE; ++e) store_out(out, base + e, l > 0.f ? acc[e] / l : 0.f, a.out_bf16);
+    for (int e = 0; e < kE; ++e) store_out(out, base + e, l > 0.f ? accf[e] / l : 0.f, a.out_bf16);
   }
 }
 
