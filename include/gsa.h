@@ -144,7 +144,9 @@ gsa_status gsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronise `stream`, copy the workspace status word (GSA_DEVERR_* bits)
  * to *flags_out and clear it.  A nonzero TIMEOUT bit means results of the
- * affected calls are invalid. */
+ * affected calls are invalid; call gsa_workspace_init before reusing the
+ * workspace after any nonzero flag (counters or the ready list may have
+ * been left mid-way). */
 gsa_status gsa_workspace_status(void *ws, size_t ws_bytes, void *stream, uint32_t *flags_out);
 
 /* ---- Flat GSA decode: three steps ------------------------------------- */
@@ -222,8 +224,11 @@ gsa_status gsa_score_select(const gsa_desc *desc, const void *q, const void *gis
                             const int32_t *n_gists, float *scores, int32_t *sel_idx, float *sel_score, void *ws,
                             size_t ws_bytes, void *stream);
 /* One decode step = score -> select -> unfold on `stream` (bf16: two
- * launches, gsa_score_select then the unfold; fp32: three).  sel_idx /
- * sel_score ([B, hq, topk]) may be NULL, in which case ws holds them. */
+ * launches, gsa_score_select then the unfold; fp32: three).  In the bf16
+ * form the scoring kernel publishes each selected row in a ready list in
+ * ws and the unfold's CTAs take rows as they are published, instead of
+ * waiting for the whole scoring kernel.  sel_idx / sel_score ([B, hq,
+ * topk]) may be NULL, in which case ws holds them. */
 gsa_status gsa_decode(const gsa_desc *desc, const void *q, const void *gist_k, const void *gist_v, const void *raw_k,
                       const void *raw_v, const int32_t *n_gists, const int32_t *own_len, void *out, float *lse,
                       int32_t *sel_idx, float *sel_score, void *ws, size_t ws_bytes, void *stream);
