@@ -513,6 +513,30 @@ def pin_prefill_bruteforce(orc):
                 np.testing.assert_allclose(res["out"][r], out, rtol=1e-12, atol=1e-12)
 
 
+def pin_prefill_large_k(orc):
+    """k above 16 (the GPU's wide scorer): rows with m > k against brute-force
+    selection and the dense mask, with k close to the number of chunks."""
+    rng = np.random.default_rng(33)
+    B, Hq, Hkv, d, c, N, k = 1, 2, 1, 3, 2, 26, 21
+    arr = rand_prefill(rng, B, Hq, Hkv, d, c, N)
+    L = N * c
+    sc = 1 / math.sqrt(d)
+    rows = [h * (L + N) + pos for h in range(Hq) for pos in range((k + 1) * c, L)]
+    for exclude in (False, True):
+        res = run_prefill(orc, arr, c, k, exclude, rows=rows)
+        for i, r in enumerate(rows):
+            h, pos = divmod(r, L + N)
+            m, j = divmod(pos, c)
+            q = arr["q_raw"][0, h, pos].astype(np.float64)
+            gk = arr["k_gist"][0, 0].astype(np.float64)
+            S = brute_topk(list(sc * (gk[:m] @ q)), k)
+            K, V, lab = interleaved(arr["k_raw"][0, 0].astype(np.float64), arr["v_raw"][0, 0].astype(np.float64),
+                                    gk, arr["v_gist"][0, 0].astype(np.float64), m, c, j + 1)
+            out, lse, _ = softmax_attend(q, K, V, decode_mask(lab, S, exclude), sc)
+            assert {int(x) for x in res["sel"][i] if x >= 0} == S
+            np.testing.assert_allclose(res["out"][i], out, rtol=1e-12, atol=1e-12)
+
+
 def pin_prefill_golden(orc):
     """Hand-derived example (tests/golden/prefill_hand.json)."""
     _check_golden(orc, json.loads((GOLDEN / "prefill_hand.json").read_text()))
@@ -770,5 +794,5 @@ DECODE_PINS = [pin_decode_bruteforce, pin_decode_dense_limit, pin_decode_k0_comp
                pin_gist_step_closed_form, pin_multiquery_bruteforce]
 HGSA_PINS = [pin_hgsa_bruteforce, pin_hgsa_reduces_to_flat, pin_hgsa_golden, pin_hgsa2_bruteforce,
              pin_hgsa2_reduces_to_one_level]
-PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_golden]
+PREFILL_PINS = [pin_prefill_dense_and_gist_rows, pin_prefill_bruteforce, pin_prefill_large_k, pin_prefill_golden]
 ALL_PINS = [pin_topk_selection, pin_topp_selection] + DECODE_PINS + HGSA_PINS + PREFILL_PINS
