@@ -220,6 +220,51 @@ def timed_steps(step, steps, flush, n_marks=1):
     return np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(n_marks)] for s in range(steps)])
 
 
+def pipelined_e2e(G, x, desc, out, sel, ssc, ws, steps):
+    """A serving loop through gsa_decode: step s's query goes host -> device
+    on one copy stream while step s-1 computes, and step s's output comes
+    back device -> host on a second copy stream while step s+1 computes
+    (two buffers each way).  Every step copies its input in and its result
+    out inside the timed region.  The loop runs back to back: its inputs
+    (gist and raw K/V) are larger than L2, so no flush runs between steps.
+    Returns the loop's total time in ms (events on the compute stream)."""
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    q_host = [x["q"].cpu().pin_memory() for _ in range(2)]
+    q_dev = [torch.empty_like(x["q"]) for _ in range(2)]
+    out_dev = [torch.empty_like(out) for _ in range(2)]
+    out_host = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for i in range(2):
+        ev_comp[i].record(comp)
+        ev_out[i].record(comp)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(comp)
+    for s in range(steps):
+        i = s & 1
+        h2d.wait_event(ev_comp[i])  # step s-2 no longer reads q_dev[i]
+        with torch.cuda.stream(h2d):
+            q_dev[i].copy_(q_host[i], non_blocking=True)
+        ev_in[i].record(h2d)
+        comp.wait_event(ev_in[i])
+        comp.wait_event(ev_out[i])  # step s-2's result has left out_dev[i]
+        G.gsa_decode(desc, q_dev[i], x["gist_k"], x["gist_v"], x["raw_k"], x["raw_v"], x["n_gists"], x["own_len"],
+                     out_dev[i], None, sel, ssc, ws)
+        ev_comp[i].record(comp)
+        d2h.wait_event(ev_comp[i])
+        with torch.cuda.stream(d2h):
+            out_host[i].copy_(out_dev[i], non_blocking=True)
+        ev_out[i].record(d2h)
+    for i in range(2):
+        comp.wait_event(ev_out[i])  # every result is on the host
+    t1.record(comp)
+    t1.synchronize()
+    return t0.elapsed_time(t1)
+
+
 def decode_setup(G, W, cfg, dev, seed):
     x = W.decode_inputs(cfg, device=dev, seed=seed)
     B, hq, d = x["q"].shape
@@ -292,7 +337,8 @@ def measure_flat(G, W, cfg, dev, args, flush, seed, e2e=False, clock_index=None)
             out_host.copy_(out, non_blocking=True)
             evs[1].record()
 
-        res["e2e_ms"] = timed_steps(step_e2e, args.steps, flush)[:, 0]
+        res["e2e_seq_ms"] = timed_steps(step_e2e, args.steps, flush)[:, 0]
+        res["e2e_pipe_ms"] = pipelined_e2e(G, x, desc, out, sel, ssc, ws, args.steps)
         res["h2d"] = int(x["q"].numel() * x["q"].element_size())
         res["d2h"] = int(out.numel() * out.element_size())
     assert G.gsa_workspace_status(ws) == 0, "device status flags set"
@@ -786,7 +832,8 @@ def run_gsa(args, world, rank, local):
         return None
     main = measure_flat(G, W, cfg, dev, args, flush, rank_seed(cfg, rank), e2e=True, clock_index=local)
     barrier()
-    total_ms, total_e2e_ms = max_over_ranks([np.sum(main["step_ms"]), np.sum(main["e2e_ms"])], world, dev)
+    total_ms, total_e2e_ms, total_seq_ms = max_over_ranks(
+        [np.sum(main["step_ms"]), main["e2e_pipe_ms"], np.sum(main["e2e_seq_ms"])], world, dev)
 
     extra = {}
     if rank == 0 and world == 1 and not args.main_only:
@@ -827,8 +874,14 @@ def run_gsa(args, world, rank, local):
             "gpu_launches": launches_per_step(cfg) * args.steps,
             "workloads": extra,
             "clocks": main["clocks"],
-            "e2e": {"value": round(job_rate(cfg.head_queries, world, args.steps, total_e2e_ms), 1), "unit": UNIT,
-                    "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"]},
+            "e2e": {"value": round(job_rate(cfg.head_queries, world, args.steps, total_seq_ms), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
+                    "mode": "each step timed alone: its query copied in, the decode, its output copied out, in "
+                            "sequence on one stream, L2 flushed between steps",
+                    "pipelined_value": round(job_rate(cfg.head_queries, world, args.steps, total_e2e_ms), 1),
+                    "pipelined_mode": "serving loop, steps back to back without L2 flushes: each step's query "
+                                      "copied in on one stream while the previous step computes, its output copied "
+                                      "out on another while the next computes"},
             "kernels_us": s["kernels_us"],
             "step_hbm": s["step_hbm"],
             "roofline": roof,
