@@ -1113,16 +1113,14 @@ __global__ void __launch_bounds__(kGatherWarps * 32) k_prefill_gather(const Gath
   // attend raw rows [first, first + n) of this kv head: up to kU steps of
   // kSlots rows with their loads in flight (steps past n are skipped)
   auto span = [&](int first, int n) {
-    const size_t off0 = (kv0 + first) * D + dd;  // this lane's slice of the span's first row
-    const __nv_bfloat16 *kb = a.k_raw + off0, *vb = a.v_raw + off0;
     for (int r0 = 0; r0 < n; r0 += kU * kSlots) {
       uint4 kw[kU][2], vw[kU][2];
 #pragma unroll
       for (int u = 0; u < kU; ++u)
         if (r0 + kSlots * u < n) {  // warp-uniform
-          const int r = min(r0 + kSlots * u + slot, n - 1) * D;  // (a span is at most 64 rows)
-          const __nv_bfloat16 *kp = kb + r;
-          const __nv_bfloat16 *vp = vb + r;
+          const int r = r0 + kSlots * u + slot;
+          const __nv_bfloat16 *kp = a.k_raw + (kv0 + first + min(r, n - 1)) * D + dd;
+          const __nv_bfloat16 *vp = a.v_raw + (kv0 + first + min(r, n - 1)) * D + dd;
           kw[u][0] = ldg_nc_v4(kp);
           kw[u][1] = ldg_nc_v4(kp + 8);
           vw[u][0] = ldg_nc_v4(vp);
