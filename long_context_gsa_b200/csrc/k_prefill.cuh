@@ -12,8 +12,9 @@
 // against every visible gist key -- on the 5th-generation tensor cores.
 // Persistent CTAs walk query tiles of 128 rows of one head (gist-query
 // tiles, then raw tiles, heaviest first).  Warp 0 issues TMA loads (Q tile,
-// then 128-gist key tiles into a 3-stage ring), warp 1 issues tcgen05.mma
-// into three 128-column TMEM accumulators, and warps 2..9 (two per TMEM lane
+// then 128-gist key tiles into a 3-stage ring, 2 stages for the wide
+// scorer at d = 128), warp 1 issues tcgen05.mma into three 128-column TMEM
+// accumulators, and warps 2..9 (two per TMEM lane
 // quadrant, so two threads per query row, each owning a 64-column half of
 // every key tile) read the scores with tcgen05.ld and apply the
 // block-causal mask.  Raw rows take the key tiles twice: a first pass of
